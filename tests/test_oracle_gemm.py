@@ -1,0 +1,157 @@
+"""Pins of the oracle's scaled GEMM.
+
+Fixed outside the oracle: exact integer dot products (every E4M3 value is an
+integer multiple of 2^-9), exact rational arithmetic for the epilogue with a
+brute-force bf16 rounding, the hand-derived worked example, and the page's
+identities: the naive two-step path equals the fused one, per-tensor scaling
+is the equal-scale special case, and transposing both operands transposes the
+output."""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from golden_io import float_array, hex_array, read_sections
+
+
+def int_units_table():
+    """E4M3 values in integer units of 2^-9, from PyTorch's decoder."""
+    v = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    out = []
+    for c in range(256):
+        if np.isnan(v[c]):
+            out.append(None)
+        else:
+            u = v[c] * 512
+            assert u == int(u)
+            out.append(int(u))
+    return out
+
+
+def random_codes(rng, shape, extreme=False):
+    if extreme:
+        return rng.choice(np.array([0x7E, 0xFE], np.uint8), size=shape)
+    c = rng.integers(0, 256, size=shape).astype(np.uint8)
+    c[(c & 0x7F) == 0x7F] = 0x7E      # no NaN codes
+    return c
+
+
+@pytest.mark.parametrize("T,Ci,Co,extreme", [(3, 5, 4, False), (7, 64, 9, False),
+                                            (2, 2048, 3, True), (5, 300, 6, False)])
+def test_acc_is_exact_integer_dot_product(T, Ci, Co, extreme):
+    rng = np.random.default_rng(T * 1000 + Ci)
+    Xq = random_codes(rng, (T, Ci), extreme)
+    Wq_t = random_codes(rng, (Co, Ci), extreme)
+    acc = oracle.gemm_acc64(Xq, Wq_t)
+    units = int_units_table()
+    for t in range(T):
+        for o in range(Co):
+            s = sum(units[a] * units[b] for a, b in zip(Xq[t], Wq_t[o]))
+            assert Fraction(acc[t, o]) == Fraction(s, 2 ** 18)
+
+
+def test_acc_exact_at_full_depth():
+    Ci = 28672
+    Xq = np.full((1, Ci), 0x7E, np.uint8)
+    Wq_t = np.full((2, Ci), 0x7E, np.uint8)
+    Wq_t[1, ::2] = 0xFE
+    acc = oracle.gemm_acc64(Xq, Wq_t)
+    assert acc[0, 0] == Ci * 448.0 * 448.0 and acc[0, 1] == 0.0
+
+
+def brute_bf16(fr: Fraction) -> int:
+    """bf16 bits of an exact rational, round-half-to-even, by bracketing."""
+    if fr == 0:
+        return 0
+    sign = 0x8000 if fr < 0 else 0
+    a = abs(fr)
+    # binary search over the monotone positive finite bf16 values
+    vals = lambda b: Fraction(float(oracle.bf16_to_float(np.array([b], np.uint16))[0]))
+    lo, hi = 0, 0x7F7F
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if vals(mid) <= a:
+            lo = mid
+        else:
+            hi = mid
+    dl, dh = a - vals(lo), vals(hi) - a
+    if dl < dh or (dl == dh and lo % 2 == 0):
+        return sign | lo
+    return sign | hi
+
+
+def test_reference_epilogue_matches_exact_rational():
+    rng = np.random.default_rng(9)
+    T, Ci, Co = 4, 96, 5
+    Xq = random_codes(rng, (T, Ci))
+    Wq_t = random_codes(rng, (Co, Ci))
+    xs = (rng.random(T) * 1e-2 + 1e-4).astype(np.float32)
+    ws = (rng.random(Co) * 1e-3 + 1e-5).astype(np.float32)
+    out = oracle.scaled_mm_reference(Xq, xs, Wq_t, ws)
+    units = int_units_table()
+    for t in range(T):
+        for o in range(Co):
+            s = sum(units[a] * units[b] for a, b in zip(Xq[t], Wq_t[o]))
+            exact = Fraction(s, 2 ** 18) * Fraction(float(xs[t])) * Fraction(float(ws[o]))
+            assert out[t, o] == brute_bf16(exact), (t, o)
+
+
+def test_hand_example_gemm():
+    g = read_sections("hand_example.txt")
+    Xq = hex_array(g["Xq_u8"], np.uint8)
+    Wq_t = hex_array(g["Wq_t_u8"], np.uint8)
+    xs = float_array(g["x_scale_f32"], np.float32)[0]
+    ws = float_array(g["w_scale_f32"], np.float32)[0]
+    assert np.array_equal(oracle.gemm_acc64(Xq, Wq_t), float_array(g["acc_f64"], np.float64))
+    expect = hex_array(g["out_bf16"], np.uint16)
+    assert np.array_equal(oracle.scaled_mm_reference(Xq, xs, Wq_t, ws), expect)
+    assert np.array_equal(oracle.fused_f32(Xq, xs, Wq_t, ws), expect)
+    out, _, _ = oracle.linear_reference(hex_array(g["X_bf16"], np.uint16), Wq_t, ws)
+    assert np.array_equal(out, expect)
+
+
+def test_naive_two_step_equals_fused():
+    w = synthetic.TINY
+    X = synthetic.make_x(w, 0, 16, 256)
+    W = synthetic.make_w(w, 0, 256, 512)
+    Xq, xs = oracle.quant_act(X)
+    Wq_t, ws = oracle.quant_weight(W)
+    y = oracle.naive_step1_f32(Xq, Wq_t)
+    naive = oracle.naive_step2_apply_scales(y, xs, ws)
+    fused = oracle.fused_f32(Xq, xs, Wq_t, ws)
+    assert np.array_equal(naive, fused)
+
+
+def test_per_tensor_special_case():
+    rng = np.random.default_rng(4)
+    Xq = random_codes(rng, (6, 128))
+    Wq_t = random_codes(rng, (10, 128))
+    sx, sw = np.float32(0.0123), np.float32(0.000456)
+    out = oracle.scaled_mm_reference(Xq, np.full(6, sx), Wq_t, np.full(10, sw))
+    acc = oracle.gemm_acc64(Xq, Wq_t)
+    assert np.array_equal(out, oracle.bf16_from_double(acc * (float(sx) * float(sw))))
+
+
+def test_transposed_operands_give_transposed_output():
+    rng = np.random.default_rng(6)
+    Xq = random_codes(rng, (9, 64))
+    Wq_t = random_codes(rng, (13, 64))
+    xs = (rng.random(9) + 0.1).astype(np.float32)
+    ws = (rng.random(13) + 0.1).astype(np.float32)
+    a = oracle.scaled_mm_reference(Xq, xs, Wq_t, ws)
+    b = oracle.scaled_mm_reference(Wq_t, ws, Xq, xs)
+    assert np.array_equal(a, b.T)
+
+
+def test_row_subset_equals_full_rows():
+    rng = np.random.default_rng(8)
+    Xq = random_codes(rng, (20, 64))
+    Wq_t = random_codes(rng, (7, 64))
+    xs = (rng.random(20) + 0.1).astype(np.float32)
+    ws = (rng.random(7) + 0.1).astype(np.float32)
+    rows = [0, 3, 19, 7]
+    full = oracle.scaled_mm_reference(Xq, xs, Wq_t, ws)
+    assert np.array_equal(oracle.scaled_mm_reference(Xq, xs, Wq_t, ws, rows), full[rows])
