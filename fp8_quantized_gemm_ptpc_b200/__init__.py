@@ -1,0 +1,272 @@
+"""PTPC-FP8 (per-token activation, per-channel weight FP8) for NVIDIA B200.
+
+Thin Python binding of the C ABI declared in ``include/ptpc.h``; it only
+marshals torch tensors (device memory and the current stream) into the
+library calls.  Every step of the computation runs in the library's sm_100a
+kernels; there is no CPU or PyTorch fallback, and importing this package
+fails if ``_lib/libptpc.so`` has not been built
+(``python -m fp8_quantized_gemm_ptpc_b200.build``).
+
+Method: "PTPC-FP8: boosting vLLM performance on AMD ROCm" (vLLM blog),
+sections "Per-Token Activation + Per-Channel Weight Quantization" and "The
+challenge: two-step vs fused".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libptpc.so")
+
+# ptpc_status
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_MISALIGNED = 2
+ERR_UNSUPPORTED_SHAPE = 3
+ERR_WORKSPACE_TOO_SMALL = 4
+ERR_UNSUPPORTED_DEVICE = 5
+ERR_CUDA = 6
+ERR_DEVICE_TIMEOUT = 7
+ERR_NOT_IMPLEMENTED = 8
+
+# ptpc_op
+OP_QUANTIZE_WEIGHTS = 1
+OP_SCALED_MM = 2
+OP_LINEAR = 3
+OP_BENCH_PER_TENSOR = 4
+OP_BENCH_UNSCALED_MM = 5
+
+# Every symbol include/ptpc.h declares, with its ctypes signature.
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+SIGNATURES = {
+    "ptpc_quantize_activations": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
+    "ptpc_quantize_weights": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _SZ, _P]),
+    "ptpc_scaled_mm": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "ptpc_linear": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "ptpc_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _I64, _I64, _I64]),
+    "ptpc_get_device_status": (ctypes.c_int, [_P, _P]),
+    "ptpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "ptpc_bench_unscaled_mm_f32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "ptpc_bench_apply_scales": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _P, _P]),
+    "ptpc_bench_quantize_activations_per_tensor": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _SZ, _P]),
+    "ptpc_bench_quantize_weights_per_tensor": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _SZ, _P]),
+}
+
+
+class PtpcError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m fp8_quantized_gemm_ptpc_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.ptpc_status_string(int(status)).decode()
+
+
+def workspace_size(op: int, T: int, Ci: int, Co: int) -> int:
+    return int(lib.ptpc_workspace_size(op, T, Ci, Co))
+
+
+def _check(fn: str, status: int):
+    if status != OK:
+        raise PtpcError(fn, status)
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t: torch.Tensor):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
+
+
+class Workspace:
+    """A zero-filled device buffer for the entry points that take (ws, ws_bytes).
+
+    The library leaves its control words zero after every successful call, so
+    one buffer serves any number of calls (not concurrently on the GPU)."""
+
+    def __init__(self, nbytes: int, device):
+        self.device = torch.device(device)
+        self.buf = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=self.device)
+
+    @property
+    def nbytes(self) -> int:
+        return self.buf.numel()
+
+    def ensure(self, nbytes: int) -> "Workspace":
+        if nbytes > self.nbytes:
+            self.buf = torch.zeros(int(nbytes), dtype=torch.uint8, device=self.device)
+        return self
+
+    def ptr(self):
+        return _ptr(self.buf)
+
+
+_ws_lock = threading.Lock()
+_ws_cache: dict = {}
+
+
+def default_workspace(nbytes: int, device) -> Workspace:
+    """Per-device, per-thread cached workspace grown on demand."""
+    key = (torch.device(device), threading.get_ident())
+    with _ws_lock:
+        ws = _ws_cache.get(key)
+        if ws is None:
+            ws = _ws_cache[key] = Workspace(nbytes, device)
+        return ws.ensure(nbytes)
+
+
+# ----------------------------------------------------------------- entry points
+
+def quantize_activations(X: torch.Tensor, Xq: torch.Tensor | None = None, x_scale: torch.Tensor | None = None):
+    """Per-token quantisation: X bf16 [T, Ci] -> (Xq uint8 [T, Ci], x_scale fp32 [T])."""
+    _need(X, "X", torch.bfloat16, 2)
+    T, Ci = X.shape
+    Xq = torch.empty((T, Ci), dtype=torch.uint8, device=X.device) if Xq is None else Xq
+    x_scale = torch.empty((T,), dtype=torch.float32, device=X.device) if x_scale is None else x_scale
+    _check("ptpc_quantize_activations",
+           lib.ptpc_quantize_activations(_ptr(X), T, Ci, _ptr(Xq), _ptr(x_scale), _stream(X.device)))
+    return Xq, x_scale
+
+
+def quantize_weights(W: torch.Tensor, ws: Workspace | None = None):
+    """Per-output-channel quantisation: W bf16 [Ci, Co] -> (Wq_t uint8 [Co, Ci], w_scale fp32 [Co])."""
+    _need(W, "W", torch.bfloat16, 2)
+    Ci, Co = W.shape
+    Wq_t = torch.empty((Co, Ci), dtype=torch.uint8, device=W.device)
+    w_scale = torch.empty((Co,), dtype=torch.float32, device=W.device)
+    need = workspace_size(OP_QUANTIZE_WEIGHTS, 0, Ci, Co)
+    ws = default_workspace(need, W.device) if ws is None else ws.ensure(need)
+    _check("ptpc_quantize_weights",
+           lib.ptpc_quantize_weights(_ptr(W), Ci, Co, _ptr(Wq_t), _ptr(w_scale), ws.ptr(), ws.nbytes,
+                                     _stream(W.device)))
+    return Wq_t, w_scale
+
+
+def scaled_mm(Xq, x_scale, Wq_t, w_scale, out: torch.Tensor | None = None, ws: Workspace | None = None):
+    """Fused scaled GEMM: out bf16 [T, Co] = bf16((Xq . Wq_t^T) * x_scale[t] * w_scale[o])."""
+    _need(Xq, "Xq", torch.uint8, 2)
+    _need(Wq_t, "Wq_t", torch.uint8, 2)
+    _need(x_scale, "x_scale", torch.float32, 1)
+    _need(w_scale, "w_scale", torch.float32, 1)
+    T, Ci = Xq.shape
+    Co = Wq_t.shape[0]
+    if Wq_t.shape[1] != Ci or x_scale.shape[0] != T or w_scale.shape[0] != Co:
+        raise ValueError("shape mismatch")
+    out = torch.empty((T, Co), dtype=torch.bfloat16, device=Xq.device) if out is None else out
+    need = workspace_size(OP_SCALED_MM, T, Ci, Co)
+    ws = default_workspace(need, Xq.device) if ws is None else ws.ensure(need)
+    _check("ptpc_scaled_mm",
+           lib.ptpc_scaled_mm(_ptr(Xq), _ptr(x_scale), _ptr(Wq_t), _ptr(w_scale), T, Ci, Co, _ptr(out),
+                              ws.ptr(), ws.nbytes, _stream(Xq.device)))
+    return out
+
+
+def linear(X, Wq_t, w_scale, out: torch.Tensor | None = None, ws: Workspace | None = None):
+    """Fused quantise + GEMM: X bf16 [T, Ci] -> out bf16 [T, Co]."""
+    _need(X, "X", torch.bfloat16, 2)
+    _need(Wq_t, "Wq_t", torch.uint8, 2)
+    _need(w_scale, "w_scale", torch.float32, 1)
+    T, Ci = X.shape
+    Co = Wq_t.shape[0]
+    if Wq_t.shape[1] != Ci or w_scale.shape[0] != Co:
+        raise ValueError("shape mismatch")
+    out = torch.empty((T, Co), dtype=torch.bfloat16, device=X.device) if out is None else out
+    need = workspace_size(OP_LINEAR, T, Ci, Co)
+    ws = default_workspace(need, X.device) if ws is None else ws.ensure(need)
+    _check("ptpc_linear",
+           lib.ptpc_linear(_ptr(X), _ptr(Wq_t), _ptr(w_scale), T, Ci, Co, _ptr(out), ws.ptr(), ws.nbytes,
+                           _stream(X.device)))
+    return out
+
+
+def device_status(ws: Workspace) -> int:
+    """Synchronise the current stream and read/clear the workspace's device status word."""
+    return int(lib.ptpc_get_device_status(ws.ptr(), _stream(ws.device)))
+
+
+# ------------------------------------------------ measurement-only entry points
+
+def unscaled_mm_f32(Xq, Wq_t, out: torch.Tensor | None = None, ws: Workspace | None = None):
+    """Naive step 1: fp32 [T, Co] = Xq . Wq_t^T (no scales)."""
+    _need(Xq, "Xq", torch.uint8, 2)
+    _need(Wq_t, "Wq_t", torch.uint8, 2)
+    T, Ci = Xq.shape
+    Co = Wq_t.shape[0]
+    out = torch.empty((T, Co), dtype=torch.float32, device=Xq.device) if out is None else out
+    need = workspace_size(OP_BENCH_UNSCALED_MM, T, Ci, Co)
+    ws = default_workspace(need, Xq.device) if ws is None else ws.ensure(need)
+    _check("ptpc_bench_unscaled_mm_f32",
+           lib.ptpc_bench_unscaled_mm_f32(_ptr(Xq), _ptr(Wq_t), T, Ci, Co, _ptr(out), ws.ptr(), ws.nbytes,
+                                          _stream(Xq.device)))
+    return out
+
+
+def apply_scales(y, x_scale, w_scale, out: torch.Tensor | None = None):
+    """Naive step 2: bf16((y * x_scale[t]) * w_scale[o])."""
+    _need(y, "y", torch.float32, 2)
+    T, Co = y.shape
+    out = torch.empty((T, Co), dtype=torch.bfloat16, device=y.device) if out is None else out
+    _check("ptpc_bench_apply_scales",
+           lib.ptpc_bench_apply_scales(_ptr(y), _ptr(x_scale), _ptr(w_scale), T, Co, _ptr(out),
+                                       _stream(y.device)))
+    return out
+
+
+def quantize_activations_per_tensor(X, Xq=None, x_scale=None, ws: Workspace | None = None):
+    """Per-tensor quantisation of X; x_scale [T] holds the one tensor scale T times."""
+    _need(X, "X", torch.bfloat16, 2)
+    T, Ci = X.shape
+    Xq = torch.empty((T, Ci), dtype=torch.uint8, device=X.device) if Xq is None else Xq
+    x_scale = torch.empty((T,), dtype=torch.float32, device=X.device) if x_scale is None else x_scale
+    need = workspace_size(OP_BENCH_PER_TENSOR, T, Ci, 0)
+    ws = default_workspace(need, X.device) if ws is None else ws.ensure(need)
+    _check("ptpc_bench_quantize_activations_per_tensor",
+           lib.ptpc_bench_quantize_activations_per_tensor(_ptr(X), T, Ci, _ptr(Xq), _ptr(x_scale), ws.ptr(),
+                                                          ws.nbytes, _stream(X.device)))
+    return Xq, x_scale
+
+
+def quantize_weights_per_tensor(W, ws: Workspace | None = None):
+    """Per-tensor quantisation of W; w_scale [Co] holds the one tensor scale Co times."""
+    _need(W, "W", torch.bfloat16, 2)
+    Ci, Co = W.shape
+    Wq_t = torch.empty((Co, Ci), dtype=torch.uint8, device=W.device)
+    w_scale = torch.empty((Co,), dtype=torch.float32, device=W.device)
+    need = workspace_size(OP_QUANTIZE_WEIGHTS, 0, Ci, Co)
+    ws = default_workspace(need, W.device) if ws is None else ws.ensure(need)
+    _check("ptpc_bench_quantize_weights_per_tensor",
+           lib.ptpc_bench_quantize_weights_per_tensor(_ptr(W), Ci, Co, _ptr(Wq_t), _ptr(w_scale), ws.ptr(),
+                                                      ws.nbytes, _stream(W.device)))
+    return Wq_t, w_scale

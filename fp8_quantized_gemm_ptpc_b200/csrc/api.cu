@@ -1,0 +1,260 @@
+// C ABI of the PTPC-FP8 library: argument checks, workspace layout and
+// dispatch to the sm_100a kernels.  Declared in include/ptpc.h.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda_runtime.h>
+
+#include "../../include/ptpc.h"
+#include "kernels.h"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int64_t kMaxDim = 0x7FFFFFFF;
+
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Workspace layout of the GEMM entry points:
+//   [0, 256)                 device status word (uint32 at offset 0)
+//   [256, 256 + C)           split-K tile counters (uint32, zero between calls)
+//   [.., .. + P)             split-K fp32 partial sums
+// ptpc_linear appends Xq [T, Ci] and x_scale [T] after the GEMM region.
+struct GemmLayout {
+  size_t counters_off, partials_off, end;
+  size_t partial_floats;
+};
+
+GemmLayout gemm_layout(int64_t T, int64_t Ci, int64_t Co) {
+  size_t cw = 0, pf = 0;
+  ptpc::gemm_workspace_needs((int)T, (int)Ci, (int)Co, &cw, &pf);
+  GemmLayout l;
+  l.counters_off = kAlign;
+  l.partials_off = l.counters_off + round_up(cw * 4);
+  l.end = l.partials_off + round_up(pf * 4);
+  l.partial_floats = pf;
+  return l;
+}
+
+// Once per device: the kernels are built for compute capability 10.0 only.
+int check_device() {
+  static std::mutex mu;
+  static int state[64] = {};  // 0 unknown, 1 ok, 2 unsupported
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PTPC_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return PTPC_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  if (state[dev] == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return PTPC_ERR_CUDA;
+    state[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return state[dev] == 1 ? PTPC_OK : PTPC_ERR_UNSUPPORTED_DEVICE;
+}
+
+int check_shape_tci(int64_t T, int64_t Ci) {
+  if (T < 0 || Ci <= 0) return Ci < 0 || T < 0 ? PTPC_ERR_INVALID_ARG : PTPC_ERR_UNSUPPORTED_SHAPE;
+  if (Ci % 16 != 0 || Ci > kMaxDim || T > kMaxDim) return PTPC_ERR_UNSUPPORTED_SHAPE;
+  return PTPC_OK;
+}
+
+int check_co(int64_t Co) {
+  if (Co < 0) return PTPC_ERR_INVALID_ARG;
+  if (Co == 0 || Co % 16 != 0 || Co > kMaxDim) return PTPC_ERR_UNSUPPORTED_SHAPE;
+  return PTPC_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? PTPC_OK : PTPC_ERR_CUDA; }
+
+int run_gemm(const uint8_t *Xq, const float *xs, const uint8_t *Wq_t, const float *ws, int64_t T, int64_t Ci,
+             int64_t Co, void *out, bool f32_out, uint8_t *wsp, bool pdl, cudaStream_t st) {
+  const GemmLayout l = gemm_layout(T, Ci, Co);
+  ptpc::GemmProblem p{};
+  p.Xq = Xq;
+  p.xs = xs;
+  p.Wq_t = Wq_t;
+  p.ws = ws;
+  p.T = (int)T;
+  p.Ci = (int)Ci;
+  p.Co = (int)Co;
+  p.out = out;
+  p.f32_out = f32_out;
+  p.status = reinterpret_cast<uint32_t *>(wsp);
+  p.counters = reinterpret_cast<uint32_t *>(wsp + l.counters_off);
+  p.partials = reinterpret_cast<float *>(wsp + l.partials_off);
+  p.partial_floats = l.partial_floats;
+  p.pdl = pdl;
+  return cuda_status(ptpc::launch_scaled_gemm(p, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ptpc_status_string(int status) {
+  switch (status) {
+    case PTPC_OK: return "PTPC_OK";
+    case PTPC_ERR_INVALID_ARG: return "PTPC_ERR_INVALID_ARG";
+    case PTPC_ERR_MISALIGNED: return "PTPC_ERR_MISALIGNED";
+    case PTPC_ERR_UNSUPPORTED_SHAPE: return "PTPC_ERR_UNSUPPORTED_SHAPE";
+    case PTPC_ERR_WORKSPACE_TOO_SMALL: return "PTPC_ERR_WORKSPACE_TOO_SMALL";
+    case PTPC_ERR_UNSUPPORTED_DEVICE: return "PTPC_ERR_UNSUPPORTED_DEVICE";
+    case PTPC_ERR_CUDA: return "PTPC_ERR_CUDA";
+    case PTPC_ERR_DEVICE_TIMEOUT: return "PTPC_ERR_DEVICE_TIMEOUT";
+    case PTPC_ERR_NOT_IMPLEMENTED: return "PTPC_ERR_NOT_IMPLEMENTED";
+    default: return "PTPC_ERR_UNKNOWN";
+  }
+}
+
+size_t ptpc_workspace_size(int op, int64_t T, int64_t Ci, int64_t Co) {
+  switch (op) {
+    case PTPC_OP_QUANTIZE_WEIGHTS:
+      if (check_shape_tci(0, Ci) != PTPC_OK || check_co(Co) != PTPC_OK) return 0;
+      return kAlign + round_up((size_t)(Co + 1) * 4);
+    case PTPC_OP_SCALED_MM:
+    case PTPC_OP_BENCH_UNSCALED_MM:
+      if (check_shape_tci(T, Ci) != PTPC_OK || check_co(Co) != PTPC_OK) return 0;
+      return gemm_layout(T, Ci, Co).end;
+    case PTPC_OP_LINEAR:
+      if (check_shape_tci(T, Ci) != PTPC_OK || check_co(Co) != PTPC_OK) return 0;
+      return gemm_layout(T, Ci, Co).end + round_up((size_t)T * (size_t)Ci) + round_up((size_t)T * 4);
+    case PTPC_OP_BENCH_PER_TENSOR:
+      if (check_shape_tci(T, Ci) != PTPC_OK) return 0;
+      return kAlign + kAlign;
+    default:
+      return 0;
+  }
+}
+
+int ptpc_quantize_activations(const void *X, int64_t T, int64_t Ci, uint8_t *Xq, float *x_scale, void *stream) {
+  int s = check_shape_tci(T, Ci);
+  if (s != PTPC_OK) return s;
+  if (T == 0) return PTPC_OK;
+  if (!X || !Xq || !x_scale) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Xq) || !aligned16(x_scale)) return PTPC_ERR_MISALIGNED;
+  if ((s = check_device()) != PTPC_OK) return s;
+  return cuda_status(ptpc::launch_quant_act(X, (int)T, (int)Ci, Xq, x_scale, (cudaStream_t)stream));
+}
+
+int ptpc_quantize_weights(const void *W, int64_t Ci, int64_t Co, uint8_t *Wq_t, float *w_scale, void *ws,
+                          size_t ws_bytes, void *stream) {
+  int s = check_shape_tci(0, Ci);
+  if (s != PTPC_OK) return s;
+  if ((s = check_co(Co)) != PTPC_OK) return s;
+  if (!W || !Wq_t || !w_scale || !ws) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(Wq_t) || !aligned16(w_scale) || !aligned16(ws)) return PTPC_ERR_MISALIGNED;
+  if (ws_bytes < ptpc_workspace_size(PTPC_OP_QUANTIZE_WEIGHTS, 0, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device()) != PTPC_OK) return s;
+  uint32_t *col_amax = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + kAlign);
+  return cuda_status(
+      ptpc::launch_quant_weight(W, (int)Ci, (int)Co, Wq_t, w_scale, col_amax, false, (cudaStream_t)stream));
+}
+
+int ptpc_scaled_mm(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq_t, const float *w_scale, int64_t T,
+                   int64_t Ci, int64_t Co, void *out, void *ws, size_t ws_bytes, void *stream) {
+  int s = check_shape_tci(T, Ci);
+  if (s != PTPC_OK) return s;
+  if ((s = check_co(Co)) != PTPC_OK) return s;
+  if (T == 0) return PTPC_OK;
+  if (!Xq || !x_scale || !Wq_t || !w_scale || !out || !ws) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(Xq) || !aligned16(x_scale) || !aligned16(Wq_t) || !aligned16(w_scale) || !aligned16(out) ||
+      !aligned16(ws))
+    return PTPC_ERR_MISALIGNED;
+  if (ws_bytes < ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device()) != PTPC_OK) return s;
+  return run_gemm(Xq, x_scale, Wq_t, w_scale, T, Ci, Co, out, false, static_cast<uint8_t *>(ws), false,
+                  (cudaStream_t)stream);
+}
+
+int ptpc_linear(const void *X, const uint8_t *Wq_t, const float *w_scale, int64_t T, int64_t Ci, int64_t Co,
+                void *out, void *ws, size_t ws_bytes, void *stream) {
+  int s = check_shape_tci(T, Ci);
+  if (s != PTPC_OK) return s;
+  if ((s = check_co(Co)) != PTPC_OK) return s;
+  if (T == 0) return PTPC_OK;
+  if (!X || !Wq_t || !w_scale || !out || !ws) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Wq_t) || !aligned16(w_scale) || !aligned16(out) || !aligned16(ws))
+    return PTPC_ERR_MISALIGNED;
+  if (ws_bytes < ptpc_workspace_size(PTPC_OP_LINEAR, T, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device()) != PTPC_OK) return s;
+  uint8_t *wsp = static_cast<uint8_t *>(ws);
+  const size_t g_end = gemm_layout(T, Ci, Co).end;
+  uint8_t *Xq = wsp + g_end;
+  float *xs = reinterpret_cast<float *>(wsp + g_end + round_up((size_t)T * (size_t)Ci));
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((s = cuda_status(ptpc::launch_quant_act(X, (int)T, (int)Ci, Xq, xs, st))) != PTPC_OK) return s;
+  return run_gemm(Xq, xs, Wq_t, w_scale, T, Ci, Co, out, false, wsp, true, st);
+}
+
+int ptpc_get_device_status(void *ws, void *stream) {
+  if (!ws) return PTPC_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  uint32_t v = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return PTPC_ERR_CUDA;
+  if (cudaMemcpy(&v, ws, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return PTPC_ERR_CUDA;
+  if (v == 0) return PTPC_OK;
+  if (cudaMemset(ws, 0, sizeof v) != cudaSuccess) return PTPC_ERR_CUDA;
+  return PTPC_ERR_DEVICE_TIMEOUT;
+}
+
+int ptpc_bench_unscaled_mm_f32(const uint8_t *Xq, const uint8_t *Wq_t, int64_t T, int64_t Ci, int64_t Co, float *y,
+                               void *ws, size_t ws_bytes, void *stream) {
+  int s = check_shape_tci(T, Ci);
+  if (s != PTPC_OK) return s;
+  if ((s = check_co(Co)) != PTPC_OK) return s;
+  if (T == 0) return PTPC_OK;
+  if (!Xq || !Wq_t || !y || !ws) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(Xq) || !aligned16(Wq_t) || !aligned16(y) || !aligned16(ws)) return PTPC_ERR_MISALIGNED;
+  if (ws_bytes < ptpc_workspace_size(PTPC_OP_BENCH_UNSCALED_MM, T, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device()) != PTPC_OK) return s;
+  return run_gemm(Xq, nullptr, Wq_t, nullptr, T, Ci, Co, y, true, static_cast<uint8_t *>(ws), false,
+                  (cudaStream_t)stream);
+}
+
+int ptpc_bench_apply_scales(const float *y, const float *x_scale, const float *w_scale, int64_t T, int64_t Co,
+                            void *out, void *stream) {
+  int s = check_co(Co);
+  if (s != PTPC_OK) return s;
+  if (T < 0) return PTPC_ERR_INVALID_ARG;
+  if (T > kMaxDim) return PTPC_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return PTPC_OK;
+  if (!y || !x_scale || !w_scale || !out) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(x_scale) || !aligned16(w_scale) || !aligned16(out)) return PTPC_ERR_MISALIGNED;
+  if ((s = check_device()) != PTPC_OK) return s;
+  return cuda_status(ptpc::launch_apply_scales(y, x_scale, w_scale, (int)T, (int)Co, out, (cudaStream_t)stream));
+}
+
+int ptpc_bench_quantize_activations_per_tensor(const void *X, int64_t T, int64_t Ci, uint8_t *Xq, float *x_scale,
+                                               void *ws, size_t ws_bytes, void *stream) {
+  int s = check_shape_tci(T, Ci);
+  if (s != PTPC_OK) return s;
+  if (T == 0) return PTPC_OK;
+  if (!X || !Xq || !x_scale || !ws) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Xq) || !aligned16(x_scale) || !aligned16(ws)) return PTPC_ERR_MISALIGNED;
+  if (ws_bytes < ptpc_workspace_size(PTPC_OP_BENCH_PER_TENSOR, T, Ci, 0)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device()) != PTPC_OK) return s;
+  uint32_t *slot = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + kAlign);
+  return cuda_status(
+      ptpc::launch_quant_act_per_tensor(X, (int)T, (int)Ci, Xq, x_scale, slot, (cudaStream_t)stream));
+}
+
+int ptpc_bench_quantize_weights_per_tensor(const void *W, int64_t Ci, int64_t Co, uint8_t *Wq_t, float *w_scale,
+                                           void *ws, size_t ws_bytes, void *stream) {
+  int s = check_shape_tci(0, Ci);
+  if (s != PTPC_OK) return s;
+  if ((s = check_co(Co)) != PTPC_OK) return s;
+  if (!W || !Wq_t || !w_scale || !ws) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(Wq_t) || !aligned16(w_scale) || !aligned16(ws)) return PTPC_ERR_MISALIGNED;
+  if (ws_bytes < ptpc_workspace_size(PTPC_OP_QUANTIZE_WEIGHTS, 0, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device()) != PTPC_OK) return s;
+  uint32_t *col_amax = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + kAlign);
+  return cuda_status(
+      ptpc::launch_quant_weight(W, (int)Ci, (int)Co, Wq_t, w_scale, col_amax, true, (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// Internal launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "sm100.cuh"
+
+namespace ptpc {
+
+// Quantisers (quant.cu).
+cudaError_t launch_quant_act(const void *X, int T, int Ci, uint8_t *Xq, float *xs, cudaStream_t st);
+cudaError_t launch_quant_act_per_tensor(const void *X, int T, int Ci, uint8_t *Xq, float *xs,
+                                        uint32_t *amax_slot, cudaStream_t st);
+// col_amax: Co + 1 32-bit words of scratch.
+cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, float *w_scale, uint32_t *col_amax,
+                                bool per_tensor, cudaStream_t st);
+cudaError_t launch_apply_scales(const float *y, const float *xs, const float *ws, int T, int Co, void *out,
+                                cudaStream_t st);
+
+// Scaled GEMM (gemm.cu).
+struct GemmProblem {
+  const uint8_t *Xq;      // [T, Ci]
+  const float *xs;        // [T]   (unused for f32 output)
+  const uint8_t *Wq_t;    // [Co, Ci]
+  const float *ws;        // [Co]  (unused for f32 output)
+  int T, Ci, Co;
+  void *out;              // bf16 [T, Co] or fp32 [T, Co]
+  bool f32_out;           // unscaled fp32 output (naive step 1)
+  uint32_t *status;       // device status word
+  uint32_t *counters;     // split-K tile counters (zero on entry, zero on exit)
+  float *partials;        // split-K fp32 partial sums
+  size_t partial_floats;  // capacity of `partials`
+  bool pdl;               // launch as a programmatic dependent of the previous kernel
+};
+
+// Workspace needs of the GEMM for a shape (counter words and partial floats).
+void gemm_workspace_needs(int T, int Ci, int Co, size_t *counter_words, size_t *partial_floats);
+cudaError_t launch_scaled_gemm(const GemmProblem &p, cudaStream_t st);
+
+int num_sms();
+
+}  // namespace ptpc

@@ -1,0 +1,480 @@
+// PTPC-FP8 quantisers for sm_100a.
+//
+// Per-token activation quantisation and per-output-channel weight
+// quantisation ("PTPC-FP8: boosting vLLM performance on AMD ROCm", section
+// "Per-Token Activation + Per-Channel Weight Quantization": Delta_X[T x 1],
+// Delta_W[1 x Co]); the per-tensor variants of the page's "standard FP8"
+// comparison (Delta_X[1], Delta_W[1]); and step 2 of the page's naive
+// two-step path (section "The challenge: two-step vs fused").
+//
+// Every code is E4M3_satRNE(fp32_RN(x / s)) with s = fp32_RN(amax / 448).  The
+// division is done without a per-element divide: with r = RN(1/s),
+//   q0 = RN(x * r),  e = x - q0 * s (one FMA, exact),  q = RN(q0 + e * r),
+// the one-step correction of Markstein ("Computation of elementary functions
+// on the IBM RISC System/6000 processor", IBM J. R&D 34(1), 1990).  For
+// s >= 2^-100 this yields the same E4M3 code as the IEEE quotient for every
+// pair of bf16 inputs (checked exhaustively against the CPU definition);
+// groups with a smaller scale take the IEEE division __fdiv_rn instead.
+#include <algorithm>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include "kernels.h"
+
+namespace ptpc {
+
+namespace {
+
+constexpr float kFastPathMinScale = 0x1p-100f;
+
+// Division mode shared by every element of a row / column.
+enum : int { kZeroGroup = 0, kFast = 1, kSlow = 2 };
+
+struct GroupScale {
+  float s;     // dequantisation scale
+  float r;     // RN(1/s) (fast mode only)
+  int mode;
+};
+
+__device__ __forceinline__ GroupScale group_scale_from_amax_bits(uint32_t amax_bits16) {
+  GroupScale g;
+  const float amax = __uint_as_float(amax_bits16 << 16);
+  if (amax == 0.0f) {
+    g.s = 1.0f;
+    g.r = 1.0f;
+    g.mode = kZeroGroup;
+  } else {
+    g.s = __fdiv_rn(amax, 448.0f);
+    g.r = __frcp_rn(g.s);
+    g.mode = g.s >= kFastPathMinScale ? kFast : kSlow;
+  }
+  return g;
+}
+
+__device__ __forceinline__ float quotient(float x, const GroupScale &g) {
+  if (g.mode == kFast) {
+    const float q0 = __fmul_rn(x, g.r);
+    const float e = __fmaf_rn(-q0, g.s, x);
+    return __fmaf_rn(e, g.r, q0);
+  }
+  return __fdiv_rn(x, g.s);
+}
+
+// Two bf16 (low half = first element) -> two E4M3 codes (low byte = first).
+__device__ __forceinline__ uint32_t quant_pair(uint32_t w, const GroupScale &g) {
+  const float lo = __uint_as_float(w << 16);
+  const float hi = __uint_as_float(w & 0xFFFF0000u);
+  float2 q;
+  q.x = quotient(lo, g);
+  q.y = quotient(hi, g);
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Eight bf16 (16 bytes) -> eight codes (8 bytes).
+__device__ __forceinline__ uint2 quant_vec(const uint4 v, const GroupScale &g) {
+  if (g.mode == kZeroGroup) return make_uint2(0u, 0u);
+  uint2 o;
+  o.x = quant_pair(v.x, g) | (quant_pair(v.y, g) << 16);
+  o.y = quant_pair(v.z, g) | (quant_pair(v.w, g) << 16);
+  return o;
+}
+
+// max(|bf16|) as 16-bit magnitude bits, two lanes per 32-bit word.  For
+// finite values the order of the magnitude bits is the order of the values.
+__device__ __forceinline__ uint32_t absmax_bits(uint32_t acc, uint4 v) {
+  acc = __vmaxu2(acc, v.x & 0x7FFF7FFFu);
+  acc = __vmaxu2(acc, v.y & 0x7FFF7FFFu);
+  acc = __vmaxu2(acc, v.z & 0x7FFF7FFFu);
+  acc = __vmaxu2(acc, v.w & 0x7FFF7FFFu);
+  return acc;
+}
+
+__device__ __forceinline__ uint32_t fold_halves(uint32_t m) { return max(m & 0xFFFFu, m >> 16); }
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
+
+// ----------------------------------------------------------------------------
+// Per-token activation quantisation.
+//
+// A group of P threads (a multiple of 32) owns one row; each thread holds V
+// 16-byte vectors of the row in registers, so the row is read from HBM once:
+// load, |x| max, group reduction (warp shuffle, then shared memory across
+// the group's warps), then quantise from registers and store 8 codes per
+// vector.  R = blockDim / P rows per CTA.
+// PER_TENSOR: the group scale comes from a tensor-wide amax computed by
+// amax_kernel (the per-tensor comparison path) instead of the row.
+// ----------------------------------------------------------------------------
+template <int V, bool PER_TENSOR>
+__global__ void __launch_bounds__(1024) quant_act_kernel(const uint4 *__restrict__ X, int T, int nvec,
+                                                         uint8_t *__restrict__ Xq, float *__restrict__ xs,
+                                                         int P, const uint32_t *__restrict__ tensor_amax) {
+  __shared__ uint32_t red[32];
+  griddep_launch_dependents();
+
+  const int tid = threadIdx.x;
+  const int rl = tid / P;
+  const int lt = tid - rl * P;
+  const int rows_per_cta = blockDim.x / P;
+  const int64_t row = (int64_t)blockIdx.x * rows_per_cta + rl;
+  const bool active = row < T;
+  const uint4 *xr = X + row * nvec;
+
+  uint4 v[V];
+  uint32_t m = 0;
+  #pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int j = lt + i * P;
+    if (active && j < nvec) {
+      v[i] = ld_stream(xr + j);
+    } else {
+      v[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  uint32_t amax_bits;
+  if constexpr (PER_TENSOR) {
+    amax_bits = *tensor_amax;
+  } else {
+    #pragma unroll
+    for (int i = 0; i < V; ++i) m = absmax_bits(m, v[i]);
+    m = __reduce_max_sync(0xffffffffu, fold_halves(m));
+    const int warps_per_row = P >> 5;
+    if (warps_per_row > 1) {
+      if ((tid & 31) == 0) red[tid >> 5] = m;
+      __syncthreads();
+      m = 0;
+      const int w0 = rl * warps_per_row;
+      for (int w = 0; w < warps_per_row; ++w) m = max(m, red[w0 + w]);
+    }
+    amax_bits = m;
+  }
+  const GroupScale g = group_scale_from_amax_bits(amax_bits);
+  if (!active) return;
+  if (lt == 0) xs[row] = g.s;
+
+  uint2 *qr = reinterpret_cast<uint2 *>(Xq + row * (int64_t)nvec * 8);
+  #pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int j = lt + i * P;
+    if (j < nvec) qr[j] = quant_vec(v[i], g);
+  }
+}
+
+// Rows too long for registers: two passes over the row (the second read is
+// normally served from L2).  One CTA per row.
+template <bool PER_TENSOR>
+__global__ void __launch_bounds__(1024) quant_act_long_kernel(const uint4 *__restrict__ X, int T, int nvec,
+                                                              uint8_t *__restrict__ Xq, float *__restrict__ xs,
+                                                              const uint32_t *__restrict__ tensor_amax) {
+  __shared__ uint32_t red[32];
+  __shared__ uint32_t row_amax;
+  griddep_launch_dependents();
+  const int64_t row = blockIdx.x;
+  const uint4 *xr = X + row * nvec;
+  uint32_t amax_bits;
+  if constexpr (PER_TENSOR) {
+    amax_bits = *tensor_amax;
+  } else {
+    uint32_t m = 0;
+    for (int j = threadIdx.x; j < nvec; j += blockDim.x) m = absmax_bits(m, xr[j]);
+    m = __reduce_max_sync(0xffffffffu, fold_halves(m));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t mm = 0;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) mm = max(mm, red[w]);
+      row_amax = mm;
+    }
+    __syncthreads();
+    amax_bits = row_amax;
+  }
+  const GroupScale g = group_scale_from_amax_bits(amax_bits);
+  if (threadIdx.x == 0) xs[row] = g.s;
+  uint2 *qr = reinterpret_cast<uint2 *>(Xq + row * (int64_t)nvec * 8);
+  for (int j = threadIdx.x; j < nvec; j += blockDim.x) qr[j] = quant_vec(ld_stream(xr + j), g);
+}
+
+// Tensor-wide max |x| of n8 16-byte vectors, as bf16 magnitude bits, into
+// *amax (atomicMax; *amax must be 0 beforehand).
+__global__ void __launch_bounds__(512) amax_kernel(const uint4 *__restrict__ X, int64_t n8,
+                                                   uint32_t *__restrict__ amax) {
+  uint32_t m = 0;
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n8; j += (int64_t)gridDim.x * blockDim.x)
+    m = absmax_bits(m, ld_stream(X + j));
+  m = __reduce_max_sync(0xffffffffu, fold_halves(m));
+  if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(amax, m);
+}
+
+// ----------------------------------------------------------------------------
+// Per-output-channel weight quantisation, pass 1: column maxima.
+// W is Ci x Co row-major.  Each thread owns 8 adjacent columns (one 16-byte
+// vector per row) and walks a slab of rows; the CTA's warps split the slab;
+// the result is merged with atomicMax into col_amax[Co] (zeroed beforehand).
+// ----------------------------------------------------------------------------
+constexpr int kColThreads = 32;   // vectors (8 columns each) per CTA row
+constexpr int kColWarps = 8;
+
+__global__ void __launch_bounds__(kColThreads * kColWarps) col_amax_kernel(const uint4 *__restrict__ W, int Ci,
+                                                                            int Co, int rows_per_cta,
+                                                                            uint32_t *__restrict__ col_amax) {
+  __shared__ uint32_t red[kColWarps][kColThreads][4];
+  const int ncv = Co / 8;
+  const int cv = blockIdx.x * kColThreads + (threadIdx.x & 31);
+  const int warp = threadIdx.x >> 5;
+  const int k0 = blockIdx.y * rows_per_cta;
+  const int k1 = min(Ci, k0 + rows_per_cta);
+  uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+  if (cv < ncv) {
+    for (int k = k0 + warp; k < k1; k += kColWarps) {
+      const uint4 v = ld_stream(W + (int64_t)k * ncv + cv);
+      m0 = __vmaxu2(m0, v.x & 0x7FFF7FFFu);
+      m1 = __vmaxu2(m1, v.y & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v.z & 0x7FFF7FFFu);
+      m3 = __vmaxu2(m3, v.w & 0x7FFF7FFFu);
+    }
+  }
+  red[warp][threadIdx.x & 31][0] = m0;
+  red[warp][threadIdx.x & 31][1] = m1;
+  red[warp][threadIdx.x & 31][2] = m2;
+  red[warp][threadIdx.x & 31][3] = m3;
+  __syncthreads();
+  if (warp == 0 && cv < ncv) {
+    const int l = threadIdx.x & 31;
+    #pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t mm = 0;
+      for (int w = 0; w < kColWarps; ++w) mm = __vmaxu2(mm, red[w][l][q]);
+      const int col = cv * 8 + q * 2;
+      if ((mm & 0xFFFFu) != 0) atomicMax(col_amax + col, mm & 0xFFFFu);
+      if ((mm >> 16) != 0) atomicMax(col_amax + col + 1, mm >> 16);
+    }
+  }
+}
+
+// Tensor-wide amax broadcast into every column's slot (per-tensor weights).
+__global__ void broadcast_amax_kernel(const uint32_t *__restrict__ src, uint32_t *__restrict__ dst, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = *src;
+}
+
+// ----------------------------------------------------------------------------
+// Weight quantisation, pass 2: quantise a 64 (k) x 64 (o) tile of W with its
+// columns' scales and write it transposed into Wq_t (Co x Ci).  The tile is
+// staged in shared memory as codes [o][k] so both the bf16 reads (along o)
+// and the code writes (along k) are coalesced.
+// ----------------------------------------------------------------------------
+constexpr int kTT = 64;
+
+__global__ void __launch_bounds__(256) quant_weight_t_kernel(const uint4 *__restrict__ W, int Ci, int Co,
+                                                             const uint32_t *__restrict__ col_amax,
+                                                             uint8_t *__restrict__ Wq_t,
+                                                             float *__restrict__ w_scale) {
+  __shared__ uint8_t tile[kTT][kTT + 4];
+  const int o0 = blockIdx.x * kTT;
+  const int k0 = blockIdx.y * kTT;
+  const int ncv = Co / 8;
+  // each thread: one 8-column vector (8 per row of 64 columns), rows step 32
+  const int cvl = threadIdx.x & 7;     // vector within the tile row
+  const int kr = threadIdx.x >> 3;     // 0..31
+  const int ocol = o0 + cvl * 8;
+  GroupScale g[8];
+  #pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const int o = ocol + c;
+    g[c] = group_scale_from_amax_bits(o < Co ? col_amax[o] : 0u);
+  }
+  if (blockIdx.y == 0 && kr == 0) {
+    #pragma unroll
+    for (int c = 0; c < 8; ++c)
+      if (ocol + c < Co) w_scale[ocol + c] = g[c].s;
+  }
+  #pragma unroll
+  for (int rr = 0; rr < kTT; rr += 32) {
+    const int k = k0 + kr + rr;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (k < Ci && ocol < Co) v = ld_stream(W + (int64_t)k * ncv + (ocol >> 3));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    #pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      GroupScale ga = g[2 * h], gb = g[2 * h + 1];
+      const float lo = __uint_as_float(w[h] << 16);
+      const float hi = __uint_as_float(w[h] & 0xFFFF0000u);
+      float2 q;
+      q.x = quotient(lo, ga);
+      q.y = quotient(hi, gb);
+      uint32_t codes = (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
+      if (ga.mode == kZeroGroup) codes &= 0xFF00u;
+      if (gb.mode == kZeroGroup) codes &= 0x00FFu;
+      tile[cvl * 8 + 2 * h][kr + rr] = (uint8_t)(codes & 0xFFu);
+      tile[cvl * 8 + 2 * h + 1][kr + rr] = (uint8_t)(codes >> 8);
+    }
+  }
+  __syncthreads();
+  // write: 64 rows (o) x 64 bytes (k): each thread writes 16 bytes
+  const int orow = threadIdx.x >> 2;        // 0..63
+  const int kc = (threadIdx.x & 3) * 16;    // 0,16,32,48
+  const int o = o0 + orow;
+  const int k = k0 + kc;
+  if (o < Co && k < Ci) {
+    uint32_t pk[4];
+    #pragma unroll
+    for (int q = 0; q < 4; ++q)
+      pk[q] = (uint32_t)tile[orow][kc + 4 * q] | ((uint32_t)tile[orow][kc + 4 * q + 1] << 8) |
+              ((uint32_t)tile[orow][kc + 4 * q + 2] << 16) | ((uint32_t)tile[orow][kc + 4 * q + 3] << 24);
+    *reinterpret_cast<uint4 *>(Wq_t + (int64_t)o * Ci + k) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Naive two-step path, step 2: out = bf16((y * x_scale[t]) * w_scale[o]).
+// Each thread handles 8 consecutive outputs (two 16-byte fp32 loads, one
+// 16-byte bf16 store).
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) apply_scales_kernel(const float4 *__restrict__ y, int T, int Co,
+                                                           const float *__restrict__ xs,
+                                                           const float *__restrict__ ws,
+                                                           uint4 *__restrict__ out) {
+  const int nv = Co / 8;
+  const int64_t total = (int64_t)T * nv;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / nv;
+    const int c = (int)(i - t * nv) * 8;
+    const float a = xs[t];
+    const float4 y0 = __ldcs(y + 2 * i);
+    const float4 y1 = __ldcs(y + 2 * i + 1);
+    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(ws + c));
+    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(ws + c + 4));
+    const float v[8] = {__fmul_rn(__fmul_rn(y0.x, a), w0.x), __fmul_rn(__fmul_rn(y0.y, a), w0.y),
+                        __fmul_rn(__fmul_rn(y0.z, a), w0.z), __fmul_rn(__fmul_rn(y0.w, a), w0.w),
+                        __fmul_rn(__fmul_rn(y1.x, a), w1.x), __fmul_rn(__fmul_rn(y1.y, a), w1.y),
+                        __fmul_rn(__fmul_rn(y1.z, a), w1.z), __fmul_rn(__fmul_rn(y1.w, a), w1.w)};
+    uint32_t p[4];
+    #pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+      p[q] = *reinterpret_cast<uint32_t *>(&b);
+    }
+    out[i] = make_uint4(p[0], p[1], p[2], p[3]);
+  }
+}
+
+// Launch shape of the register-resident activation quantiser.
+struct ActPlan {
+  int V;    // vectors per thread (0: use the two-pass kernel)
+  int P;    // threads per row
+  int R;    // rows per CTA
+};
+
+ActPlan plan_act(int nvec) {
+  ActPlan p{0, 0, 0};
+  auto roundup32 = [](int x) { return (x + 31) / 32 * 32; };
+  if (nvec <= 32 * 8) {
+    int v = (nvec + 31) / 32;
+    p.V = v <= 1 ? 1 : v <= 2 ? 2 : v <= 4 ? 4 : 8;
+    p.P = 32;
+  } else if (roundup32((nvec + 7) / 8) <= 1024) {
+    p.V = 8;
+    p.P = roundup32((nvec + 7) / 8);
+  } else if (roundup32((nvec + 15) / 16) <= 1024) {
+    p.V = 16;
+    p.P = roundup32((nvec + 15) / 16);
+  } else {
+    return p;
+  }
+  p.R = p.P >= 256 ? 1 : 256 / p.P;
+  return p;
+}
+
+template <bool PT>
+cudaError_t launch_act(const void *X, int T, int Ci, uint8_t *Xq, float *xs, const uint32_t *tensor_amax,
+                       cudaStream_t st) {
+  const int nvec = Ci / 8;
+  const ActPlan p = plan_act(nvec);
+  const uint4 *Xv = static_cast<const uint4 *>(X);
+  if (p.V == 0) {
+    quant_act_long_kernel<PT><<<T, 1024, 0, st>>>(Xv, T, nvec, Xq, xs, tensor_amax);
+    return cudaGetLastError();
+  }
+  const int grid = (T + p.R - 1) / p.R;
+  const int block = p.P * p.R;
+  switch (p.V) {
+    case 1: quant_act_kernel<1, PT><<<grid, block, 0, st>>>(Xv, T, nvec, Xq, xs, p.P, tensor_amax); break;
+    case 2: quant_act_kernel<2, PT><<<grid, block, 0, st>>>(Xv, T, nvec, Xq, xs, p.P, tensor_amax); break;
+    case 4: quant_act_kernel<4, PT><<<grid, block, 0, st>>>(Xv, T, nvec, Xq, xs, p.P, tensor_amax); break;
+    case 8: quant_act_kernel<8, PT><<<grid, block, 0, st>>>(Xv, T, nvec, Xq, xs, p.P, tensor_amax); break;
+    default: quant_act_kernel<16, PT><<<grid, block, 0, st>>>(Xv, T, nvec, Xq, xs, p.P, tensor_amax); break;
+  }
+  return cudaGetLastError();
+}
+
+int num_sms_cached() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+cudaError_t launch_quant_act(const void *X, int T, int Ci, uint8_t *Xq, float *xs, cudaStream_t st) {
+  return launch_act<false>(X, T, Ci, Xq, xs, nullptr, st);
+}
+
+cudaError_t launch_quant_act_per_tensor(const void *X, int T, int Ci, uint8_t *Xq, float *xs, uint32_t *amax_slot,
+                                        cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(amax_slot, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return e;
+  const int64_t n8 = (int64_t)T * Ci / 8;
+  int grid = (int)std::min<int64_t>((n8 + 511) / 512, (int64_t)num_sms_cached() * 4);
+  if (grid < 1) grid = 1;
+  amax_kernel<<<grid, 512, 0, st>>>(static_cast<const uint4 *>(X), n8, amax_slot);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return launch_act<true>(X, T, Ci, Xq, xs, amax_slot, st);
+}
+
+cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, float *w_scale, uint32_t *col_amax,
+                                bool per_tensor, cudaStream_t st) {
+  cudaError_t e;
+  const uint4 *Wv = static_cast<const uint4 *>(W);
+  if (per_tensor) {
+    uint32_t *slot = col_amax + Co;
+    if ((e = cudaMemsetAsync(slot, 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
+    const int64_t n8 = (int64_t)Ci * Co / 8;
+    int grid = (int)std::min<int64_t>((n8 + 511) / 512, (int64_t)num_sms_cached() * 4);
+    amax_kernel<<<grid, 512, 0, st>>>(Wv, n8, slot);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    broadcast_amax_kernel<<<(Co + 255) / 256, 256, 0, st>>>(slot, col_amax, Co);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else {
+    if ((e = cudaMemsetAsync(col_amax, 0, sizeof(uint32_t) * (size_t)Co, st)) != cudaSuccess) return e;
+    const int ncv = Co / 8;
+    const int gx = (ncv + kColThreads - 1) / kColThreads;
+    // enough row slabs to fill the GPU a few times over
+    int slabs = std::max(1, (num_sms_cached() * 4 + gx - 1) / gx);
+    int rows_per_cta = (Ci + slabs - 1) / slabs;
+    rows_per_cta = std::max(rows_per_cta, 64);
+    slabs = (Ci + rows_per_cta - 1) / rows_per_cta;
+    col_amax_kernel<<<dim3(gx, slabs), kColThreads * kColWarps, 0, st>>>(Wv, Ci, Co, rows_per_cta, col_amax);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  dim3 grid((Co + kTT - 1) / kTT, (Ci + kTT - 1) / kTT);
+  quant_weight_t_kernel<<<grid, 256, 0, st>>>(Wv, Ci, Co, col_amax, Wq_t, w_scale);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_apply_scales(const float *y, const float *xs, const float *ws, int T, int Co, void *out,
+                                cudaStream_t st) {
+  const int64_t total = (int64_t)T * (Co / 8);
+  int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)num_sms_cached() * 8);
+  if (grid < 1) grid = 1;
+  apply_scales_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4 *>(y), T, Co, xs, ws,
+                                            static_cast<uint4 *>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace ptpc

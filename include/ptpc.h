@@ -1,0 +1,186 @@
+/*
+ * ptpc.h - C ABI of the PTPC-FP8 library for NVIDIA B200 (sm_100a).
+ *
+ * PTPC-FP8 = per-token activation, per-channel weight FP8 quantisation
+ * ("PTPC-FP8: boosting vLLM performance on AMD ROCm", vLLM blog, sections
+ * "What is PTPC-FP8" and "Per-Token Activation + Per-Channel Weight
+ * Quantization").  The activation X is T x Ci (T tokens, Ci input channels),
+ * the weight W is Ci x Co (Co output channels); X gets one scale per token
+ * (Delta_X[T x 1]) and W one scale per output column (Delta_W[1 x Co]).  The
+ * GEMM applies token_scale[t] * channel_scale[o] inside its epilogue, before
+ * the single store of the result (section "The challenge: two-step vs fused",
+ * the fused `_scaled_mm(input, weight, scale_a=token_scales,
+ * scale_b=channel_scales)`).
+ *
+ * Number formats (the page names none; these are this library's readings):
+ *   - FP8 codes are OCP E4M3 ("e4m3fn", bias 7, max 448, no infinities).
+ *   - scale = amax / 448 as an IEEE fp32 division, round-to-nearest-even;
+ *     an all-zero row/column gets scale 1.0f and all codes 0x00.
+ *   - code = saturating round-half-to-even E4M3 of the fp32 quotient x / scale.
+ *   - out[t][o] = bf16_RNE((acc[t][o] * x_scale[t]) * w_scale[o]), acc the
+ *     fp32 tensor-core sum of the decoded code products.
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers named *_dev are device pointers; every buffer is owned by the
+ *     caller.  The library never allocates or frees device memory.
+ *   - Layouts are dense row-major.  bf16 tensors are passed as raw 16-bit
+ *     patterns (void*).
+ *   - Alignment: every device pointer must be 16-byte aligned
+ *     (PTPC_ERR_MISALIGNED otherwise).
+ *   - Shapes: T >= 0 (T == 0 is a no-op returning PTPC_OK); Ci and Co must be
+ *     positive multiples of 16 (PTPC_ERR_UNSUPPORTED_SHAPE otherwise), and
+ *     T, Ci, Co must each fit in 31 bits.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *     only enqueues work on it and returns; none synchronises, except
+ *     ptpc_get_device_status.
+ *   - Errors: the return value is a ptpc_status.  All argument checks run
+ *     before any launch; a failed check launches nothing.  A failed launch
+ *     returns PTPC_ERR_CUDA.  No C++ exception crosses this boundary.
+ *   - Workspace: entry points that take (ws_dev, ws_bytes) need at least
+ *     ptpc_workspace_size(op, T, Ci, Co) bytes, zero-filled before its first
+ *     use.  Each successful call leaves the workspace's control words zero
+ *     again, so a workspace is zero-filled only once.  Calls that share a
+ *     workspace must not overlap on the GPU.
+ *   - Inputs are assumed finite.  Non-finite inputs do not fault but give
+ *     unspecified codes.
+ */
+#ifndef PTPC_H_
+#define PTPC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PTPC_API __attribute__((visibility("default")))
+#else
+#define PTPC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PTPC_OK = 0,
+    PTPC_ERR_INVALID_ARG = 1,          /* null pointer, negative size, unknown op */
+    PTPC_ERR_MISALIGNED = 2,           /* a pointer is not 16-byte aligned */
+    PTPC_ERR_UNSUPPORTED_SHAPE = 3,    /* Ci or Co not a positive multiple of 16, or too large */
+    PTPC_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes < ptpc_workspace_size(...) */
+    PTPC_ERR_UNSUPPORTED_DEVICE = 5,   /* current device is not compute capability 10.0 */
+    PTPC_ERR_CUDA = 6,                 /* a CUDA runtime/driver call failed */
+    PTPC_ERR_DEVICE_TIMEOUT = 7,       /* a kernel's bounded wait ran out (device status word) */
+    PTPC_ERR_NOT_IMPLEMENTED = 8
+} ptpc_status;
+
+/* Operation ids for ptpc_workspace_size. */
+typedef enum {
+    PTPC_OP_QUANTIZE_WEIGHTS = 1,
+    PTPC_OP_SCALED_MM = 2,
+    PTPC_OP_LINEAR = 3,
+    PTPC_OP_BENCH_PER_TENSOR = 4,      /* per-tensor quantisers (measurement only) */
+    PTPC_OP_BENCH_UNSCALED_MM = 5      /* unscaled fp32 GEMM (measurement only) */
+} ptpc_op;
+
+/* Per-token activation quantisation (the page's Delta_X[T x 1]).
+ *   X_dev       bf16 [T, Ci] row-major, read only.
+ *   Xq_dev      u8   [T, Ci] row-major, written: E4M3 codes of row t with
+ *               scale x_scale[t] (the K-major A operand of the GEMM).
+ *   x_scale_dev fp32 [T], written: amax(|X[t, :]|) / 448 (1.0f if amax == 0).
+ * Codes and scales are bit-exact functions of X (see the conventions above). */
+PTPC_API int ptpc_quantize_activations(const void *X_dev, int64_t T, int64_t Ci,
+                              uint8_t *Xq_dev, float *x_scale_dev, void *stream);
+
+/* Per-output-channel weight quantisation (the page's Delta_W[1 x Co]); run
+ * once per weight, e.g. when a bf16 checkpoint is loaded.
+ *   W_dev       bf16 [Ci, Co] row-major, read only.
+ *   Wq_t_dev    u8   [Co, Ci] row-major, written: codes of column o of W,
+ *               transposed so that each output channel's codes are
+ *               contiguous along Ci (the K-major B operand of the GEMM).
+ *   w_scale_dev fp32 [Co], written: amax(|W[:, o]|) / 448 (1.0f if 0).
+ *   ws_dev      workspace of ptpc_workspace_size(PTPC_OP_QUANTIZE_WEIGHTS, 0, Ci, Co)
+ *               bytes (column maxima). */
+PTPC_API int ptpc_quantize_weights(const void *W_dev, int64_t Ci, int64_t Co,
+                          uint8_t *Wq_t_dev, float *w_scale_dev,
+                          void *ws_dev, size_t ws_bytes, void *stream);
+
+/* Fused row-wise-scaled FP8 GEMM (the page's fused `_scaled_mm` with
+ * scale_a = token scales, scale_b = channel scales):
+ *   out[t][o] = bf16_RNE((sum_k dec(Xq[t][k]) * dec(Wq_t[o][k]) * x_scale[t]) * w_scale[o])
+ *   Xq_dev      u8 [T, Ci], x_scale_dev fp32 [T]   (from ptpc_quantize_activations)
+ *   Wq_t_dev    u8 [Co, Ci], w_scale_dev fp32 [Co] (from ptpc_quantize_weights)
+ *   out_dev     bf16 [T, Co] row-major, written once (no intermediate array).
+ *   ws_dev      ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co) bytes: device
+ *               status word, split-K tile counters and fp32 partial sums.
+ * The sum over k is an fp32 tensor-core accumulation; its order is not
+ * specified.  Small T uses a split-K variant whose partial sums are reduced
+ * in a fixed order, so results are deterministic for a given shape. */
+PTPC_API int ptpc_scaled_mm(const uint8_t *Xq_dev, const float *x_scale_dev,
+                   const uint8_t *Wq_t_dev, const float *w_scale_dev,
+                   int64_t T, int64_t Ci, int64_t Co, void *out_dev,
+                   void *ws_dev, size_t ws_bytes, void *stream);
+
+/* Fused quantise + GEMM: ptpc_quantize_activations of X into the workspace,
+ * then ptpc_scaled_mm, on one stream (the GEMM is launched as a programmatic
+ * dependent of the quantiser).  The page's path with "no pre-quantization":
+ * the bf16 activation goes in, the bf16 output comes out.
+ *   X_dev bf16 [T, Ci]; Wq_t_dev / w_scale_dev as for ptpc_scaled_mm;
+ *   out_dev bf16 [T, Co];
+ *   ws_dev ptpc_workspace_size(PTPC_OP_LINEAR, T, Ci, Co) bytes (holds Xq and
+ *   x_scale as well as the GEMM's workspace). */
+PTPC_API int ptpc_linear(const void *X_dev, const uint8_t *Wq_t_dev, const float *w_scale_dev,
+                int64_t T, int64_t Ci, int64_t Co, void *out_dev,
+                void *ws_dev, size_t ws_bytes, void *stream);
+
+/* Bytes of workspace an entry point needs for the given shape (0 on invalid
+ * arguments).  The value is a multiple of 256. */
+PTPC_API size_t ptpc_workspace_size(int op, int64_t T, int64_t Ci, int64_t Co);
+
+/* Synchronises `stream`, reads the device status word at the start of ws_dev
+ * (written by kernels whose bounded waits ran out), clears it and returns
+ * PTPC_OK or PTPC_ERR_DEVICE_TIMEOUT (PTPC_ERR_CUDA if the read fails). */
+PTPC_API int ptpc_get_device_status(void *ws_dev, void *stream);
+
+/* Static, human-readable name of a status code. */
+PTPC_API const char *ptpc_status_string(int status);
+
+/* ------------------------------------------------------------------------- */
+/* Measurement-only entry points: the comparison paths the page describes.  */
+/* ------------------------------------------------------------------------- */
+
+/* Naive two-step path, step 1 (section "The challenge: two-step vs fused",
+ * `output = torch._scaled_mm(input, weight)`): the unscaled FP8 GEMM written
+ * out as an fp32 intermediate y_dev [T, Co] row-major.  Same mainloop as
+ * ptpc_scaled_mm, so y is bit-identical to that kernel's accumulator.
+ * ws_dev: ptpc_workspace_size(PTPC_OP_BENCH_UNSCALED_MM, T, Ci, Co) bytes. */
+PTPC_API int ptpc_bench_unscaled_mm_f32(const uint8_t *Xq_dev, const uint8_t *Wq_t_dev,
+                               int64_t T, int64_t Ci, int64_t Co, float *y_dev,
+                               void *ws_dev, size_t ws_bytes, void *stream);
+
+/* Naive two-step path, step 2 (`output = output * token_scales *
+ * channel_scales`): reads y_dev fp32 [T, Co] and writes
+ * out_dev[t][o] = bf16_RNE((y[t][o] * x_scale[t]) * w_scale[o]). */
+PTPC_API int ptpc_bench_apply_scales(const float *y_dev, const float *x_scale_dev,
+                            const float *w_scale_dev, int64_t T, int64_t Co,
+                            void *out_dev, void *stream);
+
+/* Per-tensor ("standard FP8", the page's Delta_X[1] / Delta_W[1]) activation
+ * quantisation: one scale for all of X.  Writes the codes to Xq_dev [T, Ci]
+ * and that one scale to every entry of x_scale_dev [T], so ptpc_scaled_mm can
+ * consume the result unchanged.  ws_dev: ptpc_workspace_size(
+ * PTPC_OP_BENCH_PER_TENSOR, T, Ci, 0) bytes. */
+PTPC_API int ptpc_bench_quantize_activations_per_tensor(const void *X_dev, int64_t T, int64_t Ci,
+                                               uint8_t *Xq_dev, float *x_scale_dev,
+                                               void *ws_dev, size_t ws_bytes, void *stream);
+
+/* Per-tensor weight quantisation: one scale for all of W (Ci x Co), codes
+ * transposed to Wq_t_dev [Co, Ci], the scale written to every entry of
+ * w_scale_dev [Co].  ws_dev as for ptpc_quantize_weights. */
+PTPC_API int ptpc_bench_quantize_weights_per_tensor(const void *W_dev, int64_t Ci, int64_t Co,
+                                           uint8_t *Wq_t_dev, float *w_scale_dev,
+                                           void *ws_dev, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PTPC_H_ */

@@ -1,0 +1,100 @@
+"""The C-ABI library loads, exports every symbol include/ptpc.h declares, and
+rejects bad arguments before touching the GPU (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def ptpc():
+    from fp8_quantized_gemm_ptpc_b200 import build
+    build.build()
+    import fp8_quantized_gemm_ptpc_b200 as p
+    return p
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "ptpc.h")).read()
+    return sorted(set(re.findall(r"PTPC_API[^;(]*?\b(ptpc_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for n in ["ptpc_quantize_activations", "ptpc_quantize_weights", "ptpc_scaled_mm", "ptpc_linear",
+              "ptpc_workspace_size", "ptpc_get_device_status", "ptpc_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(ptpc):
+    lib = ctypes.CDLL(ptpc.LIB_PATH)
+    for n in declared_symbols():
+        assert hasattr(lib, n), n
+    assert set(declared_symbols()) == set(ptpc.SIGNATURES)
+
+
+def test_status_strings(ptpc):
+    assert ptpc.status_string(0) == "PTPC_OK"
+    assert ptpc.status_string(ptpc.ERR_DEVICE_TIMEOUT) == "PTPC_ERR_DEVICE_TIMEOUT"
+    assert ptpc.status_string(999) == "PTPC_ERR_UNKNOWN"
+
+
+def test_workspace_sizes(ptpc):
+    ws = ptpc.workspace_size
+    assert ws(ptpc.OP_SCALED_MM, 2048, 4096, 6144) % 256 == 0
+    assert ws(ptpc.OP_SCALED_MM, 2048, 4096, 6144) >= 256
+    assert ws(ptpc.OP_LINEAR, 2048, 4096, 6144) >= ws(ptpc.OP_SCALED_MM, 2048, 4096, 6144) + 2048 * 4096
+    assert ws(ptpc.OP_QUANTIZE_WEIGHTS, 0, 4096, 6144) >= 256 + 4 * 6145
+    assert ws(ptpc.OP_SCALED_MM, 16, 100, 64) == 0          # Ci not a multiple of 16
+    assert ws(ptpc.OP_SCALED_MM, -1, 128, 64) == 0
+    assert ws(99, 16, 128, 64) == 0
+    # decode sizes carry room for split-K partial sums
+    assert ws(ptpc.OP_SCALED_MM, 1, 28672, 8192) > 256 + 4 * 64
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: checks fail before any access
+
+
+def call(ptpc, name, *args):
+    return getattr(ptpc.lib, name)(*args)
+
+
+def test_argument_checks_without_gpu(ptpc):
+    P = ctypes.c_void_p
+    q = lambda *a: call(ptpc, "ptpc_quantize_activations", *a)
+    assert q(P(FAKE), 16, 100, P(FAKE), P(FAKE), None) == ptpc.ERR_UNSUPPORTED_SHAPE
+    assert q(P(FAKE), -1, 128, P(FAKE), P(FAKE), None) == ptpc.ERR_INVALID_ARG
+    assert q(None, 16, 128, P(FAKE), P(FAKE), None) == ptpc.ERR_INVALID_ARG
+    assert q(P(FAKE + 8), 16, 128, P(FAKE), P(FAKE), None) == ptpc.ERR_MISALIGNED
+    assert q(None, 0, 128, None, None, None) == ptpc.OK          # T == 0: no-op
+    mm = lambda *a: call(ptpc, "ptpc_scaled_mm", *a)
+    need = ptpc.workspace_size(ptpc.OP_SCALED_MM, 16, 128, 64)
+    assert mm(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 16, 128, 64, P(FAKE), P(FAKE), need - 1, None) == \
+        ptpc.ERR_WORKSPACE_TOO_SMALL
+    assert mm(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 16, 128, 60, P(FAKE), P(FAKE), need, None) == \
+        ptpc.ERR_UNSUPPORTED_SHAPE
+    assert mm(P(FAKE), P(FAKE), P(FAKE), P(FAKE + 4), 16, 128, 64, P(FAKE), P(FAKE), need, None) == \
+        ptpc.ERR_MISALIGNED
+    assert mm(P(FAKE), None, P(FAKE), P(FAKE), 16, 128, 64, P(FAKE), P(FAKE), need, None) == \
+        ptpc.ERR_INVALID_ARG
+    lin = lambda *a: call(ptpc, "ptpc_linear", *a)
+    need = ptpc.workspace_size(ptpc.OP_LINEAR, 16, 128, 64)
+    assert lin(P(FAKE), P(FAKE), P(FAKE), 16, 128, 64, P(FAKE), P(FAKE), need - 256, None) == \
+        ptpc.ERR_WORKSPACE_TOO_SMALL
+    assert lin(None, None, None, 0, 128, 64, None, None, 0, None) == ptpc.OK
+    qw = lambda *a: call(ptpc, "ptpc_quantize_weights", *a)
+    need = ptpc.workspace_size(ptpc.OP_QUANTIZE_WEIGHTS, 0, 128, 64)
+    assert qw(P(FAKE), 128, 64, P(FAKE), P(FAKE), P(FAKE), need - 1, None) == ptpc.ERR_WORKSPACE_TOO_SMALL
+    assert qw(P(FAKE), 128, 0, P(FAKE), P(FAKE), P(FAKE), need, None) == ptpc.ERR_UNSUPPORTED_SHAPE
+    assert call(ptpc, "ptpc_get_device_status", None, None) == ptpc.ERR_INVALID_ARG
+    assert call(ptpc, "ptpc_bench_apply_scales", P(FAKE), P(FAKE), P(FAKE), -3, 64, P(FAKE), None) == \
+        ptpc.ERR_INVALID_ARG
+
+
+def test_binding_rejects_cpu_tensors(ptpc):
+    import torch
+    with pytest.raises(TypeError):
+        ptpc.quantize_activations(torch.zeros(4, 16, dtype=torch.bfloat16))

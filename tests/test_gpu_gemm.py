@@ -1,0 +1,164 @@
+"""GPU parity of the scaled GEMM, the fused entry and the comparison paths.
+
+Outputs are compared with the oracle's fp64-accumulated reference rounded to
+bf16, element by element, within |gpu - ref| <= 1e-2 |ref| + 1e-3 rms(ref).
+The GPU quantises its own inputs; the test also checks those codes are the
+oracle's, so both sides work from the same operands."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from helpers import assert_gemm_close, from_dev_bf16, to_dev, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ptpc():
+    import fp8_quantized_gemm_ptpc_b200 as p
+    return p
+
+
+def run_pair(ptpc, X, W, rows=None, check_linear=True):
+    """GPU: quantize_weights, quantize_activations, scaled_mm (and linear).
+    Oracle: the same three steps.  Returns (gpu_out, ref_out) bf16 bits."""
+    Xd, Wd = to_dev_bf16(X), to_dev_bf16(W)
+    Wq_t, ws = ptpc.quantize_weights(Wd)
+    Xq, xs = ptpc.quantize_activations(Xd)
+    out = ptpc.scaled_mm(Xq, xs, Wq_t, ws)
+    rWq, rws = oracle.quant_weight(W)
+    rXq, rxs = oracle.quant_act(X)
+    assert np.array_equal(Wq_t.cpu().numpy(), rWq) and np.array_equal(Xq.cpu().numpy(), rXq)
+    ref = oracle.scaled_mm_reference(rXq, rxs, rWq, rws, rows)
+    g = from_dev_bf16(out)
+    if check_linear:
+        lin = ptpc.linear(Xd, Wq_t, ws)
+        assert torch.equal(lin.view(torch.int16), out.view(torch.int16)), "linear != quantize + scaled_mm"
+    return (g if rows is None else g[rows]), ref
+
+
+def test_tiny_workload(ptpc):
+    w = synthetic.TINY
+    g, r = run_pair(ptpc, synthetic.make_x(w, 0, 16, 256), synthetic.make_w(w, 0, 256, 512))
+    assert_gemm_close(g, r, "tiny")
+
+
+@pytest.mark.parametrize("T,Ci,Co", [
+    (1, 16, 16), (2, 32, 48), (7, 128, 256), (77, 384, 528), (129, 256, 272), (300, 640, 1040),
+    (1000, 1024, 768), (3001, 512, 2064), (128, 4112, 256), (257, 128, 4096),
+])
+def test_ragged_shapes(ptpc, T, Ci, Co):
+    X = synthetic.with_edge_rows(synthetic.make_x(synthetic.LLAMA70B_PREFILL, 0, T, Ci))
+    W = synthetic.random_bf16((Ci, Co), seed=T + Ci + Co, scale=0.02)
+    g, r = run_pair(ptpc, X, W)
+    assert_gemm_close(g, r, f"{T}x{Ci}x{Co}")
+
+
+@pytest.mark.parametrize("layer", [0, 1, 2])
+def test_llama8b_prefill_full(ptpc, layer):
+    w = synthetic.LLAMA8B_PREFILL
+    L = w.layers[layer]
+    g, r = run_pair(ptpc, synthetic.make_x(w, layer, 2048, L.Ci), synthetic.make_w(w, layer, L.Ci, L.Co))
+    assert_gemm_close(g, r, L.name)
+
+
+@pytest.mark.parametrize("T", [1, 8, 32, 128])
+@pytest.mark.parametrize("layer", [0, 1])
+def test_decode_full(ptpc, T, layer):
+    w = synthetic.DECODE_70B
+    L = w.layers[layer]
+    g, r = run_pair(ptpc, synthetic.make_x(w, layer, T, L.Ci), synthetic.make_w(w, layer, L.Ci, L.Co))
+    assert_gemm_close(g, r, f"decode {L.name} T={T}")
+
+
+def sample_rows(T, n=256, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = {0, T - 1} | {min(T - 1, b) for b in range(127, T, 128)} | {min(T - 1, b + 1) for b in range(127, T, 128)}
+    rows |= set(rng.choice(T, size=min(T, n), replace=False).tolist())
+    return np.array(sorted(rows)[: max(n, 2)], dtype=np.int64)
+
+
+@pytest.mark.parametrize("layer", [0, 1])
+def test_llama70b_prefill_sampled(ptpc, layer):
+    w = synthetic.LLAMA70B_PREFILL
+    L = w.layers[layer]
+    rows = sample_rows(8192, 192, seed=layer)
+    g, r = run_pair(ptpc, synthetic.make_x(w, layer, 8192, L.Ci), synthetic.make_w(w, layer, L.Ci, L.Co),
+                    rows=rows, check_linear=False)
+    assert_gemm_close(g, r, f"70B {L.name}")
+
+
+@pytest.mark.parametrize("T", [77, 1000, 3001])
+def test_chain_ragged_sampled(ptpc, T):
+    w = synthetic.CHAIN_70B
+    L = w.layers[0]
+    rows = sample_rows(T, 128, seed=T)
+    g, r = run_pair(ptpc, synthetic.make_x(w, 0, T, L.Ci), synthetic.make_w(w, 0, L.Ci, L.Co), rows=rows)
+    assert_gemm_close(g, r, f"chain qkv T={T}")
+
+
+def test_naive_two_step_equals_fused(ptpc):
+    """The page's naive path (GEMM -> fp32 intermediate -> scale) gives the
+    same bits as the fused epilogue: same accumulator, same two products."""
+    for T, Ci, Co in [(300, 1024, 768), (2048, 4096, 6144), (8, 8192, 1024)]:
+        X = synthetic.make_x(synthetic.LLAMA8B_PREFILL, 0, T, Ci)
+        W = synthetic.make_w(synthetic.LLAMA8B_PREFILL, 0, Ci, Co)
+        Wq_t, ws = ptpc.quantize_weights(to_dev_bf16(W))
+        Xq, xs = ptpc.quantize_activations(to_dev_bf16(X))
+        fused = ptpc.scaled_mm(Xq, xs, Wq_t, ws)
+        y = ptpc.unscaled_mm_f32(Xq, Wq_t)
+        naive = ptpc.apply_scales(y, xs, ws)
+        assert torch.equal(fused.view(torch.int16), naive.view(torch.int16)), (T, Ci, Co)
+        # the intermediate itself is the dot product up to fp32 accumulation
+        acc = oracle.gemm_acc64(Xq.cpu().numpy(), Wq_t.cpu().numpy())
+        yy = y.cpu().numpy().astype(np.float64)
+        rms = np.sqrt(np.mean(acc * acc))
+        assert (np.abs(yy - acc) <= 1e-2 * np.abs(acc) + 1e-3 * rms).all()
+
+
+def test_per_tensor_path(ptpc):
+    X = synthetic.make_x(synthetic.LLAMA8B_PREFILL, 0, 300, 1024)
+    W = synthetic.make_w(synthetic.LLAMA8B_PREFILL, 0, 1024, 768)
+    Xq, xs = ptpc.quantize_activations_per_tensor(to_dev_bf16(X))
+    Wq_t, ws = ptpc.quantize_weights_per_tensor(to_dev_bf16(W))
+    out = from_dev_bf16(ptpc.scaled_mm(Xq, xs, Wq_t, ws))
+    rXq, sx = oracle.quant_per_tensor(X)
+    rWq, sw = oracle.quant_weight_per_tensor(W)
+    ref = oracle.scaled_mm_reference(rXq, np.full(300, sx, np.float32), rWq, np.full(768, sw, np.float32))
+    assert_gemm_close(out, ref, "per-tensor")
+
+
+def test_extreme_codes_full_depth(ptpc):
+    """All-448 operands at K = 28672: the largest dot products of the format."""
+    T, Ci, Co = 130, 28672, 272
+    rng = np.random.default_rng(1)
+    Xq = np.full((T, Ci), 0x7E, np.uint8)
+    Xq[1::2] = rng.choice(np.array([0x7E, 0xFE], np.uint8), size=(T // 2, Ci))
+    Wq_t = np.full((Co, Ci), 0x7E, np.uint8)
+    xs = np.full(T, 2.0 ** -12, np.float32)
+    ws = np.full(Co, 2.0 ** -14, np.float32)
+    out = ptpc.scaled_mm(to_dev(Xq), to_dev(xs), to_dev(Wq_t), to_dev(ws))
+    ref = oracle.scaled_mm_reference(Xq, xs, Wq_t, ws)
+    assert_gemm_close(from_dev_bf16(out), ref, "extreme")
+
+
+def test_deterministic_and_status_clean(ptpc):
+    for T, Ci, Co in [(1, 28672, 8192), (2048, 4096, 6144)]:
+        X = synthetic.make_x(synthetic.DECODE_70B, 1, T, Ci)
+        W = synthetic.make_w(synthetic.DECODE_70B, 1, Ci, Co)
+        Wq_t, ws = ptpc.quantize_weights(to_dev_bf16(W))
+        Xd = to_dev_bf16(X)
+        wsp = ptpc.Workspace(ptpc.workspace_size(ptpc.OP_LINEAR, T, Ci, Co), "cuda")
+        a = ptpc.linear(Xd, Wq_t, ws, ws=wsp)
+        b = ptpc.linear(Xd, Wq_t, ws, ws=wsp)
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+        assert ptpc.device_status(wsp) == ptpc.OK
+
+
+def test_empty_input_is_noop(ptpc):
+    Wq_t = torch.zeros((64, 128), dtype=torch.uint8, device="cuda")
+    ws = torch.ones(64, dtype=torch.float32, device="cuda")
+    out = ptpc.linear(torch.zeros((0, 128), dtype=torch.bfloat16, device="cuda"), Wq_t, ws)
+    assert out.shape == (0, 64)
