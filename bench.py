@@ -1,0 +1,441 @@
+"""PTPC-FP8 benchmark: fused quantise + scaled-GEMM linear layers on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = the PTPC-FP8 forward of every linear layer of the workload on one
+batch of synthetic activations already resident in HBM: per layer, the
+per-token activation quantiser and the fused row-wise-scaled FP8 GEMM,
+through the library's fused entry point ``ptpc_linear`` (weights are
+quantised per output channel once, before timing, as at model load).  The
+default workload is Llama-3.1-8B prefill at T = 2048 (QKV 4096->6144,
+gate+up 4096->28672, down 14336->4096).
+
+Prints one JSON line (rank 0).  ``value`` is whole-job TFLOP/s
+(2 * T * Ci * Co summed over layers and ranks / the slowest rank's device
+time).  With N > 1 every rank runs an independent replica of the workload
+(weak scaling, no data-path collective).  ``--impl reference`` times the CPU
+oracle on a bounded row sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+WORKLOADS = {
+    "llama8b_prefill": synthetic.LLAMA8B_PREFILL,
+    "decode70b": synthetic.DECODE_70B,
+    "llama70b_prefill": synthetic.LLAMA70B_PREFILL,
+    "chain70b": synthetic.CHAIN_70B,
+    "tiny": synthetic.TINY,
+}
+METRIC = "fused PTPC-FP8 GEMM TFLOP/s (% FP8 peak); quant GB/s (% HBM) on 1 B200"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="llama8b_prefill", choices=sorted(WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=None, help="override T (default: the workload's first)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extras", action="store_true", help="skip comparison paths, e2e and CPU baseline")
+    ap.add_argument("--cpu-rows", type=int, default=128, help="rows per layer in the CPU-oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+def workload_layers(wl, T):
+    return [(i, L.name, T, L.Ci, L.Co) for i, L in enumerate(wl.layers)]
+
+
+def layer_flops(layers):
+    return sum(2.0 * T * Ci * Co for _, _, T, Ci, Co in layers)
+
+
+def gemm_bytes(T, Ci, Co):
+    """Algorithmic bytes of one fused GEMM launch: Xq, Wq_t, out, both scale vectors."""
+    return T * Ci + Ci * Co + 2 * T * Co + 4 * (T + Co)
+
+
+def quant_bytes(T, Ci):
+    """Algorithmic bytes of one activation-quantiser launch: bf16 in, codes + scales out."""
+    return 3 * T * Ci + 4 * T
+
+
+def config_of(wl, layers, l2_note):
+    return {
+        "workload": wl.name + ": " + ", ".join(f"{n} {Ci}->{Co}" for _, n, _, Ci, Co in layers),
+        "tokens": layers[0][2],
+        "layers": [{"name": n, "T": T, "Ci": Ci, "Co": Co} for _, n, T, Ci, Co in layers],
+        "weights": "bf16 N(0, sigma) quantised per output channel once, before timing",
+        "l2": l2_note,
+    }
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: report clocks as unavailable
+            self.nv = None
+
+    _NAMES = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self._NAMES.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------- reference (CPU oracle) arm
+
+def cpu_oracle_sample(wl, layers, rows_per_layer, steps):
+    """Times the oracle (as it stands) on `rows_per_layer` token rows of every
+    layer: per-token quantisation of those rows and the fp64 scaled GEMM
+    against the full weight.  Returns (TFLOP/s, seconds, threads, note)."""
+    import oracle
+    prep = []
+    for i, name, T, Ci, Co in layers:
+        r = min(rows_per_layer, T)
+        X = synthetic.make_x(wl, i, r, Ci)
+        W = synthetic.make_w(wl, i, Ci, Co)
+        Wq_t, ws = oracle.quant_weight(W)
+        prep.append((X, Wq_t, ws, r, Ci, Co))
+    flops = sum(2.0 * r * Ci * Co for _, _, _, r, Ci, Co in prep)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        for X, Wq_t, ws, r, Ci, Co in prep:
+            oracle.linear_reference(X, Wq_t, ws)
+    dt = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [os.cpu_count() or 1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    note = (f"{rows_per_layer} token rows per layer x {len(prep)} layers x {steps} steps "
+            f"(oracle per-token quantisation + fp64 GEMM against the full weight)")
+    return flops * steps / dt / 1e12, dt, threads, note
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = WORKLOADS[args.workload]
+    T = args.tokens or wl.tokens[0]
+    layers = workload_layers(wl, T)
+    rows = max(1, min(args.cpu_rows, T))
+    for _ in range(max(0, min(args.warmup, 1))):
+        cpu_oracle_sample(wl, layers, rows, 1)
+    steps = max(1, min(args.steps, 3))
+    tflops, dt, threads, note = cpu_oracle_sample(wl, layers, rows, steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup, "ms_per_step": dt / steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(wl, layers, "CPU run"),
+        "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": note},
+        "e2e": {"value": tflops, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def traffic_record(kernel_src_hash):
+    """DRAM bytes per GEMM launch from a committed ncu summary, if it was
+    taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "gemm_dram_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_src_sha256") != kernel_src_hash:
+        return None
+    return d.get("dram_bytes_per_step")
+
+
+def kernel_src_hash():
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "sm100.cuh", "kernels.h"):
+        with open(os.path.join(ROOT, "fp8_quantized_gemm_ptpc_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import fp8_quantized_gemm_ptpc_b200 as ptpc
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    wl = WORKLOADS[args.workload]
+    T = args.tokens or wl.tokens[0]
+    layers = workload_layers(wl, T)
+    peaks = load_peaks()
+    fp8_peak = 2.0 * peaks["bf16_tflops"]                 # nominal fp8:bf16 ratio 2
+    fp8_peak_sus = 2.0 * peaks["bf16_tflops_sustained"]
+
+    def to_dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    # inputs, resident in HBM; weights quantised once (model load)
+    L = []
+    for i, name, T_, Ci, Co in layers:
+        X = to_dev(synthetic.make_x(wl, i, T_, Ci))
+        Wb = to_dev(synthetic.make_w(wl, i, Ci, Co))
+        Wq_t, w_scale = ptpc.quantize_weights(Wb)
+        Wq_pt, ws_pt = ptpc.quantize_weights_per_tensor(Wb)
+        del Wb
+        out = torch.empty((T_, Co), dtype=torch.bfloat16, device=dev)
+        wsp = ptpc.Workspace(ptpc.workspace_size(ptpc.OP_LINEAR, T_, Ci, Co), dev)
+        L.append(dict(name=name, T=T_, Ci=Ci, Co=Co, X=X, Wq_t=Wq_t, ws=w_scale, Wq_pt=Wq_pt, ws_pt=ws_pt,
+                      out=out, wsp=wsp))
+    torch.cuda.synchronize(dev)
+    working_set = sum(d["X"].numel() * 2 + d["Wq_t"].numel() + d["out"].numel() * 2 for d in L)
+    l2_note = (f"inputs larger than L2: {working_set / 1e6:.0f} MB touched per step > 126 MB L2, no flush"
+               if working_set > L2_BYTES else
+               f"working set {working_set / 1e6:.1f} MB fits in L2 (no flush)")
+
+    def step():
+        for d in L:
+            ptpc.linear(d["X"], d["Wq_t"], d["ws"], out=d["out"], ws=d["wsp"])
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed(fn, steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        barrier()
+        return e0.elapsed_time(e1)
+
+    K, W = args.steps, max(3, args.warmup)
+    for _ in range(W):
+        step()
+    with ClockSampler(local) as clk:
+        ms = timed(step, K)
+    ms = max_over_ranks(ms)
+    flops = layer_flops(layers)
+    value = flops * world * K / (ms / 1e3) / 1e12
+    launches = K * 2 * len(L)
+
+    # ---- per-kernel device times (events on the launch stream around each launch)
+    Kk = max(10, min(K, 200))
+    q_ms = [0.0] * len(L)
+    g_ms = [0.0] * len(L)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in L]
+    bufs = [(torch.empty((d["T"], d["Ci"]), dtype=torch.uint8, device=dev),
+             torch.empty((d["T"],), dtype=torch.float32, device=dev)) for d in L]
+    for it in range(Kk + 3):
+        for j, d in enumerate(L):
+            e = evs[j]
+            e[0].record(stream)
+            ptpc.quantize_activations(d["X"], *bufs[j])
+            e[1].record(stream)
+            ptpc.scaled_mm(bufs[j][0], bufs[j][1], d["Wq_t"], d["ws"], out=d["out"], ws=d["wsp"])
+            e[2].record(stream)
+        torch.cuda.synchronize(dev)
+        if it >= 3:
+            for j in range(len(L)):
+                q_ms[j] += evs[j][0].elapsed_time(evs[j][1]) / Kk
+                g_ms[j] += evs[j][1].elapsed_time(evs[j][2]) / Kk
+    gemm_time = sum(g_ms)
+    gemm_tflops = flops / (gemm_time / 1e3) / 1e12
+    q_bytes = sum(quant_bytes(d["T"], d["Ci"]) for d in L)
+    q_gbs = q_bytes / (sum(q_ms) / 1e3) / 1e9
+    dram = traffic_record(kernel_src_hash())
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 x e4m3 -> f32 accumulate, bf16 out", "data": "synthetic",
+        "config": dict(config_of(wl, layers, l2_note), parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
+        "frac_of_fp8_peak": value / world / fp8_peak,
+        "clocks": clk.summary(),
+        "gpu_launches": launches,
+        "roofline": {
+            "bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+            "frac": gemm_tflops / fp8_peak, "traffic": dram,
+            "kernel": "ptpc_gemm_kernel (fused scaled GEMM), all layers of one step",
+            "peak_src": f"{peaks['src']} bf16 burst x 2 (fp8:bf16 nominal ratio)",
+            "frac_of_sustained": gemm_tflops / fp8_peak_sus,
+            "per_layer_ms": {d["name"]: g for d, g in zip(L, g_ms)},
+        },
+        "quant": {
+            "value": q_gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"], "frac": q_gbs / peaks["hbm_gbs"],
+            "bytes_per_step": q_bytes, "per_layer_ms": {d["name"]: q for d, q in zip(L, q_ms)},
+            "peak_src": f"{peaks['src']} HBM copy",
+        },
+    }
+
+    if not args.no_extras:
+        # ---- comparison paths of the page: naive two-step and per-tensor scaling
+        ys = [torch.empty((d["T"], d["Co"]), dtype=torch.float32, device=dev) for d in L]
+        pt_ws = [ptpc.Workspace(ptpc.workspace_size(ptpc.OP_BENCH_PER_TENSOR, d["T"], d["Ci"], 0), dev) for d in L]
+
+        def naive():
+            for j, d in enumerate(L):
+                ptpc.quantize_activations(d["X"], *bufs[j])
+                ptpc.unscaled_mm_f32(bufs[j][0], d["Wq_t"], out=ys[j], ws=d["wsp"])
+                ptpc.apply_scales(ys[j], bufs[j][1], d["ws"], out=d["out"])
+
+        def per_tensor():
+            for j, d in enumerate(L):
+                ptpc.quantize_activations_per_tensor(d["X"], *bufs[j], ws=pt_ws[j])
+                ptpc.scaled_mm(bufs[j][0], bufs[j][1], d["Wq_pt"], d["ws_pt"], out=d["out"], ws=d["wsp"])
+
+        Kc = max(5, min(K, 100))
+        for fn in (naive, per_tensor):
+            for _ in range(3):
+                fn()
+        ms_naive = max_over_ranks(timed(naive, Kc)) / Kc
+        ms_pt = max_over_ranks(timed(per_tensor, Kc)) / Kc
+        ms_sep = sum(q_ms) + sum(g_ms)
+        line["paths"] = {
+            "fused_ptpc_linear_ms": ms / K,
+            "quantize_then_scaled_mm_ms": ms_sep,
+            "naive_two_step_ms": ms_naive,
+            "per_tensor_ms": ms_pt,
+            "fused_speedup_over_naive": ms_naive / (ms / K),
+            "ptpc_over_per_tensor_throughput": ms_pt / (ms / K),
+        }
+        del ys
+
+        # ---- end to end through the public API: pinned host in, pinned host out
+        hx = [d["X"].cpu().pin_memory() for d in L]
+        ho = [torch.empty((d["T"], d["Co"]), dtype=torch.bfloat16).pin_memory() for d in L]
+        dx = [torch.empty_like(d["X"]) for d in L]
+
+        def e2e_step():
+            for j, d in enumerate(L):
+                dx[j].copy_(hx[j], non_blocking=True)
+                ptpc.linear(dx[j], d["Wq_t"], d["ws"], out=d["out"], ws=d["wsp"])
+                ho[j].copy_(d["out"], non_blocking=True)
+
+        Ke = max(5, min(K, 30))
+        for _ in range(3):
+            e2e_step()
+        ms_e2e = max_over_ranks(timed(e2e_step, Ke)) / Ke
+        line["e2e"] = {
+            "value": flops * world / (ms_e2e / 1e3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(sum(h.numel() * 2 for h in hx)),
+            "d2h_bytes_per_step": int(sum(h.numel() * 2 for h in ho)),
+            "ms_per_step": ms_e2e,
+        }
+
+        if rank == 0 and world == 1:
+            tf, dt, threads, note = cpu_oracle_sample(wl, layers, max(1, min(args.cpu_rows, T)), 1)
+            line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                    "sample": note, "seconds": dt}
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

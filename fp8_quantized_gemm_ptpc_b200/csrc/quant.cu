@@ -9,12 +9,14 @@
 //
 // Every code is E4M3_satRNE(fp32_RN(x / s)) with s = fp32_RN(amax / 448).  The
 // division is done without a per-element divide: with r = RN(1/s),
-//   q0 = RN(x * r),  e = x - q0 * s (one FMA, exact),  q = RN(q0 + e * r),
+//   q0 = RN(x * r),  e = q0 * s - x (one FMA, exact),  q = RN(q0 - e * r),
 // the one-step correction of Markstein ("Computation of elementary functions
-// on the IBM RISC System/6000 processor", IBM J. R&D 34(1), 1990).  For
-// s >= 2^-100 this yields the same E4M3 code as the IEEE quotient for every
-// pair of bf16 inputs (checked exhaustively against the CPU definition);
-// groups with a smaller scale take the IEEE division __fdiv_rn instead.
+// on the IBM RISC System/6000 processor", IBM J. R&D 34(1), 1990).  The
+// residual is formed as q0*s - x rather than x - q0*s so that x = -0 gives
+// q = -0 (the other form returns +0 there).  For s >= 2^-100 this yields the
+// IEEE quotient itself whenever |x/s| >= 2^-11 and the same E4M3 code for
+// every pair of bf16 inputs (checked exhaustively against the CPU
+// definition); groups with a smaller scale take the IEEE division __fdiv_rn.
 #include <algorithm>
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -56,8 +58,8 @@ __device__ __forceinline__ GroupScale group_scale_from_amax_bits(uint32_t amax_b
 __device__ __forceinline__ float quotient(float x, const GroupScale &g) {
   if (g.mode == kFast) {
     const float q0 = __fmul_rn(x, g.r);
-    const float e = __fmaf_rn(-q0, g.s, x);
-    return __fmaf_rn(e, g.r, q0);
+    const float e = __fmaf_rn(q0, g.s, -x);
+    return __fmaf_rn(-e, g.r, q0);
   }
   return __fdiv_rn(x, g.s);
 }
@@ -434,7 +436,9 @@ cudaError_t launch_quant_act_per_tensor(const void *X, int T, int Ci, uint8_t *X
   if (grid < 1) grid = 1;
   amax_kernel<<<grid, 512, 0, st>>>(static_cast<const uint4 *>(X), n8, amax_slot);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  return launch_act<true>(X, T, Ci, Xq, xs, amax_slot, st);
+  if ((e = launch_act<true>(X, T, Ci, Xq, xs, amax_slot, st)) != cudaSuccess) return e;
+  // the workspace's scratch word is left zero for the next user
+  return cudaMemsetAsync(amax_slot, 0, sizeof(uint32_t), st);
 }
 
 cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, float *w_scale, uint32_t *col_amax,
@@ -464,7 +468,9 @@ cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, fl
   }
   dim3 grid((Co + kTT - 1) / kTT, (Ci + kTT - 1) / kTT);
   quant_weight_t_kernel<<<grid, 256, 0, st>>>(Wv, Ci, Co, col_amax, Wq_t, w_scale);
-  return cudaGetLastError();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // the workspace's scratch words are left zero for the next user
+  return cudaMemsetAsync(col_amax, 0, sizeof(uint32_t) * ((size_t)Co + 1), st);
 }
 
 cudaError_t launch_apply_scales(const float *y, const float *xs, const float *ws, int T, int Co, void *out,

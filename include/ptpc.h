@@ -42,7 +42,10 @@
  *     again, so a workspace is zero-filled only once.  Calls that share a
  *     workspace must not overlap on the GPU.
  *   - Inputs are assumed finite.  Non-finite inputs do not fault but give
- *     unspecified codes.
+ *     unspecified codes.  The GEMM epilogue multiplies in the order
+ *     (acc * x_scale) * w_scale in fp32; outputs are specified where that
+ *     intermediate product is finite (|acc * x_scale| < 2^128), which holds
+ *     unless a token's amax is within ~2^30 of the bf16 maximum.
  */
 #ifndef PTPC_H_
 #define PTPC_H_

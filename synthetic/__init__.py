@@ -120,11 +120,11 @@ def random_bf16(shape, seed: int, scale: float = 1.0) -> np.ndarray:
     return to_bf16_bits(rng.standard_normal(shape, dtype=np.float32) * np.float32(scale))
 
 
-def with_edge_rows(X_bits: np.ndarray, seed: int = 7) -> np.ndarray:
+def with_edge_rows(X_bits: np.ndarray, seed: int = 7, huge_bits: int = 0x7F7F) -> np.ndarray:
     """Copy of X with edge-case rows planted (when T is large enough):
     row 0 all +0, row 1 all -0, row 2 only bf16 subnormals,
     row 3 a single nonzero element, row 4 mixed +-0 and tiny normals,
-    row 5 values at the bf16 maximum magnitude."""
+    row 5 values of magnitude ``huge_bits`` (default: the bf16 maximum)."""
     X = np.array(X_bits, dtype=np.uint16, copy=True)
     T, Ci = X.shape
     rng = np.random.Generator(np.random.PCG64(seed))
@@ -145,7 +145,7 @@ def with_edge_rows(X_bits: np.ndarray, seed: int = 7) -> np.ndarray:
         r |= (rng.integers(0, 2, Ci).astype(np.uint16) << 15)
         return r
     plans.append(mixed_tiny)
-    plans.append(lambda: (np.full(Ci, 0x7F7F, np.uint16)
+    plans.append(lambda: (np.full(Ci, huge_bits, np.uint16)
                           | (rng.integers(0, 2, Ci).astype(np.uint16) << 15)))      # bf16 max
     for i, plan in enumerate(plans):
         if i < T:

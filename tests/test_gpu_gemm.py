@@ -14,6 +14,10 @@ from helpers import assert_gemm_close, from_dev_bf16, to_dev, to_dev_bf16
 
 pytestmark = pytest.mark.gpu
 
+# bf16 bits of 2^100: a row of this magnitude has x_scale ~ 2^91, and every
+# accumulator times x_scale stays far inside the fp32 range.
+BIG_BF16 = 0x7180
+
 
 @pytest.fixture(scope="module")
 def ptpc():
@@ -50,7 +54,8 @@ def test_tiny_workload(ptpc):
     (1000, 1024, 768), (3001, 512, 2064), (128, 4112, 256), (257, 128, 4096),
 ])
 def test_ragged_shapes(ptpc, T, Ci, Co):
-    X = synthetic.with_edge_rows(synthetic.make_x(synthetic.LLAMA70B_PREFILL, 0, T, Ci))
+    # the large-magnitude edge row stays where acc * x_scale fits in fp32
+    X = synthetic.with_edge_rows(synthetic.make_x(synthetic.LLAMA70B_PREFILL, 0, T, Ci), huge_bits=BIG_BF16)
     W = synthetic.random_bf16((Ci, Co), seed=T + Ci + Co, scale=0.02)
     g, r = run_pair(ptpc, X, W)
     assert_gemm_close(g, r, f"{T}x{Ci}x{Co}")
@@ -162,3 +167,24 @@ def test_empty_input_is_noop(ptpc):
     ws = torch.ones(64, dtype=torch.float32, device="cuda")
     out = ptpc.linear(torch.zeros((0, 128), dtype=torch.bfloat16, device="cuda"), Wq_t, ws)
     assert out.shape == (0, 64)
+
+
+def test_workspace_shared_across_entry_points(ptpc):
+    """Every entry point leaves the workspace's control words zero, so one
+    workspace can serve the weight quantiser and a split-K GEMM in turn."""
+    T, Ci, Co = 1, 28672, 8192
+    need = max(ptpc.workspace_size(ptpc.OP_LINEAR, T, Ci, Co),
+               ptpc.workspace_size(ptpc.OP_QUANTIZE_WEIGHTS, 0, Ci, Co),
+               ptpc.workspace_size(ptpc.OP_BENCH_PER_TENSOR, T, Ci, 0))
+    wsp = ptpc.Workspace(need, "cuda")
+    W = synthetic.make_w(synthetic.DECODE_70B, 1, Ci, Co)
+    X = synthetic.make_x(synthetic.DECODE_70B, 1, T, Ci)
+    Wq_t, ws = ptpc.quantize_weights(to_dev_bf16(W), ws=wsp)
+    ptpc.quantize_activations_per_tensor(to_dev_bf16(X), ws=wsp)
+    torch.cuda.synchronize()
+    assert int(wsp.buf[4:].count_nonzero()) == 0 or int(wsp.buf[256:].count_nonzero()) == 0
+    out = from_dev_bf16(ptpc.linear(to_dev_bf16(X), Wq_t, ws, ws=wsp))
+    rWq, rws = oracle.quant_weight(W)
+    rXq, rxs = oracle.quant_act(X)
+    assert_gemm_close(out, oracle.scaled_mm_reference(rXq, rxs, rWq, rws), "shared workspace")
+    assert ptpc.device_status(wsp) == ptpc.OK

@@ -65,6 +65,15 @@ def test_act_llama70b_prefill_full(ptpc):
     assert_act_parity(ptpc, synthetic.make_x(w, 1, 8192, 28672))
 
 
+def test_signed_zero_in_nonzero_groups(ptpc):
+    """-0.0 keeps its sign (code 0x80) in rows/columns with a normal scale."""
+    X = synthetic.random_bf16((64, 512), seed=5)
+    X[:, ::7] = 0x8000
+    X[:, 3::7] = 0x0000
+    assert_act_parity(ptpc, X)
+    assert_weight_parity(ptpc, X)
+
+
 def test_act_long_rows_two_pass_kernel(ptpc):
     # rows longer than the register-resident kernel holds (Ci > 131072)
     X = synthetic.random_bf16((3, 131072 + 4096), seed=21, scale=3.0)
