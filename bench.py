@@ -55,7 +55,9 @@ def parse():
     ap.add_argument("--tokens", type=int, default=None, help="override T (default: the workload's first)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip comparison paths, e2e and CPU baseline")
-    ap.add_argument("--cpu-rows", type=int, default=128, help="rows per layer in the CPU-oracle sample")
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="token rows per layer in the CPU-oracle sample (0: all T rows)")
+    ap.add_argument("--cpu-steps", type=int, default=2, help="steps in the CPU-oracle sample")
     return ap.parse_args()
 
 
@@ -102,9 +104,9 @@ def config_of(wl, layers, l2_note):
 class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML while running."""
 
-    def __init__(self, index: int, period_s: float = 0.02):
+    def __init__(self, index: int, period_s: float = 0.002):
         self.index, self.period = index, period_s
-        self.samples, self.reasons = [], set()
+        self.samples, self.reasons, self.power = [], set(), []
         self.max_mhz = None
         self._stop = threading.Event()
         self._t = None
@@ -128,6 +130,7 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.power.append(nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0)
                 mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
                 for bit, name in self._NAMES.items():
                     if mask & bit:
@@ -150,8 +153,11 @@ class ClockSampler:
     def summary(self):
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_min_mhz": min(self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples),
+                "power_w_median": statistics.median(self.power) if self.power else None,
+                "power_w_max": max(self.power) if self.power else None}
 
 
 # ----------------------------------------------------------------- reference (CPU oracle) arm
@@ -191,7 +197,7 @@ def run_reference(args):
     wl = WORKLOADS[args.workload]
     T = args.tokens or wl.tokens[0]
     layers = workload_layers(wl, T)
-    rows = max(1, min(args.cpu_rows, T))
+    rows = T if args.cpu_rows <= 0 else max(1, min(args.cpu_rows, T))
     for _ in range(max(0, min(args.warmup, 1))):
         cpu_oracle_sample(wl, layers, rows, 1)
     steps = max(1, min(args.steps, 3))
@@ -313,26 +319,28 @@ def run_gpu(args):
     value = flops * world * K / (ms / 1e3) / 1e12
     launches = K * 2 * len(L)
 
-    # ---- per-kernel device times (events on the launch stream around each launch)
+    # ---- per-kernel device times: events on the launch stream around each
+    # launch, no host synchronisation inside the loop
     Kk = max(10, min(K, 200))
-    q_ms = [0.0] * len(L)
-    g_ms = [0.0] * len(L)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in L]
     bufs = [(torch.empty((d["T"], d["Ci"]), dtype=torch.uint8, device=dev),
              torch.empty((d["T"],), dtype=torch.float32, device=dev)) for d in L]
-    for it in range(Kk + 3):
+    for _ in range(3):
         for j, d in enumerate(L):
-            e = evs[j]
+            ptpc.quantize_activations(d["X"], *bufs[j])
+            ptpc.scaled_mm(bufs[j][0], bufs[j][1], d["Wq_t"], d["ws"], out=d["out"], ws=d["wsp"])
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in L] for _ in range(Kk)]
+    barrier()
+    for it in range(Kk):
+        for j, d in enumerate(L):
+            e = evs[it][j]
             e[0].record(stream)
             ptpc.quantize_activations(d["X"], *bufs[j])
             e[1].record(stream)
             ptpc.scaled_mm(bufs[j][0], bufs[j][1], d["Wq_t"], d["ws"], out=d["out"], ws=d["wsp"])
             e[2].record(stream)
-        torch.cuda.synchronize(dev)
-        if it >= 3:
-            for j in range(len(L)):
-                q_ms[j] += evs[j][0].elapsed_time(evs[j][1]) / Kk
-                g_ms[j] += evs[j][1].elapsed_time(evs[j][2]) / Kk
+    barrier()
+    q_ms = [sum(evs[it][j][0].elapsed_time(evs[it][j][1]) for it in range(Kk)) / Kk for j in range(len(L))]
+    g_ms = [sum(evs[it][j][1].elapsed_time(evs[it][j][2]) for it in range(Kk)) / Kk for j in range(len(L))]
     gemm_time = sum(g_ms)
     gemm_tflops = flops / (gemm_time / 1e3) / 1e12
     q_bytes = sum(quant_bytes(d["T"], d["Ci"]) for d in L)
@@ -418,7 +426,8 @@ def run_gpu(args):
         }
 
         if rank == 0 and world == 1:
-            tf, dt, threads, note = cpu_oracle_sample(wl, layers, max(1, min(args.cpu_rows, T)), 1)
+            rows = T if args.cpu_rows <= 0 else max(1, min(args.cpu_rows, T))
+            tf, dt, threads, note = cpu_oracle_sample(wl, layers, rows, max(1, args.cpu_steps))
             line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                                     "sample": note, "seconds": dt}
 

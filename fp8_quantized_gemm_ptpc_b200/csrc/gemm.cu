@@ -96,6 +96,74 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Fused epilogue of one accumulator: 32 token rows (one TMEM lane quarter,
+// lane i = row store_row0 + i) x BN_T columns starting at global column
+// col_base.  fp32 -> (acc * x_scale) * w_scale -> bf16 (or the raw fp32
+// accumulator), staged as 32 x 128-byte chunks in 128-byte-swizzled shared
+// memory and written with TMA stores.  After the last tensor-memory read the
+// accumulator buffer is released by one arrival on `release_bar` (a
+// shared::cluster address: this CTA's barrier or the pair leader's).
+template <int BN_T, bool F32OUT>
+__device__ __forceinline__ void epilogue_store_tile(const CUtensorMap *tmC, uint32_t tbase, uint8_t *cbuf,
+                                                    float *sc, const GemmParams &p, int col_base,
+                                                    int store_row0, float xsr, int lane, uint32_t release_bar) {
+  constexpr int EPI_COLS = F32OUT ? 32 : 64;
+  #pragma unroll 1
+  for (int c0 = 0; c0 < BN_T; c0 += EPI_COLS) {
+    uint32_t packed[32];
+    if constexpr (F32OUT) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(tbase + c0, r);
+      tmem_wait_ld();
+      #pragma unroll
+      for (int j = 0; j < 32; ++j) packed[j] = r[j];
+    } else {
+      __syncwarp();
+      const int col0 = col_base + c0;
+      sc[lane] = (col0 + lane < p.Co) ? __ldg(p.ws + col0 + lane) : 0.0f;
+      sc[lane + 32] = (col0 + 32 + lane < p.Co) ? __ldg(p.ws + col0 + 32 + lane) : 0.0f;
+      uint32_t r0[32], r1[32];
+      tmem_ld_32x32b_x32(tbase + c0, r0);
+      tmem_ld_32x32b_x32(tbase + c0 + 32, r1);
+      tmem_wait_ld();
+      __syncwarp();
+      #pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float4 wv = *reinterpret_cast<const float4 *>(sc + 4 * j);
+        const uint32_t *rr = (j < 8) ? r0 : r1;
+        const int b = (j & 7) * 4;
+        const float v0 = __fmul_rn(__fmul_rn(__uint_as_float(rr[b + 0]), xsr), wv.x);
+        const float v1 = __fmul_rn(__fmul_rn(__uint_as_float(rr[b + 1]), xsr), wv.y);
+        const float v2 = __fmul_rn(__fmul_rn(__uint_as_float(rr[b + 2]), xsr), wv.z);
+        const float v3 = __fmul_rn(__fmul_rn(__uint_as_float(rr[b + 3]), xsr), wv.w);
+        packed[2 * j] = pack_bf16x2(v0, v1);
+        packed[2 * j + 1] = pack_bf16x2(v2, v3);
+      }
+    }
+    if (c0 + EPI_COLS >= BN_T) {
+      // the whole accumulator has been read: hand it back to the MMA issuer
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(release_bar);
+    }
+    // the previous TMA store from this buffer must have finished reading it
+    if (lane == 0) bulk_wait_read<0>();
+    __syncwarp();
+    #pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int pos = j ^ (lane & 7);
+      *reinterpret_cast<uint4 *>(cbuf + lane * 128 + pos * 16) =
+          make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+    }
+    fence_async_shared();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmC, cbuf, col_base + c0, store_row0);
+      bulk_commit();
+    }
+  }
+}
+
 template <int BN, int STAGES, bool F32OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     ptpc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -255,60 +323,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       if (p.nsplit == 1) {
         // ---- direct: scale, round, stage, TMA store
-        #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += C::EPI_COLS) {
-          uint32_t packed[32];
-          if constexpr (F32OUT) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(tbase + c0, r);
-            tmem_wait_ld();
-            #pragma unroll
-            for (int j = 0; j < 32; ++j) packed[j] = r[j];
-          } else {
-            __syncwarp();
-            const int col0 = n * BN + c0;
-            sc[lane] = (col0 + lane < p.Co) ? __ldg(p.ws + col0 + lane) : 0.0f;
-            sc[lane + 32] = (col0 + 32 + lane < p.Co) ? __ldg(p.ws + col0 + 32 + lane) : 0.0f;
-            uint32_t r0[32], r1[32];
-            tmem_ld_32x32b_x32(tbase + c0, r0);
-            tmem_ld_32x32b_x32(tbase + c0 + 32, r1);
-            tmem_wait_ld();
-            __syncwarp();
-            #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float4 wv = *reinterpret_cast<const float4 *>(sc + 4 * j);
-              const uint32_t *rr = (j < 8) ? r0 : r1;
-              const int b = (j & 7) * 4;
-              const float v0 = __fmul_rn(__fmul_rn(__uint_as_float(rr[b + 0]), xsr), wv.x);
-              const float v1 = __fmul_rn(__fmul_rn(__uint_as_float(rr[b + 1]), xsr), wv.y);
-              const float v2 = __fmul_rn(__fmul_rn(__uint_as_float(rr[b + 2]), xsr), wv.z);
-              const float v3 = __fmul_rn(__fmul_rn(__uint_as_float(rr[b + 3]), xsr), wv.w);
-              packed[2 * j] = pack_bf16x2(v0, v1);
-              packed[2 * j + 1] = pack_bf16x2(v2, v3);
-            }
-          }
-          if (c0 + C::EPI_COLS >= BN) {
-            // the whole accumulator has been read: hand it back to the MMA warp
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
-          }
-          // previous TMA store from this buffer must have finished reading it
-          if (lane == 0) bulk_wait_read<0>();
-          __syncwarp();
-          #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int pos = j ^ (lane & 7);
-            *reinterpret_cast<uint4 *>(cbuf + lane * 128 + pos * 16) =
-                make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-          }
-          fence_async_shared();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmC, cbuf, n * BN + c0, m * BM + q * 32);
-            bulk_commit();
-          }
-        }
+        epilogue_store_tile<BN, F32OUT>(&tmC, tbase, cbuf, sc, p, n * BN, m * BM + q * 32, xsr, lane,
+                                        smem_u32(&tempty[buf]));
       } else {
         // ---- split-K: fp32 partial of this K range, last CTA reduces
         const int prow = p.T;  // split-K runs with a single 128-row block: rows 0..T-1
@@ -385,6 +401,203 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+
+// ----------------------------------------------------------------------------
+// CTA-pair kernel (prefill): a cluster of two CTAs on two SMs computes a
+// 256 (tokens) x 256 (channels) tile with tcgen05.mma.cta_group::2 (M = 256,
+// N = 256, K = 32).  CTA r of the pair loads token rows [r*128, r*128+128)
+// of A and channel rows [r*128, r*128+128) of B into its own shared memory
+// (no multicast) and signals the leader's (r = 0) stage barrier; the leader
+// issues every MMA, reading both CTAs' shared memory, and its commits arrive
+// on the barriers of both CTAs.  Each CTA's tensor memory holds its 128 token
+// rows x 256 columns, which its own epilogue warps store.  Per SM this moves
+// 32 KB of operands per 128-deep K-block instead of 48 KB for the one-CTA
+// 128 x 256 tile, for the same tensor work.
+// ----------------------------------------------------------------------------
+constexpr int kPairBN = 256;
+constexpr int kPairHalfN = 128;
+
+template <int STAGES, bool F32OUT>
+struct PairCfg {
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = kPairHalfN * BK;
+  static constexpr int EPI_BUF = 32 * 128;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + kEpiWarps * EPI_BUF +
+                                 kEpiWarps * 64 * sizeof(float) + 256;
+  static_assert(SMEM <= 232448, "shared memory");
+};
+
+template <int STAGES, bool F32OUT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    ptpc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+  using C = PairCfg<STAGES, F32OUT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = sA + STAGES * C::A_BYTES;
+  uint8_t *sC = sB + STAGES * C::B_BYTES;
+  float *sScale = reinterpret_cast<float *>(sC + kEpiWarps * C::EPI_BUF);
+  uint64_t *full = reinterpret_cast<uint64_t *>(sScale + kEpiWarps * 64);
+  uint64_t *empty = full + STAGES;
+  uint64_t *tfull = empty + STAGES;
+  uint64_t *tempty = tfull + 2;
+  uint64_t *drain = tempty + 2;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cid = blockIdx.x >> 1;
+  const int ncl = gridDim.x >> 1;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmC);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 2 * kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (elect_one()) {
+      const uint64_t polA = policy_evict_last();
+      const uint64_t polB = policy_evict_first();
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      griddep_wait();
+      for (int u = cid; u < p.num_units && ok; u += ncl) {
+        int m, n, kb0, kb1, tile, split;
+        unit_coords(p, u, m, n, kb0, kb1, tile, split);
+        const int a_row = m * (2 * BM) + (int)rank * BM;
+        const int b_row = n * kPairBN + (int)rank * kPairHalfN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) {
+            ok = false;
+            break;
+          }
+          const uint32_t lead_full = mapa_shared(&full[stage], 0);
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (C::A_BYTES + C::B_BYTES));
+          tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, lead_full, kb * BK, a_row, polA);
+          tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, lead_full, kb * BK, b_row, polB);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        atomicOr(p.status, kStatusTimeoutProducer);
+        // the leader's stage barriers count both CTAs' bytes: once they have
+        // all completed, no copy into either CTA is still in flight
+        if (leader)
+          for (int s = 0; s < STAGES; ++s) mbar_wait(&full[s], s < stage ? phase : phase ^ 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (leader && elect_one()) {
+      constexpr uint32_t idesc = idesc_e4m3_f32(2 * BM, kPairBN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int u = cid; u < p.num_units && ok; u += ncl, ++local) {
+        int m, n, kb0, kb1, tile, split;
+        unit_coords(p, u, m, n, kb0, kb1, tile, split);
+        const int buf = local & 1;
+        const uint32_t aphase = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[buf], aphase ^ 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(buf * kPairBN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + stage * C::A_BYTES));
+          const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + stage * C::B_BYTES));
+          #pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk)
+            mma_e4m3_pair(d, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
+                          (kb > kb0 || kk > 0) ? 1u : 0u);
+          mma_commit_pair_mc(&empty[stage], 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair_mc(&tfull[buf], 0x3);
+      }
+      if (!ok) atomicOr(p.status, kStatusTimeoutMma);
+      mma_commit_pair_mc(drain, 0x1);
+      mbar_wait(drain, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int ew = warp - 2;
+    uint8_t *cbuf = sC + ew * C::EPI_BUF;
+    float *sc = sScale + ew * 64;
+    int local = 0;
+    bool ok = true;
+    griddep_wait();
+    for (int u = cid; u < p.num_units; u += ncl, ++local) {
+      int m, n, kb0, kb1, tile, split;
+      unit_coords(p, u, m, n, kb0, kb1, tile, split);
+      const int buf = local & 1;
+      const uint32_t aphase = (local >> 1) & 1;
+      const int row0 = m * (2 * BM) + (int)rank * BM + q * 32;
+      const int row = row0 + lane;
+      float xsr = 0.0f;
+      if (!F32OUT && row < p.T) xsr = __ldg(p.xs + row);
+      const bool got = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], aphase));
+      if (!got) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kPairBN);
+      epilogue_store_tile<kPairBN, F32OUT>(&tmC, tbase, cbuf, sc, p, n * kPairBN, row0, xsr, lane,
+                                           mapa_shared(&tempty[buf], 0));
+    }
+    if (!ok && lane == 0) atomicOr(p.status, kStatusTimeoutEpilogue);
+    if (lane == 0) bulk_wait<0>();
+  }
+
+  tc_fence_before();
+  cluster_sync();  // the leader's MMAs into both CTAs' tensor memory are complete
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -445,6 +658,62 @@ cudaError_t launch_cfg(const GemmProblem &pr, const GemmParams &gp, int grid, cu
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pr.pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmC, gp);
+}
+
+template <int STAGES, bool F32OUT>
+cudaError_t launch_pair(const GemmProblem &pr, GemmParams gp, cudaStream_t st) {
+  using C = PairCfg<STAGES, F32OUT>;
+  auto kernel = ptpc_gemm_pair_kernel<STAGES, F32OUT>;
+  static bool attr_done[64] = {};
+  static int max_clusters[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const bool cache = dev >= 0 && dev < 64;
+  if (!cache || !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t q = {};
+    q.gridDim = dim3(2 * 74);
+    q.blockDim = dim3(kThreads);
+    q.dynamicSmemBytes = C::SMEM;
+    int ncl = 0;
+    if (cudaOccupancyMaxActiveClusters(&ncl, kernel, &q) != cudaSuccess || ncl <= 0) {
+      cudaGetLastError();
+      ncl = num_sms() / 2;
+    }
+    if (cache) {
+      max_clusters[dev] = ncl;
+      attr_done[dev] = true;
+    } else {
+      max_clusters[0] = ncl;
+    }
+  }
+  const int ncl = std::max(1, std::min(gp.num_units, cache ? max_clusters[dev] : max_clusters[0]));
+  CUtensorMap tmA, tmB, tmC;
+  if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Xq, pr.Ci, pr.T, pr.Ci, BK, BM,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Wq_t, pr.Ci, pr.Co, pr.Ci, BK, kPairHalfN,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  bool okC;
+  if (F32OUT)
+    okC = make_map_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.out, pr.Co, pr.T, (uint64_t)pr.Co * 4, 32, 32,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  else
+    okC = make_map_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.out, pr.Co, pr.T, (uint64_t)pr.Co * 2, 64, 32,
+                      CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!okC) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * ncl);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = st;
@@ -521,6 +790,14 @@ cudaError_t launch_scaled_gemm(const GemmProblem &pr, cudaStream_t st) {
   gp.partials = pr.partials;
   if (pl.nsplit > 1 && pr.partial_floats < (size_t)gp.num_n * pl.nsplit * (size_t)pr.T * pl.bn)
     return cudaErrorInvalidValue;
+  if (pr.T > BM && pl.nsplit == 1) {
+    // CTA-pair 256 x 256 tiles
+    gp.num_m = (pr.T + 2 * BM - 1) / (2 * BM);
+    gp.num_n = (pr.Co + kPairBN - 1) / kPairBN;
+    gp.group_m = 8;
+    gp.num_units = gp.num_m * gp.num_n;
+    return pr.f32_out ? launch_pair<6, true>(pr, gp, st) : launch_pair<6, false>(pr, gp, st);
+  }
   const int grid = std::min(gp.num_units, num_sms());
   if (pl.bn == 256) {
     return pr.f32_out ? launch_cfg<256, 4, true>(pr, gp, grid, st) : launch_cfg<256, 4, false>(pr, gp, grid, st);
