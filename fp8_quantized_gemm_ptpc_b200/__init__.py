@@ -5,7 +5,7 @@ marshals torch tensors (device memory and the current stream) into the
 library calls.  Every step of the computation runs in the library's sm_100a
 kernels; there is no CPU or PyTorch fallback, and importing this package
 fails if ``_lib/libptpc.so`` has not been built
-(``python -m fp8_quantized_gemm_ptpc_b200.build``).
+(``python fp8_quantized_gemm_ptpc_b200/build.py``).
 
 Method: "PTPC-FP8: boosting vLLM performance on AMD ROCm" (vLLM blog),
 sections "Per-Token Activation + Per-Channel Weight Quantization" and "The
@@ -68,10 +68,14 @@ class PtpcError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m fp8_quantized_gemm_ptpc_b200.build` (nvcc, sm_100a)")
+                          "`python fp8_quantized_gemm_ptpc_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():
-        fn = getattr(lib, name)
+        try:
+            fn = getattr(lib, name)
+        except AttributeError as e:
+            raise ImportError(f"{LIB_PATH} does not export {name}: it is older than the sources; rebuild it with "
+                              "`python fp8_quantized_gemm_ptpc_b200/build.py`") from e
         fn.restype = res
         fn.argtypes = args
     return lib

@@ -1,6 +1,9 @@
 """Build libptpc.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m fp8_quantized_gemm_ptpc_b200.build [--force]
+    python fp8_quantized_gemm_ptpc_b200/build.py [--force]
+
+(Run it as a script, or load it by file path: importing it as a submodule
+would import the package, which loads the library it is meant to build.)
 
 The library lands in fp8_quantized_gemm_ptpc_b200/_lib/libptpc.so.  No
 fast-math: the quantisers rely on IEEE round-to-nearest fp32 arithmetic with

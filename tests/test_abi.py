@@ -11,7 +11,11 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def ptpc():
-    from fp8_quantized_gemm_ptpc_b200 import build
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_ptpc_build", os.path.join(ROOT, "fp8_quantized_gemm_ptpc_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
     build.build()
     import fp8_quantized_gemm_ptpc_b200 as p
     return p
