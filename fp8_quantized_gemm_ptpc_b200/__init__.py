@@ -52,6 +52,7 @@ SIGNATURES = {
     "ptpc_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _I64, _I64, _I64]),
     "ptpc_get_device_status": (ctypes.c_int, [_P, _P]),
     "ptpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "ptpc_scaled_mm_static_scratch": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "ptpc_bench_unscaled_mm_f32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "ptpc_bench_apply_scales": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _P, _P]),
     "ptpc_bench_quantize_activations_per_tensor": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _SZ, _P]),
@@ -212,6 +213,26 @@ def linear(X, Wq_t, w_scale, out: torch.Tensor | None = None, ws: Workspace | No
     _check("ptpc_linear",
            lib.ptpc_linear(_ptr(X), _ptr(Wq_t), _ptr(w_scale), T, Ci, Co, _ptr(out), ws.ptr(), ws.nbytes,
                            _stream(X.device)))
+    return out
+
+
+def scaled_mm_static_scratch(Xq, x_scale, Wq_t, w_scale, out: torch.Tensor | None = None):
+    """scaled_mm whose scratch is the library's own static device array (no
+    workspace argument, nothing allocated by the library; ``out`` may be
+    passed to avoid the output allocation here).  Calls must not overlap on
+    the GPU; shapes needing more than 8 MiB of scratch are rejected."""
+    _need(Xq, "Xq", torch.uint8, 2)
+    _need(Wq_t, "Wq_t", torch.uint8, 2)
+    _need(x_scale, "x_scale", torch.float32, 1)
+    _need(w_scale, "w_scale", torch.float32, 1)
+    T, Ci = Xq.shape
+    Co = Wq_t.shape[0]
+    if Wq_t.shape[1] != Ci or x_scale.shape[0] != T or w_scale.shape[0] != Co:
+        raise ValueError("shape mismatch")
+    out = torch.empty((T, Co), dtype=torch.bfloat16, device=Xq.device) if out is None else out
+    _check("ptpc_scaled_mm_static_scratch",
+           lib.ptpc_scaled_mm_static_scratch(_ptr(Xq), _ptr(x_scale), _ptr(Wq_t), _ptr(w_scale), T, Ci, Co,
+                                             _ptr(out), _stream(Xq.device)))
     return out
 
 

@@ -258,3 +258,63 @@ int ptpc_bench_quantize_weights_per_tensor(const void *W, int64_t Ci, int64_t Co
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Scaled GEMM with library-owned scratch (no allocation by the caller).
+//
+// Some callers cannot allocate device memory when they call the GEMM: an
+// inference engine that partitions all of its device memory once at start-up
+// and forbids allocation on the serving path, or a host integration that only
+// hands over input and output buffers.  This entry point needs no workspace
+// from them: its scratch (device status word, split-K tile counters and fp32
+// partial sums) lives in the file-scope array below, which every GPU that
+// loads this library holds until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;  // 8 MiB per device
+
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch for the current device.  In host code
+// the name g_static_scratch is only a host-side stand-in; the real address is
+// obtained once per device with that device current.
+int static_scratch_address(uint8_t **out) {
+  static std::mutex mu;
+  static uint8_t *addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PTPC_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return PTPC_ERR_UNSUPPORTED_DEVICE;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return PTPC_ERR_CUDA;
+    addr[dev] = static_cast<uint8_t *>(p);
+  }
+  *out = addr[dev];
+  return PTPC_OK;
+}
+
+}  // namespace
+
+extern "C" int ptpc_scaled_mm_static_scratch(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq_t,
+                                             const float *w_scale, int64_t T, int64_t Ci, int64_t Co, void *out,
+                                             void *stream) {
+  int s = check_shape_tci(T, Ci);
+  if (s != PTPC_OK) return s;
+  if ((s = check_co(Co)) != PTPC_OK) return s;
+  if (T == 0) return PTPC_OK;
+  if (!Xq || !x_scale || !Wq_t || !w_scale || !out) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(Xq) || !aligned16(x_scale) || !aligned16(Wq_t) || !aligned16(w_scale) || !aligned16(out))
+    return PTPC_ERR_MISALIGNED;
+  if (ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co) > kStaticScratchBytes) return PTPC_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device()) != PTPC_OK) return s;
+  uint8_t *scratch = nullptr;
+  if ((s = static_scratch_address(&scratch)) != PTPC_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  // The array keeps the previous call's contents: the status word and the
+  // split-K counters must start at zero (the partial sums need not).
+  const GemmLayout l = gemm_layout(T, Ci, Co);
+  if (cudaMemsetAsync(scratch, 0, l.partials_off, st) != cudaSuccess) return PTPC_ERR_CUDA;
+  return run_gemm(Xq, x_scale, Wq_t, w_scale, T, Ci, Co, out, false, scratch, false, st);
+}

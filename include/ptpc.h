@@ -146,6 +146,28 @@ PTPC_API int ptpc_get_device_status(void *ws_dev, void *stream);
 /* Static, human-readable name of a status code. */
 PTPC_API const char *ptpc_status_string(int status);
 
+/* ptpc_scaled_mm without a caller-provided workspace.  The page has no
+ * counterpart: this exists for callers that cannot allocate device memory
+ * when they call the GEMM (an engine that partitions all device memory at
+ * start-up and forbids allocation on its serving path, or an integration that
+ * only hands over input and output buffers).  Same arguments, layouts and
+ * results as ptpc_scaled_mm minus (ws_dev, ws_bytes).
+ *   Scratch: a file-scope 8 MiB device array inside the library, held by
+ *   every GPU that loads the library until the process exits.  Shapes whose
+ *   ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co) exceeds 8 MiB are
+ *   rejected with PTPC_ERR_WORKSPACE_TOO_SMALL (for example decode shapes with
+ *   many split-K partial sums, such as T = 128, Ci = 28672, Co = 8192); prefill
+ *   shapes need only a few KiB.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress), so make that first call before any stream capture.
+ *   Every call zeroes the array's control words with cudaMemsetAsync on
+ *   `stream` and allocates nothing.  All calls share the one array: calls
+ *   that overlap on the GPU (different streams, or different host threads)
+ *   race on it and give wrong results. */
+PTPC_API int ptpc_scaled_mm_static_scratch(const uint8_t *Xq_dev, const float *x_scale_dev,
+                                           const uint8_t *Wq_t_dev, const float *w_scale_dev,
+                                           int64_t T, int64_t Ci, int64_t Co, void *out_dev, void *stream);
+
 /* ------------------------------------------------------------------------- */
 /* Measurement-only entry points: the comparison paths the page describes.  */
 /* ------------------------------------------------------------------------- */

@@ -1,0 +1,69 @@
+"""ptpc_scaled_mm_static_scratch: the scaled GEMM for callers that cannot
+allocate device memory when they call it (an engine whose device memory is
+partitioned once at start-up, or an integration that only passes its input
+and output buffers).  Its scratch is the library's own static device array,
+so the caller passes no workspace.
+
+Checked through the C ABI against ptpc_scaled_mm (which takes a caller
+workspace) on two calls in a row, with shapes that use the scratch (split-K
+partial sums and tile counters) and one that does not fit and must be
+rejected.  This file is collected last on purpose."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import synthetic
+from helpers import assert_gemm_close, from_dev_bf16, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ptpc():
+    import fp8_quantized_gemm_ptpc_b200 as p
+    return p
+
+
+def _abi_call(ptpc, Xq, xs, Wq_t, ws, out):
+    T, Ci = Xq.shape
+    Co = Wq_t.shape[0]
+    P = ctypes.c_void_p
+    return ptpc.lib.ptpc_scaled_mm_static_scratch(
+        P(Xq.data_ptr()), P(xs.data_ptr()), P(Wq_t.data_ptr()), P(ws.data_ptr()), T, Ci, Co, P(out.data_ptr()),
+        P(torch.cuda.current_stream().cuda_stream))
+
+
+@pytest.mark.parametrize("T,layer", [(8, 1), (32, 1), (1, 0), (300, 0)])
+def test_static_scratch_matches_workspace_entry_point(ptpc, T, layer):
+    w = synthetic.DECODE_70B
+    L = w.layers[layer]
+    Ci, Co = L.Ci, L.Co
+    if T > 128:  # a prefill-sized case (no split-K); keep the weight small
+        Co = 4096
+    X = synthetic.make_x(w, layer, T, Ci)
+    W = synthetic.make_w(w, layer, Ci, Co)
+    Wq_t, ws = ptpc.quantize_weights(to_dev_bf16(W))
+    Xq, xs = ptpc.quantize_activations(to_dev_bf16(X))
+    ref = ptpc.scaled_mm(Xq, xs, Wq_t, ws)
+    ref_bits = from_dev_bf16(ref)
+    for _ in range(2):
+        out = torch.full((T, Co), float("nan"), dtype=torch.bfloat16, device="cuda")
+        assert _abi_call(ptpc, Xq, xs, Wq_t, ws, out) == ptpc.OK
+        torch.cuda.synchronize()
+        got = from_dev_bf16(out)
+        assert_gemm_close(got, ref_bits, f"static scratch T={T} {Ci}->{Co}")
+        # same kernels, same fixed reduction order: the bits agree as well
+        assert np.array_equal(got, ref_bits)
+
+
+def test_static_scratch_rejects_shapes_beyond_its_size(ptpc):
+    T, Ci, Co = 128, 28672, 8192
+    assert ptpc.workspace_size(ptpc.OP_SCALED_MM, T, Ci, Co) > 8 << 20
+    Xq = torch.zeros((T, Ci), dtype=torch.uint8, device="cuda")
+    xs = torch.ones(T, dtype=torch.float32, device="cuda")
+    Wq_t = torch.zeros((Co, Ci), dtype=torch.uint8, device="cuda")
+    ws = torch.ones(Co, dtype=torch.float32, device="cuda")
+    out = torch.empty((T, Co), dtype=torch.bfloat16, device="cuda")
+    assert _abi_call(ptpc, Xq, xs, Wq_t, ws, out) == ptpc.ERR_WORKSPACE_TOO_SMALL
