@@ -58,6 +58,11 @@ def parse():
     ap.add_argument("--cpu-rows", type=int, default=0,
                     help="token rows per layer in the CPU-oracle sample (0: all T rows)")
     ap.add_argument("--cpu-steps", type=int, default=2, help="steps in the CPU-oracle sample")
+    ap.add_argument("--quant-only", action="store_true",
+                    help="time only the per-token activation quantiser on the workload's inputs")
+    ap.add_argument("--sweep", action="store_true",
+                    help="70B 4-linear chain: fused vs naive two-step vs per-tensor, one JSON line per T")
+    ap.add_argument("--sweep-tokens", default=None, help="comma-separated T values for --sweep")
     return ap.parse_args()
 
 
@@ -69,6 +74,24 @@ def load_peaks():
         return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
                 "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+def dist_max(value: float, device=None) -> float:
+    """Maximum of a per-rank value over all ranks of the default process group
+    (the slowest rank's time decides a multi-GPU step)."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step: float, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank runs `steps` steps of the same work
+    (weak scaling); the job takes as long as its slowest rank."""
+    return flops_per_rank_step * world * steps / (max_ms / 1e3) / 1e12
 
 
 def workload_layers(wl, T):
@@ -271,10 +294,9 @@ def run_gpu(args):
         Wb = to_dev(synthetic.make_w(wl, i, Ci, Co))
         Wq_t, w_scale = ptpc.quantize_weights(Wb)
         Wq_pt, ws_pt = ptpc.quantize_weights_per_tensor(Wb)
-        del Wb
         out = torch.empty((T_, Co), dtype=torch.bfloat16, device=dev)
         wsp = ptpc.Workspace(ptpc.workspace_size(ptpc.OP_LINEAR, T_, Ci, Co), dev)
-        L.append(dict(name=name, T=T_, Ci=Ci, Co=Co, X=X, Wq_t=Wq_t, ws=w_scale, Wq_pt=Wq_pt, ws_pt=ws_pt,
+        L.append(dict(name=name, T=T_, Ci=Ci, Co=Co, X=X, W=Wb, Wq_t=Wq_t, ws=w_scale, Wq_pt=Wq_pt, ws_pt=ws_pt,
                       out=out, wsp=wsp))
     torch.cuda.synchronize(dev)
     working_set = sum(d["X"].numel() * 2 + d["Wq_t"].numel() + d["out"].numel() * 2 for d in L)
@@ -292,11 +314,7 @@ def run_gpu(args):
         torch.cuda.synchronize(dev)
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return dist_max(v, dev)
 
     def timed(fn, steps):
         e0 = torch.cuda.Event(enable_timing=True)
@@ -316,7 +334,7 @@ def run_gpu(args):
         ms = timed(step, K)
     ms = max_over_ranks(ms)
     flops = layer_flops(layers)
-    value = flops * world * K / (ms / 1e3) / 1e12
+    value = whole_job_tflops(flops, world, K, ms)
     launches = K * 2 * len(L)
 
     # ---- per-kernel device times: events on the launch stream around each
@@ -343,6 +361,10 @@ def run_gpu(args):
     g_ms = [sum(evs[it][j][1].elapsed_time(evs[it][j][2]) for it in range(Kk)) / Kk for j in range(len(L))]
     gemm_time = sum(g_ms)
     gemm_tflops = flops / (gemm_time / 1e3) / 1e12
+    g_bytes = sum(gemm_bytes(d["T"], d["Ci"], d["Co"]) for d in L)
+    gemm_gbs = g_bytes / (gemm_time / 1e3) / 1e9
+    ridge = fp8_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)      # FLOP per byte
+    hbm_bound = flops / g_bytes < ridge
     q_bytes = sum(quant_bytes(d["T"], d["Ci"]) for d in L)
     q_gbs = q_bytes / (sum(q_ms) / 1e3) / 1e9
     dram = traffic_record(kernel_src_hash())
@@ -355,12 +377,19 @@ def run_gpu(args):
         "frac_of_fp8_peak": value / world / fp8_peak,
         "clocks": clk.summary(),
         "gpu_launches": launches,
-        "roofline": {
+        "roofline": ({
+            "bound": "hbm", "achieved": gemm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gemm_gbs / peaks["hbm_gbs"], "traffic": dram,
+            "peak_src": f"{peaks['src']} HBM copy",
+        } if hbm_bound else {
             "bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
             "frac": gemm_tflops / fp8_peak, "traffic": dram,
-            "kernel": "ptpc_gemm_kernel (fused scaled GEMM), all layers of one step",
             "peak_src": f"{peaks['src']} bf16 burst x 2 (fp8:bf16 nominal ratio)",
             "frac_of_sustained": gemm_tflops / fp8_peak_sus,
+        }) | {
+            "kernel": "ptpc scaled GEMM (fused epilogue), all layers of one step",
+            "algorithmic_flops_per_step": flops, "algorithmic_bytes_per_step": g_bytes,
+            "gemm_tflops": gemm_tflops, "gemm_gbs": gemm_gbs,
             "per_layer_ms": {d["name"]: g for d, g in zip(L, g_ms)},
         },
         "quant": {
@@ -368,6 +397,26 @@ def run_gpu(args):
             "bytes_per_step": q_bytes, "per_layer_ms": {d["name"]: q for d, q in zip(L, q_ms)},
             "peak_src": f"{peaks['src']} HBM copy",
         },
+    }
+
+    # ---- per-output-channel weight quantiser (run once per weight at load time)
+    wq_ms = []
+    for d in L:
+        Wb = d.pop("W")
+        wsq = ptpc.Workspace(ptpc.workspace_size(ptpc.OP_QUANTIZE_WEIGHTS, 0, d["Ci"], d["Co"]), dev)
+        for _ in range(2):
+            ptpc.quantize_weights(Wb, ws=wsq)
+        n_it = 5
+        wq_ms.append(max_over_ranks(timed(lambda: ptpc.quantize_weights(Wb, ws=wsq), n_it)) / n_it)
+        del Wb
+    wq_elems = sum(d["Ci"] * d["Co"] for d in L)
+    wq_bytes = sum(3 * d["Ci"] * d["Co"] + 4 * d["Co"] for d in L)
+    line["quant_weights"] = {
+        "value": wq_bytes / (sum(wq_ms) / 1e3) / 1e9, "unit": "GB/s", "peak": peaks["hbm_gbs"],
+        "frac": wq_bytes / (sum(wq_ms) / 1e3) / 1e9 / peaks["hbm_gbs"],
+        "algorithmic_bytes": wq_bytes, "kernel_bytes": 5 * wq_elems + 8 * sum(d["Co"] for d in L),
+        "per_layer_ms": {d["name"]: t for d, t in zip(L, wq_ms)},
+        "note": "one-time, at weight load; the kernel reads W twice (column maxima, then codes)",
     }
 
     if not args.no_extras:
@@ -439,10 +488,139 @@ def run_gpu(args):
     return 0
 
 
+def run_quant_only(args):
+    """Times ptpc_quantize_activations alone on every layer input of the
+    workload (no weights are generated)."""
+    import torch
+
+    import fp8_quantized_gemm_ptpc_b200 as ptpc
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    wl = WORKLOADS[args.workload]
+    T = args.tokens or wl.tokens[0]
+    layers = workload_layers(wl, T)
+    peaks = load_peaks()
+    bufs = []
+    for i, name, T_, Ci, Co in layers:
+        X = torch.from_numpy(synthetic.make_x(wl, i, T_, Ci).view(np.int16)).to(dev).view(torch.bfloat16)
+        bufs.append((name, X, torch.empty((T_, Ci), dtype=torch.uint8, device=dev),
+                     torch.empty((T_,), dtype=torch.float32, device=dev)))
+    K, W = args.steps, max(3, args.warmup)
+    for _ in range(W):
+        for _, X, Xq, xs in bufs:
+            ptpc.quantize_activations(X, Xq, xs)
+    per = {}
+    with ClockSampler(dev.index or 0) as clk:
+        for name, X, Xq, xs in bufs:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record(stream)
+            for _ in range(K):
+                ptpc.quantize_activations(X, Xq, xs)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            per[name] = e0.elapsed_time(e1) / K
+    total_bytes = sum(quant_bytes(X.shape[0], X.shape[1]) for _, X, _, _ in bufs)
+    gbs = total_bytes / (sum(per.values()) / 1e3) / 1e9
+    print(json.dumps({
+        "metric": "per-token activation quantiser GB/s (algorithmic 3 B/element + 4 B/row)", "value": gbs,
+        "unit": "GB/s", "n_gpus": 1, "steps": K, "warmup": W, "higher_is_better": True,
+        "frac_of_hbm": gbs / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"], "data": "synthetic",
+        "config": {"workload": wl.name, "tokens": T, "inputs": [[X.shape[0], X.shape[1]] for _, X, _, _ in bufs]},
+        "per_input_ms": per, "clocks": clk.summary(),
+    }), flush=True)
+    return 0
+
+
+def run_sweep(args):
+    """The 70B-shaped chain QKV -> O -> gate+up -> down with dynamic per-token
+    re-quantisation between layers: O reads QKV output columns [0, 8192) and
+    down reads gate+up output columns [0, 28672) (column slices, no copies).
+    Three paths are timed side by side for every T: the fused PTPC entry
+    point, the page's naive two-step path (unscaled fp32 GEMM, then a scaling
+    kernel) and per-tensor scaling."""
+    import torch
+
+    import fp8_quantized_gemm_ptpc_b200 as ptpc
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    wl = synthetic.CHAIN_70B
+    tokens = ([int(t) for t in args.sweep_tokens.split(",")] if args.sweep_tokens else list(wl.tokens))
+    peaks = load_peaks()
+    Ws = []
+    for i, L in enumerate(wl.layers):
+        Wb = torch.from_numpy(synthetic.make_w(wl, i, L.Ci, L.Co).view(np.int16)).to(dev).view(torch.bfloat16)
+        Ws.append((L, ptpc.quantize_weights(Wb), ptpc.quantize_weights_per_tensor(Wb)))
+        del Wb
+    # chain inputs: layer l reads columns [0, Ci) of the previous layer's output
+    flops_tok = sum(2.0 * L.Ci * L.Co for L, _, _ in Ws)
+    for T in tokens:
+        X0 = torch.from_numpy(synthetic.make_x(wl, 0, T, wl.layers[0].Ci).view(np.int16)).to(dev).view(torch.bfloat16)
+        outs = [torch.empty((T, L.Co), dtype=torch.bfloat16, device=dev) for L, _, _ in Ws]
+        wsps = [ptpc.Workspace(ptpc.workspace_size(ptpc.OP_LINEAR, T, L.Ci, L.Co), dev) for L, _, _ in Ws]
+        ys = [torch.empty((T, L.Co), dtype=torch.float32, device=dev) for L, _, _ in Ws]
+        qs = [(torch.empty((T, L.Ci), dtype=torch.uint8, device=dev), torch.empty((T,), dtype=torch.float32, device=dev))
+              for L, _, _ in Ws]
+        pts = [ptpc.Workspace(ptpc.workspace_size(ptpc.OP_BENCH_PER_TENSOR, T, L.Ci, 0), dev) for L, _, _ in Ws]
+
+        def layer_input(i):
+            return X0 if i == 0 else outs[i - 1][:, :Ws[i][0].Ci]
+
+        def fused():
+            for i, (L, (Wq, ws), _) in enumerate(Ws):
+                ptpc.linear(layer_input(i), Wq, ws, out=outs[i], ws=wsps[i])
+
+        def naive():
+            for i, (L, (Wq, ws), _) in enumerate(Ws):
+                Xq, xs = ptpc.quantize_activations(layer_input(i), *qs[i])
+                ptpc.unscaled_mm_f32(Xq, Wq, out=ys[i], ws=wsps[i])
+                ptpc.apply_scales(ys[i], xs, ws, out=outs[i])
+
+        def per_tensor():
+            for i, (L, _, (Wq, ws)) in enumerate(Ws):
+                Xq, xs = ptpc.quantize_activations_per_tensor(layer_input(i), *qs[i], ws=pts[i])
+                ptpc.scaled_mm(Xq, xs, Wq, ws, out=outs[i], ws=wsps[i])
+
+        K = max(3, min(200, int(4e13 / (flops_tok * T))))
+        res = {}
+        for name, fn in (("fused", fused), ("naive", naive), ("per_tensor", per_tensor)):
+            for _ in range(3):
+                fn()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record(stream)
+            for _ in range(K):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            res[name] = e0.elapsed_time(e1) / K
+        print(json.dumps({
+            "kind": "chain_sweep", "workload": wl.name, "T": T, "steps": K,
+            "fused_ms": res["fused"], "naive_ms": res["naive"], "per_tensor_ms": res["per_tensor"],
+            "fused_tflops": flops_tok * T / (res["fused"] / 1e3) / 1e12,
+            "fused_frac_of_fp8_peak": flops_tok * T / (res["fused"] / 1e3) / 1e12 / (2.0 * peaks["bf16_tflops"]),
+            "fused_speedup_over_naive": res["naive"] / res["fused"],
+            "ptpc_over_per_tensor_throughput": res["per_tensor"] / res["fused"],
+        }), flush=True)
+        del X0, outs, wsps, ys, qs, pts
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.quant_only:
+        return run_quant_only(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_gpu(args)
 
 

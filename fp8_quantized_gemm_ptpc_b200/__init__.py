@@ -45,17 +45,17 @@ _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
 _SZ = ctypes.c_size_t
 SIGNATURES = {
-    "ptpc_quantize_activations": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P]),
+    "ptpc_quantize_activations": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "ptpc_quantize_weights": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "ptpc_scaled_mm": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
-    "ptpc_linear": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "ptpc_linear": (ctypes.c_int, [_P, _I64, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "ptpc_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _I64, _I64, _I64]),
     "ptpc_get_device_status": (ctypes.c_int, [_P, _P]),
     "ptpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ptpc_scaled_mm_static_scratch": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "ptpc_bench_unscaled_mm_f32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "ptpc_bench_apply_scales": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _P, _P]),
-    "ptpc_bench_quantize_activations_per_tensor": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _SZ, _P]),
+    "ptpc_bench_quantize_activations_per_tensor": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "ptpc_bench_quantize_weights_per_tensor": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _SZ, _P]),
 }
 
@@ -115,6 +115,18 @@ def _need(t: torch.Tensor, name: str, dtype, ndim: int):
         raise ValueError(f"{name} must be a contiguous {ndim}-d tensor")
 
 
+def _need_rows(t: torch.Tensor, name: str) -> int:
+    """A bf16 [rows, cols] tensor whose rows are contiguous (a dense tensor or
+    a column slice of one); returns the row pitch in elements."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be torch.bfloat16, got {t.dtype}")
+    if t.dim() != 2 or (t.shape[1] > 1 and t.stride(1) != 1):
+        raise ValueError(f"{name} must be a 2-d tensor with contiguous rows")
+    return t.stride(0) if t.shape[0] > 1 else t.shape[1]
+
+
 class Workspace:
     """A zero-filled device buffer for the entry points that take (ws, ws_bytes).
 
@@ -155,13 +167,14 @@ def default_workspace(nbytes: int, device) -> Workspace:
 # ----------------------------------------------------------------- entry points
 
 def quantize_activations(X: torch.Tensor, Xq: torch.Tensor | None = None, x_scale: torch.Tensor | None = None):
-    """Per-token quantisation: X bf16 [T, Ci] -> (Xq uint8 [T, Ci], x_scale fp32 [T])."""
-    _need(X, "X", torch.bfloat16, 2)
+    """Per-token quantisation: X bf16 [T, Ci] (rows contiguous; a column slice
+    is fine) -> (Xq uint8 [T, Ci], x_scale fp32 [T])."""
+    ldx = _need_rows(X, "X")
     T, Ci = X.shape
     Xq = torch.empty((T, Ci), dtype=torch.uint8, device=X.device) if Xq is None else Xq
     x_scale = torch.empty((T,), dtype=torch.float32, device=X.device) if x_scale is None else x_scale
     _check("ptpc_quantize_activations",
-           lib.ptpc_quantize_activations(_ptr(X), T, Ci, _ptr(Xq), _ptr(x_scale), _stream(X.device)))
+           lib.ptpc_quantize_activations(_ptr(X), T, Ci, ldx, _ptr(Xq), _ptr(x_scale), _stream(X.device)))
     return Xq, x_scale
 
 
@@ -199,8 +212,9 @@ def scaled_mm(Xq, x_scale, Wq_t, w_scale, out: torch.Tensor | None = None, ws: W
 
 
 def linear(X, Wq_t, w_scale, out: torch.Tensor | None = None, ws: Workspace | None = None):
-    """Fused quantise + GEMM: X bf16 [T, Ci] -> out bf16 [T, Co]."""
-    _need(X, "X", torch.bfloat16, 2)
+    """Fused quantise + GEMM: X bf16 [T, Ci] (rows contiguous; a column slice
+    is fine) -> out bf16 [T, Co]."""
+    ldx = _need_rows(X, "X")
     _need(Wq_t, "Wq_t", torch.uint8, 2)
     _need(w_scale, "w_scale", torch.float32, 1)
     T, Ci = X.shape
@@ -211,7 +225,7 @@ def linear(X, Wq_t, w_scale, out: torch.Tensor | None = None, ws: Workspace | No
     need = workspace_size(OP_LINEAR, T, Ci, Co)
     ws = default_workspace(need, X.device) if ws is None else ws.ensure(need)
     _check("ptpc_linear",
-           lib.ptpc_linear(_ptr(X), _ptr(Wq_t), _ptr(w_scale), T, Ci, Co, _ptr(out), ws.ptr(), ws.nbytes,
+           lib.ptpc_linear(_ptr(X), ldx, _ptr(Wq_t), _ptr(w_scale), T, Ci, Co, _ptr(out), ws.ptr(), ws.nbytes,
                            _stream(X.device)))
     return out
 
@@ -271,14 +285,14 @@ def apply_scales(y, x_scale, w_scale, out: torch.Tensor | None = None):
 
 def quantize_activations_per_tensor(X, Xq=None, x_scale=None, ws: Workspace | None = None):
     """Per-tensor quantisation of X; x_scale [T] holds the one tensor scale T times."""
-    _need(X, "X", torch.bfloat16, 2)
+    ldx = _need_rows(X, "X")
     T, Ci = X.shape
     Xq = torch.empty((T, Ci), dtype=torch.uint8, device=X.device) if Xq is None else Xq
     x_scale = torch.empty((T,), dtype=torch.float32, device=X.device) if x_scale is None else x_scale
     need = workspace_size(OP_BENCH_PER_TENSOR, T, Ci, 0)
     ws = default_workspace(need, X.device) if ws is None else ws.ensure(need)
     _check("ptpc_bench_quantize_activations_per_tensor",
-           lib.ptpc_bench_quantize_activations_per_tensor(_ptr(X), T, Ci, _ptr(Xq), _ptr(x_scale), ws.ptr(),
+           lib.ptpc_bench_quantize_activations_per_tensor(_ptr(X), T, Ci, ldx, _ptr(Xq), _ptr(x_scale), ws.ptr(),
                                                           ws.nbytes, _stream(X.device)))
     return Xq, x_scale
 

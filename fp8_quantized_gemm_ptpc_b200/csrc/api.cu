@@ -28,9 +28,9 @@ struct GemmLayout {
   size_t partial_floats;
 };
 
-GemmLayout gemm_layout(int64_t T, int64_t Ci, int64_t Co) {
+GemmLayout gemm_layout(int64_t T, int64_t Ci, int64_t Co, size_t max_partial_floats = SIZE_MAX) {
   size_t cw = 0, pf = 0;
-  ptpc::gemm_workspace_needs((int)T, (int)Ci, (int)Co, &cw, &pf);
+  ptpc::gemm_workspace_needs((int)T, (int)Ci, (int)Co, max_partial_floats, &cw, &pf);
   GemmLayout l;
   l.counters_off = kAlign;
   l.partials_off = l.counters_off + round_up(cw * 4);
@@ -63,6 +63,13 @@ int check_shape_tci(int64_t T, int64_t Ci) {
   return PTPC_OK;
 }
 
+// Row pitch of an activation: at least Ci elements, 16-byte rows.
+int check_ldx(int64_t ldx, int64_t Ci) {
+  if (ldx < Ci) return PTPC_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || ldx > kMaxDim) return PTPC_ERR_MISALIGNED;
+  return PTPC_OK;
+}
+
 int check_co(int64_t Co) {
   if (Co < 0) return PTPC_ERR_INVALID_ARG;
   if (Co == 0 || Co % 16 != 0 || Co > kMaxDim) return PTPC_ERR_UNSUPPORTED_SHAPE;
@@ -72,8 +79,9 @@ int check_co(int64_t Co) {
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? PTPC_OK : PTPC_ERR_CUDA; }
 
 int run_gemm(const uint8_t *Xq, const float *xs, const uint8_t *Wq_t, const float *ws, int64_t T, int64_t Ci,
-             int64_t Co, void *out, bool f32_out, uint8_t *wsp, bool pdl, cudaStream_t st) {
-  const GemmLayout l = gemm_layout(T, Ci, Co);
+             int64_t Co, void *out, bool f32_out, uint8_t *wsp, bool pdl, cudaStream_t st,
+             size_t max_partial_floats = SIZE_MAX) {
+  const GemmLayout l = gemm_layout(T, Ci, Co, max_partial_floats);
   ptpc::GemmProblem p{};
   p.Xq = Xq;
   p.xs = xs;
@@ -131,14 +139,16 @@ size_t ptpc_workspace_size(int op, int64_t T, int64_t Ci, int64_t Co) {
   }
 }
 
-int ptpc_quantize_activations(const void *X, int64_t T, int64_t Ci, uint8_t *Xq, float *x_scale, void *stream) {
+int ptpc_quantize_activations(const void *X, int64_t T, int64_t Ci, int64_t ldx, uint8_t *Xq, float *x_scale,
+                              void *stream) {
   int s = check_shape_tci(T, Ci);
   if (s != PTPC_OK) return s;
   if (T == 0) return PTPC_OK;
+  if ((s = check_ldx(ldx, Ci)) != PTPC_OK) return s;
   if (!X || !Xq || !x_scale) return PTPC_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(Xq) || !aligned16(x_scale)) return PTPC_ERR_MISALIGNED;
   if ((s = check_device()) != PTPC_OK) return s;
-  return cuda_status(ptpc::launch_quant_act(X, (int)T, (int)Ci, Xq, x_scale, (cudaStream_t)stream));
+  return cuda_status(ptpc::launch_quant_act(X, (int)T, (int)Ci, ldx, Xq, x_scale, (cudaStream_t)stream));
 }
 
 int ptpc_quantize_weights(const void *W, int64_t Ci, int64_t Co, uint8_t *Wq_t, float *w_scale, void *ws,
@@ -171,12 +181,13 @@ int ptpc_scaled_mm(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq_t,
                   (cudaStream_t)stream);
 }
 
-int ptpc_linear(const void *X, const uint8_t *Wq_t, const float *w_scale, int64_t T, int64_t Ci, int64_t Co,
-                void *out, void *ws, size_t ws_bytes, void *stream) {
+int ptpc_linear(const void *X, int64_t ldx, const uint8_t *Wq_t, const float *w_scale, int64_t T, int64_t Ci,
+                int64_t Co, void *out, void *ws, size_t ws_bytes, void *stream) {
   int s = check_shape_tci(T, Ci);
   if (s != PTPC_OK) return s;
   if ((s = check_co(Co)) != PTPC_OK) return s;
   if (T == 0) return PTPC_OK;
+  if ((s = check_ldx(ldx, Ci)) != PTPC_OK) return s;
   if (!X || !Wq_t || !w_scale || !out || !ws) return PTPC_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(Wq_t) || !aligned16(w_scale) || !aligned16(out) || !aligned16(ws))
     return PTPC_ERR_MISALIGNED;
@@ -187,7 +198,7 @@ int ptpc_linear(const void *X, const uint8_t *Wq_t, const float *w_scale, int64_
   uint8_t *Xq = wsp + g_end;
   float *xs = reinterpret_cast<float *>(wsp + g_end + round_up((size_t)T * (size_t)Ci));
   cudaStream_t st = (cudaStream_t)stream;
-  if ((s = cuda_status(ptpc::launch_quant_act(X, (int)T, (int)Ci, Xq, xs, st))) != PTPC_OK) return s;
+  if ((s = cuda_status(ptpc::launch_quant_act(X, (int)T, (int)Ci, ldx, Xq, xs, st))) != PTPC_OK) return s;
   return run_gemm(Xq, xs, Wq_t, w_scale, T, Ci, Co, out, false, wsp, true, st);
 }
 
@@ -229,18 +240,19 @@ int ptpc_bench_apply_scales(const float *y, const float *x_scale, const float *w
   return cuda_status(ptpc::launch_apply_scales(y, x_scale, w_scale, (int)T, (int)Co, out, (cudaStream_t)stream));
 }
 
-int ptpc_bench_quantize_activations_per_tensor(const void *X, int64_t T, int64_t Ci, uint8_t *Xq, float *x_scale,
-                                               void *ws, size_t ws_bytes, void *stream) {
+int ptpc_bench_quantize_activations_per_tensor(const void *X, int64_t T, int64_t Ci, int64_t ldx, uint8_t *Xq,
+                                               float *x_scale, void *ws, size_t ws_bytes, void *stream) {
   int s = check_shape_tci(T, Ci);
   if (s != PTPC_OK) return s;
   if (T == 0) return PTPC_OK;
+  if ((s = check_ldx(ldx, Ci)) != PTPC_OK) return s;
   if (!X || !Xq || !x_scale || !ws) return PTPC_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(Xq) || !aligned16(x_scale) || !aligned16(ws)) return PTPC_ERR_MISALIGNED;
   if (ws_bytes < ptpc_workspace_size(PTPC_OP_BENCH_PER_TENSOR, T, Ci, 0)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
   if ((s = check_device()) != PTPC_OK) return s;
   uint32_t *slot = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + kAlign);
   return cuda_status(
-      ptpc::launch_quant_act_per_tensor(X, (int)T, (int)Ci, Xq, x_scale, slot, (cudaStream_t)stream));
+      ptpc::launch_quant_act_per_tensor(X, (int)T, (int)Ci, ldx, Xq, x_scale, slot, (cudaStream_t)stream));
 }
 
 int ptpc_bench_quantize_weights_per_tensor(const void *W, int64_t Ci, int64_t Co, uint8_t *Wq_t, float *w_scale,
@@ -307,14 +319,17 @@ extern "C" int ptpc_scaled_mm_static_scratch(const uint8_t *Xq, const float *x_s
   if (!Xq || !x_scale || !Wq_t || !w_scale || !out) return PTPC_ERR_INVALID_ARG;
   if (!aligned16(Xq) || !aligned16(x_scale) || !aligned16(Wq_t) || !aligned16(w_scale) || !aligned16(out))
     return PTPC_ERR_MISALIGNED;
-  if (ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co) > kStaticScratchBytes) return PTPC_ERR_WORKSPACE_TOO_SMALL;
   if ((s = check_device()) != PTPC_OK) return s;
+  // Plan within the array: stream-K partial sums only when they fit in what
+  // is left after the status word and (at most 64 KiB of) tile counters.
+  const size_t budget_floats = (kStaticScratchBytes - kAlign - (size_t(64) << 10)) / sizeof(float);
+  const GemmLayout l = gemm_layout(T, Ci, Co, budget_floats);
+  if (l.end > kStaticScratchBytes) return PTPC_ERR_WORKSPACE_TOO_SMALL;
   uint8_t *scratch = nullptr;
   if ((s = static_scratch_address(&scratch)) != PTPC_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   // The array keeps the previous call's contents: the status word and the
-  // split-K counters must start at zero (the partial sums need not).
-  const GemmLayout l = gemm_layout(T, Ci, Co);
+  // stream-K tile counters must start at zero (the partial sums need not).
   if (cudaMemsetAsync(scratch, 0, l.partials_off, st) != cudaSuccess) return PTPC_ERR_CUDA;
-  return run_gemm(Xq, x_scale, Wq_t, w_scale, T, Ci, Co, out, false, scratch, false, st);
+  return run_gemm(Xq, x_scale, Wq_t, w_scale, T, Ci, Co, out, false, scratch, false, st, budget_floats);
 }

@@ -6,24 +6,33 @@
 // on AMD ROCm" (section "The challenge: two-step vs fused"): the two scale
 // vectors are applied to the accumulator on chip, between the tensor-memory
 // load and the single store of the output, so no T x Co intermediate is ever
-// written.  The page's kernel is AMD's (MI300X); this one is written for B200:
+// written.  The page's kernel is AMD's (MI300X); these are written for B200.
 //
-//   * persistent CTAs (one per SM) walk output tiles of 128 tokens x BN
-//     channels in an L2-friendly grouped order;
-//   * warp 0 (one thread) streams 128-byte-wide K slices of Xq and Wq_t with
-//     TMA into a STAGES-deep shared-memory ring (128-byte swizzle);
-//   * warp 1 (one thread) issues tcgen05.mma kind::f8f6f4 (E4M3 x E4M3 ->
-//     fp32, M = 128, N = BN, K = 32) into one of two tensor-memory
-//     accumulators, and commits each stage back to the producer;
-//   * warps 2-5 read the finished accumulator with tcgen05.ld (each warp owns
-//     one 32-lane quarter of tensor memory = 32 token rows), scale, round to
-//     bf16, stage the tile in swizzled shared memory and store it with TMA,
-//     while the MMA warp already fills the other accumulator.
-//   * For decode-sized T (one 128-row block) the K loop can be split over
-//     several CTAs (split-K).  Each writes an fp32 partial; the CTA that
-//     finishes a tile last (atomic counter, no waiting) sums the partials in
-//     split order, scales and stores.  The reduction order is fixed, so the
-//     result does not depend on which CTA finishes last.
+// Two kernels share the structure below.
+//   * ptpc_gemm_pair_kernel (T > 128, prefill): a cluster of two CTAs on two
+//     SMs computes 256 x 256 tiles with tcgen05.mma.cta_group::2.
+//   * ptpc_gemm_decode_kernel (T <= 128, decode): one CTA per SM, operands
+//     swapped — 128 weight rows are the MMA's M operand and the T tokens
+//     (padded to a multiple of 16) its N operand.
+// In both, warp 0 (one thread) streams 128-byte-wide K slices of Xq and Wq_t
+// with TMA into a shared-memory ring (128-byte swizzle, no multicast); warp 1
+// (one thread) issues the MMAs (E4M3 x E4M3 -> fp32, K = 32 each) into one of
+// two tensor-memory accumulators and commits every stage back to the
+// producer; warps 2-5 read the finished accumulator with tcgen05.ld (each
+// warp owns one 32-lane quarter), apply the two scales, round to bf16 and
+// store, while the MMA warp fills the other accumulator.
+//
+// Work schedule: the prefill kernel takes whole tiles round-robin over the
+// CTA pairs.  The decode kernel has few tiles (Co / 128) and each is a long
+// stream of weight bytes, so when there are fewer tiles than SMs it shares
+// them "stream-K" style: each CTA takes an equal contiguous range of all
+// tiles' K-blocks, so every SM streams the same number of weight bytes and a
+// tile may be computed in several K segments.  A segment that is not the
+// whole tile writes its fp32 partial sum to the workspace and bumps the
+// tile's arrival counter; the CTA that arrives last (no CTA ever waits for
+// another) adds the partials in segment order — a fixed order, so the result
+// does not depend on which CTA finishes last — applies the scales, stores,
+// and resets the counter for the next call.
 //
 // Every wait on an mbarrier is bounded (see mbar_wait); a wait that runs out
 // sets a bit in the device status word, and the CTA stops issuing work, lets
@@ -40,17 +49,26 @@ namespace ptpc {
 
 namespace {
 
-constexpr int BM = 128;      // tokens per tile (MMA M, tensor-memory lanes)
+constexpr int BM = 128;      // token rows per CTA tile (tensor-memory lanes)
 constexpr int BK = 128;      // K bytes per stage (= one 128-byte swizzle row)
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kPairBN = 256;    // CTA-pair tile width (MMA N)
+constexpr int kPairHalfN = 128; // weight rows each CTA of a pair loads
 
 struct GemmParams {
   int T, Co;
-  int num_m, num_n, num_kb;
-  int group_m;
-  int nsplit;
-  int num_units;
+  int num_m, num_n, num_kb;   // tile grid (rows of tiles are 128 or 256 tokens)
+  int group_m;                // tile rows visited together (L2 reuse of weights)
+  int num_tiles;
+  int dp_tiles;               // tiles [0, dp_tiles): whole, round-robin
+  int sk_ctas;                // CTAs (pairs) sharing tiles [dp_tiles, num_tiles)
+  int seg_slots;              // partial-sum slots per shared tile
+  long long sk_iters;         // (num_tiles - dp_tiles) * num_kb
+  int part_rows;              // rows of one partial-sum slot
+  int np;                     // decode kernel: tokens padded to the MMA's N (multiple of 16)
+  int stages;                 // decode kernel: shared-memory ring depth
+  int tmem_cols;              // decode kernel: tensor-memory columns allocated (two accumulators)
   const float *xs;
   const float *ws;
   void *out;
@@ -59,35 +77,67 @@ struct GemmParams {
   float *partials;
 };
 
-template <int BN, int STAGES, bool F32OUT>
-struct Cfg {
-  static constexpr int A_BYTES = BM * BK;
-  static constexpr int B_BYTES = BN * BK;
-  static constexpr int EPI_COLS = F32OUT ? 32 : 64;     // columns in one 128-byte output row chunk
-  static constexpr int EPI_BUF = 32 * 128;              // one warp's staging: 32 rows x 128 bytes
-  static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
-                                   : (2 * BN <= 256) ? 256 : 512;
-  static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + kEpiWarps * EPI_BUF +
-                                 kEpiWarps * 64 * sizeof(float) + 256;
-  static_assert(BN % EPI_COLS == 0, "BN must be a multiple of the epilogue chunk");
-  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
-  static_assert(SMEM <= 232448, "shared memory");
+// One piece of work: K-blocks [kb0, kb1) of tile `tile`, segment `seg` of
+// `nseg` (nseg == 1: the whole tile).
+struct Unit {
+  int tile, m, n, kb0, kb1, seg, nseg;
 };
 
-__device__ __forceinline__ void unit_coords(const GemmParams &p, int unit, int &m, int &n, int &kb0, int &kb1,
-                                            int &tile, int &split) {
-  tile = unit / p.nsplit;
-  split = unit - tile * p.nsplit;
-  const int per_group = p.group_m * p.num_n;
-  const int g = tile / per_group;
-  const int first_m = g * p.group_m;
-  const int gm = min(p.group_m, p.num_m - first_m);
-  const int r = tile - g * per_group;
-  m = first_m + r % gm;
-  n = r / gm;
-  kb0 = (int)(((long long)split * p.num_kb) / p.nsplit);
-  kb1 = (int)(((long long)(split + 1) * p.num_kb) / p.nsplit);
+__device__ __forceinline__ int sk_owner(const GemmParams &p, long long x) {
+  return (int)(((x + 1) * (long long)p.sk_ctas - 1) / p.sk_iters);
 }
+
+// The same sequence of units for the producer, the MMA issuer and the
+// epilogue of one CTA (pair) `id` out of `count`.
+struct Sched {
+  int id, dp_next, dp_step;
+  long long pos, end;
+
+  __device__ __forceinline__ void init(const GemmParams &p, int id_, int count) {
+    id = id_;
+    dp_next = id_;
+    dp_step = count;
+    if (id_ < p.sk_ctas) {
+      pos = (long long)id_ * p.sk_iters / p.sk_ctas;
+      end = (long long)(id_ + 1) * p.sk_iters / p.sk_ctas;
+    } else {
+      pos = end = 0;
+    }
+  }
+
+  __device__ __forceinline__ bool next(const GemmParams &p, Unit &u) {
+    if (dp_next < p.dp_tiles) {
+      u.tile = dp_next;
+      dp_next += dp_step;
+      u.kb0 = 0;
+      u.kb1 = p.num_kb;
+      u.seg = 0;
+      u.nseg = 1;
+    } else if (pos < end) {
+      const long long t = pos / p.num_kb;
+      const long long t_begin = t * p.num_kb, t_end = t_begin + p.num_kb;
+      const long long s_end = end < t_end ? end : t_end;
+      u.tile = p.dp_tiles + (int)t;
+      u.kb0 = (int)(pos - t_begin);
+      u.kb1 = (int)(s_end - t_begin);
+      const int first = sk_owner(p, t_begin);
+      u.seg = id - first;
+      u.nseg = sk_owner(p, t_end - 1) - first + 1;
+      pos = s_end;
+    } else {
+      return false;
+    }
+    // grouped raster: group_m tile rows, all tile columns, rows fastest
+    const int per_group = p.group_m * p.num_n;
+    const int g = u.tile / per_group;
+    const int first_m = g * p.group_m;
+    const int gm = min(p.group_m, p.num_m - first_m);
+    const int r = u.tile - g * per_group;
+    u.m = first_m + r % gm;
+    u.n = r / gm;
+    return true;
+  }
+};
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
 
@@ -96,13 +146,56 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Fused epilogue of one accumulator: 32 token rows (one TMEM lane quarter,
-// lane i = row store_row0 + i) x BN_T columns starting at global column
-// col_base.  fp32 -> (acc * x_scale) * w_scale -> bf16 (or the raw fp32
-// accumulator), staged as 32 x 128-byte chunks in 128-byte-swizzled shared
-// memory and written with TMA stores.  After the last tensor-memory read the
-// accumulator buffer is released by one arrival on `release_bar` (a
-// shared::cluster address: this CTA's barrier or the pair leader's).
+// Stages one warp's 32 rows x 128 bytes in 128-byte-swizzled shared memory and
+// stores them with TMA at (col, row).  `packed` holds this lane's row.
+__device__ __forceinline__ void stage_and_store(const CUtensorMap *tmC, uint8_t *cbuf, const uint32_t (&packed)[32],
+                                                int col, int row, int lane) {
+  // the previous TMA store from this buffer must have finished reading it
+  if (lane == 0) bulk_wait_read<0>();
+  __syncwarp();
+  #pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int pos = j ^ (lane & 7);
+    *reinterpret_cast<uint4 *>(cbuf + lane * 128 + pos * 16) =
+        make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+  }
+  fence_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmC, cbuf, col, row);
+    bulk_commit();
+  }
+}
+
+// Column scales of a 64-column chunk into this warp's scratch `sc`.
+__device__ __forceinline__ void load_col_scales(float *sc, const GemmParams &p, int col0, int lane) {
+  __syncwarp();
+  sc[lane] = (col0 + lane < p.Co) ? __ldg(p.ws + col0 + lane) : 0.0f;
+  sc[lane + 32] = (col0 + 32 + lane < p.Co) ? __ldg(p.ws + col0 + 32 + lane) : 0.0f;
+  __syncwarp();
+}
+
+// (acc * x_scale) * w_scale for 32 accumulators (raw fp32 bits), packed to
+// 16 bf16 pairs at packed[off .. off+15].
+__device__ __forceinline__ void scale_pack32(const uint32_t (&r)[32], float xsr, const float *sc,
+                                             uint32_t (&packed)[32], int off) {
+  #pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float4 wv = *reinterpret_cast<const float4 *>(sc + 4 * j);
+    const float v0 = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 0]), xsr), wv.x);
+    const float v1 = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 1]), xsr), wv.y);
+    const float v2 = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 2]), xsr), wv.z);
+    const float v3 = __fmul_rn(__fmul_rn(__uint_as_float(r[4 * j + 3]), xsr), wv.w);
+    packed[off + 2 * j] = pack_bf16x2(v0, v1);
+    packed[off + 2 * j + 1] = pack_bf16x2(v2, v3);
+  }
+}
+
+// Fused epilogue of one accumulator held in tensor memory: 32 token rows (one
+// lane quarter; lane i = row store_row0 + i) x BN_T columns from global
+// column col_base.  After the last tensor-memory read the accumulator buffer
+// is released by one arrival on `release_bar` (a shared::cluster address:
+// this CTA's barrier or the pair leader's).
 template <int BN_T, bool F32OUT>
 __device__ __forceinline__ void epilogue_store_tile(const CUtensorMap *tmC, uint32_t tbase, uint8_t *cbuf,
                                                     float *sc, const GemmParams &p, int col_base,
@@ -112,33 +205,17 @@ __device__ __forceinline__ void epilogue_store_tile(const CUtensorMap *tmC, uint
   for (int c0 = 0; c0 < BN_T; c0 += EPI_COLS) {
     uint32_t packed[32];
     if constexpr (F32OUT) {
+      tmem_ld_32x32b_x32(tbase + c0, packed);
+      tmem_wait_ld();
+    } else {
+      load_col_scales(sc, p, col_base + c0, lane);
       uint32_t r[32];
       tmem_ld_32x32b_x32(tbase + c0, r);
       tmem_wait_ld();
-      #pragma unroll
-      for (int j = 0; j < 32; ++j) packed[j] = r[j];
-    } else {
-      __syncwarp();
-      const int col0 = col_base + c0;
-      sc[lane] = (col0 + lane < p.Co) ? __ldg(p.ws + col0 + lane) : 0.0f;
-      sc[lane + 32] = (col0 + 32 + lane < p.Co) ? __ldg(p.ws + col0 + 32 + lane) : 0.0f;
-      uint32_t r0[32], r1[32];
-      tmem_ld_32x32b_x32(tbase + c0, r0);
-      tmem_ld_32x32b_x32(tbase + c0 + 32, r1);
+      scale_pack32(r, xsr, sc, packed, 0);
+      tmem_ld_32x32b_x32(tbase + c0 + 32, r);
       tmem_wait_ld();
-      __syncwarp();
-      #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float4 wv = *reinterpret_cast<const float4 *>(sc + 4 * j);
-        const uint32_t *rr = (j < 8) ? r0 : r1;
-        const int b = (j & 7) * 4;
-        const float v0 = __fmul_rn(__fmul_rn(__uint_as_float(rr[b + 0]), xsr), wv.x);
-        const float v1 = __fmul_rn(__fmul_rn(__uint_as_float(rr[b + 1]), xsr), wv.y);
-        const float v2 = __fmul_rn(__fmul_rn(__uint_as_float(rr[b + 2]), xsr), wv.z);
-        const float v3 = __fmul_rn(__fmul_rn(__uint_as_float(rr[b + 3]), xsr), wv.w);
-        packed[2 * j] = pack_bf16x2(v0, v1);
-        packed[2 * j + 1] = pack_bf16x2(v2, v3);
-      }
+      scale_pack32(r, xsr, sc + 32, packed, 16);
     }
     if (c0 + EPI_COLS >= BN_T) {
       // the whole accumulator has been read: hand it back to the MMA issuer
@@ -146,51 +223,192 @@ __device__ __forceinline__ void epilogue_store_tile(const CUtensorMap *tmC, uint
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(release_bar);
     }
-    // the previous TMA store from this buffer must have finished reading it
-    if (lane == 0) bulk_wait_read<0>();
-    __syncwarp();
-    #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int pos = j ^ (lane & 7);
-      *reinterpret_cast<uint4 *>(cbuf + lane * 128 + pos * 16) =
-          make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+    stage_and_store(tmC, cbuf, packed, col_base + c0, store_row0, lane);
+  }
+}
+
+// Last arriver of a shared decode tile: adds the nseg partial slots
+// ([token][channel], BM floats per token) in slot order, applies the scales
+// (or keeps fp32) and stores each token's 128 channels.  The four epilogue
+// warps split the tokens (warp ew takes tokens ew, ew + 4, ...), each lane
+// owns 4 consecutive channels (one 16-byte load per slot and token), and the
+// loads of RB tokens x SB slots are issued together (16 loads in flight per
+// lane), so a tile of 128 tokens in three slots costs about eight L2 round
+// trips per warp instead of one per token and slot.
+template <bool F32OUT>
+__device__ __forceinline__ void decode_reduce_tile(const GemmParams &p, const float *slot0, size_t slot_stride,
+                                                   int nseg, int col_base, int ew, int lane) {
+  constexpr int RB = 8;  // tokens per batch
+  constexpr int SB = 2;  // slots loaded together
+  const int c = lane * 4;
+  const bool col_ok = col_base + c < p.Co;  // Co % 16 == 0: the lane's 4 columns are valid together
+  float4 wv = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (!F32OUT && col_ok) wv = __ldg(reinterpret_cast<const float4 *>(p.ws + col_base + c));
+  for (int r0 = ew; r0 < p.T; r0 += kEpiWarps * RB) {
+    float4 acc[RB];
+    for (int sg0 = 0; sg0 < nseg; sg0 += SB) {
+      float4 v[SB][RB];
+      #pragma unroll
+      for (int k = 0; k < SB; ++k) {
+        #pragma unroll
+        for (int i = 0; i < RB; ++i) {
+          const int row = r0 + i * kEpiWarps;
+          v[k][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (sg0 + k < nseg && row < p.T)
+            v[k][i] = __ldcg(reinterpret_cast<const float4 *>(slot0 + (size_t)(sg0 + k) * slot_stride +
+                                                              (size_t)row * BM + c));
+        }
+      }
+      #pragma unroll
+      for (int k = 0; k < SB; ++k) {
+        if (sg0 + k >= nseg) break;
+        #pragma unroll
+        for (int i = 0; i < RB; ++i) {
+          if (sg0 + k == 0) {
+            acc[i] = v[k][i];
+          } else {
+            acc[i].x = __fadd_rn(acc[i].x, v[k][i].x);
+            acc[i].y = __fadd_rn(acc[i].y, v[k][i].y);
+            acc[i].z = __fadd_rn(acc[i].z, v[k][i].z);
+            acc[i].w = __fadd_rn(acc[i].w, v[k][i].w);
+          }
+        }
+      }
     }
-    fence_async_shared();
-    __syncwarp();
-    if (lane == 0) {
-      tma_store_2d(tmC, cbuf, col_base + c0, store_row0);
-      bulk_commit();
+    if (!col_ok) continue;
+    #pragma unroll
+    for (int i = 0; i < RB; ++i) {
+      const int row = r0 + i * kEpiWarps;
+      if (row >= p.T) continue;
+      if constexpr (F32OUT) {
+        *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (size_t)row * p.Co + col_base + c) = acc[i];
+      } else {
+        const float a = __ldg(p.xs + row);
+        const uint32_t lo = pack_bf16x2(__fmul_rn(__fmul_rn(acc[i].x, a), wv.x), __fmul_rn(__fmul_rn(acc[i].y, a), wv.y));
+        const uint32_t hi = pack_bf16x2(__fmul_rn(__fmul_rn(acc[i].z, a), wv.z), __fmul_rn(__fmul_rn(acc[i].w, a), wv.w));
+        *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) + (size_t)row * p.Co + col_base + c) =
+            make_uint2(lo, hi);
+      }
     }
   }
 }
 
-template <int BN, int STAGES, bool F32OUT>
+// ----------------------------------------------------------------------------
+// Decode kernel (T <= 128), operands swapped: acc^T = Wq_t . Xq^T.
+// The 128 weight rows of a channel tile are the MMA's M = 128 operand and the
+// T tokens, padded to NP (a multiple of 16), are its N operand.  A stage then
+// carries 16 KB of weights and only NP x 128 bytes of activations, instead of
+// a 128-row activation box that is mostly out-of-bounds fill, and the ring is
+// as deep as shared memory allows (12 stages at NP = 16).  Tensor-memory lane
+// = output channel, column = token: each epilogue thread owns one channel, so
+// w_scale is one register and every token's 32 channels of a warp are one
+// contiguous store.  Work is shared stream-K style as in the one-CTA kernel.
+// ----------------------------------------------------------------------------
+constexpr int kDecMaxStages = 16;
+constexpr int kDecWBytes = BM * BK;   // weight tile of one stage
+constexpr size_t kDecBarBytes = 512;  // barriers and flags after the ring
+constexpr size_t kDecSmemMax = 232448;
+
+__host__ __device__ constexpr size_t dec_smem_bytes(int np, int stages) {
+  return 1024 + (size_t)stages * (kDecWBytes + (size_t)np * BK) + kDecBarBytes;
+}
+
+// Whole tile: scales applied per (token, channel), one bf16 (or fp32) store
+// per token; the accumulator is released after its last tensor-memory read.
+template <bool F32OUT>
+__device__ __forceinline__ void decode_store_tile(const GemmParams &p, uint32_t tbase, int ch, float wsr,
+                                                  int lane, uint32_t release_bar) {
+  const bool ch_ok = ch < p.Co;
+  #pragma unroll 1
+  for (int c0 = 0; c0 < p.np; c0 += 16) {
+    uint32_t r[16];
+    tmem_ld_32x32b_x16(tbase + c0, r);
+    tmem_wait_ld();
+    if (c0 + 16 >= p.np) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(release_bar);
+    }
+    if (!ch_ok) continue;
+    #pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int t = c0 + j;
+      if (t < p.T) {
+        const float acc = __uint_as_float(r[j]);
+        if constexpr (F32OUT) {
+          static_cast<float *>(p.out)[(size_t)t * p.Co + ch] = acc;
+        } else {
+          const float v = __fmul_rn(__fmul_rn(acc, __ldg(p.xs + t)), wsr);
+          static_cast<__nv_bfloat16 *>(p.out)[(size_t)t * p.Co + ch] = __float2bfloat16_rn(v);
+        }
+      }
+    }
+  }
+}
+
+// Shared tile: this segment's partial sums go to its slot ([token][channel],
+// BM floats per token row, so a warp writes 128 contiguous bytes per token);
+// the last of the tile's segments to arrive adds all slots in slot order.
+template <bool F32OUT>
+__device__ __noinline__ void decode_segment(const GemmParams &p, const Unit &u, uint32_t tbase, float *slot0,
+                                            size_t slot_stride, uint32_t *counter, int q, int lane, int et,
+                                            int *last_flag, uint32_t release_bar) {
+  float *slot = slot0 + (size_t)u.seg * slot_stride + q * 32 + lane;
+  #pragma unroll 1
+  for (int c0 = 0; c0 < p.np; c0 += 16) {
+    uint32_t r[16];
+    tmem_ld_32x32b_x16(tbase + c0, r);
+    tmem_wait_ld();
+    #pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int t = c0 + j;
+      if (t < p.T) __stcg(slot + (size_t)t * BM, __uint_as_float(r[j]));
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive_cluster(release_bar);
+  __threadfence();
+  epi_bar();
+  if (et == 0) {
+    const uint32_t prev = atomicAdd(counter, 1u);
+    *last_flag = (prev == (uint32_t)(u.nseg - 1)) ? 1 : 0;
+  }
+  epi_bar();
+  if (*last_flag) {
+    __threadfence();
+    decode_reduce_tile<F32OUT>(p, slot0, slot_stride, u.nseg, u.n * BM, et >> 5, lane);
+    if (et == 0) *counter = 0u;  // ready for the next call
+  }
+  epi_bar();
+}
+
+template <bool F32OUT>
 __global__ void __launch_bounds__(kThreads, 1)
-    ptpc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
-  using C = Cfg<BN, STAGES, F32OUT>;
+    ptpc_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                            const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sA = smem;
-  uint8_t *sB = sA + STAGES * C::A_BYTES;
-  uint8_t *sC = sB + STAGES * C::B_BYTES;
-  float *sScale = reinterpret_cast<float *>(sC + kEpiWarps * C::EPI_BUF);
-  uint64_t *full = reinterpret_cast<uint64_t *>(sScale + kEpiWarps * 64);
-  uint64_t *empty = full + STAGES;
-  uint64_t *tfull = empty + STAGES;
+  const int STAGES = p.stages;
+  const int X_BYTES = p.np * BK;
+  uint8_t *sW = smem;
+  uint8_t *sX = sW + STAGES * kDecWBytes;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sX + STAGES * X_BYTES);
+  uint64_t *empty = full + kDecMaxStages;
+  uint64_t *tfull = empty + kDecMaxStages;
   uint64_t *tempty = tfull + 2;
   uint64_t *drain = tempty + 2;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
   int *last_flag = reinterpret_cast<int *>(tmem_holder + 1);
   int *vote = last_flag + 1;  // [kEpiWarps]
+  const uint32_t acc_cols = (uint32_t)p.tmem_cols / 2;  // column stride of the two accumulators
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
-    prefetch_tmap(&tmC);
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmX);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -203,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_alloc(tmem_holder, (uint32_t)p.tmem_cols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -214,65 +432,83 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (elect_one()) {
-      const uint64_t polA = policy_evict_last();
-      const uint64_t polB = policy_evict_first();
+      const uint64_t polW = policy_evict_first();  // every weight byte is read once
+      const uint64_t polX = policy_evict_last();   // every CTA reads the activations
+      const uint32_t stage_tx = (uint32_t)(kDecWBytes + X_BYTES);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      Sched sc;
+      Unit u;
+      // The weights never depend on the kernel launched just before this one:
+      // the first stages' weight tiles are requested before waiting for it.
+      int pre = 0;
+      sc.init(p, blockIdx.x, gridDim.x);
+      if (sc.next(p, u)) {
+        for (; pre < STAGES && u.kb0 + pre < u.kb1; ++pre) {
+          mbar_arrive_expect_tx(&full[pre], stage_tx);
+          tma_load_2d(sW + pre * kDecWBytes, &tmW, &full[pre], (u.kb0 + pre) * BK, u.n * BM, polW);
+        }
+      }
       griddep_wait();  // Xq may come from the kernel launched just before
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-        int m, n, kb0, kb1, tile, split;
-        unit_coords(p, u, m, n, kb0, kb1, tile, split);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1)) {
-            ok = false;
-            break;
+      int issued = 0;
+      sc.init(p, blockIdx.x, gridDim.x);
+      while (ok && sc.next(p, u)) {
+        for (int kb = u.kb0; kb < u.kb1; ++kb, ++issued) {
+          if (issued >= pre) {
+            if (!mbar_wait(&empty[stage], phase ^ 1)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[stage], stage_tx);
+            tma_load_2d(sW + stage * kDecWBytes, &tmW, &full[stage], kb * BK, u.n * BM, polW);
           }
-          mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES);
-          tma_load_2d(sA + stage * C::A_BYTES, &tmA, &full[stage], kb * BK, m * BM, polA);
-          tma_load_2d(sB + stage * C::B_BYTES, &tmB, &full[stage], kb * BK, n * BN, polB);
+          tma_load_2d(sX + stage * X_BYTES, &tmX, &full[stage], kb * BK, 0, polX);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
+      griddep_launch_dependents();
       if (!ok) {
         atomicOr(p.status, kStatusTimeoutProducer);
-        // let the loads already issued land before the CTA can exit
         for (int s = 0; s < STAGES; ++s) mbar_wait(&full[s], s < stage ? phase : phase ^ 1);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(BM, BN);
+      const uint32_t idesc = idesc_e4m3_f32(BM, p.np);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x, ++local) {
-        int m, n, kb0, kb1, tile, split;
-        unit_coords(p, u, m, n, kb0, kb1, tile, split);
+      Sched sc;
+      sc.init(p, blockIdx.x, gridDim.x);
+      Unit u;
+      while (ok && sc.next(p, u)) {
         const int buf = local & 1;
         const uint32_t aphase = (local >> 1) & 1;
+        ++local;
         if (!mbar_wait(&tempty[buf], aphase ^ 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem_base + (uint32_t)(buf * BN);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        const uint32_t d = tmem_base + (uint32_t)buf * acc_cols;
+        for (int kb = u.kb0; kb < u.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t ad = sw128_kmajor_desc(smem_u32(sA + stage * C::A_BYTES));
-          const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + stage * C::B_BYTES));
+          const uint64_t ad = sw128_kmajor_desc(smem_u32(sW + stage * kDecWBytes));
+          const uint64_t bd = sw128_kmajor_desc(smem_u32(sX + stage * X_BYTES));
           #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)
-            mma_e4m3(d, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+            mma_e4m3(d, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
+                     (kb > u.kb0 || kk > 0) ? 1u : 0u);
           mma_commit(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
@@ -283,124 +519,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&tfull[buf]);
       }
       if (!ok) atomicOr(p.status, kStatusTimeoutMma);
-      // every MMA issued above completes before the tensor memory is freed
       mma_commit(drain);
       mbar_wait(drain, 0);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;              // tensor-memory lane quarter = token rows q*32 .. q*32+31
-    const int ew = warp - 2;             // staging buffer index
-    const int et = threadIdx.x - 64;     // 0..127 within the epilogue warps
-    uint8_t *cbuf = sC + ew * C::EPI_BUF;
-    float *sc = sScale + ew * 64;
+    const int q = warp & 3;           // tensor-memory lane quarter = channels q*32 .. q*32+31
+    const int ew = warp - 2;
+    const int et = threadIdx.x - 64;  // 0..127 within the epilogue warps
     int local = 0;
     bool ok = true;
     griddep_wait();  // x_scale may come from the kernel launched just before
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++local) {
-      int m, n, kb0, kb1, tile, split;
-      unit_coords(p, u, m, n, kb0, kb1, tile, split);
+    Sched sc;
+    sc.init(p, blockIdx.x, gridDim.x);
+    Unit u;
+    while (sc.next(p, u)) {
       const int buf = local & 1;
       const uint32_t aphase = (local >> 1) & 1;
-      const int row = m * BM + q * 32 + lane;
-      float xsr = 0.0f;
-      if (!F32OUT && row < p.T) xsr = __ldg(p.xs + row);
-      // The decision to stop must be the same for every lane (tcgen05.ld is
-      // warp-collective) and, in split-K mode, for all four epilogue warps
-      // (they meet at named barriers below).
+      ++local;
+      const int ch = u.n * BM + q * 32 + lane;
+      const float wsr = (!F32OUT && ch < p.Co) ? __ldg(p.ws + ch) : 0.0f;
       bool got = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], aphase));
-      if (p.nsplit > 1) {
+      if (p.sk_ctas > 0) {
         if (lane == 0) vote[ew] = got ? 1 : 0;
         epi_bar();
         got = vote[0] && vote[1] && vote[2] && vote[3];
+        epi_bar();
       }
       if (!got) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
-
-      if (p.nsplit == 1) {
-        // ---- direct: scale, round, stage, TMA store
-        epilogue_store_tile<BN, F32OUT>(&tmC, tbase, cbuf, sc, p, n * BN, m * BM + q * 32, xsr, lane,
-                                        smem_u32(&tempty[buf]));
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * acc_cols;
+      if (u.nseg == 1) {
+        decode_store_tile<F32OUT>(p, tbase, ch, wsr, lane, smem_u32(&tempty[buf]));
       } else {
-        // ---- split-K: fp32 partial of this K range, last CTA reduces
-        const int prow = p.T;  // split-K runs with a single 128-row block: rows 0..T-1
-        float *part = p.partials + ((size_t)tile * p.nsplit + split) * (size_t)prow * BN;
-        const bool warp_has_rows = q * 32 < prow;
-        if (warp_has_rows) {
-          #pragma unroll 1
-          for (int c0 = 0; c0 < BN; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(tbase + c0, r);
-            tmem_wait_ld();
-            if (row < prow) {
-              float4 *dst = reinterpret_cast<float4 *>(part + (size_t)row * BN + c0);
-              #pragma unroll
-              for (int j = 0; j < 8; ++j)
-                __stcg(dst + j, make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                            __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[buf]);
-        __threadfence();
-        epi_bar();
-        if (et == 0) {
-          const uint32_t prev = atomicAdd(p.counters + tile, 1u);
-          *last_flag = (prev == (uint32_t)(p.nsplit - 1)) ? 1 : 0;
-        }
-        epi_bar();
-        if (*last_flag) {
-          __threadfence();
-          const float *base = p.partials + (size_t)tile * p.nsplit * (size_t)prow * BN;
-          const int nv = prow * (BN / 4);
-          for (int i = et; i < nv; i += 32 * kEpiWarps) {
-            const int r = i / (BN / 4);
-            const int c = (i - r * (BN / 4)) * 4;
-            float4 acc = __ldcg(reinterpret_cast<const float4 *>(base + (size_t)r * BN + c));
-            for (int s = 1; s < p.nsplit; ++s) {
-              const float4 v = __ldcg(reinterpret_cast<const float4 *>(base + ((size_t)s * prow + r) * BN + c));
-              acc.x = __fadd_rn(acc.x, v.x);
-              acc.y = __fadd_rn(acc.y, v.y);
-              acc.z = __fadd_rn(acc.z, v.z);
-              acc.w = __fadd_rn(acc.w, v.w);
-            }
-            const int col = n * BN + c;
-            if (col < p.Co) {  // Co % 16 == 0: the 4 columns are all in range
-              if constexpr (F32OUT) {
-                *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (size_t)r * p.Co + col) = acc;
-              } else {
-                const float a = __ldg(p.xs + r);
-                const float4 wv = __ldg(reinterpret_cast<const float4 *>(p.ws + col));
-                uint2 o;
-                o.x = pack_bf16x2(__fmul_rn(__fmul_rn(acc.x, a), wv.x), __fmul_rn(__fmul_rn(acc.y, a), wv.y));
-                o.y = pack_bf16x2(__fmul_rn(__fmul_rn(acc.z, a), wv.z), __fmul_rn(__fmul_rn(acc.w, a), wv.w));
-                *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) + (size_t)r * p.Co + col) = o;
-              }
-            }
-          }
-          if (et == 0) p.counters[tile] = 0u;  // ready for the next call
-        }
-        epi_bar();
+        const int sk_tile = u.tile - p.dp_tiles;
+        const size_t slot_stride = (size_t)p.part_rows * BM;
+        float *slot0 = p.partials + (size_t)sk_tile * p.seg_slots * slot_stride;
+        decode_segment<F32OUT>(p, u, tbase, slot0, slot_stride, p.counters + sk_tile, q, lane, et, last_flag,
+                               smem_u32(&tempty[buf]));
       }
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeoutEpilogue);
-    if (lane == 0) bulk_wait<0>();
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    tmem_dealloc(tmem_base, (uint32_t)p.tmem_cols);
   }
 }
-
 
 // ----------------------------------------------------------------------------
 // CTA-pair kernel (prefill): a cluster of two CTAs on two SMs computes a
@@ -411,12 +582,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // issues every MMA, reading both CTAs' shared memory, and its commits arrive
 // on the barriers of both CTAs.  Each CTA's tensor memory holds its 128 token
 // rows x 256 columns, which its own epilogue warps store.  Per SM this moves
-// 32 KB of operands per 128-deep K-block instead of 48 KB for the one-CTA
+// 32 KB of operands per 128-deep K-block instead of 48 KB for a one-CTA
 // 128 x 256 tile, for the same tensor work.
 // ----------------------------------------------------------------------------
-constexpr int kPairBN = 256;
-constexpr int kPairHalfN = 128;
-
 template <int STAGES, bool F32OUT>
 struct PairCfg {
   static constexpr int A_BYTES = BM * BK;
@@ -485,27 +653,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
+      Sched sc;
+      Unit u;
+      // weight tiles of the first stages before waiting for the previous kernel
+      int pre = 0;
+      sc.init(p, cid, ncl);
+      if (sc.next(p, u)) {
+        const int b_row = u.n * kPairBN + (int)rank * kPairHalfN;
+        for (; pre < STAGES && u.kb0 + pre < u.kb1; ++pre) {
+          if (leader) mbar_arrive_expect_tx(&full[pre], 2 * (C::A_BYTES + C::B_BYTES));
+          tma_load_2d_pair(sB + pre * C::B_BYTES, &tmB, mapa_shared(&full[pre], 0), (u.kb0 + pre) * BK, b_row,
+                           polB);
+        }
+      }
       griddep_wait();
-      for (int u = cid; u < p.num_units && ok; u += ncl) {
-        int m, n, kb0, kb1, tile, split;
-        unit_coords(p, u, m, n, kb0, kb1, tile, split);
-        const int a_row = m * (2 * BM) + (int)rank * BM;
-        const int b_row = n * kPairBN + (int)rank * kPairHalfN;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1)) {
-            ok = false;
-            break;
-          }
+      int issued = 0;
+      sc.init(p, cid, ncl);
+      while (ok && sc.next(p, u)) {
+        const int a_row = u.m * (2 * BM) + (int)rank * BM;
+        const int b_row = u.n * kPairBN + (int)rank * kPairHalfN;
+        for (int kb = u.kb0; kb < u.kb1; ++kb, ++issued) {
           const uint32_t lead_full = mapa_shared(&full[stage], 0);
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (C::A_BYTES + C::B_BYTES));
+          if (issued >= pre) {
+            if (!mbar_wait(&empty[stage], phase ^ 1)) {
+              ok = false;
+              break;
+            }
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (C::A_BYTES + C::B_BYTES));
+            tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, lead_full, kb * BK, b_row, polB);
+          }
           tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, lead_full, kb * BK, a_row, polA);
-          tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, lead_full, kb * BK, b_row, polB);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
+      griddep_launch_dependents();
       if (!ok) {
         atomicOr(p.status, kStatusTimeoutProducer);
         // the leader's stage barriers count both CTAs' bytes: once they have
@@ -522,18 +706,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int u = cid; u < p.num_units && ok; u += ncl, ++local) {
-        int m, n, kb0, kb1, tile, split;
-        unit_coords(p, u, m, n, kb0, kb1, tile, split);
+      Sched sc;
+      sc.init(p, cid, ncl);
+      Unit u;
+      while (ok && sc.next(p, u)) {
         const int buf = local & 1;
         const uint32_t aphase = (local >> 1) & 1;
+        ++local;
         if (!mbar_wait(&tempty[buf], aphase ^ 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d = tmem_base + (uint32_t)(buf * kPairBN);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = u.kb0; kb < u.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase)) {
             ok = false;
             break;
@@ -544,7 +730,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)
             mma_e4m3_pair(d, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
-                          (kb > kb0 || kk > 0) ? 1u : 0u);
+                          (kb > u.kb0 || kk > 0) ? 1u : 0u);
           mma_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == STAGES) {
             stage = 0;
@@ -563,27 +749,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int ew = warp - 2;
     uint8_t *cbuf = sC + ew * C::EPI_BUF;
-    float *sc = sScale + ew * 64;
+    float *scl = sScale + ew * 64;
     int local = 0;
     bool ok = true;
     griddep_wait();
-    for (int u = cid; u < p.num_units; u += ncl, ++local) {
-      int m, n, kb0, kb1, tile, split;
-      unit_coords(p, u, m, n, kb0, kb1, tile, split);
+    Sched sc;
+    sc.init(p, cid, ncl);
+    Unit u;
+    while (sc.next(p, u)) {
       const int buf = local & 1;
       const uint32_t aphase = (local >> 1) & 1;
-      const int row0 = m * (2 * BM) + (int)rank * BM + q * 32;
+      ++local;
+      const int row0 = u.m * (2 * BM) + (int)rank * BM + q * 32;
       const int row = row0 + lane;
       float xsr = 0.0f;
       if (!F32OUT && row < p.T) xsr = __ldg(p.xs + row);
-      const bool got = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], aphase));
-      if (!got) {
+      // tcgen05.ld is warp-collective: the whole warp stops or none of it
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], aphase))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kPairBN);
-      epilogue_store_tile<kPairBN, F32OUT>(&tmC, tbase, cbuf, sc, p, n * kPairBN, row0, xsr, lane,
+      epilogue_store_tile<kPairBN, F32OUT>(&tmC, tbase, cbuf, scl, p, u.n * kPairBN, row0, xsr, lane,
                                            mapa_shared(&tempty[buf], 0));
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeoutEpilogue);
@@ -629,180 +817,232 @@ bool make_map_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, bool F32OUT>
-cudaError_t launch_cfg(const GemmProblem &pr, const GemmParams &gp, int grid, cudaStream_t st) {
-  using C = Cfg<BN, STAGES, F32OUT>;
-  auto kernel = ptpc_gemm_kernel<BN, STAGES, F32OUT>;
-  static bool attr_done[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_done[dev] = true;
-  }
-  CUtensorMap tmA, tmB, tmC;
-  if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Xq, pr.Ci, pr.T, pr.Ci, BK, BM,
+bool make_maps(const GemmProblem &pr, uint32_t b_rows, CUtensorMap *tmA, CUtensorMap *tmB, CUtensorMap *tmC) {
+  if (!make_map_2d(tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Xq, pr.Ci, pr.T, pr.Ci, BK, BM,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Wq_t, pr.Ci, pr.Co, pr.Ci, BK, BN,
+      !make_map_2d(tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Wq_t, pr.Ci, pr.Co, pr.Ci, BK, b_rows,
                    CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  bool okC;
-  if (F32OUT)
-    okC = make_map_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.out, pr.Co, pr.T, (uint64_t)pr.Co * 4, 32, 32,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
-  else
-    okC = make_map_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.out, pr.Co, pr.T, (uint64_t)pr.Co * 2, 64, 32,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!okC) return cudaErrorInvalidValue;
+    return false;
+  if (pr.f32_out)
+    return make_map_2d(tmC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.out, pr.Co, pr.T, (uint64_t)pr.Co * 4, 32, 32,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  return make_map_2d(tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.out, pr.Co, pr.T, (uint64_t)pr.Co * 2, 64, 32,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
 
+constexpr int kPairStages = 6;
+
+// Per device: dynamic shared-memory opt-in of every kernel variant, the SM
+// count, and the number of CTA pairs that can be resident at once.
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 148;
+  int pair_clusters = 74;
+};
+
+DeviceInfo &device_info() {
+  static DeviceInfo info[64];
+  static DeviceInfo fallback;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return fallback;
+  }
+  DeviceInfo &d = info[dev];
+  if (!d.ready) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) d.sms = v;
+    cudaFuncSetAttribute(ptpc_gemm_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)kDecSmemMax);
+    cudaFuncSetAttribute(ptpc_gemm_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)kDecSmemMax);
+    cudaFuncSetAttribute(ptpc_gemm_pair_kernel<kPairStages, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)PairCfg<kPairStages, false>::SMEM);
+    cudaFuncSetAttribute(ptpc_gemm_pair_kernel<kPairStages, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)PairCfg<kPairStages, true>::SMEM);
+    cudaLaunchConfig_t q = {};
+    q.gridDim = dim3(2 * (d.sms / 2));
+    q.blockDim = dim3(kThreads);
+    q.dynamicSmemBytes = PairCfg<kPairStages, false>::SMEM;
+    int ncl = 0;
+    if (cudaOccupancyMaxActiveClusters(&ncl, ptpc_gemm_pair_kernel<kPairStages, false>, &q) == cudaSuccess &&
+        ncl > 0)
+      d.pair_clusters = ncl;
+    else
+      d.pair_clusters = d.sms / 2;
+    cudaGetLastError();
+    d.ready = true;
+  }
+  return d;
+}
+
+// The launch plan of one problem; the workspace query and the launch both
+// derive from it, so they always agree.
+struct Plan {
+  bool pair;
+  int tile_rows, bn;
+  int num_m, num_n, num_kb, num_tiles;
+  int group_m;
+  int ctas;            // CTAs (one-CTA kernel) or CTA pairs (pair kernel) launched
+  int dp_tiles, sk_ctas, seg_slots, part_rows;
+  long long sk_iters;
+  int np, stages, tmem_cols;  // decode kernel only
+  size_t counter_words, partial_floats;
+};
+
+Plan make_plan(int T, int Ci, int Co, size_t max_partial_floats) {
+  const DeviceInfo &d = device_info();
+  Plan pl = {};
+  pl.num_kb = (Ci + BK - 1) / BK;
+  pl.pair = T > BM;
+  if (pl.pair) {
+    pl.tile_rows = 2 * BM;
+    pl.bn = kPairBN;
+    pl.group_m = 8;
+  } else {
+    // decode kernel: one tile row holds every token; tiles are 128 channels
+    pl.tile_rows = std::max(T, 1);
+    pl.bn = BM;
+    pl.group_m = 1;
+    pl.np = std::max(16, (T + 15) / 16 * 16);
+    const size_t stage_bytes = kDecWBytes + (size_t)pl.np * BK;
+    pl.stages = (int)std::min<size_t>(kDecMaxStages, (kDecSmemMax - dec_smem_bytes(pl.np, 0)) / stage_bytes);
+    pl.tmem_cols = 64;  // each accumulator starts on a 32-column boundary
+    while (pl.tmem_cols < 2 * pl.np) pl.tmem_cols <<= 1;
+  }
+  pl.num_m = (T + pl.tile_rows - 1) / pl.tile_rows;
+  pl.num_n = (Co + pl.bn - 1) / pl.bn;
+  pl.num_tiles = pl.num_m * pl.num_n;
+  const int slots = pl.pair ? d.pair_clusters : d.sms;
+  pl.dp_tiles = pl.num_tiles;
+  pl.sk_ctas = 0;
+  pl.seg_slots = 1;
+  pl.sk_iters = 0;
+  if (pl.pair) {
+    // Whole tiles only.  Sharing the last partial wave stream-K style was
+    // measured slower on B200 for 256 x 256 tiles (e.g. 2048 x 4096 -> 6144:
+    // 73.8 us shared vs 43.1 us whole; 2048 x 14336 -> 4096: 136.8 vs 109.7):
+    // the fixup of 256 KB fp32 partials costs more than the idle pairs.
+    pl.part_rows = BM;
+  } else {
+    // decode: every SM streams the same number of weight K-blocks; segments
+    // long enough that partial sums stay small next to the weights they cover
+    const long long iters = (long long)pl.num_tiles * pl.num_kb;
+    const int min_seg = std::max(4, (T + 3) / 4);
+    const int sk = (int)std::min<long long>(slots, iters / min_seg);
+    if (sk > pl.num_tiles) {
+      pl.dp_tiles = 0;
+      pl.sk_ctas = sk;
+      pl.sk_iters = iters;
+    }
+    pl.part_rows = T;
+  }
+  if (pl.sk_ctas > 0) {
+    const long long per = pl.sk_iters / pl.sk_ctas;  // >= min_seg >= 4
+    pl.seg_slots = (int)((pl.num_kb + per - 1) / per) + 1;
+    const size_t sk_tiles = (size_t)(pl.num_tiles - pl.dp_tiles);
+    pl.counter_words = sk_tiles;
+    pl.partial_floats = sk_tiles * pl.seg_slots * (size_t)pl.part_rows * pl.bn;
+    if (pl.partial_floats > max_partial_floats) {
+      // no room for the partial sums: whole tiles only
+      pl.dp_tiles = pl.num_tiles;
+      pl.sk_ctas = 0;
+      pl.seg_slots = 1;
+      pl.sk_iters = 0;
+      pl.counter_words = 0;
+      pl.partial_floats = 0;
+    }
+  }
+  pl.ctas = std::max(1, std::min(pl.num_tiles, slots));
+  if (pl.sk_ctas > 0) pl.ctas = std::max(pl.ctas, std::min(slots, pl.sk_ctas));
+  return pl;
+}
+
+template <typename Kernel>
+cudaError_t launch_decode(Kernel kernel, int grid, size_t smem, const CUtensorMap &tmW, const CUtensorMap &tmX,
+                          const GemmParams &gp, bool pdl, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = pr.pdl ? 1 : 0;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmC, gp);
+  return cudaLaunchKernelEx(&cfg, kernel, tmW, tmX, gp);
 }
 
-template <int STAGES, bool F32OUT>
-cudaError_t launch_pair(const GemmProblem &pr, GemmParams gp, cudaStream_t st) {
-  using C = PairCfg<STAGES, F32OUT>;
-  auto kernel = ptpc_gemm_pair_kernel<STAGES, F32OUT>;
-  static bool attr_done[64] = {};
-  static int max_clusters[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const bool cache = dev >= 0 && dev < 64;
-  if (!cache || !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t q = {};
-    q.gridDim = dim3(2 * 74);
-    q.blockDim = dim3(kThreads);
-    q.dynamicSmemBytes = C::SMEM;
-    int ncl = 0;
-    if (cudaOccupancyMaxActiveClusters(&ncl, kernel, &q) != cudaSuccess || ncl <= 0) {
-      cudaGetLastError();
-      ncl = num_sms() / 2;
-    }
-    if (cache) {
-      max_clusters[dev] = ncl;
-      attr_done[dev] = true;
-    } else {
-      max_clusters[0] = ncl;
-    }
-  }
-  const int ncl = std::max(1, std::min(gp.num_units, cache ? max_clusters[dev] : max_clusters[0]));
-  CUtensorMap tmA, tmB, tmC;
-  if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Xq, pr.Ci, pr.T, pr.Ci, BK, BM,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Wq_t, pr.Ci, pr.Co, pr.Ci, BK, kPairHalfN,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  bool okC;
-  if (F32OUT)
-    okC = make_map_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.out, pr.Co, pr.T, (uint64_t)pr.Co * 4, 32, 32,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
-  else
-    okC = make_map_2d(&tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.out, pr.Co, pr.T, (uint64_t)pr.Co * 2, 64, 32,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!okC) return cudaErrorInvalidValue;
+template <typename Kernel>
+cudaError_t launch(Kernel kernel, int grid, size_t smem, const CUtensorMap &tmA, const CUtensorMap &tmB,
+                   const CUtensorMap &tmC, const GemmParams &gp, bool pdl, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * ncl);
+  cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = pr.pdl ? 1 : 0;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmC, gp);
-}
-
-struct Plan {
-  int bn;
-  int nsplit;
-};
-
-// Split-K only for a single 128-row block (decode-sized T): enough work units
-// to keep the SMs streaming weights, bounded partial-sum traffic.
-Plan choose_plan(int T, int Ci, int Co) {
-  Plan pl{256, 1};
-  const int sms = num_sms();
-  const int num_kb = (Ci + BK - 1) / BK;
-  if (T <= BM) {
-    pl.bn = 128;
-    const int tiles = (Co + pl.bn - 1) / pl.bn;
-    int best = 1;
-    for (int s = 1; s <= 16 && s <= num_kb / 2; ++s) {
-      // partial traffic (write + read) relative to the weight bytes of a tile
-      const double extra = (s > 1) ? (2.0 * s * T * 4.0) / (double)Ci : 0.0;
-      if (extra > 0.15) break;
-      best = s;
-      if (tiles * s >= sms) break;
-    }
-    pl.nsplit = best;
-  }
-  return pl;
 }
 
 }  // namespace
 
-int num_sms() {
-  static int n = []() {
-    int dev = 0, v = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    return v > 0 ? v : 148;
-  }();
-  return n;
-}
+int num_sms() { return device_info().sms; }
 
-void gemm_workspace_needs(int T, int Ci, int Co, size_t *counter_words, size_t *partial_floats) {
-  const Plan pl = choose_plan(T, Ci, Co);
-  const size_t tiles = (size_t)((T + BM - 1) / BM) * (size_t)((Co + pl.bn - 1) / pl.bn);
-  *counter_words = tiles;
-  *partial_floats = pl.nsplit > 1 ? tiles * pl.nsplit * (size_t)T * pl.bn : 0;
+void gemm_workspace_needs(int T, int Ci, int Co, size_t max_partial_floats, size_t *counter_words,
+                          size_t *partial_floats) {
+  const Plan pl = make_plan(T, Ci, Co, max_partial_floats);
+  *counter_words = pl.counter_words;
+  *partial_floats = pl.partial_floats;
 }
 
 cudaError_t launch_scaled_gemm(const GemmProblem &pr, cudaStream_t st) {
-  const Plan pl = choose_plan(pr.T, pr.Ci, pr.Co);
+  const Plan pl = make_plan(pr.T, pr.Ci, pr.Co, pr.partial_floats);
   GemmParams gp = {};
   gp.T = pr.T;
   gp.Co = pr.Co;
-  gp.num_m = (pr.T + BM - 1) / BM;
-  gp.num_n = (pr.Co + pl.bn - 1) / pl.bn;
-  gp.num_kb = (pr.Ci + BK - 1) / BK;
-  gp.group_m = 16;
-  gp.nsplit = pl.nsplit;
-  gp.num_units = gp.num_m * gp.num_n * gp.nsplit;
+  gp.num_m = pl.num_m;
+  gp.num_n = pl.num_n;
+  gp.num_kb = pl.num_kb;
+  gp.group_m = pl.group_m;
+  gp.num_tiles = pl.num_tiles;
+  gp.dp_tiles = pl.dp_tiles;
+  gp.sk_ctas = pl.sk_ctas;
+  gp.seg_slots = pl.seg_slots;
+  gp.sk_iters = pl.sk_iters;
+  gp.part_rows = pl.part_rows;
   gp.xs = pr.xs;
   gp.ws = pr.ws;
   gp.out = pr.out;
   gp.status = pr.status;
   gp.counters = pr.counters;
   gp.partials = pr.partials;
-  if (pl.nsplit > 1 && pr.partial_floats < (size_t)gp.num_n * pl.nsplit * (size_t)pr.T * pl.bn)
-    return cudaErrorInvalidValue;
-  if (pr.T > BM && pl.nsplit == 1) {
-    // CTA-pair 256 x 256 tiles
-    gp.num_m = (pr.T + 2 * BM - 1) / (2 * BM);
-    gp.num_n = (pr.Co + kPairBN - 1) / kPairBN;
-    gp.group_m = 8;
-    gp.num_units = gp.num_m * gp.num_n;
-    return pr.f32_out ? launch_pair<6, true>(pr, gp, st) : launch_pair<6, false>(pr, gp, st);
+  gp.np = pl.np;
+  gp.stages = pl.stages;
+  gp.tmem_cols = pl.tmem_cols;
+  if (!pl.pair) {
+    CUtensorMap tmW, tmX;
+    if (!make_map_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Wq_t, pr.Ci, pr.Co, pr.Ci, BK, BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Xq, pr.Ci, pr.T, pr.Ci, BK, pl.np,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+    const size_t smem = dec_smem_bytes(pl.np, pl.stages);
+    return pr.f32_out ? launch_decode(ptpc_gemm_decode_kernel<true>, pl.ctas, smem, tmW, tmX, gp, pr.pdl, st)
+                      : launch_decode(ptpc_gemm_decode_kernel<false>, pl.ctas, smem, tmW, tmX, gp, pr.pdl, st);
   }
-  const int grid = std::min(gp.num_units, num_sms());
-  if (pl.bn == 256) {
-    return pr.f32_out ? launch_cfg<256, 4, true>(pr, gp, grid, st) : launch_cfg<256, 4, false>(pr, gp, grid, st);
-  }
-  return pr.f32_out ? launch_cfg<128, 6, true>(pr, gp, grid, st) : launch_cfg<128, 6, false>(pr, gp, grid, st);
+  CUtensorMap tmA, tmB, tmC;
+  if (!make_maps(pr, kPairHalfN, &tmA, &tmB, &tmC)) return cudaErrorInvalidValue;
+  const int grid = 2 * pl.ctas;
+  return pr.f32_out ? launch(ptpc_gemm_pair_kernel<kPairStages, true>, grid, PairCfg<kPairStages, true>::SMEM, tmA,
+                             tmB, tmC, gp, pr.pdl, st)
+                    : launch(ptpc_gemm_pair_kernel<kPairStages, false>, grid, PairCfg<kPairStages, false>::SMEM,
+                             tmA, tmB, tmC, gp, pr.pdl, st);
 }
 
 }  // namespace ptpc

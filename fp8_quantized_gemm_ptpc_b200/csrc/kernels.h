@@ -9,8 +9,9 @@
 namespace ptpc {
 
 // Quantisers (quant.cu).
-cudaError_t launch_quant_act(const void *X, int T, int Ci, uint8_t *Xq, float *xs, cudaStream_t st);
-cudaError_t launch_quant_act_per_tensor(const void *X, int T, int Ci, uint8_t *Xq, float *xs,
+// ldx: row pitch of X in elements (>= Ci, multiple of 8).
+cudaError_t launch_quant_act(const void *X, int T, int Ci, int64_t ldx, uint8_t *Xq, float *xs, cudaStream_t st);
+cudaError_t launch_quant_act_per_tensor(const void *X, int T, int Ci, int64_t ldx, uint8_t *Xq, float *xs,
                                         uint32_t *amax_slot, cudaStream_t st);
 // col_amax: Co + 1 32-bit words of scratch.
 cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, float *w_scale, uint32_t *col_amax,
@@ -30,12 +31,16 @@ struct GemmProblem {
   uint32_t *status;       // device status word
   uint32_t *counters;     // split-K tile counters (zero on entry, zero on exit)
   float *partials;        // split-K fp32 partial sums
-  size_t partial_floats;  // capacity of `partials`
+  size_t partial_floats;  // capacity of `partials` (also caps the plan's partial sums)
   bool pdl;               // launch as a programmatic dependent of the previous kernel
 };
 
-// Workspace needs of the GEMM for a shape (counter words and partial floats).
-void gemm_workspace_needs(int T, int Ci, int Co, size_t *counter_words, size_t *partial_floats);
+// Workspace needs of the GEMM for a shape (counter words and partial floats)
+// when at most max_partial_floats partial-sum floats may be used (stream-K is
+// dropped for whole tiles when its partial sums would not fit).  A launch with
+// GemmProblem::partial_floats = the value returned here runs the same plan.
+void gemm_workspace_needs(int T, int Ci, int Co, size_t max_partial_floats, size_t *counter_words,
+                          size_t *partial_floats);
 cudaError_t launch_scaled_gemm(const GemmProblem &p, cudaStream_t st);
 
 int num_sms();

@@ -74,7 +74,36 @@ __device__ __forceinline__ uint32_t quant_pair(uint32_t w, const GroupScale &g) 
   return (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
 }
 
-// Eight bf16 (16 bytes) -> eight codes (8 bytes).
+// Fast path for two bf16 of one 32-bit word, with Blackwell's packed fp32x2
+// arithmetic: the same three IEEE operations as quotient(), two lanes per
+// instruction.  nx = -x is built during unpacking, so that
+//   q0 = RN((-x) * (-r)) = RN(x * r),  e = RN(q0 * s + (-x)),  q = RN(e * (-r) + q0)
+// (the residual form that keeps -0 as -0).  Returns the two E4M3 codes,
+// first element in the low byte.
+__device__ __forceinline__ uint32_t quant_pair_fast(uint32_t w, uint64_t s2, uint64_t nr2) {
+  const uint32_t nlo = (w << 16) ^ 0x80000000u;       // -x of the first element
+  const uint32_t nhi = (w & 0xFFFF0000u) ^ 0x80000000u;  // -x of the second element
+  uint64_t nx2, q0, e, q;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(nx2) : "r"(nlo), "r"(nhi));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(q0) : "l"(nx2), "l"(nr2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(e) : "l"(q0), "l"(s2), "l"(nx2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(q) : "l"(e), "l"(nr2), "l"(q0));
+  uint32_t qlo, qhi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(qlo), "=r"(qhi) : "l"(q));
+  uint16_t c;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "r"(qhi), "r"(qlo));
+  return (uint32_t)c;
+}
+
+// Eight bf16 (16 bytes) -> eight codes (8 bytes), fast path.
+__device__ __forceinline__ uint2 quant_vec_fast(const uint4 v, uint64_t s2, uint64_t nr2) {
+  uint2 o;
+  o.x = quant_pair_fast(v.x, s2, nr2) | (quant_pair_fast(v.y, s2, nr2) << 16);
+  o.y = quant_pair_fast(v.z, s2, nr2) | (quant_pair_fast(v.w, s2, nr2) << 16);
+  return o;
+}
+
+// Eight bf16 (16 bytes) -> eight codes (8 bytes), any mode.
 __device__ __forceinline__ uint2 quant_vec(const uint4 v, const GroupScale &g) {
   if (g.mode == kZeroGroup) return make_uint2(0u, 0u);
   uint2 o;
@@ -83,17 +112,41 @@ __device__ __forceinline__ uint2 quant_vec(const uint4 v, const GroupScale &g) {
   return o;
 }
 
-// max(|bf16|) as 16-bit magnitude bits, two lanes per 32-bit word.  For
-// finite values the order of the magnitude bits is the order of the values.
+__device__ __forceinline__ uint64_t pack2(float a) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "r"(__float_as_uint(a)));
+  return r;
+}
+
+// Quantises n vectors src[j0], src[j0 + step], ... of one group into
+// dst[j] (8 codes each), choosing the arithmetic once for the whole run.
+template <typename Src>
+__device__ __forceinline__ void quant_run(Src src, uint2 *dst, int j0, int n, int step, const GroupScale &g) {
+  if (g.mode == kFast) {
+    const uint64_t s2 = pack2(g.s), nr2 = pack2(-g.r);
+    for (int j = j0; j < n; j += step) dst[j] = quant_vec_fast(src(j), s2, nr2);
+  } else if (g.mode == kSlow) {
+    for (int j = j0; j < n; j += step) dst[j] = quant_vec(src(j), g);
+  } else {
+    for (int j = j0; j < n; j += step) dst[j] = make_uint2(0u, 0u);
+  }
+}
+
+// max(|bf16|) of a 16-byte vector folded into acc (bf16x2 magnitudes; the
+// sign bits of acc are meaningless).  One max.xorsign.abs per two elements.
 __device__ __forceinline__ uint32_t absmax_bits(uint32_t acc, uint4 v) {
-  acc = __vmaxu2(acc, v.x & 0x7FFF7FFFu);
-  acc = __vmaxu2(acc, v.y & 0x7FFF7FFFu);
-  acc = __vmaxu2(acc, v.z & 0x7FFF7FFFu);
-  acc = __vmaxu2(acc, v.w & 0x7FFF7FFFu);
+  asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(acc) : "r"(v.x));
+  asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(acc) : "r"(v.y));
+  asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(acc) : "r"(v.z));
+  asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(acc) : "r"(v.w));
   return acc;
 }
 
-__device__ __forceinline__ uint32_t fold_halves(uint32_t m) { return max(m & 0xFFFFu, m >> 16); }
+// Larger of the two 16-bit magnitudes of a folded accumulator.
+__device__ __forceinline__ uint32_t fold_halves(uint32_t m) {
+  m &= 0x7FFF7FFFu;
+  return max(m & 0xFFFFu, m >> 16);
+}
 
 __device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
 
@@ -109,11 +162,15 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
 // amax_kernel (the per-tensor comparison path) instead of the row.
 // ----------------------------------------------------------------------------
 template <int V, bool PER_TENSOR>
-__global__ void __launch_bounds__(1024) quant_act_kernel(const uint4 *__restrict__ X, int T, int nvec,
-                                                         uint8_t *__restrict__ Xq, float *__restrict__ xs,
-                                                         int P, const uint32_t *__restrict__ tensor_amax) {
+__global__ void __launch_bounds__(V >= 16 ? 512 : 1024) quant_act_kernel(const uint4 *__restrict__ X, int T, int nvec,
+                                                         int64_t ldv, uint8_t *__restrict__ Xq,
+                                                         float *__restrict__ xs, int P,
+                                                         const uint32_t *__restrict__ tensor_amax) {
   __shared__ uint32_t red[32];
   griddep_launch_dependents();
+  // Launched as a programmatic dependent: X (and the buffers written below)
+  // may belong to the kernel launched just before, which must finish first.
+  griddep_wait();
 
   const int tid = threadIdx.x;
   const int rl = tid / P;
@@ -121,7 +178,7 @@ __global__ void __launch_bounds__(1024) quant_act_kernel(const uint4 *__restrict
   const int rows_per_cta = blockDim.x / P;
   const int64_t row = (int64_t)blockIdx.x * rows_per_cta + rl;
   const bool active = row < T;
-  const uint4 *xr = X + row * nvec;
+  const uint4 *xr = X + row * ldv;
 
   uint4 v[V];
   uint32_t m = 0;
@@ -156,10 +213,19 @@ __global__ void __launch_bounds__(1024) quant_act_kernel(const uint4 *__restrict
   if (lt == 0) xs[row] = g.s;
 
   uint2 *qr = reinterpret_cast<uint2 *>(Xq + row * (int64_t)nvec * 8);
-  #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const int j = lt + i * P;
-    if (j < nvec) qr[j] = quant_vec(v[i], g);
+  if (g.mode == kFast) {
+    const uint64_t s2 = pack2(g.s), nr2 = pack2(-g.r);
+    #pragma unroll
+    for (int i = 0; i < V; ++i) {
+      const int j = lt + i * P;
+      if (j < nvec) qr[j] = quant_vec_fast(v[i], s2, nr2);
+    }
+  } else {
+    #pragma unroll
+    for (int i = 0; i < V; ++i) {
+      const int j = lt + i * P;
+      if (j < nvec) qr[j] = quant_vec(v[i], g);
+    }
   }
 }
 
@@ -167,13 +233,15 @@ __global__ void __launch_bounds__(1024) quant_act_kernel(const uint4 *__restrict
 // normally served from L2).  One CTA per row.
 template <bool PER_TENSOR>
 __global__ void __launch_bounds__(1024) quant_act_long_kernel(const uint4 *__restrict__ X, int T, int nvec,
-                                                              uint8_t *__restrict__ Xq, float *__restrict__ xs,
+                                                              int64_t ldv, uint8_t *__restrict__ Xq,
+                                                              float *__restrict__ xs,
                                                               const uint32_t *__restrict__ tensor_amax) {
   __shared__ uint32_t red[32];
   __shared__ uint32_t row_amax;
   griddep_launch_dependents();
+  griddep_wait();
   const int64_t row = blockIdx.x;
-  const uint4 *xr = X + row * nvec;
+  const uint4 *xr = X + row * ldv;
   uint32_t amax_bits;
   if constexpr (PER_TENSOR) {
     amax_bits = *tensor_amax;
@@ -194,16 +262,20 @@ __global__ void __launch_bounds__(1024) quant_act_long_kernel(const uint4 *__res
   const GroupScale g = group_scale_from_amax_bits(amax_bits);
   if (threadIdx.x == 0) xs[row] = g.s;
   uint2 *qr = reinterpret_cast<uint2 *>(Xq + row * (int64_t)nvec * 8);
-  for (int j = threadIdx.x; j < nvec; j += blockDim.x) qr[j] = quant_vec(ld_stream(xr + j), g);
+  quant_run([&](int j) { return ld_stream(xr + j); }, qr, threadIdx.x, nvec, blockDim.x, g);
 }
 
-// Tensor-wide max |x| of n8 16-byte vectors, as bf16 magnitude bits, into
-// *amax (atomicMax; *amax must be 0 beforehand).
-__global__ void __launch_bounds__(512) amax_kernel(const uint4 *__restrict__ X, int64_t n8,
-                                                   uint32_t *__restrict__ amax) {
+// Tensor-wide max |x| of rows x nvec 16-byte vectors (row pitch ldv
+// vectors), as bf16 magnitude bits, into *amax (atomicMax; *amax must be 0
+// beforehand).
+__global__ void __launch_bounds__(512) amax_kernel(const uint4 *__restrict__ X, int64_t rows, int nvec,
+                                                   int64_t ldv, uint32_t *__restrict__ amax) {
   uint32_t m = 0;
-  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n8; j += (int64_t)gridDim.x * blockDim.x)
-    m = absmax_bits(m, ld_stream(X + j));
+  const int64_t n8 = rows * nvec;
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < n8; j += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = j / nvec;
+    m = absmax_bits(m, ld_stream(X + r * ldv + (j - r * nvec)));
+  }
   m = __reduce_max_sync(0xffffffffu, fold_halves(m));
   if ((threadIdx.x & 31) == 0 && m != 0) atomicMax(amax, m);
 }
@@ -261,70 +333,67 @@ __global__ void broadcast_amax_kernel(const uint32_t *__restrict__ src, uint32_t
 }
 
 // ----------------------------------------------------------------------------
-// Weight quantisation, pass 2: quantise a 64 (k) x 64 (o) tile of W with its
-// columns' scales and write it transposed into Wq_t (Co x Ci).  The tile is
-// staged in shared memory as codes [o][k] so both the bf16 reads (along o)
-// and the code writes (along k) are coalesced.
+// Weight quantisation, pass 2: quantise a 128 (k) x 64 (o) tile of W with its
+// columns' scales and write it transposed into Wq_t (Co x Ci).  Thread
+// (cv, kq) converts rows 4*kq .. 4*kq+3 of the 8 columns of vector cv, so for
+// each column it holds 4 consecutive K codes: one 32-bit word into the
+// shared tile [o][k], which is then written out as 16-byte row chunks.  Both
+// the bf16 reads (along Co) and the code writes (along Ci) are coalesced.
 // ----------------------------------------------------------------------------
-constexpr int kTT = 64;
+constexpr int kTK = 128;   // K rows per tile
+constexpr int kTO = 64;    // output channels per tile
+constexpr int kTPitch = kTK + 4;
 
 __global__ void __launch_bounds__(256) quant_weight_t_kernel(const uint4 *__restrict__ W, int Ci, int Co,
                                                              const uint32_t *__restrict__ col_amax,
                                                              uint8_t *__restrict__ Wq_t,
                                                              float *__restrict__ w_scale) {
-  __shared__ uint8_t tile[kTT][kTT + 4];
-  const int o0 = blockIdx.x * kTT;
-  const int k0 = blockIdx.y * kTT;
+  __shared__ __align__(16) uint8_t tile[kTO][kTPitch];
+  const int o0 = blockIdx.x * kTO;
+  const int k0 = blockIdx.y * kTK;
   const int ncv = Co / 8;
-  // each thread: one 8-column vector (8 per row of 64 columns), rows step 32
-  const int cvl = threadIdx.x & 7;     // vector within the tile row
-  const int kr = threadIdx.x >> 3;     // 0..31
-  const int ocol = o0 + cvl * 8;
-  GroupScale g[8];
+  const int cv = threadIdx.x & 7;      // 8-column vector within the tile
+  const int kq = threadIdx.x >> 3;     // rows 4*kq .. 4*kq+3
+  const int ocol = o0 + cv * 8;
+  uint4 v[4];
+  #pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int k = k0 + 4 * kq + r;
+    v[r] = (k < Ci && ocol < Co) ? ld_stream(W + (int64_t)k * ncv + (ocol >> 3)) : make_uint4(0u, 0u, 0u, 0u);
+  }
   #pragma unroll
   for (int c = 0; c < 8; ++c) {
     const int o = ocol + c;
-    g[c] = group_scale_from_amax_bits(o < Co ? col_amax[o] : 0u);
-  }
-  if (blockIdx.y == 0 && kr == 0) {
-    #pragma unroll
-    for (int c = 0; c < 8; ++c)
-      if (ocol + c < Co) w_scale[ocol + c] = g[c].s;
-  }
-  #pragma unroll
-  for (int rr = 0; rr < kTT; rr += 32) {
-    const int k = k0 + kr + rr;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (k < Ci && ocol < Co) v = ld_stream(W + (int64_t)k * ncv + (ocol >> 3));
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      GroupScale ga = g[2 * h], gb = g[2 * h + 1];
-      const float lo = __uint_as_float(w[h] << 16);
-      const float hi = __uint_as_float(w[h] & 0xFFFF0000u);
-      float2 q;
-      q.x = quotient(lo, ga);
-      q.y = quotient(hi, gb);
-      uint32_t codes = (uint32_t)__nv_cvt_float2_to_fp8x2(q, __NV_SATFINITE, __NV_E4M3);
-      if (ga.mode == kZeroGroup) codes &= 0xFF00u;
-      if (gb.mode == kZeroGroup) codes &= 0x00FFu;
-      tile[cvl * 8 + 2 * h][kr + rr] = (uint8_t)(codes & 0xFFu);
-      tile[cvl * 8 + 2 * h + 1][kr + rr] = (uint8_t)(codes >> 8);
+    const GroupScale g = group_scale_from_amax_bits(o < Co ? col_amax[o] : 0u);
+    if (blockIdx.y == 0 && kq == 0 && o < Co) w_scale[o] = g.s;
+    uint32_t word = 0;
+    if (g.mode != kZeroGroup) {
+      float q[4];
+      #pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const uint32_t w2 = (c < 2) ? v[r].x : (c < 4) ? v[r].y : (c < 6) ? v[r].z : v[r].w;
+        const float x = (c & 1) ? __uint_as_float(w2 & 0xFFFF0000u) : __uint_as_float(w2 << 16);
+        q[r] = quotient(x, g);
+      }
+      const uint32_t lo = (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(q[0], q[1]), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t hi = (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(q[2], q[3]), __NV_SATFINITE, __NV_E4M3);
+      word = lo | (hi << 16);
     }
+    *reinterpret_cast<uint32_t *>(&tile[cv * 8 + c][4 * kq]) = word;
   }
   __syncthreads();
-  // write: 64 rows (o) x 64 bytes (k): each thread writes 16 bytes
-  const int orow = threadIdx.x >> 2;        // 0..63
-  const int kc = (threadIdx.x & 3) * 16;    // 0,16,32,48
-  const int o = o0 + orow;
-  const int k = k0 + kc;
-  if (o < Co && k < Ci) {
-    uint32_t pk[4];
-    #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      pk[q] = (uint32_t)tile[orow][kc + 4 * q] | ((uint32_t)tile[orow][kc + 4 * q + 1] << 8) |
-              ((uint32_t)tile[orow][kc + 4 * q + 2] << 16) | ((uint32_t)tile[orow][kc + 4 * q + 3] << 24);
-    *reinterpret_cast<uint4 *>(Wq_t + (int64_t)o * Ci + k) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  // write: 64 rows (o) x 128 bytes (k), 16 bytes per thread, two passes
+  #pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int idx = threadIdx.x + pass * 256;
+    const int orow = idx >> 3;           // 0..63
+    const int kc = (idx & 7) * 16;       // 0..112
+    const int o = o0 + orow;
+    const int k = k0 + kc;
+    if (o < Co && k < Ci) {
+      const uint32_t *src = reinterpret_cast<const uint32_t *>(&tile[orow][kc]);
+      *reinterpret_cast<uint4 *>(Wq_t + (int64_t)o * Ci + k) = make_uint4(src[0], src[1], src[2], src[3]);
+    }
   }
 }
 
@@ -378,7 +447,7 @@ ActPlan plan_act(int nvec) {
   } else if (roundup32((nvec + 7) / 8) <= 1024) {
     p.V = 8;
     p.P = roundup32((nvec + 7) / 8);
-  } else if (roundup32((nvec + 15) / 16) <= 1024) {
+  } else if (roundup32((nvec + 15) / 16) <= 512) {  // 64 data registers a thread: at most 512 threads
     p.V = 16;
     p.P = roundup32((nvec + 15) / 16);
   } else {
@@ -388,26 +457,41 @@ ActPlan plan_act(int nvec) {
   return p;
 }
 
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous kernel in the stream finishes, and waits for it with
+// griddepcontrol.wait before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 template <bool PT>
-cudaError_t launch_act(const void *X, int T, int Ci, uint8_t *Xq, float *xs, const uint32_t *tensor_amax,
-                       cudaStream_t st) {
+cudaError_t launch_act(const void *X, int T, int Ci, int64_t ldx, uint8_t *Xq, float *xs,
+                       const uint32_t *tensor_amax, cudaStream_t st) {
   const int nvec = Ci / 8;
+  const int64_t ldv = ldx / 8;
   const ActPlan p = plan_act(nvec);
   const uint4 *Xv = static_cast<const uint4 *>(X);
-  if (p.V == 0) {
-    quant_act_long_kernel<PT><<<T, 1024, 0, st>>>(Xv, T, nvec, Xq, xs, tensor_amax);
-    return cudaGetLastError();
-  }
+  if (p.V == 0) return launch_pdl(quant_act_long_kernel<PT>, T, 1024, st, Xv, T, nvec, ldv, Xq, xs, tensor_amax);
   const int grid = (T + p.R - 1) / p.R;
   const int block = p.P * p.R;
   switch (p.V) {
-    case 1: quant_act_kernel<1, PT><<<grid, block, 0, st>>>(Xv, T, nvec, Xq, xs, p.P, tensor_amax); break;
-    case 2: quant_act_kernel<2, PT><<<grid, block, 0, st>>>(Xv, T, nvec, Xq, xs, p.P, tensor_amax); break;
-    case 4: quant_act_kernel<4, PT><<<grid, block, 0, st>>>(Xv, T, nvec, Xq, xs, p.P, tensor_amax); break;
-    case 8: quant_act_kernel<8, PT><<<grid, block, 0, st>>>(Xv, T, nvec, Xq, xs, p.P, tensor_amax); break;
-    default: quant_act_kernel<16, PT><<<grid, block, 0, st>>>(Xv, T, nvec, Xq, xs, p.P, tensor_amax); break;
+    case 1: return launch_pdl(quant_act_kernel<1, PT>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax);
+    case 2: return launch_pdl(quant_act_kernel<2, PT>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax);
+    case 4: return launch_pdl(quant_act_kernel<4, PT>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax);
+    case 8: return launch_pdl(quant_act_kernel<8, PT>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax);
+    default: return launch_pdl(quant_act_kernel<16, PT>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax);
   }
-  return cudaGetLastError();
 }
 
 int num_sms_cached() {
@@ -423,20 +507,20 @@ int num_sms_cached() {
 
 }  // namespace
 
-cudaError_t launch_quant_act(const void *X, int T, int Ci, uint8_t *Xq, float *xs, cudaStream_t st) {
-  return launch_act<false>(X, T, Ci, Xq, xs, nullptr, st);
+cudaError_t launch_quant_act(const void *X, int T, int Ci, int64_t ldx, uint8_t *Xq, float *xs, cudaStream_t st) {
+  return launch_act<false>(X, T, Ci, ldx, Xq, xs, nullptr, st);
 }
 
-cudaError_t launch_quant_act_per_tensor(const void *X, int T, int Ci, uint8_t *Xq, float *xs, uint32_t *amax_slot,
-                                        cudaStream_t st) {
+cudaError_t launch_quant_act_per_tensor(const void *X, int T, int Ci, int64_t ldx, uint8_t *Xq, float *xs,
+                                        uint32_t *amax_slot, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(amax_slot, 0, sizeof(uint32_t), st);
   if (e != cudaSuccess) return e;
   const int64_t n8 = (int64_t)T * Ci / 8;
   int grid = (int)std::min<int64_t>((n8 + 511) / 512, (int64_t)num_sms_cached() * 4);
   if (grid < 1) grid = 1;
-  amax_kernel<<<grid, 512, 0, st>>>(static_cast<const uint4 *>(X), n8, amax_slot);
+  amax_kernel<<<grid, 512, 0, st>>>(static_cast<const uint4 *>(X), T, Ci / 8, ldx / 8, amax_slot);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = launch_act<true>(X, T, Ci, Xq, xs, amax_slot, st)) != cudaSuccess) return e;
+  if ((e = launch_act<true>(X, T, Ci, ldx, Xq, xs, amax_slot, st)) != cudaSuccess) return e;
   // the workspace's scratch word is left zero for the next user
   return cudaMemsetAsync(amax_slot, 0, sizeof(uint32_t), st);
 }
@@ -450,7 +534,7 @@ cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, fl
     if ((e = cudaMemsetAsync(slot, 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
     const int64_t n8 = (int64_t)Ci * Co / 8;
     int grid = (int)std::min<int64_t>((n8 + 511) / 512, (int64_t)num_sms_cached() * 4);
-    amax_kernel<<<grid, 512, 0, st>>>(Wv, n8, slot);
+    amax_kernel<<<grid, 512, 0, st>>>(Wv, Ci, Co / 8, Co / 8, slot);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     broadcast_amax_kernel<<<(Co + 255) / 256, 256, 0, st>>>(slot, col_amax, Co);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -466,7 +550,7 @@ cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, fl
     col_amax_kernel<<<dim3(gx, slabs), kColThreads * kColWarps, 0, st>>>(Wv, Ci, Co, rows_per_cta, col_amax);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  dim3 grid((Co + kTT - 1) / kTT, (Ci + kTT - 1) / kTT);
+  dim3 grid((Co + kTO - 1) / kTO, (Ci + kTK - 1) / kTK);
   quant_weight_t_kernel<<<grid, 256, 0, st>>>(Wv, Ci, Co, col_amax, Wq_t, w_scale);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // the workspace's scratch words are left zero for the next user

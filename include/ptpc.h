@@ -26,7 +26,7 @@
  *   - Layouts are dense row-major.  bf16 tensors are passed as raw 16-bit
  *     patterns (void*).
  *   - Alignment: every device pointer must be 16-byte aligned
- *     (PTPC_ERR_MISALIGNED otherwise).
+ *     (PTPC_ERR_MISALIGNED otherwise); so must every row of X (ldx % 8 == 0).
  *   - Shapes: T >= 0 (T == 0 is a no-op returning PTPC_OK); Ci and Co must be
  *     positive multiples of 16 (PTPC_ERR_UNSUPPORTED_SHAPE otherwise), and
  *     T, Ci, Co must each fit in 31 bits.
@@ -85,12 +85,14 @@ typedef enum {
 } ptpc_op;
 
 /* Per-token activation quantisation (the page's Delta_X[T x 1]).
- *   X_dev       bf16 [T, Ci] row-major, read only.
+ *   X_dev       bf16 [T, Ci] row-major with row pitch ldx elements, read only
+ *               (ldx >= Ci, ldx % 8 == 0: e.g. a column slice of a wider
+ *               tensor; ldx == Ci for a dense tensor).
  *   Xq_dev      u8   [T, Ci] row-major, written: E4M3 codes of row t with
  *               scale x_scale[t] (the K-major A operand of the GEMM).
  *   x_scale_dev fp32 [T], written: amax(|X[t, :]|) / 448 (1.0f if amax == 0).
  * Codes and scales are bit-exact functions of X (see the conventions above). */
-PTPC_API int ptpc_quantize_activations(const void *X_dev, int64_t T, int64_t Ci,
+PTPC_API int ptpc_quantize_activations(const void *X_dev, int64_t T, int64_t Ci, int64_t ldx,
                               uint8_t *Xq_dev, float *x_scale_dev, void *stream);
 
 /* Per-output-channel weight quantisation (the page's Delta_W[1 x Co]); run
@@ -126,11 +128,12 @@ PTPC_API int ptpc_scaled_mm(const uint8_t *Xq_dev, const float *x_scale_dev,
  * then ptpc_scaled_mm, on one stream (the GEMM is launched as a programmatic
  * dependent of the quantiser).  The page's path with "no pre-quantization":
  * the bf16 activation goes in, the bf16 output comes out.
- *   X_dev bf16 [T, Ci]; Wq_t_dev / w_scale_dev as for ptpc_scaled_mm;
+ *   X_dev bf16 [T, Ci] with row pitch ldx (as for ptpc_quantize_activations);
+ *   Wq_t_dev / w_scale_dev as for ptpc_scaled_mm;
  *   out_dev bf16 [T, Co];
  *   ws_dev ptpc_workspace_size(PTPC_OP_LINEAR, T, Ci, Co) bytes (holds Xq and
  *   x_scale as well as the GEMM's workspace). */
-PTPC_API int ptpc_linear(const void *X_dev, const uint8_t *Wq_t_dev, const float *w_scale_dev,
+PTPC_API int ptpc_linear(const void *X_dev, int64_t ldx, const uint8_t *Wq_t_dev, const float *w_scale_dev,
                 int64_t T, int64_t Ci, int64_t Co, void *out_dev,
                 void *ws_dev, size_t ws_bytes, void *stream);
 
@@ -153,11 +156,12 @@ PTPC_API const char *ptpc_status_string(int status);
  * only hands over input and output buffers).  Same arguments, layouts and
  * results as ptpc_scaled_mm minus (ws_dev, ws_bytes).
  *   Scratch: a file-scope 8 MiB device array inside the library, held by
- *   every GPU that loads the library until the process exits.  Shapes whose
- *   ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co) exceeds 8 MiB are
- *   rejected with PTPC_ERR_WORKSPACE_TOO_SMALL (for example decode shapes with
- *   many split-K partial sums, such as T = 128, Ci = 28672, Co = 8192); prefill
- *   shapes need only a few KiB.
+ *   every GPU that loads the library until the process exits.  The GEMM's
+ *   stream-K partial sums are kept within it: a shape whose partial sums
+ *   would not fit runs on whole tiles instead (same results within the GEMM
+ *   tolerance, possibly slower than ptpc_scaled_mm).  A shape whose remaining
+ *   scratch (status word and tile counters) still exceeds the array is
+ *   rejected with PTPC_ERR_WORKSPACE_TOO_SMALL.
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress), so make that first call before any stream capture.
  *   Every call zeroes the array's control words with cudaMemsetAsync on
@@ -193,7 +197,7 @@ PTPC_API int ptpc_bench_apply_scales(const float *y_dev, const float *x_scale_de
  * and that one scale to every entry of x_scale_dev [T], so ptpc_scaled_mm can
  * consume the result unchanged.  ws_dev: ptpc_workspace_size(
  * PTPC_OP_BENCH_PER_TENSOR, T, Ci, 0) bytes. */
-PTPC_API int ptpc_bench_quantize_activations_per_tensor(const void *X_dev, int64_t T, int64_t Ci,
+PTPC_API int ptpc_bench_quantize_activations_per_tensor(const void *X_dev, int64_t T, int64_t Ci, int64_t ldx,
                                                uint8_t *Xq_dev, float *x_scale_dev,
                                                void *ws_dev, size_t ws_bytes, void *stream);
 

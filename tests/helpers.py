@@ -21,7 +21,7 @@ def assert_gemm_close(gpu_bits: np.ndarray, ref_bits: np.ndarray, what: str = ""
     rms = float(np.sqrt(np.mean(r * r))) if r.size else 0.0
     err = np.abs(g - r)
     bound = REL * np.abs(r) + ABS_RMS * rms
-    bad = err > bound
+    bad = ~(err <= bound)   # NaN or inf on either side counts as a mismatch
     if bad.any():
         i = np.argwhere(bad)[0]
         raise AssertionError(f"{what}: {int(bad.sum())} of {bad.size} outside tolerance; first at {tuple(i)}: "

@@ -69,11 +69,13 @@ def call(ptpc, name, *args):
 def test_argument_checks_without_gpu(ptpc):
     P = ctypes.c_void_p
     q = lambda *a: call(ptpc, "ptpc_quantize_activations", *a)
-    assert q(P(FAKE), 16, 100, P(FAKE), P(FAKE), None) == ptpc.ERR_UNSUPPORTED_SHAPE
-    assert q(P(FAKE), -1, 128, P(FAKE), P(FAKE), None) == ptpc.ERR_INVALID_ARG
-    assert q(None, 16, 128, P(FAKE), P(FAKE), None) == ptpc.ERR_INVALID_ARG
-    assert q(P(FAKE + 8), 16, 128, P(FAKE), P(FAKE), None) == ptpc.ERR_MISALIGNED
-    assert q(None, 0, 128, None, None, None) == ptpc.OK          # T == 0: no-op
+    assert q(P(FAKE), 16, 100, 100, P(FAKE), P(FAKE), None) == ptpc.ERR_UNSUPPORTED_SHAPE
+    assert q(P(FAKE), -1, 128, 128, P(FAKE), P(FAKE), None) == ptpc.ERR_INVALID_ARG
+    assert q(None, 16, 128, 128, P(FAKE), P(FAKE), None) == ptpc.ERR_INVALID_ARG
+    assert q(P(FAKE + 8), 16, 128, 128, P(FAKE), P(FAKE), None) == ptpc.ERR_MISALIGNED
+    assert q(P(FAKE), 16, 128, 100, P(FAKE), P(FAKE), None) == ptpc.ERR_INVALID_ARG   # ldx < Ci
+    assert q(P(FAKE), 16, 128, 132, P(FAKE), P(FAKE), None) == ptpc.ERR_MISALIGNED    # 16-byte rows
+    assert q(None, 0, 128, 128, None, None, None) == ptpc.OK     # T == 0: no-op
     mm = lambda *a: call(ptpc, "ptpc_scaled_mm", *a)
     need = ptpc.workspace_size(ptpc.OP_SCALED_MM, 16, 128, 64)
     assert mm(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 16, 128, 64, P(FAKE), P(FAKE), need - 1, None) == \
@@ -86,9 +88,10 @@ def test_argument_checks_without_gpu(ptpc):
         ptpc.ERR_INVALID_ARG
     lin = lambda *a: call(ptpc, "ptpc_linear", *a)
     need = ptpc.workspace_size(ptpc.OP_LINEAR, 16, 128, 64)
-    assert lin(P(FAKE), P(FAKE), P(FAKE), 16, 128, 64, P(FAKE), P(FAKE), need - 256, None) == \
+    assert lin(P(FAKE), 128, P(FAKE), P(FAKE), 16, 128, 64, P(FAKE), P(FAKE), need - 256, None) == \
         ptpc.ERR_WORKSPACE_TOO_SMALL
-    assert lin(None, None, None, 0, 128, 64, None, None, 0, None) == ptpc.OK
+    assert lin(P(FAKE), 64, P(FAKE), P(FAKE), 16, 128, 64, P(FAKE), P(FAKE), need, None) == ptpc.ERR_INVALID_ARG
+    assert lin(None, 128, None, None, 0, 128, 64, None, None, 0, None) == ptpc.OK
     qw = lambda *a: call(ptpc, "ptpc_quantize_weights", *a)
     need = ptpc.workspace_size(ptpc.OP_QUANTIZE_WEIGHTS, 0, 128, 64)
     assert qw(P(FAKE), 128, 64, P(FAKE), P(FAKE), P(FAKE), need - 1, None) == ptpc.ERR_WORKSPACE_TOO_SMALL

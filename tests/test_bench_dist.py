@@ -1,0 +1,64 @@
+"""Host-side logic of bench.py's multi-GPU path, run as world-size-2 gloo
+ranks on CPU: the slowest rank's time decides the step, whole-job
+throughput counts every rank's work, and under torchrun only rank 0 runs the
+reference arm."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    from datetime import timedelta
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        ms = [12.5, 20.0][rank]
+        mx = bench.dist_max(ms)
+        out[rank] = (mx, bench.whole_job_tflops(1e12, world, 10, mx))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_whole_job_throughput():
+    world = 2
+    port = _free_port()
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+    for r in range(world):
+        mx, tf = out[r]
+        assert mx == 20.0                       # the slowest rank
+        assert tf == pytest.approx(1e12 * 2 * 10 / 0.020 / 1e12)
+
+
+def test_single_process_helpers():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.dist_max(3.5) == 3.5
+    assert bench.whole_job_tflops(2e12, 1, 4, 8.0) == pytest.approx(1000.0)
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setattr(sys, "argv", ["bench.py", "--impl", "reference", "--gpus", "2"])
+    assert bench.main() == 0
+    assert capsys.readouterr().out == ""

@@ -188,3 +188,18 @@ def test_workspace_shared_across_entry_points(ptpc):
     rXq, rxs = oracle.quant_act(X)
     assert_gemm_close(out, oracle.scaled_mm_reference(rXq, rxs, rWq, rws), "shared workspace")
     assert ptpc.device_status(wsp) == ptpc.OK
+
+
+def test_linear_on_column_slice(ptpc):
+    """The fused entry reads a layer input that is a column slice of the
+    previous layer's output (row pitch > Ci) without a copy."""
+    T, Ci, Co, wide = 300, 1024, 768, 1536
+    Xw = synthetic.make_x(synthetic.LLAMA70B_PREFILL, 0, T, wide)
+    W = synthetic.make_w(synthetic.LLAMA70B_PREFILL, 0, Ci, Co)
+    Wq_t, ws = ptpc.quantize_weights(to_dev_bf16(W))
+    out = ptpc.linear(to_dev_bf16(Xw)[:, :Ci], Wq_t, ws)
+    X = np.ascontiguousarray(Xw[:, :Ci])
+    ref, _, _ = oracle.linear_reference(X, *oracle.quant_weight(W))
+    assert_gemm_close(from_dev_bf16(out), ref, "column slice")
+    dense = ptpc.linear(to_dev_bf16(X), Wq_t, ws)
+    assert torch.equal(dense.view(torch.int16), out.view(torch.int16))

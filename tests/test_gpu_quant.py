@@ -145,3 +145,18 @@ def test_codes_do_not_depend_on_stream_or_repeat(ptpc):
         b = ptpc.quantize_activations(Xd)
     s.synchronize()
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("T,Ci,extra", [(7, 4096, 64), (300, 8192, 2048), (1000, 256, 8), (2048, 28672, 28672)])
+def test_act_row_pitch(ptpc, T, Ci, extra):
+    """X given as a column slice of a wider tensor (row pitch ldx = Ci + extra)."""
+    full = synthetic.make_x(synthetic.LLAMA70B_PREFILL, 1, T, Ci + extra)
+    view = to_dev_bf16(full)[:, :Ci]
+    assert view.stride(0) == Ci + extra
+    gq, gs = ptpc.quantize_activations(view)
+    rq, rs = oracle.quant_act(np.ascontiguousarray(full[:, :Ci]))
+    assert np.array_equal(gs.cpu().numpy().view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(gq.cpu().numpy(), rq)
+    pq, ps = ptpc.quantize_activations_per_tensor(view)
+    oq, osc = oracle.quant_per_tensor(np.ascontiguousarray(full[:, :Ci]))
+    assert np.array_equal(pq.cpu().numpy(), oq) and (ps.cpu().numpy() == np.float32(osc)).all()
