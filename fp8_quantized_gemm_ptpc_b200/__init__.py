@@ -52,6 +52,7 @@ SIGNATURES = {
     "ptpc_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _I64, _I64, _I64]),
     "ptpc_get_device_status": (ctypes.c_int, [_P, _P]),
     "ptpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "ptpc_gemm_ksplit": (ctypes.c_int, [_I64, _I64, _I64]),
     "ptpc_scaled_mm_static_scratch": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "ptpc_bench_unscaled_mm_f32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "ptpc_bench_apply_scales": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _P, _P]),
@@ -91,6 +92,12 @@ def status_string(status: int) -> str:
 
 def workspace_size(op: int, T: int, Ci: int, Co: int) -> int:
     return int(lib.ptpc_workspace_size(op, T, Ci, Co))
+
+
+def gemm_ksplit(T: int, Ci: int, Co: int) -> int:
+    """CTAs sharing each output tile for this shape on the current device
+    (1: whole tiles; 2/4/8: K split over a cluster; 0: invalid)."""
+    return int(lib.ptpc_gemm_ksplit(T, Ci, Co))
 
 
 def _check(fn: str, status: int):

@@ -20,24 +20,8 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Workspace layout of the GEMM entry points:
 //   [0, 256)                 device status word (uint32 at offset 0)
-//   [256, 256 + C)           split-K tile counters (uint32, zero between calls)
-//   [.., .. + P)             split-K fp32 partial sums
-// ptpc_linear appends Xq [T, Ci] and x_scale [T] after the GEMM region.
-struct GemmLayout {
-  size_t counters_off, partials_off, end;
-  size_t partial_floats;
-};
-
-GemmLayout gemm_layout(int64_t T, int64_t Ci, int64_t Co, size_t max_partial_floats = SIZE_MAX) {
-  size_t cw = 0, pf = 0;
-  ptpc::gemm_workspace_needs((int)T, (int)Ci, (int)Co, max_partial_floats, &cw, &pf);
-  GemmLayout l;
-  l.counters_off = kAlign;
-  l.partials_off = l.counters_off + round_up(cw * 4);
-  l.end = l.partials_off + round_up(pf * 4);
-  l.partial_floats = pf;
-  return l;
-}
+// ptpc_linear appends Xq [T, Ci] and x_scale [T] after it.
+constexpr size_t kGemmWorkspace = kAlign;
 
 // Once per device: the kernels are built for compute capability 10.0 only.
 int check_device() {
@@ -79,9 +63,7 @@ int check_co(int64_t Co) {
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? PTPC_OK : PTPC_ERR_CUDA; }
 
 int run_gemm(const uint8_t *Xq, const float *xs, const uint8_t *Wq_t, const float *ws, int64_t T, int64_t Ci,
-             int64_t Co, void *out, bool f32_out, uint8_t *wsp, bool pdl, cudaStream_t st,
-             size_t max_partial_floats = SIZE_MAX) {
-  const GemmLayout l = gemm_layout(T, Ci, Co, max_partial_floats);
+             int64_t Co, void *out, bool f32_out, uint8_t *wsp, bool pdl, cudaStream_t st) {
   ptpc::GemmProblem p{};
   p.Xq = Xq;
   p.xs = xs;
@@ -93,9 +75,6 @@ int run_gemm(const uint8_t *Xq, const float *xs, const uint8_t *Wq_t, const floa
   p.out = out;
   p.f32_out = f32_out;
   p.status = reinterpret_cast<uint32_t *>(wsp);
-  p.counters = reinterpret_cast<uint32_t *>(wsp + l.counters_off);
-  p.partials = reinterpret_cast<float *>(wsp + l.partials_off);
-  p.partial_floats = l.partial_floats;
   p.pdl = pdl;
   return cuda_status(ptpc::launch_scaled_gemm(p, st));
 }
@@ -127,10 +106,10 @@ size_t ptpc_workspace_size(int op, int64_t T, int64_t Ci, int64_t Co) {
     case PTPC_OP_SCALED_MM:
     case PTPC_OP_BENCH_UNSCALED_MM:
       if (check_shape_tci(T, Ci) != PTPC_OK || check_co(Co) != PTPC_OK) return 0;
-      return gemm_layout(T, Ci, Co).end;
+      return kGemmWorkspace;
     case PTPC_OP_LINEAR:
       if (check_shape_tci(T, Ci) != PTPC_OK || check_co(Co) != PTPC_OK) return 0;
-      return gemm_layout(T, Ci, Co).end + round_up((size_t)T * (size_t)Ci) + round_up((size_t)T * 4);
+      return kGemmWorkspace + round_up((size_t)T * (size_t)Ci) + round_up((size_t)T * 4);
     case PTPC_OP_BENCH_PER_TENSOR:
       if (check_shape_tci(T, Ci) != PTPC_OK) return 0;
       return kAlign + kAlign;
@@ -194,12 +173,17 @@ int ptpc_linear(const void *X, int64_t ldx, const uint8_t *Wq_t, const float *w_
   if (ws_bytes < ptpc_workspace_size(PTPC_OP_LINEAR, T, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
   if ((s = check_device()) != PTPC_OK) return s;
   uint8_t *wsp = static_cast<uint8_t *>(ws);
-  const size_t g_end = gemm_layout(T, Ci, Co).end;
-  uint8_t *Xq = wsp + g_end;
-  float *xs = reinterpret_cast<float *>(wsp + g_end + round_up((size_t)T * (size_t)Ci));
+  uint8_t *Xq = wsp + kGemmWorkspace;
+  float *xs = reinterpret_cast<float *>(wsp + kGemmWorkspace + round_up((size_t)T * (size_t)Ci));
   cudaStream_t st = (cudaStream_t)stream;
   if ((s = cuda_status(ptpc::launch_quant_act(X, (int)T, (int)Ci, ldx, Xq, xs, st))) != PTPC_OK) return s;
   return run_gemm(Xq, xs, Wq_t, w_scale, T, Ci, Co, out, false, wsp, true, st);
+}
+
+int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co) {
+  if (check_shape_tci(T, Ci) != PTPC_OK || check_co(Co) != PTPC_OK || T == 0) return 0;
+  if (check_device() != PTPC_OK) return 0;
+  return ptpc::gemm_ksplit((int)T, (int)Ci, (int)Co);
 }
 
 int ptpc_get_device_status(void *ws, void *stream) {
@@ -278,13 +262,13 @@ int ptpc_bench_quantize_weights_per_tensor(const void *W, int64_t Ci, int64_t Co
 // inference engine that partitions all of its device memory once at start-up
 // and forbids allocation on the serving path, or a host integration that only
 // hands over input and output buffers.  This entry point needs no workspace
-// from them: its scratch (device status word, split-K tile counters and fp32
-// partial sums) lives in the file-scope array below, which every GPU that
-// loads this library holds until the process exits.
+// from them: its scratch (the GEMM's device status word) lives in the
+// file-scope array below, which every GPU that loads this library holds until
+// the process exits.
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr size_t kStaticScratchBytes = size_t(8) << 20;  // 8 MiB per device
+constexpr size_t kStaticScratchBytes = 4096;  // per device
 
 static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 
@@ -320,16 +304,12 @@ extern "C" int ptpc_scaled_mm_static_scratch(const uint8_t *Xq, const float *x_s
   if (!aligned16(Xq) || !aligned16(x_scale) || !aligned16(Wq_t) || !aligned16(w_scale) || !aligned16(out))
     return PTPC_ERR_MISALIGNED;
   if ((s = check_device()) != PTPC_OK) return s;
-  // Plan within the array: stream-K partial sums only when they fit in what
-  // is left after the status word and (at most 64 KiB of) tile counters.
-  const size_t budget_floats = (kStaticScratchBytes - kAlign - (size_t(64) << 10)) / sizeof(float);
-  const GemmLayout l = gemm_layout(T, Ci, Co, budget_floats);
-  if (l.end > kStaticScratchBytes) return PTPC_ERR_WORKSPACE_TOO_SMALL;
+  if (kGemmWorkspace > kStaticScratchBytes) return PTPC_ERR_WORKSPACE_TOO_SMALL;
   uint8_t *scratch = nullptr;
   if ((s = static_scratch_address(&scratch)) != PTPC_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  // The array keeps the previous call's contents: the status word and the
-  // stream-K tile counters must start at zero (the partial sums need not).
-  if (cudaMemsetAsync(scratch, 0, l.partials_off, st) != cudaSuccess) return PTPC_ERR_CUDA;
-  return run_gemm(Xq, x_scale, Wq_t, w_scale, T, Ci, Co, out, false, scratch, false, st, budget_floats);
+  // The array keeps the previous call's contents: the status word must start
+  // at zero.
+  if (cudaMemsetAsync(scratch, 0, kGemmWorkspace, st) != cudaSuccess) return PTPC_ERR_CUDA;
+  return run_gemm(Xq, x_scale, Wq_t, w_scale, T, Ci, Co, out, false, scratch, false, st);
 }

@@ -22,17 +22,15 @@
 // warp owns one 32-lane quarter), apply the two scales, round to bf16 and
 // store, while the MMA warp fills the other accumulator.
 //
-// Work schedule: the prefill kernel takes whole tiles round-robin over the
-// CTA pairs.  The decode kernel has few tiles (Co / 128) and each is a long
-// stream of weight bytes, so when there are fewer tiles than SMs it shares
-// them "stream-K" style: each CTA takes an equal contiguous range of all
-// tiles' K-blocks, so every SM streams the same number of weight bytes and a
-// tile may be computed in several K segments.  A segment that is not the
-// whole tile writes its fp32 partial sum to the workspace and bumps the
-// tile's arrival counter; the CTA that arrives last (no CTA ever waits for
-// another) adds the partials in segment order — a fixed order, so the result
-// does not depend on which CTA finishes last — applies the scales, stores,
-// and resets the counter for the next call.
+// Work schedule: whole tiles, round-robin over the CTAs (CTA pairs), except
+// that a decode problem with fewer than half as many tiles as SMs splits K:
+// the S CTAs of a thread-block cluster (S = 2, 4 or 8) share one tile, each
+// streaming 1/S of its K-blocks, so S times as many SMs stream weights.  Each
+// CTA leaves its fp32 partial sums in its own shared memory; after a cluster
+// barrier every CTA finishes 128/S of the tile's channels by reading the S
+// partial sums over distributed shared memory and adding them in rank order
+// (a fixed order: the result does not depend on timing), then applies the
+// scales and stores.  No partial sum goes through global memory.
 //
 // Every wait on an mbarrier is bounded (see mbar_wait); a wait that runs out
 // sets a bit in the device status word, and the CTA stops issuing work, lets
@@ -61,11 +59,7 @@ struct GemmParams {
   int num_m, num_n, num_kb;   // tile grid (rows of tiles are 128 or 256 tokens)
   int group_m;                // tile rows visited together (L2 reuse of weights)
   int num_tiles;
-  int dp_tiles;               // tiles [0, dp_tiles): whole, round-robin
-  int sk_ctas;                // CTAs (pairs) sharing tiles [dp_tiles, num_tiles)
-  int seg_slots;              // partial-sum slots per shared tile
-  long long sk_iters;         // (num_tiles - dp_tiles) * num_kb
-  int part_rows;              // rows of one partial-sum slot
+  int ksplit;                 // decode kernel: CTAs (one cluster) per tile, 1 = whole tiles
   int np;                     // decode kernel: tokens padded to the MMA's N (multiple of 16)
   int stages;                 // decode kernel: shared-memory ring depth
   int tmem_cols;              // decode kernel: tensor-memory columns allocated (two accumulators)
@@ -73,60 +67,41 @@ struct GemmParams {
   const float *ws;
   void *out;
   uint32_t *status;
-  uint32_t *counters;
-  float *partials;
 };
 
-// One piece of work: K-blocks [kb0, kb1) of tile `tile`, segment `seg` of
-// `nseg` (nseg == 1: the whole tile).
+// One piece of work: K-blocks [kb0, kb1) of tile `tile` (row m, column n).
 struct Unit {
-  int tile, m, n, kb0, kb1, seg, nseg;
+  int tile, m, n, kb0, kb1;
 };
-
-__device__ __forceinline__ int sk_owner(const GemmParams &p, long long x) {
-  return (int)(((x + 1) * (long long)p.sk_ctas - 1) / p.sk_iters);
-}
 
 // The same sequence of units for the producer, the MMA issuer and the
-// epilogue of one CTA (pair) `id` out of `count`.
+// epilogue of one CTA (pair) `id` out of `count`: tiles id, id + count, ...
+// whole, or, when the decode kernel splits K (ksplit > 1), the one tile of
+// this CTA's cluster and this CTA's share of its K-blocks.
 struct Sched {
-  int id, dp_next, dp_step;
-  long long pos, end;
+  int next_tile, step, kb0, kb1;
 
-  __device__ __forceinline__ void init(const GemmParams &p, int id_, int count) {
-    id = id_;
-    dp_next = id_;
-    dp_step = count;
-    if (id_ < p.sk_ctas) {
-      pos = (long long)id_ * p.sk_iters / p.sk_ctas;
-      end = (long long)(id_ + 1) * p.sk_iters / p.sk_ctas;
+  __device__ __forceinline__ void init(const GemmParams &p, int id, int count) {
+    if (p.ksplit > 1) {
+      const int r = id % p.ksplit;  // == %cluster_ctarank for a 1-D cluster
+      next_tile = id / p.ksplit;
+      step = p.num_tiles;  // one tile per cluster
+      kb0 = r * p.num_kb / p.ksplit;
+      kb1 = (r + 1) * p.num_kb / p.ksplit;
     } else {
-      pos = end = 0;
+      next_tile = id;
+      step = count;
+      kb0 = 0;
+      kb1 = p.num_kb;
     }
   }
 
   __device__ __forceinline__ bool next(const GemmParams &p, Unit &u) {
-    if (dp_next < p.dp_tiles) {
-      u.tile = dp_next;
-      dp_next += dp_step;
-      u.kb0 = 0;
-      u.kb1 = p.num_kb;
-      u.seg = 0;
-      u.nseg = 1;
-    } else if (pos < end) {
-      const long long t = pos / p.num_kb;
-      const long long t_begin = t * p.num_kb, t_end = t_begin + p.num_kb;
-      const long long s_end = end < t_end ? end : t_end;
-      u.tile = p.dp_tiles + (int)t;
-      u.kb0 = (int)(pos - t_begin);
-      u.kb1 = (int)(s_end - t_begin);
-      const int first = sk_owner(p, t_begin);
-      u.seg = id - first;
-      u.nseg = sk_owner(p, t_end - 1) - first + 1;
-      pos = s_end;
-    } else {
-      return false;
-    }
+    if (next_tile >= p.num_tiles) return false;
+    u.tile = next_tile;
+    next_tile += step;
+    u.kb0 = kb0;
+    u.kb1 = kb1;
     // grouped raster: group_m tile rows, all tile columns, rows fastest
     const int per_group = p.group_m * p.num_n;
     const int g = u.tile / per_group;
@@ -138,8 +113,6 @@ struct Sched {
     return true;
   }
 };
-
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -227,72 +200,6 @@ __device__ __forceinline__ void epilogue_store_tile(const CUtensorMap *tmC, uint
   }
 }
 
-// Last arriver of a shared decode tile: adds the nseg partial slots
-// ([token][channel], BM floats per token) in slot order, applies the scales
-// (or keeps fp32) and stores each token's 128 channels.  The four epilogue
-// warps split the tokens (warp ew takes tokens ew, ew + 4, ...), each lane
-// owns 4 consecutive channels (one 16-byte load per slot and token), and the
-// loads of RB tokens x SB slots are issued together (16 loads in flight per
-// lane), so a tile of 128 tokens in three slots costs about eight L2 round
-// trips per warp instead of one per token and slot.
-template <bool F32OUT>
-__device__ __forceinline__ void decode_reduce_tile(const GemmParams &p, const float *slot0, size_t slot_stride,
-                                                   int nseg, int col_base, int ew, int lane) {
-  constexpr int RB = 8;  // tokens per batch
-  constexpr int SB = 2;  // slots loaded together
-  const int c = lane * 4;
-  const bool col_ok = col_base + c < p.Co;  // Co % 16 == 0: the lane's 4 columns are valid together
-  float4 wv = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (!F32OUT && col_ok) wv = __ldg(reinterpret_cast<const float4 *>(p.ws + col_base + c));
-  for (int r0 = ew; r0 < p.T; r0 += kEpiWarps * RB) {
-    float4 acc[RB];
-    for (int sg0 = 0; sg0 < nseg; sg0 += SB) {
-      float4 v[SB][RB];
-      #pragma unroll
-      for (int k = 0; k < SB; ++k) {
-        #pragma unroll
-        for (int i = 0; i < RB; ++i) {
-          const int row = r0 + i * kEpiWarps;
-          v[k][i] = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (sg0 + k < nseg && row < p.T)
-            v[k][i] = __ldcg(reinterpret_cast<const float4 *>(slot0 + (size_t)(sg0 + k) * slot_stride +
-                                                              (size_t)row * BM + c));
-        }
-      }
-      #pragma unroll
-      for (int k = 0; k < SB; ++k) {
-        if (sg0 + k >= nseg) break;
-        #pragma unroll
-        for (int i = 0; i < RB; ++i) {
-          if (sg0 + k == 0) {
-            acc[i] = v[k][i];
-          } else {
-            acc[i].x = __fadd_rn(acc[i].x, v[k][i].x);
-            acc[i].y = __fadd_rn(acc[i].y, v[k][i].y);
-            acc[i].z = __fadd_rn(acc[i].z, v[k][i].z);
-            acc[i].w = __fadd_rn(acc[i].w, v[k][i].w);
-          }
-        }
-      }
-    }
-    if (!col_ok) continue;
-    #pragma unroll
-    for (int i = 0; i < RB; ++i) {
-      const int row = r0 + i * kEpiWarps;
-      if (row >= p.T) continue;
-      if constexpr (F32OUT) {
-        *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (size_t)row * p.Co + col_base + c) = acc[i];
-      } else {
-        const float a = __ldg(p.xs + row);
-        const uint32_t lo = pack_bf16x2(__fmul_rn(__fmul_rn(acc[i].x, a), wv.x), __fmul_rn(__fmul_rn(acc[i].y, a), wv.y));
-        const uint32_t hi = pack_bf16x2(__fmul_rn(__fmul_rn(acc[i].z, a), wv.z), __fmul_rn(__fmul_rn(acc[i].w, a), wv.w));
-        *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) + (size_t)row * p.Co + col_base + c) =
-            make_uint2(lo, hi);
-      }
-    }
-  }
-}
-
 // ----------------------------------------------------------------------------
 // Decode kernel (T <= 128), operands swapped: acc^T = Wq_t . Xq^T.
 // The 128 weight rows of a channel tile are the MMA's M = 128 operand and the
@@ -302,7 +209,9 @@ __device__ __forceinline__ void decode_reduce_tile(const GemmParams &p, const fl
 // as deep as shared memory allows (12 stages at NP = 16).  Tensor-memory lane
 // = output channel, column = token: each epilogue thread owns one channel, so
 // w_scale is one register and every token's 32 channels of a warp are one
-// contiguous store.  Work is shared stream-K style as in the one-CTA kernel.
+// contiguous store.  With ksplit = S > 1 the grid is made of S-CTA clusters,
+// one tile each, and the epilogue leaves the partial sums in shared memory
+// for the cluster reduction instead of storing.
 // ----------------------------------------------------------------------------
 constexpr int kDecMaxStages = 16;
 constexpr int kDecWBytes = BM * BK;   // weight tile of one stage
@@ -346,41 +255,80 @@ __device__ __forceinline__ void decode_store_tile(const GemmParams &p, uint32_t 
   }
 }
 
-// Shared tile: this segment's partial sums go to its slot ([token][channel],
-// BM floats per token row, so a warp writes 128 contiguous bytes per token);
-// the last of the tile's segments to arrive adds all slots in slot order.
-template <bool F32OUT>
-__device__ __noinline__ void decode_segment(const GemmParams &p, const Unit &u, uint32_t tbase, float *slot0,
-                                            size_t slot_stride, uint32_t *counter, int q, int lane, int et,
-                                            int *last_flag, uint32_t release_bar) {
-  float *slot = slot0 + (size_t)u.seg * slot_stride + q * 32 + lane;
+// K split over a cluster, step 1: this CTA's partial sums of the tile, from
+// tensor memory to red[t][c] (fp32, BM floats per token) in its own shared
+// memory.  Each warp writes 32 consecutive floats per token (no bank
+// conflicts).
+__device__ __forceinline__ void decode_dump_tile(const GemmParams &p, uint32_t tbase, float *red, int q, int lane) {
+  float *dst = red + q * 32 + lane;
   #pragma unroll 1
   for (int c0 = 0; c0 < p.np; c0 += 16) {
     uint32_t r[16];
     tmem_ld_32x32b_x16(tbase + c0, r);
     tmem_wait_ld();
     #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int t = c0 + j;
-      if (t < p.T) __stcg(slot + (size_t)t * BM, __uint_as_float(r[j]));
+    for (int j = 0; j < 16; ++j) dst[(c0 + j) * BM] = __uint_as_float(r[j]);
+  }
+}
+
+// K split over a cluster, step 2 (after a cluster barrier): this CTA (rank)
+// finishes channels [rank * 128/S, (rank + 1) * 128/S) of the tile for every
+// token.  Each thread takes 4 consecutive channels of one token, loads them
+// from all S CTAs' red arrays over distributed shared memory (16 bytes per
+// load; U groups, U * S loads in flight), adds the S partial sums in rank
+// order, applies the scales and stores.
+template <int S, bool F32OUT>
+__device__ __forceinline__ void decode_cluster_reduce(const GemmParams &p, const float *red, int tile,
+                                                      uint32_t rank) {
+  constexpr int CS = BM / S;                // channels this CTA finishes
+  constexpr int G = CS / 4;                 // 4-channel groups per token
+  constexpr int U = S >= 8 ? 1 : 8 / S;     // groups per thread in flight
+  uint32_t base[S];
+  #pragma unroll
+  for (int s = 0; s < S; ++s) base[s] = mapa_shared(red, (uint32_t)s);
+  const int total = p.T * G;
+  const int c_first = (int)rank * CS;
+  for (int i0 = threadIdx.x; i0 < total; i0 += U * kThreads) {
+    float4 v[U][S];
+    #pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int idx = i0 + u * kThreads;
+      if (idx < total) {
+        const int t = idx / G;
+        const int c = c_first + (idx - t * G) * 4;
+        const uint32_t off = (uint32_t)(t * BM + c) * 4u;
+        #pragma unroll
+        for (int s = 0; s < S; ++s) v[u][s] = ld_shared_cluster_f32x4(base[s] + off);
+      }
+    }
+    #pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int idx = i0 + u * kThreads;
+      if (idx >= total) continue;
+      const int t = idx / G;
+      const int c = c_first + (idx - t * G) * 4;
+      const int ch = tile * BM + c;
+      if (ch >= p.Co) continue;  // Co % 16 == 0: the 4 channels are valid together
+      float4 acc = v[u][0];
+      #pragma unroll
+      for (int s = 1; s < S; ++s) {
+        acc.x = __fadd_rn(acc.x, v[u][s].x);
+        acc.y = __fadd_rn(acc.y, v[u][s].y);
+        acc.z = __fadd_rn(acc.z, v[u][s].z);
+        acc.w = __fadd_rn(acc.w, v[u][s].w);
+      }
+      if constexpr (F32OUT) {
+        *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + (size_t)t * p.Co + ch) = acc;
+      } else {
+        const float a = __ldg(p.xs + t);
+        const float4 w = __ldg(reinterpret_cast<const float4 *>(p.ws + ch));
+        const uint32_t lo = pack_bf16x2(__fmul_rn(__fmul_rn(acc.x, a), w.x), __fmul_rn(__fmul_rn(acc.y, a), w.y));
+        const uint32_t hi = pack_bf16x2(__fmul_rn(__fmul_rn(acc.z, a), w.z), __fmul_rn(__fmul_rn(acc.w, a), w.w));
+        *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) + (size_t)t * p.Co + ch) =
+            make_uint2(lo, hi);
+      }
     }
   }
-  tc_fence_before();
-  __syncwarp();
-  if (lane == 0) mbar_arrive_cluster(release_bar);
-  __threadfence();
-  epi_bar();
-  if (et == 0) {
-    const uint32_t prev = atomicAdd(counter, 1u);
-    *last_flag = (prev == (uint32_t)(u.nseg - 1)) ? 1 : 0;
-  }
-  epi_bar();
-  if (*last_flag) {
-    __threadfence();
-    decode_reduce_tile<F32OUT>(p, slot0, slot_stride, u.nseg, u.n * BM, et >> 5, lane);
-    if (et == 0) *counter = 0u;  // ready for the next call
-  }
-  epi_bar();
 }
 
 template <bool F32OUT>
@@ -399,9 +347,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t *tempty = tfull + 2;
   uint64_t *drain = tempty + 2;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
-  int *last_flag = reinterpret_cast<int *>(tmem_holder + 1);
-  int *vote = last_flag + 1;  // [kEpiWarps]
   const uint32_t acc_cols = (uint32_t)p.tmem_cols / 2;  // column stride of the two accumulators
+  // K split: partial sums of the tile, [NP tokens][BM channels] fp32, in the
+  // weight ring (idle once the accumulator is complete; NP * 512 <= 64 KB,
+  // the ring holds at least 7 x 16 KB)
+  float *red = reinterpret_cast<float *>(sW);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -524,9 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;           // tensor-memory lane quarter = channels q*32 .. q*32+31
-    const int ew = warp - 2;
-    const int et = threadIdx.x - 64;  // 0..127 within the epilogue warps
+    const int q = warp & 3;  // tensor-memory lane quarter = channels q*32 .. q*32+31
     int local = 0;
     bool ok = true;
     griddep_wait();  // x_scale may come from the kernel launched just before
@@ -539,30 +487,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++local;
       const int ch = u.n * BM + q * 32 + lane;
       const float wsr = (!F32OUT && ch < p.Co) ? __ldg(p.ws + ch) : 0.0f;
-      bool got = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], aphase));
-      if (p.sk_ctas > 0) {
-        if (lane == 0) vote[ew] = got ? 1 : 0;
-        epi_bar();
-        got = vote[0] && vote[1] && vote[2] && vote[3];
-        epi_bar();
-      }
-      if (!got) {
+      // tcgen05.ld is warp-collective: the whole warp stops or none of it
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], aphase))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)buf * acc_cols;
-      if (u.nseg == 1) {
+      if (p.ksplit == 1)
         decode_store_tile<F32OUT>(p, tbase, ch, wsr, lane, smem_u32(&tempty[buf]));
-      } else {
-        const int sk_tile = u.tile - p.dp_tiles;
-        const size_t slot_stride = (size_t)p.part_rows * BM;
-        float *slot0 = p.partials + (size_t)sk_tile * p.seg_slots * slot_stride;
-        decode_segment<F32OUT>(p, u, tbase, slot0, slot_stride, p.counters + sk_tile, q, lane, et, last_flag,
-                               smem_u32(&tempty[buf]));
-      }
+      else
+        decode_dump_tile(p, tbase, red, q, lane);
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeoutEpilogue);
+  }
+
+  if (p.ksplit > 1) {
+    // Every CTA of the cluster reaches both barriers on every path (a timed
+    // out wait above only skips work), so neither can wait forever.
+    __syncwarp();    // warps 0 and 1 arrive from a one-lane branch
+    cluster_sync();  // all partial sums of the tile are in shared memory
+    const int tile = blockIdx.x / p.ksplit;
+    const uint32_t rank = cluster_ctarank();
+    if (p.ksplit == 2)
+      decode_cluster_reduce<2, F32OUT>(p, red, tile, rank);
+    else if (p.ksplit == 4)
+      decode_cluster_reduce<4, F32OUT>(p, red, tile, rank);
+    else
+      decode_cluster_reduce<8, F32OUT>(p, red, tile, rank);
+    cluster_sync();  // no CTA reads another's shared memory any more
   }
 
   tc_fence_before();
@@ -838,7 +791,31 @@ struct DeviceInfo {
   bool ready = false;
   int sms = 148;
   int pair_clusters = 74;
+  int dec_clusters[9] = {};  // resident decode clusters of 2, 4 and 8 CTAs
 };
+
+// Most clusters of `size` CTAs of `kernel` (with `smem` bytes each) that can
+// be resident at once; 0 if unknown.
+template <typename Kernel>
+int max_clusters(Kernel kernel, int sms, int size, size_t smem) {
+  cudaLaunchConfig_t q = {};
+  q.gridDim = dim3(size * (sms / size));
+  q.blockDim = dim3(kThreads);
+  q.dynamicSmemBytes = smem;
+  cudaLaunchAttribute a[1];
+  a[0].id = cudaLaunchAttributeClusterDimension;
+  a[0].val.clusterDim.x = size;
+  a[0].val.clusterDim.y = 1;
+  a[0].val.clusterDim.z = 1;
+  q.attrs = a;
+  q.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &q) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
 
 DeviceInfo &device_info() {
   static DeviceInfo info[64];
@@ -860,6 +837,7 @@ DeviceInfo &device_info() {
                          (int)PairCfg<kPairStages, false>::SMEM);
     cudaFuncSetAttribute(ptpc_gemm_pair_kernel<kPairStages, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)PairCfg<kPairStages, true>::SMEM);
+    // the pair kernel's cluster size is compiled in (__cluster_dims__)
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3(2 * (d.sms / 2));
     q.blockDim = dim3(kThreads);
@@ -871,30 +849,38 @@ DeviceInfo &device_info() {
     else
       d.pair_clusters = d.sms / 2;
     cudaGetLastError();
+    // the decode kernel takes its cluster size at launch; ask for the largest
+    // shared-memory footprint it launches with
+    for (int size = 2; size <= 8; size *= 2) {
+      const int a = max_clusters(ptpc_gemm_decode_kernel<false>, d.sms, size, kDecSmemMax);
+      const int b = max_clusters(ptpc_gemm_decode_kernel<true>, d.sms, size, kDecSmemMax);
+      d.dec_clusters[size] = std::min(a, b);
+    }
     d.ready = true;
   }
   return d;
 }
 
-// The launch plan of one problem; the workspace query and the launch both
-// derive from it, so they always agree.
+// The launch plan of one problem.
 struct Plan {
   bool pair;
   int tile_rows, bn;
   int num_m, num_n, num_kb, num_tiles;
   int group_m;
-  int ctas;            // CTAs (one-CTA kernel) or CTA pairs (pair kernel) launched
-  int dp_tiles, sk_ctas, seg_slots, part_rows;
-  long long sk_iters;
+  int ctas;     // CTAs (decode kernel) or CTA pairs (pair kernel) launched
+  int ksplit;   // decode kernel: CTAs per tile (cluster size), 1 = whole tiles
   int np, stages, tmem_cols;  // decode kernel only
-  size_t counter_words, partial_floats;
 };
 
-Plan make_plan(int T, int Ci, int Co, size_t max_partial_floats) {
+// Fewest K-blocks a CTA of a K-split cluster streams.
+constexpr int kMinSplitKb = 4;
+
+Plan make_plan(int T, int Ci, int Co) {
   const DeviceInfo &d = device_info();
   Plan pl = {};
   pl.num_kb = (Ci + BK - 1) / BK;
   pl.pair = T > BM;
+  pl.ksplit = 1;
   if (pl.pair) {
     pl.tile_rows = 2 * BM;
     pl.bn = kPairBN;
@@ -913,64 +899,44 @@ Plan make_plan(int T, int Ci, int Co, size_t max_partial_floats) {
   pl.num_m = (T + pl.tile_rows - 1) / pl.tile_rows;
   pl.num_n = (Co + pl.bn - 1) / pl.bn;
   pl.num_tiles = pl.num_m * pl.num_n;
-  const int slots = pl.pair ? d.pair_clusters : d.sms;
-  pl.dp_tiles = pl.num_tiles;
-  pl.sk_ctas = 0;
-  pl.seg_slots = 1;
-  pl.sk_iters = 0;
   if (pl.pair) {
-    // Whole tiles only.  Sharing the last partial wave stream-K style was
-    // measured slower on B200 for 256 x 256 tiles (e.g. 2048 x 4096 -> 6144:
-    // 73.8 us shared vs 43.1 us whole; 2048 x 14336 -> 4096: 136.8 vs 109.7):
-    // the fixup of 256 KB fp32 partials costs more than the idle pairs.
-    pl.part_rows = BM;
-  } else {
-    // decode: every SM streams the same number of weight K-blocks; segments
-    // long enough that partial sums stay small next to the weights they cover
-    const long long iters = (long long)pl.num_tiles * pl.num_kb;
-    const int min_seg = std::max(4, (T + 3) / 4);
-    const int sk = (int)std::min<long long>(slots, iters / min_seg);
-    if (sk > pl.num_tiles) {
-      pl.dp_tiles = 0;
-      pl.sk_ctas = sk;
-      pl.sk_iters = iters;
-    }
-    pl.part_rows = T;
+    // Whole tiles only.  Sharing the last partial wave stream-K style (fp32
+    // partial sums through global memory, fixed-order fixup) was measured
+    // slower on B200 for 256 x 256 tiles (e.g. 2048 x 4096 -> 6144: 73.8 us
+    // shared vs 43.1 us whole; 2048 x 14336 -> 4096: 136.8 vs 109.7).
+    pl.ctas = std::max(1, std::min(pl.num_tiles, d.pair_clusters));
+    return pl;
   }
-  if (pl.sk_ctas > 0) {
-    const long long per = pl.sk_iters / pl.sk_ctas;  // >= min_seg >= 4
-    pl.seg_slots = (int)((pl.num_kb + per - 1) / per) + 1;
-    const size_t sk_tiles = (size_t)(pl.num_tiles - pl.dp_tiles);
-    pl.counter_words = sk_tiles;
-    pl.partial_floats = sk_tiles * pl.seg_slots * (size_t)pl.part_rows * pl.bn;
-    if (pl.partial_floats > max_partial_floats) {
-      // no room for the partial sums: whole tiles only
-      pl.dp_tiles = pl.num_tiles;
-      pl.sk_ctas = 0;
-      pl.seg_slots = 1;
-      pl.sk_iters = 0;
-      pl.counter_words = 0;
-      pl.partial_floats = 0;
+  // Decode: split K over a cluster when that puts at least twice as many SMs
+  // on the weight stream, all tiles in one wave.
+  for (int size = 8; size >= 2; size /= 2) {
+    if ((long long)pl.num_tiles * size <= d.sms && pl.num_tiles <= d.dec_clusters[size] &&
+        pl.num_kb >= size * kMinSplitKb) {
+      pl.ksplit = size;
+      break;
     }
   }
-  pl.ctas = std::max(1, std::min(pl.num_tiles, slots));
-  if (pl.sk_ctas > 0) pl.ctas = std::max(pl.ctas, std::min(slots, pl.sk_ctas));
+  pl.ctas = pl.ksplit > 1 ? pl.num_tiles * pl.ksplit : std::max(1, std::min(pl.num_tiles, d.sms));
   return pl;
 }
 
 template <typename Kernel>
-cudaError_t launch_decode(Kernel kernel, int grid, size_t smem, const CUtensorMap &tmW, const CUtensorMap &tmX,
-                          const GemmParams &gp, bool pdl, cudaStream_t st) {
+cudaError_t launch_decode(Kernel kernel, int grid, int cluster, size_t smem, const CUtensorMap &tmW,
+                          const CUtensorMap &tmX, const GemmParams &gp, bool pdl, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, tmW, tmX, gp);
 }
 
@@ -994,15 +960,10 @@ cudaError_t launch(Kernel kernel, int grid, size_t smem, const CUtensorMap &tmA,
 
 int num_sms() { return device_info().sms; }
 
-void gemm_workspace_needs(int T, int Ci, int Co, size_t max_partial_floats, size_t *counter_words,
-                          size_t *partial_floats) {
-  const Plan pl = make_plan(T, Ci, Co, max_partial_floats);
-  *counter_words = pl.counter_words;
-  *partial_floats = pl.partial_floats;
-}
+int gemm_ksplit(int T, int Ci, int Co) { return make_plan(T, Ci, Co).ksplit; }
 
 cudaError_t launch_scaled_gemm(const GemmProblem &pr, cudaStream_t st) {
-  const Plan pl = make_plan(pr.T, pr.Ci, pr.Co, pr.partial_floats);
+  const Plan pl = make_plan(pr.T, pr.Ci, pr.Co);
   GemmParams gp = {};
   gp.T = pr.T;
   gp.Co = pr.Co;
@@ -1011,20 +972,14 @@ cudaError_t launch_scaled_gemm(const GemmProblem &pr, cudaStream_t st) {
   gp.num_kb = pl.num_kb;
   gp.group_m = pl.group_m;
   gp.num_tiles = pl.num_tiles;
-  gp.dp_tiles = pl.dp_tiles;
-  gp.sk_ctas = pl.sk_ctas;
-  gp.seg_slots = pl.seg_slots;
-  gp.sk_iters = pl.sk_iters;
-  gp.part_rows = pl.part_rows;
+  gp.ksplit = pl.ksplit;
+  gp.np = pl.np;
+  gp.stages = pl.stages;
+  gp.tmem_cols = pl.tmem_cols;
   gp.xs = pr.xs;
   gp.ws = pr.ws;
   gp.out = pr.out;
   gp.status = pr.status;
-  gp.counters = pr.counters;
-  gp.partials = pr.partials;
-  gp.np = pl.np;
-  gp.stages = pl.stages;
-  gp.tmem_cols = pl.tmem_cols;
   if (!pl.pair) {
     CUtensorMap tmW, tmX;
     if (!make_map_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Wq_t, pr.Ci, pr.Co, pr.Ci, BK, BM,
@@ -1033,8 +988,10 @@ cudaError_t launch_scaled_gemm(const GemmProblem &pr, cudaStream_t st) {
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
     const size_t smem = dec_smem_bytes(pl.np, pl.stages);
-    return pr.f32_out ? launch_decode(ptpc_gemm_decode_kernel<true>, pl.ctas, smem, tmW, tmX, gp, pr.pdl, st)
-                      : launch_decode(ptpc_gemm_decode_kernel<false>, pl.ctas, smem, tmW, tmX, gp, pr.pdl, st);
+    return pr.f32_out ? launch_decode(ptpc_gemm_decode_kernel<true>, pl.ctas, pl.ksplit, smem, tmW, tmX, gp,
+                                      pr.pdl, st)
+                      : launch_decode(ptpc_gemm_decode_kernel<false>, pl.ctas, pl.ksplit, smem, tmW, tmX, gp,
+                                      pr.pdl, st);
   }
   CUtensorMap tmA, tmB, tmC;
   if (!make_maps(pr, kPairHalfN, &tmA, &tmB, &tmC)) return cudaErrorInvalidValue;

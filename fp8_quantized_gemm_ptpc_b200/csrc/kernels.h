@@ -19,7 +19,7 @@ cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, fl
 cudaError_t launch_apply_scales(const float *y, const float *xs, const float *ws, int T, int Co, void *out,
                                 cudaStream_t st);
 
-// Scaled GEMM (gemm.cu).
+// Scaled GEMM (gemm.cu).  Its only scratch is the device status word.
 struct GemmProblem {
   const uint8_t *Xq;      // [T, Ci]
   const float *xs;        // [T]   (unused for f32 output)
@@ -29,19 +29,14 @@ struct GemmProblem {
   void *out;              // bf16 [T, Co] or fp32 [T, Co]
   bool f32_out;           // unscaled fp32 output (naive step 1)
   uint32_t *status;       // device status word
-  uint32_t *counters;     // split-K tile counters (zero on entry, zero on exit)
-  float *partials;        // split-K fp32 partial sums
-  size_t partial_floats;  // capacity of `partials` (also caps the plan's partial sums)
   bool pdl;               // launch as a programmatic dependent of the previous kernel
 };
 
-// Workspace needs of the GEMM for a shape (counter words and partial floats)
-// when at most max_partial_floats partial-sum floats may be used (stream-K is
-// dropped for whole tiles when its partial sums would not fit).  A launch with
-// GemmProblem::partial_floats = the value returned here runs the same plan.
-void gemm_workspace_needs(int T, int Ci, int Co, size_t max_partial_floats, size_t *counter_words,
-                          size_t *partial_floats);
 cudaError_t launch_scaled_gemm(const GemmProblem &p, cudaStream_t st);
+
+// CTAs per tile the decode kernel uses for a shape (1: whole tiles; larger:
+// K split over a cluster of that many CTAs).  For tests and reports.
+int gemm_ksplit(int T, int Ci, int Co);
 
 int num_sms();
 

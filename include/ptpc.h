@@ -114,11 +114,12 @@ PTPC_API int ptpc_quantize_weights(const void *W_dev, int64_t Ci, int64_t Co,
  *   Xq_dev      u8 [T, Ci], x_scale_dev fp32 [T]   (from ptpc_quantize_activations)
  *   Wq_t_dev    u8 [Co, Ci], w_scale_dev fp32 [Co] (from ptpc_quantize_weights)
  *   out_dev     bf16 [T, Co] row-major, written once (no intermediate array).
- *   ws_dev      ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co) bytes: device
- *               status word, split-K tile counters and fp32 partial sums.
+ *   ws_dev      ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co) bytes: the
+ *               device status word.
  * The sum over k is an fp32 tensor-core accumulation; its order is not
- * specified.  Small T uses a split-K variant whose partial sums are reduced
- * in a fixed order, so results are deterministic for a given shape. */
+ * specified.  For T <= 128 and few output tiles, K is split over a cluster of
+ * 2, 4 or 8 CTAs (see ptpc_gemm_ksplit) whose fp32 partial sums are added in
+ * a fixed order, so results are deterministic for a given shape. */
 PTPC_API int ptpc_scaled_mm(const uint8_t *Xq_dev, const float *x_scale_dev,
                    const uint8_t *Wq_t_dev, const float *w_scale_dev,
                    int64_t T, int64_t Ci, int64_t Co, void *out_dev,
@@ -149,22 +150,26 @@ PTPC_API int ptpc_get_device_status(void *ws_dev, void *stream);
 /* Static, human-readable name of a status code. */
 PTPC_API const char *ptpc_status_string(int status);
 
+/* How ptpc_scaled_mm / ptpc_linear run a shape on the current device: the
+ * number of CTAs that share each output tile (1: every tile whole; 2, 4 or 8:
+ * K split over a cluster of that many CTAs, decode-sized T only).  0 on
+ * invalid arguments, T == 0 or an unsupported device.  Launches nothing. */
+PTPC_API int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co);
+
 /* ptpc_scaled_mm without a caller-provided workspace.  The page has no
  * counterpart: this exists for callers that cannot allocate device memory
  * when they call the GEMM (an engine that partitions all device memory at
  * start-up and forbids allocation on its serving path, or an integration that
  * only hands over input and output buffers).  Same arguments, layouts and
  * results as ptpc_scaled_mm minus (ws_dev, ws_bytes).
- *   Scratch: a file-scope 8 MiB device array inside the library, held by
- *   every GPU that loads the library until the process exits.  The GEMM's
- *   stream-K partial sums are kept within it: a shape whose partial sums
- *   would not fit runs on whole tiles instead (same results within the GEMM
- *   tolerance, possibly slower than ptpc_scaled_mm).  A shape whose remaining
- *   scratch (status word and tile counters) still exceeds the array is
+ *   Scratch: a file-scope 4 KiB device array inside the library, held by
+ *   every GPU that loads the library until the process exits; the GEMM uses
+ *   its first 256 bytes (the device status word).  Results are bit-identical
+ *   to ptpc_scaled_mm's.  A GEMM whose scratch exceeded the array would be
  *   rejected with PTPC_ERR_WORKSPACE_TOO_SMALL.
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress), so make that first call before any stream capture.
- *   Every call zeroes the array's control words with cudaMemsetAsync on
+ *   Every call zeroes the status word with cudaMemsetAsync on
  *   `stream` and allocates nothing.  All calls share the one array: calls
  *   that overlap on the GPU (different streams, or different host threads)
  *   race on it and give wrong results. */

@@ -55,8 +55,16 @@ def test_workspace_sizes(ptpc):
     assert ws(ptpc.OP_SCALED_MM, 16, 100, 64) == 0          # Ci not a multiple of 16
     assert ws(ptpc.OP_SCALED_MM, -1, 128, 64) == 0
     assert ws(99, 16, 128, 64) == 0
-    # decode sizes carry room for split-K partial sums
-    assert ws(ptpc.OP_SCALED_MM, 1, 28672, 8192) > 256 + 4 * 64
+    # the GEMM's only scratch is the device status word, at every size
+    assert ws(ptpc.OP_SCALED_MM, 1, 28672, 8192) == 256
+    assert ws(ptpc.OP_SCALED_MM, 8192, 28672, 8192) == 256
+
+
+def test_ksplit_query_rejects_bad_shapes(ptpc):
+    assert ptpc.gemm_ksplit(16, 100, 64) == 0     # Ci not a multiple of 16
+    assert ptpc.gemm_ksplit(16, 128, 60) == 0     # Co not a multiple of 16
+    assert ptpc.gemm_ksplit(-1, 128, 64) == 0
+    assert ptpc.gemm_ksplit(0, 128, 64) == 0      # nothing to run
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: checks fail before any access

@@ -78,6 +78,41 @@ def test_decode_full(ptpc, T, layer):
     assert_gemm_close(g, r, f"decode {L.name} T={T}")
 
 
+# Decode shapes whose tile counts (Co / 128) select each K split on a 148-SM
+# B200: 16 tiles -> 8 CTAs per tile (or 4, when fewer than 16 clusters of 8
+# fit at once), 32 -> 4, 64 -> 2, 80 -> whole tiles; 8 tiles -> 8.  Ci 4112
+# leaves a partial last K-block and uneven shares; Co 2064 a partial last
+# tile.
+@pytest.mark.parametrize("Ci,Co,splits", [
+    (4096, 1024, (8,)), (4096, 2048, (4, 8)), (4112, 2064, (4, 8)), (2048, 4096, (4,)), (1024, 8192, (2,)),
+    (4112, 8192, (2,)), (1024, 10240, (1,)),
+])
+@pytest.mark.parametrize("T", [1, 13, 77, 128])
+def test_decode_cluster_split(ptpc, T, Ci, Co, splits):
+    got_split = ptpc.gemm_ksplit(T, Ci, Co)
+    assert got_split in splits, f"{T}x{Ci}x{Co}: K split {got_split}, expected one of {splits}"
+    X = synthetic.with_edge_rows(synthetic.make_x(synthetic.DECODE_70B, 0, T, Ci), huge_bits=BIG_BF16)
+    W = synthetic.random_bf16((Ci, Co), seed=T * 7 + Ci + Co, scale=0.02)
+    g, r = run_pair(ptpc, X, W)
+    assert_gemm_close(g, r, f"decode {T}x{Ci}x{Co} split {got_split}")
+
+
+def test_decode_split_matches_naive_step1(ptpc):
+    """The K-split path's fp32 output (naive step 1) is what the fused path
+    scales: applying the scales to it gives the fused output bit for bit."""
+    T, Ci, Co = 32, 2048, 4096
+    assert ptpc.gemm_ksplit(T, Ci, Co) > 1
+    X = synthetic.make_x(synthetic.DECODE_70B, 1, T, Ci)
+    W = synthetic.random_bf16((Ci, Co), seed=5, scale=0.02)
+    Xd, Wd = to_dev_bf16(X), to_dev_bf16(W)
+    Wq_t, ws = ptpc.quantize_weights(Wd)
+    Xq, xs = ptpc.quantize_activations(Xd)
+    y = ptpc.unscaled_mm_f32(Xq, Wq_t)
+    naive = ptpc.apply_scales(y, xs, ws)
+    fused = ptpc.scaled_mm(Xq, xs, Wq_t, ws)
+    assert torch.equal(naive.view(torch.int16), fused.view(torch.int16))
+
+
 def sample_rows(T, n=256, seed=0):
     rng = np.random.default_rng(seed)
     rows = {0, T - 1} | {min(T - 1, b) for b in range(127, T, 128)} | {min(T - 1, b + 1) for b in range(127, T, 128)}

@@ -5,10 +5,10 @@ and output buffers).  Its scratch is the library's own static device array,
 so the caller passes no workspace.
 
 Checked through the C ABI against ptpc_scaled_mm (which takes a caller
-workspace) on two calls in a row, with shapes that use the scratch for
-stream-K partial sums and tile counters, and shapes whose partial sums do
-not fit (the entry point then runs whole tiles).  This file is collected
-last on purpose."""
+workspace) on two calls in a row, on decode shapes (K split over a cluster
+and whole tiles) and a prefill shape: the two entry points run the same plan,
+so the outputs agree within the GEMM tolerance and, in fact, bit for bit.
+This file is collected last on purpose."""
 import ctypes
 
 import numpy as np
@@ -36,12 +36,12 @@ def _abi_call(ptpc, Xq, xs, Wq_t, ws, out):
         P(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("T,layer", [(8, 1), (32, 1), (128, 1), (1, 0), (300, 0)])
+@pytest.mark.parametrize("T,layer", [(8, 1), (32, 1), (128, 1), (1, 0), (128, 0), (300, 0)])
 def test_static_scratch_matches_workspace_entry_point(ptpc, T, layer):
     w = synthetic.DECODE_70B
     L = w.layers[layer]
     Ci, Co = L.Ci, L.Co
-    if T > 128:  # a prefill-sized case (no split-K); keep the weight small
+    if T > 128:  # a prefill-sized case; keep the weight small
         Co = 4096
     X = synthetic.make_x(w, layer, T, Ci)
     W = synthetic.make_w(w, layer, Ci, Co)
@@ -55,8 +55,4 @@ def test_static_scratch_matches_workspace_entry_point(ptpc, T, layer):
         torch.cuda.synchronize()
         got = from_dev_bf16(out)
         assert_gemm_close(got, ref_bits, f"static scratch T={T} {Ci}->{Co}")
-        assert np.isfinite(bf16_bits_as_float(got)).all()
-
-
-def bf16_bits_as_float(bits):
-    return (bits.astype(np.uint32) << 16).view(np.float32)
+        assert np.array_equal(got, ref_bits)
