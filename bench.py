@@ -239,9 +239,10 @@ def run_reference(args):
 
 # ----------------------------------------------------------------- GPU arm
 
-def traffic_record(kernel_src_hash):
-    """DRAM bytes per GEMM launch from a committed ncu summary, if it was
-    taken on the current kernel source."""
+def traffic_record(kernel_src_hash, key):
+    """DRAM bytes (read + write) of one step's GEMM launches for workload
+    `key`, from the committed ncu summary, if that was taken on the current
+    kernel source; None otherwise."""
     path = os.path.join(ROOT, "profiles", "gemm_dram_traffic.json")
     if not os.path.exists(path):
         return None
@@ -249,7 +250,8 @@ def traffic_record(kernel_src_hash):
         d = json.load(f)
     if d.get("kernel_src_sha256") != kernel_src_hash:
         return None
-    return d.get("dram_bytes_per_step")
+    e = d.get("entries", {}).get(key)
+    return None if e is None else e.get("dram_bytes_per_step")
 
 
 def kernel_src_hash():
@@ -367,7 +369,7 @@ def run_gpu(args):
     hbm_bound = flops / g_bytes < ridge
     q_bytes = sum(quant_bytes(d["T"], d["Ci"]) for d in L)
     q_gbs = q_bytes / (sum(q_ms) / 1e3) / 1e9
-    dram = traffic_record(kernel_src_hash())
+    dram = traffic_record(kernel_src_hash(), f"{args.workload}:T={T}")
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W,
@@ -388,6 +390,7 @@ def run_gpu(args):
             "frac_of_sustained": gemm_tflops / fp8_peak_sus,
         }) | {
             "kernel": "ptpc scaled GEMM (fused epilogue), all layers of one step",
+            "traffic_unit": "bytes per step (dram__bytes_read.sum + dram__bytes_write.sum over the step's GEMM launches)",
             "algorithmic_flops_per_step": flops, "algorithmic_bytes_per_step": g_bytes,
             "gemm_tflops": gemm_tflops, "gemm_gbs": gemm_gbs,
             "per_layer_ms": {d["name"]: g for d, g in zip(L, g_ms)},
