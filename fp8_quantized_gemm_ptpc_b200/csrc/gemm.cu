@@ -9,9 +9,9 @@
 // written.  The page's kernel is AMD's (MI300X); these are written for B200.
 //
 // Two kernels share the structure below.
-//   * ptpc_gemm_pair_kernel (T > 128, prefill): a cluster of two CTAs on two
+//   * ptpc_gemm_pair_kernel (prefill): a cluster of two CTAs on two
 //     SMs computes 256 x 256 tiles with tcgen05.mma.cta_group::2.
-//   * ptpc_gemm_decode_kernel (T <= 128, decode): one CTA per SM, operands
+//   * ptpc_gemm_decode_kernel (decode, T <= 256; see make_plan): one CTA per SM, operands
 //     swapped — 128 weight rows are the MMA's M operand and the T tokens
 //     (padded to a multiple of 16) its N operand.
 // In both, warp 0 (one thread) streams 128-byte-wide K slices of Xq and Wq_t
@@ -201,18 +201,21 @@ __device__ __forceinline__ void epilogue_store_tile(const CUtensorMap *tmC, uint
 }
 
 // ----------------------------------------------------------------------------
-// Decode kernel (T <= 128), operands swapped: acc^T = Wq_t . Xq^T.
+// Decode kernel (T <= kDecodeMaxT), operands swapped: acc^T = Wq_t . Xq^T.
 // The 128 weight rows of a channel tile are the MMA's M = 128 operand and the
-// T tokens, padded to NP (a multiple of 16), are its N operand.  A stage then
-// carries 16 KB of weights and only NP x 128 bytes of activations, instead of
-// a 128-row activation box that is mostly out-of-bounds fill, and the ring is
-// as deep as shared memory allows (12 stages at NP = 16).  Tensor-memory lane
+// T tokens, padded to NP (a multiple of 16, at most 256), are its N operand.
+// A stage then carries 16 KB of weights and only NP x 128 bytes of
+// activations, instead of a 128-row activation box that is mostly
+// out-of-bounds fill, and the ring is as deep as shared memory allows (12
+// stages at NP = 16, 4 at NP = 256).  Tensor-memory lane
 // = output channel, column = token: each epilogue thread owns one channel, so
 // w_scale is one register and every token's 32 channels of a warp are one
 // contiguous store.  With ksplit = S > 1 the grid is made of S-CTA clusters,
 // one tile each, and the epilogue leaves the partial sums in shared memory
 // for the cluster reduction instead of storing.
 // ----------------------------------------------------------------------------
+constexpr int kDecodeMaxT = 256;       // largest T the decode kernel takes (MMA N <= 256)
+constexpr int kDecodeWholeMaxT = 192;  // above this, the decode kernel only when it splits K
 constexpr int kDecMaxStages = 16;
 constexpr int kDecWBytes = BM * BK;   // weight tile of one stage
 constexpr size_t kDecBarBytes = 512;  // barriers and flags after the ring
@@ -349,8 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
   const uint32_t acc_cols = (uint32_t)p.tmem_cols / 2;  // column stride of the two accumulators
   // K split: partial sums of the tile, [NP tokens][BM channels] fp32, in the
-  // weight ring (idle once the accumulator is complete; NP * 512 <= 64 KB,
-  // the ring holds at least 7 x 16 KB)
+  // ring (idle once the accumulator is complete; the weight and activation
+  // stages are contiguous, and NP * 512 bytes fit in them: checked by the plan)
   float *red = reinterpret_cast<float *>(sW);
 
   const int warp = threadIdx.x >> 5;
@@ -870,54 +873,77 @@ struct Plan {
   int ctas;     // CTAs (decode kernel) or CTA pairs (pair kernel) launched
   int ksplit;   // decode kernel: CTAs per tile (cluster size), 1 = whole tiles
   int np, stages, tmem_cols;  // decode kernel only
+  bool red_fits;              // decode kernel: the K-split buffer fits in the ring
 };
 
 // Fewest K-blocks a CTA of a K-split cluster streams.
 constexpr int kMinSplitKb = 4;
 
-Plan make_plan(int T, int Ci, int Co) {
-  const DeviceInfo &d = device_info();
+// The decode kernel's plan for T <= kDecodeMaxT: whole 128-channel tiles, or
+// K split over a cluster when that puts at least twice as many SMs on the
+// weight stream, all tiles in one wave.
+Plan decode_plan(int T, int Ci, int Co, const DeviceInfo &d) {
   Plan pl = {};
+  pl.pair = false;
   pl.num_kb = (Ci + BK - 1) / BK;
-  pl.pair = T > BM;
+  pl.tile_rows = std::max(T, 1);  // one tile row holds every token
+  pl.bn = BM;
+  pl.group_m = 1;
+  pl.np = std::max(16, (T + 15) / 16 * 16);
+  const size_t stage_bytes = kDecWBytes + (size_t)pl.np * BK;
+  pl.stages = (int)std::min<size_t>(kDecMaxStages, (kDecSmemMax - dec_smem_bytes(pl.np, 0)) / stage_bytes);
+  pl.tmem_cols = 64;  // each accumulator starts on a 32-column boundary
+  while (pl.tmem_cols < 2 * pl.np) pl.tmem_cols <<= 1;
+  // the K-split reduction buffer must fit in the ring (true for every NP <= 256)
+  pl.red_fits = (size_t)pl.np * BM * sizeof(float) <= (size_t)pl.stages * stage_bytes;
+  pl.num_m = 1;
+  pl.num_n = (Co + BM - 1) / BM;
+  pl.num_tiles = pl.num_n;
   pl.ksplit = 1;
-  if (pl.pair) {
-    pl.tile_rows = 2 * BM;
-    pl.bn = kPairBN;
-    pl.group_m = 8;
-  } else {
-    // decode kernel: one tile row holds every token; tiles are 128 channels
-    pl.tile_rows = std::max(T, 1);
-    pl.bn = BM;
-    pl.group_m = 1;
-    pl.np = std::max(16, (T + 15) / 16 * 16);
-    const size_t stage_bytes = kDecWBytes + (size_t)pl.np * BK;
-    pl.stages = (int)std::min<size_t>(kDecMaxStages, (kDecSmemMax - dec_smem_bytes(pl.np, 0)) / stage_bytes);
-    pl.tmem_cols = 64;  // each accumulator starts on a 32-column boundary
-    while (pl.tmem_cols < 2 * pl.np) pl.tmem_cols <<= 1;
-  }
-  pl.num_m = (T + pl.tile_rows - 1) / pl.tile_rows;
-  pl.num_n = (Co + pl.bn - 1) / pl.bn;
-  pl.num_tiles = pl.num_m * pl.num_n;
-  if (pl.pair) {
-    // Whole tiles only.  Sharing the last partial wave stream-K style (fp32
-    // partial sums through global memory, fixed-order fixup) was measured
-    // slower on B200 for 256 x 256 tiles (e.g. 2048 x 4096 -> 6144: 73.8 us
-    // shared vs 43.1 us whole; 2048 x 14336 -> 4096: 136.8 vs 109.7).
-    pl.ctas = std::max(1, std::min(pl.num_tiles, d.pair_clusters));
-    return pl;
-  }
-  // Decode: split K over a cluster when that puts at least twice as many SMs
-  // on the weight stream, all tiles in one wave.
   for (int size = 8; size >= 2; size /= 2) {
     if ((long long)pl.num_tiles * size <= d.sms && pl.num_tiles <= d.dec_clusters[size] &&
-        pl.num_kb >= size * kMinSplitKb) {
+        pl.num_kb >= size * kMinSplitKb && pl.red_fits) {
       pl.ksplit = size;
       break;
     }
   }
   pl.ctas = pl.ksplit > 1 ? pl.num_tiles * pl.ksplit : std::max(1, std::min(pl.num_tiles, d.sms));
   return pl;
+}
+
+// The prefill kernel's plan: whole 256 x 256 tiles on the CTA pairs.
+// Sharing the last partial wave stream-K style (fp32 partial sums through
+// global memory, fixed-order fixup) was measured slower on B200 for these
+// tiles (e.g. 2048 x 4096 -> 6144: 73.8 us shared vs 43.1 us whole;
+// 2048 x 14336 -> 4096: 136.8 vs 109.7).
+Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d) {
+  Plan pl = {};
+  pl.pair = true;
+  pl.ksplit = 1;
+  pl.num_kb = (Ci + BK - 1) / BK;
+  pl.tile_rows = 2 * BM;
+  pl.bn = kPairBN;
+  pl.group_m = 8;
+  pl.num_m = (T + pl.tile_rows - 1) / pl.tile_rows;
+  pl.num_n = (Co + pl.bn - 1) / pl.bn;
+  pl.num_tiles = pl.num_m * pl.num_n;
+  pl.ctas = std::max(1, std::min(pl.num_tiles, d.pair_clusters));
+  return pl;
+}
+
+// Which kernel runs a shape.  Measured on B200 with weights streamed from
+// HBM (70B layer shapes): the decode kernel is faster than the pair kernel
+// for every T <= 160; between 192 and 256 only where it splits K (e.g.
+// T = 256, 28672 -> 8192: 63.5 us vs 93.2 us), while with whole tiles it
+// ties at T = 192 and falls behind above (T = 256, 8192 -> 28672: 67.1 us vs
+// 59.0 us).
+Plan make_plan(int T, int Ci, int Co) {
+  const DeviceInfo &d = device_info();
+  if (T <= kDecodeMaxT) {
+    const Plan pl = decode_plan(T, Ci, Co, d);
+    if (T <= kDecodeWholeMaxT || pl.ksplit > 1) return pl;
+  }
+  return pair_plan(T, Ci, Co, d);
 }
 
 template <typename Kernel>

@@ -117,7 +117,7 @@ PTPC_API int ptpc_quantize_weights(const void *W_dev, int64_t Ci, int64_t Co,
  *   ws_dev      ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co) bytes: the
  *               device status word.
  * The sum over k is an fp32 tensor-core accumulation; its order is not
- * specified.  For T <= 128 and few output tiles, K is split over a cluster of
+ * specified.  For T <= 256 and few output tiles, K is split over a cluster of
  * 2, 4 or 8 CTAs (see ptpc_gemm_ksplit) whose fp32 partial sums are added in
  * a fixed order, so results are deterministic for a given shape. */
 PTPC_API int ptpc_scaled_mm(const uint8_t *Xq_dev, const float *x_scale_dev,

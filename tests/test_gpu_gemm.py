@@ -69,7 +69,7 @@ def test_llama8b_prefill_full(ptpc, layer):
     assert_gemm_close(g, r, L.name)
 
 
-@pytest.mark.parametrize("T", [1, 8, 32, 128])
+@pytest.mark.parametrize("T", [1, 8, 32, 128, 200])
 @pytest.mark.parametrize("layer", [0, 1])
 def test_decode_full(ptpc, T, layer):
     w = synthetic.DECODE_70B
@@ -87,7 +87,7 @@ def test_decode_full(ptpc, T, layer):
     (4096, 1024, (8,)), (4096, 2048, (4, 8)), (4112, 2064, (4, 8)), (2048, 4096, (4,)), (1024, 8192, (2,)),
     (4112, 8192, (2,)), (1024, 10240, (1,)),
 ])
-@pytest.mark.parametrize("T", [1, 13, 77, 128])
+@pytest.mark.parametrize("T", [1, 13, 77, 128, 160, 256])
 def test_decode_cluster_split(ptpc, T, Ci, Co, splits):
     got_split = ptpc.gemm_ksplit(T, Ci, Co)
     assert got_split in splits, f"{T}x{Ci}x{Co}: K split {got_split}, expected one of {splits}"
