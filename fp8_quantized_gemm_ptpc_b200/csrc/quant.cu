@@ -333,6 +333,21 @@ __global__ void broadcast_amax_kernel(const uint32_t *__restrict__ src, uint32_t
 }
 
 // ----------------------------------------------------------------------------
+// Weight quantisation, between the passes: each column's scale from its
+// maximum, once per column.  w_scale[o] = s; the column-maximum word is
+// replaced by the bits of RN(1/s) (never 0 for a nonzero column), or 0 for an
+// all-zero column, so pass 2 needs no division.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) weight_scales_kernel(uint32_t *__restrict__ col_amax,
+                                                            float *__restrict__ w_scale, int Co) {
+  const int o = blockIdx.x * blockDim.x + threadIdx.x;
+  if (o >= Co) return;
+  const GroupScale g = group_scale_from_amax_bits(col_amax[o]);
+  w_scale[o] = g.s;
+  col_amax[o] = g.mode == kZeroGroup ? 0u : __float_as_uint(g.r);
+}
+
+// ----------------------------------------------------------------------------
 // Weight quantisation, pass 2: quantise a 128 (k) x 64 (o) tile of W with its
 // columns' scales and write it transposed into Wq_t (Co x Ci).  Thread
 // (cv, kq) converts rows 4*kq .. 4*kq+3 of the 8 columns of vector cv, so for
@@ -345,9 +360,9 @@ constexpr int kTO = 64;    // output channels per tile
 constexpr int kTPitch = kTK + 4;
 
 __global__ void __launch_bounds__(256) quant_weight_t_kernel(const uint4 *__restrict__ W, int Ci, int Co,
-                                                             const uint32_t *__restrict__ col_amax,
+                                                             const uint32_t *__restrict__ col_rcp,
                                                              uint8_t *__restrict__ Wq_t,
-                                                             float *__restrict__ w_scale) {
+                                                             const float *__restrict__ w_scale) {
   __shared__ __align__(16) uint8_t tile[kTO][kTPitch];
   const int o0 = blockIdx.x * kTO;
   const int k0 = blockIdx.y * kTK;
@@ -361,11 +376,32 @@ __global__ void __launch_bounds__(256) quant_weight_t_kernel(const uint4 *__rest
     const int k = k0 + 4 * kq + r;
     v[r] = (k < Ci && ocol < Co) ? ld_stream(W + (int64_t)k * ncv + (ocol >> 3)) : make_uint4(0u, 0u, 0u, 0u);
   }
+  // this vector's 8 column scales and reciprocals (Co % 16 == 0: all valid or none)
+  float sc[8], rc[8];
+  if (ocol < Co) {
+    const float4 s0 = __ldg(reinterpret_cast<const float4 *>(w_scale + ocol));
+    const float4 s1 = __ldg(reinterpret_cast<const float4 *>(w_scale + ocol + 4));
+    const uint4 r0 = __ldg(reinterpret_cast<const uint4 *>(col_rcp + ocol));
+    const uint4 r1 = __ldg(reinterpret_cast<const uint4 *>(col_rcp + ocol + 4));
+    sc[0] = s0.x; sc[1] = s0.y; sc[2] = s0.z; sc[3] = s0.w;
+    sc[4] = s1.x; sc[5] = s1.y; sc[6] = s1.z; sc[7] = s1.w;
+    rc[0] = __uint_as_float(r0.x); rc[1] = __uint_as_float(r0.y);
+    rc[2] = __uint_as_float(r0.z); rc[3] = __uint_as_float(r0.w);
+    rc[4] = __uint_as_float(r1.x); rc[5] = __uint_as_float(r1.y);
+    rc[6] = __uint_as_float(r1.z); rc[7] = __uint_as_float(r1.w);
+  } else {
+    #pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      sc[c] = 1.0f;
+      rc[c] = 0.0f;
+    }
+  }
   #pragma unroll
   for (int c = 0; c < 8; ++c) {
-    const int o = ocol + c;
-    const GroupScale g = group_scale_from_amax_bits(o < Co ? col_amax[o] : 0u);
-    if (blockIdx.y == 0 && kq == 0 && o < Co) w_scale[o] = g.s;
+    GroupScale g;
+    g.s = sc[c];
+    g.r = rc[c];
+    g.mode = __float_as_uint(rc[c]) == 0u ? kZeroGroup : (sc[c] >= kFastPathMinScale ? kFast : kSlow);
     uint32_t word = 0;
     if (g.mode != kZeroGroup) {
       float q[4];
@@ -550,6 +586,8 @@ cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, fl
     col_amax_kernel<<<dim3(gx, slabs), kColThreads * kColWarps, 0, st>>>(Wv, Ci, Co, rows_per_cta, col_amax);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  weight_scales_kernel<<<(Co + 255) / 256, 256, 0, st>>>(col_amax, w_scale, Co);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 grid((Co + kTO - 1) / kTO, (Ci + kTK - 1) / kTK);
   quant_weight_t_kernel<<<grid, 256, 0, st>>>(Wv, Ci, Co, col_amax, Wq_t, w_scale);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
