@@ -167,8 +167,8 @@ PTPC_API int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co);
  *   its first 256 bytes (the device status word).  Results are bit-identical
  *   to ptpc_scaled_mm's.  A GEMM whose scratch exceeded the array would be
  *   rejected with PTPC_ERR_WORKSPACE_TOO_SMALL.
- *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress), so make that first call before any stream capture.
+ *   The first call on a device looks up the array's device address once
+ *   (cudaGetSymbolAddress; its failure returns PTPC_ERR_CUDA).
  *   Every call zeroes the status word with cudaMemsetAsync on
  *   `stream` and allocates nothing.  All calls share the one array: calls
  *   that overlap on the GPU (different streams, or different host threads)
