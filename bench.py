@@ -318,10 +318,12 @@ def run_gpu(args):
     def max_over_ranks(v):
         return dist_max(v, dev)
 
-    def timed(fn, steps):
+    def timed(fn, steps, before=None):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         barrier()
+        if before is not None:
+            before()
         e0.record(stream)
         for _ in range(steps):
             fn()
@@ -334,6 +336,12 @@ def run_gpu(args):
         step()
     with ClockSampler(local) as clk:
         ms = timed(step, K)
+    # The SM clock seen by the device over the same loop, repeated right
+    # after: the clock probe runs beside it on a side stream (kept out of the
+    # timed region above, which it could perturb).
+    probe = ptpc.ClockProbe(dev)
+    ms_probe = timed(step, K, before=lambda: probe.start(ms * 1.05 / 1e3))
+    probe_mhz = probe.mhz()
     ms = max_over_ranks(ms)
     flops = layer_flops(layers)
     value = whole_job_tflops(flops, world, K, ms)
@@ -377,7 +385,10 @@ def run_gpu(args):
         "dtype": "e4m3 x e4m3 -> f32 accumulate, bf16 out", "data": "synthetic",
         "config": dict(config_of(wl, layers, l2_note), parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
         "frac_of_fp8_peak": value / world / fp8_peak,
-        "clocks": clk.summary(),
+        "clocks": clk.summary() | {"sm_mhz_device": probe_mhz,
+                                   "sm_mhz_device_src": "median over 1 ms intervals of clock64 / globaltimer on "
+                                                        "one SM, during a repeat of the timed loop",
+                                   "repeat_ms_per_step": ms_probe / K},
         "gpu_launches": launches,
         "roofline": ({
             "bound": "hbm", "achieved": gemm_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -56,6 +56,7 @@ SIGNATURES = {
     "ptpc_scaled_mm_static_scratch": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "ptpc_bench_unscaled_mm_f32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "ptpc_bench_apply_scales": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _P, _P]),
+    "ptpc_bench_clock_probe": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_uint64, ctypes.c_uint64, _P, _P]),
     "ptpc_bench_quantize_activations_per_tensor": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "ptpc_bench_quantize_weights_per_tensor": (ctypes.c_int, [_P, _I64, _I64, _P, _P, _P, _SZ, _P]),
 }
@@ -288,6 +289,42 @@ def apply_scales(y, x_scale, w_scale, out: torch.Tensor | None = None):
            lib.ptpc_bench_apply_scales(_ptr(y), _ptr(x_scale), _ptr(w_scale), T, Co, _ptr(out),
                                        _stream(y.device)))
     return out
+
+
+class ClockProbe:
+    """Effective SM clock over a measured region (measurement only).
+
+    start(seconds) launches the library's clock probe on a side stream of the
+    current device (one sleeping thread, no shared memory); after the region,
+    mhz() synchronises the device and returns the median SM clock (MHz) over
+    the probe's 1 ms intervals, or None if it recorded fewer than two."""
+
+    def __init__(self, device, max_records: int = 16384):
+        self.device = torch.device(device)
+        self.records = torch.zeros((max_records, 2), dtype=torch.int64, device=self.device)
+        self.count = torch.zeros((1,), dtype=torch.int32, device=self.device)
+        self.stream = torch.cuda.Stream(self.device)
+
+    def start(self, seconds: float, period_ns: int = 1_000_000):
+        duration = int(max(0.0, min(seconds, 120.0)) * 1e9)
+        n = int(min(self.records.shape[0], duration // period_ns + 2))
+        _check("ptpc_bench_clock_probe",
+               lib.ptpc_bench_clock_probe(_ptr(self.records), max(2, n), period_ns, duration, _ptr(self.count),
+                                          ctypes.c_void_p(self.stream.cuda_stream)))
+
+    def mhz(self):
+        torch.cuda.synchronize(self.device)
+        n = int(self.count.item())
+        if n < 2:
+            return None
+        r = self.records[:n].cpu().numpy().astype("float64")
+        dt = r[1:, 0] - r[:-1, 0]
+        dc = r[1:, 1] - r[:-1, 1]
+        ok = dt > 0
+        if not ok.any():
+            return None
+        import numpy as np
+        return float(np.median(dc[ok] / dt[ok] * 1e3))
 
 
 def quantize_activations_per_tensor(X, Xq=None, x_scale=None, ws: Workspace | None = None):

@@ -7,6 +7,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/ptpc.h"
+#include "bench_probe.h"
 #include "kernels.h"
 
 namespace {
@@ -209,6 +210,18 @@ int ptpc_bench_unscaled_mm_f32(const uint8_t *Xq, const uint8_t *Wq_t, int64_t T
   if ((s = check_device()) != PTPC_OK) return s;
   return run_gemm(Xq, nullptr, Wq_t, nullptr, T, Ci, Co, y, true, static_cast<uint8_t *>(ws), false,
                   (cudaStream_t)stream);
+}
+
+int ptpc_bench_clock_probe(uint64_t *records_dev, int max_records, uint64_t period_ns, uint64_t duration_ns,
+                           int *count_dev, void *stream) {
+  if (!records_dev || !count_dev || max_records < 2) return PTPC_ERR_INVALID_ARG;
+  if (period_ns < 1000 || duration_ns > 120ull * 1000000000ull) return PTPC_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(records_dev) & 7u) != 0 || (reinterpret_cast<uintptr_t>(count_dev) & 3u) != 0)
+    return PTPC_ERR_MISALIGNED;
+  int s = check_device();
+  if (s != PTPC_OK) return s;
+  return cuda_status(ptpc::launch_clock_probe(reinterpret_cast<unsigned long long *>(records_dev), max_records,
+                                              period_ns, duration_ns, count_dev, (cudaStream_t)stream));
 }
 
 int ptpc_bench_apply_scales(const float *y, const float *x_scale, const float *w_scale, int64_t T, int64_t Co,

@@ -190,6 +190,17 @@ PTPC_API int ptpc_bench_unscaled_mm_f32(const uint8_t *Xq_dev, const uint8_t *Wq
                                int64_t T, int64_t Ci, int64_t Co, float *y_dev,
                                void *ws_dev, size_t ws_bytes, void *stream);
 
+/* Effective SM clock during a measurement: one sleeping thread on one SM
+ * writes (globaltimer ns, clock64 cycles) pairs to records_dev
+ * (uint64 [max_records][2], 8-byte aligned) about every period_ns (>= 1000)
+ * until duration_ns (<= 120 s) have passed or max_records (>= 2) are
+ * written, and the number written to *count_dev.  Launched on `stream`,
+ * typically a side stream that runs alongside the kernels being timed; it
+ * uses no shared memory.  Clock = cycles / ns between records.  Every wait
+ * inside is bounded.  No counterpart on the page. */
+PTPC_API int ptpc_bench_clock_probe(uint64_t *records_dev, int max_records, uint64_t period_ns,
+                                    uint64_t duration_ns, int *count_dev, void *stream);
+
 /* Naive two-step path, step 2 (`output = output * token_scales *
  * channel_scales`): reads y_dev fp32 [T, Co] and writes
  * out_dev[t][o] = bf16_RNE((y[t][o] * x_scale[t]) * w_scale[o]). */

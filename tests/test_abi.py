@@ -107,6 +107,12 @@ def test_argument_checks_without_gpu(ptpc):
     assert call(ptpc, "ptpc_get_device_status", None, None) == ptpc.ERR_INVALID_ARG
     assert call(ptpc, "ptpc_bench_apply_scales", P(FAKE), P(FAKE), P(FAKE), -3, 64, P(FAKE), None) == \
         ptpc.ERR_INVALID_ARG
+    probe = lambda *a: call(ptpc, "ptpc_bench_clock_probe", *a)
+    assert probe(P(FAKE), 1, 1000000, 1000000, P(FAKE), None) == ptpc.ERR_INVALID_ARG      # < 2 records
+    assert probe(P(FAKE), 64, 10, 1000000, P(FAKE), None) == ptpc.ERR_INVALID_ARG          # period < 1 us
+    assert probe(P(FAKE), 64, 1000000, 121 * 10**9, P(FAKE), None) == ptpc.ERR_INVALID_ARG  # > 120 s
+    assert probe(P(FAKE + 4), 64, 1000000, 1000000, P(FAKE), None) == ptpc.ERR_MISALIGNED
+    assert probe(None, 64, 1000000, 1000000, P(FAKE), None) == ptpc.ERR_INVALID_ARG
 
 
 def test_binding_rejects_cpu_tensors(ptpc):
