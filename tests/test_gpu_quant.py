@@ -136,6 +136,16 @@ def test_per_tensor(ptpc):
     assert (ws.cpu().numpy() == np.float32(wsc)).all()
 
 
+def test_per_tensor_weights_long_columns(ptpc):
+    """Per-tensor weight scale on long columns (Ci = 28672, the 70B down-proj
+    input width) and a narrow output (Co = 64)."""
+    W = synthetic.make_w(synthetic.DECODE_70B, 1, 28672, 64)
+    Wq_t, ws = ptpc.quantize_weights_per_tensor(to_dev_bf16(W))
+    wq, wsc = oracle.quant_weight_per_tensor(W)
+    assert np.array_equal(Wq_t.cpu().numpy(), wq)
+    assert (ws.cpu().numpy() == np.float32(wsc)).all()
+
+
 def test_codes_do_not_depend_on_stream_or_repeat(ptpc):
     X = synthetic.make_x(synthetic.LLAMA8B_PREFILL, 1, 333, 4096)
     Xd = to_dev_bf16(X)
