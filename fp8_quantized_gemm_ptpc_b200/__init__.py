@@ -53,6 +53,7 @@ SIGNATURES = {
     "ptpc_get_device_status": (ctypes.c_int, [_P, _P]),
     "ptpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ptpc_gemm_ksplit": (ctypes.c_int, [_I64, _I64, _I64]),
+    "ptpc_selftest_wait_timeout": (ctypes.c_int, [_P, _P]),
     "ptpc_scaled_mm_static_scratch": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "ptpc_bench_unscaled_mm_f32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "ptpc_bench_apply_scales": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _P, _P]),
@@ -241,8 +242,9 @@ def linear(X, Wq_t, w_scale, out: torch.Tensor | None = None, ws: Workspace | No
 def scaled_mm_static_scratch(Xq, x_scale, Wq_t, w_scale, out: torch.Tensor | None = None):
     """scaled_mm whose scratch is the library's own static device array (no
     workspace argument, nothing allocated by the library; ``out`` may be
-    passed to avoid the output allocation here).  Calls must not overlap on
-    the GPU; shapes needing more than 8 MiB of scratch are rejected."""
+    passed to avoid the output allocation here).  The array is 4 KiB per
+    device, of which the GEMM uses its 256-byte status word; calls must not
+    overlap on the GPU."""
     _need(Xq, "Xq", torch.uint8, 2)
     _need(Wq_t, "Wq_t", torch.uint8, 2)
     _need(x_scale, "x_scale", torch.float32, 1)
@@ -256,6 +258,12 @@ def scaled_mm_static_scratch(Xq, x_scale, Wq_t, w_scale, out: torch.Tensor | Non
            lib.ptpc_scaled_mm_static_scratch(_ptr(Xq), _ptr(x_scale), _ptr(Wq_t), _ptr(w_scale), T, Ci, Co,
                                              _ptr(out), _stream(Xq.device)))
     return out
+
+
+def selftest_wait_timeout(ws: Workspace):
+    """Launch the failure-path self-test on the current stream: a bounded
+    wait that must run out (about 2 s) and set the workspace's status word."""
+    _check("ptpc_selftest_wait_timeout", lib.ptpc_selftest_wait_timeout(ws.ptr(), _stream(ws.device)))
 
 
 def device_status(ws: Workspace) -> int:

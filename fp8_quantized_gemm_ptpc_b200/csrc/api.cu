@@ -187,6 +187,14 @@ int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co) {
   return ptpc::gemm_ksplit((int)T, (int)Ci, (int)Co);
 }
 
+int ptpc_selftest_wait_timeout(void *ws, void *stream) {
+  if (!ws) return PTPC_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return PTPC_ERR_MISALIGNED;
+  int s = check_device();
+  if (s != PTPC_OK) return s;
+  return cuda_status(ptpc::launch_wait_timeout_selftest(static_cast<uint32_t *>(ws), (cudaStream_t)stream));
+}
+
 int ptpc_get_device_status(void *ws, void *stream) {
   if (!ws) return PTPC_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;

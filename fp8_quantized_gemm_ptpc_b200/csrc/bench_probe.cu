@@ -1,4 +1,5 @@
-// Measurement support: the effective SM clock during a timed region.
+// Measurement support: the effective SM clock during a timed region; and a
+// self-test of the bounded waits' failure path.
 //
 // One thread records (%globaltimer, %clock64) pairs about every period_ns
 // for duration_ns, sleeping in between (the warp issues almost nothing and
@@ -36,7 +37,27 @@ __global__ void clock_probe_kernel(unsigned long long *__restrict__ out, int max
   *count = n;
 }
 
+// Status bit set by the wait self-test below.
+constexpr uint32_t kStatusTimeoutSelftest = 1u << 3;
+
+// One thread waits, with the kernels' own bounded mbar_wait, on a barrier
+// that nothing ever arrives at: the wait runs out after its limit (2 s of
+// %globaltimer), the kernel records the timeout in the status word and
+// returns.  Nothing faults or hangs; the context stays usable.
+__global__ void wait_timeout_selftest_kernel(uint32_t *status) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  if (!mbar_wait(&bar, 0)) atomicOr(status, kStatusTimeoutSelftest);
+}
+
 }  // namespace
+
+cudaError_t launch_wait_timeout_selftest(uint32_t *status, cudaStream_t st) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(status);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_clock_probe(unsigned long long *out, int max_records, uint64_t period_ns, uint64_t duration_ns,
                                int *count, cudaStream_t st) {

@@ -1,4 +1,4 @@
-// Measurement support (bench_probe.cu), kept apart from the kernels' interface.
+// Measurement and self-test support (bench_probe.cu), kept apart from the kernels' interface.
 #pragma once
 
 #include <cstdint>
@@ -10,5 +10,9 @@ namespace ptpc {
 // duration_ns into out[2 * max_records]; the number written goes to *count.
 cudaError_t launch_clock_probe(unsigned long long *out, int max_records, uint64_t period_ns, uint64_t duration_ns,
                                int *count, cudaStream_t st);
+
+// Launches a kernel whose bounded wait must run out (about 2 s) and record a
+// timeout bit in *status.
+cudaError_t launch_wait_timeout_selftest(uint32_t *status, cudaStream_t st);
 
 }  // namespace ptpc

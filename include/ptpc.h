@@ -147,6 +147,16 @@ PTPC_API size_t ptpc_workspace_size(int op, int64_t T, int64_t Ci, int64_t Co);
  * PTPC_OK or PTPC_ERR_DEVICE_TIMEOUT (PTPC_ERR_CUDA if the read fails). */
 PTPC_API int ptpc_get_device_status(void *ws_dev, void *stream);
 
+/* Self-test of the failure path: launches on `stream` one thread that waits,
+ * with the same bounded wait the GEMM kernels use, on an mbarrier that
+ * nothing arrives at.  The wait runs out after its limit (about 2 s of GPU
+ * time), the kernel sets a bit in the status word at the start of ws_dev
+ * (256-byte aligned workspace of at least 256 bytes) and returns; nothing
+ * faults or hangs and the context stays usable.  A following
+ * ptpc_get_device_status(ws_dev, stream) returns PTPC_ERR_DEVICE_TIMEOUT and
+ * clears the word.  No counterpart on the page. */
+PTPC_API int ptpc_selftest_wait_timeout(void *ws_dev, void *stream);
+
 /* Static, human-readable name of a status code. */
 PTPC_API const char *ptpc_status_string(int status);
 

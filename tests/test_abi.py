@@ -113,6 +113,8 @@ def test_argument_checks_without_gpu(ptpc):
     assert probe(P(FAKE), 64, 1000000, 121 * 10**9, P(FAKE), None) == ptpc.ERR_INVALID_ARG  # > 120 s
     assert probe(P(FAKE + 4), 64, 1000000, 1000000, P(FAKE), None) == ptpc.ERR_MISALIGNED
     assert probe(None, 64, 1000000, 1000000, P(FAKE), None) == ptpc.ERR_INVALID_ARG
+    assert call(ptpc, "ptpc_selftest_wait_timeout", None, None) == ptpc.ERR_INVALID_ARG
+    assert call(ptpc, "ptpc_selftest_wait_timeout", P(FAKE + 16), None) == ptpc.ERR_MISALIGNED
 
 
 def test_binding_rejects_cpu_tensors(ptpc):

@@ -206,7 +206,8 @@ def test_empty_input_is_noop(ptpc):
 
 def test_workspace_shared_across_entry_points(ptpc):
     """Every entry point leaves the workspace's control words zero, so one
-    workspace can serve the weight quantiser and a split-K GEMM in turn."""
+    workspace can serve the weight quantiser, the per-tensor quantiser and a
+    decode GEMM with K split over a cluster in turn."""
     T, Ci, Co = 1, 28672, 8192
     need = max(ptpc.workspace_size(ptpc.OP_LINEAR, T, Ci, Co),
                ptpc.workspace_size(ptpc.OP_QUANTIZE_WEIGHTS, 0, Ci, Co),
