@@ -652,9 +652,25 @@ def run_sweep(args):
                 Xq, xs = ptpc.quantize_activations_per_tensor(layer_input(i), *qs[i], ws=pts[i])
                 ptpc.scaled_mm(Xq, xs, Wq, ws, out=outs[i], ws=wsps[i])
 
+        # the fused chain captured once into a CUDA graph and replayed (the
+        # library only enqueues work on the current stream)
+        for _ in range(2):
+            fused()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        capture_stream = torch.cuda.Stream(dev)
+        with torch.cuda.stream(capture_stream):
+            with torch.cuda.graph(graph, stream=capture_stream):
+                fused()
+        torch.cuda.synchronize(dev)
+
+        def fused_graph():
+            graph.replay()
+
         K = max(3, min(200, int(4e13 / (flops_tok * T))))
         res = {}
-        for name, fn in (("fused", fused), ("naive", naive), ("per_tensor", per_tensor)):
+        for name, fn in (("fused", fused), ("fused_graph", fused_graph), ("naive", naive),
+                         ("per_tensor", per_tensor)):
             for _ in range(3):
                 fn()
             e0 = torch.cuda.Event(enable_timing=True)
@@ -668,13 +684,14 @@ def run_sweep(args):
             res[name] = e0.elapsed_time(e1) / K
         print(json.dumps({
             "kind": "chain_sweep", "workload": wl.name, "T": T, "steps": K,
-            "fused_ms": res["fused"], "naive_ms": res["naive"], "per_tensor_ms": res["per_tensor"],
+            "fused_ms": res["fused"], "fused_graph_ms": res["fused_graph"], "naive_ms": res["naive"],
+            "per_tensor_ms": res["per_tensor"],
             "fused_tflops": flops_tok * T / (res["fused"] / 1e3) / 1e12,
             "fused_frac_of_fp8_peak": flops_tok * T / (res["fused"] / 1e3) / 1e12 / (2.0 * peaks["bf16_tflops"]),
             "fused_speedup_over_naive": res["naive"] / res["fused"],
             "ptpc_over_per_tensor_throughput": res["per_tensor"] / res["fused"],
         }), flush=True)
-        del X0, outs, wsps, ys, qs, pts
+        del graph, X0, outs, wsps, ys, qs, pts
         torch.cuda.empty_cache()
     return 0
 
