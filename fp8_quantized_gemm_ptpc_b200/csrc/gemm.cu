@@ -11,9 +11,9 @@
 // Two kernels share the structure below.
 //   * ptpc_gemm_pair_kernel (prefill): a cluster of two CTAs on two
 //     SMs computes 256 x 256 tiles with tcgen05.mma.cta_group::2.
-//   * ptpc_gemm_decode_kernel (decode, T <= 256; see make_plan): one CTA per SM, operands
-//     swapped — 128 weight rows are the MMA's M operand and the T tokens
-//     (padded to a multiple of 16) its N operand.
+//   * ptpc_gemm_decode_kernel (decode-sized T, at most 256; see make_plan):
+//     one CTA per SM, operands swapped — 128 weight rows are the MMA's M
+//     operand and the T tokens (padded to a multiple of 16) its N operand.
 // In both, warp 0 (one thread) streams 128-byte-wide K slices of Xq and Wq_t
 // with TMA into a shared-memory ring (128-byte swizzle, no multicast); warp 1
 // (one thread) issues the MMAs (E4M3 x E4M3 -> fp32, K = 32 each) into one of
@@ -56,7 +56,7 @@ constexpr int kPairHalfN = 128; // weight rows each CTA of a pair loads
 
 struct GemmParams {
   int T, Co;
-  int num_m, num_n, num_kb;   // tile grid (rows of tiles are 128 or 256 tokens)
+  int num_m, num_n, num_kb;   // tile grid (pair kernel: 256-token tile rows; decode: one row of all tokens)
   int group_m;                // tile rows visited together (L2 reuse of weights)
   int num_tiles;
   int ksplit;                 // decode kernel: CTAs (one cluster) per tile, 1 = whole tiles
