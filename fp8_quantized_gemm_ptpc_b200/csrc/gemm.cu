@@ -37,6 +37,7 @@
 // its own copies and MMAs drain, frees its tensor memory and exits.
 #include <algorithm>
 #include <cstdint>
+#include <mutex>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -820,14 +821,16 @@ int max_clusters(Kernel kernel, int sms, int size, size_t smem) {
   return n;
 }
 
-DeviceInfo &device_info() {
+const DeviceInfo &device_info() {
   static DeviceInfo info[64];
   static DeviceInfo fallback;
+  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
     return fallback;
   }
+  std::lock_guard<std::mutex> lock(mu);  // first use of a device may come from several host threads
   DeviceInfo &d = info[dev];
   if (!d.ready) {
     int v = 0;

@@ -530,16 +530,6 @@ cudaError_t launch_act(const void *X, int T, int Ci, int64_t ldx, uint8_t *Xq, f
   }
 }
 
-int num_sms_cached() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
 
 }  // namespace
 
@@ -552,7 +542,7 @@ cudaError_t launch_quant_act_per_tensor(const void *X, int T, int Ci, int64_t ld
   cudaError_t e = cudaMemsetAsync(amax_slot, 0, sizeof(uint32_t), st);
   if (e != cudaSuccess) return e;
   const int64_t n8 = (int64_t)T * Ci / 8;
-  int grid = (int)std::min<int64_t>((n8 + 511) / 512, (int64_t)num_sms_cached() * 4);
+  int grid = (int)std::min<int64_t>((n8 + 511) / 512, (int64_t)num_sms() * 4);
   if (grid < 1) grid = 1;
   amax_kernel<<<grid, 512, 0, st>>>(static_cast<const uint4 *>(X), T, Ci / 8, ldx / 8, amax_slot);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -569,7 +559,7 @@ cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, fl
     uint32_t *slot = col_amax + Co;
     if ((e = cudaMemsetAsync(slot, 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
     const int64_t n8 = (int64_t)Ci * Co / 8;
-    int grid = (int)std::min<int64_t>((n8 + 511) / 512, (int64_t)num_sms_cached() * 4);
+    int grid = (int)std::min<int64_t>((n8 + 511) / 512, (int64_t)num_sms() * 4);
     amax_kernel<<<grid, 512, 0, st>>>(Wv, Ci, Co / 8, Co / 8, slot);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     broadcast_amax_kernel<<<(Co + 255) / 256, 256, 0, st>>>(slot, col_amax, Co);
@@ -579,7 +569,7 @@ cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, fl
     const int ncv = Co / 8;
     const int gx = (ncv + kColThreads - 1) / kColThreads;
     // enough row slabs to fill the GPU a few times over
-    int slabs = std::max(1, (num_sms_cached() * 4 + gx - 1) / gx);
+    int slabs = std::max(1, (num_sms() * 4 + gx - 1) / gx);
     int rows_per_cta = (Ci + slabs - 1) / slabs;
     rows_per_cta = std::max(rows_per_cta, 64);
     slabs = (Ci + rows_per_cta - 1) / rows_per_cta;
@@ -598,7 +588,7 @@ cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, fl
 cudaError_t launch_apply_scales(const float *y, const float *xs, const float *ws, int T, int Co, void *out,
                                 cudaStream_t st) {
   const int64_t total = (int64_t)T * (Co / 8);
-  int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)num_sms_cached() * 8);
+  int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)num_sms() * 8);
   if (grid < 1) grid = 1;
   apply_scales_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4 *>(y), T, Co, xs, ws,
                                             static_cast<uint4 *>(out));
