@@ -410,6 +410,9 @@ def run_gpu(args):
             "value": q_gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"], "frac": q_gbs / peaks["hbm_gbs"],
             "bytes_per_step": q_bytes, "per_layer_ms": {d["name"]: q for d, q in zip(L, q_ms)},
             "peak_src": f"{peaks['src']} HBM copy",
+            "note": "inside the step: each launch timed by events between the GEMMs (launch gap included), "
+                    "at the clock the GEMMs' power draw leaves; the quantiser alone on inputs larger than L2: "
+                    "bench.py --quant-only --workload llama70b_prefill",
         },
     }
 
