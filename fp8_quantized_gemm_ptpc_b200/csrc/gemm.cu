@@ -52,8 +52,6 @@ constexpr int BM = 128;      // token rows per CTA tile (tensor-memory lanes)
 constexpr int BK = 128;      // K bytes per stage (= one 128-byte swizzle row)
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
-constexpr int kPairBN = 256;    // CTA-pair tile width (MMA N)
-constexpr int kPairHalfN = 128; // weight rows each CTA of a pair loads
 
 struct GemmParams {
   int T, Co;
@@ -542,22 +540,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 // 32 KB of operands per 128-deep K-block instead of 48 KB for a one-CTA
 // 128 x 256 tile, for the same tensor work.
 // ----------------------------------------------------------------------------
-template <int STAGES, bool F32OUT>
+// BN: tile width (MMA N), 256 or 128; each CTA of the pair loads BN / 2
+// weight rows.
+template <int STAGES, bool F32OUT, int BN>
 struct PairCfg {
   static constexpr int A_BYTES = BM * BK;
-  static constexpr int B_BYTES = kPairHalfN * BK;
+  static constexpr int B_BYTES = (BN / 2) * BK;
   static constexpr int EPI_BUF = 32 * 128;
-  static constexpr int TMEM_COLS = 512;
+  static constexpr int TMEM_COLS = 2 * BN;  // two accumulators (a power of two >= 32)
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + kEpiWarps * EPI_BUF +
                                  kEpiWarps * 64 * sizeof(float) + 256;
   static_assert(SMEM <= 232448, "shared memory");
 };
 
-template <int STAGES, bool F32OUT>
+template <int STAGES, bool F32OUT, int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ptpc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
-  using C = PairCfg<STAGES, F32OUT>;
+  using C = PairCfg<STAGES, F32OUT, BN>;
+  constexpr int HALF_N = BN / 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sA = smem;
@@ -616,7 +617,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int pre = 0;
       sc.init(p, cid, ncl);
       if (sc.next(p, u)) {
-        const int b_row = u.n * kPairBN + (int)rank * kPairHalfN;
+        const int b_row = u.n * BN + (int)rank * HALF_N;
         for (; pre < STAGES && u.kb0 + pre < u.kb1; ++pre) {
           if (leader) mbar_arrive_expect_tx(&full[pre], 2 * (C::A_BYTES + C::B_BYTES));
           tma_load_2d_pair(sB + pre * C::B_BYTES, &tmB, mapa_shared(&full[pre], 0), (u.kb0 + pre) * BK, b_row,
@@ -628,7 +629,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       sc.init(p, cid, ncl);
       while (ok && sc.next(p, u)) {
         const int a_row = u.m * (2 * BM) + (int)rank * BM;
-        const int b_row = u.n * kPairBN + (int)rank * kPairHalfN;
+        const int b_row = u.n * BN + (int)rank * HALF_N;
         for (int kb = u.kb0; kb < u.kb1; ++kb, ++issued) {
           const uint32_t lead_full = mapa_shared(&full[stage], 0);
           if (issued >= pre) {
@@ -658,7 +659,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (leader && elect_one()) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(2 * BM, kPairBN);
+      constexpr uint32_t idesc = idesc_e4m3_f32(2 * BM, BN);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -675,7 +676,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem_base + (uint32_t)(buf * kPairBN);
+        const uint32_t d = tmem_base + (uint32_t)(buf * BN);
         for (int kb = u.kb0; kb < u.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase)) {
             ok = false;
@@ -727,8 +728,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * kPairBN);
-      epilogue_store_tile<kPairBN, F32OUT>(&tmC, tbase, cbuf, scl, p, u.n * kPairBN, row0, xsr, lane,
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
+      epilogue_store_tile<BN, F32OUT>(&tmC, tbase, cbuf, scl, p, u.n * BN, row0, xsr, lane,
                                            mapa_shared(&tempty[buf], 0));
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeoutEpilogue);
@@ -787,14 +788,41 @@ bool make_maps(const GemmProblem &pr, uint32_t b_rows, CUtensorMap *tmA, CUtenso
                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-constexpr int kPairStages = 6;
+// Ring depth of the pair kernel per tile width (the stages fill ~192 KB).
+template <int BN>
+constexpr int pair_stages() {
+  return BN == 256 ? 6 : 8;
+}
+
+template <bool F32OUT, int BN>
+void set_pair_smem() {
+  cudaFuncSetAttribute(ptpc_gemm_pair_kernel<pair_stages<BN>(), F32OUT, BN>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)PairCfg<pair_stages<BN>(), F32OUT, BN>::SMEM);
+}
+
+// CTA pairs of the BN-wide pair kernel that can be resident at once.
+template <int BN>
+int pair_resident(int sms) {
+  cudaLaunchConfig_t q = {};
+  q.gridDim = dim3(2 * (sms / 2));
+  q.blockDim = dim3(kThreads);
+  q.dynamicSmemBytes = PairCfg<pair_stages<BN>(), false, BN>::SMEM;
+  int ncl = 0;
+  if (cudaOccupancyMaxActiveClusters(&ncl, ptpc_gemm_pair_kernel<pair_stages<BN>(), false, BN>, &q) != cudaSuccess ||
+      ncl <= 0)
+    ncl = sms / 2;
+  cudaGetLastError();
+  return ncl;
+}
 
 // Per device: dynamic shared-memory opt-in of every kernel variant, the SM
 // count, and the number of CTA pairs that can be resident at once.
 struct DeviceInfo {
   bool ready = false;
   int sms = 148;
-  int pair_clusters = 74;
+  int pair_clusters = 74;     // resident CTA pairs, 256-wide tiles
+  int pair_clusters128 = 74;  // resident CTA pairs, 128-wide tiles
   int dec_clusters[9] = {};  // resident decode clusters of 2, 4 and 8 CTAs
 };
 
@@ -839,22 +867,13 @@ const DeviceInfo &device_info() {
                          (int)kDecSmemMax);
     cudaFuncSetAttribute(ptpc_gemm_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)kDecSmemMax);
-    cudaFuncSetAttribute(ptpc_gemm_pair_kernel<kPairStages, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)PairCfg<kPairStages, false>::SMEM);
-    cudaFuncSetAttribute(ptpc_gemm_pair_kernel<kPairStages, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)PairCfg<kPairStages, true>::SMEM);
+    set_pair_smem<false, 256>();
+    set_pair_smem<true, 256>();
+    set_pair_smem<false, 128>();
+    set_pair_smem<true, 128>();
     // the pair kernel's cluster size is compiled in (__cluster_dims__)
-    cudaLaunchConfig_t q = {};
-    q.gridDim = dim3(2 * (d.sms / 2));
-    q.blockDim = dim3(kThreads);
-    q.dynamicSmemBytes = PairCfg<kPairStages, false>::SMEM;
-    int ncl = 0;
-    if (cudaOccupancyMaxActiveClusters(&ncl, ptpc_gemm_pair_kernel<kPairStages, false>, &q) == cudaSuccess &&
-        ncl > 0)
-      d.pair_clusters = ncl;
-    else
-      d.pair_clusters = d.sms / 2;
-    cudaGetLastError();
+    d.pair_clusters = pair_resident<256>(d.sms);
+    d.pair_clusters128 = pair_resident<128>(d.sms);
     // the decode kernel takes its cluster size at launch; ask for the largest
     // shared-memory footprint it launches with
     for (int size = 2; size <= 8; size *= 2) {
@@ -878,6 +897,14 @@ struct Plan {
   int np, stages, tmem_cols;  // decode kernel only
   bool red_fits;              // decode kernel: the K-split buffer fits in the ring
 };
+
+// Time of a 128-wide pair tile relative to half a 256-wide one.  Measured on
+// B200 from wave counts and times of both widths: 1.05-1.09 where the GEMM is
+// short, 1.14-1.18 on longer ones, 1.32 on the 70B gate+up at T = 8192 (more
+// operand bytes per FLOP under the power cap).  1.15 picks the faster width
+// on every measured shape, e.g. 512 x 8192 -> 10240: 53.7 us (128-wide, 3
+// waves) against 68.1 us (256-wide, 2 waves of which the second is 8% full).
+constexpr double kPairN128Cost = 1.15;
 
 // Fewest K-blocks a CTA of a K-split cluster streams.
 constexpr int kMinSplitKb = 4;
@@ -914,7 +941,18 @@ Plan decode_plan(int T, int Ci, int Co, const DeviceInfo &d) {
   return pl;
 }
 
-// The prefill kernel's plan: whole 256 x 256 tiles on the CTA pairs.
+// Tile width of the pair kernel for a shape: 128-wide tiles halve the size of
+// the last partial wave but move more operand bytes per FLOP, so they are
+// taken only when they finish the waves sooner by a margin.
+int choose_pair_bn(int T, int Co, const DeviceInfo &d) {
+  const long long m = (T + 2 * BM - 1) / (2 * BM);
+  const long long w256 = (m * ((Co + 255) / 256) + d.pair_clusters - 1) / d.pair_clusters;
+  const long long w128 = (m * ((Co + 127) / 128) + d.pair_clusters128 - 1) / d.pair_clusters128;
+  // cost in 128-wide tile-times; a 128-wide tile costs kPairN128Cost of half a 256-wide one
+  return (double)w128 * kPairN128Cost < (double)(2 * w256) ? 128 : 256;
+}
+
+// The prefill kernel's plan: whole tiles on the CTA pairs.
 // Sharing the last partial wave stream-K style (fp32 partial sums through
 // global memory, fixed-order fixup) was measured slower on B200 for these
 // tiles (e.g. 2048 x 4096 -> 6144: 73.8 us shared vs 43.1 us whole;
@@ -925,12 +963,12 @@ Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d) {
   pl.ksplit = 1;
   pl.num_kb = (Ci + BK - 1) / BK;
   pl.tile_rows = 2 * BM;
-  pl.bn = kPairBN;
+  pl.bn = choose_pair_bn(T, Co, d);
   pl.group_m = 8;
   pl.num_m = (T + pl.tile_rows - 1) / pl.tile_rows;
   pl.num_n = (Co + pl.bn - 1) / pl.bn;
   pl.num_tiles = pl.num_m * pl.num_n;
-  pl.ctas = std::max(1, std::min(pl.num_tiles, d.pair_clusters));
+  pl.ctas = std::max(1, std::min(pl.num_tiles, pl.bn == 128 ? d.pair_clusters128 : d.pair_clusters));
   return pl;
 }
 
@@ -985,6 +1023,13 @@ cudaError_t launch(Kernel kernel, int grid, size_t smem, const CUtensorMap &tmA,
   return cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmC, gp);
 }
 
+template <bool F32OUT, int BN>
+cudaError_t launch_pair(int grid, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC,
+                        const GemmParams &gp, bool pdl, cudaStream_t st) {
+  return launch(ptpc_gemm_pair_kernel<pair_stages<BN>(), F32OUT, BN>, grid,
+                PairCfg<pair_stages<BN>(), F32OUT, BN>::SMEM, tmA, tmB, tmC, gp, pdl, st);
+}
+
 }  // namespace
 
 int num_sms() { return device_info().sms; }
@@ -1023,12 +1068,13 @@ cudaError_t launch_scaled_gemm(const GemmProblem &pr, cudaStream_t st) {
                                       pr.pdl, st);
   }
   CUtensorMap tmA, tmB, tmC;
-  if (!make_maps(pr, kPairHalfN, &tmA, &tmB, &tmC)) return cudaErrorInvalidValue;
+  if (!make_maps(pr, pl.bn / 2, &tmA, &tmB, &tmC)) return cudaErrorInvalidValue;
   const int grid = 2 * pl.ctas;
-  return pr.f32_out ? launch(ptpc_gemm_pair_kernel<kPairStages, true>, grid, PairCfg<kPairStages, true>::SMEM, tmA,
-                             tmB, tmC, gp, pr.pdl, st)
-                    : launch(ptpc_gemm_pair_kernel<kPairStages, false>, grid, PairCfg<kPairStages, false>::SMEM,
-                             tmA, tmB, tmC, gp, pr.pdl, st);
+  if (pl.bn == 128)
+    return pr.f32_out ? launch_pair<true, 128>(grid, tmA, tmB, tmC, gp, pr.pdl, st)
+                      : launch_pair<false, 128>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
+  return pr.f32_out ? launch_pair<true, 256>(grid, tmA, tmB, tmC, gp, pr.pdl, st)
+                    : launch_pair<false, 256>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
 }
 
 }  // namespace ptpc
