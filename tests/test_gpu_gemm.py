@@ -114,10 +114,19 @@ def test_decode_split_matches_naive_step1(ptpc):
 
 
 def sample_rows(T, n=256, seed=0):
+    """About n output rows spread over all of T: the first and last rows, both
+    sides of evenly spaced 128-row tile boundaries (up to n / 4 boundaries),
+    and random rows for the rest."""
     rng = np.random.default_rng(seed)
-    rows = {0, T - 1} | {min(T - 1, b) for b in range(127, T, 128)} | {min(T - 1, b + 1) for b in range(127, T, 128)}
-    rows |= set(rng.choice(T, size=min(T, n), replace=False).tolist())
-    return np.array(sorted(rows)[: max(n, 2)], dtype=np.int64)
+    rows = {0, T - 1}
+    bounds = np.arange(128, T, 128)
+    if bounds.size:
+        pick = bounds[np.unique(np.linspace(0, bounds.size - 1, min(bounds.size, max(1, n // 4))).astype(np.int64))]
+        for b in pick.tolist():
+            rows |= {b - 1, b}
+    extra = max(0, n - len(rows))
+    rows |= set(rng.choice(T, size=min(T, extra), replace=False).tolist())
+    return np.array(sorted(rows), dtype=np.int64)
 
 
 @pytest.mark.parametrize("layer", [0, 1])
@@ -137,6 +146,20 @@ def test_chain_ragged_sampled(ptpc, T):
     rows = sample_rows(T, 128, seed=T)
     g, r = run_pair(ptpc, synthetic.make_x(w, 0, T, L.Ci), synthetic.make_w(w, 0, L.Ci, L.Co), rows=rows)
     assert_gemm_close(g, r, f"chain qkv T={T}")
+
+
+@pytest.mark.parametrize("layer", [2, 3])
+def test_chain_largest_T_sampled(ptpc, layer):
+    """The chain's largest size (T = 16384) on its two largest layers, gate+up
+    8192 -> 57344 and down 28672 -> 8192: codes bit-exact everywhere, outputs
+    checked on sampled rows (both sides of every 128-row boundary included)."""
+    w = synthetic.CHAIN_70B
+    L = w.layers[layer]
+    T = 16384
+    rows = sample_rows(T, 128, seed=layer)
+    g, r = run_pair(ptpc, synthetic.make_x(w, layer, T, L.Ci), synthetic.make_w(w, layer, L.Ci, L.Co), rows=rows,
+                    check_linear=False)
+    assert_gemm_close(g, r, f"chain {L.name} T={T}")
 
 
 def test_naive_two_step_equals_fused(ptpc):
