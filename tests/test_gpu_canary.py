@@ -1,0 +1,105 @@
+"""Stray-write checks: every output buffer (and the workspace) is placed
+inside a larger allocation whose guard bytes before and after must come back
+unchanged, over shapes that exercise every tail path (ragged rows and
+columns, both prefill tile widths, the decode kernel with and without a K
+split, the long-row quantiser, the naive path)."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import synthetic
+from helpers import to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+GUARD = 4096          # bytes on each side; keeps 256-byte alignment
+PATTERN = 0xA5
+
+
+@pytest.fixture(scope="module")
+def ptpc():
+    import fp8_quantized_gemm_ptpc_b200 as p
+    return p
+
+
+class Guarded:
+    """nbytes of device memory between two guard regions filled with PATTERN."""
+
+    def __init__(self, nbytes: int):
+        self.nbytes = nbytes
+        self.buf = torch.full((GUARD + nbytes + GUARD,), PATTERN, dtype=torch.uint8, device="cuda")
+
+    def view(self, dtype, shape):
+        return self.buf[GUARD:GUARD + self.nbytes].view(dtype).view(shape)
+
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.data_ptr() + GUARD)
+
+    def check(self, what):
+        torch.cuda.synchronize()
+        head = self.buf[:GUARD]
+        tail = self.buf[GUARD + self.nbytes:]
+        assert bool((head == PATTERN).all()), f"{what}: write before the buffer"
+        assert bool((tail == PATTERN).all()), f"{what}: write past the end of the buffer"
+
+
+@pytest.mark.parametrize("T,Ci", [(1, 16), (77, 4112), (1000, 256), (3, 65552)])
+def test_activation_quantiser_stays_in_bounds(ptpc, T, Ci):
+    X = to_dev_bf16(synthetic.make_x(synthetic.LLAMA8B_PREFILL, 0, T, Ci))
+    q, s = Guarded(T * Ci), Guarded(T * 4)
+    ptpc.quantize_activations(X, q.view(torch.uint8, (T, Ci)), s.view(torch.float32, (T,)))
+    q.check(f"Xq {T}x{Ci}")
+    s.check(f"x_scale {T}x{Ci}")
+
+
+@pytest.mark.parametrize("Ci,Co", [(16, 16), (384, 4112), (4112, 48), (4096, 6144)])
+def test_weight_quantiser_stays_in_bounds(ptpc, Ci, Co):
+    W = to_dev_bf16(synthetic.random_bf16((Ci, Co), seed=Ci + 3 * Co, scale=0.02))
+    q, s = Guarded(Co * Ci), Guarded(Co * 4)
+    need = ptpc.workspace_size(ptpc.OP_QUANTIZE_WEIGHTS, 0, Ci, Co)
+    ws = Guarded(need)
+    ws.view(torch.uint8, (need,)).zero_()
+    P = ctypes.c_void_p
+    st = P(torch.cuda.current_stream().cuda_stream)
+    assert ptpc.lib.ptpc_quantize_weights(P(W.data_ptr()), Ci, Co, q.ptr(), s.ptr(), ws.ptr(), need, st) == ptpc.OK
+    q.check(f"Wq_t {Ci}x{Co}")
+    s.check(f"w_scale {Ci}x{Co}")
+    ws.check(f"weight workspace {Ci}x{Co}")
+
+
+@pytest.mark.parametrize("T,Ci,Co", [
+    (1, 4096, 2048), (13, 2048, 4096), (128, 1024, 8192), (200, 4112, 8192), (77, 384, 528),
+    (300, 640, 1040), (512, 8192, 10240), (2048, 4096, 6144), (1000, 1024, 2064),
+])
+def test_gemm_and_linear_stay_in_bounds(ptpc, T, Ci, Co):
+    X = to_dev_bf16(synthetic.make_x(synthetic.DECODE_70B, 0, T, Ci))
+    Wq_t, ws = ptpc.quantize_weights(to_dev_bf16(synthetic.random_bf16((Ci, Co), seed=T + Ci, scale=0.02)))
+    Xq, xs = ptpc.quantize_activations(X)
+    out = Guarded(T * Co * 2)
+    need = ptpc.workspace_size(ptpc.OP_LINEAR, T, Ci, Co)
+    wsg = Guarded(need)
+    wsg.view(torch.uint8, (need,)).zero_()
+    ws_obj = ptpc.Workspace(0, "cuda")
+    ws_obj.buf = wsg.view(torch.uint8, (need,))
+    ptpc.scaled_mm(Xq, xs, Wq_t, ws, out=out.view(torch.bfloat16, (T, Co)), ws=ws_obj)
+    out.check(f"scaled_mm out {T}x{Ci}x{Co}")
+    wsg.check(f"scaled_mm workspace {T}x{Ci}x{Co}")
+    ptpc.linear(X, Wq_t, ws, out=out.view(torch.bfloat16, (T, Co)), ws=ws_obj)
+    out.check(f"linear out {T}x{Ci}x{Co}")
+    wsg.check(f"linear workspace {T}x{Ci}x{Co}")
+    assert ptpc.device_status(ws_obj) == ptpc.OK
+
+
+@pytest.mark.parametrize("T,Ci,Co", [(7, 1024, 2048), (300, 512, 1040)])
+def test_naive_path_stays_in_bounds(ptpc, T, Ci, Co):
+    X = to_dev_bf16(synthetic.make_x(synthetic.DECODE_70B, 1, T, Ci))
+    Wq_t, ws = ptpc.quantize_weights(to_dev_bf16(synthetic.random_bf16((Ci, Co), seed=11, scale=0.02)))
+    Xq, xs = ptpc.quantize_activations(X)
+    y, out = Guarded(T * Co * 4), Guarded(T * Co * 2)
+    ptpc.unscaled_mm_f32(Xq, Wq_t, out=y.view(torch.float32, (T, Co)))
+    y.check(f"naive step 1 {T}x{Ci}x{Co}")
+    ptpc.apply_scales(y.view(torch.float32, (T, Co)), xs, ws, out=out.view(torch.bfloat16, (T, Co)))
+    out.check(f"naive step 2 {T}x{Ci}x{Co}")
+    assert np.isfinite(out.view(torch.bfloat16, (T, Co)).float().cpu().numpy()).all()
