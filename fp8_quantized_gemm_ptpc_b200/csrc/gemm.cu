@@ -37,6 +37,8 @@
 // its own copies and MMAs drain, frees its tensor memory and exits.
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -906,6 +908,16 @@ struct Plan {
 // waves) against 68.1 us (256-wide, 2 waves of which the second is 8% full).
 constexpr double kPairN128Cost = 1.15;
 
+// Tuning overrides (not for production use): an integer environment
+// variable, or `fallback` when unset or not a number.
+int env_int(const char *name, int fallback) {
+  const char *v = std::getenv(name);
+  if (v == nullptr || *v == '\0') return fallback;
+  char *end = nullptr;
+  const long x = std::strtol(v, &end, 10);
+  return (end != nullptr && *end == '\0') ? (int)x : fallback;
+}
+
 // Fewest K-blocks a CTA of a K-split cluster streams.
 constexpr int kMinSplitKb = 4;
 
@@ -930,13 +942,19 @@ Plan decode_plan(int T, int Ci, int Co, const DeviceInfo &d) {
   pl.num_n = (Co + BM - 1) / BM;
   pl.num_tiles = pl.num_n;
   pl.ksplit = 1;
+  auto feasible = [&](int size) {
+    return (long long)pl.num_tiles * size <= d.sms && pl.num_tiles <= d.dec_clusters[size] &&
+           pl.num_kb >= size * kMinSplitKb && pl.red_fits;
+  };
   for (int size = 8; size >= 2; size /= 2) {
-    if ((long long)pl.num_tiles * size <= d.sms && pl.num_tiles <= d.dec_clusters[size] &&
-        pl.num_kb >= size * kMinSplitKb && pl.red_fits) {
+    if (feasible(size)) {
       pl.ksplit = size;
       break;
     }
   }
+  // PTPC_FORCE_KSPLIT = 1, 2, 4 or 8 (tuning only; ignored where infeasible)
+  const int forced = env_int("PTPC_FORCE_KSPLIT", 0);
+  if (forced == 1 || ((forced == 2 || forced == 4 || forced == 8) && feasible(forced))) pl.ksplit = forced;
   pl.ctas = pl.ksplit > 1 ? pl.num_tiles * pl.ksplit : std::max(1, std::min(pl.num_tiles, d.sms));
   return pl;
 }
@@ -945,6 +963,8 @@ Plan decode_plan(int T, int Ci, int Co, const DeviceInfo &d) {
 // the last partial wave but move more operand bytes per FLOP, so they are
 // taken only when they finish the waves sooner by a margin.
 int choose_pair_bn(int T, int Co, const DeviceInfo &d) {
+  const int forced = env_int("PTPC_FORCE_PAIR_BN", 0);  // 128 or 256 (tuning only)
+  if (forced == 128 || forced == 256) return forced;
   const long long m = (T + 2 * BM - 1) / (2 * BM);
   const long long w256 = (m * ((Co + 255) / 256) + d.pair_clusters - 1) / d.pair_clusters;
   const long long w128 = (m * ((Co + 127) / 128) + d.pair_clusters128 - 1) / d.pair_clusters128;
@@ -978,10 +998,15 @@ Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d) {
 // T = 256, 28672 -> 8192: 63.5 us vs 93.2 us), while with whole tiles it
 // ties at T = 192 and falls behind above (T = 256, 8192 -> 28672: 67.1 us vs
 // 59.0 us).
+// PTPC_FORCE_KERNEL = "pair" or "decode" overrides the choice (tuning only;
+// the decode kernel takes T <= 256 only).
 Plan make_plan(int T, int Ci, int Co) {
   const DeviceInfo &d = device_info();
+  const char *force = std::getenv("PTPC_FORCE_KERNEL");
+  if (force != nullptr && std::strcmp(force, "pair") == 0) return pair_plan(T, Ci, Co, d);
   if (T <= kDecodeMaxT) {
     const Plan pl = decode_plan(T, Ci, Co, d);
+    if (force != nullptr && std::strcmp(force, "decode") == 0) return pl;
     if (T <= kDecodeWholeMaxT || pl.ksplit > 1) return pl;
   }
   return pair_plan(T, Ci, Co, d);

@@ -162,6 +162,34 @@ def test_chain_largest_T_sampled(ptpc, layer):
     assert_gemm_close(g, r, f"chain {L.name} T={T}")
 
 
+def test_tuning_overrides(ptpc, monkeypatch):
+    """PTPC_FORCE_KSPLIT / PTPC_FORCE_PAIR_BN / PTPC_FORCE_KERNEL change the
+    plan (where feasible) and every forced plan still matches the oracle."""
+    T, Ci, Co = 32, 2048, 4096                 # 32 channel tiles: K split over 4 by default
+    assert ptpc.gemm_ksplit(T, Ci, Co) == 4
+    monkeypatch.setenv("PTPC_FORCE_KSPLIT", "2")
+    assert ptpc.gemm_ksplit(T, Ci, Co) == 2
+    monkeypatch.setenv("PTPC_FORCE_KSPLIT", "8")   # 32 x 8 CTAs do not fit in one wave: ignored
+    assert ptpc.gemm_ksplit(T, Ci, Co) == 4
+    monkeypatch.setenv("PTPC_FORCE_KSPLIT", "1")
+    assert ptpc.gemm_ksplit(T, Ci, Co) == 1
+    monkeypatch.delenv("PTPC_FORCE_KSPLIT")
+    X = synthetic.with_edge_rows(synthetic.make_x(synthetic.DECODE_70B, 0, 256, 1024), huge_bits=BIG_BF16)
+    W = synthetic.random_bf16((1024, 2064), seed=17, scale=0.02)
+    cases = [({"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_PAIR_BN": "128"}, 100),
+             ({"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_PAIR_BN": "256"}, 7),
+             ({"PTPC_FORCE_KERNEL": "decode"}, 256),
+             ({"PTPC_FORCE_KERNEL": "decode", "PTPC_FORCE_KSPLIT": "1"}, 64),
+             ({"PTPC_FORCE_KSPLIT": "2"}, 13)]
+    for env, t in cases:
+        for k, v in env.items():
+            monkeypatch.setenv(k, v)
+        g, r = run_pair(ptpc, X[:t].copy(), W)
+        assert_gemm_close(g, r, f"forced {env} T={t}")
+        for k in env:
+            monkeypatch.delenv(k)
+
+
 def test_naive_two_step_equals_fused(ptpc):
     """The page's naive path (GEMM -> fp32 intermediate -> scale) gives the
     same bits as the fused epilogue: same accumulator, same two products."""
