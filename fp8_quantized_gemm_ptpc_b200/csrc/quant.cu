@@ -80,9 +80,17 @@ __device__ __forceinline__ uint32_t quant_pair(uint32_t w, const GroupScale &g) 
 //   q0 = RN((-x) * (-r)) = RN(x * r),  e = RN(q0 * s + (-x)),  q = RN(e * (-r) + q0)
 // (the residual form that keeps -0 as -0).  Returns the two E4M3 codes,
 // first element in the low byte.
+__device__ __forceinline__ uint32_t quant_nx2_fast(uint32_t nlo, uint32_t nhi, uint64_t s2, uint64_t nr2);
+
 __device__ __forceinline__ uint32_t quant_pair_fast(uint32_t w, uint64_t s2, uint64_t nr2) {
   const uint32_t nlo = (w << 16) ^ 0x80000000u;       // -x of the first element
   const uint32_t nhi = (w & 0xFFFF0000u) ^ 0x80000000u;  // -x of the second element
+  return quant_nx2_fast(nlo, nhi, s2, nr2);
+}
+
+// The fast-path arithmetic of quant_pair_fast on two elements given as the
+// fp32 bits of their negations (first element -> low byte of the result).
+__device__ __forceinline__ uint32_t quant_nx2_fast(uint32_t nlo, uint32_t nhi, uint64_t s2, uint64_t nr2) {
   uint64_t nx2, q0, e, q;
   asm("mov.b64 %0, {%1, %2};" : "=l"(nx2) : "r"(nlo), "r"(nhi));
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(q0) : "l"(nx2), "l"(nr2));
@@ -403,7 +411,18 @@ __global__ void __launch_bounds__(256) quant_weight_t_kernel(const uint4 *__rest
     g.r = rc[c];
     g.mode = __float_as_uint(rc[c]) == 0u ? kZeroGroup : (sc[c] >= kFastPathMinScale ? kFast : kSlow);
     uint32_t word = 0;
-    if (g.mode != kZeroGroup) {
+    if (g.mode == kFast) {
+      // rows (0, 1) and (2, 3) of the column as packed pairs, the same IEEE
+      // steps as the activation quantiser's fast path
+      const uint64_t s2 = pack2(g.s), nr2 = pack2(-g.r);
+      uint32_t nx[4];
+      #pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const uint32_t w2 = (c < 2) ? v[r].x : (c < 4) ? v[r].y : (c < 6) ? v[r].z : v[r].w;
+        nx[r] = ((c & 1) ? (w2 & 0xFFFF0000u) : (w2 << 16)) ^ 0x80000000u;
+      }
+      word = quant_nx2_fast(nx[0], nx[1], s2, nr2) | (quant_nx2_fast(nx[2], nx[3], s2, nr2) << 16);
+    } else if (g.mode == kSlow) {
       float q[4];
       #pragma unroll
       for (int r = 0; r < 4; ++r) {
