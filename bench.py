@@ -7,14 +7,19 @@ batch of synthetic activations already resident in HBM: per layer, the
 per-token activation quantiser and the fused row-wise-scaled FP8 GEMM,
 through the library's fused entry point ``ptpc_linear`` (weights are
 quantised per output channel once, before timing, as at model load).  The
-default workload is Llama-3.1-8B prefill at T = 2048 (QKV 4096->6144,
-gate+up 4096->28672, down 14336->4096).
+default workload is the largest single-GPU configuration, Llama-3.1-70B
+prefill at T = 8192 (fused gate+up 8192->57344, down 28672->8192).
 
 Prints one JSON line (rank 0).  ``value`` is whole-job TFLOP/s
 (2 * T * Ci * Co summed over layers and ranks / the slowest rank's device
-time).  With N > 1 every rank runs an independent replica of the workload
-(weak scaling, no data-path collective).  ``--impl reference`` times the CPU
-oracle on a bounded row sample of the same workload instead.
+time).  The same line carries the GEMM's roofline record, the activation
+quantiser inside the step and alone, the weight quantiser, the page's
+comparison paths, the end-to-end figure through pinned host memory, the
+decode regime (70B up/down at T = 1, 8, 32, 128), a short ragged-T chain
+summary and the CPU oracle's throughput on a row sample.  With N > 1 every
+rank runs an independent replica of the workload (weak scaling, no data-path
+collective).  ``--impl reference`` times the CPU oracle on a bounded row
+sample of the same workload instead.
 """
 from __future__ import annotations
 
@@ -49,13 +54,13 @@ L2_BYTES = 126 * 1024 * 1024
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="llama8b_prefill", choices=sorted(WORKLOADS))
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama70b_prefill", choices=sorted(WORKLOADS))
     ap.add_argument("--tokens", type=int, default=None, help="override T (default: the workload's first)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip comparison paths, e2e and CPU baseline")
-    ap.add_argument("--cpu-rows", type=int, default=0,
+    ap.add_argument("--cpu-rows", type=int, default=512,
                     help="token rows per layer in the CPU-oracle sample (0: all T rows)")
     ap.add_argument("--cpu-steps", type=int, default=2, help="steps in the CPU-oracle sample")
     ap.add_argument("--quant-only", action="store_true",
@@ -63,6 +68,10 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="70B 4-linear chain: fused vs naive two-step vs per-tensor, one JSON line per T")
     ap.add_argument("--sweep-tokens", default=None, help="comma-separated T values for --sweep")
+    ap.add_argument("--chain-tokens", default="1,256,3001",
+                    help="T values of the chain summary inside the default line ('' to skip)")
+    ap.add_argument("--decode-tokens", default="1,8,32,128",
+                    help="T values of the decode record inside the default line ('' to skip)")
     return ap.parse_args()
 
 
@@ -185,32 +194,60 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- reference (CPU oracle) arm
 
-def cpu_oracle_sample(wl, layers, rows_per_layer, steps):
-    """Times the oracle (as it stands) on `rows_per_layer` token rows of every
-    layer: per-token quantisation of those rows and the fp64 scaled GEMM
-    against the full weight.  Returns (TFLOP/s, seconds, threads, note)."""
-    import oracle
-    prep = []
-    for i, name, T, Ci, Co in layers:
-        r = min(rows_per_layer, T)
-        X = synthetic.make_x(wl, i, r, Ci)
-        W = synthetic.make_w(wl, i, Ci, Co)
-        Wq_t, ws = oracle.quant_weight(W)
-        prep.append((X, Wq_t, ws, r, Ci, Co))
-    flops = sum(2.0 * r * Ci * Co for _, _, _, r, Ci, Co in prep)
-    t0 = time.perf_counter()
-    for _ in range(steps):
-        for X, Wq_t, ws, r, Ci, Co in prep:
-            oracle.linear_reference(X, Wq_t, ws)
-    dt = time.perf_counter() - t0
+def sample_rows(T, n, seed=0):
+    """Token rows of the CPU-oracle sample: all T rows if n >= T; otherwise
+    the first and last row, both rows at every 128-row tile boundary, and a
+    seeded uniform draw up to n rows in all, sorted."""
+    if n <= 0 or n >= T:
+        return np.arange(T)
+    fixed = {0, T - 1}
+    for b in range(128, T, 128):
+        fixed.update((b - 1, b))
+    fixed = sorted(fixed)
+    if len(fixed) >= n:
+        pick = np.linspace(0, len(fixed) - 1, n).round().astype(int)
+        return np.unique(np.asarray(fixed)[pick])
+    rng = np.random.Generator(np.random.PCG64(seed))
+    rest = np.setdiff1d(np.arange(T), fixed)
+    extra = rng.choice(rest, size=n - len(fixed), replace=False)
+    return np.sort(np.concatenate([fixed, extra]))
+
+
+def cpu_threads():
     try:
         from threadpoolctl import threadpool_info
-        threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [os.cpu_count() or 1])
+        return max([d.get("num_threads", 1) for d in threadpool_info()] + [os.cpu_count() or 1])
     except Exception:
-        threads = os.cpu_count() or 1
-    note = (f"{rows_per_layer} token rows per layer x {len(prep)} layers x {steps} steps "
-            f"(oracle per-token quantisation + fp64 GEMM against the full weight)")
-    return flops * steps / dt / 1e12, dt, threads, note
+        return os.cpu_count() or 1
+
+
+def cpu_oracle_sample(wl, layers, rows_per_layer, steps, W_bits=None):
+    """Times the oracle (as it stands) on a sample of token rows of every
+    layer (sample_rows: first/last, every 128-row tile boundary, seeded
+    draw): per-token quantisation of those rows and the fp64 scaled GEMM
+    against the full weight, which the oracle quantises beforehand (not
+    timed).  W_bits optionally passes the layers' bf16 weights already drawn.
+    Returns (TFLOP/s, seconds, threads, note)."""
+    import oracle
+    prep = []
+    for j, (i, name, T, Ci, Co) in enumerate(layers):
+        rows = sample_rows(T, rows_per_layer, seed=10 + i)
+        X = synthetic.make_x(wl, i, T, Ci)[rows]
+        W = W_bits[j] if W_bits is not None else synthetic.make_w(wl, i, Ci, Co)
+        Wq_t, ws = oracle.quant_weight(W)
+        prep.append((np.ascontiguousarray(X), Wq_t, ws, len(rows), T, Ci, Co))
+    flops = sum(2.0 * r * Ci * Co for _, _, _, r, _, Ci, Co in prep)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        for X, Wq_t, ws, r, T, Ci, Co in prep:
+            oracle.linear_reference(X, Wq_t, ws)
+    dt = time.perf_counter() - t0
+    sampled = all(r < T for _, _, _, r, T, _, _ in prep)
+    note = (f"{prep[0][3]} of {prep[0][4]} token rows per layer (first/last, every 128-row tile boundary, seeded "
+            f"draw) x {len(prep)} layers x {steps} steps: oracle per-token quantisation + fp64 GEMM against the "
+            f"full weight; TFLOP/s of the sample"
+            + ("; the oracle's time for a whole step is extrapolated from it (per row x T)" if sampled else ""))
+    return flops * steps / dt / 1e12, dt, cpu_threads(), note
 
 
 def run_reference(args):
@@ -221,13 +258,18 @@ def run_reference(args):
     T = args.tokens or wl.tokens[0]
     layers = workload_layers(wl, T)
     rows = T if args.cpu_rows <= 0 else max(1, min(args.cpu_rows, T))
-    for _ in range(max(0, min(args.warmup, 1))):
-        cpu_oracle_sample(wl, layers, rows, 1)
+    W_bits = [synthetic.make_w(wl, i, Ci, Co) for i, _, _, Ci, Co in layers]
+    if args.warmup > 0:
+        cpu_oracle_sample(wl, layers, min(rows, 16), 1, W_bits)
     steps = max(1, min(args.steps, 3))
-    tflops, dt, threads, note = cpu_oracle_sample(wl, layers, rows, steps)
+    tflops, dt, threads, note = cpu_oracle_sample(wl, layers, rows, steps, W_bits)
+    flops = layer_flops(layers)
     line = {
         "impl": "reference", "metric": METRIC, "value": tflops, "unit": "TFLOP/s",
-        "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup, "ms_per_step": dt / steps * 1e3,
+        "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": flops / (tflops * 1e12) * 1e3,
+        "ms_per_step_note": "whole step of the workload at the sample's rate (extrapolated per row x T)"
+                            if rows < T else "measured",
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(wl, layers, "CPU run"),
         "cpu_baseline": {"value": tflops, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": note},
@@ -262,6 +304,107 @@ def kernel_src_hash():
     return h.hexdigest()
 
 
+def decode_record(ptpc, dev, peaks, tokens, steps):
+    """The decode regime on its own: the 70B up (8192 -> 28672) and down
+    (28672 -> 8192) layers through ptpc_linear at small T, weights quantised
+    once.  Each layer's weight (235 MB of codes) is larger than L2, and the two
+    alternate, so every weight byte comes from HBM on every call.  Reports
+    the step time, the GEMM launches against the HBM roofline (algorithmic
+    bytes: weight codes, activation codes, output, scales), the K split each
+    layer runs with, and the host time per call (library and binding)."""
+    import ctypes
+
+    import torch
+    wl = synthetic.DECODE_70B
+    stream = torch.cuda.current_stream(dev)
+    Ls = []
+    for i, L in enumerate(wl.layers):
+        Wb = torch.from_numpy(synthetic.make_w(wl, i, L.Ci, L.Co).view(np.int16)).to(dev).view(torch.bfloat16)
+        Wq, ws = ptpc.quantize_weights(Wb)
+        del Wb
+        Ls.append((L, Wq, ws))
+    out = {}
+    for T in tokens:
+        Xs = [torch.from_numpy(synthetic.make_x(wl, i, T, L.Ci).view(np.int16)).to(dev).view(torch.bfloat16)
+              for i, (L, _, _) in enumerate(Ls)]
+        outs = [torch.empty((T, L.Co), dtype=torch.bfloat16, device=dev) for L, _, _ in Ls]
+        wsps = [ptpc.Workspace(ptpc.workspace_size(ptpc.OP_LINEAR, T, L.Ci, L.Co), dev) for L, _, _ in Ls]
+        q = [(torch.empty((T, L.Ci), dtype=torch.uint8, device=dev), torch.empty((T,), dtype=torch.float32, device=dev))
+             for L, _, _ in Ls]
+
+        def step():
+            for j, (L, Wq, ws) in enumerate(Ls):
+                ptpc.linear(Xs[j], Wq, ws, out=outs[j], ws=wsps[j])
+
+        for _ in range(3):
+            step()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_step = e0.elapsed_time(e1) / steps
+        # per launch: events around the quantiser and the GEMM of every layer
+        ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in Ls] for _ in range(steps)]
+        for it in range(steps):
+            for j, (L, Wq, ws) in enumerate(Ls):
+                ev[it][j][0].record(stream)
+                ptpc.quantize_activations(Xs[j], *q[j])
+                ev[it][j][1].record(stream)
+                ptpc.scaled_mm(q[j][0], q[j][1], Wq, ws, out=outs[j], ws=wsps[j])
+                ev[it][j][2].record(stream)
+        torch.cuda.synchronize(dev)
+        g_ms = [sum(ev[it][j][1].elapsed_time(ev[it][j][2]) for it in range(steps)) / steps for j in range(len(Ls))]
+        q_ms = [sum(ev[it][j][0].elapsed_time(ev[it][j][1]) for it in range(steps)) / steps for j in range(len(Ls))]
+        g_bytes = [gemm_bytes(T, L.Ci, L.Co) for L, _, _ in Ls]
+        g_gbs = sum(g_bytes) / (sum(g_ms) / 1e3) / 1e9
+        step_bytes = sum(g_bytes) + sum(quant_bytes(T, L.Ci) for L, _, _ in Ls)
+        # host time per call: the C ABI through ctypes with arguments marshalled
+        # once, and the Python binding (argument checks, stream lookup); the
+        # GPU stays busy, so these are enqueue costs
+        L0, Wq0, ws0 = Ls[0]
+        P = ctypes.c_void_p
+        args = (P(Xs[0].data_ptr()), L0.Ci, P(Wq0.data_ptr()), P(ws0.data_ptr()), T, L0.Ci, L0.Co,
+                P(outs[0].data_ptr()), wsps[0].ptr(), wsps[0].nbytes, P(stream.cuda_stream))
+        n_calls = 100
+        h0, m0 = ptpc.map_cache_stats()
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        for _ in range(n_calls):
+            ptpc.lib.ptpc_linear(*args)
+        t1 = time.perf_counter()
+        torch.cuda.synchronize(dev)
+        t2 = time.perf_counter()
+        for _ in range(n_calls):
+            ptpc.linear(Xs[0], Wq0, ws0, out=outs[0], ws=wsps[0])
+        t3 = time.perf_counter()
+        torch.cuda.synchronize(dev)
+        h1, m1 = ptpc.map_cache_stats()
+        out[str(T)] = {
+            "ms_per_step": ms_step, "layers": [f"{L.name} {L.Ci}->{L.Co}" for L, _, _ in Ls],
+            "gemm_ms": {L.name: g for (L, _, _), g in zip(Ls, g_ms)},
+            "quant_ms": {L.name: x for (L, _, _), x in zip(Ls, q_ms)},
+            "ksplit": {L.name: ptpc.gemm_ksplit(T, L.Ci, L.Co) for L, _, _ in Ls},
+            "roofline": {"bound": "hbm", "achieved": g_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": g_gbs / peaks["hbm_gbs"], "algorithmic_bytes": sum(g_bytes),
+                         "peak_src": f"{peaks['src']} HBM copy"},
+            "step_gbs": step_bytes / (ms_step / 1e3) / 1e9,
+            "step_frac_of_hbm": step_bytes / (ms_step / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "host_us_per_call_abi": (t1 - t0) / n_calls * 1e6,
+            "host_us_per_call_binding": (t3 - t2) / n_calls * 1e6,
+            "tensor_map_cache": {"hits": h1 - h0, "misses": m1 - m0},
+        }
+        del Xs, outs, wsps, q, ev
+    del Ls
+    torch.cuda.empty_cache()
+    return {"workload": wl.name, "steps": steps,
+            "l2": "each layer's weight (235 MB of codes) exceeds the 126 MB L2 and the layers alternate: "
+                  "weights stream from HBM on every call",
+            "per_T": out}
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -285,15 +428,21 @@ def run_gpu(args):
     peaks = load_peaks()
     fp8_peak = 2.0 * peaks["bf16_tflops"]                 # nominal fp8:bf16 ratio 2
     fp8_peak_sus = 2.0 * peaks["bf16_tflops_sustained"]
+    cpu_baseline_here = rank == 0 and world == 1 and not args.no_extras
 
     def to_dev(bits):
         return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
 
     # inputs, resident in HBM; weights quantised once (model load)
     L = []
+    W_bits = []
     for i, name, T_, Ci, Co in layers:
         X = to_dev(synthetic.make_x(wl, i, T_, Ci))
-        Wb = to_dev(synthetic.make_w(wl, i, Ci, Co))
+        wb = synthetic.make_w(wl, i, Ci, Co)
+        if cpu_baseline_here:
+            W_bits.append(wb)
+        Wb = to_dev(wb)
+        del wb
         Wq_t, w_scale = ptpc.quantize_weights(Wb)
         Wq_pt, ws_pt = ptpc.quantize_weights_per_tensor(Wb)
         out = torch.empty((T_, Co), dtype=torch.bfloat16, device=dev)
@@ -385,7 +534,6 @@ def run_gpu(args):
         "dtype": "e4m3 x e4m3 -> f32 accumulate, bf16 out", "data": "synthetic",
         "config": dict(config_of(wl, layers, l2_note), parallelism=f"replicas x{world}" if world > 1 else "1 GPU"),
         "frac_of_fp8_peak": value / world / fp8_peak,
-        "frac_of_fp8_peak_sustained": value / world / fp8_peak_sus,
         "clocks": clk.summary() | {"sm_mhz_device": probe_mhz,
                                    "sm_mhz_device_src": "median over 1 ms intervals of clock64 / globaltimer on "
                                                         "one SM, during a repeat of the timed loop",
@@ -396,28 +544,46 @@ def run_gpu(args):
             "frac": gemm_gbs / peaks["hbm_gbs"], "traffic": dram,
             "peak_src": f"{peaks['src']} HBM copy",
         } if hbm_bound else {
-            # timed inside a long step (after the timed loop and its repeat, at the clock the
-            # power cap leaves), so the sustained figure is the denominator; burst beside it
-            "bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak_sus, "unit": "TFLOP/s",
-            "frac": gemm_tflops / fp8_peak_sus, "traffic": dram,
-            "peak_src": f"{peaks['src']} bf16 sustained x 2 (fp8:bf16 nominal ratio); kernel timed inside "
-                        "a long step",
-            "burst_peak": fp8_peak, "frac_of_burst": gemm_tflops / fp8_peak,
+            # the timed loop lasts milliseconds, not seconds: the burst FP8
+            # figure is the denominator; the sustained one is reported beside it
+            "bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+            "frac": gemm_tflops / fp8_peak, "traffic": dram,
+            "peak_src": f"{peaks['src']} bf16 burst x 2 (fp8:bf16 nominal ratio 4.5 : 2.25 PFLOP/s)",
+            "sustained_peak": fp8_peak_sus, "frac_of_sustained": gemm_tflops / fp8_peak_sus,
         }) | {
             "kernel": "ptpc scaled GEMM (fused epilogue), all layers of one step",
             "traffic_unit": "bytes per step (dram__bytes_read.sum + dram__bytes_write.sum over the step's GEMM launches)",
             "algorithmic_flops_per_step": flops, "algorithmic_bytes_per_step": g_bytes,
             "gemm_tflops": gemm_tflops, "gemm_gbs": gemm_gbs,
             "per_layer_ms": {d["name"]: g for d, g in zip(L, g_ms)},
+            "sm_mhz_device": probe_mhz,
         },
         "quant": {
             "value": q_gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"], "frac": q_gbs / peaks["hbm_gbs"],
             "bytes_per_step": q_bytes, "per_layer_ms": {d["name"]: q for d, q in zip(L, q_ms)},
             "peak_src": f"{peaks['src']} HBM copy",
             "note": "inside the step: each launch timed by events between the GEMMs (launch gap included), "
-                    "at the clock the GEMMs' power draw leaves; the quantiser alone on inputs larger than L2: "
-                    "bench.py --quant-only --workload llama70b_prefill",
+                    "at the clock the GEMMs' power draw leaves",
         },
+    }
+
+    # ---- the activation quantiser alone on the same inputs (no GEMM in
+    # between; every input is larger than L2, so each pass reads X from HBM)
+    Kq = max(10, min(4 * K, 200))
+    qfn = lambda: [ptpc.quantize_activations(d["X"], *bufs[j]) for j, d in enumerate(L)]
+    for _ in range(3):
+        qfn()
+    ms_q = max_over_ranks(timed(qfn, Kq)) / Kq
+    qprobe = ptpc.ClockProbe(dev)
+    timed(qfn, Kq, before=lambda: qprobe.start(ms_q * Kq * 1.05 / 1e3))
+    q_alone = q_bytes / (ms_q / 1e3) / 1e9
+    line["quant_isolated"] = {
+        "value": q_alone, "unit": "GB/s", "achieved": q_alone, "peak": peaks["hbm_gbs"],
+        "frac": q_alone / peaks["hbm_gbs"], "bytes_per_pass": q_bytes, "ms_per_pass": ms_q, "passes": Kq,
+        "inputs": [[d["T"], d["Ci"]] for d in L], "sm_mhz_device": qprobe.mhz(),
+        "peak_src": f"{peaks['src']} HBM copy",
+        "note": "ptpc_quantize_activations alone, every layer input of the step in turn, back to back; "
+                "algorithmic bytes 3 per element + 4 per row",
     }
 
     # ---- per-output-channel weight quantiser (run once per weight at load time)
@@ -472,6 +638,10 @@ def run_gpu(args):
             "ptpc_over_per_tensor_throughput": ms_pt / (ms / K),
         }
         del ys
+        for d in L:
+            d.pop("Wq_pt")
+            d.pop("ws_pt")
+        torch.cuda.empty_cache()
 
         # ---- end to end through the public API: pinned host in, pinned host out.
         # Every step copies each layer's input host -> device, runs ptpc.linear
@@ -546,12 +716,36 @@ def run_gpu(args):
             "ms_per_step": ms_e2e,
             "pipelining": "per-direction copy streams, two device buffer sets",
         }
+        del hx, ho, dx, dout
 
-        if rank == 0 and world == 1:
+    # the step's own buffers are no longer needed
+    del L, bufs, evs
+    torch.cuda.empty_cache()
+
+    if not args.no_extras:
+        # ---- the decode regime and a short ragged-T chain summary
+        dec_tokens = [int(t) for t in args.decode_tokens.split(",") if t.strip()]
+        if dec_tokens:
+            line["decode"] = decode_record(ptpc, dev, peaks, dec_tokens, steps=max(20, min(K * 2, 100)))
+        chain_tokens = [int(t) for t in args.chain_tokens.split(",") if t.strip()]
+        if chain_tokens:
+            Ws = chain_weights(ptpc, dev)
+            line["chain"] = {
+                "workload": synthetic.CHAIN_70B.name + ": qkv 8192->10240, o 8192->8192, gate_up 8192->57344, "
+                                                       "down 28672->8192, dynamic re-quantisation between layers",
+                "per_T": [chain_measure(ptpc, dev, Ws, t, peaks, graph=False) for t in chain_tokens],
+                "roofline_note": "roofline_ms = max(algorithmic FLOPs / burst FP8 peak, algorithmic bytes of "
+                                 "quantisers and GEMMs / HBM copy bandwidth)",
+            }
+            del Ws
+            torch.cuda.empty_cache()
+
+        if cpu_baseline_here:
             rows = T if args.cpu_rows <= 0 else max(1, min(args.cpu_rows, T))
-            tf, dt, threads, note = cpu_oracle_sample(wl, layers, rows, max(1, args.cpu_steps))
+            tf, dt, threads, note = cpu_oracle_sample(wl, layers, rows, max(1, args.cpu_steps), W_bits)
             line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                                     "sample": note, "seconds": dt}
+    del W_bits
 
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -608,98 +802,125 @@ def run_quant_only(args):
     return 0
 
 
-def run_sweep(args):
-    """The 70B-shaped chain QKV -> O -> gate+up -> down with dynamic per-token
+def chain_weights(ptpc, dev):
+    """The 70B chain's four weights, quantised per output channel and per
+    tensor: [(Layer, (Wq_t, w_scale), (Wq_t_pt, w_scale_pt))]."""
+    import torch
+    wl = synthetic.CHAIN_70B
+    Ws = []
+    for i, L in enumerate(wl.layers):
+        Wb = torch.from_numpy(synthetic.make_w(wl, i, L.Ci, L.Co).view(np.int16)).to(dev).view(torch.bfloat16)
+        Ws.append((L, ptpc.quantize_weights(Wb), ptpc.quantize_weights_per_tensor(Wb)))
+        del Wb
+    return Ws
+
+
+def chain_roofline_ms(T, layers, peaks):
+    """Roofline time of one chain pass: the slower of its algorithmic FP8
+    FLOPs at the burst FP8 peak and its algorithmic bytes (quantiser + GEMM of
+    every layer) at the HBM copy bandwidth."""
+    flops = sum(2.0 * T * L.Ci * L.Co for L in layers)
+    nbytes = sum(quant_bytes(T, L.Ci) + gemm_bytes(T, L.Ci, L.Co) for L in layers)
+    return max(flops / (2.0 * peaks["bf16_tflops"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9)) * 1e3
+
+
+def chain_measure(ptpc, dev, Ws, T, peaks, graph=True, K=None):
+    """One T of the chain QKV -> O -> gate+up -> down with dynamic per-token
     re-quantisation between layers: O reads QKV output columns [0, 8192) and
     down reads gate+up output columns [0, 28672) (column slices, no copies).
-    Three paths are timed side by side for every T: the fused PTPC entry
-    point, the page's naive two-step path (unscaled fp32 GEMM, then a scaling
-    kernel) and per-tensor scaling."""
+    The fused PTPC entry point, the page's naive two-step path (unscaled fp32
+    GEMM, then a scaling kernel) and per-tensor scaling are timed side by side
+    (CUDA events on the launch stream, after 3 warm-up passes)."""
+    import torch
+    wl = synthetic.CHAIN_70B
+    stream = torch.cuda.current_stream(dev)
+    flops_tok = sum(2.0 * L.Ci * L.Co for L, _, _ in Ws)
+    X0 = torch.from_numpy(synthetic.make_x(wl, 0, T, wl.layers[0].Ci).view(np.int16)).to(dev).view(torch.bfloat16)
+    outs = [torch.empty((T, L.Co), dtype=torch.bfloat16, device=dev) for L, _, _ in Ws]
+    wsps = [ptpc.Workspace(ptpc.workspace_size(ptpc.OP_LINEAR, T, L.Ci, L.Co), dev) for L, _, _ in Ws]
+    ys = [torch.empty((T, L.Co), dtype=torch.float32, device=dev) for L, _, _ in Ws]
+    qs = [(torch.empty((T, L.Ci), dtype=torch.uint8, device=dev), torch.empty((T,), dtype=torch.float32, device=dev))
+          for L, _, _ in Ws]
+    pts = [ptpc.Workspace(ptpc.workspace_size(ptpc.OP_BENCH_PER_TENSOR, T, L.Ci, 0), dev) for L, _, _ in Ws]
+
+    def layer_input(i):
+        return X0 if i == 0 else outs[i - 1][:, :Ws[i][0].Ci]
+
+    def fused():
+        for i, (L, (Wq, ws), _) in enumerate(Ws):
+            ptpc.linear(layer_input(i), Wq, ws, out=outs[i], ws=wsps[i])
+
+    def naive():
+        for i, (L, (Wq, ws), _) in enumerate(Ws):
+            Xq, xs = ptpc.quantize_activations(layer_input(i), *qs[i])
+            ptpc.unscaled_mm_f32(Xq, Wq, out=ys[i], ws=wsps[i])
+            ptpc.apply_scales(ys[i], xs, ws, out=outs[i])
+
+    def per_tensor():
+        for i, (L, _, (Wq, ws)) in enumerate(Ws):
+            Xq, xs = ptpc.quantize_activations_per_tensor(layer_input(i), *qs[i], ws=pts[i])
+            ptpc.scaled_mm(Xq, xs, Wq, ws, out=outs[i], ws=wsps[i])
+
+    paths = [("fused", fused), ("naive", naive), ("per_tensor", per_tensor)]
+    g = None
+    if graph:
+        # the fused chain captured once into a CUDA graph and replayed (the
+        # library only enqueues work on the current stream)
+        for _ in range(2):
+            fused()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        capture_stream = torch.cuda.Stream(dev)
+        with torch.cuda.stream(capture_stream):
+            with torch.cuda.graph(g, stream=capture_stream):
+                fused()
+        torch.cuda.synchronize(dev)
+        paths.insert(1, ("fused_graph", g.replay))
+
+    K = K or max(3, min(200, int(4e13 / (flops_tok * T))))
+    res = {}
+    for name, fn in paths:
+        for _ in range(3):
+            fn()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(K):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        res[name] = e0.elapsed_time(e1) / K
+    roof = chain_roofline_ms(T, [L for L, _, _ in Ws], peaks)
+    rec = {
+        "T": T, "steps": K, "fused_ms": res["fused"], "naive_ms": res["naive"], "per_tensor_ms": res["per_tensor"],
+        "fused_tflops": flops_tok * T / (res["fused"] / 1e3) / 1e12,
+        "roofline_ms": roof, "fused_frac_of_roofline": roof / res["fused"],
+        "fused_speedup_over_naive": res["naive"] / res["fused"],
+        "ptpc_over_per_tensor_throughput": res["per_tensor"] / res["fused"],
+    }
+    if graph:
+        rec["fused_graph_ms"] = res["fused_graph"]
+    del g, X0, outs, wsps, ys, qs, pts
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_sweep(args):
+    """Every T of the 70B chain (or --sweep-tokens), one JSON line each."""
     import torch
 
     import fp8_quantized_gemm_ptpc_b200 as ptpc
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
-    stream = torch.cuda.current_stream(dev)
     wl = synthetic.CHAIN_70B
     tokens = ([int(t) for t in args.sweep_tokens.split(",")] if args.sweep_tokens else list(wl.tokens))
     peaks = load_peaks()
-    Ws = []
-    for i, L in enumerate(wl.layers):
-        Wb = torch.from_numpy(synthetic.make_w(wl, i, L.Ci, L.Co).view(np.int16)).to(dev).view(torch.bfloat16)
-        Ws.append((L, ptpc.quantize_weights(Wb), ptpc.quantize_weights_per_tensor(Wb)))
-        del Wb
-    # chain inputs: layer l reads columns [0, Ci) of the previous layer's output
-    flops_tok = sum(2.0 * L.Ci * L.Co for L, _, _ in Ws)
+    Ws = chain_weights(ptpc, dev)
     for T in tokens:
-        X0 = torch.from_numpy(synthetic.make_x(wl, 0, T, wl.layers[0].Ci).view(np.int16)).to(dev).view(torch.bfloat16)
-        outs = [torch.empty((T, L.Co), dtype=torch.bfloat16, device=dev) for L, _, _ in Ws]
-        wsps = [ptpc.Workspace(ptpc.workspace_size(ptpc.OP_LINEAR, T, L.Ci, L.Co), dev) for L, _, _ in Ws]
-        ys = [torch.empty((T, L.Co), dtype=torch.float32, device=dev) for L, _, _ in Ws]
-        qs = [(torch.empty((T, L.Ci), dtype=torch.uint8, device=dev), torch.empty((T,), dtype=torch.float32, device=dev))
-              for L, _, _ in Ws]
-        pts = [ptpc.Workspace(ptpc.workspace_size(ptpc.OP_BENCH_PER_TENSOR, T, L.Ci, 0), dev) for L, _, _ in Ws]
-
-        def layer_input(i):
-            return X0 if i == 0 else outs[i - 1][:, :Ws[i][0].Ci]
-
-        def fused():
-            for i, (L, (Wq, ws), _) in enumerate(Ws):
-                ptpc.linear(layer_input(i), Wq, ws, out=outs[i], ws=wsps[i])
-
-        def naive():
-            for i, (L, (Wq, ws), _) in enumerate(Ws):
-                Xq, xs = ptpc.quantize_activations(layer_input(i), *qs[i])
-                ptpc.unscaled_mm_f32(Xq, Wq, out=ys[i], ws=wsps[i])
-                ptpc.apply_scales(ys[i], xs, ws, out=outs[i])
-
-        def per_tensor():
-            for i, (L, _, (Wq, ws)) in enumerate(Ws):
-                Xq, xs = ptpc.quantize_activations_per_tensor(layer_input(i), *qs[i], ws=pts[i])
-                ptpc.scaled_mm(Xq, xs, Wq, ws, out=outs[i], ws=wsps[i])
-
-        # the fused chain captured once into a CUDA graph and replayed (the
-        # library only enqueues work on the current stream)
-        for _ in range(2):
-            fused()
-        torch.cuda.synchronize(dev)
-        graph = torch.cuda.CUDAGraph()
-        capture_stream = torch.cuda.Stream(dev)
-        with torch.cuda.stream(capture_stream):
-            with torch.cuda.graph(graph, stream=capture_stream):
-                fused()
-        torch.cuda.synchronize(dev)
-
-        def fused_graph():
-            graph.replay()
-
-        K = max(3, min(200, int(4e13 / (flops_tok * T))))
-        res = {}
-        for name, fn in (("fused", fused), ("fused_graph", fused_graph), ("naive", naive),
-                         ("per_tensor", per_tensor)):
-            for _ in range(3):
-                fn()
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            torch.cuda.synchronize(dev)
-            e0.record(stream)
-            for _ in range(K):
-                fn()
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            res[name] = e0.elapsed_time(e1) / K
-        print(json.dumps({
-            "kind": "chain_sweep", "workload": wl.name, "T": T, "steps": K,
-            "fused_ms": res["fused"], "fused_graph_ms": res["fused_graph"], "naive_ms": res["naive"],
-            "per_tensor_ms": res["per_tensor"],
-            "fused_tflops": flops_tok * T / (res["fused"] / 1e3) / 1e12,
-            "fused_frac_of_fp8_peak": flops_tok * T / (res["fused"] / 1e3) / 1e12 / (2.0 * peaks["bf16_tflops"]),
-            "fused_speedup_over_naive": res["naive"] / res["fused"],
-            "ptpc_over_per_tensor_throughput": res["per_tensor"] / res["fused"],
-        }), flush=True)
-        del graph, X0, outs, wsps, ys, qs, pts
-        torch.cuda.empty_cache()
+        rec = chain_measure(ptpc, dev, Ws, T, peaks)
+        print(json.dumps({"kind": "chain_sweep", "workload": wl.name} | rec), flush=True)
     return 0
 
 

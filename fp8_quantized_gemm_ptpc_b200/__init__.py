@@ -55,6 +55,9 @@ SIGNATURES = {
     "ptpc_gemm_ksplit": (ctypes.c_int, [_I64, _I64, _I64]),
     "ptpc_selftest_wait_timeout": (ctypes.c_int, [_P, _P]),
     "ptpc_scaled_mm_static_scratch": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
+    "ptpc_static_scratch_status": (ctypes.c_int, [_P]),
+    "ptpc_reload_tuning_overrides": (ctypes.c_int, []),
+    "ptpc_bench_map_cache_stats": (ctypes.c_int, [_P, _P]),
     "ptpc_bench_unscaled_mm_f32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "ptpc_bench_apply_scales": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _P, _P]),
     "ptpc_bench_clock_probe": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_uint64, ctypes.c_uint64, _P, _P]),
@@ -140,7 +143,10 @@ class Workspace:
     """A zero-filled device buffer for the entry points that take (ws, ws_bytes).
 
     The library leaves its control words zero after every successful call, so
-    one buffer serves any number of calls (not concurrently on the GPU)."""
+    one buffer serves any number of calls that do not overlap on the GPU.  A
+    workspace belongs to one stream: the buffer is allocated (and zeroed) on
+    the stream that is current when it is created or grown, and the caller
+    must not use it on two streams at once."""
 
     def __init__(self, nbytes: int, device):
         self.device = torch.device(device)
@@ -151,6 +157,10 @@ class Workspace:
         return self.buf.numel()
 
     def ensure(self, nbytes: int) -> "Workspace":
+        """Grow to at least nbytes.  The old buffer goes back to PyTorch's
+        caching allocator, which hands it out again only to work ordered after
+        what is already queued on the stream it was allocated on, so a kernel
+        of that stream that still reads it is not overtaken."""
         if nbytes > self.nbytes:
             self.buf = torch.zeros(int(nbytes), dtype=torch.uint8, device=self.device)
         return self
@@ -164,12 +174,20 @@ _ws_cache: dict = {}
 
 
 def default_workspace(nbytes: int, device) -> Workspace:
-    """Per-device, per-thread cached workspace grown on demand."""
-    key = (torch.device(device), threading.get_ident())
+    """The cached workspace of (device, current stream), grown on demand.
+
+    Keyed by stream, not by host thread: calls on two streams get two
+    workspaces and never share the quantised activations or the status word
+    a ``linear`` call keeps there, while calls on one stream are ordered by
+    that stream, which is what makes sharing one buffer between them safe."""
+    dev = torch.device(device)
+    stream = torch.cuda.current_stream(dev)
+    key = (dev, stream.cuda_stream)
     with _ws_lock:
         ws = _ws_cache.get(key)
         if ws is None:
-            ws = _ws_cache[key] = Workspace(nbytes, device)
+            with torch.cuda.stream(stream):
+                ws = _ws_cache[key] = Workspace(nbytes, dev)
         return ws.ensure(nbytes)
 
 
@@ -244,7 +262,7 @@ def scaled_mm_static_scratch(Xq, x_scale, Wq_t, w_scale, out: torch.Tensor | Non
     workspace argument, nothing allocated by the library; ``out`` may be
     passed to avoid the output allocation here).  The array is 4 KiB per
     device, of which the GEMM uses its 256-byte status word; calls must not
-    overlap on the GPU."""
+    overlap on the GPU.  Timeouts are read with static_scratch_status()."""
     _need(Xq, "Xq", torch.uint8, 2)
     _need(Wq_t, "Wq_t", torch.uint8, 2)
     _need(x_scale, "x_scale", torch.float32, 1)
@@ -258,6 +276,26 @@ def scaled_mm_static_scratch(Xq, x_scale, Wq_t, w_scale, out: torch.Tensor | Non
            lib.ptpc_scaled_mm_static_scratch(_ptr(Xq), _ptr(x_scale), _ptr(Wq_t), _ptr(w_scale), T, Ci, Co,
                                              _ptr(out), _stream(Xq.device)))
     return out
+
+
+def static_scratch_status() -> int:
+    """Synchronise the current stream and read/clear the status word of the
+    static scratch array (timeouts of scaled_mm_static_scratch since the last
+    read): OK or ERR_DEVICE_TIMEOUT."""
+    return int(lib.ptpc_static_scratch_status(_stream(torch.device("cuda", torch.cuda.current_device()))))
+
+
+def reload_tuning_overrides():
+    """Re-read PTPC_FORCE_KERNEL / PTPC_FORCE_PAIR_BN / PTPC_FORCE_KSPLIT from
+    the environment (the library reads them once otherwise; tuning only)."""
+    _check("ptpc_reload_tuning_overrides", lib.ptpc_reload_tuning_overrides())
+
+
+def map_cache_stats():
+    """(hits, misses) of the library's host-side tensor-map cache."""
+    h, m = ctypes.c_uint64(0), ctypes.c_uint64(0)
+    _check("ptpc_bench_map_cache_stats", lib.ptpc_bench_map_cache_stats(ctypes.byref(h), ctypes.byref(m)))
+    return int(h.value), int(m.value)
 
 
 def selftest_wait_timeout(ws: Workspace):

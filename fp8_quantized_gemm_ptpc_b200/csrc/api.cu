@@ -187,6 +187,17 @@ int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co) {
   return ptpc::gemm_ksplit((int)T, (int)Ci, (int)Co);
 }
 
+int ptpc_reload_tuning_overrides(void) {
+  ptpc::reload_tuning();
+  return PTPC_OK;
+}
+
+int ptpc_bench_map_cache_stats(uint64_t *hits, uint64_t *misses) {
+  if (!hits || !misses) return PTPC_ERR_INVALID_ARG;
+  ptpc::map_cache_stats(hits, misses);
+  return PTPC_OK;
+}
+
 int ptpc_selftest_wait_timeout(void *ws, void *stream) {
   if (!ws) return PTPC_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return PTPC_ERR_MISALIGNED;
@@ -314,6 +325,8 @@ int static_scratch_address(uint8_t **out) {
 
 }  // namespace
 
+static_assert(kGemmWorkspace <= kStaticScratchBytes, "the GEMM's scratch must fit in the static array");
+
 extern "C" int ptpc_scaled_mm_static_scratch(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq_t,
                                              const float *w_scale, int64_t T, int64_t Ci, int64_t Co, void *out,
                                              void *stream) {
@@ -325,12 +338,19 @@ extern "C" int ptpc_scaled_mm_static_scratch(const uint8_t *Xq, const float *x_s
   if (!aligned16(Xq) || !aligned16(x_scale) || !aligned16(Wq_t) || !aligned16(w_scale) || !aligned16(out))
     return PTPC_ERR_MISALIGNED;
   if ((s = check_device()) != PTPC_OK) return s;
-  if (kGemmWorkspace > kStaticScratchBytes) return PTPC_ERR_WORKSPACE_TOO_SMALL;
   uint8_t *scratch = nullptr;
   if ((s = static_scratch_address(&scratch)) != PTPC_OK) return s;
-  cudaStream_t st = (cudaStream_t)stream;
-  // The array keeps the previous call's contents: the status word must start
-  // at zero.
-  if (cudaMemsetAsync(scratch, 0, kGemmWorkspace, st) != cudaSuccess) return PTPC_ERR_CUDA;
-  return run_gemm(Xq, x_scale, Wq_t, w_scale, T, Ci, Co, out, false, scratch, false, st);
+  // The GEMM only ORs timeout bits into the status word at the start of the
+  // array and needs nothing else to start at zero.  The word is not cleared
+  // here, so a timeout stays recorded until ptpc_static_scratch_status reads
+  // it (the array is zero when the library is loaded).
+  return run_gemm(Xq, x_scale, Wq_t, w_scale, T, Ci, Co, out, false, scratch, false, (cudaStream_t)stream);
+}
+
+extern "C" int ptpc_static_scratch_status(void *stream) {
+  int s = check_device();
+  if (s != PTPC_OK) return s;
+  uint8_t *scratch = nullptr;
+  if ((s = static_scratch_address(&scratch)) != PTPC_OK) return s;
+  return ptpc_get_device_status(scratch, stream);
 }

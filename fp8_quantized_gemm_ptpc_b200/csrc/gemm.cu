@@ -36,10 +36,12 @@
 // sets a bit in the device status word, and the CTA stops issuing work, lets
 // its own copies and MMAs drain, frees its tensor memory and exits.
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -765,16 +767,68 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-bool make_map_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
-                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+// What a 2-D tensor map encodes.  The encoding depends on nothing else (not
+// on the current device or context), so equal keys give identical maps.
+struct MapKey {
+  const void *base;
+  uint64_t inner, outer, row_bytes;
+  uint32_t box_inner, box_outer;
+  int dt, sw;
+  bool operator==(const MapKey &o) const {
+    return base == o.base && inner == o.inner && outer == o.outer && row_bytes == o.row_bytes &&
+           box_inner == o.box_inner && box_outer == o.box_outer && dt == o.dt && sw == o.sw;
+  }
+};
+
+struct MapKeyHash {
+  size_t operator()(const MapKey &k) const {
+    uint64_t h = reinterpret_cast<uintptr_t>(k.base);
+    for (uint64_t v : {k.inner, k.outer, k.row_bytes, (uint64_t)k.box_inner << 32 | k.box_outer,
+                       (uint64_t)k.dt << 8 | (uint64_t)k.sw})
+      h = (h ^ v) * 0x100000001B3ull + (h >> 29);
+    return (size_t)h;
+  }
+};
+
+// Encoded tensor maps, shared by every device and host thread.  Layers call
+// the GEMM with the same buffers again and again, so after the first call of
+// a layer its maps come from here instead of being encoded anew.  Bounded:
+// the cache is emptied when it reaches kMapCacheMax entries.
+constexpr size_t kMapCacheMax = 4096;
+std::mutex g_map_mu;
+std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_map_cache;
+std::atomic<uint64_t> g_map_hits{0}, g_map_misses{0};
+
+bool encode_map_2d(CUtensorMap *m, const MapKey &k) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint64_t dims[2] = {k.inner, k.outer};
+  cuuint64_t strides[1] = {k.row_bytes};
+  cuuint32_t box[2] = {k.box_inner, k.box_outer};
   cuuint32_t estr[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, (CUtensorMapDataType)k.dt, 2, const_cast<void *>(k.base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, (CUtensorMapSwizzle)k.sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+                 uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+  const MapKey k{base, inner, outer, row_bytes, box_inner, box_outer, (int)dt, (int)sw};
+  {
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    auto it = g_map_cache.find(k);
+    if (it != g_map_cache.end()) {
+      *m = it->second;
+      g_map_hits.fetch_add(1, std::memory_order_relaxed);
+      return true;
+    }
+  }
+  if (!encode_map_2d(m, k)) return false;
+  g_map_misses.fetch_add(1, std::memory_order_relaxed);
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  if (g_map_cache.size() >= kMapCacheMax) g_map_cache.clear();
+  g_map_cache.emplace(k, *m);
+  return true;
 }
 
 bool make_maps(const GemmProblem &pr, uint32_t b_rows, CUtensorMap *tmA, CUtensorMap *tmB, CUtensorMap *tmC) {
@@ -853,6 +907,7 @@ int max_clusters(Kernel kernel, int sms, int size, size_t smem) {
 
 const DeviceInfo &device_info() {
   static DeviceInfo info[64];
+  static std::atomic<bool> ready[64];
   static DeviceInfo fallback;
   static std::mutex mu;
   int dev = 0;
@@ -860,9 +915,10 @@ const DeviceInfo &device_info() {
     cudaGetLastError();
     return fallback;
   }
+  if (ready[dev].load(std::memory_order_acquire)) return info[dev];
   std::lock_guard<std::mutex> lock(mu);  // first use of a device may come from several host threads
   DeviceInfo &d = info[dev];
-  if (!d.ready) {
+  if (!ready[dev].load(std::memory_order_relaxed)) {
     int v = 0;
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) d.sms = v;
     cudaFuncSetAttribute(ptpc_gemm_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -884,6 +940,7 @@ const DeviceInfo &device_info() {
       d.dec_clusters[size] = std::min(a, b);
     }
     d.ready = true;
+    ready[dev].store(true, std::memory_order_release);
   }
   return d;
 }
@@ -908,14 +965,50 @@ struct Plan {
 // waves) against 68.1 us (256-wide, 2 waves of which the second is 8% full).
 constexpr double kPairN128Cost = 1.15;
 
-// Tuning overrides (not for production use): an integer environment
-// variable, or `fallback` when unset or not a number.
+// Tuning overrides (not for production use), from the environment:
+// PTPC_FORCE_KERNEL = pair | decode, PTPC_FORCE_PAIR_BN = 128 | 256,
+// PTPC_FORCE_KSPLIT = 1 | 2 | 4 | 8.  Read once, at the first GEMM call of
+// the process (or again by reload_tuning), not on every call.
+struct Tuning {
+  int kernel;   // 0 automatic, 1 pair, 2 decode
+  int pair_bn;  // 0 automatic, 128, 256
+  int ksplit;   // 0 automatic, 1, 2, 4, 8
+};
+
 int env_int(const char *name, int fallback) {
   const char *v = std::getenv(name);
   if (v == nullptr || *v == '\0') return fallback;
   char *end = nullptr;
   const long x = std::strtol(v, &end, 10);
   return (end != nullptr && *end == '\0') ? (int)x : fallback;
+}
+
+Tuning read_tuning() {
+  Tuning t{0, 0, 0};
+  const char *k = std::getenv("PTPC_FORCE_KERNEL");
+  if (k != nullptr && std::strcmp(k, "pair") == 0) t.kernel = 1;
+  if (k != nullptr && std::strcmp(k, "decode") == 0) t.kernel = 2;
+  const int bn = env_int("PTPC_FORCE_PAIR_BN", 0);
+  if (bn == 128 || bn == 256) t.pair_bn = bn;
+  const int ks = env_int("PTPC_FORCE_KSPLIT", 0);
+  if (ks == 1 || ks == 2 || ks == 4 || ks == 8) t.ksplit = ks;
+  return t;
+}
+
+// Packed as kernel | pair_bn / 128 << 2 | ksplit << 4, plus bit 8 once read.
+std::atomic<uint32_t> g_tuning{0};
+
+uint32_t pack_tuning(const Tuning &t) {
+  return 0x100u | (uint32_t)t.kernel | (uint32_t)(t.pair_bn / 128) << 2 | (uint32_t)t.ksplit << 4;
+}
+
+Tuning tuning() {
+  uint32_t v = g_tuning.load(std::memory_order_relaxed);
+  if ((v & 0x100u) == 0) {
+    v = pack_tuning(read_tuning());
+    g_tuning.store(v, std::memory_order_relaxed);
+  }
+  return Tuning{(int)(v & 3u), (int)((v >> 2) & 3u) * 128, (int)((v >> 4) & 15u)};
 }
 
 // Fewest K-blocks a CTA of a K-split cluster streams.
@@ -953,7 +1046,7 @@ Plan decode_plan(int T, int Ci, int Co, const DeviceInfo &d) {
     }
   }
   // PTPC_FORCE_KSPLIT = 1, 2, 4 or 8 (tuning only; ignored where infeasible)
-  const int forced = env_int("PTPC_FORCE_KSPLIT", 0);
+  const int forced = tuning().ksplit;
   if (forced == 1 || ((forced == 2 || forced == 4 || forced == 8) && feasible(forced))) pl.ksplit = forced;
   pl.ctas = pl.ksplit > 1 ? pl.num_tiles * pl.ksplit : std::max(1, std::min(pl.num_tiles, d.sms));
   return pl;
@@ -963,8 +1056,8 @@ Plan decode_plan(int T, int Ci, int Co, const DeviceInfo &d) {
 // the last partial wave but move more operand bytes per FLOP, so they are
 // taken only when they finish the waves sooner by a margin.
 int choose_pair_bn(int T, int Co, const DeviceInfo &d) {
-  const int forced = env_int("PTPC_FORCE_PAIR_BN", 0);  // 128 or 256 (tuning only)
-  if (forced == 128 || forced == 256) return forced;
+  const int forced = tuning().pair_bn;  // 128 or 256 (tuning only)
+  if (forced != 0) return forced;
   const long long m = (T + 2 * BM - 1) / (2 * BM);
   const long long w256 = (m * ((Co + 255) / 256) + d.pair_clusters - 1) / d.pair_clusters;
   const long long w128 = (m * ((Co + 127) / 128) + d.pair_clusters128 - 1) / d.pair_clusters128;
@@ -1002,11 +1095,11 @@ Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d) {
 // the decode kernel takes T <= 256 only).
 Plan make_plan(int T, int Ci, int Co) {
   const DeviceInfo &d = device_info();
-  const char *force = std::getenv("PTPC_FORCE_KERNEL");
-  if (force != nullptr && std::strcmp(force, "pair") == 0) return pair_plan(T, Ci, Co, d);
+  const int force = tuning().kernel;
+  if (force == 1) return pair_plan(T, Ci, Co, d);
   if (T <= kDecodeMaxT) {
     const Plan pl = decode_plan(T, Ci, Co, d);
-    if (force != nullptr && std::strcmp(force, "decode") == 0) return pl;
+    if (force == 2) return pl;
     if (T <= kDecodeWholeMaxT || pl.ksplit > 1) return pl;
   }
   return pair_plan(T, Ci, Co, d);
@@ -1058,6 +1151,13 @@ cudaError_t launch_pair(int grid, const CUtensorMap &tmA, const CUtensorMap &tmB
 }  // namespace
 
 int num_sms() { return device_info().sms; }
+
+void reload_tuning() { g_tuning.store(pack_tuning(read_tuning()), std::memory_order_relaxed); }
+
+void map_cache_stats(uint64_t *hits, uint64_t *misses) {
+  *hits = g_map_hits.load(std::memory_order_relaxed);
+  *misses = g_map_misses.load(std::memory_order_relaxed);
+}
 
 int gemm_ksplit(int T, int Ci, int Co) { return make_plan(T, Ci, Co).ksplit; }
 

@@ -40,4 +40,11 @@ int gemm_ksplit(int T, int Ci, int Co);
 
 int num_sms();
 
+// Re-reads the PTPC_FORCE_* tuning overrides from the environment (they are
+// otherwise read once, at the first GEMM call).
+void reload_tuning();
+
+// Tensor-map cache counters since the library was loaded.
+void map_cache_stats(uint64_t *hits, uint64_t *misses);
+
 }  // namespace ptpc

@@ -317,7 +317,3 @@ __device__ __forceinline__ void mma_commit_pair_mc(uint64_t *bar, uint16_t cta_m
 }
 
 }  // namespace ptpc
-
-namespace ptpc {
-
-}  // namespace ptpc

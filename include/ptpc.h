@@ -8,9 +8,8 @@
  * the weight W is Ci x Co (Co output channels); X gets one scale per token
  * (Delta_X[T x 1]) and W one scale per output column (Delta_W[1 x Co]).  The
  * GEMM applies token_scale[t] * channel_scale[o] inside its epilogue, before
- * the single store of the result (section "The challenge: two-step vs fused",
- * the fused `_scaled_mm(input, weight, scale_a=token_scales,
- * scale_b=channel_scales)`).
+ * the single store of the result (section "The challenge: two-step vs fused":
+ * the fused call that hands both scale vectors to the FP8 GEMM).
  *
  * Number formats (the page names none; these are this library's readings):
  *   - FP8 codes are OCP E4M3 ("e4m3fn", bias 7, max 448, no infinities).
@@ -22,7 +21,9 @@
  *
  * Conventions shared by every entry point:
  *   - Pointers named *_dev are device pointers; every buffer is owned by the
- *     caller.  The library never allocates or frees device memory.
+ *     caller.  Apart from the 4 KiB static scratch array that
+ *     ptpc_scaled_mm_static_scratch uses (held by every GPU that loads the
+ *     library), the library never allocates or frees device memory.
  *   - Layouts are dense row-major.  bf16 tensors are passed as raw 16-bit
  *     patterns (void*).
  *   - Alignment: every device pointer must be 16-byte aligned
@@ -32,7 +33,7 @@
  *     T, Ci, Co must each fit in 31 bits.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
  *     only enqueues work on it and returns; none synchronises, except
- *     ptpc_get_device_status.
+ *     ptpc_get_device_status and ptpc_static_scratch_status.
  *   - Errors: the return value is a ptpc_status.  All argument checks run
  *     before any launch; a failed check launches nothing.  A failed launch
  *     returns PTPC_ERR_CUDA.  No C++ exception crosses this boundary.
@@ -108,8 +109,8 @@ PTPC_API int ptpc_quantize_weights(const void *W_dev, int64_t Ci, int64_t Co,
                           uint8_t *Wq_t_dev, float *w_scale_dev,
                           void *ws_dev, size_t ws_bytes, void *stream);
 
-/* Fused row-wise-scaled FP8 GEMM (the page's fused `_scaled_mm` with
- * scale_a = token scales, scale_b = channel scales):
+/* Fused row-wise-scaled FP8 GEMM (the page's fused path: the token scales
+ * scale the rows of the product, the channel scales its columns):
  *   out[t][o] = bf16_RNE((sum_k dec(Xq[t][k]) * dec(Wq_t[o][k]) * x_scale[t]) * w_scale[o])
  *   Xq_dev      u8 [T, Ci], x_scale_dev fp32 [T]   (from ptpc_quantize_activations)
  *   Wq_t_dev    u8 [Co, Ci], w_scale_dev fp32 [Co] (from ptpc_quantize_weights)
@@ -127,8 +128,9 @@ PTPC_API int ptpc_scaled_mm(const uint8_t *Xq_dev, const float *x_scale_dev,
 
 /* Fused quantise + GEMM: ptpc_quantize_activations of X into the workspace,
  * then ptpc_scaled_mm, on one stream (the GEMM is launched as a programmatic
- * dependent of the quantiser).  The page's path with "no pre-quantization":
- * the bf16 activation goes in, the bf16 output comes out.
+ * dependent of the quantiser).  The page's dynamic path, in which activations
+ * are quantised on every call rather than ahead of time: the bf16 activation
+ * goes in, the bf16 output comes out.
  *   X_dev bf16 [T, Ci] with row pitch ldx (as for ptpc_quantize_activations);
  *   Wq_t_dev / w_scale_dev as for ptpc_scaled_mm;
  *   out_dev bf16 [T, Co];
@@ -166,6 +168,18 @@ PTPC_API const char *ptpc_status_string(int status);
  * invalid arguments, T == 0 or an unsupported device.  Launches nothing. */
 PTPC_API int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co);
 
+/* Re-reads the GEMM's tuning overrides from the environment.  They are
+ * otherwise read once, at the first GEMM call of the process, so that no call
+ * pays for environment lookups:
+ *   PTPC_FORCE_KERNEL  = pair | decode   which GEMM kernel runs a shape,
+ *   PTPC_FORCE_PAIR_BN = 128 | 256       tile width of the prefill kernel,
+ *   PTPC_FORCE_KSPLIT  = 1 | 2 | 4 | 8   CTAs per tile of the decode kernel.
+ * Each is honoured only where the forced choice is feasible for the shape;
+ * results stay within the GEMM's tolerance under every choice.  For tuning
+ * and tests, not for production.  Not thread-safe with concurrent GEMM calls
+ * that should see a consistent setting.  No counterpart on the page. */
+PTPC_API int ptpc_reload_tuning_overrides(void);
+
 /* ptpc_scaled_mm without a caller-provided workspace.  The page has no
  * counterpart: this exists for callers that cannot allocate device memory
  * when they call the GEMM (an engine that partitions all device memory at
@@ -175,30 +189,47 @@ PTPC_API int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co);
  *   Scratch: a file-scope 4 KiB device array inside the library, held by
  *   every GPU that loads the library until the process exits; the GEMM uses
  *   its first 256 bytes (the device status word).  Results are bit-identical
- *   to ptpc_scaled_mm's.  A GEMM whose scratch exceeded the array would be
- *   rejected with PTPC_ERR_WORKSPACE_TOO_SMALL.
+ *   to ptpc_scaled_mm's.  The GEMM's scratch fits the array for every shape
+ *   (checked when the library is compiled).
  *   The first call on a device looks up the array's device address once
  *   (cudaGetSymbolAddress; its failure returns PTPC_ERR_CUDA).
- *   Every call zeroes the status word with cudaMemsetAsync on
- *   `stream` and allocates nothing.  All calls share the one array: calls
- *   that overlap on the GPU (different streams, or different host threads)
- *   race on it and give wrong results. */
+ *   Nothing is allocated and nothing is cleared per call: the status word is
+ *   zero when the library is loaded, the GEMM only sets timeout bits in it,
+ *   and those stay set until ptpc_static_scratch_status reads and clears
+ *   them.  All calls share the one array: calls that overlap on the GPU
+ *   (different streams, or different host threads) race on it, and a timeout
+ *   of one of them cannot be told apart from the other's. */
 PTPC_API int ptpc_scaled_mm_static_scratch(const uint8_t *Xq_dev, const float *x_scale_dev,
                                            const uint8_t *Wq_t_dev, const float *w_scale_dev,
                                            int64_t T, int64_t Ci, int64_t Co, void *out_dev, void *stream);
+
+/* Device status of ptpc_scaled_mm_static_scratch on the current device: like
+ * ptpc_get_device_status, synchronises `stream`, reads the status word of the
+ * static scratch array, clears it and returns PTPC_OK or
+ * PTPC_ERR_DEVICE_TIMEOUT (a bounded wait of some static-scratch GEMM since the
+ * last read ran out; its output is then incomplete).  Allocates nothing.
+ * No counterpart on the page. */
+PTPC_API int ptpc_static_scratch_status(void *stream);
 
 /* ------------------------------------------------------------------------- */
 /* Measurement-only entry points: the comparison paths the page describes.  */
 /* ------------------------------------------------------------------------- */
 
-/* Naive two-step path, step 1 (section "The challenge: two-step vs fused",
- * `output = torch._scaled_mm(input, weight)`): the unscaled FP8 GEMM written
- * out as an fp32 intermediate y_dev [T, Co] row-major.  Same mainloop as
+/* Naive two-step path, step 1 (section "The challenge: two-step vs fused":
+ * the FP8 GEMM called without scales): the unscaled FP8 GEMM written out as
+ * an fp32 intermediate y_dev [T, Co] row-major.  Same mainloop as
  * ptpc_scaled_mm, so y is bit-identical to that kernel's accumulator.
  * ws_dev: ptpc_workspace_size(PTPC_OP_BENCH_UNSCALED_MM, T, Ci, Co) bytes. */
 PTPC_API int ptpc_bench_unscaled_mm_f32(const uint8_t *Xq_dev, const uint8_t *Wq_t_dev,
                                int64_t T, int64_t Ci, int64_t Co, float *y_dev,
                                void *ws_dev, size_t ws_bytes, void *stream);
+
+/* Host-side tensor-map cache of the GEMM entry points: how many maps were
+ * taken from the cache (*hits) and how many were encoded (*misses) since the
+ * library was loaded.  A GEMM call needs two or three maps, keyed by pointer,
+ * shape, tile box and element type; repeated calls on the same buffers hit.
+ * No counterpart on the page. */
+PTPC_API int ptpc_bench_map_cache_stats(uint64_t *hits, uint64_t *misses);
 
 /* Effective SM clock during a measurement: one sleeping thread on one SM
  * writes (globaltimer ns, clock64 cycles) pairs to records_dev
@@ -211,8 +242,9 @@ PTPC_API int ptpc_bench_unscaled_mm_f32(const uint8_t *Xq_dev, const uint8_t *Wq
 PTPC_API int ptpc_bench_clock_probe(uint64_t *records_dev, int max_records, uint64_t period_ns,
                                     uint64_t duration_ns, int *count_dev, void *stream);
 
-/* Naive two-step path, step 2 (`output = output * token_scales *
- * channel_scales`): reads y_dev fp32 [T, Co] and writes
+/* Naive two-step path, step 2 (same section: the rank-1 rescale of the
+ * intermediate by the token scales, then the channel scales): reads y_dev
+ * fp32 [T, Co] and writes
  * out_dev[t][o] = bf16_RNE((y[t][o] * x_scale[t]) * w_scale[o]). */
 PTPC_API int ptpc_bench_apply_scales(const float *y_dev, const float *x_scale_dev,
                             const float *w_scale_dev, int64_t T, int64_t Co,

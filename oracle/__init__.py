@@ -8,9 +8,9 @@ this package imports nothing from the product.
 Source: "PTPC-FP8: boosting vLLM performance on AMD ROCm" (vLLM blog), sections
 "What is PTPC-FP8", "Per-Token Activation + Per-Channel Weight Quantization"
 (tensor shapes X: T x Ci, W: Ci x Co, scale vectors Delta_X[T x 1] and
-Delta_W[1 x Co]) and "The challenge: two-step vs fused" (the naive path
-``out = _scaled_mm(x, w); out = out * token_scales * channel_scales`` and the
-fused ``_scaled_mm(x, w, scale_a=token_scales, scale_b=channel_scales)``).
+Delta_W[1 x Co]) and "The challenge: two-step vs fused" (the naive path: an
+unscaled FP8 GEMM into an intermediate, then a rescale by the token scales and
+then the channel scales; the fused path: the GEMM given both scale vectors).
 
 The element-wise steps (E4M3 codec, bf16 rounding, quantisers, fp32
 epilogues) are plain C in ``ptpc_oracle.c``; the dot products use a library

@@ -4,6 +4,7 @@ throughput, and the workloads' shapes against the stated configurations."""
 import importlib.util
 import os
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -62,3 +63,34 @@ def test_roofline_bound_by_arithmetic_intensity(bench):
                                 / sum(bench.gemm_bytes(T, Ci, Co) for T, Ci, Co in shapes))
     assert intensity(pre) > ridge
     assert intensity(dec) < ridge
+
+
+def test_cpu_sample_rows(bench):
+    """The CPU-oracle row sample: first/last rows, both rows at every 128-row
+    tile boundary, then a seeded draw; all rows when the sample covers T."""
+    r = bench.sample_rows(8192, 512, seed=3)
+    assert len(r) == 512 and len(set(r.tolist())) == 512
+    assert r[0] == 0 and r[-1] == 8191 and (np.diff(r) > 0).all()
+    for b in range(128, 8192, 128):
+        assert b - 1 in r and b in r
+    assert np.array_equal(r, bench.sample_rows(8192, 512, seed=3))
+    assert np.array_equal(bench.sample_rows(100, 512), np.arange(100))
+    assert np.array_equal(bench.sample_rows(300, 0), np.arange(300))
+    small = bench.sample_rows(8192, 64)
+    assert len(small) == 64 and small[0] == 0 and small[-1] == 8191
+
+
+def test_chain_roofline(bench):
+    """The chain's roofline time is the slower of its FLOPs at the FP8 peak and
+    its algorithmic bytes at HBM bandwidth: bytes decide at T = 1, FLOPs at
+    T = 8192."""
+    import synthetic
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1650.0}
+    layers = synthetic.CHAIN_70B.layers
+    w_bytes = sum(L.Ci * L.Co for L in layers)
+    t1 = bench.chain_roofline_ms(1, layers, peaks)
+    assert t1 == pytest.approx(sum(bench.quant_bytes(1, L.Ci) + bench.gemm_bytes(1, L.Ci, L.Co) for L in layers)
+                               / 6500e9 * 1e3)
+    assert t1 > w_bytes / 6500e9 * 1e3
+    t8k = bench.chain_roofline_ms(8192, layers, peaks)
+    assert t8k == pytest.approx(sum(2.0 * 8192 * L.Ci * L.Co for L in layers) / 3300e12 * 1e3)

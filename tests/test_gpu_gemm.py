@@ -164,30 +164,70 @@ def test_chain_largest_T_sampled(ptpc, layer):
 
 def test_tuning_overrides(ptpc, monkeypatch):
     """PTPC_FORCE_KSPLIT / PTPC_FORCE_PAIR_BN / PTPC_FORCE_KERNEL change the
-    plan (where feasible) and every forced plan still matches the oracle."""
-    T, Ci, Co = 32, 2048, 4096                 # 32 channel tiles: K split over 4 by default
-    assert ptpc.gemm_ksplit(T, Ci, Co) == 4
-    monkeypatch.setenv("PTPC_FORCE_KSPLIT", "2")
-    assert ptpc.gemm_ksplit(T, Ci, Co) == 2
-    monkeypatch.setenv("PTPC_FORCE_KSPLIT", "8")   # 32 x 8 CTAs do not fit in one wave: ignored
-    assert ptpc.gemm_ksplit(T, Ci, Co) == 4
-    monkeypatch.setenv("PTPC_FORCE_KSPLIT", "1")
-    assert ptpc.gemm_ksplit(T, Ci, Co) == 1
-    monkeypatch.delenv("PTPC_FORCE_KSPLIT")
-    X = synthetic.with_edge_rows(synthetic.make_x(synthetic.DECODE_70B, 0, 256, 1024), huge_bits=BIG_BF16)
-    W = synthetic.random_bf16((1024, 2064), seed=17, scale=0.02)
-    cases = [({"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_PAIR_BN": "128"}, 100),
-             ({"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_PAIR_BN": "256"}, 7),
-             ({"PTPC_FORCE_KERNEL": "decode"}, 256),
-             ({"PTPC_FORCE_KERNEL": "decode", "PTPC_FORCE_KSPLIT": "1"}, 64),
-             ({"PTPC_FORCE_KSPLIT": "2"}, 13)]
-    for env, t in cases:
+    plan (where feasible) and every forced plan still matches the oracle.  The
+    library reads them once, so every change is followed by a reload."""
+    names = ("PTPC_FORCE_KSPLIT", "PTPC_FORCE_PAIR_BN", "PTPC_FORCE_KERNEL")
+
+    def setenv(env):
+        for k in names:
+            monkeypatch.delenv(k, raising=False)
         for k, v in env.items():
             monkeypatch.setenv(k, v)
-        g, r = run_pair(ptpc, X[:t].copy(), W)
-        assert_gemm_close(g, r, f"forced {env} T={t}")
-        for k in env:
-            monkeypatch.delenv(k)
+        ptpc.reload_tuning_overrides()
+
+    T, Ci, Co = 32, 2048, 4096                 # 32 channel tiles: K split over 4 by default
+    try:
+        setenv({})
+        assert ptpc.gemm_ksplit(T, Ci, Co) == 4
+        monkeypatch.setenv("PTPC_FORCE_KSPLIT", "2")
+        assert ptpc.gemm_ksplit(T, Ci, Co) == 4    # not re-read until a reload
+        setenv({"PTPC_FORCE_KSPLIT": "2"})
+        assert ptpc.gemm_ksplit(T, Ci, Co) == 2
+        setenv({"PTPC_FORCE_KSPLIT": "8"})         # 32 x 8 CTAs do not fit in one wave: ignored
+        assert ptpc.gemm_ksplit(T, Ci, Co) == 4
+        setenv({"PTPC_FORCE_KSPLIT": "1"})
+        assert ptpc.gemm_ksplit(T, Ci, Co) == 1
+        X = synthetic.with_edge_rows(synthetic.make_x(synthetic.DECODE_70B, 0, 256, 1024), huge_bits=BIG_BF16)
+        W = synthetic.random_bf16((1024, 2064), seed=17, scale=0.02)
+        cases = [({"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_PAIR_BN": "128"}, 100),
+                 ({"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_PAIR_BN": "256"}, 7),
+                 ({"PTPC_FORCE_KERNEL": "decode"}, 256),
+                 ({"PTPC_FORCE_KERNEL": "decode", "PTPC_FORCE_KSPLIT": "1"}, 64),
+                 ({"PTPC_FORCE_KSPLIT": "2"}, 13)]
+        for env, t in cases:
+            setenv(env)
+            g, r = run_pair(ptpc, X[:t].copy(), W)
+            assert_gemm_close(g, r, f"forced {env} T={t}")
+    finally:
+        setenv({})
+    assert ptpc.gemm_ksplit(T, Ci, Co) == 4
+
+
+def test_tensor_map_cache(ptpc):
+    """Repeated GEMM calls on the same buffers take their tensor maps from the
+    library's host-side cache; another buffer of the same shape is a miss and
+    still computes its own result."""
+    T, Ci, Co = 64, 1024, 2048
+    X = synthetic.make_x(synthetic.DECODE_70B, 0, T, Ci)
+    W = synthetic.random_bf16((Ci, Co), seed=5, scale=0.02)
+    Wq_t, ws = ptpc.quantize_weights(to_dev_bf16(W))
+    Xq, xs = ptpc.quantize_activations(to_dev_bf16(X))
+    out = ptpc.scaled_mm(Xq, xs, Wq_t, ws)
+    h0, m0 = ptpc.map_cache_stats()
+    for _ in range(5):
+        ptpc.scaled_mm(Xq, xs, Wq_t, ws, out=out)
+    h1, m1 = ptpc.map_cache_stats()
+    assert m1 == m0 and h1 - h0 >= 10, (h0, m0, h1, m1)
+    # same shape, other buffers (the second weight is the first one negated)
+    Wq2, ws2 = ptpc.quantize_weights(to_dev_bf16(W ^ np.uint16(0x8000)))
+    out2 = ptpc.scaled_mm(Xq, xs, Wq2, ws2)
+    h2, m2 = ptpc.map_cache_stats()
+    assert m2 > m1
+    torch.cuda.synchronize()
+    a = from_dev_bf16(out).astype(np.uint16)
+    b = from_dev_bf16(out2).astype(np.uint16)
+    nz = (a & 0x7FFF) != 0
+    assert np.array_equal(a[nz] ^ np.uint16(0x8000), b[nz])
 
 
 def test_naive_two_step_equals_fused(ptpc):
