@@ -72,6 +72,14 @@ def _load():
             lib.oracle_quantize_value.argtypes = [ctypes.c_float, ctypes.c_float, ctypes.c_float]
             lib.oracle_bf16_from_double.restype = ctypes.c_uint16
             lib.oracle_bf16_from_double.argtypes = [ctypes.c_double]
+            lib.oracle_fmt_decode.restype = ctypes.c_double
+            lib.oracle_fmt_decode.argtypes = [ctypes.c_uint8, ctypes.c_int]
+            lib.oracle_fmt_encode.restype = ctypes.c_uint8
+            lib.oracle_fmt_encode.argtypes = [ctypes.c_float, ctypes.c_int]
+            lib.oracle_fmt_max.restype = ctypes.c_double
+            lib.oracle_fmt_max.argtypes = [ctypes.c_int]
+            lib.oracle_packed_row_bytes.restype = ctypes.c_int64
+            lib.oracle_packed_row_bytes.argtypes = [ctypes.c_int64, ctypes.c_int]
             for name, args in {
                 "oracle_quant_act": [P, I64, I64, P, P],
                 "oracle_quant_weight": [P, I64, I64, P, P],
@@ -82,6 +90,9 @@ def _load():
                 "oracle_reference_epilogue_f64": [P, I64, I64, P, P, P],
                 "oracle_e4m3_encode_array": [P, I64, P],
                 "oracle_bf16_from_double_array": [P, I64, P],
+                "oracle_quant_weight_fmt": [P, I64, I64, ctypes.c_int, P, P],
+                "oracle_pack_fmt": [P, I64, I64, ctypes.c_int, P],
+                "oracle_fmt_encode_array": [P, I64, ctypes.c_int, P],
             }.items():
                 fn = getattr(lib, name)
                 fn.restype = None
@@ -253,3 +264,94 @@ def fused_f32(Xq, x_scale, Wq_t, w_scale, rows=None) -> np.ndarray:
     _load().oracle_fused_epilogue_f32(_ptr(acc), acc.shape[0], acc.shape[1],
                                       _ptr(xs), _ptr(ws), _ptr(out))
     return out
+
+
+# --------------------------------------------------------------------------
+# Sub-byte weight formats (FP6 E3M2 / E2M3, FP4 E2M1)
+# --------------------------------------------------------------------------
+# Source: the llminfo.tech summary of "Running LLMs at custom floating-points
+# (near-lossless FP6)" (FP4-FP7 weights with per-channel quantisation, the
+# MX formats named as the likely standard) with the PTPC page's per-output-
+# channel weight scale.  The readings are listed in ptpc_oracle.c.
+
+FORMATS = {"e4m3": 0, "e2m1": 1, "e2m3": 2, "e3m2": 3}
+FORMAT_BITS = {"e4m3": 8, "e2m1": 4, "e2m3": 6, "e3m2": 6}
+
+
+def fmt_max(fmt: str) -> float:
+    """Largest finite magnitude of a format."""
+    return float(_load().oracle_fmt_max(FORMATS[fmt]))
+
+
+def fmt_decode_table(fmt: str) -> np.ndarray:
+    """fp64 value of every code of a format (2^bits entries, sign in the top bit)."""
+    lib = _load()
+    f = FORMATS[fmt]
+    return np.array([lib.oracle_fmt_decode(c, f) for c in range(1 << FORMAT_BITS[fmt])], dtype=np.float64)
+
+
+def fmt_encode(v, fmt: str) -> np.ndarray:
+    """Saturating round-half-to-even codes of fp32 values in a format."""
+    a = np.ascontiguousarray(np.asarray(v, dtype=np.float32))
+    out = np.empty(a.shape, dtype=np.uint8)
+    _load().oracle_fmt_encode_array(_ptr(a), a.size, FORMATS[fmt], _ptr(out))
+    return out
+
+
+def quant_weight_fmt(W_bits: np.ndarray, fmt: str):
+    """Per-output-channel quantisation of W (Ci x Co bf16 bits) to a format:
+    (codes_t [Co, Ci] u8, one code per byte; w_scale [Co] f32 = amax / max)."""
+    W = np.ascontiguousarray(W_bits, dtype=np.uint16)
+    Ci, Co = W.shape
+    codes = np.empty((Co, Ci), dtype=np.uint8)
+    ws = np.empty((Co,), dtype=np.float32)
+    _load().oracle_quant_weight_fmt(_ptr(W), Ci, Co, FORMATS[fmt], _ptr(codes), _ptr(ws))
+    return codes, ws
+
+
+def pack_fmt(codes: np.ndarray, fmt: str) -> np.ndarray:
+    """Packs [rows, K] codes (one per byte) into the bytes the weight occupies
+    in memory: [rows, K * bits / 8]."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    rows, K = c.shape
+    assert K % 16 == 0
+    lib = _load()
+    out = np.empty((rows, int(lib.oracle_packed_row_bytes(K, FORMATS[fmt]))), dtype=np.uint8)
+    lib.oracle_pack_fmt(_ptr(c), rows, K, FORMATS[fmt], _ptr(out))
+    return out
+
+
+def gemm_acc64_fmt(Xq: np.ndarray, codes_t: np.ndarray, fmt: str, rows=None, col_chunk: int = 4096) -> np.ndarray:
+    """acc[t, o] = sum_k dec_e4m3(Xq[t, k]) * dec_fmt(codes_t[o, k]) in fp64.
+
+    Exact: E4M3 values are integer multiples of 2^-9 and the sub-byte formats'
+    of 2^-4 or coarser, every product an integer multiple of 2^-13 below 2^14,
+    so sums of up to 2^17 products stay below 2^44 units."""
+    Ci = Xq.shape[1]
+    assert codes_t.shape[1] == Ci and Ci <= MAX_EXACT_K
+    A = e4m3_decode_table()[Xq if rows is None else Xq[np.asarray(rows)]]
+    dec = fmt_decode_table(fmt)
+    Co = codes_t.shape[0]
+    acc = np.empty((A.shape[0], Co), dtype=np.float64)
+    for o0 in range(0, Co, col_chunk):
+        acc[:, o0:o0 + col_chunk] = A @ dec[codes_t[o0:o0 + col_chunk]].T
+    return acc
+
+
+def scaled_mm_reference_fmt(Xq, x_scale, codes_t, w_scale, fmt: str, rows=None) -> np.ndarray:
+    """Tolerance reference of the scaled GEMM with format-f weights:
+    bf16_RNE(x_scale[t] * w_scale[o] * acc[t, o]) in fp64 (bf16 bits)."""
+    acc = gemm_acc64_fmt(Xq, codes_t, fmt, rows)
+    xs = np.ascontiguousarray(np.asarray(x_scale, dtype=np.float32)[
+        slice(None) if rows is None else np.asarray(rows)])
+    ws = np.ascontiguousarray(w_scale, dtype=np.float32)
+    out = np.empty(acc.shape, dtype=np.uint16)
+    _load().oracle_reference_epilogue_f64(_ptr(acc), acc.shape[0], acc.shape[1], _ptr(xs), _ptr(ws), _ptr(out))
+    return out
+
+
+def linear_reference_fmt(X_bits, codes_t, w_scale, fmt: str, rows=None):
+    """Per-token FP8 quantisation of X, then the scaled GEMM against format-f
+    weights.  Returns (out bf16 bits, Xq, x_scale)."""
+    Xq, xs = quant_act(X_bits)
+    return scaled_mm_reference_fmt(Xq, xs, codes_t, w_scale, fmt, rows), Xq, xs

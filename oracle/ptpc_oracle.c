@@ -332,3 +332,182 @@ void oracle_bf16_from_double_array(const double *v, int64_t n, uint16_t *out)
     for (i = 0; i < n; ++i)
         out[i] = oracle_bf16_from_double(v[i]);
 }
+
+/* ------------------------------------------------------------------------- */
+/* Sub-byte weight formats: FP6 (E3M2, E2M3) and FP4 (E2M1)                  */
+/* ------------------------------------------------------------------------- */
+/*
+ * Source: the llminfo.tech summary of "Running LLMs at custom floating-points
+ * (near-lossless FP6)" (FP6-LLM extended to FP4-FP7 with per-channel
+ * quantisation; the exponent/mantissa split is a free choice, and the author
+ * names the MX formats as the likely standard), combined with the PTPC page's
+ * per-output-channel weight scale.  Readings (the pages give no formula):
+ *   - the formats are the OCP MX element types, which the B200 tensor cores
+ *     consume natively: E2M1 (bias 1, max 6), E2M3 (bias 1, max 7.5), E3M2
+ *     (bias 3, max 28); none has infinities or NaN;
+ *   - per output channel o: s = amax_o / max_format (IEEE fp32 division),
+ *     1.0f for an all-zero column; code = saturating round-half-to-even of
+ *     fp32_RN(w / s) to the format's grid, sign kept (-0 -> sign bit set);
+ *   - a code is held in the low bits of a byte: sign at bit (E + M), then E
+ *     exponent bits, then M mantissa bits;
+ *   - packing along K (the input channels) into the bytes that the weight
+ *     occupies in memory: FP4 two codes per byte, the even position in the
+ *     low nibble; FP6 sixteen codes per twelve bytes, code j of the group at
+ *     bits [6j, 6j + 6) of the group read as a little-endian 96-bit integer.
+ * Format ids: 0 E4M3 (the PTPC format, for cross-checks), 1 E2M1, 2 E2M3,
+ * 3 E3M2.
+ */
+
+typedef struct {
+    int ebits, mbits, bias;
+    double maxval;
+} oracle_fmt;
+
+static oracle_fmt oracle_fmt_of(int f)
+{
+    oracle_fmt r;
+    switch (f) {
+    case 1: r.ebits = 2; r.mbits = 1; r.bias = 1; r.maxval = 6.0; break;
+    case 2: r.ebits = 2; r.mbits = 3; r.bias = 1; r.maxval = 7.5; break;
+    case 3: r.ebits = 3; r.mbits = 2; r.bias = 3; r.maxval = 28.0; break;
+    default: r.ebits = 4; r.mbits = 3; r.bias = 7; r.maxval = 448.0; break;
+    }
+    return r;
+}
+
+double oracle_fmt_max(int f)
+{
+    return oracle_fmt_of(f).maxval;
+}
+
+/* Value of a code: exponent field e, mantissa field m.  e == 0 is subnormal,
+ * m * 2^(1 - bias - M); otherwise (2^M + m) * 2^(e - bias - M).  E4M3's
+ * S.1111.111 is NaN; the sub-byte formats have none. */
+double oracle_fmt_decode(uint8_t code, int f)
+{
+    oracle_fmt t = oracle_fmt_of(f);
+    int nb = t.ebits + t.mbits;
+    int sign = (code >> nb) & 1;
+    int e = (code >> t.mbits) & ((1 << t.ebits) - 1);
+    int m = code & ((1 << t.mbits) - 1);
+    double mag;
+    if (f == 0 && e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        mag = ldexp((double)m, 1 - t.bias - t.mbits);
+    else
+        mag = ldexp((double)((1 << t.mbits) + m), e - t.bias - t.mbits);
+    return sign ? -mag : mag;
+}
+
+/* Saturating round-half-to-even of an fp32 value to the format's grid: the
+ * same steps as oracle_e4m3_encode, with the format's parameters. */
+uint8_t oracle_fmt_encode(float v, int f)
+{
+    oracle_fmt t = oracle_fmt_of(f);
+    int nb = t.ebits + t.mbits;
+    uint8_t sign = signbit(v) ? (uint8_t)(1u << nb) : 0;
+    double a, step, n, fl, rem, q, min_normal = ldexp(1.0, 1 - t.bias);
+    int E;
+
+    if (isnan(v))
+        return (uint8_t)(sign | ((1u << nb) - 1u)); /* outside the contract */
+    a = fabs((double)v);
+    if (a >= t.maxval)
+        q = t.maxval;
+    else {
+        if (a < min_normal) {
+            step = ldexp(1.0, 1 - t.bias - t.mbits);
+        } else {
+            frexp(a, &E);                      /* a in [2^(E-1), 2^E) */
+            step = ldexp(1.0, (E - 1) - t.mbits);
+        }
+        n = a / step;                          /* exact: step is a power of two */
+        fl = floor(n);
+        rem = n - fl;
+        if (rem > 0.5 || (rem == 0.5 && fmod(fl, 2.0) == 1.0))
+            fl += 1.0;
+        q = fl * step;
+        if (q > t.maxval)
+            q = t.maxval;
+    }
+    if (q < min_normal)
+        return (uint8_t)(sign | (uint8_t)(q / ldexp(1.0, 1 - t.bias - t.mbits)));
+    frexp(q, &E);
+    {
+        int e = (E - 1) + t.bias;
+        int m = (int)(q / ldexp(1.0, E - 1) * (double)(1 << t.mbits)) - (1 << t.mbits);
+        return (uint8_t)(sign | (uint8_t)((e << t.mbits) | m));
+    }
+}
+
+/* Per-output-channel weight quantisation to format f: W is Ci x Co bf16
+ * (row-major); writes one code per byte, transposed (codes_t is Co x Ci),
+ * and w_scale[Co] = amax / max_format. */
+void oracle_quant_weight_fmt(const uint16_t *W, int64_t Ci, int64_t Co, int f,
+                             uint8_t *codes_t, float *w_scale)
+{
+    const float fmax = (float)oracle_fmt_of(f).maxval;
+    int64_t o;
+#pragma omp parallel for schedule(static)
+    for (o = 0; o < Co; ++o) {
+        float amax = 0.0f, s;
+        int64_t k;
+        for (k = 0; k < Ci; ++k) {
+            float a = fabsf(oracle_bf16_to_float(W[k * Co + o]));
+            if (a > amax)
+                amax = a;
+        }
+        s = amax == 0.0f ? 1.0f : amax / fmax;
+        w_scale[o] = s;
+        for (k = 0; k < Ci; ++k) {
+            float x = oracle_bf16_to_float(W[k * Co + o]);
+            codes_t[o * Ci + k] = amax == 0.0f ? 0 : oracle_fmt_encode(x / s, f);
+        }
+    }
+}
+
+/* Bytes a row of K codes of format f occupies once packed. */
+int64_t oracle_packed_row_bytes(int64_t K, int f)
+{
+    if (f == 1)
+        return K / 2;
+    if (f == 2 || f == 3)
+        return K / 16 * 12;
+    return K;
+}
+
+/* Packs rows x K codes (one per byte) into rows x oracle_packed_row_bytes
+ * bytes, bit by bit: code k of a row occupies bits [b*k, b*k + b) of the
+ * packed row read as a little-endian bit string (b = 4 for E2M1, 6 for the
+ * FP6 formats, 8 for E4M3).  K must be a multiple of 16. */
+void oracle_pack_fmt(const uint8_t *codes, int64_t rows, int64_t K, int f, uint8_t *packed)
+{
+    const int b = f == 1 ? 4 : (f == 2 || f == 3) ? 6 : 8;
+    const int64_t rb = oracle_packed_row_bytes(K, f);
+    int64_t r;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < rows; ++r) {
+        int64_t k;
+        uint8_t *dst = packed + r * rb;
+        memset(dst, 0, (size_t)rb);
+        for (k = 0; k < K; ++k) {
+            int bit;
+            uint8_t c = codes[r * K + k];
+            for (bit = 0; bit < b; ++bit) {
+                int64_t pos = k * b + bit;
+                if ((c >> bit) & 1)
+                    dst[pos / 8] |= (uint8_t)(1u << (pos % 8));
+            }
+        }
+    }
+}
+
+/* Array form of oracle_fmt_encode, for the tests. */
+void oracle_fmt_encode_array(const float *v, int64_t n, int f, uint8_t *out)
+{
+    int64_t i;
+#pragma omp parallel for schedule(static)
+    for (i = 0; i < n; ++i)
+        out[i] = oracle_fmt_encode(v[i], f);
+}
