@@ -33,6 +33,10 @@ ERR_CUDA = 6
 ERR_DEVICE_TIMEOUT = 7
 ERR_NOT_IMPLEMENTED = 8
 
+# ptpc_weight_format
+WEIGHT_FORMATS = {"e4m3": 0, "e2m1": 1, "e2m3": 2, "e3m2": 3}
+WEIGHT_BITS = {"e4m3": 8, "e2m1": 4, "e2m3": 6, "e3m2": 6}
+
 # ptpc_op
 OP_QUANTIZE_WEIGHTS = 1
 OP_SCALED_MM = 2
@@ -56,6 +60,12 @@ SIGNATURES = {
     "ptpc_selftest_wait_timeout": (ctypes.c_int, [_P, _P]),
     "ptpc_scaled_mm_static_scratch": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "ptpc_static_scratch_status": (ctypes.c_int, [_P]),
+    "ptpc_weight_bytes": (ctypes.c_size_t, [ctypes.c_int, _I64, _I64]),
+    "ptpc_act_row_amax": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P]),
+    "ptpc_quantize_activations_amax": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P]),
+    "ptpc_quantize_weights_fmt": (ctypes.c_int, [_P, _I64, _I64, ctypes.c_int, _P, _P, _P, _SZ, _P]),
+    "ptpc_scaled_mm_fmt": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "ptpc_linear_fmt": (ctypes.c_int, [_P, _I64, _P, _P, ctypes.c_int, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "ptpc_reload_tuning_overrides": (ctypes.c_int, []),
     "ptpc_bench_map_cache_stats": (ctypes.c_int, [_P, _P]),
     "ptpc_bench_unscaled_mm_f32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
@@ -205,6 +215,30 @@ def quantize_activations(X: torch.Tensor, Xq: torch.Tensor | None = None, x_scal
     return Xq, x_scale
 
 
+def row_amax(X: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """fp32 [T]: max |x| of every row of X bf16 [T, Ci] (rows contiguous)."""
+    ldx = _need_rows(X, "X")
+    T, Ci = X.shape
+    out = torch.empty((T,), dtype=torch.float32, device=X.device) if out is None else out
+    _check("ptpc_act_row_amax", lib.ptpc_act_row_amax(_ptr(X), T, Ci, ldx, _ptr(out), _stream(X.device)))
+    return out
+
+
+def quantize_activations_amax(X: torch.Tensor, amax: torch.Tensor, Xq: torch.Tensor | None = None,
+                              x_scale: torch.Tensor | None = None):
+    """Per-token quantisation of a row slice X [T, Ci] with the given row
+    maxima (combined over the slices) -> (Xq uint8 [T, Ci], x_scale fp32 [T])."""
+    ldx = _need_rows(X, "X")
+    _need(amax, "amax", torch.float32, 1)
+    T, Ci = X.shape
+    Xq = torch.empty((T, Ci), dtype=torch.uint8, device=X.device) if Xq is None else Xq
+    x_scale = torch.empty((T,), dtype=torch.float32, device=X.device) if x_scale is None else x_scale
+    _check("ptpc_quantize_activations_amax",
+           lib.ptpc_quantize_activations_amax(_ptr(X), T, Ci, ldx, _ptr(amax), _ptr(Xq), _ptr(x_scale),
+                                              _stream(X.device)))
+    return Xq, x_scale
+
+
 def quantize_weights(W: torch.Tensor, ws: Workspace | None = None):
     """Per-output-channel quantisation: W bf16 [Ci, Co] -> (Wq_t uint8 [Co, Ci], w_scale fp32 [Co])."""
     _need(W, "W", torch.bfloat16, 2)
@@ -217,6 +251,74 @@ def quantize_weights(W: torch.Tensor, ws: Workspace | None = None):
            lib.ptpc_quantize_weights(_ptr(W), Ci, Co, _ptr(Wq_t), _ptr(w_scale), ws.ptr(), ws.nbytes,
                                      _stream(W.device)))
     return Wq_t, w_scale
+
+
+def _fmt(fmt: str) -> int:
+    if fmt not in WEIGHT_FORMATS:
+        raise ValueError(f"weight format must be one of {sorted(WEIGHT_FORMATS)}, got {fmt!r}")
+    return WEIGHT_FORMATS[fmt]
+
+
+def quantize_weights_fmt(W: torch.Tensor, fmt: str, ws: Workspace | None = None):
+    """Per-output-channel quantisation of W bf16 [Ci, Co] to a weight format
+    ('e4m3', 'e2m1', 'e2m3', 'e3m2') -> (Wq uint8 [Co, Ci * bits / 8] packed
+    along Ci, w_scale fp32 [Co])."""
+    _need(W, "W", torch.bfloat16, 2)
+    Ci, Co = W.shape
+    f = _fmt(fmt)
+    nbytes = int(lib.ptpc_weight_bytes(f, Ci, Co))
+    if nbytes == 0:
+        raise ValueError(f"unsupported shape {Ci}x{Co} for weight format {fmt}")
+    # 32-byte aligned rows: the caching allocator returns 512-byte aligned blocks
+    Wq = torch.empty((Co, nbytes // Co), dtype=torch.uint8, device=W.device)
+    w_scale = torch.empty((Co,), dtype=torch.float32, device=W.device)
+    need = workspace_size(OP_QUANTIZE_WEIGHTS, 0, Ci, Co)
+    ws = default_workspace(need, W.device) if ws is None else ws.ensure(need)
+    _check("ptpc_quantize_weights_fmt",
+           lib.ptpc_quantize_weights_fmt(_ptr(W), Ci, Co, f, _ptr(Wq), _ptr(w_scale), ws.ptr(), ws.nbytes,
+                                         _stream(W.device)))
+    return Wq, w_scale
+
+
+def _packed_ci(Wq: torch.Tensor, fmt: str) -> int:
+    return Wq.shape[1] * 8 // WEIGHT_BITS[fmt]
+
+
+def scaled_mm_fmt(Xq, x_scale, Wq, w_scale, fmt: str, out: torch.Tensor | None = None, ws: Workspace | None = None):
+    """Scaled GEMM against weights of a format (from quantize_weights_fmt)."""
+    _need(Xq, "Xq", torch.uint8, 2)
+    _need(Wq, "Wq", torch.uint8, 2)
+    _need(x_scale, "x_scale", torch.float32, 1)
+    _need(w_scale, "w_scale", torch.float32, 1)
+    T, Ci = Xq.shape
+    Co = Wq.shape[0]
+    if _packed_ci(Wq, fmt) != Ci or x_scale.shape[0] != T or w_scale.shape[0] != Co:
+        raise ValueError("shape mismatch")
+    out = torch.empty((T, Co), dtype=torch.bfloat16, device=Xq.device) if out is None else out
+    need = workspace_size(OP_SCALED_MM, T, Ci, Co)
+    ws = default_workspace(need, Xq.device) if ws is None else ws.ensure(need)
+    _check("ptpc_scaled_mm_fmt",
+           lib.ptpc_scaled_mm_fmt(_ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), _fmt(fmt), T, Ci, Co,
+                                  _ptr(out), ws.ptr(), ws.nbytes, _stream(Xq.device)))
+    return out
+
+
+def linear_fmt(X, Wq, w_scale, fmt: str, out: torch.Tensor | None = None, ws: Workspace | None = None):
+    """Fused per-token FP8 quantisation + GEMM against weights of a format."""
+    ldx = _need_rows(X, "X")
+    _need(Wq, "Wq", torch.uint8, 2)
+    _need(w_scale, "w_scale", torch.float32, 1)
+    T, Ci = X.shape
+    Co = Wq.shape[0]
+    if _packed_ci(Wq, fmt) != Ci or w_scale.shape[0] != Co:
+        raise ValueError("shape mismatch")
+    out = torch.empty((T, Co), dtype=torch.bfloat16, device=X.device) if out is None else out
+    need = workspace_size(OP_LINEAR, T, Ci, Co)
+    ws = default_workspace(need, X.device) if ws is None else ws.ensure(need)
+    _check("ptpc_linear_fmt",
+           lib.ptpc_linear_fmt(_ptr(X), ldx, _ptr(Wq), _ptr(w_scale), _fmt(fmt), T, Ci, Co, _ptr(out), ws.ptr(),
+                               ws.nbytes, _stream(X.device)))
+    return out
 
 
 def scaled_mm(Xq, x_scale, Wq_t, w_scale, out: torch.Tensor | None = None, ws: Workspace | None = None):

@@ -63,9 +63,24 @@ int check_co(int64_t Co) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? PTPC_OK : PTPC_ERR_CUDA; }
 
+// Weight formats (ptpc_weight_format): bits per code.
+int wfmt_bits(int fmt) { return fmt == PTPC_WFMT_E4M3 ? 8 : fmt == PTPC_WFMT_E2M1 ? 4 : 6; }
+
+bool valid_wfmt(int fmt) { return fmt >= PTPC_WFMT_E4M3 && fmt <= PTPC_WFMT_E3M2; }
+
+// Packed sub-byte weights: TMA's 4- and 6-bit tensor types read rows of whole
+// 128-code boxes from 32-byte aligned addresses.
+int check_subbyte(int fmt, int64_t Ci, const void *Wq) {
+  if (fmt == PTPC_WFMT_E4M3) return PTPC_OK;
+  if (Ci % 128 != 0) return PTPC_ERR_UNSUPPORTED_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(Wq) & 31u) != 0) return PTPC_ERR_MISALIGNED;
+  return PTPC_OK;
+}
+
 int run_gemm(const uint8_t *Xq, const float *xs, const uint8_t *Wq_t, const float *ws, int64_t T, int64_t Ci,
-             int64_t Co, void *out, bool f32_out, uint8_t *wsp, bool pdl, cudaStream_t st) {
+             int64_t Co, void *out, bool f32_out, uint8_t *wsp, bool pdl, cudaStream_t st, int wfmt = 0) {
   ptpc::GemmProblem p{};
+  p.wfmt = wfmt;
   p.Xq = Xq;
   p.xs = xs;
   p.Wq_t = Wq_t;
@@ -131,6 +146,30 @@ int ptpc_quantize_activations(const void *X, int64_t T, int64_t Ci, int64_t ldx,
   return cuda_status(ptpc::launch_quant_act(X, (int)T, (int)Ci, ldx, Xq, x_scale, (cudaStream_t)stream));
 }
 
+int ptpc_act_row_amax(const void *X, int64_t T, int64_t Ci, int64_t ldx, float *amax, void *stream) {
+  int s = check_shape_tci(T, Ci);
+  if (s != PTPC_OK) return s;
+  if (T == 0) return PTPC_OK;
+  if ((s = check_ldx(ldx, Ci)) != PTPC_OK) return s;
+  if (!X || !amax) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(amax)) return PTPC_ERR_MISALIGNED;
+  if ((s = check_device()) != PTPC_OK) return s;
+  return cuda_status(ptpc::launch_row_amax(X, (int)T, (int)Ci, ldx, amax, (cudaStream_t)stream));
+}
+
+int ptpc_quantize_activations_amax(const void *X, int64_t T, int64_t Ci, int64_t ldx, const float *amax,
+                                   uint8_t *Xq, float *x_scale, void *stream) {
+  int s = check_shape_tci(T, Ci);
+  if (s != PTPC_OK) return s;
+  if (T == 0) return PTPC_OK;
+  if ((s = check_ldx(ldx, Ci)) != PTPC_OK) return s;
+  if (!X || !amax || !Xq || !x_scale) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(amax) || !aligned16(Xq) || !aligned16(x_scale)) return PTPC_ERR_MISALIGNED;
+  if ((s = check_device()) != PTPC_OK) return s;
+  return cuda_status(
+      ptpc::launch_quant_act_amax(X, (int)T, (int)Ci, ldx, amax, Xq, x_scale, (cudaStream_t)stream));
+}
+
 int ptpc_quantize_weights(const void *W, int64_t Ci, int64_t Co, uint8_t *Wq_t, float *w_scale, void *ws,
                           size_t ws_bytes, void *stream) {
   int s = check_shape_tci(0, Ci);
@@ -179,6 +218,69 @@ int ptpc_linear(const void *X, int64_t ldx, const uint8_t *Wq_t, const float *w_
   cudaStream_t st = (cudaStream_t)stream;
   if ((s = cuda_status(ptpc::launch_quant_act(X, (int)T, (int)Ci, ldx, Xq, xs, st))) != PTPC_OK) return s;
   return run_gemm(Xq, xs, Wq_t, w_scale, T, Ci, Co, out, false, wsp, true, st);
+}
+
+size_t ptpc_weight_bytes(int fmt, int64_t Ci, int64_t Co) {
+  if (!valid_wfmt(fmt) || check_shape_tci(0, Ci) != PTPC_OK || check_co(Co) != PTPC_OK) return 0;
+  if (fmt != PTPC_WFMT_E4M3 && Ci % 128 != 0) return 0;
+  return (size_t)Co * (size_t)Ci * (size_t)wfmt_bits(fmt) / 8;
+}
+
+int ptpc_quantize_weights_fmt(const void *W, int64_t Ci, int64_t Co, int fmt, uint8_t *Wq, float *w_scale, void *ws,
+                              size_t ws_bytes, void *stream) {
+  if (!valid_wfmt(fmt)) return PTPC_ERR_INVALID_ARG;
+  if (fmt == PTPC_WFMT_E4M3) return ptpc_quantize_weights(W, Ci, Co, Wq, w_scale, ws, ws_bytes, stream);
+  int s = check_shape_tci(0, Ci);
+  if (s != PTPC_OK) return s;
+  if ((s = check_co(Co)) != PTPC_OK) return s;
+  if (!W || !Wq || !w_scale || !ws) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(w_scale) || !aligned16(ws)) return PTPC_ERR_MISALIGNED;
+  if ((s = check_subbyte(fmt, Ci, Wq)) != PTPC_OK) return s;
+  if (ws_bytes < ptpc_workspace_size(PTPC_OP_QUANTIZE_WEIGHTS, 0, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device()) != PTPC_OK) return s;
+  uint32_t *col_amax = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + kAlign);
+  return cuda_status(
+      ptpc::launch_quant_weight_sub(W, (int)Ci, (int)Co, fmt, Wq, w_scale, col_amax, (cudaStream_t)stream));
+}
+
+int ptpc_scaled_mm_fmt(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq, const float *w_scale, int fmt,
+                       int64_t T, int64_t Ci, int64_t Co, void *out, void *ws, size_t ws_bytes, void *stream) {
+  if (!valid_wfmt(fmt)) return PTPC_ERR_INVALID_ARG;
+  int s = check_shape_tci(T, Ci);
+  if (s != PTPC_OK) return s;
+  if ((s = check_co(Co)) != PTPC_OK) return s;
+  if (T == 0) return PTPC_OK;
+  if (!Xq || !x_scale || !Wq || !w_scale || !out || !ws) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(Xq) || !aligned16(x_scale) || !aligned16(Wq) || !aligned16(w_scale) || !aligned16(out) ||
+      !aligned16(ws))
+    return PTPC_ERR_MISALIGNED;
+  if ((s = check_subbyte(fmt, Ci, Wq)) != PTPC_OK) return s;
+  if (ws_bytes < ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device()) != PTPC_OK) return s;
+  return run_gemm(Xq, x_scale, Wq, w_scale, T, Ci, Co, out, false, static_cast<uint8_t *>(ws), false,
+                  (cudaStream_t)stream, fmt);
+}
+
+int ptpc_linear_fmt(const void *X, int64_t ldx, const uint8_t *Wq, const float *w_scale, int fmt, int64_t T,
+                    int64_t Ci, int64_t Co, void *out, void *ws, size_t ws_bytes, void *stream) {
+  if (!valid_wfmt(fmt)) return PTPC_ERR_INVALID_ARG;
+  int s = check_shape_tci(T, Ci);
+  if (s != PTPC_OK) return s;
+  if ((s = check_co(Co)) != PTPC_OK) return s;
+  if (T == 0) return PTPC_OK;
+  if ((s = check_ldx(ldx, Ci)) != PTPC_OK) return s;
+  if (!X || !Wq || !w_scale || !out || !ws) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(Wq) || !aligned16(w_scale) || !aligned16(out) || !aligned16(ws))
+    return PTPC_ERR_MISALIGNED;
+  if ((s = check_subbyte(fmt, Ci, Wq)) != PTPC_OK) return s;
+  if (ws_bytes < ptpc_workspace_size(PTPC_OP_LINEAR, T, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device()) != PTPC_OK) return s;
+  uint8_t *wsp = static_cast<uint8_t *>(ws);
+  uint8_t *Xq = wsp + kGemmWorkspace;
+  float *xs = reinterpret_cast<float *>(wsp + kGemmWorkspace + round_up((size_t)T * (size_t)Ci));
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((s = cuda_status(ptpc::launch_quant_act(X, (int)T, (int)Ci, ldx, Xq, xs, st))) != PTPC_OK) return s;
+  return run_gemm(Xq, xs, Wq, w_scale, T, Ci, Co, out, false, wsp, true, st, fmt);
 }
 
 int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co) {

@@ -57,6 +57,16 @@ constexpr int BK = 128;      // K bytes per stage (= one 128-byte swizzle row)
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 
+// Weight formats: 0 E4M3 (PTPC-FP8), 1 E2M1 (FP4), 2 E2M3 and 3 E3M2 (FP6).
+// The sub-byte weights sit packed in global memory and are unpacked by TMA
+// into the same one-byte-per-element shared-memory layout as E4M3 (16 codes
+// per 16-byte chunk), so only the bytes a stage transfers and the MMA's
+// operand format change.
+__host__ __device__ constexpr int wf_bits(int wf) { return wf == 0 ? 8 : wf == 1 ? 4 : 6; }
+__host__ __device__ constexpr uint32_t wf_mma(int wf) {
+  return wf == 0 ? kMmaE4M3 : wf == 1 ? kMmaE2M1 : wf == 2 ? kMmaE2M3 : kMmaE3M2;
+}
+
 struct GemmParams {
   int T, Co;
   int num_m, num_n, num_kb;   // tile grid (pair kernel: 256-token tile rows; decode: one row of all tokens)
@@ -337,7 +347,7 @@ __device__ __forceinline__ void decode_cluster_reduce(const GemmParams &p, const
   }
 }
 
-template <bool F32OUT>
+template <bool F32OUT, int WF>
 __global__ void __launch_bounds__(kThreads, 1)
     ptpc_gemm_decode_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                             const GemmParams p) {
@@ -390,7 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (elect_one()) {
       const uint64_t polW = policy_evict_first();  // every weight byte is read once
       const uint64_t polX = policy_evict_last();   // every CTA reads the activations
-      const uint32_t stage_tx = (uint32_t)(kDecWBytes + X_BYTES);
+      // bytes TMA moves per stage: the weights at their packed size
+      const uint32_t stage_tx = (uint32_t)(kDecWBytes * wf_bits(WF) / 8 + X_BYTES);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -435,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      const uint32_t idesc = idesc_e4m3_f32(BM, p.np);
+      const uint32_t idesc = idesc_f8f6f4_f32(BM, p.np, wf_mma(WF), kMmaE4M3);  // A = weights
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -463,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = sw128_kmajor_desc(smem_u32(sX + stage * X_BYTES));
           #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)
-            mma_e4m3(d, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
+            mma_f8f6f4(d, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
                      (kb > u.kb0 || kk > 0) ? 1u : 0u);
           mma_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -546,10 +557,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ----------------------------------------------------------------------------
 // BN: tile width (MMA N), 256 or 128; each CTA of the pair loads BN / 2
 // weight rows.
-template <int STAGES, bool F32OUT, int BN>
+template <int STAGES, bool F32OUT, int BN, int WF = 0>
 struct PairCfg {
   static constexpr int A_BYTES = BM * BK;
   static constexpr int B_BYTES = (BN / 2) * BK;
+  static constexpr int B_TX = B_BYTES * wf_bits(WF) / 8;  // weight bytes TMA moves (packed size)
   static constexpr int EPI_BUF = 32 * 128;
   static constexpr int TMEM_COLS = 2 * BN;  // two accumulators (a power of two >= 32)
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + kEpiWarps * EPI_BUF +
@@ -557,11 +569,11 @@ struct PairCfg {
   static_assert(SMEM <= 232448, "shared memory");
 };
 
-template <int STAGES, bool F32OUT, int BN>
+template <int STAGES, bool F32OUT, int BN, int WF>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     ptpc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
-  using C = PairCfg<STAGES, F32OUT, BN>;
+  using C = PairCfg<STAGES, F32OUT, BN, WF>;
   constexpr int HALF_N = BN / 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -623,7 +635,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (sc.next(p, u)) {
         const int b_row = u.n * BN + (int)rank * HALF_N;
         for (; pre < STAGES && u.kb0 + pre < u.kb1; ++pre) {
-          if (leader) mbar_arrive_expect_tx(&full[pre], 2 * (C::A_BYTES + C::B_BYTES));
+          if (leader) mbar_arrive_expect_tx(&full[pre], 2 * (C::A_BYTES + C::B_TX));
           tma_load_2d_pair(sB + pre * C::B_BYTES, &tmB, mapa_shared(&full[pre], 0), (u.kb0 + pre) * BK, b_row,
                            polB);
         }
@@ -641,7 +653,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
-            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (C::A_BYTES + C::B_BYTES));
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (C::A_BYTES + C::B_TX));
             tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, lead_full, kb * BK, b_row, polB);
           }
           tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, lead_full, kb * BK, a_row, polA);
@@ -663,7 +675,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (leader && elect_one()) {
-      constexpr uint32_t idesc = idesc_e4m3_f32(2 * BM, BN);
+      constexpr uint32_t idesc = idesc_f8f6f4_f32(2 * BM, BN, kMmaE4M3, wf_mma(WF));  // B = weights
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -691,7 +703,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint64_t bd = sw128_kmajor_desc(smem_u32(sB + stage * C::B_BYTES));
           #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk)
-            mma_e4m3_pair(d, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
+            mma_f8f6f4_pair(d, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc,
                           (kb > u.kb0 || kk > 0) ? 1u : 0u);
           mma_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == STAGES) {
@@ -831,11 +843,23 @@ bool make_map_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint6
   return true;
 }
 
+// Tensor map of the weight codes Wq [Co, Ci]: one byte per code (E4M3), or
+// packed 4-bit / 6-bit codes that TMA unpacks into 16-byte chunks of 16 codes
+// in shared memory (box inner extent 128 codes, rows 32-byte aligned).
+bool make_weight_map(CUtensorMap *m, const GemmProblem &pr, uint32_t rows) {
+  if (pr.wfmt == 0)
+    return make_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Wq_t, pr.Ci, pr.Co, pr.Ci, BK, rows,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+  const CUtensorMapDataType dt =
+      pr.wfmt == 1 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_16U6_ALIGN16B;
+  return make_map_2d(m, dt, pr.Wq_t, pr.Ci, pr.Co, (uint64_t)pr.Ci * wf_bits(pr.wfmt) / 8, BK, rows,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 bool make_maps(const GemmProblem &pr, uint32_t b_rows, CUtensorMap *tmA, CUtensorMap *tmB, CUtensorMap *tmC) {
   if (!make_map_2d(tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Xq, pr.Ci, pr.T, pr.Ci, BK, BM,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_2d(tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Wq_t, pr.Ci, pr.Co, pr.Ci, BK, b_rows,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_weight_map(tmB, pr, b_rows))
     return false;
   if (pr.f32_out)
     return make_map_2d(tmC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.out, pr.Co, pr.T, (uint64_t)pr.Co * 4, 32, 32,
@@ -850,11 +874,11 @@ constexpr int pair_stages() {
   return BN == 256 ? 6 : 8;
 }
 
-template <bool F32OUT, int BN>
+template <bool F32OUT, int BN, int WF = 0>
 void set_pair_smem() {
-  cudaFuncSetAttribute(ptpc_gemm_pair_kernel<pair_stages<BN>(), F32OUT, BN>,
+  cudaFuncSetAttribute(ptpc_gemm_pair_kernel<pair_stages<BN>(), F32OUT, BN, WF>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)PairCfg<pair_stages<BN>(), F32OUT, BN>::SMEM);
+                       (int)PairCfg<pair_stages<BN>(), F32OUT, BN, WF>::SMEM);
 }
 
 // CTA pairs of the BN-wide pair kernel that can be resident at once.
@@ -865,7 +889,7 @@ int pair_resident(int sms) {
   q.blockDim = dim3(kThreads);
   q.dynamicSmemBytes = PairCfg<pair_stages<BN>(), false, BN>::SMEM;
   int ncl = 0;
-  if (cudaOccupancyMaxActiveClusters(&ncl, ptpc_gemm_pair_kernel<pair_stages<BN>(), false, BN>, &q) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveClusters(&ncl, ptpc_gemm_pair_kernel<pair_stages<BN>(), false, BN, 0>, &q) != cudaSuccess ||
       ncl <= 0)
     ncl = sms / 2;
   cudaGetLastError();
@@ -921,22 +945,28 @@ const DeviceInfo &device_info() {
   if (!ready[dev].load(std::memory_order_relaxed)) {
     int v = 0;
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0) d.sms = v;
-    cudaFuncSetAttribute(ptpc_gemm_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kDecSmemMax);
-    cudaFuncSetAttribute(ptpc_gemm_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kDecSmemMax);
+    for (auto k : {ptpc_gemm_decode_kernel<false, 0>, ptpc_gemm_decode_kernel<true, 0>,
+                   ptpc_gemm_decode_kernel<false, 1>, ptpc_gemm_decode_kernel<false, 2>,
+                   ptpc_gemm_decode_kernel<false, 3>})
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecSmemMax);
     set_pair_smem<false, 256>();
     set_pair_smem<true, 256>();
     set_pair_smem<false, 128>();
     set_pair_smem<true, 128>();
+    set_pair_smem<false, 256, 1>();
+    set_pair_smem<false, 128, 1>();
+    set_pair_smem<false, 256, 2>();
+    set_pair_smem<false, 128, 2>();
+    set_pair_smem<false, 256, 3>();
+    set_pair_smem<false, 128, 3>();
     // the pair kernel's cluster size is compiled in (__cluster_dims__)
     d.pair_clusters = pair_resident<256>(d.sms);
     d.pair_clusters128 = pair_resident<128>(d.sms);
     // the decode kernel takes its cluster size at launch; ask for the largest
     // shared-memory footprint it launches with
     for (int size = 2; size <= 8; size *= 2) {
-      const int a = max_clusters(ptpc_gemm_decode_kernel<false>, d.sms, size, kDecSmemMax);
-      const int b = max_clusters(ptpc_gemm_decode_kernel<true>, d.sms, size, kDecSmemMax);
+      const int a = max_clusters(ptpc_gemm_decode_kernel<false, 0>, d.sms, size, kDecSmemMax);
+      const int b = max_clusters(ptpc_gemm_decode_kernel<true, 0>, d.sms, size, kDecSmemMax);
       d.dec_clusters[size] = std::min(a, b);
     }
     d.ready = true;
@@ -1141,11 +1171,11 @@ cudaError_t launch(Kernel kernel, int grid, size_t smem, const CUtensorMap &tmA,
   return cudaLaunchKernelEx(&cfg, kernel, tmA, tmB, tmC, gp);
 }
 
-template <bool F32OUT, int BN>
+template <bool F32OUT, int BN, int WF = 0>
 cudaError_t launch_pair(int grid, const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmC,
                         const GemmParams &gp, bool pdl, cudaStream_t st) {
-  return launch(ptpc_gemm_pair_kernel<pair_stages<BN>(), F32OUT, BN>, grid,
-                PairCfg<pair_stages<BN>(), F32OUT, BN>::SMEM, tmA, tmB, tmC, gp, pdl, st);
+  return launch(ptpc_gemm_pair_kernel<pair_stages<BN>(), F32OUT, BN, WF>, grid,
+                PairCfg<pair_stages<BN>(), F32OUT, BN, WF>::SMEM, tmA, tmB, tmC, gp, pdl, st);
 }
 
 }  // namespace
@@ -1179,27 +1209,42 @@ cudaError_t launch_scaled_gemm(const GemmProblem &pr, cudaStream_t st) {
   gp.ws = pr.ws;
   gp.out = pr.out;
   gp.status = pr.status;
+  if (pr.f32_out && pr.wfmt != 0) return cudaErrorInvalidValue;  // the naive path is E4M3 only
   if (!pl.pair) {
     CUtensorMap tmW, tmX;
-    if (!make_map_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Wq_t, pr.Ci, pr.Co, pr.Ci, BK, BM,
-                     CU_TENSOR_MAP_SWIZZLE_128B) ||
+    if (!make_weight_map(&tmW, pr, BM) ||
         !make_map_2d(&tmX, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Xq, pr.Ci, pr.T, pr.Ci, BK, pl.np,
                      CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
     const size_t smem = dec_smem_bytes(pl.np, pl.stages);
-    return pr.f32_out ? launch_decode(ptpc_gemm_decode_kernel<true>, pl.ctas, pl.ksplit, smem, tmW, tmX, gp,
-                                      pr.pdl, st)
-                      : launch_decode(ptpc_gemm_decode_kernel<false>, pl.ctas, pl.ksplit, smem, tmW, tmX, gp,
-                                      pr.pdl, st);
+    switch (pr.f32_out ? -1 : pr.wfmt) {
+      case -1: return launch_decode(ptpc_gemm_decode_kernel<true, 0>, pl.ctas, pl.ksplit, smem, tmW, tmX, gp, pr.pdl, st);
+      case 1: return launch_decode(ptpc_gemm_decode_kernel<false, 1>, pl.ctas, pl.ksplit, smem, tmW, tmX, gp, pr.pdl, st);
+      case 2: return launch_decode(ptpc_gemm_decode_kernel<false, 2>, pl.ctas, pl.ksplit, smem, tmW, tmX, gp, pr.pdl, st);
+      case 3: return launch_decode(ptpc_gemm_decode_kernel<false, 3>, pl.ctas, pl.ksplit, smem, tmW, tmX, gp, pr.pdl, st);
+      default: return launch_decode(ptpc_gemm_decode_kernel<false, 0>, pl.ctas, pl.ksplit, smem, tmW, tmX, gp, pr.pdl, st);
+    }
   }
   CUtensorMap tmA, tmB, tmC;
   if (!make_maps(pr, pl.bn / 2, &tmA, &tmB, &tmC)) return cudaErrorInvalidValue;
   const int grid = 2 * pl.ctas;
-  if (pl.bn == 128)
-    return pr.f32_out ? launch_pair<true, 128>(grid, tmA, tmB, tmC, gp, pr.pdl, st)
-                      : launch_pair<false, 128>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
-  return pr.f32_out ? launch_pair<true, 256>(grid, tmA, tmB, tmC, gp, pr.pdl, st)
-                    : launch_pair<false, 256>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
+  if (pr.f32_out)
+    return pl.bn == 128 ? launch_pair<true, 128>(grid, tmA, tmB, tmC, gp, pr.pdl, st)
+                        : launch_pair<true, 256>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
+  if (pl.bn == 128) {
+    switch (pr.wfmt) {
+      case 1: return launch_pair<false, 128, 1>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
+      case 2: return launch_pair<false, 128, 2>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
+      case 3: return launch_pair<false, 128, 3>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
+      default: return launch_pair<false, 128, 0>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
+    }
+  }
+  switch (pr.wfmt) {
+    case 1: return launch_pair<false, 256, 1>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
+    case 2: return launch_pair<false, 256, 2>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
+    case 3: return launch_pair<false, 256, 3>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
+    default: return launch_pair<false, 256, 0>(grid, tmA, tmB, tmC, gp, pr.pdl, st);
+  }
 }
 
 }  // namespace ptpc

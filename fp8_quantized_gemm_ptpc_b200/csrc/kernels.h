@@ -11,11 +11,20 @@ namespace ptpc {
 // Quantisers (quant.cu).
 // ldx: row pitch of X in elements (>= Ci, multiple of 8).
 cudaError_t launch_quant_act(const void *X, int T, int Ci, int64_t ldx, uint8_t *Xq, float *xs, cudaStream_t st);
+// Row split over tensor-parallel ranks: the slice's row maxima (fp32 [T]),
+// and the quantisation of the slice with given (combined) row maxima.
+cudaError_t launch_row_amax(const void *X, int T, int Ci, int64_t ldx, float *amax, cudaStream_t st);
+cudaError_t launch_quant_act_amax(const void *X, int T, int Ci, int64_t ldx, const float *amax, uint8_t *Xq,
+                                  float *xs, cudaStream_t st);
 cudaError_t launch_quant_act_per_tensor(const void *X, int T, int Ci, int64_t ldx, uint8_t *Xq, float *xs,
                                         uint32_t *amax_slot, cudaStream_t st);
 // col_amax: Co + 1 32-bit words of scratch.
 cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, float *w_scale, uint32_t *col_amax,
                                 bool per_tensor, cudaStream_t st);
+// Sub-byte per-output-channel weight quantisation: fmt 1 = E2M1 (FP4),
+// 2 = E2M3, 3 = E3M2 (FP6); Wp [Co, Ci * bits / 8] packed along K; Ci % 128 == 0.
+cudaError_t launch_quant_weight_sub(const void *W, int Ci, int Co, int fmt, uint8_t *Wp, float *w_scale,
+                                    uint32_t *col_amax, cudaStream_t st);
 cudaError_t launch_apply_scales(const float *y, const float *xs, const float *ws, int T, int Co, void *out,
                                 cudaStream_t st);
 
@@ -30,6 +39,7 @@ struct GemmProblem {
   bool f32_out;           // unscaled fp32 output (naive step 1)
   uint32_t *status;       // device status word
   bool pdl;               // launch as a programmatic dependent of the previous kernel
+  int wfmt;               // weight format: 0 E4M3, 1 E2M1, 2 E2M3, 3 E3M2 (packed along Ci)
 };
 
 cudaError_t launch_scaled_gemm(const GemmProblem &p, cudaStream_t st);

@@ -20,6 +20,8 @@
 #include <algorithm>
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp6.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
@@ -40,7 +42,9 @@ struct GroupScale {
   int mode;
 };
 
-__device__ __forceinline__ GroupScale group_scale_from_amax_bits(uint32_t amax_bits16) {
+// Scale of a group from its largest magnitude (bf16 bits): amax / fmax, the
+// format's largest finite value (448 for E4M3).
+__device__ __forceinline__ GroupScale group_scale_from_amax_bits(uint32_t amax_bits16, float fmax = 448.0f) {
   GroupScale g;
   const float amax = __uint_as_float(amax_bits16 << 16);
   if (amax == 0.0f) {
@@ -48,7 +52,7 @@ __device__ __forceinline__ GroupScale group_scale_from_amax_bits(uint32_t amax_b
     g.r = 1.0f;
     g.mode = kZeroGroup;
   } else {
-    g.s = __fdiv_rn(amax, 448.0f);
+    g.s = __fdiv_rn(amax, fmax);
     g.r = __frcp_rn(g.s);
     g.mode = g.s >= kFastPathMinScale ? kFast : kSlow;
   }
@@ -166,14 +170,19 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *p) { return __ldcs(p); }
 // load, |x| max, group reduction (warp shuffle, then shared memory across
 // the group's warps), then quantise from registers and store 8 codes per
 // vector.  R = blockDim / P rows per CTA.
-// PER_TENSOR: the group scale comes from a tensor-wide amax computed by
-// amax_kernel (the per-tensor comparison path) instead of the row.
+// SRC: where the group scale's maximum comes from: kAmaxRow the row itself;
+// kAmaxTensor a tensor-wide maximum computed by amax_kernel (the per-tensor
+// comparison path, bf16 magnitude bits); kAmaxGiven an fp32 maximum per row
+// supplied by the caller (the row split over tensor-parallel ranks).
 // ----------------------------------------------------------------------------
-template <int V, bool PER_TENSOR>
+enum : int { kAmaxRow = 0, kAmaxTensor = 1, kAmaxGiven = 2 };
+
+template <int V, int SRC>
 __global__ void __launch_bounds__(V >= 16 ? 512 : 1024) quant_act_kernel(const uint4 *__restrict__ X, int T, int nvec,
                                                          int64_t ldv, uint8_t *__restrict__ Xq,
                                                          float *__restrict__ xs, int P,
-                                                         const uint32_t *__restrict__ tensor_amax) {
+                                                         const uint32_t *__restrict__ tensor_amax,
+                                                         const float *__restrict__ given_amax) {
   __shared__ uint32_t red[32];
   griddep_launch_dependents();
   // Launched as a programmatic dependent: X (and the buffers written below)
@@ -200,8 +209,10 @@ __global__ void __launch_bounds__(V >= 16 ? 512 : 1024) quant_act_kernel(const u
     }
   }
   uint32_t amax_bits;
-  if constexpr (PER_TENSOR) {
+  if constexpr (SRC == kAmaxTensor) {
     amax_bits = *tensor_amax;
+  } else if constexpr (SRC == kAmaxGiven) {
+    amax_bits = active ? __float_as_uint(given_amax[row]) >> 16 : 0u;
   } else {
     #pragma unroll
     for (int i = 0; i < V; ++i) m = absmax_bits(m, v[i]);
@@ -239,11 +250,12 @@ __global__ void __launch_bounds__(V >= 16 ? 512 : 1024) quant_act_kernel(const u
 
 // Rows too long for registers: two passes over the row (the second read is
 // normally served from L2).  One CTA per row.
-template <bool PER_TENSOR>
+template <int SRC>
 __global__ void __launch_bounds__(1024) quant_act_long_kernel(const uint4 *__restrict__ X, int T, int nvec,
                                                               int64_t ldv, uint8_t *__restrict__ Xq,
                                                               float *__restrict__ xs,
-                                                              const uint32_t *__restrict__ tensor_amax) {
+                                                              const uint32_t *__restrict__ tensor_amax,
+                                                              const float *__restrict__ given_amax) {
   __shared__ uint32_t red[32];
   __shared__ uint32_t row_amax;
   griddep_launch_dependents();
@@ -251,8 +263,10 @@ __global__ void __launch_bounds__(1024) quant_act_long_kernel(const uint4 *__res
   const int64_t row = blockIdx.x;
   const uint4 *xr = X + row * ldv;
   uint32_t amax_bits;
-  if constexpr (PER_TENSOR) {
+  if constexpr (SRC == kAmaxTensor) {
     amax_bits = *tensor_amax;
+  } else if constexpr (SRC == kAmaxGiven) {
+    amax_bits = __float_as_uint(given_amax[row]) >> 16;
   } else {
     uint32_t m = 0;
     for (int j = threadIdx.x; j < nvec; j += blockDim.x) m = absmax_bits(m, xr[j]);
@@ -347,10 +361,10 @@ __global__ void broadcast_amax_kernel(const uint32_t *__restrict__ src, uint32_t
 // all-zero column, so pass 2 needs no division.
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) weight_scales_kernel(uint32_t *__restrict__ col_amax,
-                                                            float *__restrict__ w_scale, int Co) {
+                                                            float *__restrict__ w_scale, int Co, float fmax) {
   const int o = blockIdx.x * blockDim.x + threadIdx.x;
   if (o >= Co) return;
-  const GroupScale g = group_scale_from_amax_bits(col_amax[o]);
+  const GroupScale g = group_scale_from_amax_bits(col_amax[o], fmax);
   w_scale[o] = g.s;
   col_amax[o] = g.mode == kZeroGroup ? 0u : __float_as_uint(g.r);
 }
@@ -453,6 +467,148 @@ __global__ void __launch_bounds__(256) quant_weight_t_kernel(const uint4 *__rest
 }
 
 // ----------------------------------------------------------------------------
+// Sub-byte weight formats: FP4 E2M1 and FP6 E2M3 / E3M2 (the OCP MX element
+// types that tcgen05.mma.kind::f8f6f4 reads), one scale per output channel
+// s = amax / max_format, codes packed along K the way TMA's packed 4- and
+// 6-bit tensor types read them: FP4 two codes a byte (the even K position in
+// the low nibble), FP6 code j of every 16 at bits [6j, 6j + 6) of 12 bytes
+// read as a little-endian integer.  The quotient is the activation
+// quantiser's divide-free one (exhaustively equal in code to the IEEE
+// quotient for these divisors too), computed on x as is with -r, which gives
+// -q, so the sign bits of the finished codes are flipped once per word.
+//
+// A CTA quantises a 128 (K) x 64 (channel) tile: thread (cv, kq) converts K
+// rows 8 kq .. 8 kq + 7 of the 8 channels of vector cv into 8 codes per
+// channel (4 bytes of FP4 or 6 of FP6), placed in a shared tile [channel][K
+// bytes], which is written out as 16-byte row chunks (the bf16 reads run
+// along Co, the packed writes along Ci; both coalesced).  Ci % 128 == 0.
+// ----------------------------------------------------------------------------
+constexpr int kSbThreads = 128;
+
+template <int WF>
+struct SubFmt;
+template <>
+struct SubFmt<1> {  // E2M1
+  static constexpr int bits = 4;
+  static constexpr float fmax = 6.0f;
+};
+template <>
+struct SubFmt<2> {  // E2M3
+  static constexpr int bits = 6;
+  static constexpr float fmax = 7.5f;
+};
+template <>
+struct SubFmt<3> {  // E3M2
+  static constexpr int bits = 6;
+  static constexpr float fmax = 28.0f;
+};
+
+// Codes of two fp32 values (a: even K position, b: odd) in the format, a in
+// the low nibble (FP4) or the low byte (FP6).
+template <int WF>
+__device__ __forceinline__ uint32_t cvt_sub_pair(float a, float b) {
+  if constexpr (WF == 1)
+    return (uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(a, b), __NV_E2M1, cudaRoundNearest) & 0xFFu;
+  else if constexpr (WF == 2)
+    return (uint32_t)__nv_cvt_float2_to_fp6x2(make_float2(a, b), __NV_E2M3, cudaRoundNearest);
+  else
+    return (uint32_t)__nv_cvt_float2_to_fp6x2(make_float2(a, b), __NV_E3M2, cudaRoundNearest);
+}
+
+// Eight consecutive-K values of one channel (fp32 bits) -> packed codes:
+// FP4 in the low 32 bits, FP6 in the low 48.  `flip`: the values are -q.
+template <int WF>
+__device__ __forceinline__ uint64_t pack8_sub(const float (&q)[8], bool flip) {
+  uint64_t acc = 0;
+  #pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const uint32_t c = cvt_sub_pair<WF>(q[2 * p], q[2 * p + 1]);
+    if constexpr (WF == 1) {
+      acc |= (uint64_t)c << (8 * p);
+    } else {
+      acc |= (uint64_t)(c & 0x3Fu) << (12 * p);
+      acc |= (uint64_t)((c >> 8) & 0x3Fu) << (12 * p + 6);
+    }
+  }
+  if (flip) acc ^= (WF == 1) ? 0x88888888ull : 0x820820820820ull;
+  return acc;
+}
+
+template <int WF>
+__global__ void __launch_bounds__(kSbThreads) quant_weight_sub_kernel(const uint4 *__restrict__ W, int Ci, int Co,
+                                                                     const uint32_t *__restrict__ col_rcp,
+                                                                     uint8_t *__restrict__ Wp,
+                                                                     const float *__restrict__ w_scale) {
+  constexpr int B = SubFmt<WF>::bits;
+  constexpr int RB = kTK * B / 8;      // packed bytes of 128 K codes: 64 (FP4) or 96 (FP6)
+  constexpr int PITCH = RB + 16;
+  constexpr int CB = 8 * B / 8;        // packed bytes of 8 codes: 4 or 6
+  __shared__ __align__(16) uint8_t tile[kTO][PITCH];
+  const int o0 = blockIdx.x * kTO;
+  const int k0 = blockIdx.y * kTK;
+  const int ncv = Co / 8;
+  const int cv = threadIdx.x & 7;
+  const int kq = threadIdx.x >> 3;     // K rows 8 kq .. 8 kq + 7
+  const int ocol = o0 + cv * 8;
+  const bool col_ok = ocol < Co;       // Co % 16 == 0: the 8 columns are valid together
+  uint4 v[8];
+  #pragma unroll
+  for (int r = 0; r < 8; ++r)
+    v[r] = col_ok ? ld_stream(W + (int64_t)(k0 + 8 * kq + r) * ncv + (ocol >> 3)) : make_uint4(0u, 0u, 0u, 0u);
+  #pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float s = 1.0f, rc = 0.0f;
+    if (col_ok) {
+      s = __ldg(w_scale + ocol + c);
+      rc = __uint_as_float(__ldg(col_rcp + ocol + c));
+    }
+    float x[8];
+    #pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const uint32_t w2 = (c < 2) ? v[r].x : (c < 4) ? v[r].y : (c < 6) ? v[r].z : v[r].w;
+      x[r] = (c & 1) ? __uint_as_float(w2 & 0xFFFF0000u) : __uint_as_float(w2 << 16);
+    }
+    uint64_t packed = 0;
+    if (__float_as_uint(rc) == 0u) {
+      packed = 0;  // all-zero column (or a column past Co)
+    } else if (s >= kFastPathMinScale) {
+      float q[8];
+      #pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const float nq0 = __fmul_rn(x[r], -rc);
+        const float e = __fmaf_rn(nq0, s, x[r]);
+        q[r] = __fmaf_rn(e, -rc, nq0);
+      }
+      packed = pack8_sub<WF>(q, true);
+    } else {
+      float q[8];
+      #pragma unroll
+      for (int r = 0; r < 8; ++r) q[r] = __fdiv_rn(x[r], s);
+      packed = pack8_sub<WF>(q, false);
+    }
+    uint8_t *dst = &tile[cv * 8 + c][kq * CB];
+    if constexpr (CB == 4) {
+      *reinterpret_cast<uint32_t *>(dst) = (uint32_t)packed;
+    } else {
+      reinterpret_cast<uint16_t *>(dst)[0] = (uint16_t)packed;
+      reinterpret_cast<uint16_t *>(dst)[1] = (uint16_t)(packed >> 16);
+      reinterpret_cast<uint16_t *>(dst)[2] = (uint16_t)(packed >> 32);
+    }
+  }
+  __syncthreads();
+  constexpr int CHUNKS = RB / 16;      // 16-byte chunks per channel row
+  const int64_t row_bytes = (int64_t)Ci * B / 8;
+  for (int i = threadIdx.x; i < kTO * CHUNKS; i += kSbThreads) {
+    const int orow = i / CHUNKS;
+    const int ch = i - orow * CHUNKS;
+    const int o = o0 + orow;
+    if (o < Co)
+      *reinterpret_cast<uint4 *>(Wp + (int64_t)o * row_bytes + (int64_t)k0 * B / 8 + ch * 16) =
+          *reinterpret_cast<const uint4 *>(&tile[orow][ch * 16]);
+  }
+}
+
+// ----------------------------------------------------------------------------
 // Naive two-step path, step 2: out = bf16((y * x_scale[t]) * w_scale[o]).
 // Each thread handles 8 consecutive outputs (two 16-byte fp32 loads, one
 // 16-byte bf16 store).
@@ -530,30 +686,58 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, cudaStream
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-template <bool PT>
+template <int SRC>
 cudaError_t launch_act(const void *X, int T, int Ci, int64_t ldx, uint8_t *Xq, float *xs,
-                       const uint32_t *tensor_amax, cudaStream_t st) {
+                       const uint32_t *tensor_amax, const float *given_amax, cudaStream_t st) {
   const int nvec = Ci / 8;
   const int64_t ldv = ldx / 8;
   const ActPlan p = plan_act(nvec);
   const uint4 *Xv = static_cast<const uint4 *>(X);
-  if (p.V == 0) return launch_pdl(quant_act_long_kernel<PT>, T, 1024, st, Xv, T, nvec, ldv, Xq, xs, tensor_amax);
+  if (p.V == 0)
+    return launch_pdl(quant_act_long_kernel<SRC>, T, 1024, st, Xv, T, nvec, ldv, Xq, xs, tensor_amax, given_amax);
   const int grid = (T + p.R - 1) / p.R;
   const int block = p.P * p.R;
   switch (p.V) {
-    case 1: return launch_pdl(quant_act_kernel<1, PT>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax);
-    case 2: return launch_pdl(quant_act_kernel<2, PT>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax);
-    case 4: return launch_pdl(quant_act_kernel<4, PT>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax);
-    case 8: return launch_pdl(quant_act_kernel<8, PT>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax);
-    default: return launch_pdl(quant_act_kernel<16, PT>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax);
+    case 1: return launch_pdl(quant_act_kernel<1, SRC>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax, given_amax);
+    case 2: return launch_pdl(quant_act_kernel<2, SRC>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax, given_amax);
+    case 4: return launch_pdl(quant_act_kernel<4, SRC>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax, given_amax);
+    case 8: return launch_pdl(quant_act_kernel<8, SRC>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax, given_amax);
+    default: return launch_pdl(quant_act_kernel<16, SRC>, grid, block, st, Xv, T, nvec, ldv, Xq, xs, p.P, tensor_amax, given_amax);
   }
 }
 
+// ----------------------------------------------------------------------------
+// Row maxima of a T x Ci bf16 slice (fp32, exact): one warp per row, 8 rows
+// per CTA, 16-byte streaming loads, warp reduction.  The first half of the
+// row-split quantisation (the second is quant_act_kernel<., kAmaxGiven>).
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) row_amax_kernel(const uint4 *__restrict__ X, int T, int nvec, int64_t ldv,
+                                                       float *__restrict__ amax) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= T) return;
+  const uint4 *xr = X + (int64_t)row * ldv;
+  uint32_t m = 0;
+  for (int j = lane; j < nvec; j += 32) m = absmax_bits(m, ld_stream(xr + j));
+  m = __reduce_max_sync(0xffffffffu, fold_halves(m));
+  if (lane == 0) amax[row] = __uint_as_float(m << 16);
+}
 
 }  // namespace
 
 cudaError_t launch_quant_act(const void *X, int T, int Ci, int64_t ldx, uint8_t *Xq, float *xs, cudaStream_t st) {
-  return launch_act<false>(X, T, Ci, ldx, Xq, xs, nullptr, st);
+  return launch_act<kAmaxRow>(X, T, Ci, ldx, Xq, xs, nullptr, nullptr, st);
+}
+
+cudaError_t launch_quant_act_amax(const void *X, int T, int Ci, int64_t ldx, const float *amax, uint8_t *Xq,
+                                  float *xs, cudaStream_t st) {
+  return launch_act<kAmaxGiven>(X, T, Ci, ldx, Xq, xs, nullptr, amax, st);
+}
+
+cudaError_t launch_row_amax(const void *X, int T, int Ci, int64_t ldx, float *amax, cudaStream_t st) {
+  return launch_pdl(row_amax_kernel, (T + 7) / 8, 256, st, static_cast<const uint4 *>(X), T, Ci / 8, ldx / 8, amax);
 }
 
 cudaError_t launch_quant_act_per_tensor(const void *X, int T, int Ci, int64_t ldx, uint8_t *Xq, float *xs,
@@ -565,7 +749,7 @@ cudaError_t launch_quant_act_per_tensor(const void *X, int T, int Ci, int64_t ld
   if (grid < 1) grid = 1;
   amax_kernel<<<grid, 512, 0, st>>>(static_cast<const uint4 *>(X), T, Ci / 8, ldx / 8, amax_slot);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = launch_act<true>(X, T, Ci, ldx, Xq, xs, amax_slot, st)) != cudaSuccess) return e;
+  if ((e = launch_act<kAmaxTensor>(X, T, Ci, ldx, Xq, xs, amax_slot, nullptr, st)) != cudaSuccess) return e;
   // the workspace's scratch word is left zero for the next user
   return cudaMemsetAsync(amax_slot, 0, sizeof(uint32_t), st);
 }
@@ -595,10 +779,39 @@ cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, fl
     col_amax_kernel<<<dim3(gx, slabs), kColThreads * kColWarps, 0, st>>>(Wv, Ci, Co, rows_per_cta, col_amax);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  weight_scales_kernel<<<(Co + 255) / 256, 256, 0, st>>>(col_amax, w_scale, Co);
+  weight_scales_kernel<<<(Co + 255) / 256, 256, 0, st>>>(col_amax, w_scale, Co, 448.0f);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 grid((Co + kTO - 1) / kTO, (Ci + kTK - 1) / kTK);
   quant_weight_t_kernel<<<grid, 256, 0, st>>>(Wv, Ci, Co, col_amax, Wq_t, w_scale);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // the workspace's scratch words are left zero for the next user
+  return cudaMemsetAsync(col_amax, 0, sizeof(uint32_t) * ((size_t)Co + 1), st);
+}
+
+cudaError_t launch_quant_weight_sub(const void *W, int Ci, int Co, int fmt, uint8_t *Wp, float *w_scale,
+                                    uint32_t *col_amax, cudaStream_t st) {
+  if (fmt < 1 || fmt > 3 || Ci % kTK != 0) return cudaErrorInvalidValue;
+  cudaError_t e;
+  const uint4 *Wv = static_cast<const uint4 *>(W);
+  if ((e = cudaMemsetAsync(col_amax, 0, sizeof(uint32_t) * (size_t)Co, st)) != cudaSuccess) return e;
+  const int ncv = Co / 8;
+  const int gx = (ncv + kColThreads - 1) / kColThreads;
+  int slabs = std::max(1, (num_sms() * 4 + gx - 1) / gx);
+  int rows_per_cta = (Ci + slabs - 1) / slabs;
+  rows_per_cta = std::max(rows_per_cta, 64);
+  slabs = (Ci + rows_per_cta - 1) / rows_per_cta;
+  col_amax_kernel<<<dim3(gx, slabs), kColThreads * kColWarps, 0, st>>>(Wv, Ci, Co, rows_per_cta, col_amax);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const float fmax = fmt == 1 ? SubFmt<1>::fmax : fmt == 2 ? SubFmt<2>::fmax : SubFmt<3>::fmax;
+  weight_scales_kernel<<<(Co + 255) / 256, 256, 0, st>>>(col_amax, w_scale, Co, fmax);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const dim3 grid((Co + kTO - 1) / kTO, Ci / kTK);
+  if (fmt == 1)
+    quant_weight_sub_kernel<1><<<grid, kSbThreads, 0, st>>>(Wv, Ci, Co, col_amax, Wp, w_scale);
+  else if (fmt == 2)
+    quant_weight_sub_kernel<2><<<grid, kSbThreads, 0, st>>>(Wv, Ci, Co, col_amax, Wp, w_scale);
+  else
+    quant_weight_sub_kernel<3><<<grid, kSbThreads, 0, st>>>(Wv, Ci, Co, col_amax, Wp, w_scale);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // the workspace's scratch words are left zero for the next user
   return cudaMemsetAsync(col_amax, 0, sizeof(uint32_t) * ((size_t)Co + 1), st);

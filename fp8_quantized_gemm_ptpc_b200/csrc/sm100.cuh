@@ -162,8 +162,9 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, E4M3 x E4M3 -> fp32, one CTA.
-__device__ __forceinline__ void mma_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 (operand formats from the
+// instruction descriptor) -> fp32, one CTA.
+__device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -222,13 +223,21 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor: dense E4M3 x E4M3 -> fp32, both operands K-major.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+// Operand formats of tcgen05.mma.kind::f8f6f4 (instruction-descriptor codes).
+constexpr uint32_t kMmaE4M3 = 0, kMmaE2M3 = 3, kMmaE3M2 = 4, kMmaE2M1 = 5;
+
+// Instruction descriptor: dense kind::f8f6f4 MMA with fp32 accumulation, both
+// operands K-major; afmt / bfmt are the operand formats above.
+__host__ __device__ constexpr uint32_t idesc_f8f6f4_f32(int M, int N, uint32_t afmt, uint32_t bfmt) {
   return (1u << 4)                        // D format: fp32
-         | (0u << 7)                      // A format: E4M3
-         | (0u << 10)                     // B format: E4M3
+         | (afmt << 7)                    // A format
+         | (bfmt << 10)                   // B format
          | ((uint32_t)(N >> 3) << 17)     // N / 8
          | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return idesc_f8f6f4_f32(M, N, kMmaE4M3, kMmaE4M3);
 }
 
 }  // namespace ptpc
@@ -295,8 +304,8 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 }
 
 // D[tmem of both CTAs] (+)= A[smem of both CTAs] * B[smem of both CTAs]^T,
-// E4M3 x E4M3 -> fp32, issued by one thread of the pair's first CTA.
-__device__ __forceinline__ void mma_e4m3_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+// kind::f8f6f4 -> fp32, issued by one thread of the pair's first CTA.
+__device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                               uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"

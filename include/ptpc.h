@@ -76,6 +76,20 @@ typedef enum {
     PTPC_ERR_NOT_IMPLEMENTED = 8
 } ptpc_status;
 
+/* Weight formats.  E4M3 is the PTPC-FP8 format of the entry points above;
+ * the others are the sub-byte formats of FP4-FP7 runtime weight quantisation
+ * (the llminfo.tech summary "Running LLMs at custom floating-points
+ * (near-lossless FP6)": FP6-LLM extended to FP4-FP7 with per-channel
+ * quantisation), taken as the OCP MX element types that the tensor cores
+ * read natively.  Every format keeps one fp32 scale per output channel,
+ * amax / (largest value of the format), and per-token FP8 activations. */
+typedef enum {
+    PTPC_WFMT_E4M3 = 0,   /* FP8, 1 byte a code, max 448 */
+    PTPC_WFMT_E2M1 = 1,   /* FP4, max 6; two codes a byte, even K position in the low nibble */
+    PTPC_WFMT_E2M3 = 2,   /* FP6, max 7.5; 16 codes in 12 bytes, code j at bits [6j, 6j+6) little-endian */
+    PTPC_WFMT_E3M2 = 3    /* FP6, max 28; packed like E2M3 */
+} ptpc_weight_format;
+
 /* Operation ids for ptpc_workspace_size. */
 typedef enum {
     PTPC_OP_QUANTIZE_WEIGHTS = 1,
@@ -95,6 +109,28 @@ typedef enum {
  * Codes and scales are bit-exact functions of X (see the conventions above). */
 PTPC_API int ptpc_quantize_activations(const void *X_dev, int64_t T, int64_t Ci, int64_t ldx,
                               uint8_t *Xq_dev, float *x_scale_dev, void *stream);
+
+/* Tensor parallelism with the input channels split over ranks (a
+ * row-parallel linear, as in the page's TP = 2 evaluation setup in its
+ * benchmark section): a rank holds a column slice X_r [T, Ci_r] of every
+ * token, but the token's scale comes from the whole row.  The ranks combine
+ * their slice maxima (maximum over ranks, exact in any order) and quantise
+ * their slice with the combined maxima; the codes and scales are then exactly
+ * those ptpc_quantize_activations gives the whole row.
+ *
+ * ptpc_act_row_amax: amax_dev fp32 [T] = max_k |X[t, k]| of the slice (exact;
+ * 0 for an all-zero row).  X as for ptpc_quantize_activations. */
+PTPC_API int ptpc_act_row_amax(const void *X_dev, int64_t T, int64_t Ci, int64_t ldx, float *amax_dev,
+                               void *stream);
+
+/* ptpc_quantize_activations with the row maxima given: x_scale[t] =
+ * amax[t] / 448 (1.0f and all codes 0x00 when amax[t] == 0), codes of the
+ * slice with that scale.  amax_dev fp32 [T] must hold maxima of bf16
+ * magnitudes that are at least the slice's own (the combined maxima from
+ * ptpc_act_row_amax). */
+PTPC_API int ptpc_quantize_activations_amax(const void *X_dev, int64_t T, int64_t Ci, int64_t ldx,
+                                            const float *amax_dev, uint8_t *Xq_dev, float *x_scale_dev,
+                                            void *stream);
 
 /* Per-output-channel weight quantisation (the page's Delta_W[1 x Co]); run
  * once per weight, e.g. when a bf16 checkpoint is loaded.
@@ -167,6 +203,39 @@ PTPC_API const char *ptpc_status_string(int status);
  * K split over a cluster of that many CTAs, decode-sized T only).  0 on
  * invalid arguments, T == 0 or an unsupported device.  Launches nothing. */
 PTPC_API int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co);
+
+/* Bytes of a quantised weight of format fmt: Co * Ci * bits / 8 (0 on
+ * invalid arguments; the sub-byte formats need Ci % 128 == 0). */
+PTPC_API size_t ptpc_weight_bytes(int fmt, int64_t Ci, int64_t Co);
+
+/* Per-output-channel weight quantisation to format fmt (ptpc_weight_format):
+ * w_scale[o] = amax(|W[:, o]|) / max_format (1.0f for an all-zero column),
+ * code = saturating round-half-to-even of the fp32 quotient W[k][o] / w_scale[o]
+ * in the format (sign kept), written transposed and packed along Ci:
+ *   Wq_dev  u8 [Co, ptpc_weight_bytes(fmt, Ci, Co) / Co], row o = channel o's
+ *           Ci codes in K order (E4M3: exactly ptpc_quantize_weights' Wq_t).
+ * Sub-byte formats need Ci % 128 == 0 (PTPC_ERR_UNSUPPORTED_SHAPE) and a
+ * 32-byte aligned Wq_dev (PTPC_ERR_MISALIGNED), as TMA reads them.
+ * ws_dev: ptpc_workspace_size(PTPC_OP_QUANTIZE_WEIGHTS, 0, Ci, Co) bytes. */
+PTPC_API int ptpc_quantize_weights_fmt(const void *W_dev, int64_t Ci, int64_t Co, int fmt,
+                                       uint8_t *Wq_dev, float *w_scale_dev,
+                                       void *ws_dev, size_t ws_bytes, void *stream);
+
+/* ptpc_scaled_mm with weights of format fmt (from ptpc_quantize_weights_fmt):
+ *   out[t][o] = bf16_RNE((sum_k dec_e4m3(Xq[t][k]) * dec_fmt(Wq[o][k]) * x_scale[t]) * w_scale[o]).
+ * The tensor cores read the packed FP4/FP6 codes directly (mixed-format
+ * kind::f8f6f4 MMA), so decode-sized T streams 1/2 (FP4) or 3/4 (FP6) of the
+ * FP8 weight bytes.  Same plans, workspace and conventions as ptpc_scaled_mm. */
+PTPC_API int ptpc_scaled_mm_fmt(const uint8_t *Xq_dev, const float *x_scale_dev,
+                                const uint8_t *Wq_dev, const float *w_scale_dev, int fmt,
+                                int64_t T, int64_t Ci, int64_t Co, void *out_dev,
+                                void *ws_dev, size_t ws_bytes, void *stream);
+
+/* ptpc_linear with weights of format fmt: per-token FP8 quantisation of X,
+ * then ptpc_scaled_mm_fmt, on one stream; workspace as for ptpc_linear. */
+PTPC_API int ptpc_linear_fmt(const void *X_dev, int64_t ldx, const uint8_t *Wq_dev, const float *w_scale_dev,
+                             int fmt, int64_t T, int64_t Ci, int64_t Co, void *out_dev,
+                             void *ws_dev, size_t ws_bytes, void *stream);
 
 /* Re-reads the GEMM's tuning overrides from the environment.  They are
  * otherwise read once, at the first GEMM call of the process, so that no call

@@ -93,6 +93,8 @@ def _load():
                 "oracle_quant_weight_fmt": [P, I64, I64, ctypes.c_int, P, P],
                 "oracle_pack_fmt": [P, I64, I64, ctypes.c_int, P],
                 "oracle_fmt_encode_array": [P, I64, ctypes.c_int, P],
+                "oracle_row_amax": [P, I64, I64, P],
+                "oracle_quant_act_amax": [P, I64, I64, P, P, P],
             }.items():
                 fn = getattr(lib, name)
                 fn.restype = None
@@ -355,3 +357,38 @@ def linear_reference_fmt(X_bits, codes_t, w_scale, fmt: str, rows=None):
     weights.  Returns (out bf16 bits, Xq, x_scale)."""
     Xq, xs = quant_act(X_bits)
     return scaled_mm_reference_fmt(Xq, xs, codes_t, w_scale, fmt, rows), Xq, xs
+
+
+# --------------------------------------------------------------------------
+# Row-split (tensor-parallel) activation quantisation
+# --------------------------------------------------------------------------
+
+def row_amax(X_bits: np.ndarray) -> np.ndarray:
+    """max |x| of every row of a bf16 [T, Ci] slice (fp32, exact)."""
+    X = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    out = np.empty((X.shape[0],), dtype=np.float32)
+    _load().oracle_row_amax(_ptr(X), X.shape[0], X.shape[1], _ptr(out))
+    return out
+
+
+def quant_act_amax(X_bits: np.ndarray, amax: np.ndarray):
+    """Per-token quantisation of a slice with given row maxima (the maxima of
+    the whole rows, combined over the slices): (Xq [T, Ci], x_scale [T])."""
+    X = np.ascontiguousarray(X_bits, dtype=np.uint16)
+    a = np.ascontiguousarray(amax, dtype=np.float32)
+    T, Ci = X.shape
+    Xq = np.empty((T, Ci), dtype=np.uint8)
+    xs = np.empty((T,), dtype=np.float32)
+    _load().oracle_quant_act_amax(_ptr(X), T, Ci, _ptr(a), _ptr(Xq), _ptr(xs))
+    return Xq, xs
+
+
+def reference_epilogue(acc64: np.ndarray, x_scale, w_scale) -> np.ndarray:
+    """bf16_RNE(x_scale[t] * w_scale[o] * acc[t, o]) in fp64 of a given fp64
+    accumulator (the epilogue of scaled_mm_reference)."""
+    acc = np.ascontiguousarray(acc64, dtype=np.float64)
+    xs = np.ascontiguousarray(x_scale, dtype=np.float32)
+    ws = np.ascontiguousarray(w_scale, dtype=np.float32)
+    out = np.empty(acc.shape, dtype=np.uint16)
+    _load().oracle_reference_epilogue_f64(_ptr(acc), acc.shape[0], acc.shape[1], _ptr(xs), _ptr(ws), _ptr(out))
+    return out

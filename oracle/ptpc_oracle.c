@@ -511,3 +511,50 @@ void oracle_fmt_encode_array(const float *v, int64_t n, int f, uint8_t *out)
     for (i = 0; i < n; ++i)
         out[i] = oracle_fmt_encode(v[i], f);
 }
+
+/* ------------------------------------------------------------------------- */
+/* Per-token quantisation with a given row maximum (tensor parallelism)      */
+/* ------------------------------------------------------------------------- */
+/*
+ * When the input channels of a layer are split over ranks (the row-parallel
+ * linear of the PTPC page's TP = 2 evaluation), a rank holds only a slice of
+ * every token's row.  The token's scale still comes from the whole row: the
+ * ranks combine their slice maxima (a maximum is exact in any order) and each
+ * rank quantises its slice with the combined maximum.  These two functions
+ * are the two halves of that split: the slice maximum, and the quantisation
+ * with a given maximum (s = amax / 448 as for oracle_quant_act; with the row's
+ * own maximum it is oracle_quant_act).
+ */
+
+/* amax[t] = max_k |X[t, k]| over a T x Ci bf16 slice (fp32, exact). */
+void oracle_row_amax(const uint16_t *X, int64_t T, int64_t Ci, float *amax)
+{
+    int64_t t;
+#pragma omp parallel for schedule(static)
+    for (t = 0; t < T; ++t) {
+        float m = 0.0f;
+        int64_t k;
+        for (k = 0; k < Ci; ++k) {
+            float a = fabsf(oracle_bf16_to_float(X[t * Ci + k]));
+            if (a > m)
+                m = a;
+        }
+        amax[t] = m;
+    }
+}
+
+/* Codes of a T x Ci slice with the given per-row maxima: x_scale[t] =
+ * amax[t] / 448 (1.0f and all codes 0x00 when amax[t] == 0). */
+void oracle_quant_act_amax(const uint16_t *X, int64_t T, int64_t Ci, const float *amax,
+                           uint8_t *Xq, float *x_scale)
+{
+    int64_t t;
+#pragma omp parallel for schedule(static)
+    for (t = 0; t < T; ++t) {
+        float s = oracle_scale_from_amax(amax[t]);
+        int64_t k;
+        x_scale[t] = s;
+        for (k = 0; k < Ci; ++k)
+            Xq[t * Ci + k] = oracle_quantize_value(oracle_bf16_to_float(X[t * Ci + k]), s, amax[t]);
+    }
+}

@@ -121,3 +121,35 @@ def test_binding_rejects_cpu_tensors(ptpc):
     import torch
     with pytest.raises(TypeError):
         ptpc.quantize_activations(torch.zeros(4, 16, dtype=torch.bfloat16))
+
+
+def test_weight_format_argument_checks(ptpc):
+    P = ctypes.c_void_p
+    wb = lambda *a: call(ptpc, "ptpc_weight_bytes", *a)
+    assert wb(0, 4096, 6144) == 4096 * 6144
+    assert wb(1, 4096, 6144) == 4096 * 6144 // 2
+    assert wb(2, 4096, 6144) == 4096 * 6144 * 3 // 4
+    assert wb(3, 8192, 16) == 8192 * 16 * 3 // 4
+    assert wb(1, 4112, 16) == 0          # sub-byte rows need Ci % 128 == 0
+    assert wb(4, 4096, 16) == 0          # unknown format
+    need = ptpc.workspace_size(ptpc.OP_QUANTIZE_WEIGHTS, 0, 256, 64)
+    qw = lambda *a: call(ptpc, "ptpc_quantize_weights_fmt", *a)
+    assert qw(P(FAKE), 256, 64, 7, P(FAKE), P(FAKE), P(FAKE), need, None) == ptpc.ERR_INVALID_ARG
+    assert qw(P(FAKE), 144, 64, 1, P(FAKE), P(FAKE), P(FAKE), need, None) == ptpc.ERR_UNSUPPORTED_SHAPE
+    assert qw(P(FAKE), 256, 64, 2, P(FAKE + 16), P(FAKE), P(FAKE), need, None) == ptpc.ERR_MISALIGNED
+    assert qw(P(FAKE), 256, 64, 3, P(FAKE), P(FAKE), P(FAKE), need - 1, None) == ptpc.ERR_WORKSPACE_TOO_SMALL
+    mm = lambda *a: call(ptpc, "ptpc_scaled_mm_fmt", *a)
+    need = ptpc.workspace_size(ptpc.OP_SCALED_MM, 16, 256, 64)
+    assert mm(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 9, 16, 256, 64, P(FAKE), P(FAKE), need, None) == \
+        ptpc.ERR_INVALID_ARG
+    assert mm(P(FAKE), P(FAKE), P(FAKE), P(FAKE), 1, 16, 272, 64, P(FAKE), P(FAKE), need, None) == \
+        ptpc.ERR_UNSUPPORTED_SHAPE
+    assert mm(P(FAKE), P(FAKE), P(FAKE + 16), P(FAKE), 2, 16, 256, 64, P(FAKE), P(FAKE), need, None) == \
+        ptpc.ERR_MISALIGNED
+    assert mm(None, None, None, None, 1, 0, 256, 64, None, None, 0, None) == ptpc.OK
+    lin = lambda *a: call(ptpc, "ptpc_linear_fmt", *a)
+    need = ptpc.workspace_size(ptpc.OP_LINEAR, 16, 256, 64)
+    assert lin(P(FAKE), 256, P(FAKE), P(FAKE), 3, 16, 256, 64, P(FAKE), P(FAKE), need - 256, None) == \
+        ptpc.ERR_WORKSPACE_TOO_SMALL
+    assert lin(P(FAKE), 256, P(FAKE + 16), P(FAKE), 1, 16, 256, 64, P(FAKE), P(FAKE), need, None) == \
+        ptpc.ERR_MISALIGNED

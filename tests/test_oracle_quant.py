@@ -146,3 +146,22 @@ def test_quantize_value_single_element():
     assert oracle.quantize_value(-0.0, 1.0, 0.0) == 0x00
     assert oracle.scale_from_amax(0.0) == 1.0
     assert oracle.scale_from_amax(448.0) == 1.0
+
+
+def test_row_split_quantisation_equals_whole_rows():
+    """Tensor-parallel split of the input channels: the maximum of the slices'
+    row maxima is the row maximum (checked against numpy), and quantising each
+    slice with it reproduces the whole-row codes and scales of quant_act."""
+    X = synthetic.with_edge_rows(synthetic.make_x(synthetic.LLAMA70B_PREFILL, 0, 40, 1024))
+    Xq, xs = oracle.quant_act(X)
+    full_amax = np.abs(oracle.bf16_to_float(X)).max(axis=1)
+    assert np.array_equal(oracle.row_amax(X), full_amax)
+    for parts in (2, 4, 8):
+        w = 1024 // parts
+        slices = [X[:, r * w:(r + 1) * w] for r in range(parts)]
+        amax = np.max(np.stack([oracle.row_amax(s) for s in slices]), axis=0)
+        assert np.array_equal(amax, full_amax)
+        got = [oracle.quant_act_amax(s, amax) for s in slices]
+        assert np.array_equal(np.concatenate([g[0] for g in got], axis=1), Xq)
+        for g in got:
+            assert np.array_equal(g[1].view(np.uint32), xs.view(np.uint32))
