@@ -57,6 +57,7 @@ SIGNATURES = {
     "ptpc_get_device_status": (ctypes.c_int, [_P, _P]),
     "ptpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ptpc_gemm_ksplit": (ctypes.c_int, [_I64, _I64, _I64]),
+    "ptpc_gemm_tail_split": (ctypes.c_int, [_I64, _I64, _I64, _SZ]),
     "ptpc_selftest_wait_timeout": (ctypes.c_int, [_P, _P]),
     "ptpc_scaled_mm_static_scratch": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "ptpc_static_scratch_status": (ctypes.c_int, [_P]),
@@ -113,6 +114,15 @@ def gemm_ksplit(T: int, Ci: int, Co: int) -> int:
     """CTAs sharing each output tile for this shape on the current device
     (1: whole tiles; 2/4/8: K split over a cluster; 0: invalid)."""
     return int(lib.ptpc_gemm_ksplit(T, Ci, Co))
+
+
+def gemm_tail_split(T: int, Ci: int, Co: int, ws_bytes: int | None = None) -> int:
+    """CTA pairs sharing each tile of the prefill GEMM's split last wave for
+    this shape (0: every tile whole), with ws_bytes of GEMM workspace
+    (default: what ptpc_workspace_size asks for)."""
+    if ws_bytes is None:
+        ws_bytes = workspace_size(OP_SCALED_MM, T, Ci, Co)
+    return int(lib.ptpc_gemm_tail_split(T, Ci, Co, ws_bytes))
 
 
 def _check(fn: str, status: int):

@@ -21,8 +21,12 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Workspace layout of the GEMM entry points:
 //   [0, 256)                 device status word (uint32 at offset 0)
-// ptpc_linear appends Xq [T, Ci] and x_scale [T] after it.
-constexpr size_t kGemmWorkspace = kAlign;
+//   [256, gemm bytes)        prefill shapes only: the split tail's counters and
+//                            fp32 partial accumulators (ptpc::gemm_workspace_bytes)
+// ptpc_linear appends Xq [T, Ci] and x_scale [T] after the GEMM's part.
+constexpr size_t kGemmWorkspace = kAlign;  // the part every GEMM call needs
+
+size_t gemm_ws(int64_t T, int64_t Ci, int64_t Co) { return ptpc::gemm_workspace_bytes((int)T, (int)Ci, (int)Co); }
 
 // Once per device: the kernels are built for compute capability 10.0 only.
 int check_device() {
@@ -78,9 +82,11 @@ int check_subbyte(int fmt, int64_t Ci, const void *Wq) {
 }
 
 int run_gemm(const uint8_t *Xq, const float *xs, const uint8_t *Wq_t, const float *ws, int64_t T, int64_t Ci,
-             int64_t Co, void *out, bool f32_out, uint8_t *wsp, bool pdl, cudaStream_t st, int wfmt = 0) {
+             int64_t Co, void *out, bool f32_out, uint8_t *wsp, size_t ws_bytes, bool pdl, cudaStream_t st,
+             int wfmt = 0) {
   ptpc::GemmProblem p{};
   p.wfmt = wfmt;
+  p.ws_bytes = ws_bytes;
   p.Xq = Xq;
   p.xs = xs;
   p.Wq_t = Wq_t;
@@ -120,12 +126,14 @@ size_t ptpc_workspace_size(int op, int64_t T, int64_t Ci, int64_t Co) {
       if (check_shape_tci(0, Ci) != PTPC_OK || check_co(Co) != PTPC_OK) return 0;
       return kAlign + round_up((size_t)(Co + 1) * 4);
     case PTPC_OP_SCALED_MM:
+      if (check_shape_tci(T, Ci) != PTPC_OK || check_co(Co) != PTPC_OK) return 0;
+      return gemm_ws(T, Ci, Co);
     case PTPC_OP_BENCH_UNSCALED_MM:
       if (check_shape_tci(T, Ci) != PTPC_OK || check_co(Co) != PTPC_OK) return 0;
       return kGemmWorkspace;
     case PTPC_OP_LINEAR:
       if (check_shape_tci(T, Ci) != PTPC_OK || check_co(Co) != PTPC_OK) return 0;
-      return kGemmWorkspace + round_up((size_t)T * (size_t)Ci) + round_up((size_t)T * 4);
+      return gemm_ws(T, Ci, Co) + round_up((size_t)T * (size_t)Ci) + round_up((size_t)T * 4);
     case PTPC_OP_BENCH_PER_TENSOR:
       if (check_shape_tci(T, Ci) != PTPC_OK) return 0;
       return kAlign + kAlign;
@@ -196,8 +204,8 @@ int ptpc_scaled_mm(const uint8_t *Xq, const float *x_scale, const uint8_t *Wq_t,
     return PTPC_ERR_MISALIGNED;
   if (ws_bytes < ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
   if ((s = check_device()) != PTPC_OK) return s;
-  return run_gemm(Xq, x_scale, Wq_t, w_scale, T, Ci, Co, out, false, static_cast<uint8_t *>(ws), false,
-                  (cudaStream_t)stream);
+  return run_gemm(Xq, x_scale, Wq_t, w_scale, T, Ci, Co, out, false, static_cast<uint8_t *>(ws), gemm_ws(T, Ci, Co),
+                  false, (cudaStream_t)stream);
 }
 
 int ptpc_linear(const void *X, int64_t ldx, const uint8_t *Wq_t, const float *w_scale, int64_t T, int64_t Ci,
@@ -213,11 +221,12 @@ int ptpc_linear(const void *X, int64_t ldx, const uint8_t *Wq_t, const float *w_
   if (ws_bytes < ptpc_workspace_size(PTPC_OP_LINEAR, T, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
   if ((s = check_device()) != PTPC_OK) return s;
   uint8_t *wsp = static_cast<uint8_t *>(ws);
-  uint8_t *Xq = wsp + kGemmWorkspace;
-  float *xs = reinterpret_cast<float *>(wsp + kGemmWorkspace + round_up((size_t)T * (size_t)Ci));
+  const size_t gws = gemm_ws(T, Ci, Co);
+  uint8_t *Xq = wsp + gws;
+  float *xs = reinterpret_cast<float *>(wsp + gws + round_up((size_t)T * (size_t)Ci));
   cudaStream_t st = (cudaStream_t)stream;
   if ((s = cuda_status(ptpc::launch_quant_act(X, (int)T, (int)Ci, ldx, Xq, xs, st))) != PTPC_OK) return s;
-  return run_gemm(Xq, xs, Wq_t, w_scale, T, Ci, Co, out, false, wsp, true, st);
+  return run_gemm(Xq, xs, Wq_t, w_scale, T, Ci, Co, out, false, wsp, gws, true, st);
 }
 
 size_t ptpc_weight_bytes(int fmt, int64_t Ci, int64_t Co) {
@@ -257,8 +266,8 @@ int ptpc_scaled_mm_fmt(const uint8_t *Xq, const float *x_scale, const uint8_t *W
   if ((s = check_subbyte(fmt, Ci, Wq)) != PTPC_OK) return s;
   if (ws_bytes < ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
   if ((s = check_device()) != PTPC_OK) return s;
-  return run_gemm(Xq, x_scale, Wq, w_scale, T, Ci, Co, out, false, static_cast<uint8_t *>(ws), false,
-                  (cudaStream_t)stream, fmt);
+  return run_gemm(Xq, x_scale, Wq, w_scale, T, Ci, Co, out, false, static_cast<uint8_t *>(ws), gemm_ws(T, Ci, Co),
+                  false, (cudaStream_t)stream, fmt);
 }
 
 int ptpc_linear_fmt(const void *X, int64_t ldx, const uint8_t *Wq, const float *w_scale, int fmt, int64_t T,
@@ -276,11 +285,18 @@ int ptpc_linear_fmt(const void *X, int64_t ldx, const uint8_t *Wq, const float *
   if (ws_bytes < ptpc_workspace_size(PTPC_OP_LINEAR, T, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
   if ((s = check_device()) != PTPC_OK) return s;
   uint8_t *wsp = static_cast<uint8_t *>(ws);
-  uint8_t *Xq = wsp + kGemmWorkspace;
-  float *xs = reinterpret_cast<float *>(wsp + kGemmWorkspace + round_up((size_t)T * (size_t)Ci));
+  const size_t gws = gemm_ws(T, Ci, Co);
+  uint8_t *Xq = wsp + gws;
+  float *xs = reinterpret_cast<float *>(wsp + gws + round_up((size_t)T * (size_t)Ci));
   cudaStream_t st = (cudaStream_t)stream;
   if ((s = cuda_status(ptpc::launch_quant_act(X, (int)T, (int)Ci, ldx, Xq, xs, st))) != PTPC_OK) return s;
-  return run_gemm(Xq, xs, Wq, w_scale, T, Ci, Co, out, false, wsp, true, st, fmt);
+  return run_gemm(Xq, xs, Wq, w_scale, T, Ci, Co, out, false, wsp, gws, true, st, fmt);
+}
+
+int ptpc_gemm_tail_split(int64_t T, int64_t Ci, int64_t Co, size_t ws_bytes) {
+  if (check_shape_tci(T, Ci) != PTPC_OK || check_co(Co) != PTPC_OK || T == 0) return 0;
+  if (check_device() != PTPC_OK) return 0;
+  return ptpc::gemm_tail_split((int)T, (int)Ci, (int)Co, ws_bytes);
 }
 
 int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co) {
@@ -329,8 +345,8 @@ int ptpc_bench_unscaled_mm_f32(const uint8_t *Xq, const uint8_t *Wq_t, int64_t T
   if (!aligned16(Xq) || !aligned16(Wq_t) || !aligned16(y) || !aligned16(ws)) return PTPC_ERR_MISALIGNED;
   if (ws_bytes < ptpc_workspace_size(PTPC_OP_BENCH_UNSCALED_MM, T, Ci, Co)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
   if ((s = check_device()) != PTPC_OK) return s;
-  return run_gemm(Xq, nullptr, Wq_t, nullptr, T, Ci, Co, y, true, static_cast<uint8_t *>(ws), false,
-                  (cudaStream_t)stream);
+  return run_gemm(Xq, nullptr, Wq_t, nullptr, T, Ci, Co, y, true, static_cast<uint8_t *>(ws), kGemmWorkspace,
+                  false, (cudaStream_t)stream);
 }
 
 int ptpc_bench_clock_probe(uint64_t *records_dev, int max_records, uint64_t period_ns, uint64_t duration_ns,
@@ -446,7 +462,8 @@ extern "C" int ptpc_scaled_mm_static_scratch(const uint8_t *Xq, const float *x_s
   // array and needs nothing else to start at zero.  The word is not cleared
   // here, so a timeout stays recorded until ptpc_static_scratch_status reads
   // it (the array is zero when the library is loaded).
-  return run_gemm(Xq, x_scale, Wq_t, w_scale, T, Ci, Co, out, false, scratch, false, (cudaStream_t)stream);
+  return run_gemm(Xq, x_scale, Wq_t, w_scale, T, Ci, Co, out, false, scratch, kStaticScratchBytes, false,
+                  (cudaStream_t)stream);
 }
 
 extern "C" int ptpc_static_scratch_status(void *stream) {

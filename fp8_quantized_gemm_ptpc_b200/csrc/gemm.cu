@@ -53,6 +53,7 @@ namespace ptpc {
 namespace {
 
 constexpr int BM = 128;      // token rows per CTA tile (tensor-memory lanes)
+constexpr size_t kGemmStatusBytes = 256;  // the workspace's device status word (and its padding)
 constexpr int BK = 128;      // K bytes per stage (= one 128-byte swizzle row)
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
@@ -76,6 +77,12 @@ struct GemmParams {
   int np;                     // decode kernel: tokens padded to the MMA's N (multiple of 16)
   int stages;                 // decode kernel: shared-memory ring depth
   int tmem_cols;              // decode kernel: tensor-memory columns allocated (two accumulators)
+  // pair kernel, split tail: the last tail_tiles tiles of the raster (the
+  // under-filled last wave) are split along K over tail_split CTA pairs each
+  int full_tiles;             // tiles done whole (num_tiles - tail_tiles)
+  int tail_tiles, tail_split;
+  float *partials;            // fp32 [tail_tiles][tail_split][256][BN] partial accumulators
+  uint32_t *tail_count;       // [2][tail_tiles]: CTAs that stored their partial / finished reducing
   const float *xs;
   const float *ws;
   void *out;
@@ -83,8 +90,9 @@ struct GemmParams {
 };
 
 // One piece of work: K-blocks [kb0, kb1) of tile `tile` (row m, column n).
+// split >= 0: a K range of a split tail tile (the partial is reduced later).
 struct Unit {
-  int tile, m, n, kb0, kb1;
+  int tile, m, n, kb0, kb1, split;
 };
 
 // The same sequence of units for the producer, the MMA issuer and the
@@ -93,8 +101,10 @@ struct Unit {
 // this CTA's cluster and this CTA's share of its K-blocks.
 struct Sched {
   int next_tile, step, kb0, kb1;
+  int tail_unit;  // pair kernel: index of this pair's unit in the split tail, -1 if none (or done)
 
   __device__ __forceinline__ void init(const GemmParams &p, int id, int count) {
+    tail_unit = -1;
     if (p.ksplit > 1) {
       const int r = id % p.ksplit;  // == %cluster_ctarank for a 1-D cluster
       next_tile = id / p.ksplit;
@@ -106,15 +116,11 @@ struct Sched {
       step = count;
       kb0 = 0;
       kb1 = p.num_kb;
+      if (p.tail_tiles > 0 && id < p.tail_tiles * p.tail_split) tail_unit = id;
     }
   }
 
-  __device__ __forceinline__ bool next(const GemmParams &p, Unit &u) {
-    if (next_tile >= p.num_tiles) return false;
-    u.tile = next_tile;
-    next_tile += step;
-    u.kb0 = kb0;
-    u.kb1 = kb1;
+  __device__ __forceinline__ void raster(const GemmParams &p, Unit &u) {
     // grouped raster: group_m tile rows, all tile columns, rows fastest
     const int per_group = p.group_m * p.num_n;
     const int g = u.tile / per_group;
@@ -123,7 +129,30 @@ struct Sched {
     const int r = u.tile - g * per_group;
     u.m = first_m + r % gm;
     u.n = r / gm;
-    return true;
+  }
+
+  __device__ __forceinline__ bool next(const GemmParams &p, Unit &u) {
+    if (next_tile < p.full_tiles) {
+      u.tile = next_tile;
+      next_tile += step;
+      u.kb0 = kb0;
+      u.kb1 = kb1;
+      u.split = -1;
+      raster(p, u);
+      return true;
+    }
+    if (tail_unit >= 0) {
+      const int j = tail_unit / p.tail_split;
+      const int r = tail_unit - j * p.tail_split;
+      tail_unit = -1;
+      u.tile = p.full_tiles + j;
+      u.kb0 = r * p.num_kb / p.tail_split;
+      u.kb1 = (r + 1) * p.num_kb / p.tail_split;
+      u.split = r;
+      raster(p, u);
+      return true;
+    }
+    return false;
   }
 };
 
@@ -544,6 +573,91 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------------
+// Split tail of the pair kernel.  The tiles of the last, under-filled wave are
+// split along K over tail_split CTA pairs each; every CTA of those pairs
+// stores its 128 rows x BN fp32 partial accumulator in the workspace, counts
+// itself in, waits (bounded) until the tile's 2 * tail_split CTAs have all
+// stored theirs, and then finishes 1 / (2 * tail_split) of the tile: the
+// partials added in split order (a fixed order: deterministic), the two
+// scales applied, bf16 stored.  The last CTA to finish zeroes the tile's
+// counters for the next call.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// This lane's row of the partial accumulator: tensor memory -> global.
+template <int BN_T>
+__device__ __forceinline__ void dump_partial(uint32_t tbase, float *row_dst, int lane, uint32_t release_bar) {
+  #pragma unroll 1
+  for (int c0 = 0; c0 < BN_T; c0 += 32) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(tbase + c0, r);
+    tmem_wait_ld();
+    if (c0 + 32 >= BN_T) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(release_bar);
+    }
+    float4 *d = reinterpret_cast<float4 *>(row_dst + c0);
+    #pragma unroll
+    for (int j = 0; j < 8; ++j)
+      __stcg(d + j, make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+  }
+}
+
+// Reducer `ridx` (0 .. 2 * split - 1) of tail tile j at tile position (m, n):
+// groups of 8 output columns, [ridx * G / (2 S), (ridx + 1) * G / (2 S)).
+template <int BN_T>
+__device__ __forceinline__ void reduce_tail_tile(const GemmParams &p, int j, int m, int n, int ridx, int etid) {
+  const int S = p.tail_split;
+  constexpr int G8 = BN_T / 8;
+  constexpr int G = 2 * BM * G8;
+  const int g0 = (int)((long long)ridx * G / (2 * S));
+  const int g1 = (int)((long long)(ridx + 1) * G / (2 * S));
+  const float *base = p.partials + (size_t)j * S * (2 * BM) * BN_T;
+  for (int g = g0 + etid; g < g1; g += 32 * kEpiWarps) {
+    const int row = g / G8;
+    const int c8 = (g - row * G8) * 8;
+    const int t = m * (2 * BM) + row;
+    const int col = n * BN_T + c8;
+    if (t >= p.T || col >= p.Co) continue;  // Co % 16 == 0: the 8 columns are valid together
+    float a[8];
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = 0.0f;
+    for (int sp = 0; sp < S; ++sp) {
+      const float4 *src = reinterpret_cast<const float4 *>(base + ((size_t)sp * (2 * BM) + row) * BN_T + c8);
+      const float4 v0 = __ldcg(src), v1 = __ldcg(src + 1);
+      if (sp == 0) {
+        a[0] = v0.x; a[1] = v0.y; a[2] = v0.z; a[3] = v0.w;
+        a[4] = v1.x; a[5] = v1.y; a[6] = v1.z; a[7] = v1.w;
+      } else {
+        a[0] = __fadd_rn(a[0], v0.x); a[1] = __fadd_rn(a[1], v0.y);
+        a[2] = __fadd_rn(a[2], v0.z); a[3] = __fadd_rn(a[3], v0.w);
+        a[4] = __fadd_rn(a[4], v1.x); a[5] = __fadd_rn(a[5], v1.y);
+        a[6] = __fadd_rn(a[6], v1.z); a[7] = __fadd_rn(a[7], v1.w);
+      }
+    }
+    const float xs = __ldg(p.xs + t);
+    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.ws + col));
+    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.ws + col + 4));
+    const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    uint32_t o[4];
+    #pragma unroll
+    for (int i = 0; i < 4; ++i)
+      o[i] = pack_bf16x2(__fmul_rn(__fmul_rn(a[2 * i], xs), w[2 * i]),
+                         __fmul_rn(__fmul_rn(a[2 * i + 1], xs), w[2 * i + 1]));
+    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + (size_t)t * p.Co + col) =
+        make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// ----------------------------------------------------------------------------
 // CTA-pair kernel (prefill): a cluster of two CTAs on two SMs computes a
 // 256 (tokens) x 256 (channels) tile with tcgen05.mma.cta_group::2 (M = 256,
 // N = 256, K = 32).  CTA r of the pair loads token rows [r*128, r*128+128)
@@ -587,6 +701,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   uint64_t *tempty = tfull + 2;
   uint64_t *drain = tempty + 2;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
+  uint32_t *tail_flag = tmem_holder + 1;  // split tail: 1 while this CTA's protocol is intact
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -722,10 +837,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;
     const int ew = warp - 2;
+    const int etid = threadIdx.x - 64;
     uint8_t *cbuf = sC + ew * C::EPI_BUF;
     float *scl = sScale + ew * 64;
     int local = 0;
     bool ok = true;
+    // a member of the split tail: decided by the schedule alone, so every
+    // epilogue warp runs the tail protocol's barriers whatever happens above
+    const bool tail_member = p.tail_tiles > 0 && !F32OUT && cid < p.tail_tiles * p.tail_split;
+    int tail_j = 0, tail_m = 0, tail_n = 0, tail_r = 0;
+    bool dumped = false;
+    if (tail_member) {
+      if (etid == 0) *tail_flag = 1u;
+      epi_bar();
+    }
     griddep_wait();
     Sched sc;
     sc.init(p, cid, ncl);
@@ -745,11 +870,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
-      epilogue_store_tile<BN, F32OUT>(&tmC, tbase, cbuf, scl, p, u.n * BN, row0, xsr, lane,
-                                           mapa_shared(&tempty[buf], 0));
+      if (u.split < 0) {
+        epilogue_store_tile<BN, F32OUT>(&tmC, tbase, cbuf, scl, p, u.n * BN, row0, xsr, lane,
+                                        mapa_shared(&tempty[buf], 0));
+      } else if constexpr (!F32OUT) {
+        tail_j = u.tile - p.full_tiles;
+        tail_m = u.m;
+        tail_n = u.n;
+        tail_r = u.split;
+        float *dst = p.partials +
+                     ((size_t)(tail_j * p.tail_split + u.split) * (2 * BM) + rank * BM + q * 32 + lane) * BN;
+        dump_partial<BN>(tbase, dst, lane, mapa_shared(&tempty[buf], 0));
+        dumped = true;
+      }
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeoutEpilogue);
     if (lane == 0) bulk_wait<0>();
+    if (tail_member) {
+      // 1. count this CTA in once all four warps have stored their rows
+      __threadfence();
+      if (!dumped && lane == 0) atomicAnd(tail_flag, 0u);
+      epi_bar();
+      uint32_t *arrived = p.tail_count + tail_j;
+      uint32_t *finished = p.tail_count + p.tail_tiles + tail_j;
+      const uint32_t members = 2u * (uint32_t)p.tail_split;
+      if (etid == 0) {
+        if (*tail_flag) {
+          __threadfence();  // after the barrier: releases every warp's partial stores
+          atomicAdd(arrived, 1u);
+          // 2. wait (bounded) for every member CTA of the tile
+          bool all = ld_acquire_u32(arrived) >= members;
+          const uint64_t t0 = global_timer_ns();
+          while (!all) {
+            __nanosleep(256);
+            all = ld_acquire_u32(arrived) >= members;
+            if (!all && global_timer_ns() - t0 > kWaitLimitNs) break;
+          }
+          if (!all) {
+            atomicOr(p.status, kStatusTimeoutEpilogue);
+            *tail_flag = 0u;
+          }
+        }
+      }
+      epi_bar();
+      __threadfence();
+      // 3. this CTA's share of the tile
+      if (*tail_flag) reduce_tail_tile<BN>(p, tail_j, tail_m, tail_n, tail_r * 2 + (int)rank, etid);
+      __threadfence();
+      epi_bar();
+      // 4. the last member to finish leaves the counters zero
+      if (etid == 0 && *tail_flag) {
+        if (atomicAdd(finished, 1u) == members - 1u) {
+          atomicExch(arrived, 0u);
+          atomicExch(finished, 0u);
+        }
+      }
+    }
   }
 
   tc_fence_before();
@@ -985,6 +1161,7 @@ struct Plan {
   int ksplit;   // decode kernel: CTAs per tile (cluster size), 1 = whole tiles
   int np, stages, tmem_cols;  // decode kernel only
   bool red_fits;              // decode kernel: the K-split buffer fits in the ring
+  int tail_tiles, tail_split; // pair kernel: split tail (0: every tile whole)
 };
 
 // Time of a 128-wide pair tile relative to half a 256-wide one.  Measured on
@@ -997,12 +1174,14 @@ constexpr double kPairN128Cost = 1.15;
 
 // Tuning overrides (not for production use), from the environment:
 // PTPC_FORCE_KERNEL = pair | decode, PTPC_FORCE_PAIR_BN = 128 | 256,
-// PTPC_FORCE_KSPLIT = 1 | 2 | 4 | 8.  Read once, at the first GEMM call of
-// the process (or again by reload_tuning), not on every call.
+// PTPC_FORCE_KSPLIT = 1 | 2 | 4 | 8, PTPC_FORCE_SPLIT_TAIL = 0 | 1 (the pair
+// kernel's split tail off, or on wherever it is feasible).  Read once, at the
+// first GEMM call of the process (or again by reload_tuning), not on every call.
 struct Tuning {
   int kernel;   // 0 automatic, 1 pair, 2 decode
   int pair_bn;  // 0 automatic, 128, 256
   int ksplit;   // 0 automatic, 1, 2, 4, 8
+  int streamk;  // 0 automatic, 1 off, 2 on wherever feasible
 };
 
 int env_int(const char *name, int fallback) {
@@ -1022,14 +1201,19 @@ Tuning read_tuning() {
   if (bn == 128 || bn == 256) t.pair_bn = bn;
   const int ks = env_int("PTPC_FORCE_KSPLIT", 0);
   if (ks == 1 || ks == 2 || ks == 4 || ks == 8) t.ksplit = ks;
+  const int sk = env_int("PTPC_FORCE_SPLIT_TAIL", -1);
+  if (sk == 0) t.streamk = 1;
+  if (sk == 1) t.streamk = 2;
   return t;
 }
 
-// Packed as kernel | pair_bn / 128 << 2 | ksplit << 4, plus bit 8 once read.
+// Packed as kernel | pair_bn / 128 << 2 | ksplit << 4 | streamk << 9, plus
+// bit 8 once read.
 std::atomic<uint32_t> g_tuning{0};
 
 uint32_t pack_tuning(const Tuning &t) {
-  return 0x100u | (uint32_t)t.kernel | (uint32_t)(t.pair_bn / 128) << 2 | (uint32_t)t.ksplit << 4;
+  return 0x100u | (uint32_t)t.kernel | (uint32_t)(t.pair_bn / 128) << 2 | (uint32_t)t.ksplit << 4 |
+         (uint32_t)t.streamk << 9;
 }
 
 Tuning tuning() {
@@ -1038,7 +1222,7 @@ Tuning tuning() {
     v = pack_tuning(read_tuning());
     g_tuning.store(v, std::memory_order_relaxed);
   }
-  return Tuning{(int)(v & 3u), (int)((v >> 2) & 3u) * 128, (int)((v >> 4) & 15u)};
+  return Tuning{(int)(v & 3u), (int)((v >> 2) & 3u) * 128, (int)((v >> 4) & 15u), (int)((v >> 9) & 3u)};
 }
 
 // Fewest K-blocks a CTA of a K-split cluster streams.
@@ -1095,12 +1279,43 @@ int choose_pair_bn(int T, int Co, const DeviceInfo &d) {
   return (double)w128 * kPairN128Cost < (double)(2 * w256) ? 128 : 256;
 }
 
+// Split tail of the pair kernel.  With W whole waves and R < pairs tiles
+// left, the last wave keeps only R of the pairs busy for a whole tile time.
+// Splitting those R tiles along K over S = pairs / R pairs each (S >= 2, at
+// least kMinTailKb K-blocks per split) finishes them in about 1/S of a tile
+// time plus the partials' round trip through L2 and the distributed
+// reduction.  Taken only where the caller's workspace holds the partials.
+constexpr int kMinTailKb = 4;
+constexpr int kMaxTailPairs = 74;      // bound of the workspace size (a B200's 148 SMs in pairs)
+constexpr size_t kTailCountBytes = 1024;
+
+size_t tail_workspace(int tail_tiles, int split, int bn) {
+  return kTailCountBytes + (size_t)tail_tiles * split * (2 * BM) * bn * sizeof(float);
+}
+
+void choose_tail(Plan &pl, size_t ws_bytes) {
+  pl.tail_tiles = 0;
+  pl.tail_split = 0;
+  const int forced = tuning().streamk;          // 0 automatic, 1 off, 2 on
+  if (forced == 1 || pl.num_tiles <= pl.ctas) return;
+  const int rem = pl.num_tiles % pl.ctas;
+  if (rem == 0) return;
+  const int pairs = std::min(pl.ctas, kMaxTailPairs);
+  int split = std::min(pairs / rem, pl.num_kb / kMinTailKb);
+  if (split < 2) return;
+  // worth it only if the last wave is mostly idle: at most half the pairs busy
+  if (forced != 2 && 2 * rem > pl.ctas) return;
+  if (kGemmStatusBytes + tail_workspace(rem, split, pl.bn) > ws_bytes) return;
+  pl.tail_tiles = rem;
+  pl.tail_split = split;
+}
+
 // The prefill kernel's plan: whole tiles on the CTA pairs.
 // Sharing the last partial wave stream-K style (fp32 partial sums through
 // global memory, fixed-order fixup) was measured slower on B200 for these
 // tiles (e.g. 2048 x 4096 -> 6144: 73.8 us shared vs 43.1 us whole;
 // 2048 x 14336 -> 4096: 136.8 vs 109.7).
-Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d) {
+Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d, size_t ws_bytes) {
   Plan pl = {};
   pl.pair = true;
   pl.ksplit = 1;
@@ -1112,6 +1327,7 @@ Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d) {
   pl.num_n = (Co + pl.bn - 1) / pl.bn;
   pl.num_tiles = pl.num_m * pl.num_n;
   pl.ctas = std::max(1, std::min(pl.num_tiles, pl.bn == 128 ? d.pair_clusters128 : d.pair_clusters));
+  choose_tail(pl, ws_bytes);
   return pl;
 }
 
@@ -1123,16 +1339,16 @@ Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d) {
 // 59.0 us).
 // PTPC_FORCE_KERNEL = "pair" or "decode" overrides the choice (tuning only;
 // the decode kernel takes T <= 256 only).
-Plan make_plan(int T, int Ci, int Co) {
+Plan make_plan(int T, int Ci, int Co, size_t ws_bytes) {
   const DeviceInfo &d = device_info();
   const int force = tuning().kernel;
-  if (force == 1) return pair_plan(T, Ci, Co, d);
+  if (force == 1) return pair_plan(T, Ci, Co, d, ws_bytes);
   if (T <= kDecodeMaxT) {
     const Plan pl = decode_plan(T, Ci, Co, d);
     if (force == 2) return pl;
     if (T <= kDecodeWholeMaxT || pl.ksplit > 1) return pl;
   }
-  return pair_plan(T, Ci, Co, d);
+  return pair_plan(T, Ci, Co, d, ws_bytes);
 }
 
 template <typename Kernel>
@@ -1189,10 +1405,21 @@ void map_cache_stats(uint64_t *hits, uint64_t *misses) {
   *misses = g_map_misses.load(std::memory_order_relaxed);
 }
 
-int gemm_ksplit(int T, int Ci, int Co) { return make_plan(T, Ci, Co).ksplit; }
+int gemm_ksplit(int T, int Ci, int Co) { return make_plan(T, Ci, Co, gemm_workspace_bytes(T, Ci, Co)).ksplit; }
+
+int gemm_tail_split(int T, int Ci, int Co, size_t ws_bytes) { return make_plan(T, Ci, Co, ws_bytes).tail_split; }
+
+size_t gemm_workspace_bytes(int T, int Ci, int Co) {
+  // the status word, plus the split tail's counters and partials where the
+  // pair kernel could split one (more than one wave, K long enough), sized
+  // for kMaxTailPairs pairs of 256-wide tiles
+  const int num_kb = (Ci + BK - 1) / BK;
+  if (T <= kDecodeWholeMaxT || num_kb < 2 * kMinTailKb) return kGemmStatusBytes;
+  return kGemmStatusBytes + tail_workspace(1, kMaxTailPairs, 256);
+}
 
 cudaError_t launch_scaled_gemm(const GemmProblem &pr, cudaStream_t st) {
-  const Plan pl = make_plan(pr.T, pr.Ci, pr.Co);
+  const Plan pl = make_plan(pr.T, pr.Ci, pr.Co, pr.f32_out ? 0 : pr.ws_bytes);
   GemmParams gp = {};
   gp.T = pr.T;
   gp.Co = pr.Co;
@@ -1205,6 +1432,14 @@ cudaError_t launch_scaled_gemm(const GemmProblem &pr, cudaStream_t st) {
   gp.np = pl.np;
   gp.stages = pl.stages;
   gp.tmem_cols = pl.tmem_cols;
+  gp.tail_tiles = pl.tail_tiles;
+  gp.tail_split = pl.tail_split;
+  gp.full_tiles = pl.num_tiles - pl.tail_tiles;
+  if (pl.tail_tiles > 0) {
+    uint8_t *w = reinterpret_cast<uint8_t *>(pr.status);
+    gp.tail_count = reinterpret_cast<uint32_t *>(w + kGemmStatusBytes);
+    gp.partials = reinterpret_cast<float *>(w + kGemmStatusBytes + kTailCountBytes);
+  }
   gp.xs = pr.xs;
   gp.ws = pr.ws;
   gp.out = pr.out;

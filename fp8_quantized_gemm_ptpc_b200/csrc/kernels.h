@@ -28,7 +28,9 @@ cudaError_t launch_quant_weight_sub(const void *W, int Ci, int Co, int fmt, uint
 cudaError_t launch_apply_scales(const float *y, const float *xs, const float *ws, int T, int Co, void *out,
                                 cudaStream_t st);
 
-// Scaled GEMM (gemm.cu).  Its only scratch is the device status word.
+// Scaled GEMM (gemm.cu).  Its workspace holds the device status word and,
+// for shapes whose last wave of prefill tiles is split along K, the split's
+// counters and fp32 partial accumulators (gemm_workspace_bytes).
 struct GemmProblem {
   const uint8_t *Xq;      // [T, Ci]
   const float *xs;        // [T]   (unused for f32 output)
@@ -40,6 +42,7 @@ struct GemmProblem {
   uint32_t *status;       // device status word
   bool pdl;               // launch as a programmatic dependent of the previous kernel
   int wfmt;               // weight format: 0 E4M3, 1 E2M1, 2 E2M3, 3 E3M2 (packed along Ci)
+  size_t ws_bytes;        // workspace at `status` (the split tail needs gemm_workspace_bytes)
 };
 
 cudaError_t launch_scaled_gemm(const GemmProblem &p, cudaStream_t st);
@@ -47,6 +50,13 @@ cudaError_t launch_scaled_gemm(const GemmProblem &p, cudaStream_t st);
 // CTAs per tile the decode kernel uses for a shape (1: whole tiles; larger:
 // K split over a cluster of that many CTAs).  For tests and reports.
 int gemm_ksplit(int T, int Ci, int Co);
+
+// Tail tiles' split of the pair kernel for a shape with ws_bytes of
+// workspace (0: every tile whole).  For tests and reports.
+int gemm_tail_split(int T, int Ci, int Co, size_t ws_bytes);
+
+// Workspace bytes of a GEMM call (a multiple of 256).
+size_t gemm_workspace_bytes(int T, int Ci, int Co);
 
 int num_sms();
 

@@ -152,11 +152,17 @@ PTPC_API int ptpc_quantize_weights(const void *W_dev, int64_t Ci, int64_t Co,
  *   Wq_t_dev    u8 [Co, Ci], w_scale_dev fp32 [Co] (from ptpc_quantize_weights)
  *   out_dev     bf16 [T, Co] row-major, written once (no intermediate array).
  *   ws_dev      ptpc_workspace_size(PTPC_OP_SCALED_MM, T, Ci, Co) bytes: the
- *               device status word.
+ *               device status word and, for prefill-sized T, room for the
+ *               split tail (below), about 19 MB.
  * The sum over k is an fp32 tensor-core accumulation; its order is not
  * specified.  For T <= 256 and few output tiles, K is split over a cluster of
  * 2, 4 or 8 CTAs (see ptpc_gemm_ksplit) whose fp32 partial sums are added in
- * a fixed order, so results are deterministic for a given shape. */
+ * a fixed order.  For prefill-sized T whose last wave of output tiles would
+ * keep at most half the SMs busy, those tiles are split along K over the
+ * whole GPU (see ptpc_gemm_tail_split): their fp32 partial sums go through
+ * the workspace and are added in a fixed order.  Results are deterministic
+ * for a given shape and workspace size.  With a smaller workspace (at least
+ * the status word) every tile is computed whole. */
 PTPC_API int ptpc_scaled_mm(const uint8_t *Xq_dev, const float *x_scale_dev,
                    const uint8_t *Wq_t_dev, const float *w_scale_dev,
                    int64_t T, int64_t Ci, int64_t Co, void *out_dev,
@@ -242,12 +248,20 @@ PTPC_API int ptpc_linear_fmt(const void *X_dev, int64_t ldx, const uint8_t *Wq_d
  * pays for environment lookups:
  *   PTPC_FORCE_KERNEL  = pair | decode   which GEMM kernel runs a shape,
  *   PTPC_FORCE_PAIR_BN = 128 | 256       tile width of the prefill kernel,
- *   PTPC_FORCE_KSPLIT  = 1 | 2 | 4 | 8   CTAs per tile of the decode kernel.
+ *   PTPC_FORCE_KSPLIT  = 1 | 2 | 4 | 8   CTAs per tile of the decode kernel,
+ *   PTPC_FORCE_SPLIT_TAIL = 0 | 1        the prefill kernel's split tail off,
+ *                                        or on wherever the workspace allows.
  * Each is honoured only where the forced choice is feasible for the shape;
  * results stay within the GEMM's tolerance under every choice.  For tuning
  * and tests, not for production.  Not thread-safe with concurrent GEMM calls
  * that should see a consistent setting.  No counterpart on the page. */
 PTPC_API int ptpc_reload_tuning_overrides(void);
+
+/* The split-tail plan of ptpc_scaled_mm / ptpc_linear for a shape on the
+ * current device with ws_bytes of GEMM workspace: 0 if every output tile is
+ * computed whole, else the number of CTA pairs that share each tile of the
+ * last wave (split along K).  Launches nothing.  No counterpart on the page. */
+PTPC_API int ptpc_gemm_tail_split(int64_t T, int64_t Ci, int64_t Co, size_t ws_bytes);
 
 /* ptpc_scaled_mm without a caller-provided workspace.  The page has no
  * counterpart: this exists for callers that cannot allocate device memory
@@ -257,9 +271,10 @@ PTPC_API int ptpc_reload_tuning_overrides(void);
  * results as ptpc_scaled_mm minus (ws_dev, ws_bytes).
  *   Scratch: a file-scope 4 KiB device array inside the library, held by
  *   every GPU that loads the library until the process exits; the GEMM uses
- *   its first 256 bytes (the device status word).  Results are bit-identical
- *   to ptpc_scaled_mm's.  The GEMM's scratch fits the array for every shape
- *   (checked when the library is compiled).
+ *   its first 256 bytes (the device status word).  The array has no room
+ *   for the split tail, so every output tile is computed whole; results are
+ *   bit-identical to ptpc_scaled_mm's wherever that plan has no split tail
+ *   (ptpc_gemm_tail_split), and within the GEMM's tolerance of them elsewhere.
  *   The first call on a device looks up the array's device address once
  *   (cudaGetSymbolAddress; its failure returns PTPC_ERR_CUDA).
  *   Nothing is allocated and nothing is cleared per call: the status word is

@@ -55,9 +55,15 @@ def test_workspace_sizes(ptpc):
     assert ws(ptpc.OP_SCALED_MM, 16, 100, 64) == 0          # Ci not a multiple of 16
     assert ws(ptpc.OP_SCALED_MM, -1, 128, 64) == 0
     assert ws(99, 16, 128, 64) == 0
-    # the GEMM's only scratch is the device status word, at every size
+    # decode-sized T: the device status word only; prefill-sized T: room for
+    # the split tail (74 CTA pairs x a 256 x 256 fp32 partial + counters)
     assert ws(ptpc.OP_SCALED_MM, 1, 28672, 8192) == 256
-    assert ws(ptpc.OP_SCALED_MM, 8192, 28672, 8192) == 256
+    assert ws(ptpc.OP_SCALED_MM, 192, 8192, 57344) == 256
+    big = 256 + 1024 + 74 * 256 * 256 * 4
+    assert ws(ptpc.OP_SCALED_MM, 8192, 28672, 8192) == big
+    assert ws(ptpc.OP_SCALED_MM, 300, 768, 1040) == 256           # K too short to split
+    assert ws(ptpc.OP_LINEAR, 8192, 28672, 8192) == big + 8192 * 28672 + 8192 * 4
+    assert ws(ptpc.OP_BENCH_UNSCALED_MM, 8192, 28672, 8192) == 256
 
 
 def test_ksplit_query_rejects_bad_shapes(ptpc):

@@ -330,3 +330,53 @@ def test_linear_on_column_slice(ptpc):
     assert_gemm_close(from_dev_bf16(out), ref, "column slice")
     dense = ptpc.linear(to_dev_bf16(X), Wq_t, ws)
     assert torch.equal(dense.view(torch.int16), out.view(torch.int16))
+
+
+@pytest.mark.parametrize("T,Ci,Co,fmt", [(256, 8192, 57344, "e4m3"), (300, 2048, 28672, "e4m3"),
+                                         (512, 4096, 10240, "e4m3"), (1000, 1024, 5120, "e4m3"),
+                                         (300, 2048, 28672, "e2m1"), (512, 4096, 10240, "e3m2")])
+def test_split_tail(ptpc, monkeypatch, T, Ci, Co, fmt):
+    """Prefill shapes whose last wave of tiles is split along K over the GPU
+    (partials through the workspace, distributed fixed-order reduction):
+    parity with the oracle, agreement with the whole-tile plan, repeated
+    calls on one workspace (its counters back at zero after each), no
+    timeout in the status word."""
+    assert ptpc.gemm_tail_split(T, Ci, Co) >= 2, "shape does not exercise the split tail"
+    X = synthetic.with_edge_rows(synthetic.make_x(synthetic.CHAIN_70B, 2, T, Ci), huge_bits=BIG_BF16)
+    W = synthetic.make_w(synthetic.CHAIN_70B, 2, Ci, Co)
+    Xd = to_dev_bf16(X)
+    Wq, ws_ = ptpc.quantize_weights_fmt(to_dev_bf16(W), fmt)
+    Xq, xs = ptpc.quantize_activations(Xd)
+    wsp = ptpc.Workspace(ptpc.workspace_size(ptpc.OP_LINEAR, T, Ci, Co), "cuda")
+    outs = [ptpc.scaled_mm_fmt(Xq, xs, Wq, ws_, fmt, ws=wsp) for _ in range(3)]
+    lin = ptpc.linear_fmt(Xd, Wq, ws_, fmt, ws=wsp)
+    assert ptpc.device_status(wsp) == ptpc.OK
+    assert int(wsp.buf[256:256 + 1024].count_nonzero()) == 0          # counters left at zero
+    for o in outs[1:] + [lin]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))   # deterministic
+    rXq, rxs = oracle.quant_act(X)
+    rows = np.unique(np.concatenate([np.arange(0, T, 7), [T - 1]]))
+    if fmt == "e4m3":
+        rWq, rws = oracle.quant_weight(W)
+        ref = oracle.scaled_mm_reference(rXq, rxs, rWq, rws, rows)
+    else:
+        codes, rws = oracle.quant_weight_fmt(W, fmt)
+        ref = oracle.scaled_mm_reference_fmt(rXq, rxs, codes, rws, fmt, rows)
+    assert_gemm_close(from_dev_bf16(outs[0])[rows], ref, f"split tail {fmt} T={T} {Ci}->{Co}")
+    # the whole-tile plan of the same shape agrees within the tolerance
+    try:
+        monkeypatch.setenv("PTPC_FORCE_SPLIT_TAIL", "0")
+        ptpc.reload_tuning_overrides()
+        assert ptpc.gemm_tail_split(T, Ci, Co) == 0
+        whole = ptpc.scaled_mm_fmt(Xq, xs, Wq, ws_, fmt, ws=wsp)
+    finally:
+        monkeypatch.delenv("PTPC_FORCE_SPLIT_TAIL")
+        ptpc.reload_tuning_overrides()
+    assert_gemm_close(from_dev_bf16(outs[0]), from_dev_bf16(whole), "split tail vs whole tiles")
+
+
+def test_split_tail_needs_the_workspace(ptpc):
+    """With only the status word of workspace the same shape runs whole tiles."""
+    assert ptpc.gemm_tail_split(256, 8192, 57344) >= 2
+    assert ptpc.gemm_tail_split(256, 8192, 57344, ws_bytes=256) == 0
+    assert ptpc.gemm_tail_split(8192, 8192, 57344) == 0       # last wave mostly full: no split
