@@ -62,6 +62,10 @@ SIGNATURES = {
     "ptpc_scaled_mm_static_scratch": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "ptpc_static_scratch_status": (ctypes.c_int, [_P]),
     "ptpc_weight_bytes": (ctypes.c_size_t, [ctypes.c_int, _I64, _I64]),
+    "ptpc_kv_cache_append": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
+    "ptpc_decode_attention_workspace_size": (ctypes.c_size_t, [_I64, _I64, _I64, _I64]),
+    "ptpc_decode_attention": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64,
+                                             _I64, _I64, ctypes.c_float, _P, _P, _SZ, _P]),
     "ptpc_act_row_amax": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P]),
     "ptpc_quantize_activations_amax": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P, _P]),
     "ptpc_quantize_weights_fmt": (ctypes.c_int, [_P, _I64, _I64, ctypes.c_int, _P, _P, _P, _SZ, _P]),
@@ -511,3 +515,48 @@ def quantize_weights_per_tensor(W, ws: Workspace | None = None):
            lib.ptpc_bench_quantize_weights_per_tensor(_ptr(W), Ci, Co, _ptr(Wq_t), _ptr(w_scale), ws.ptr(),
                                                       ws.nbytes, _stream(W.device)))
     return Wq_t, w_scale
+
+
+# ------------------------------------------------------------ FP8 KV cache
+
+def kv_cache_append(K, V, slots, k_cache, v_cache, k_scale, v_scale):
+    """Quantise K, V bf16 [T, H, D] per (token, head) to E4M3 and write them
+    to their slots of the paged caches: k_cache / v_cache uint8
+    [num_blocks, block_size, H, D], k_scale / v_scale fp32 [num_blocks,
+    block_size, H]; slots int64 [T] (block * block_size + offset, -1 skips)."""
+    _need(K, "K", torch.bfloat16, 3)
+    _need(V, "V", torch.bfloat16, 3)
+    _need(slots, "slots", torch.int64, 1)
+    _need(k_cache, "k_cache", torch.uint8, 4)
+    _need(v_cache, "v_cache", torch.uint8, 4)
+    _need(k_scale, "k_scale", torch.float32, 3)
+    _need(v_scale, "v_scale", torch.float32, 3)
+    T, H, D = K.shape
+    nb, bs = k_cache.shape[:2]
+    if V.shape != K.shape or k_cache.shape != (nb, bs, H, D) or v_cache.shape != k_cache.shape or \
+            k_scale.shape != (nb, bs, H) or v_scale.shape != k_scale.shape or slots.shape[0] != T:
+        raise ValueError("shape mismatch")
+    _check("ptpc_kv_cache_append",
+           lib.ptpc_kv_cache_append(_ptr(K), _ptr(V), _ptr(slots), T, H, D, bs, nb, _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(k_scale), _ptr(v_scale), _stream(K.device)))
+
+
+def decode_attention(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, max_context: int,
+                     softmax_scale: float, out: torch.Tensor | None = None, ws: Workspace | None = None):
+    """Decode attention over the FP8 paged cache: q bf16 [B, Hq, D],
+    block_tables int32 [B, max_blocks], context_lens int32 [B] (each at most
+    max_context) -> out bf16 [B, Hq, D]."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(block_tables, "block_tables", torch.int32, 2)
+    _need(context_lens, "context_lens", torch.int32, 1)
+    B, Hq, D = q.shape
+    nb, bs, Hkv, _ = k_cache.shape
+    out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device) if out is None else out
+    need = int(lib.ptpc_decode_attention_workspace_size(B, Hq, D, max_context))
+    ws = default_workspace(need, q.device) if ws is None else ws.ensure(need)
+    _check("ptpc_decode_attention",
+           lib.ptpc_decode_attention(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+                                     _ptr(block_tables), _ptr(context_lens), B, Hq, Hkv, D, bs, nb,
+                                     block_tables.shape[1], max_context, float(softmax_scale), _ptr(out), ws.ptr(),
+                                     ws.nbytes, _stream(q.device)))
+    return out

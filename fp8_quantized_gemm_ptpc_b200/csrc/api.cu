@@ -299,6 +299,65 @@ int ptpc_gemm_tail_split(int64_t T, int64_t Ci, int64_t Co, size_t ws_bytes) {
   return ptpc::gemm_tail_split((int)T, (int)Ci, (int)Co, ws_bytes);
 }
 
+// ------------------------------------------------------------------ FP8 KV cache
+
+namespace {
+int check_kv_dims(int64_t H, int64_t D, int64_t block_size, int64_t num_blocks) {
+  if (H <= 0 || D <= 0 || block_size <= 0 || num_blocks <= 0) return PTPC_ERR_INVALID_ARG;
+  if ((D != 64 && D != 128) || H > 1024 || block_size > 65536 || num_blocks > kMaxDim) return PTPC_ERR_UNSUPPORTED_SHAPE;
+  return PTPC_OK;
+}
+}  // namespace
+
+int ptpc_kv_cache_append(const void *K, const void *V, const int64_t *slots, int64_t T, int64_t H, int64_t D,
+                         int64_t block_size, int64_t num_blocks, uint8_t *k_cache, uint8_t *v_cache, float *k_scale,
+                         float *v_scale, void *stream) {
+  int s = check_kv_dims(H, D, block_size, num_blocks);
+  if (s != PTPC_OK) return s;
+  if (T < 0) return PTPC_ERR_INVALID_ARG;
+  if (T > kMaxDim || T * H > kMaxDim) return PTPC_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return PTPC_OK;
+  if (!K || !V || !slots || !k_cache || !v_cache || !k_scale || !v_scale) return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(K) || !aligned16(V) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (reinterpret_cast<uintptr_t>(slots) & 7u) || (reinterpret_cast<uintptr_t>(k_scale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+    return PTPC_ERR_MISALIGNED;
+  if ((s = check_device()) != PTPC_OK) return s;
+  return cuda_status(ptpc::launch_kv_append(K, V, slots, (int)T, (int)H, (int)D, num_blocks * block_size, k_cache,
+                                            v_cache, k_scale, v_scale, (cudaStream_t)stream));
+}
+
+size_t ptpc_decode_attention_workspace_size(int64_t B, int64_t Hq, int64_t D, int64_t max_context) {
+  if (B <= 0 || Hq <= 0 || (D != 64 && D != 128) || max_context < 0 || max_context > kMaxDim) return 0;
+  return round_up(ptpc::attn_workspace_bytes((int)B, (int)Hq, (int)D, (int)max_context));
+}
+
+int ptpc_decode_attention(const void *q, const uint8_t *k_cache, const uint8_t *v_cache, const float *k_scale,
+                          const float *v_scale, const int32_t *block_tables, const int32_t *context_lens, int64_t B,
+                          int64_t Hq, int64_t Hkv, int64_t D, int64_t block_size, int64_t num_blocks,
+                          int64_t max_blocks, int64_t max_context, float softmax_scale, void *out, void *ws,
+                          size_t ws_bytes, void *stream) {
+  int s = check_kv_dims(Hkv, D, block_size, num_blocks);
+  if (s != PTPC_OK) return s;
+  if (B < 0 || Hq <= 0 || max_blocks <= 0 || max_context < 0) return PTPC_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0 || Hq / Hkv > 16 || B > 65535 || Hkv > 65535 || max_context > kMaxDim ||
+      max_blocks > kMaxDim / block_size)
+    return PTPC_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0) return PTPC_OK;
+  if (!q || !k_cache || !v_cache || !k_scale || !v_scale || !block_tables || !context_lens || !out || !ws)
+    return PTPC_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned16(ws) ||
+      (reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u) ||
+      (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+    return PTPC_ERR_MISALIGNED;
+  if (ws_bytes < ptpc_decode_attention_workspace_size(B, Hq, D, max_context)) return PTPC_ERR_WORKSPACE_TOO_SMALL;
+  if ((s = check_device()) != PTPC_OK) return s;
+  return cuda_status(ptpc::launch_decode_attention(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                                                   (int)B, (int)Hq, (int)Hkv, (int)D, (int)block_size,
+                                                   (int)max_blocks, num_blocks * block_size, (int)max_context,
+                                                   softmax_scale, out, ws, (cudaStream_t)stream));
+}
+
 int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co) {
   if (check_shape_tci(T, Ci) != PTPC_OK || check_co(Co) != PTPC_OK || T == 0) return 0;
   if (check_device() != PTPC_OK) return 0;

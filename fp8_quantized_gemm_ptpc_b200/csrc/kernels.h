@@ -25,6 +25,17 @@ cudaError_t launch_quant_weight(const void *W, int Ci, int Co, uint8_t *Wq_t, fl
 // 2 = E2M3, 3 = E3M2 (FP6); Wp [Co, Ci * bits / 8] packed along K; Ci % 128 == 0.
 cudaError_t launch_quant_weight_sub(const void *W, int Ci, int Co, int fmt, uint8_t *Wp, float *w_scale,
                                     uint32_t *col_amax, cudaStream_t st);
+// FP8 KV cache (quant.cu, attention.cu): append K/V [T, H, D] bf16 rows to
+// slot-major caches ([num_slots, H, D] codes, [num_slots, H] scales), and
+// decode attention over them (workspace attn_workspace_bytes).
+cudaError_t launch_kv_append(const void *K, const void *V, const int64_t *slots, int T, int H, int D,
+                             int64_t num_slots, uint8_t *kc, uint8_t *vc, float *ks, float *vs, cudaStream_t st);
+size_t attn_workspace_bytes(int B, int Hq, int D, int max_context);
+cudaError_t launch_decode_attention(const void *q, const uint8_t *kc, const uint8_t *vc, const float *ks,
+                                    const float *vs, const int32_t *block_tables, const int32_t *context_lens,
+                                    int B, int Hq, int Hkv, int D, int block_size, int max_blocks,
+                                    int64_t num_slots, int max_context, float softmax_scale, void *out, void *ws,
+                                    cudaStream_t st);
 cudaError_t launch_apply_scales(const float *y, const float *xs, const float *ws, int T, int Co, void *out,
                                 cudaStream_t st);
 

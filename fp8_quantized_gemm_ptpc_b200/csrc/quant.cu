@@ -609,6 +609,52 @@ __global__ void __launch_bounds__(kSbThreads) quant_weight_sub_kernel(const uint
 }
 
 // ----------------------------------------------------------------------------
+// FP8 KV cache, append: every (token, head) vector of D values of K and V is
+// quantised with the per-token rule (s = amax / 448, the activation
+// quantiser's exact quotient) and written to its paged-cache slot:
+//   codes  cache[(slot * H + h) * D + d],  scale  scales[slot * H + h],
+// slot = slots[t] (block * block_size + offset; a negative slot skips the
+// token, a slot past the cache is skipped too).  D / 8 lanes own a vector
+// (one 16-byte load, 8 codes each); a warp holds 32 * 8 / D vectors.
+// ----------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) kv_append_kernel(const uint4 *__restrict__ K, const uint4 *__restrict__ V,
+                                                        const int64_t *__restrict__ slots, int T, int H,
+                                                        int64_t num_slots, uint8_t *__restrict__ kc,
+                                                        uint8_t *__restrict__ vc, float *__restrict__ ks,
+                                                        float *__restrict__ vs) {
+  constexpr int L = D / 8;              // lanes per vector
+  griddep_launch_dependents();
+  griddep_wait();
+  const int64_t vec = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / L;   // (t, h) row of K and V
+  const int lane = threadIdx.x % L;
+  const bool active = vec < (int64_t)T * H;
+  const int64_t t = active ? vec / H : 0;
+  const int h = active ? (int)(vec - t * H) : 0;
+  const int64_t slot = active ? slots[t] : -1;
+  const bool write = active && slot >= 0 && slot < num_slots;
+  #pragma unroll
+  for (int which = 0; which < 2; ++which) {
+    const uint4 *src = which == 0 ? K : V;
+    const uint4 v = active ? ld_stream(src + vec * L + lane) : make_uint4(0u, 0u, 0u, 0u);
+    uint32_t m = fold_halves(absmax_bits(0u, v));
+    #pragma unroll
+    for (int o = L / 2; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const GroupScale g = group_scale_from_amax_bits(m);
+    uint2 q;
+    if (g.mode == kFast)
+      q = quant_vec_fast(v, pack2(g.s), pack2(-g.r));
+    else
+      q = quant_vec(v, g);
+    if (write) {
+      uint8_t *dst = (which == 0 ? kc : vc) + (slot * H + h) * D;
+      reinterpret_cast<uint2 *>(dst)[lane] = q;
+      if (lane == 0) (which == 0 ? ks : vs)[slot * H + h] = g.s;
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
 // Naive two-step path, step 2: out = bf16((y * x_scale[t]) * w_scale[o]).
 // Each thread handles 8 consecutive outputs (two 16-byte fp32 loads, one
 // 16-byte bf16 store).
@@ -815,6 +861,20 @@ cudaError_t launch_quant_weight_sub(const void *W, int Ci, int Co, int fmt, uint
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // the workspace's scratch words are left zero for the next user
   return cudaMemsetAsync(col_amax, 0, sizeof(uint32_t) * ((size_t)Co + 1), st);
+}
+
+cudaError_t launch_kv_append(const void *K, const void *V, const int64_t *slots, int T, int H, int D,
+                             int64_t num_slots, uint8_t *kc, uint8_t *vc, float *ks, float *vs, cudaStream_t st) {
+  const int64_t threads = (int64_t)T * H * (D / 8);
+  const int grid = (int)((threads + 255) / 256);
+  const uint4 *Kv = static_cast<const uint4 *>(K);
+  const uint4 *Vv = static_cast<const uint4 *>(V);
+  switch (D) {
+    case 64: return launch_pdl(kv_append_kernel<64>, grid, 256, st, Kv, Vv, slots, T, H, num_slots, kc, vc, ks, vs);
+    case 128: return launch_pdl(kv_append_kernel<128>, grid, 256, st, Kv, Vv, slots, T, H, num_slots, kc, vc, ks, vs);
+    case 256: return launch_pdl(kv_append_kernel<256>, grid, 256, st, Kv, Vv, slots, T, H, num_slots, kc, vc, ks, vs);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_apply_scales(const float *y, const float *xs, const float *ws, int T, int Co, void *out,

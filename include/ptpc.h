@@ -296,6 +296,51 @@ PTPC_API int ptpc_scaled_mm_static_scratch(const uint8_t *Xq_dev, const float *x
 PTPC_API int ptpc_static_scratch_status(void *stream);
 
 /* ------------------------------------------------------------------------- */
+/* FP8 (E4M3) KV cache.  The PTPC page runs every evaluation with            */
+/* kv_cache_dtype=fp8_e4m3 (its lm-evaluation-harness commands).  The page    */
+/* gives no scale rule; this library applies the PTPC per-token rule to       */
+/* every (token, KV head) vector of D values: scale = amax / 448, codes       */
+/* E4M3_satRNE(x / scale), exactly as ptpc_quantize_activations on the rows   */
+/* of a [T * H, D] view.  The cache is paged and slot-major:                  */
+/*   codes  cache[(slot * H + h) * D + d]  (u8),  scale  scales[slot * H + h], */
+/*   slot = block * block_size + offset.                                      */
+/* ------------------------------------------------------------------------- */
+
+/* Appends T tokens: K_dev, V_dev bf16 [T, H, D]; slots_dev int64 [T] (a
+ * negative slot skips the token, as does a slot >= num_blocks * block_size);
+ * k_cache / v_cache u8 [num_blocks * block_size, H, D]; k_scale / v_scale
+ * fp32 [num_blocks * block_size, H].  D is 64 or 128.  Tokens with equal
+ * slots race. */
+PTPC_API int ptpc_kv_cache_append(const void *K_dev, const void *V_dev, const int64_t *slots_dev, int64_t T,
+                                  int64_t H, int64_t D, int64_t block_size, int64_t num_blocks,
+                                  uint8_t *k_cache_dev, uint8_t *v_cache_dev, float *k_scale_dev,
+                                  float *v_scale_dev, void *stream);
+
+/* Workspace bytes of ptpc_decode_attention (0 on invalid arguments). */
+PTPC_API size_t ptpc_decode_attention_workspace_size(int64_t B, int64_t Hq, int64_t D, int64_t max_context);
+
+/* Decode attention (one query per sequence) over the FP8 cache:
+ *   q_dev bf16 [B, Hq, D] (|q| < 65504), query head h reads KV head
+ *   h / (Hq / Hkv) (Hq / Hkv <= 16);
+ *   block_tables_dev int32 [B, max_blocks]: the cache blocks of each
+ *   sequence in order; context_lens_dev int32 [B]: positions to attend to
+ *   (<= max_context; positions whose block-table entry is missing, negative
+ *   or past the cache are left out);
+ *   out[b][h][d] = bf16_RNE(sum_l p_l * v_scale_l * dec(V_l[d])),
+ *   p = softmax_l(softmax_scale * k_scale_l * sum_d q[d] * dec(K_l[d]))
+ *   (0 for a sequence with no position), computed in fp32 with f16 tensor-
+ *   core products of the exactly decoded codes.  out_dev bf16 [B, Hq, D].
+ *   ws_dev: ptpc_decode_attention_workspace_size(B, Hq, D, max_context)
+ *   bytes (the context is split into chunks of 512 positions whose partial
+ *   results are combined by a second kernel). */
+PTPC_API int ptpc_decode_attention(const void *q_dev, const uint8_t *k_cache_dev, const uint8_t *v_cache_dev,
+                                   const float *k_scale_dev, const float *v_scale_dev,
+                                   const int32_t *block_tables_dev, const int32_t *context_lens_dev, int64_t B,
+                                   int64_t Hq, int64_t Hkv, int64_t D, int64_t block_size, int64_t num_blocks,
+                                   int64_t max_blocks, int64_t max_context, float softmax_scale, void *out_dev,
+                                   void *ws_dev, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------- */
 /* Measurement-only entry points: the comparison paths the page describes.  */
 /* ------------------------------------------------------------------------- */
 

@@ -392,3 +392,61 @@ def reference_epilogue(acc64: np.ndarray, x_scale, w_scale) -> np.ndarray:
     out = np.empty(acc.shape, dtype=np.uint16)
     _load().oracle_reference_epilogue_f64(_ptr(acc), acc.shape[0], acc.shape[1], _ptr(xs), _ptr(ws), _ptr(out))
     return out
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) KV cache and decode attention
+# --------------------------------------------------------------------------
+# Source: the PTPC page's evaluation commands, which run PTPC-FP8 with
+# kv_cache_dtype=fp8_e4m3 (the KV cache stored in E4M3).  The page gives no
+# scale rule; the reading here is the PTPC per-token rule applied to every
+# (token, KV head) vector of D values: s = amax / 448, codes E4M3_satRNE(x/s)
+# (quant_act on the rows of a [T * H, D] view).  The cache is paged: slot
+# = block * block_size + offset, codes [num_blocks, block_size, H, D] u8,
+# scales [num_blocks, block_size, H] f32.  Decode attention over it is the
+# plain definition, in fp64: for query head h (KV head g = h // (Hq / Hkv)),
+#   s_l = softmax_scale * sum_d q[h, d] * dec(K[l, g, d]) * k_scale[l, g],
+#   p = softmax(s),  out[h, d] = sum_l p_l * dec(V[l, g, d]) * v_scale[l, g],
+# rounded to bf16.
+
+def kv_quantize(KV_bits: np.ndarray):
+    """Per-(token, head) E4M3 quantisation of K or V, bf16 [T, H, D]:
+    (codes [T, H, D] u8, scales [T, H] f32)."""
+    T, H, D = KV_bits.shape
+    q, s = quant_act(np.ascontiguousarray(KV_bits).reshape(T * H, D))
+    return q.reshape(T, H, D), s.reshape(T, H)
+
+
+def kv_cache_write(cache_codes, cache_scales, codes, scales, slots, block_size: int):
+    """Scatter token rows into the paged cache (in place): token t goes to
+    block slots[t] // block_size, offset slots[t] % block_size."""
+    for t, slot in enumerate(np.asarray(slots)):
+        b, o = divmod(int(slot), block_size)
+        cache_codes[b, o] = codes[t]
+        cache_scales[b, o] = scales[t]
+
+
+def decode_attention_reference(q_bits, k_codes, k_scales, v_codes, v_scales, block_tables, context_lens,
+                               block_size: int, softmax_scale: float) -> np.ndarray:
+    """Decode attention over an E4M3 paged cache, fp64, rounded to bf16.
+    q_bits bf16 [B, Hq, D]; returns bf16 bits [B, Hq, D]."""
+    B, Hq, D = q_bits.shape
+    Hkv = k_codes.shape[2]
+    group = Hq // Hkv
+    dec = e4m3_decode_table()
+    q = bf16_to_float(q_bits).astype(np.float64)
+    out = np.empty((B, Hq, D), dtype=np.float64)
+    for b in range(B):
+        L = int(context_lens[b])
+        pos = np.arange(L)
+        blocks = np.asarray(block_tables[b])[pos // block_size]
+        offs = pos % block_size
+        K = dec[k_codes[blocks, offs]] * k_scales[blocks, offs][:, :, None].astype(np.float64)   # [L, Hkv, D]
+        V = dec[v_codes[blocks, offs]] * v_scales[blocks, offs][:, :, None].astype(np.float64)
+        for h in range(Hq):
+            g = h // group
+            s = softmax_scale * (K[:, g, :] @ q[b, h])
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            out[b, h] = p @ V[:, g, :]
+    return bf16_from_double(out)

@@ -159,3 +159,31 @@ def test_weight_format_argument_checks(ptpc):
         ptpc.ERR_WORKSPACE_TOO_SMALL
     assert lin(P(FAKE), 256, P(FAKE + 16), P(FAKE), 1, 16, 256, 64, P(FAKE), P(FAKE), need, None) == \
         ptpc.ERR_MISALIGNED
+
+
+def test_kv_cache_argument_checks(ptpc):
+    P = ctypes.c_void_p
+    ap = lambda *a: call(ptpc, "ptpc_kv_cache_append", *a)
+    args = [P(FAKE), P(FAKE), P(FAKE), 4, 8, 128, 16, 10, P(FAKE), P(FAKE), P(FAKE), P(FAKE), None]
+    bad = list(args); bad[5] = 96
+    assert ap(*bad) == ptpc.ERR_UNSUPPORTED_SHAPE          # head size 64 or 128
+    bad = list(args); bad[3] = -1
+    assert ap(*bad) == ptpc.ERR_INVALID_ARG
+    bad = list(args); bad[2] = P(FAKE + 4)
+    assert ap(*bad) == ptpc.ERR_MISALIGNED                 # int64 slots
+    bad = list(args); bad[3] = 0
+    assert ap(*bad) == ptpc.OK
+    wsz = lambda *a: call(ptpc, "ptpc_decode_attention_workspace_size", *a)
+    assert wsz(32, 64, 128, 4096) == 32 * 64 * 8 * (2 + 128) * 4
+    assert wsz(32, 64, 96, 4096) == 0
+    at = lambda *a: call(ptpc, "ptpc_decode_attention", *a)
+    need = wsz(2, 16, 128, 100)
+    base = [P(FAKE)] * 7 + [2, 16, 8, 128, 16, 10, 7, 100, ctypes.c_float(0.1), P(FAKE), P(FAKE), need, None]
+    bad = list(base); bad[8] = 12
+    assert at(*bad) == ptpc.ERR_UNSUPPORTED_SHAPE           # Hq not a multiple of Hkv
+    bad = list(base); bad[8] = 256; bad[9] = 8
+    assert at(*bad) == ptpc.ERR_UNSUPPORTED_SHAPE           # group of 32 query heads
+    bad = list(base); bad[-2] = need - 1
+    assert at(*bad) == ptpc.ERR_WORKSPACE_TOO_SMALL
+    bad = list(base); bad[7] = 0
+    assert at(*bad) == ptpc.OK

@@ -1,0 +1,152 @@
+"""GPU parity of the FP8 (E4M3) KV cache against the oracle: the append
+kernel's codes and scales bit for bit (the per-token rule on every
+(token, KV head) vector), and decode attention over the paged cache within
+|gpu - ref| <= 1e-2 |ref| + 1e-3 rms(ref) of the oracle's fp64 attention,
+over context lengths around the 16-position tiles and 512-position chunks,
+GQA groups of 1 to 16 query heads, head sizes 64 and 128, and block tables
+with missing entries."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from helpers import assert_gemm_close, from_dev_bf16, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ptpc():
+    import fp8_quantized_gemm_ptpc_b200 as p
+    return p
+
+
+def make_kv(T, H, D, seed):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = rng.standard_normal((T, H, D)).astype(np.float32)
+    x *= rng.lognormal(0.0, 1.0, size=(T, H, 1)).astype(np.float32)
+    x[:, :, rng.choice(D, 2, replace=False)] *= 20.0          # a few outlier channels per head
+    return synthetic.to_bf16_bits(x)
+
+
+def build_cache(ptpc, lens, Hkv, D, bs, seed, holes=False):
+    """Random block tables, K/V appended through the library; returns device
+    caches and the oracle's copies."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    B = len(lens)
+    max_blocks = max(1, max((l + bs - 1) // bs for l in lens))
+    nb = B * max_blocks + 3
+    perm = rng.permutation(nb)
+    tables = np.full((B, max_blocks), -1, np.int32)
+    k = 0
+    for b, l in enumerate(lens):
+        n = (l + bs - 1) // bs
+        tables[b, :n] = perm[k:k + n]
+        k += n
+    slots = []
+    for b, l in enumerate(lens):
+        for pos in range(l):
+            slots.append(tables[b, pos // bs] * bs + pos % bs)
+    T = len(slots)
+    K = make_kv(max(T, 1), Hkv, D, seed + 1)[:T]
+    V = make_kv(max(T, 1), Hkv, D, seed + 2)[:T]
+    kc = torch.zeros((nb, bs, Hkv, D), dtype=torch.uint8, device="cuda")
+    vc = torch.zeros_like(kc)
+    ksc = torch.zeros((nb, bs, Hkv), dtype=torch.float32, device="cuda")
+    vsc = torch.zeros_like(ksc)
+    if T:
+        ptpc.kv_cache_append(to_dev_bf16(K), to_dev_bf16(V), torch.tensor(slots, dtype=torch.int64, device="cuda"),
+                             kc, vc, ksc, vsc)
+    rk = np.zeros((nb, bs, Hkv, D), np.uint8); rv = np.zeros_like(rk)
+    rks = np.zeros((nb, bs, Hkv), np.float32); rvs = np.zeros_like(rks)
+    if T:
+        qk, sk = oracle.kv_quantize(K)
+        qv, sv = oracle.kv_quantize(V)
+        oracle.kv_cache_write(rk, rks, qk, sk, slots, bs)
+        oracle.kv_cache_write(rv, rvs, qv, sv, slots, bs)
+    if holes and max_blocks > 2:
+        tables[0, 1] = -1          # a missing block: its positions are left out on both sides
+    return (kc, vc, ksc, vsc, tables), (rk, rv, rks, rvs)
+
+
+def test_append_bit_exact(ptpc):
+    T, H, D, bs, nb = 300, 8, 128, 16, 32
+    K = make_kv(T, H, D, 1)
+    V = make_kv(T, H, D, 2)
+    K[3] = 0x8000                      # an all -0 token: scale 1, codes 0
+    rng = np.random.Generator(np.random.PCG64(3))
+    slots = rng.permutation(nb * bs)[:T].astype(np.int64)
+    slots[5] = -1                      # skipped
+    slots[6] = nb * bs + 7             # past the cache: skipped
+    kc = torch.full((nb, bs, H, D), 0xAB, dtype=torch.uint8, device="cuda")
+    vc = kc.clone()
+    ksc = torch.full((nb, bs, H), -7.0, device="cuda")
+    vsc = ksc.clone()
+    ptpc.kv_cache_append(to_dev_bf16(K), to_dev_bf16(V), torch.from_numpy(slots).cuda(), kc, vc, ksc, vsc)
+    rk = np.full((nb, bs, H, D), 0xAB, np.uint8); rv = rk.copy()
+    rks = np.full((nb, bs, H), -7.0, np.float32); rvs = rks.copy()
+    keep = [t for t in range(T) if 0 <= slots[t] < nb * bs]
+    qk, sk = oracle.kv_quantize(K[keep])
+    qv, sv = oracle.kv_quantize(V[keep])
+    oracle.kv_cache_write(rk, rks, qk, sk, slots[keep], bs)
+    oracle.kv_cache_write(rv, rvs, qv, sv, slots[keep], bs)
+    assert np.array_equal(kc.cpu().numpy(), rk) and np.array_equal(vc.cpu().numpy(), rv)
+    assert np.array_equal(ksc.cpu().numpy().view(np.uint32), rks.view(np.uint32))
+    assert np.array_equal(vsc.cpu().numpy().view(np.uint32), rvs.view(np.uint32))
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,D,bs", [
+    ([1, 15, 16, 17, 100], 8, 1, 128, 16),
+    ([511, 512, 513, 1030], 64, 8, 128, 16),
+    ([33, 700], 16, 16, 128, 32),
+    ([257, 1500], 32, 2, 64, 16),
+    ([0, 5, 2049], 28, 4, 128, 16),
+])
+def test_decode_attention(ptpc, lens, Hq, Hkv, D, bs):
+    dev, ref = build_cache(ptpc, lens, Hkv, D, bs, seed=sum(lens) + Hq, holes=True)
+    kc, vc, ksc, vsc, tables = dev
+    rk, rv, rks, rvs = ref
+    assert np.array_equal(kc.cpu().numpy(), rk) and np.array_equal(vsc.cpu().numpy(), rvs)
+    B = len(lens)
+    rng = np.random.Generator(np.random.PCG64(11))
+    q = synthetic.to_bf16_bits(rng.standard_normal((B, Hq, D)).astype(np.float32) * 2.0)
+    scale = 1.0 / math.sqrt(D)
+    max_ctx = max(lens)
+    out = ptpc.decode_attention(to_dev_bf16(q), kc, vc, ksc, vsc, torch.from_numpy(tables).cuda(),
+                                torch.tensor(lens, dtype=torch.int32, device="cuda"), max_ctx, scale)
+    # the oracle over the same table (missing entries: positions left out)
+    got = from_dev_bf16(out)
+    for b in range(B):
+        L = lens[b]
+        pos = [p for p in range(L) if tables[b, p // bs] >= 0]
+        if not pos:
+            assert not got[b].any() or np.all((got[b] & 0x7FFF) == 0)
+            continue
+        bt = np.array([[tables[b, p // bs] for p in pos]])
+        offs = [p % bs for p in pos]
+        # gather the positions into a one-position-per-block table for the reference
+        ck = rk[bt[0], offs][None].transpose(1, 0, 2, 3)     # [n, 1, Hkv, D]
+        cv = rv[bt[0], offs][None].transpose(1, 0, 2, 3)
+        cks = rks[bt[0], offs][:, None, :]
+        cvs = rvs[bt[0], offs][:, None, :]
+        r = oracle.decode_attention_reference(q[b:b + 1], ck, cks, cv, cvs, np.arange(len(pos))[None],
+                                              [len(pos)], 1, scale)
+        assert_gemm_close(got[b:b + 1], r, f"attention b={b} L={L} Hq={Hq} Hkv={Hkv} D={D}")
+
+
+def test_decode_attention_70b_shape(ptpc):
+    """Llama-3.1-70B attention at decode: 64 query heads on 8 KV heads, D =
+    128, 16-position blocks; a batch of mixed context lengths."""
+    lens = [4096, 1, 3000, 2048, 777, 4095]
+    dev, ref = build_cache(ptpc, lens, 8, 128, 16, seed=70)
+    kc, vc, ksc, vsc, tables = dev
+    rk, rv, rks, rvs = ref
+    rng = np.random.Generator(np.random.PCG64(12))
+    q = synthetic.to_bf16_bits(rng.standard_normal((len(lens), 64, 128)).astype(np.float32))
+    out = ptpc.decode_attention(to_dev_bf16(q), kc, vc, ksc, vsc, torch.from_numpy(tables).cuda(),
+                                torch.tensor(lens, dtype=torch.int32, device="cuda"), 4096, 1 / math.sqrt(128))
+    r = oracle.decode_attention_reference(q, rk, rks, rv, rvs, tables, lens, 16, 1 / math.sqrt(128))
+    assert_gemm_close(from_dev_bf16(out), r, "70B decode attention")

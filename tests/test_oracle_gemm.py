@@ -155,3 +155,44 @@ def test_row_subset_equals_full_rows():
     rows = [0, 3, 19, 7]
     full = oracle.scaled_mm_reference(Xq, xs, Wq_t, ws)
     assert np.array_equal(oracle.scaled_mm_reference(Xq, xs, Wq_t, ws, rows), full[rows])
+
+
+def test_kv_cache_oracle():
+    """The FP8 KV-cache oracle: per-(token, head) codes are the per-token
+    quantiser's on the [T * H, D] rows (scale = amax / 448, bit-exact), the
+    paged scatter puts every token at its slot, and decode attention reduces
+    to textbook cases: one context token returns its dequantised V exactly
+    (softmax of one score is 1), identical keys average the values, and a
+    dominant score selects its value."""
+    rng = np.random.Generator(np.random.PCG64(5))
+    T, H, D, bs = 20, 2, 64, 4
+    Kb = synthetic.to_bf16_bits(rng.standard_normal((T, H, D)).astype(np.float32))
+    codes, scales = oracle.kv_quantize(Kb)
+    q2, s2 = oracle.quant_act(Kb.reshape(T * H, D))
+    assert np.array_equal(codes.reshape(T * H, D), q2) and np.array_equal(scales.ravel(), s2)
+    amax = np.abs(oracle.bf16_to_float(Kb)).max(axis=2)
+    assert np.array_equal(scales, (amax / np.float32(448.0)).astype(np.float32))
+    nblk = 8
+    cc = np.zeros((nblk, bs, H, D), np.uint8)
+    cs = np.zeros((nblk, bs, H), np.float32)
+    slots = rng.permutation(nblk * bs)[:T]
+    oracle.kv_cache_write(cc, cs, codes, scales, slots, bs)
+    for t in range(T):
+        assert np.array_equal(cc[slots[t] // bs, slots[t] % bs], codes[t])
+    dec = oracle.e4m3_decode_table()
+    # one context token: the output is that token's dequantised V (p = 1)
+    qb = synthetic.to_bf16_bits(rng.standard_normal((1, 4, D)).astype(np.float32))
+    bt = np.array([[slots[0] // bs] + [0] * 7])
+    cc1 = np.zeros_like(cc); cs1 = np.zeros_like(cs)
+    cc1[slots[0] // bs, 0] = codes[0]; cs1[slots[0] // bs, 0] = scales[0]
+    out = oracle.decode_attention_reference(qb, cc1, cs1, cc1, cs1, bt, [1], bs, 0.125)
+    v = dec[codes[0]] * scales[0][:, None].astype(np.float64)
+    for h in range(4):
+        assert np.array_equal(out[0, h], oracle.bf16_from_double(v[h // 2]))
+    # identical keys: the output is the mean of the values
+    cc2 = np.zeros((2, bs, 1, D), np.uint8); cs2 = np.ones((2, bs, 1), np.float32)
+    cc2[:, :, 0, :] = codes[0, 0]
+    vc = np.zeros_like(cc2); vc[0, :, 0, :] = codes[:4, 0]; vc[1, :, 0, :] = codes[4:8, 0]
+    out = oracle.decode_attention_reference(qb[:, :1], cc2, cs2, vc, cs2, np.array([[0, 1]]), [8], bs, 0.5)
+    mean = dec[codes[:8, 0]].mean(axis=0)
+    assert np.allclose(oracle.bf16_to_float(out[0, 0]), mean, rtol=2 ** -8, atol=1e-12)
