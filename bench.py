@@ -70,6 +70,9 @@ def parse():
     ap.add_argument("--sweep-tokens", default=None, help="comma-separated T values for --sweep")
     ap.add_argument("--chain-tokens", default="1,256,3001",
                     help="T values of the chain summary inside the default line ('' to skip)")
+    ap.add_argument("--tp", action="store_true",
+                    help="tensor-parallel 70B MLP pair (column- then row-parallel) over the torchrun ranks")
+    ap.add_argument("--no-kv", action="store_true", help="skip the FP8 KV-cache decode-attention record")
     ap.add_argument("--decode-tokens", default="1,8,32,128",
                     help="T values of the decode record inside the default line ('' to skip)")
     return ap.parse_args()
@@ -405,6 +408,147 @@ def decode_record(ptpc, dev, peaks, tokens, steps):
             "per_T": out}
 
 
+def decode_subbyte_record(ptpc, dev, peaks, tokens, steps, fmts=("e3m2", "e2m1")):
+    """The 70B decode layers with FP6 (E3M2) and FP4 (E2M1) per-channel
+    weights: the same step as the decode record (per-token FP8 activations
+    quantised per call), the weights streaming 3/4 or 1/2 of the FP8 bytes.
+    Reports per T the step time, the weight bytes a step streams and the
+    GEMM launches against the HBM roofline on their algorithmic bytes."""
+    import torch
+    wl = synthetic.DECODE_70B
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    for fmt in fmts:
+        bits = ptpc.WEIGHT_BITS[fmt]
+        Ls = []
+        for i, L in enumerate(wl.layers):
+            Wb = torch.from_numpy(synthetic.make_w(wl, i, L.Ci, L.Co).view(np.int16)).to(dev).view(torch.bfloat16)
+            Wq, ws = ptpc.quantize_weights_fmt(Wb, fmt)
+            del Wb
+            Ls.append((L, Wq, ws))
+        per_T = {}
+        for T in tokens:
+            Xs = [torch.from_numpy(synthetic.make_x(wl, i, T, L.Ci).view(np.int16)).to(dev).view(torch.bfloat16)
+                  for i, (L, _, _) in enumerate(Ls)]
+            outs = [torch.empty((T, L.Co), dtype=torch.bfloat16, device=dev) for L, _, _ in Ls]
+            wsps = [ptpc.Workspace(ptpc.workspace_size(ptpc.OP_LINEAR, T, L.Ci, L.Co), dev) for L, _, _ in Ls]
+            q = [(torch.empty((T, L.Ci), dtype=torch.uint8, device=dev),
+                  torch.empty((T,), dtype=torch.float32, device=dev)) for L, _, _ in Ls]
+
+            def step():
+                for j, (L, Wq, ws) in enumerate(Ls):
+                    ptpc.linear_fmt(Xs[j], Wq, ws, fmt, out=outs[j], ws=wsps[j])
+
+            for _ in range(3):
+                step()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            e0.record(stream)
+            for _ in range(steps):
+                step()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms_step = e0.elapsed_time(e1) / steps
+            ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in Ls] for _ in range(steps)]
+            for j, (L, Wq, ws) in enumerate(Ls):
+                ptpc.quantize_activations(Xs[j], *q[j])
+            for it in range(steps):
+                for j, (L, Wq, ws) in enumerate(Ls):
+                    ev[it][j][0].record(stream)
+                    ptpc.scaled_mm_fmt(q[j][0], q[j][1], Wq, ws, fmt, out=outs[j], ws=wsps[j])
+                    ev[it][j][1].record(stream)
+            torch.cuda.synchronize(dev)
+            g_ms = [sum(ev[it][j][0].elapsed_time(ev[it][j][1]) for it in range(steps)) / steps
+                    for j in range(len(Ls))]
+            w_bytes = sum(L.Ci * L.Co * bits // 8 for L, _, _ in Ls)
+            g_bytes = sum(L.Ci * L.Co * bits // 8 + T * L.Ci + 2 * T * L.Co + 4 * (T + L.Co) for L, _, _ in Ls)
+            g_gbs = g_bytes / (sum(g_ms) / 1e3) / 1e9
+            per_T[str(T)] = {
+                "ms_per_step": ms_step, "weight_bytes_per_step": w_bytes,
+                "weight_bytes_vs_fp8": w_bytes / sum(L.Ci * L.Co for L, _, _ in Ls),
+                "gemm_ms": {L.name: g for (L, _, _), g in zip(Ls, g_ms)},
+                "roofline": {"bound": "hbm", "achieved": g_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": g_gbs / peaks["hbm_gbs"], "algorithmic_bytes": g_bytes},
+            }
+            del Xs, outs, wsps, q, ev
+        res[fmt] = per_T
+        del Ls
+        torch.cuda.empty_cache()
+    return {"workload": wl.name + ", sub-byte per-channel weights, FP8 per-token activations", "steps": steps,
+            "per_format": res}
+
+
+def kv_decode_record(ptpc, dev, peaks, B=32, ctx=4096, Hq=64, Hkv=8, D=128, bs=16, steps=50):
+    """Decode attention of a Llama-3.1-70B-shaped layer (64 query heads on 8
+    KV heads, D = 128) over the FP8 paged cache: B sequences of ctx cached
+    positions, blocks of bs positions in a shuffled order.  Algorithmic bytes
+    per step: the codes of K and V, their scales, q and the output.  Also
+    times appending one new token per sequence (the decode step's write)."""
+    import math
+
+    import torch
+    rng = np.random.Generator(np.random.PCG64(1234))
+    nblk = B * ctx // bs
+    tables = rng.permutation(nblk).astype(np.int32).reshape(B, ctx // bs)
+    kc = torch.empty((nblk, bs, Hkv, D), dtype=torch.uint8, device=dev)
+    vc = torch.empty_like(kc)
+    ksc = torch.empty((nblk, bs, Hkv), dtype=torch.float32, device=dev)
+    vsc = torch.empty_like(ksc)
+    # fill the cache through the append kernel, one chunk of tokens at a time
+    slots_all = (tables[:, :, None] * bs + np.arange(bs)[None, None, :]).reshape(-1)
+    g = torch.Generator(device=dev)
+    g.manual_seed(99)
+    for c0 in range(0, slots_all.size, 65536):
+        sl = torch.from_numpy(slots_all[c0:c0 + 65536].astype(np.int64)).to(dev)
+        K = torch.randn((sl.numel(), Hkv, D), device=dev, generator=g).to(torch.bfloat16)
+        V = torch.randn((sl.numel(), Hkv, D), device=dev, generator=g).to(torch.bfloat16)
+        ptpc.kv_cache_append(K, V, sl, kc, vc, ksc, vsc)
+        del K, V
+    q = torch.randn((B, Hq, D), device=dev, generator=g).to(torch.bfloat16)
+    bt = torch.from_numpy(tables).to(dev)
+    lens = torch.full((B,), ctx, dtype=torch.int32, device=dev)
+    out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=dev)
+    ws = ptpc.Workspace(int(ptpc.lib.ptpc_decode_attention_workspace_size(B, Hq, D, ctx)), dev)
+    stream = torch.cuda.current_stream(dev)
+    fn = lambda: ptpc.decode_attention(q, kc, vc, ksc, vsc, bt, lens, ctx, 1 / math.sqrt(D), out=out, ws=ws)
+    for _ in range(3):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    nbytes = B * ctx * Hkv * (2 * D + 8) + 2 * (2 * B * Hq * D)
+    # one new token per sequence: the decode step's cache write
+    Kn = torch.randn((B, Hkv, D), device=dev, generator=g).to(torch.bfloat16)
+    sl = torch.from_numpy(slots_all[:B].astype(np.int64)).to(dev)
+    for _ in range(3):
+        ptpc.kv_cache_append(Kn, Kn, sl, kc, vc, ksc, vsc)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(steps):
+        ptpc.kv_cache_append(Kn, Kn, sl, kc, vc, ksc, vsc)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_app = e0.elapsed_time(e1) / steps
+    gbs = nbytes / (ms / 1e3) / 1e9
+    rec = {
+        "workload": f"Llama-3.1-70B decode attention: {B} sequences x {ctx} cached positions, {Hq} query / "
+                    f"{Hkv} KV heads, D = {D}, {bs}-position blocks (shuffled), E4M3 codes + per-(token, head) scales",
+        "ms_per_step": ms, "algorithmic_bytes": nbytes,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "peak_src": f"{peaks['src']} HBM copy"},
+        "bf16_cache_bytes_would_be": B * ctx * Hkv * 2 * D * 2,
+        "append_one_token_per_sequence_us": ms_app * 1e3,
+    }
+    del kc, vc, ksc, vsc, q, out, ws
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -727,6 +871,10 @@ def run_gpu(args):
         dec_tokens = [int(t) for t in args.decode_tokens.split(",") if t.strip()]
         if dec_tokens:
             line["decode"] = decode_record(ptpc, dev, peaks, dec_tokens, steps=max(20, min(K * 2, 100)))
+            line["decode_subbyte"] = decode_subbyte_record(ptpc, dev, peaks, [t for t in dec_tokens if t in (1, 128)]
+                                                           or dec_tokens[:1], steps=max(20, min(K * 2, 100)))
+        if not args.no_kv:
+            line["kv_decode"] = kv_decode_record(ptpc, dev, peaks)
         chain_tokens = [int(t) for t in args.chain_tokens.split(",") if t.strip()]
         if chain_tokens:
             Ws = chain_weights(ptpc, dev)
@@ -924,6 +1072,68 @@ def run_sweep(args):
     return 0
 
 
+def run_tp(args):
+    """Tensor-parallel 70B MLP pair on N ranks (one GPU each, NCCL between
+    them): gate+up 8192 -> 57344 column-parallel (no collective), then down
+    28672 -> 8192 row-parallel on each rank's slice of the gate+up output
+    (the first 28672 / N of its columns, standing in for the SwiGLU between
+    the layers): a MAX all-reduce of T row maxima and a SUM all-reduce of the
+    T x 8192 fp32 accumulators.  Prints one JSON line (rank 0) with the step
+    time as the maximum over ranks and whole-job TFLOP/s."""
+    import torch
+    import torch.distributed as dist
+
+    from fp8_quantized_gemm_ptpc_b200.tp import ColumnParallelLinear, RowParallelLinear
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    wl = synthetic.LLAMA70B_PREFILL
+    T = args.tokens or wl.tokens[0]
+    to_dev = lambda bits: torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    X = to_dev(synthetic.make_x(wl, 0, T, 8192))
+    gate_up = ColumnParallelLinear(to_dev(synthetic.make_w(wl, 0, 8192, 57344)), rank, world)
+    down = RowParallelLinear(to_dev(synthetic.make_w(wl, 1, 28672, 8192)), rank, world)
+    width = down.k1 - down.k0
+
+    def step():
+        h = gate_up.forward(X)
+        return down.forward(h[:, :width])
+
+    stream = torch.cuda.current_stream(dev)
+    K, W = args.steps, max(3, args.warmup)
+    for _ in range(W):
+        step()
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = dist_max(e0.elapsed_time(e1), dev) / K
+    flops = 2.0 * T * 8192 * 57344 + 2.0 * T * 28672 * 8192        # the whole layer pair, over all ranks
+    if rank == 0:
+        print(json.dumps({
+            "metric": "tensor-parallel PTPC-FP8 70B MLP pair TFLOP/s", "value": flops / (ms / 1e3) / 1e12,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": K, "warmup": W, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "strong", "data": "synthetic",
+            "config": {"workload": f"70B gate_up 8192->57344 column-parallel + down 28672->8192 row-parallel, T={T}",
+                       "parallelism": f"tp{world}"},
+        }), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -932,6 +1142,8 @@ def main():
         return run_quant_only(args)
     if args.sweep:
         return run_sweep(args)
+    if args.tp:
+        return run_tp(args)
     return run_gpu(args)
 
 
