@@ -115,6 +115,32 @@ __device__ __forceinline__ uint2 quant_vec_fast(const uint4 v, uint64_t s2, uint
   return o;
 }
 
+// The fast path on x as it is: with -r in place of r the three steps give
+// -q exactly (signed zeros included: checked against the form above for every
+// (bf16 amax, bf16 x) pair with s >= 2^-100), so the codes come out with
+// their sign bits flipped, which one XOR per four codes undoes.  This saves
+// building -x for every element.
+__device__ __forceinline__ uint32_t quant_x2_negated(uint32_t w, uint64_t s2, uint64_t nr2) {
+  const uint32_t lo = w << 16, hi = w & 0xFFFF0000u;
+  uint64_t x2, nq0, e, nq;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x2) : "r"(lo), "r"(hi));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(nq0) : "l"(x2), "l"(nr2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(e) : "l"(nq0), "l"(s2), "l"(x2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(nq) : "l"(e), "l"(nr2), "l"(nq0));
+  uint32_t a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(nq));
+  uint16_t c;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c) : "r"(b), "r"(a));
+  return (uint32_t)c;
+}
+
+__device__ __forceinline__ uint2 quant_vec_fast_flip(const uint4 v, uint64_t s2, uint64_t nr2) {
+  uint2 o;
+  o.x = (quant_x2_negated(v.x, s2, nr2) | (quant_x2_negated(v.y, s2, nr2) << 16)) ^ 0x80808080u;
+  o.y = (quant_x2_negated(v.z, s2, nr2) | (quant_x2_negated(v.w, s2, nr2) << 16)) ^ 0x80808080u;
+  return o;
+}
+
 // Eight bf16 (16 bytes) -> eight codes (8 bytes), any mode.
 __device__ __forceinline__ uint2 quant_vec(const uint4 v, const GroupScale &g) {
   if (g.mode == kZeroGroup) return make_uint2(0u, 0u);
@@ -245,6 +271,80 @@ __global__ void __launch_bounds__(V >= 16 ? 512 : 1024) quant_act_kernel(const u
       const int j = lt + i * P;
       if (j < nvec) qr[j] = quant_vec(v[i], g);
     }
+  }
+}
+
+// Rows that split exactly into V vectors per thread x P threads (P a
+// multiple of 32): the same algorithm as quant_act_kernel without any
+// per-vector bounds check, with P known at compile time for the common model
+// widths (PC; 0 = P at run time) so every load and store takes an immediate
+// offset, and the row's scale computed once by its first thread and
+// broadcast through shared memory.  Measured with the same counters: 5.4
+// instead of 9.7 instructions per element at 8192 columns, which is what
+// decides the throughput when the power cap holds the SM clock near 1 GHz.
+template <int V, int SRC, int PC>
+__global__ void __launch_bounds__(V >= 16 ? 512 : 1024) quant_act_exact_kernel(
+    const uint4 *__restrict__ X, int T, int64_t ldv, uint8_t *__restrict__ Xq, float *__restrict__ xs, int p_rt,
+    const uint32_t *__restrict__ tensor_amax, const float *__restrict__ given_amax) {
+  __shared__ uint32_t red[32];
+  __shared__ float sb_s[32], sb_r[32];
+  __shared__ int sb_mode[32];
+  griddep_launch_dependents();
+  griddep_wait();
+  const int P = PC ? PC : p_rt;
+  const int tid = threadIdx.x;
+  const int rl = tid / P;
+  const int lt = tid - rl * P;
+  const int R = blockDim.x / P;
+  const int64_t row = (int64_t)blockIdx.x * R + rl;
+  const bool active = row < T;
+  const uint4 *xr = X + row * ldv + lt;
+  uint4 v[V];
+  if (active) {
+    #pragma unroll
+    for (int i = 0; i < V; ++i) v[i] = ld_stream(xr + i * P);
+  } else {
+    #pragma unroll
+    for (int i = 0; i < V; ++i) v[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if constexpr (SRC == kAmaxRow) {
+    uint32_t m = 0;
+    #pragma unroll
+    for (int i = 0; i < V; ++i) m = absmax_bits(m, v[i]);
+    m = __reduce_max_sync(0xffffffffu, fold_halves(m));
+    if ((tid & 31) == 0) red[tid >> 5] = m;
+    __syncthreads();
+  }
+  if (lt == 0) {
+    uint32_t amax_bits = 0;
+    if constexpr (SRC == kAmaxTensor) {
+      amax_bits = *tensor_amax;
+    } else if constexpr (SRC == kAmaxGiven) {
+      amax_bits = active ? __float_as_uint(given_amax[row]) >> 16 : 0u;
+    } else {
+      const int w0 = rl * (P >> 5);
+      for (int w = 0; w < (P >> 5); ++w) amax_bits = max(amax_bits, red[w0 + w]);
+    }
+    const GroupScale g = group_scale_from_amax_bits(amax_bits);
+    sb_s[rl] = g.s;
+    sb_r[rl] = g.r;
+    sb_mode[rl] = g.mode;
+    if (active) xs[row] = g.s;
+  }
+  __syncthreads();
+  if (!active) return;
+  GroupScale g;
+  g.s = sb_s[rl];
+  g.r = sb_r[rl];
+  g.mode = sb_mode[rl];
+  uint2 *qr = reinterpret_cast<uint2 *>(Xq + row * (int64_t)V * P * 8) + lt;
+  if (g.mode == kFast) {
+    const uint64_t s2 = pack2(g.s), nr2 = pack2(-g.r);
+    #pragma unroll
+    for (int i = 0; i < V; ++i) qr[i * P] = quant_vec_fast_flip(v[i], s2, nr2);
+  } else {
+    #pragma unroll
+    for (int i = 0; i < V; ++i) qr[i * P] = quant_vec(v[i], g);
   }
 }
 
@@ -732,13 +832,47 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, cudaStream
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Exact split of a row of nvec vectors: V vectors per thread x P threads, P
+// a multiple of 32 (at most 1024 threads, 512 with 16 vectors); V = 0 if no
+// such split exists.
+ActPlan plan_act_exact(int nvec) {
+  for (int V : {8, 4, 16}) {
+    if (nvec % (32 * V) != 0) continue;
+    const int P = nvec / V;
+    if (P > (V >= 16 ? 512 : 1024)) continue;
+    return ActPlan{V, P, P >= 256 ? 1 : 256 / P};
+  }
+  return ActPlan{0, 0, 0};
+}
+
+template <int V, int SRC, int PC>
+cudaError_t launch_exact(const ActPlan &p, const uint4 *Xv, int T, int64_t ldv, uint8_t *Xq, float *xs,
+                         const uint32_t *tensor_amax, const float *given_amax, cudaStream_t st) {
+  const int grid = (T + p.R - 1) / p.R;
+  return launch_pdl(quant_act_exact_kernel<V, SRC, PC>, grid, p.P * p.R, st, Xv, T, ldv, Xq, xs, p.P, tensor_amax,
+                    given_amax);
+}
+
 template <int SRC>
 cudaError_t launch_act(const void *X, int T, int Ci, int64_t ldx, uint8_t *Xq, float *xs,
                        const uint32_t *tensor_amax, const float *given_amax, cudaStream_t st) {
   const int nvec = Ci / 8;
   const int64_t ldv = ldx / 8;
-  const ActPlan p = plan_act(nvec);
   const uint4 *Xv = static_cast<const uint4 *>(X);
+  const ActPlan e = plan_act_exact(nvec);
+  if (e.V == 8) {
+    // the model widths of the workloads: 4096, 8192, 14336, 28672 columns
+    switch (e.P) {
+      case 64: return launch_exact<8, SRC, 64>(e, Xv, T, ldv, Xq, xs, tensor_amax, given_amax, st);
+      case 128: return launch_exact<8, SRC, 128>(e, Xv, T, ldv, Xq, xs, tensor_amax, given_amax, st);
+      case 224: return launch_exact<8, SRC, 224>(e, Xv, T, ldv, Xq, xs, tensor_amax, given_amax, st);
+      case 448: return launch_exact<8, SRC, 448>(e, Xv, T, ldv, Xq, xs, tensor_amax, given_amax, st);
+      default: return launch_exact<8, SRC, 0>(e, Xv, T, ldv, Xq, xs, tensor_amax, given_amax, st);
+    }
+  }
+  if (e.V == 4) return launch_exact<4, SRC, 0>(e, Xv, T, ldv, Xq, xs, tensor_amax, given_amax, st);
+  if (e.V == 16) return launch_exact<16, SRC, 0>(e, Xv, T, ldv, Xq, xs, tensor_amax, given_amax, st);
+  const ActPlan p = plan_act(nvec);
   if (p.V == 0)
     return launch_pdl(quant_act_long_kernel<SRC>, T, 1024, st, Xv, T, nvec, ldv, Xq, xs, tensor_amax, given_amax);
   const int grid = (T + p.R - 1) / p.R;
