@@ -68,7 +68,7 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="70B 4-linear chain: fused vs naive two-step vs per-tensor, one JSON line per T")
     ap.add_argument("--sweep-tokens", default=None, help="comma-separated T values for --sweep")
-    ap.add_argument("--chain-tokens", default="1,256,3001",
+    ap.add_argument("--chain-tokens", default="1,256,300,512,1000,3001",
                     help="T values of the chain summary inside the default line ('' to skip)")
     ap.add_argument("--tp", action="store_true",
                     help="tensor-parallel 70B MLP pair (column- then row-parallel) over the torchrun ranks")
