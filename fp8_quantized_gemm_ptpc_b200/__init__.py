@@ -73,6 +73,7 @@ SIGNATURES = {
     "ptpc_linear_fmt": (ctypes.c_int, [_P, _I64, _P, _P, ctypes.c_int, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "ptpc_reload_tuning_overrides": (ctypes.c_int, []),
     "ptpc_bench_map_cache_stats": (ctypes.c_int, [_P, _P]),
+    "ptpc_bench_map_cache_selftest": (ctypes.c_int, []),
     "ptpc_bench_unscaled_mm_f32": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "ptpc_bench_apply_scales": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _P, _P]),
     "ptpc_bench_clock_probe": (ctypes.c_int, [_P, ctypes.c_int, ctypes.c_uint64, ctypes.c_uint64, _P, _P]),

@@ -369,6 +369,8 @@ int ptpc_reload_tuning_overrides(void) {
   return PTPC_OK;
 }
 
+int ptpc_bench_map_cache_selftest(void) { return ptpc::map_cache_selftest() == 0 ? PTPC_OK : PTPC_ERR_INVALID_ARG; }
+
 int ptpc_bench_map_cache_stats(uint64_t *hits, uint64_t *misses) {
   if (!hits || !misses) return PTPC_ERR_INVALID_ARG;
   ptpc::map_cache_stats(hits, misses);

@@ -978,14 +978,49 @@ struct MapKeyHash {
   }
 };
 
-// Encoded tensor maps, shared by every device and host thread.  Layers call
-// the GEMM with the same buffers again and again, so after the first call of
-// a layer its maps come from here instead of being encoded anew.  Bounded:
-// the cache is emptied when it reaches kMapCacheMax entries.
+// Encoded tensor maps, keyed by what they encode.  Layers call the GEMM with
+// the same buffers again and again, so after the first call of a layer its
+// maps come from here instead of being encoded anew.  Bounded: emptied when
+// it reaches `cap` entries.  Thread-safe; the encoder runs outside the lock.
+class MapCache {
+ public:
+  explicit MapCache(size_t cap) : cap_(cap) {}
+
+  template <typename Encoder>
+  bool get(CUtensorMap *m, const MapKey &k, Encoder encode) {
+    {
+      std::lock_guard<std::mutex> lock(mu_);
+      auto it = map_.find(k);
+      if (it != map_.end()) {
+        *m = it->second;
+        hits_.fetch_add(1, std::memory_order_relaxed);
+        return true;
+      }
+    }
+    if (!encode(m, k)) return false;
+    misses_.fetch_add(1, std::memory_order_relaxed);
+    std::lock_guard<std::mutex> lock(mu_);
+    if (map_.size() >= cap_) map_.clear();
+    map_.emplace(k, *m);
+    return true;
+  }
+
+  uint64_t hits() const { return hits_.load(std::memory_order_relaxed); }
+  uint64_t misses() const { return misses_.load(std::memory_order_relaxed); }
+  size_t size() {
+    std::lock_guard<std::mutex> lock(mu_);
+    return map_.size();
+  }
+
+ private:
+  size_t cap_;
+  std::mutex mu_;
+  std::unordered_map<MapKey, CUtensorMap, MapKeyHash> map_;
+  std::atomic<uint64_t> hits_{0}, misses_{0};
+};
+
 constexpr size_t kMapCacheMax = 4096;
-std::mutex g_map_mu;
-std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_map_cache;
-std::atomic<uint64_t> g_map_hits{0}, g_map_misses{0};
+MapCache g_maps(kMapCacheMax);   // shared by every device and host thread
 
 bool encode_map_2d(CUtensorMap *m, const MapKey &k) {
   EncodeTiledFn fn = encode_fn();
@@ -1002,21 +1037,7 @@ bool encode_map_2d(CUtensorMap *m, const MapKey &k) {
 bool make_map_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
   const MapKey k{base, inner, outer, row_bytes, box_inner, box_outer, (int)dt, (int)sw};
-  {
-    std::lock_guard<std::mutex> lock(g_map_mu);
-    auto it = g_map_cache.find(k);
-    if (it != g_map_cache.end()) {
-      *m = it->second;
-      g_map_hits.fetch_add(1, std::memory_order_relaxed);
-      return true;
-    }
-  }
-  if (!encode_map_2d(m, k)) return false;
-  g_map_misses.fetch_add(1, std::memory_order_relaxed);
-  std::lock_guard<std::mutex> lock(g_map_mu);
-  if (g_map_cache.size() >= kMapCacheMax) g_map_cache.clear();
-  g_map_cache.emplace(k, *m);
-  return true;
+  return g_maps.get(m, k, encode_map_2d);
 }
 
 // Tensor map of the weight codes Wq [Co, Ci]: one byte per code (E4M3), or
@@ -1401,8 +1422,44 @@ int num_sms() { return device_info().sms; }
 void reload_tuning() { g_tuning.store(pack_tuning(read_tuning()), std::memory_order_relaxed); }
 
 void map_cache_stats(uint64_t *hits, uint64_t *misses) {
-  *hits = g_map_hits.load(std::memory_order_relaxed);
-  *misses = g_map_misses.load(std::memory_order_relaxed);
+  *hits = g_maps.hits();
+  *misses = g_maps.misses();
+}
+
+int map_cache_selftest() {
+  // a private cache of 4 entries and an encoder that only counts its calls
+  // and stamps the key's pointer into the map
+  MapCache c(4);
+  int encodes = 0;
+  auto fake = [&](CUtensorMap *m, const MapKey &k) {
+    ++encodes;
+    std::memset(m, 0, sizeof(*m));
+    std::memcpy(m, &k.base, sizeof(k.base));
+    return true;
+  };
+  auto key = [](uintptr_t base, uint64_t rows) {
+    return MapKey{reinterpret_cast<const void *>(base), 4096, rows, 4096, 128, 128, 0, 3};
+  };
+  CUtensorMap m;
+  const void *got = nullptr;
+  int fails = 0;
+  auto check = [&](bool ok) { fails += ok ? 0 : 1; };
+  check(c.get(&m, key(0x1000, 64), fake) && encodes == 1 && c.misses() == 1 && c.hits() == 0);
+  check(c.get(&m, key(0x1000, 64), fake) && encodes == 1 && c.hits() == 1);          // hit
+  std::memcpy(&got, &m, sizeof(got));
+  check(got == reinterpret_cast<const void *>(0x1000));
+  check(c.get(&m, key(0x2000, 64), fake) && encodes == 2);                           // same shape, other pointer
+  std::memcpy(&got, &m, sizeof(got));
+  check(got == reinterpret_cast<const void *>(0x2000));
+  check(c.get(&m, key(0x1000, 128), fake) && encodes == 3);                          // same pointer, other shape
+  check(c.get(&m, key(0x1000, 64), fake) && encodes == 3 && c.hits() == 2);          // still cached
+  check(c.size() == 3);
+  check(c.get(&m, key(0x3000, 64), fake) && c.size() == 4);
+  check(c.get(&m, key(0x4000, 64), fake) && c.size() == 1 && encodes == 5);          // full: emptied, then added
+  check(c.get(&m, key(0x1000, 64), fake) && encodes == 6);                           // gone with the rest
+  auto failing = [](CUtensorMap *, const MapKey &) { return false; };
+  check(!c.get(&m, key(0x5000, 64), failing) && c.size() == 2);                      // a failed encode is not stored
+  return fails;
 }
 
 int gemm_ksplit(int T, int Ci, int Co) { return make_plan(T, Ci, Co, gemm_workspace_bytes(T, Ci, Co)).ksplit; }

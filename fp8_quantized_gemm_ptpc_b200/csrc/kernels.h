@@ -78,4 +78,8 @@ void reload_tuning();
 // Tensor-map cache counters since the library was loaded.
 void map_cache_stats(uint64_t *hits, uint64_t *misses);
 
+// The cache's own logic on a private instance with a stand-in encoder (no
+// GPU needed): number of failed checks, 0 when it behaves.
+int map_cache_selftest();
+
 }  // namespace ptpc

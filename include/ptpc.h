@@ -360,6 +360,12 @@ PTPC_API int ptpc_bench_unscaled_mm_f32(const uint8_t *Xq_dev, const uint8_t *Wq
  * No counterpart on the page. */
 PTPC_API int ptpc_bench_map_cache_stats(uint64_t *hits, uint64_t *misses);
 
+/* Self-test of the tensor-map cache's logic on a private instance with a
+ * stand-in encoder (no GPU needed): hits, misses for another pointer or shape,
+ * emptying at capacity, failed encodes not stored.  PTPC_OK if every check
+ * holds.  No counterpart on the page. */
+PTPC_API int ptpc_bench_map_cache_selftest(void);
+
 /* Effective SM clock during a measurement: one sleeping thread on one SM
  * writes (globaltimer ns, clock64 cycles) pairs to records_dev
  * (uint64 [max_records][2], 8-byte aligned) about every period_ns (>= 1000)

@@ -187,3 +187,10 @@ def test_kv_cache_argument_checks(ptpc):
     assert at(*bad) == ptpc.ERR_WORKSPACE_TOO_SMALL
     bad = list(base); bad[7] = 0
     assert at(*bad) == ptpc.OK
+
+
+def test_tensor_map_cache_logic(ptpc):
+    """The host-side tensor-map cache (hits, misses for another pointer or
+    shape, emptying at capacity, failed encodes) on a private instance with a
+    stand-in encoder: no GPU needed."""
+    assert call(ptpc, "ptpc_bench_map_cache_selftest") == ptpc.OK
