@@ -304,7 +304,8 @@ int ptpc_gemm_tail_split(int64_t T, int64_t Ci, int64_t Co, size_t ws_bytes) {
 namespace {
 int check_kv_dims(int64_t H, int64_t D, int64_t block_size, int64_t num_blocks) {
   if (H <= 0 || D <= 0 || block_size <= 0 || num_blocks <= 0) return PTPC_ERR_INVALID_ARG;
-  if ((D != 64 && D != 128) || H > 1024 || block_size > 65536 || num_blocks > kMaxDim) return PTPC_ERR_UNSUPPORTED_SHAPE;
+  if ((D != 64 && D != 128) || H > 1024 || block_size < 8 || block_size > 65536 || num_blocks > kMaxDim)
+    return PTPC_ERR_UNSUPPORTED_SHAPE;
   return PTPC_OK;
 }
 }  // namespace

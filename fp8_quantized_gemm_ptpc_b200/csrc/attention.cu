@@ -12,18 +12,21 @@
 //   out[h, d] = sum_l softmax(s)_l * v_scale[l] * dec(V[l, d]).
 //
 // Decode is bound by the bytes of the cache it streams (one byte per code).
-// A CTA takes one (sequence, KV head) and a chunk of kChunk context
-// positions; its four warps take 16-position tiles in turn.  A warp gathers a
-// tile's K and V codes through the block table (16-byte loads), decodes them
-// exactly to f16 in shared memory (cvt e4m3x2 -> f16x2; every E4M3 value is an
-// f16 value) and runs FlashAttention-style tensor-core MMAs (mma.sync
-// m16n8k16, f16 inputs, fp32 accumulation) with the GQA group's query heads
-// as the 16 rows: S = Q K^T, an online softmax in base 2, O += P V.  The key
-// scales multiply the scores; the value scales enter P relative to the
-// chunk's largest one (so P stays in [0, 1] in f16) and that one multiplies
-// the accumulator at the end.  The warps' states are combined in shared
-// memory and every CTA writes (max, sum, accumulator) for its chunk; a second
-// kernel combines the chunks of a head and rounds to bf16.
+// A CTA takes one (sequence, KV head) and a chunk of 512 context positions,
+// whose block-table entries it first reads into shared memory; its four warps
+// take 16-position tiles in turn.  A warp gathers a tile's K and V codes and
+// scales with asynchronous copies (cp.async, 16 bytes per copy, zero-filled
+// for positions that are not read) into one of two shared-memory stages, so
+// the next tile's bytes are in flight while it decodes this one exactly to
+// f16 (cvt e4m3x2 -> f16x2; every E4M3 value is an f16 value) and runs
+// FlashAttention-style tensor-core MMAs (mma.sync m16n8k16, f16 inputs, fp32
+// accumulation) with the GQA group's query heads as the 16 rows: S = Q K^T,
+// an online softmax in base 2, O += P V.  The key scales multiply the scores;
+// the value scales enter P relative to the tile's largest one (so P stays in
+// [0, 1] in f16), and the accumulator is kept in units of that value scale
+// (moved between tiles with the softmax's own rescale).  The warps' states
+// are combined in shared memory and every CTA writes (max, sum, accumulator)
+// for its chunk; a second kernel combines the chunks and rounds to bf16.
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -111,44 +114,97 @@ __device__ __forceinline__ int64_t kv_slot(const AttnParams &p, int b, int pos) 
   return (blk < 0 || slot >= p.num_slots) ? -1 : slot;
 }
 
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+constexpr int kMinBlockSize = 8;   // the chunk's block-table entries fit in shared memory
+
+// Shared memory of one CTA: every warp's two code stages (K and V codes and
+// scales of 16 positions) and its decoded f16 K and V tiles, which at the end
+// double as the warps' accumulators; the chunk's block-table entries.
+template <int D, int CHUNK>
+struct AttnSmem {
+  static constexpr int PITCH = D + 8;                                   // f16 per decoded row
+  static constexpr int CODE_STAGE = 2 * 16 * D;                         // bytes: K and V codes
+  static constexpr int CODES = kAttnWarps * 2 * CODE_STAGE;
+  static constexpr int TILES = kAttnWarps * 2 * 16 * PITCH * 2;         // bytes: decoded K and V
+  static constexpr int SCALES = kAttnWarps * 2 * 2 * 16 * 4;            // bytes: k and v scales
+  static constexpr int BLOCKS = (CHUNK / kMinBlockSize + 2) * 4;
+  static constexpr size_t BYTES = (size_t)CODES + TILES + SCALES + BLOCKS;
+  static_assert(kAttnWarps * 16 * D * 4 <= TILES, "combine buffer");
+};
+
 template <int D, int CHUNK>
 __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnParams p) {
+  using SM = AttnSmem<D, CHUNK>;
   constexpr int KS = D / 16;        // 16-wide K steps of S = Q K^T
   constexpr int NT = D / 8;         // 8-wide column tiles of O
-  constexpr int PITCH = D + 8;      // f16 per shared row (conflict-free ldmatrix)
-  constexpr int CB = D / 2;         // code bytes a lane loads per tile row (two lanes per position)
-  // K and V tiles of every warp; reused as the combine buffer at the end
-  constexpr int TILE_BYTES = kAttnWarps * 2 * 16 * PITCH * 2;
-  constexpr int ACC_BYTES = kAttnWarps * 16 * D * 4;
-  static_assert(ACC_BYTES <= TILE_BYTES, "combine buffer");
-  __shared__ __align__(16) uint8_t smem[TILE_BYTES];
+  constexpr int PITCH = SM::PITCH;
+  constexpr int CB = D / 2;         // code bytes a lane moves per tile row (two lanes per position)
+  extern __shared__ __align__(16) uint8_t dsmem[];
+  uint8_t *s_codes = dsmem;
+  uint8_t *s_tiles = dsmem + SM::CODES;
+  float *s_scl = reinterpret_cast<float *>(dsmem + SM::CODES + SM::TILES);
+  int *s_blk = reinterpret_cast<int *>(dsmem + SM::CODES + SM::TILES + SM::SCALES);
   __shared__ float s_ml[kAttnWarps][16][2];
-  __shared__ float s_sc[kAttnWarps][16][2];   // per position: k scale * softmax scale, v scale / vs_ref
-  __shared__ uint32_t s_valid[kAttnWarps];     // per warp: bit i set if tile position i is read
-  __shared__ float s_red[kAttnWarps];
+  __shared__ float s_unit[kAttnWarps];
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int L = __ldg(p.context_lens + b);
   const int c0 = split * CHUNK;
   const int c1 = min(c0 + CHUNK, L);
-  __half *sK = reinterpret_cast<__half *>(smem) + warp * 2 * 16 * PITCH;
-  __half *sV = sK + 16 * PITCH;
 
-  // largest value scale of the chunk (every scale is positive)
-  float vmax = 0.0f;
-  for (int pos = c0 + threadIdx.x; pos < c1; pos += kAttnThreads) {
-    const int64_t slot = kv_slot(p, b, pos);
-    if (slot >= 0) vmax = fmaxf(vmax, __ldg(p.vs + slot * p.Hkv + g));
+  // the chunk's block-table entries (-1 where there is none)
+  const int bi0 = c0 / p.block_size;
+  const int nbi = c1 > c0 ? (c1 - 1) / p.block_size - bi0 + 1 : 0;
+  for (int i = threadIdx.x; i < nbi; i += kAttnThreads) {
+    const int bi = bi0 + i;
+    s_blk[i] = bi < p.max_blocks ? __ldg(p.block_tables + (int64_t)b * p.max_blocks + bi) : -1;
   }
-  #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-  if (lane == 0) s_red[warp] = vmax;
   __syncthreads();
-  float vs_ref = s_red[0];
-  #pragma unroll
-  for (int w = 1; w < kAttnWarps; ++w) vs_ref = fmaxf(vs_ref, s_red[w]);
-  const float inv_ref = vs_ref > 0.0f ? 1.0f / vs_ref : 0.0f;
+  auto slot_of = [&](int pos) -> int64_t {
+    if (pos >= c1) return -1;
+    const int blk = s_blk[pos / p.block_size - bi0];
+    const int64_t slot = (int64_t)blk * p.block_size + pos % p.block_size;
+    return (blk < 0 || slot >= p.num_slots) ? -1 : slot;
+  };
+
+  __half *sK = reinterpret_cast<__half *>(s_tiles) + warp * 2 * 16 * PITCH;
+  __half *sV = sK + 16 * PITCH;
+  uint8_t *wcodes = s_codes + warp * 2 * SM::CODE_STAGE;
+  float *wscl = s_scl + warp * 2 * 2 * 16;
+
+  // issue the copies of the tile at `base` into code stage `st`
+  auto prefetch = [&](int base, int st) {
+    const int kk = lane >> 1, half = lane & 1;
+    const int64_t slot = slot_of(base + kk);
+    const bool valid = slot >= 0;
+    const int64_t off = (valid ? slot * p.Hkv + g : 0) * D + half * CB;
+    uint8_t *dk = wcodes + st * SM::CODE_STAGE + kk * D + half * CB;
+    uint8_t *dv = dk + 16 * D;
+    #pragma unroll
+    for (int i = 0; i < CB / 16; ++i) {
+      cp_async16(dk + 16 * i, p.kc + off + 16 * i, valid);
+      cp_async16(dv + 16 * i, p.vc + off + 16 * i, valid);
+    }
+    if (half == 0) {
+      const int64_t si = valid ? slot * p.Hkv + g : 0;
+      cp_async4(wscl + (st * 2 + 0) * 16 + kk, p.ks + si, valid);
+      cp_async4(wscl + (st * 2 + 1) * 16 + kk, p.vs + si, valid);
+    }
+  };
 
   // query fragments (A operand; rows = the group's heads, padded to 16)
   const int r0 = lane >> 2, cq = (lane & 3) * 2;
@@ -167,42 +223,44 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnPar
     }
   }
 
-  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.0f, 0.0f};
+  // the accumulator is kept in units of `unit` (a value scale): O = acc * unit
+  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.0f, 0.0f}, unit = 1.0f;
   float acc[NT][4];
   #pragma unroll
   for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
 
-  for (int base = c0 + warp * 16; base < c1; base += kAttnWarps * 16) {
-    // gather this tile's codes: position base + lane / 2, half (lane & 1) of its D bytes
+  int st = 0;
+  int base = c0 + warp * 16;
+  if (base < c1) prefetch(base, 0);
+  cp_async_commit();
+  for (; base < c1; base += kAttnWarps * 16, st ^= 1) {
+    const int next = base + kAttnWarps * 16;
+    if (next < c1) prefetch(next, st ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();     // this tile's copies have landed (the next tile's may not)
+    __syncwarp();
+    // decode this lane's codes to f16
     {
       const int kk = lane >> 1, half = lane & 1;
-      const int pos = base + kk;
-      int64_t slot = pos < c1 ? kv_slot(p, b, pos) : -1;
-      const bool valid = slot >= 0;
-      if (!valid) slot = 0;
-      const int64_t off = (slot * p.Hkv + g) * D + half * CB;
-      uint4 kc[CB / 16], vc[CB / 16];
+      const uint8_t *ck = wcodes + st * SM::CODE_STAGE + kk * D + half * CB;
       #pragma unroll
       for (int i = 0; i < CB / 16; ++i) {
-        kc[i] = valid ? __ldcs(reinterpret_cast<const uint4 *>(p.kc + off) + i) : make_uint4(0u, 0u, 0u, 0u);
-        vc[i] = valid ? __ldcs(reinterpret_cast<const uint4 *>(p.vc + off) + i) : make_uint4(0u, 0u, 0u, 0u);
+        decode16(*reinterpret_cast<const uint4 *>(ck + 16 * i), sK + kk * PITCH + half * CB + i * 16);
+        decode16(*reinterpret_cast<const uint4 *>(ck + 16 * D + 16 * i), sV + kk * PITCH + half * CB + i * 16);
       }
-      if (half == 0) {
-        s_sc[warp][kk][0] = valid ? __ldg(p.ks + slot * p.Hkv + g) * p.scale_log2 : 0.0f;
-        s_sc[warp][kk][1] = valid ? __ldg(p.vs + slot * p.Hkv + g) * inv_ref : 0.0f;
-      }
-      const uint32_t vb = __ballot_sync(0xffffffffu, valid && half == 0);   // bit 2 kk: position kk
-      if (lane == 0) {
-        uint32_t bits = 0;
-        #pragma unroll
-        for (int i = 0; i < 16; ++i) bits |= ((vb >> (2 * i)) & 1u) << i;
-        s_valid[warp] = bits;
-      }
+    }
+    const float *ksc = wscl + (st * 2 + 0) * 16;
+    const float *vsc = wscl + (st * 2 + 1) * 16;
+    // the tile's readable positions and its largest value scale
+    uint32_t vbits = 0;
+    float vmax = 0.0f;
+    {
+      const int pos = base + (lane & 15);
+      const bool valid = slot_of(pos) >= 0;
+      vbits = __ballot_sync(0xffffffffu, valid && lane < 16);
+      vmax = valid ? vsc[lane & 15] : 0.0f;
       #pragma unroll
-      for (int i = 0; i < CB / 16; ++i) {
-        decode16(kc[i], sK + kk * PITCH + half * CB + i * 16);
-        decode16(vc[i], sV + kk * PITCH + half * CB + i * 16);
-      }
+      for (int o = 8; o >= 1; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
     }
     __syncwarp();
 
@@ -220,7 +278,6 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnPar
       }
     }
     // key scales, masking, online softmax (rows r0 and r0 + 8)
-    const uint32_t vbits = s_valid[warp];
     float mx[2] = {-INFINITY, -INFINITY};
     #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -228,13 +285,14 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnPar
       for (int e = 0; e < 2; ++e) {
         const int kp = j * 8 + cq + e;
         const bool valid = (vbits >> kp) & 1u;
-        const float ksc = s_sc[warp][kp][0];
-        s[j][e] = valid ? s[j][e] * ksc : -INFINITY;
-        s[j][2 + e] = valid ? s[j][2 + e] * ksc : -INFINITY;
+        const float k2 = ksc[kp] * p.scale_log2;
+        s[j][e] = valid ? s[j][e] * k2 : -INFINITY;
+        s[j][2 + e] = valid ? s[j][2 + e] * k2 : -INFINITY;
         mx[0] = fmaxf(mx[0], s[j][e]);
         mx[1] = fmaxf(mx[1], s[j][2 + e]);
       }
     }
+    const float inv_vmax = vmax > 0.0f ? 1.0f / vmax : 0.0f;
     float alpha[2], psum[2] = {0.0f, 0.0f};
     #pragma unroll
     for (int r = 0; r < 2; ++r) {
@@ -251,22 +309,26 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnPar
       float pv[4];
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const float vsc = s_sc[warp][j * 8 + cq + e][1];
+        const float vr = vsc[j * 8 + cq + e] * inv_vmax;   // this position's value scale / the tile's largest
         const float p0 = m_r[0] == -INFINITY ? 0.0f : exp2f(s[j][e] - m_r[0]);
         const float p1 = m_r[1] == -INFINITY ? 0.0f : exp2f(s[j][2 + e] - m_r[1]);
         psum[0] += p0;
         psum[1] += p1;
-        pv[e] = p0 * vsc;
-        pv[2 + e] = p1 * vsc;
+        pv[e] = p0 * vr;
+        pv[2 + e] = p1 * vr;
       }
       pa[2 * j] = h2_bits(__floats2half2_rn(pv[0], pv[1]));       // row r0, positions j*8 + cq, +1
       pa[2 * j + 1] = h2_bits(__floats2half2_rn(pv[2], pv[3]));   // row r0 + 8
     }
+    // move the accumulator to this tile's units (vmax), with the softmax factor
+    const float to_tile = vmax > 0.0f ? unit * inv_vmax : 1.0f;
+    if (vmax > 0.0f) unit = vmax;
     #pragma unroll
     for (int r = 0; r < 2; ++r) {
       psum[r] += __shfl_xor_sync(0xffffffffu, psum[r], 1);
       psum[r] += __shfl_xor_sync(0xffffffffu, psum[r], 2);
       l_r[r] = l_r[r] * alpha[r] + psum[r];
+      alpha[r] *= to_tile;
     }
     #pragma unroll
     for (int n = 0; n < NT; ++n) {
@@ -286,24 +348,26 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnPar
     }
     __syncwarp();  // the next tile overwrites this warp's tiles
   }
+  cp_async_wait<0>();
 
-  // combine the four warps' states
+  // combine the four warps' states (each accumulator times its unit)
   if ((lane & 3) == 0) {
     s_ml[warp][r0][0] = m_r[0];
     s_ml[warp][r0][1] = l_r[0];
     s_ml[warp][r0 + 8][0] = m_r[1];
     s_ml[warp][r0 + 8][1] = l_r[1];
   }
+  if (lane == 0) s_unit[warp] = unit;
   __syncthreads();  // every warp has finished with its tiles: the buffer is free
-  float *s_acc = reinterpret_cast<float *>(smem);   // [warp][16][D]
+  float *s_acc = reinterpret_cast<float *>(s_tiles);   // [warp][16][D]
   #pragma unroll
   for (int n = 0; n < NT; ++n) {
     float *row0 = s_acc + ((size_t)warp * 16 + r0) * D + n * 8 + cq;
     float *row1 = s_acc + ((size_t)warp * 16 + r0 + 8) * D + n * 8 + cq;
-    row0[0] = acc[n][0];
-    row0[1] = acc[n][1];
-    row1[0] = acc[n][2];
-    row1[1] = acc[n][3];
+    row0[0] = acc[n][0] * unit;
+    row0[1] = acc[n][1] * unit;
+    row1[0] = acc[n][2] * unit;
+    row1[1] = acc[n][3] * unit;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < p.G * D; i += kAttnThreads) {
@@ -321,7 +385,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnPar
       }
     }
     const int64_t idx = (((int64_t)b * p.Hq + (int64_t)g * p.G + h) * p.splits + split);
-    p.part_acc[idx * D + d] = o * vs_ref;
+    p.part_acc[idx * D + d] = o;
     if (d == 0) {
       p.part_ml[idx * 2] = m;
       p.part_ml[idx * 2 + 1] = l;
@@ -354,7 +418,17 @@ constexpr int kAttnChunk = 512;
 
 template <int D>
 cudaError_t launch_attn(const AttnParams &p, int B, __nv_bfloat16 *out, cudaStream_t st) {
-  decode_attn_kernel<D, kAttnChunk><<<dim3(p.splits, p.Hkv, B), kAttnThreads, 0, st>>>(p);
+  const size_t smem = AttnSmem<D, kAttnChunk>::BYTES;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t a = cudaFuncSetAttribute(decode_attn_kernel<D, kAttnChunk>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (a != cudaSuccess) return a;
+    attr_set[dev] = true;
+  }
+  decode_attn_kernel<D, kAttnChunk><<<dim3(p.splits, p.Hkv, B), kAttnThreads, smem, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};

@@ -613,47 +613,83 @@ __device__ __forceinline__ void dump_partial(uint32_t tbase, float *row_dst, int
 
 // Reducer `ridx` (0 .. 2 * split - 1) of tail tile j at tile position (m, n):
 // groups of 8 output columns, [ridx * G / (2 S), (ridx + 1) * G / (2 S)).
+// A thread takes U groups at a time and loads four splits of all of them
+// before adding (8 U independent 16-byte loads in flight: the partials come
+// from L2, and a load-add chain per split would leave the reduction waiting on
+// latency); the additions stay in split order 0, 1, 2, ...
 template <int BN_T>
 __device__ __forceinline__ void reduce_tail_tile(const GemmParams &p, int j, int m, int n, int ridx, int etid) {
+  constexpr int U = 2;
+  constexpr int SU = 4;
   const int S = p.tail_split;
   constexpr int G8 = BN_T / 8;
   constexpr int G = 2 * BM * G8;
   const int g0 = (int)((long long)ridx * G / (2 * S));
   const int g1 = (int)((long long)(ridx + 1) * G / (2 * S));
   const float *base = p.partials + (size_t)j * S * (2 * BM) * BN_T;
-  for (int g = g0 + etid; g < g1; g += 32 * kEpiWarps) {
-    const int row = g / G8;
-    const int c8 = (g - row * G8) * 8;
-    const int t = m * (2 * BM) + row;
-    const int col = n * BN_T + c8;
-    if (t >= p.T || col >= p.Co) continue;  // Co % 16 == 0: the 8 columns are valid together
-    float a[8];
+  const size_t split_stride = (size_t)(2 * BM) * BN_T;
+  for (int gb = g0 + etid; gb < g1; gb += U * 32 * kEpiWarps) {
+    float a[U][8];
+    size_t off[U];
+    bool live[U];
     #pragma unroll
-    for (int i = 0; i < 8; ++i) a[i] = 0.0f;
-    for (int sp = 0; sp < S; ++sp) {
-      const float4 *src = reinterpret_cast<const float4 *>(base + ((size_t)sp * (2 * BM) + row) * BN_T + c8);
-      const float4 v0 = __ldcg(src), v1 = __ldcg(src + 1);
-      if (sp == 0) {
-        a[0] = v0.x; a[1] = v0.y; a[2] = v0.z; a[3] = v0.w;
-        a[4] = v1.x; a[5] = v1.y; a[6] = v1.z; a[7] = v1.w;
-      } else {
-        a[0] = __fadd_rn(a[0], v0.x); a[1] = __fadd_rn(a[1], v0.y);
-        a[2] = __fadd_rn(a[2], v0.z); a[3] = __fadd_rn(a[3], v0.w);
-        a[4] = __fadd_rn(a[4], v1.x); a[5] = __fadd_rn(a[5], v1.y);
-        a[6] = __fadd_rn(a[6], v1.z); a[7] = __fadd_rn(a[7], v1.w);
+    for (int u = 0; u < U; ++u) {
+      const int g = gb + u * 32 * kEpiWarps;
+      live[u] = g < g1;
+      const int row = live[u] ? g / G8 : 0;
+      const int c8 = live[u] ? (g - row * G8) * 8 : 0;
+      off[u] = (size_t)row * BN_T + c8;
+      #pragma unroll
+      for (int i = 0; i < 8; ++i) a[u][i] = 0.0f;
+    }
+    for (int sp0 = 0; sp0 < S; sp0 += SU) {
+      float4 v[SU][U][2];
+      #pragma unroll
+      for (int k = 0; k < SU; ++k) {
+        #pragma unroll
+        for (int u = 0; u < U; ++u) {
+          if (sp0 + k < S && live[u]) {
+            const float4 *src = reinterpret_cast<const float4 *>(base + (size_t)(sp0 + k) * split_stride + off[u]);
+            v[k][u][0] = __ldcg(src);
+            v[k][u][1] = __ldcg(src + 1);
+          } else {
+            v[k][u][0] = v[k][u][1] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          }
+        }
+      }
+      #pragma unroll
+      for (int k = 0; k < SU; ++k) {
+        if (sp0 + k >= S) break;
+        #pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const float w[8] = {v[k][u][0].x, v[k][u][0].y, v[k][u][0].z, v[k][u][0].w,
+                              v[k][u][1].x, v[k][u][1].y, v[k][u][1].z, v[k][u][1].w};
+          #pragma unroll
+          for (int i = 0; i < 8; ++i) a[u][i] = (sp0 + k == 0) ? w[i] : __fadd_rn(a[u][i], w[i]);
+        }
       }
     }
-    const float xs = __ldg(p.xs + t);
-    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.ws + col));
-    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.ws + col + 4));
-    const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    uint32_t o[4];
     #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      o[i] = pack_bf16x2(__fmul_rn(__fmul_rn(a[2 * i], xs), w[2 * i]),
-                         __fmul_rn(__fmul_rn(a[2 * i + 1], xs), w[2 * i + 1]));
-    *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + (size_t)t * p.Co + col) =
-        make_uint4(o[0], o[1], o[2], o[3]);
+    for (int u = 0; u < U; ++u) {
+      if (!live[u]) continue;
+      const int g = gb + u * 32 * kEpiWarps;
+      const int row = g / G8;
+      const int c8 = (g - row * G8) * 8;
+      const int t = m * (2 * BM) + row;
+      const int col = n * BN_T + c8;
+      if (t >= p.T || col >= p.Co) continue;  // Co % 16 == 0: the 8 columns are valid together
+      const float xs = __ldg(p.xs + t);
+      const float4 w0 = __ldg(reinterpret_cast<const float4 *>(p.ws + col));
+      const float4 w1 = __ldg(reinterpret_cast<const float4 *>(p.ws + col + 4));
+      const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      uint32_t o[4];
+      #pragma unroll
+      for (int i = 0; i < 4; ++i)
+        o[i] = pack_bf16x2(__fmul_rn(__fmul_rn(a[u][2 * i], xs), w[2 * i]),
+                           __fmul_rn(__fmul_rn(a[u][2 * i + 1], xs), w[2 * i + 1]));
+      *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + (size_t)t * p.Co + col) =
+          make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 

@@ -309,8 +309,8 @@ PTPC_API int ptpc_static_scratch_status(void *stream);
 /* Appends T tokens: K_dev, V_dev bf16 [T, H, D]; slots_dev int64 [T] (a
  * negative slot skips the token, as does a slot >= num_blocks * block_size);
  * k_cache / v_cache u8 [num_blocks * block_size, H, D]; k_scale / v_scale
- * fp32 [num_blocks * block_size, H].  D is 64 or 128.  Tokens with equal
- * slots race. */
+ * fp32 [num_blocks * block_size, H].  D is 64 or 128; block_size >= 8.
+ * Tokens with equal slots race. */
 PTPC_API int ptpc_kv_cache_append(const void *K_dev, const void *V_dev, const int64_t *slots_dev, int64_t T,
                                   int64_t H, int64_t D, int64_t block_size, int64_t num_blocks,
                                   uint8_t *k_cache_dev, uint8_t *v_cache_dev, float *k_scale_dev,
