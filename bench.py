@@ -75,6 +75,10 @@ def parse():
     ap.add_argument("--no-kv", action="store_true", help="skip the FP8 KV-cache decode-attention record")
     ap.add_argument("--decode-tokens", default="1,8,32,128",
                     help="T values of the decode record inside the default line ('' to skip)")
+    ap.add_argument("--weight-formats", default="e3m2,e2m1",
+                    help="sub-byte weight formats of the decode_subbyte record")
+    ap.add_argument("--record", default=None, choices=["decode", "decode_subbyte", "kv_decode"],
+                    help="print only this sub-record of the default line (a short run for profiling)")
     return ap.parse_args()
 
 
@@ -625,26 +629,38 @@ def run_gpu(args):
         return e0.elapsed_time(e1)
 
     K, W = args.steps, max(3, args.warmup)
+    # ---- the activation quantiser alone on the step's inputs, measured
+    # before any GEMM has run (a kernel timed alone: burst conditions; every
+    # input is larger than L2, so each pass reads X from HBM)
+    bufs = [(torch.empty((d["T"], d["Ci"]), dtype=torch.uint8, device=dev),
+             torch.empty((d["T"],), dtype=torch.float32, device=dev)) for d in L]
+    q_bytes = sum(quant_bytes(d["T"], d["Ci"]) for d in L)
+    Kq = max(10, min(4 * K, 200))
+    qfn = lambda: [ptpc.quantize_activations(d["X"], *bufs[j]) for j, d in enumerate(L)]
+    for _ in range(3):
+        qfn()
+    ms_q = max_over_ranks(timed(qfn, Kq)) / Kq
+    qprobe = ptpc.ClockProbe(dev)
+    timed(qfn, Kq, before=lambda: qprobe.start(ms_q * Kq * 1.05 / 1e3))
+    q_alone = q_bytes / (ms_q / 1e3) / 1e9
+    quant_isolated = {
+        "value": q_alone, "unit": "GB/s", "achieved": q_alone, "peak": peaks["hbm_gbs"],
+        "frac": q_alone / peaks["hbm_gbs"], "bytes_per_pass": q_bytes, "ms_per_pass": ms_q, "passes": Kq,
+        "inputs": [[d["T"], d["Ci"]] for d in L], "sm_mhz_device": qprobe.mhz(),
+        "peak_src": f"{peaks['src']} HBM copy",
+        "note": "ptpc_quantize_activations alone, every layer input of the step in turn, back to back, "
+                "before the GEMM loops; algorithmic bytes 3 per element + 4 per row",
+    }
+
     for _ in range(W):
         step()
     with ClockSampler(local) as clk:
         ms = timed(step, K)
-    # The SM clock seen by the device over the same loop, repeated right
-    # after: the clock probe runs beside it on a side stream (kept out of the
-    # timed region above, which it could perturb).
-    probe = ptpc.ClockProbe(dev)
-    ms_probe = timed(step, K, before=lambda: probe.start(ms * 1.05 / 1e3))
-    probe_mhz = probe.mhz()
-    ms = max_over_ranks(ms)
-    flops = layer_flops(layers)
-    value = whole_job_tflops(flops, world, K, ms)
-    launches = K * 2 * len(L)
-
-    # ---- per-kernel device times: events on the launch stream around each
-    # launch, no host synchronisation inside the loop
+    # ---- per-kernel device times, right after the timed loop: the same
+    # launches as ptpc_linear (quantiser, then GEMM) through the two separate
+    # entry points, with events on the launch stream around each launch and no
+    # host synchronisation inside the loop
     Kk = max(10, min(K, 200))
-    bufs = [(torch.empty((d["T"], d["Ci"]), dtype=torch.uint8, device=dev),
-             torch.empty((d["T"],), dtype=torch.float32, device=dev)) for d in L]
     for _ in range(3):
         for j, d in enumerate(L):
             ptpc.quantize_activations(d["X"], *bufs[j])
@@ -662,13 +678,27 @@ def run_gpu(args):
     barrier()
     q_ms = [sum(evs[it][j][0].elapsed_time(evs[it][j][1]) for it in range(Kk)) / Kk for j in range(len(L))]
     g_ms = [sum(evs[it][j][1].elapsed_time(evs[it][j][2]) for it in range(Kk)) / Kk for j in range(len(L))]
-    gemm_time = sum(g_ms)
-    gemm_tflops = flops / (gemm_time / 1e3) / 1e12
+    # The SM clock seen by the device over the same loop, repeated: the clock
+    # probe runs beside it on a side stream (kept out of the timed region
+    # above, which it could perturb).
+    probe = ptpc.ClockProbe(dev)
+    ms_probe = timed(step, K, before=lambda: probe.start(ms * 1.05 / 1e3))
+    probe_mhz = probe.mhz()
+    ms = max_over_ranks(ms)
+    flops = layer_flops(layers)
+    value = whole_job_tflops(flops, world, K, ms)
+    launches = K * 2 * len(L)
+
+    # The GEMM's time inside the timed steps: the step's device time less its
+    # quantiser launches (launch gaps stay charged to the GEMM, so this is an
+    # upper bound on its launch durations and `achieved` a lower bound).
+    gemm_step_ms = ms / K - sum(q_ms)
+    gemm_tflops = flops / (gemm_step_ms / 1e3) / 1e12
     g_bytes = sum(gemm_bytes(d["T"], d["Ci"], d["Co"]) for d in L)
-    gemm_gbs = g_bytes / (gemm_time / 1e3) / 1e9
+    gemm_gbs = g_bytes / (gemm_step_ms / 1e3) / 1e9
+    loop_tflops = flops / (sum(g_ms) / 1e3) / 1e12
     ridge = fp8_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)      # FLOP per byte
     hbm_bound = flops / g_bytes < ridge
-    q_bytes = sum(quant_bytes(d["T"], d["Ci"]) for d in L)
     q_gbs = q_bytes / (sum(q_ms) / 1e3) / 1e9
     dram = traffic_record(kernel_src_hash(), f"{args.workload}:T={T}")
 
@@ -698,10 +728,17 @@ def run_gpu(args):
             "kernel": "ptpc scaled GEMM (fused epilogue), all layers of one step",
             "traffic_unit": "bytes per step (dram__bytes_read.sum + dram__bytes_write.sum over the step's GEMM launches)",
             "algorithmic_flops_per_step": flops, "algorithmic_bytes_per_step": g_bytes,
-            "gemm_tflops": gemm_tflops, "gemm_gbs": gemm_gbs,
-            "per_layer_ms": {d["name"]: g for d, g in zip(L, g_ms)},
+            "gemm_tflops": gemm_tflops, "gemm_gbs": gemm_gbs, "gemm_ms_per_step": gemm_step_ms,
+            "achieved_src": "algorithmic FLOPs / (timed step device time - its quantiser launches, "
+                            "the latter timed by events in a loop of the same launches right after)",
+            "per_launch_loop": {
+                "tflops": loop_tflops, "ms_per_step": sum(g_ms),
+                "per_layer_ms": {d["name"]: g for d, g in zip(L, g_ms)},
+                "note": "events around each GEMM launch in that loop; it runs later than the timed "
+                        "steps, so at the lower clock that the power cap has reached by then"},
             "sm_mhz_device": probe_mhz,
         },
+        "quant_isolated": quant_isolated,
         "quant": {
             "value": q_gbs, "unit": "GB/s", "peak": peaks["hbm_gbs"], "frac": q_gbs / peaks["hbm_gbs"],
             "bytes_per_step": q_bytes, "per_layer_ms": {d["name"]: q for d, q in zip(L, q_ms)},
@@ -709,25 +746,6 @@ def run_gpu(args):
             "note": "inside the step: each launch timed by events between the GEMMs (launch gap included), "
                     "at the clock the GEMMs' power draw leaves",
         },
-    }
-
-    # ---- the activation quantiser alone on the same inputs (no GEMM in
-    # between; every input is larger than L2, so each pass reads X from HBM)
-    Kq = max(10, min(4 * K, 200))
-    qfn = lambda: [ptpc.quantize_activations(d["X"], *bufs[j]) for j, d in enumerate(L)]
-    for _ in range(3):
-        qfn()
-    ms_q = max_over_ranks(timed(qfn, Kq)) / Kq
-    qprobe = ptpc.ClockProbe(dev)
-    timed(qfn, Kq, before=lambda: qprobe.start(ms_q * Kq * 1.05 / 1e3))
-    q_alone = q_bytes / (ms_q / 1e3) / 1e9
-    line["quant_isolated"] = {
-        "value": q_alone, "unit": "GB/s", "achieved": q_alone, "peak": peaks["hbm_gbs"],
-        "frac": q_alone / peaks["hbm_gbs"], "bytes_per_pass": q_bytes, "ms_per_pass": ms_q, "passes": Kq,
-        "inputs": [[d["T"], d["Ci"]] for d in L], "sm_mhz_device": qprobe.mhz(),
-        "peak_src": f"{peaks['src']} HBM copy",
-        "note": "ptpc_quantize_activations alone, every layer input of the step in turn, back to back; "
-                "algorithmic bytes 3 per element + 4 per row",
     }
 
     # ---- per-output-channel weight quantiser (run once per weight at load time)
@@ -1134,6 +1152,29 @@ def run_tp(args):
     return 0
 
 
+def run_record(args):
+    """One sub-record of the default line on its own (1 GPU), printed as one
+    JSON line: a short command to profile the decode GEMMs or the decode
+    attention with."""
+    import torch
+
+    import fp8_quantized_gemm_ptpc_b200 as ptpc
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    steps = max(3, args.steps)
+    tokens = [int(t) for t in args.decode_tokens.split(",") if t.strip()]
+    if args.record == "decode":
+        rec = decode_record(ptpc, dev, peaks, tokens, steps=steps)
+    elif args.record == "decode_subbyte":
+        rec = decode_subbyte_record(ptpc, dev, peaks, tokens, steps=steps,
+                                    fmts=tuple(f for f in args.weight_formats.split(",") if f))
+    else:
+        rec = kv_decode_record(ptpc, dev, peaks, steps=steps)
+    print(json.dumps({"record": args.record} | rec), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -1144,6 +1185,8 @@ def main():
         return run_sweep(args)
     if args.tp:
         return run_tp(args)
+    if args.record:
+        return run_record(args)
     return run_gpu(args)
 
 
