@@ -58,6 +58,7 @@ SIGNATURES = {
     "ptpc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ptpc_gemm_ksplit": (ctypes.c_int, [_I64, _I64, _I64]),
     "ptpc_gemm_tail_split": (ctypes.c_int, [_I64, _I64, _I64, _SZ]),
+    "ptpc_gemm_swap_tokens": (ctypes.c_int, [_I64, _I64, _I64, _SZ]),
     "ptpc_selftest_wait_timeout": (ctypes.c_int, [_P, _P]),
     "ptpc_scaled_mm_static_scratch": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "ptpc_static_scratch_status": (ctypes.c_int, [_P]),
@@ -128,6 +129,15 @@ def gemm_tail_split(T: int, Ci: int, Co: int, ws_bytes: int | None = None) -> in
     if ws_bytes is None:
         ws_bytes = workspace_size(OP_SCALED_MM, T, Ci, Co)
     return int(lib.ptpc_gemm_tail_split(T, Ci, Co, ws_bytes))
+
+
+def gemm_swap_tokens(T: int, Ci: int, Co: int, ws_bytes: int | None = None) -> int:
+    """Tokens a tile holds when the prefill GEMM's plan for this shape swaps
+    its operands (weights as the 256-row operand), 0 otherwise; ws_bytes of
+    GEMM workspace (default: what ptpc_workspace_size asks for)."""
+    if ws_bytes is None:
+        ws_bytes = workspace_size(OP_SCALED_MM, T, Ci, Co)
+    return int(lib.ptpc_gemm_swap_tokens(T, Ci, Co, ws_bytes))
 
 
 def _check(fn: str, status: int):

@@ -299,6 +299,12 @@ int ptpc_gemm_tail_split(int64_t T, int64_t Ci, int64_t Co, size_t ws_bytes) {
   return ptpc::gemm_tail_split((int)T, (int)Ci, (int)Co, ws_bytes);
 }
 
+int ptpc_gemm_swap_tokens(int64_t T, int64_t Ci, int64_t Co, size_t ws_bytes) {
+  if (check_shape_tci(T, Ci) != PTPC_OK || check_co(Co) != PTPC_OK || T == 0) return 0;
+  if (check_device() != PTPC_OK) return 0;
+  return ptpc::gemm_swap_tokens((int)T, (int)Ci, (int)Co, ws_bytes);
+}
+
 // ------------------------------------------------------------------ FP8 KV cache
 
 namespace {

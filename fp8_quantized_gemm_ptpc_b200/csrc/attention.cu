@@ -11,22 +11,28 @@
 //   s_l = softmax_scale * k_scale[l] * sum_d q[h, d] * dec(K[l, d]),
 //   out[h, d] = sum_l softmax(s)_l * v_scale[l] * dec(V[l, d]).
 //
-// Decode is bound by the bytes of the cache it streams (one byte per code).
-// A CTA takes one (sequence, KV head) and a chunk of 512 context positions,
-// whose block-table entries it first reads into shared memory; its four warps
-// take 16-position tiles in turn.  A warp gathers a tile's K and V codes and
-// scales with asynchronous copies (cp.async, 16 bytes per copy, zero-filled
-// for positions that are not read) into one of two shared-memory stages, so
-// the next tile's bytes are in flight while it decodes this one exactly to
-// f16 (cvt e4m3x2 -> f16x2; every E4M3 value is an f16 value) and runs
-// FlashAttention-style tensor-core MMAs (mma.sync m16n8k16, f16 inputs, fp32
-// accumulation) with the GQA group's query heads as the 16 rows: S = Q K^T,
-// an online softmax in base 2, O += P V.  The key scales multiply the scores;
-// the value scales enter P relative to the tile's largest one (so P stays in
-// [0, 1] in f16), and the accumulator is kept in units of that value scale
-// (moved between tiles with the softmax's own rescale).  The warps' states
-// are combined in shared memory and every CTA writes (max, sum, accumulator)
-// for its chunk; a second kernel combines the chunks and rounds to bf16.
+// Decode is bound by the bytes of the cache it streams (one byte per code),
+// so the kernel spends as few instructions per code byte as it can.  A CTA
+// takes one (sequence, KV head) and a chunk of 512 context positions, whose
+// block-table entries it first reads into shared memory; its four warps take
+// 16-position tiles in turn.  A warp gathers a tile's K and V codes and scales
+// with asynchronous copies (cp.async, 16 bytes per copy, zero-filled for
+// positions that are not read) into a ring of three shared-memory stages, so
+// two tiles' bytes are in flight while it computes on a third.  The codes go
+// from shared memory straight into the registers of FlashAttention-style
+// tensor-core MMAs (mma.sync m16n8k16, f16 inputs, fp32 accumulation; the
+// GQA group's query heads are the 16 rows), converted exactly to f16 on the
+// way (cvt e4m3x2 -> f16x2: every E4M3 value is an f16 value).  To make that
+// possible the contraction over d in S = Q K^T runs in a permuted order (the
+// same for Q and K) in which each lane's codes of a position are contiguous,
+// and O's columns are ordered so that each lane's V codes of a position are
+// contiguous too; the two positions a V register pairs are joined by one byte
+// permute.  Online softmax in base 2; the key scales multiply the scores; the
+// value scales enter P relative to the largest value scale seen so far (so P
+// stays in [0, 1] in f16), and the accumulator is kept in units of it.  The
+// warps' states are combined in shared memory and every CTA writes (max, sum,
+// accumulator) for its chunk; a second kernel combines the chunks and rounds
+// to bf16.
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -69,31 +75,6 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   return (uint32_t)r.x | ((uint32_t)r.y << 16);
 }
 
-// 16 codes -> 16 f16 at dst (32 bytes, 16-byte aligned).
-__device__ __forceinline__ void decode16(uint4 c, __half *dst) {
-  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-  uint32_t o[8];
-  #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    o[2 * i] = e4m3x2_to_f16x2(w[i] & 0xFFFFu);
-    o[2 * i + 1] = e4m3x2_to_f16x2(w[i] >> 16);
-  }
-  reinterpret_cast<uint4 *>(dst)[0] = make_uint4(o[0], o[1], o[2], o[3]);
-  reinterpret_cast<uint4 *>(dst)[1] = make_uint4(o[4], o[5], o[6], o[7]);
-}
-
-__device__ __forceinline__ void ldsm_x2(uint32_t &r0, uint32_t &r1, const void *p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
-               : "=r"(r0), "=r"(r1)
-               : "r"((uint32_t)__cvta_generic_to_shared(p)));
-}
-
-__device__ __forceinline__ void ldsm_x2_trans(uint32_t &r0, uint32_t &r1, const void *p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
-               : "=r"(r0), "=r"(r1)
-               : "r"((uint32_t)__cvta_generic_to_shared(p)));
-}
-
 // D (16x8 fp32) += A (16x16 f16, row) * B (16x8 f16, col).
 __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -101,17 +82,6 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Cache slot of position pos of sequence b, or -1 where the block table has
-// no entry for it or names a block outside the cache (such positions are
-// masked instead of read).
-__device__ __forceinline__ int64_t kv_slot(const AttnParams &p, int b, int pos) {
-  const int bi = pos / p.block_size;
-  if (bi >= p.max_blocks) return -1;
-  const int blk = __ldg(p.block_tables + (int64_t)b * p.max_blocks + bi);
-  const int64_t slot = (int64_t)blk * p.block_size + pos % p.block_size;
-  return (blk < 0 || slot >= p.num_slots) ? -1 : slot;
 }
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
@@ -129,36 +99,45 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 constexpr int kMinBlockSize = 8;   // the chunk's block-table entries fit in shared memory
+constexpr int kAttnStages = 3;     // code stages a warp keeps in flight (two tiles ahead)
 
-// Shared memory of one CTA: every warp's two code stages (K and V codes and
-// scales of 16 positions) and its decoded f16 K and V tiles, which at the end
-// double as the warps' accumulators; the chunk's block-table entries.
+// Shared memory of one CTA: every warp's ring of code stages (K and V codes of
+// 16 positions, their scales and the tile's validity mask), which at the end
+// doubles as the warps' accumulators, and the chunk's block-table entries.
+// A position's D code bytes are stored as D/16 16-byte chunks, chunk i at
+// chunk index i ^ (position mod D/16), so that the fragment loads below hit
+// distinct shared-memory banks.
 template <int D, int CHUNK>
 struct AttnSmem {
-  static constexpr int PITCH = D + 8;                                   // f16 per decoded row
-  static constexpr int CODE_STAGE = 2 * 16 * D;                         // bytes: K and V codes
-  static constexpr int CODES = kAttnWarps * 2 * CODE_STAGE;
-  static constexpr int TILES = kAttnWarps * 2 * 16 * PITCH * 2;         // bytes: decoded K and V
-  static constexpr int SCALES = kAttnWarps * 2 * 2 * 16 * 4;            // bytes: k and v scales
+  static constexpr int CODES_TILE = 2 * 16 * D;                       // K then V codes
+  static constexpr int STAGE = CODES_TILE + 2 * 16 * 4 + 16;          // + k, v scales + validity mask
+  static constexpr int RING = kAttnStages * STAGE;
+  static constexpr int CODES = kAttnWarps * RING;
   static constexpr int BLOCKS = (CHUNK / kMinBlockSize + 2) * 4;
-  static constexpr size_t BYTES = (size_t)CODES + TILES + SCALES + BLOCKS;
-  static_assert(kAttnWarps * 16 * D * 4 <= TILES, "combine buffer");
+  static constexpr size_t BYTES = (size_t)CODES + BLOCKS;
+  static_assert(kAttnWarps * 16 * D * 4 <= CODES, "combine buffer");
+  static_assert(STAGE % 16 == 0, "stage alignment");
 };
 
+// Byte offset of 16-byte chunk i of tile-local position pos in a code tile.
+template <int D>
+__device__ __forceinline__ int code_off(int pos, int i) {
+  return pos * D + ((i ^ (pos & (D / 16 - 1))) << 4);
+}
+
+__device__ __forceinline__ uint32_t lo16(uint32_t w) { return w & 0xFFFFu; }
+__device__ __forceinline__ uint32_t hi16(uint32_t w) { return w >> 16; }
+
 template <int D, int CHUNK>
-__global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(kAttnThreads, 3) decode_attn_kernel(const AttnParams p) {
   using SM = AttnSmem<D, CHUNK>;
-  constexpr int KS = D / 16;        // 16-wide K steps of S = Q K^T
+  constexpr int KS = D / 16;        // 16-deep K steps of S = Q K^T
   constexpr int NT = D / 8;         // 8-wide column tiles of O
-  constexpr int PITCH = SM::PITCH;
-  constexpr int CB = D / 2;         // code bytes a lane moves per tile row (two lanes per position)
+  constexpr int KB = D / 4;         // K code bytes a lane holds per position (its share of D)
+  constexpr int VB = D / 8;         // V code bytes a lane holds per position
   extern __shared__ __align__(16) uint8_t dsmem[];
-  uint8_t *s_codes = dsmem;
-  uint8_t *s_tiles = dsmem + SM::CODES;
-  float *s_scl = reinterpret_cast<float *>(dsmem + SM::CODES + SM::TILES);
-  int *s_blk = reinterpret_cast<int *>(dsmem + SM::CODES + SM::TILES + SM::SCALES);
+  int *s_blk = reinterpret_cast<int *>(dsmem + SM::CODES);
   __shared__ float s_ml[kAttnWarps][16][2];
-  __shared__ float s_unit[kAttnWarps];
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -174,40 +153,50 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnPar
     s_blk[i] = bi < p.max_blocks ? __ldg(p.block_tables + (int64_t)b * p.max_blocks + bi) : -1;
   }
   __syncthreads();
-  auto slot_of = [&](int pos) -> int64_t {
-    if (pos >= c1) return -1;
-    const int blk = s_blk[pos / p.block_size - bi0];
-    const int64_t slot = (int64_t)blk * p.block_size + pos % p.block_size;
-    return (blk < 0 || slot >= p.num_slots) ? -1 : slot;
-  };
 
-  __half *sK = reinterpret_cast<__half *>(s_tiles) + warp * 2 * 16 * PITCH;
-  __half *sV = sK + 16 * PITCH;
-  uint8_t *wcodes = s_codes + warp * 2 * SM::CODE_STAGE;
-  float *wscl = s_scl + warp * 2 * 2 * 16;
+  uint8_t *ring = dsmem + warp * SM::RING;
 
-  // issue the copies of the tile at `base` into code stage `st`
+  // Copies of the tile at `base` into stage `st`: lane pair (2 kk, 2 kk + 1)
+  // takes position kk, each lane half of its K and V codes; even lanes the
+  // scales; the tile's validity mask by lane 0.  Positions that are not read
+  // (past the context, no block-table entry, block outside the cache) are
+  // zero-filled and masked.
   auto prefetch = [&](int base, int st) {
     const int kk = lane >> 1, half = lane & 1;
-    const int64_t slot = slot_of(base + kk);
+    const int pos = base + kk;
+    int64_t slot = -1;
+    if (pos < c1) {
+      const int blk = s_blk[pos / p.block_size - bi0];
+      slot = (int64_t)blk * p.block_size + pos % p.block_size;
+      if (blk < 0 || slot >= p.num_slots) slot = -1;
+    }
     const bool valid = slot >= 0;
-    const int64_t off = (valid ? slot * p.Hkv + g : 0) * D + half * CB;
-    uint8_t *dk = wcodes + st * SM::CODE_STAGE + kk * D + half * CB;
-    uint8_t *dv = dk + 16 * D;
+    const int64_t row = valid ? slot * p.Hkv + g : 0;
+    uint8_t *sk = ring + st * SM::STAGE;
+    uint8_t *sv = sk + 16 * D;
+    const uint8_t *gk = p.kc + row * D;
+    const uint8_t *gv = p.vc + row * D;
     #pragma unroll
-    for (int i = 0; i < CB / 16; ++i) {
-      cp_async16(dk + 16 * i, p.kc + off + 16 * i, valid);
-      cp_async16(dv + 16 * i, p.vc + off + 16 * i, valid);
+    for (int i = 0; i < D / 32; ++i) {
+      const int ci = half * (D / 32) + i;
+      cp_async16(sk + code_off<D>(kk, ci), gk + 16 * ci, valid);
+      cp_async16(sv + code_off<D>(kk, ci), gv + 16 * ci, valid);
     }
+    float *sc = reinterpret_cast<float *>(sk + SM::CODES_TILE);
     if (half == 0) {
-      const int64_t si = valid ? slot * p.Hkv + g : 0;
-      cp_async4(wscl + (st * 2 + 0) * 16 + kk, p.ks + si, valid);
-      cp_async4(wscl + (st * 2 + 1) * 16 + kk, p.vs + si, valid);
+      cp_async4(sc + kk, p.ks + row, valid);
+      cp_async4(sc + 16 + kk, p.vs + row, valid);
     }
+    const uint32_t m = __ballot_sync(0xffffffffu, valid);   // bit 2 kk (and 2 kk + 1): position kk
+    if (lane == 0) *reinterpret_cast<uint32_t *>(sc + 32) = m;
   };
 
-  // query fragments (A operand; rows = the group's heads, padded to 16)
-  const int r0 = lane >> 2, cq = (lane & 3) * 2;
+  // Query fragments (A operand of S = Q K^T; rows = the group's heads, padded
+  // to 16).  The contraction over d is taken in a permuted order: in K step
+  // s, lane column c (lane & 3) holds d = c*KB + 4s + {0, 1} (logical k =
+  // 2c, 2c+1) and c*KB + 4s + {2, 3} (logical 2c+8, 2c+9), so that a lane's K
+  // codes for a position are the KB contiguous bytes [c*KB, (c+1)*KB).
+  const int r0 = lane >> 2, cq = lane & 3;
   uint32_t qa[KS][4];
   {
     const uint32_t *q32 = reinterpret_cast<const uint32_t *>(p.q);
@@ -217,82 +206,100 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnPar
       #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int row = r0 + ((i & 1) ? 8 : 0);
-        const int col = kk * 16 + cq + ((i & 2) ? 8 : 0);
+        const int col = cq * KB + 4 * kk + ((i & 2) ? 2 : 0);
         qa[kk][i] = row < p.G ? bf16x2_to_f16x2(__ldg(q32 + ((hrow0 + row) * D + col) / 2)) : 0u;
       }
     }
   }
 
-  // the accumulator is kept in units of `unit` (a value scale): O = acc * unit
-  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.0f, 0.0f}, unit = 1.0f;
+  // The accumulator is kept in units of `unit`, the largest value scale seen
+  // so far (O = acc * unit); column tile n, columns 2cq, 2cq+1 hold
+  // d = VB*(2cq) + n and VB*(2cq+1) + n (the V operand's d order: lane row r0
+  // holds d = VB*r0 + n, so its V codes for a position are the VB contiguous
+  // bytes [VB*r0, VB*(r0+1))).
+  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.0f, 0.0f}, unit = 0.0f;
   float acc[NT][4];
   #pragma unroll
   for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
 
-  int st = 0;
-  int base = c0 + warp * 16;
-  if (base < c1) prefetch(base, 0);
-  cp_async_commit();
-  for (; base < c1; base += kAttnWarps * 16, st ^= 1) {
-    const int next = base + kAttnWarps * 16;
-    if (next < c1) prefetch(next, st ^ 1);
+  constexpr int STEP = kAttnWarps * 16;
+  const int first = c0 + warp * 16;
+  #pragma unroll
+  for (int i = 0; i < kAttnStages - 1; ++i) {
+    if (first + i * STEP < c1) prefetch(first + i * STEP, i);
     cp_async_commit();
-    cp_async_wait<1>();     // this tile's copies have landed (the next tile's may not)
-    __syncwarp();
-    // decode this lane's codes to f16
+  }
+  int st = 0;
+  for (int base = first; base < c1; base += STEP) {
     {
-      const int kk = lane >> 1, half = lane & 1;
-      const uint8_t *ck = wcodes + st * SM::CODE_STAGE + kk * D + half * CB;
-      #pragma unroll
-      for (int i = 0; i < CB / 16; ++i) {
-        decode16(*reinterpret_cast<const uint4 *>(ck + 16 * i), sK + kk * PITCH + half * CB + i * 16);
-        decode16(*reinterpret_cast<const uint4 *>(ck + 16 * D + 16 * i), sV + kk * PITCH + half * CB + i * 16);
-      }
+      const int ahead = base + (kAttnStages - 1) * STEP;
+      int st_ahead = st + kAttnStages - 1;
+      if (st_ahead >= kAttnStages) st_ahead -= kAttnStages;
+      if (ahead < c1) prefetch(ahead, st_ahead);
+      cp_async_commit();
     }
-    const float *ksc = wscl + (st * 2 + 0) * 16;
-    const float *vsc = wscl + (st * 2 + 1) * 16;
-    // the tile's readable positions and its largest value scale
-    uint32_t vbits = 0;
-    float vmax = 0.0f;
-    {
-      const int pos = base + (lane & 15);
-      const bool valid = slot_of(pos) >= 0;
-      vbits = __ballot_sync(0xffffffffu, valid && lane < 16);
-      vmax = valid ? vsc[lane & 15] : 0.0f;
-      #pragma unroll
-      for (int o = 8; o >= 1; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-    }
+    cp_async_wait<kAttnStages - 1>();   // this tile's copies have landed
     __syncwarp();
+    const uint8_t *sk = ring + st * SM::STAGE;
+    const uint8_t *sv = sk + 16 * D;
+    const float *ksc = reinterpret_cast<const float *>(sk + SM::CODES_TILE);
+    const float *vsc = ksc + 16;
+    const uint32_t vmask = *reinterpret_cast<const uint32_t *>(ksc + 32);
 
-    // S = Q K^T: two 8-position column tiles
+    // S = Q K^T: column tile j holds positions 8j .. 8j+7 (B operand: lane
+    // row r0 = position 8j + r0, its KB code bytes)
     float s[2][4];
     #pragma unroll
     for (int j = 0; j < 2; ++j) {
+      const int pos = 8 * j + r0;
+      uint32_t kw[KB / 4];
+      #pragma unroll
+      for (int i = 0; i < KB / 16; ++i) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(sk + code_off<D>(pos, cq * (KB / 16) + i));
+        kw[4 * i] = v.x;
+        kw[4 * i + 1] = v.y;
+        kw[4 * i + 2] = v.z;
+        kw[4 * i + 3] = v.w;
+      }
       s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
       #pragma unroll
-      for (int kk = 0; kk < KS; ++kk) {
-        uint32_t b0, b1;
-        const int l8 = lane & 7, m = (lane >> 3) & 1;
-        ldsm_x2(b0, b1, sK + (j * 8 + l8) * PITCH + kk * 16 + m * 8);
-        mma_f16(s[j], qa[kk], b0, b1);
+      for (int kk = 0; kk < KS; ++kk)
+        mma_f16(s[j], qa[kk], e4m3x2_to_f16x2(lo16(kw[kk])), e4m3x2_to_f16x2(hi16(kw[kk])));
+    }
+
+    // this lane's positions: 2cq, 2cq+1 (column tile 0) and 2cq+8, 2cq+9 (tile 1)
+    const float2 ks01 = *reinterpret_cast<const float2 *>(ksc + 2 * cq);
+    const float2 ks89 = *reinterpret_cast<const float2 *>(ksc + 2 * cq + 8);
+    const float2 vs01 = *reinterpret_cast<const float2 *>(vsc + 2 * cq);
+    const float2 vs89 = *reinterpret_cast<const float2 *>(vsc + 2 * cq + 8);
+    const float kscl[2][2] = {{ks01.x, ks01.y}, {ks89.x, ks89.y}};
+    const float vscl[2][2] = {{vs01.x, vs01.y}, {vs89.x, vs89.y}};
+    bool ok[2][2];
+    float vmax = 0.0f;
+    #pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      #pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        ok[j][e] = (vmask >> (2 * (8 * j + 2 * cq + e))) & 1u;
+        if (ok[j][e]) vmax = fmaxf(vmax, vscl[j][e]);
       }
     }
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 1));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 2));
+
     // key scales, masking, online softmax (rows r0 and r0 + 8)
     float mx[2] = {-INFINITY, -INFINITY};
     #pragma unroll
     for (int j = 0; j < 2; ++j) {
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int kp = j * 8 + cq + e;
-        const bool valid = (vbits >> kp) & 1u;
-        const float k2 = ksc[kp] * p.scale_log2;
-        s[j][e] = valid ? s[j][e] * k2 : -INFINITY;
-        s[j][2 + e] = valid ? s[j][2 + e] * k2 : -INFINITY;
+        const float k2 = kscl[j][e] * p.scale_log2;
+        s[j][e] = ok[j][e] ? s[j][e] * k2 : -INFINITY;
+        s[j][2 + e] = ok[j][e] ? s[j][2 + e] * k2 : -INFINITY;
         mx[0] = fmaxf(mx[0], s[j][e]);
         mx[1] = fmaxf(mx[1], s[j][2 + e]);
       }
     }
-    const float inv_vmax = vmax > 0.0f ? 1.0f / vmax : 0.0f;
     float alpha[2], psum[2] = {0.0f, 0.0f};
     #pragma unroll
     for (int r = 0; r < 2; ++r) {
@@ -303,13 +310,18 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnPar
       alpha[r] = m_new == -INFINITY ? 1.0f : exp2f(m_r[r] - m_new);
       m_r[r] = m_new;
     }
+    // the unit grows to this tile's largest value scale where that is larger
+    const float new_unit = fmaxf(unit, vmax);
+    const float to_unit = new_unit > unit && unit > 0.0f ? __fdividef(unit, new_unit) : 1.0f;
+    unit = new_unit;
+    const float inv_unit = unit > 0.0f ? __fdividef(1.0f, unit) : 0.0f;
     uint32_t pa[4];
     #pragma unroll
     for (int j = 0; j < 2; ++j) {
       float pv[4];
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const float vr = vsc[j * 8 + cq + e] * inv_vmax;   // this position's value scale / the tile's largest
+        const float vr = vscl[j][e] * inv_unit;   // this position's value scale / the unit
         const float p0 = m_r[0] == -INFINITY ? 0.0f : exp2f(s[j][e] - m_r[0]);
         const float p1 = m_r[1] == -INFINITY ? 0.0f : exp2f(s[j][2 + e] - m_r[1]);
         psum[0] += p0;
@@ -317,57 +329,80 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const AttnPar
         pv[e] = p0 * vr;
         pv[2 + e] = p1 * vr;
       }
-      pa[2 * j] = h2_bits(__floats2half2_rn(pv[0], pv[1]));       // row r0, positions j*8 + cq, +1
+      pa[2 * j] = h2_bits(__floats2half2_rn(pv[0], pv[1]));       // row r0, positions 8j + 2cq, +1
       pa[2 * j + 1] = h2_bits(__floats2half2_rn(pv[2], pv[3]));   // row r0 + 8
     }
-    // move the accumulator to this tile's units (vmax), with the softmax factor
-    const float to_tile = vmax > 0.0f ? unit * inv_vmax : 1.0f;
-    if (vmax > 0.0f) unit = vmax;
     #pragma unroll
     for (int r = 0; r < 2; ++r) {
       psum[r] += __shfl_xor_sync(0xffffffffu, psum[r], 1);
       psum[r] += __shfl_xor_sync(0xffffffffu, psum[r], 2);
       l_r[r] = l_r[r] * alpha[r] + psum[r];
-      alpha[r] *= to_tile;
+      alpha[r] *= to_unit;
     }
-    #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      acc[n][0] *= alpha[0];
-      acc[n][1] *= alpha[0];
-      acc[n][2] *= alpha[1];
-      acc[n][3] *= alpha[1];
+    // rescale the accumulator only where a factor differs from one
+    if (__any_sync(0xffffffffu, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
+      #pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        acc[n][0] *= alpha[0];
+        acc[n][1] *= alpha[0];
+        acc[n][2] *= alpha[1];
+        acc[n][3] *= alpha[1];
+      }
     }
-    // O += P V (A = P: rows r0 / r0 + 8, positions cq.. and cq + 8..)
+
+    // O += P V.  A = P (rows r0 / r0 + 8; k = positions 2cq, 2cq+1 and
+    // 2cq+8, 2cq+9); B = V (k = those positions, n = d of column tile n):
+    // lane row r0 holds d = VB*r0 + n, so the two codes of a B register (two
+    // positions, one d) are byte n of two positions' VB-byte runs, paired
+    // with a byte permute before the conversion.
     const uint32_t a[4] = {pa[0], pa[1], pa[2], pa[3]};
+    uint32_t vw[4][VB / 4];
     #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      uint32_t b0, b1;
-      const int l8 = lane & 7, m = (lane >> 3) & 1;
-      ldsm_x2_trans(b0, b1, sV + (m * 8 + l8) * PITCH + n * 8);
-      mma_f16(acc[n], a, b0, b1);
+    for (int q = 0; q < 4; ++q) {
+      const int pos = 2 * cq + (q & 1) + ((q & 2) ? 8 : 0);
+      if constexpr (VB == 16) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(sv + code_off<D>(pos, r0));
+        vw[q][0] = v.x;
+        vw[q][1] = v.y;
+        vw[q][2] = v.z;
+        vw[q][3] = v.w;
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2 *>(sv + code_off<D>(pos, r0 >> 1) + 8 * (r0 & 1));
+        vw[q][0] = v.x;
+        vw[q][1] = v.y;
+      }
     }
-    __syncwarp();  // the next tile overwrites this warp's tiles
+    #pragma unroll
+    for (int n = 0; n < NT; n += 2) {
+      const uint32_t sel = (n & 2) ? 0x7362u : 0x5140u;
+      const uint32_t x01 = __byte_perm(vw[0][n >> 2], vw[1][n >> 2], sel);   // positions 2cq, 2cq+1
+      const uint32_t x89 = __byte_perm(vw[2][n >> 2], vw[3][n >> 2], sel);   // positions 2cq+8, 2cq+9
+      mma_f16(acc[n], a, e4m3x2_to_f16x2(lo16(x01)), e4m3x2_to_f16x2(lo16(x89)));
+      mma_f16(acc[n + 1], a, e4m3x2_to_f16x2(hi16(x01)), e4m3x2_to_f16x2(hi16(x89)));
+    }
+    __syncwarp();  // this stage is refilled two tiles later
+    if (++st == kAttnStages) st = 0;
   }
   cp_async_wait<0>();
 
   // combine the four warps' states (each accumulator times its unit)
-  if ((lane & 3) == 0) {
+  if (cq == 0) {
     s_ml[warp][r0][0] = m_r[0];
     s_ml[warp][r0][1] = l_r[0];
     s_ml[warp][r0 + 8][0] = m_r[1];
     s_ml[warp][r0 + 8][1] = l_r[1];
   }
-  if (lane == 0) s_unit[warp] = unit;
-  __syncthreads();  // every warp has finished with its tiles: the buffer is free
-  float *s_acc = reinterpret_cast<float *>(s_tiles);   // [warp][16][D]
+  __syncthreads();  // every warp has finished with its ring: the buffer is free
+  float *s_acc = reinterpret_cast<float *>(dsmem);   // [warp][16][D]
   #pragma unroll
   for (int n = 0; n < NT; ++n) {
-    float *row0 = s_acc + ((size_t)warp * 16 + r0) * D + n * 8 + cq;
-    float *row1 = s_acc + ((size_t)warp * 16 + r0 + 8) * D + n * 8 + cq;
-    row0[0] = acc[n][0] * unit;
-    row0[1] = acc[n][1] * unit;
-    row1[0] = acc[n][2] * unit;
-    row1[1] = acc[n][3] * unit;
+    const int d0 = VB * (2 * cq) + n, d1 = VB * (2 * cq + 1) + n;
+    float *row0 = s_acc + ((size_t)warp * 16 + r0) * D;
+    float *row1 = s_acc + ((size_t)warp * 16 + r0 + 8) * D;
+    row0[d0] = acc[n][0] * unit;
+    row0[d1] = acc[n][1] * unit;
+    row1[d0] = acc[n][2] * unit;
+    row1[d1] = acc[n][3] * unit;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < p.G * D; i += kAttnThreads) {

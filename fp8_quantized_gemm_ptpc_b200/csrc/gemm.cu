@@ -70,7 +70,11 @@ __host__ __device__ constexpr uint32_t wf_mma(int wf) {
 
 struct GemmParams {
   int T, Co;
-  int num_m, num_n, num_kb;   // tile grid (pair kernel: 256-token tile rows; decode: one row of all tokens)
+  int num_m, num_n, num_kb;   // tile grid (pair kernel: token tile rows; decode: one row of all tokens)
+  // pair kernel, operands swapped: the weights are the MMA's M = 256 operand
+  // (256 channels a tile) and nt tokens (a multiple of 32, at most 256) its N
+  // operand; swap = 0: 256 tokens x BN channels a tile
+  int swap, nt;
   int group_m;                // tile rows visited together (L2 reuse of weights)
   int num_tiles;
   int ksplit;                 // decode kernel: CTAs (one cluster) per tile, 1 = whole tiles
@@ -257,11 +261,12 @@ __device__ __forceinline__ void epilogue_store_tile(const CUtensorMap *tmC, uint
 // for the cluster reduction instead of storing.
 // ----------------------------------------------------------------------------
 constexpr int kDecodeMaxT = 256;       // largest T the decode kernel takes (MMA N <= 256)
-constexpr int kDecodeWholeMaxT = 192;  // above this, the decode kernel only when it splits K
+constexpr int kDecodeWholeMaxT = 192;  // above this, the pair kernel (unless forced)
 constexpr int kDecMaxStages = 16;
 constexpr int kDecWBytes = BM * BK;   // weight tile of one stage
 constexpr size_t kDecBarBytes = 512;  // barriers and flags after the ring
 constexpr size_t kDecSmemMax = 232448;
+constexpr int kDecPrefetchBytes = 192 * 1024;  // weight bytes an SM prefetches into L2 ahead of its loads
 
 __host__ __device__ constexpr size_t dec_smem_bytes(int np, int stages) {
   return 1024 + (size_t)stages * (kDecWBytes + (size_t)np * BK) + kDecBarBytes;
@@ -436,6 +441,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       Sched sc;
       Unit u;
+      // L2 prefetch of the weight tiles kDecPrefetchBytes ahead of the loads
+      // (a second walk of the same schedule): the ring holds the weights
+      // unpacked, so a sub-byte format keeps only half (FP4) or 3/4 (FP6) of
+      // the ring's bytes in flight from HBM; with the tiles already in L2 the
+      // ring's loads return sooner and the SM's stream keeps up.
+      Sched sa;
+      Unit ua;
+      sa.init(p, blockIdx.x, gridDim.x);
+      bool more_a = sa.next(p, ua);
+      int kba = ua.kb0;
+      auto advance_a = [&]() {
+        if (more_a && ++kba >= ua.kb1) {
+          more_a = sa.next(p, ua);
+          kba = ua.kb0;
+        }
+      };
+      const int pf_ahead = kDecPrefetchBytes / (kDecWBytes * wf_bits(WF) / 8);
+      for (int i = 0; i < pf_ahead; ++i) advance_a();
+      auto prefetch_next = [&]() {
+        if (more_a) tma_prefetch_2d(&tmW, kba * BK, ua.n * BM);
+        advance_a();
+      };
       // The weights never depend on the kernel launched just before this one:
       // the first stages' weight tiles are requested before waiting for it.
       int pre = 0;
@@ -444,6 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (; pre < STAGES && u.kb0 + pre < u.kb1; ++pre) {
           mbar_arrive_expect_tx(&full[pre], stage_tx);
           tma_load_2d(sW + pre * kDecWBytes, &tmW, &full[pre], (u.kb0 + pre) * BK, u.n * BM, polW);
+          prefetch_next();
         }
       }
       griddep_wait();  // Xq may come from the kernel launched just before
@@ -458,6 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mbar_arrive_expect_tx(&full[stage], stage_tx);
             tma_load_2d(sW + stage * kDecWBytes, &tmW, &full[stage], kb * BK, u.n * BM, polW);
+            prefetch_next();
           }
           tma_load_2d(sX + stage * X_BYTES, &tmX, &full[stage], kb * BK, 0, polX);
           if (++stage == STAGES) {
@@ -611,8 +640,83 @@ __device__ __forceinline__ void dump_partial(uint32_t tbase, float *row_dst, int
   }
 }
 
+// Operands swapped: tensor-memory lane = output channel, column = token.
+// This warp's 32 channels [ch0, ch0 + 32) of tokens [t0, t0 + nt): each
+// chunk of 32 tokens is scaled ((acc * x_scale) * w_scale, the same order as
+// the unswapped tile), transposed through shared memory ([32 tokens][32
+// channels], unswizzled) and stored by TMA; the output map clips tokens >= T
+// and channels >= Co.  The accumulator buffer is released after its last
+// tensor-memory read.
+template <bool F32OUT>
+__device__ __forceinline__ void epilogue_store_swap(const CUtensorMap *tmC, uint32_t tbase, uint8_t *cbuf,
+                                                    const GemmParams &p, int ch0, int t0, int lane,
+                                                    uint32_t release_bar) {
+  const int ch = ch0 + lane;
+  float wsr = 0.0f;
+  if constexpr (!F32OUT) wsr = ch < p.Co ? __ldg(p.ws + ch) : 0.0f;
+  #pragma unroll 1
+  for (int c0 = 0; c0 < p.nt; c0 += 32) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(tbase + c0, r);
+    tmem_wait_ld();
+    if (c0 + 32 >= p.nt) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(release_bar);
+    }
+    float xsl = 0.0f;  // lane j holds the scale of token t0 + c0 + j
+    if constexpr (!F32OUT) {
+      const int t = t0 + c0 + lane;
+      xsl = t < p.T ? __ldg(p.xs + t) : 0.0f;
+    }
+    // the previous TMA store from this buffer must have finished reading it
+    if (lane == 0) bulk_wait_read<0>();
+    __syncwarp();
+    if constexpr (F32OUT) {
+      float *s = reinterpret_cast<float *>(cbuf);
+      #pragma unroll
+      for (int j = 0; j < 32; ++j) s[j * 32 + lane] = __uint_as_float(r[j]);
+    } else {
+      __nv_bfloat16 *s = reinterpret_cast<__nv_bfloat16 *>(cbuf);
+      #pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float xs = __shfl_sync(0xffffffffu, xsl, j);
+        s[j * 32 + lane] = __float2bfloat16_rn(__fmul_rn(__fmul_rn(__uint_as_float(r[j]), xs), wsr));
+      }
+    }
+    fence_async_shared();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmC, cbuf, ch0, t0 + c0);
+      bulk_commit();
+    }
+  }
+}
+
+// Operands swapped, split tail: this lane's channel of the partial
+// accumulator, stored transposed (partial[token][channel], 256 channels a
+// token row) so that the reduction reads and writes whole channel runs.
+__device__ __forceinline__ void dump_partial_swap(uint32_t tbase, float *col_dst, int nt, int lane,
+                                                  uint32_t release_bar) {
+  #pragma unroll 1
+  for (int c0 = 0; c0 < nt; c0 += 32) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(tbase + c0, r);
+    tmem_wait_ld();
+    if (c0 + 32 >= nt) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(release_bar);
+    }
+    #pragma unroll
+    for (int j = 0; j < 32; ++j) __stcg(col_dst + (size_t)(c0 + j) * 256, __uint_as_float(r[j]));
+  }
+}
+
 // Reducer `ridx` (0 .. 2 * split - 1) of tail tile j at tile position (m, n):
 // groups of 8 output columns, [ridx * G / (2 S), (ridx + 1) * G / (2 S)).
+// A partial tile is R token rows x BN_T channels (R = 256, or nt when the
+// operands are swapped).
 // A thread takes U groups at a time and loads four splits of all of them
 // before adding (8 U independent 16-byte loads in flight: the partials come
 // from L2, and a load-add chain per split would leave the reduction waiting on
@@ -622,12 +726,13 @@ __device__ __forceinline__ void reduce_tail_tile(const GemmParams &p, int j, int
   constexpr int U = 2;
   constexpr int SU = 4;
   const int S = p.tail_split;
+  const int R = p.swap ? p.nt : 2 * BM;
   constexpr int G8 = BN_T / 8;
-  constexpr int G = 2 * BM * G8;
+  const int G = R * G8;
   const int g0 = (int)((long long)ridx * G / (2 * S));
   const int g1 = (int)((long long)(ridx + 1) * G / (2 * S));
-  const float *base = p.partials + (size_t)j * S * (2 * BM) * BN_T;
-  const size_t split_stride = (size_t)(2 * BM) * BN_T;
+  const float *base = p.partials + (size_t)j * S * R * BN_T;
+  const size_t split_stride = (size_t)R * BN_T;
   for (int gb = g0 + etid; gb < g1; gb += U * 32 * kEpiWarps) {
     float a[U][8];
     size_t off[U];
@@ -675,7 +780,7 @@ __device__ __forceinline__ void reduce_tail_tile(const GemmParams &p, int j, int
       const int g = gb + u * 32 * kEpiWarps;
       const int row = g / G8;
       const int c8 = (g - row * G8) * 8;
-      const int t = m * (2 * BM) + row;
+      const int t = m * R + row;
       const int col = n * BN_T + c8;
       if (t >= p.T || col >= p.Co) continue;  // Co % 16 == 0: the 8 columns are valid together
       const float xs = __ldg(p.xs + t);
@@ -707,6 +812,15 @@ __device__ __forceinline__ void reduce_tail_tile(const GemmParams &p, int j, int
 // ----------------------------------------------------------------------------
 // BN: tile width (MMA N), 256 or 128; each CTA of the pair loads BN / 2
 // weight rows.
+//
+// Swapped operands (BN = 256 variants, p.swap): for token counts that leave
+// most of a 256-row tile empty (e.g. T = 300: 512 rows computed for 300), the
+// weights become the M = 256 operand (CTA r loads channel rows [r*128,
+// r*128+128) of a 256-channel tile) and nt tokens the N operand (CTA r loads
+// nt / 2 token rows), nt a multiple of 32 chosen so that the token tiles
+// divide T evenly.  Tensor-memory lane = channel, column = token; the
+// epilogue transposes through shared memory.  Same ring, barriers, schedule
+// and split tail.
 template <int STAGES, bool F32OUT, int BN, int WF = 0>
 struct PairCfg {
   static constexpr int A_BYTES = BM * BK;
@@ -780,14 +894,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool ok = true;
       Sched sc;
       Unit u;
+      // Which shared-memory slot takes the weight tile and which the token
+      // tile: unswapped, tokens are the A operand (128 rows a CTA) and
+      // weights B (HALF_N rows); swapped, the weights are A (128 channel rows
+      // a CTA) and the tokens B (nt / 2 rows a CTA).
+      bool swap = false;
+      if constexpr (BN == 256) swap = p.swap != 0;
+      uint8_t *const sW = swap ? sA : sB;
+      uint8_t *const sX = swap ? sB : sA;
+      const int w_stride = swap ? C::A_BYTES : C::B_BYTES;
+      const int x_stride = swap ? C::B_BYTES : C::A_BYTES;
+      const uint32_t stage_tx = swap ? 2u * (uint32_t)(C::B_TX + (p.nt / 2) * BK) : 2u * (C::A_BYTES + C::B_TX);
+      const int x_rows = swap ? p.nt : 2 * BM;
       // weight tiles of the first stages before waiting for the previous kernel
       int pre = 0;
       sc.init(p, cid, ncl);
       if (sc.next(p, u)) {
-        const int b_row = u.n * BN + (int)rank * HALF_N;
+        const int w_row = u.n * BN + (int)rank * HALF_N;
         for (; pre < STAGES && u.kb0 + pre < u.kb1; ++pre) {
-          if (leader) mbar_arrive_expect_tx(&full[pre], 2 * (C::A_BYTES + C::B_TX));
-          tma_load_2d_pair(sB + pre * C::B_BYTES, &tmB, mapa_shared(&full[pre], 0), (u.kb0 + pre) * BK, b_row,
+          if (leader) mbar_arrive_expect_tx(&full[pre], stage_tx);
+          tma_load_2d_pair(sW + pre * w_stride, &tmB, mapa_shared(&full[pre], 0), (u.kb0 + pre) * BK, w_row,
                            polB);
         }
       }
@@ -795,8 +921,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int issued = 0;
       sc.init(p, cid, ncl);
       while (ok && sc.next(p, u)) {
-        const int a_row = u.m * (2 * BM) + (int)rank * BM;
-        const int b_row = u.n * BN + (int)rank * HALF_N;
+        const int x_row = u.m * x_rows + (int)rank * (x_rows / 2);
+        const int w_row = u.n * BN + (int)rank * HALF_N;
         for (int kb = u.kb0; kb < u.kb1; ++kb, ++issued) {
           const uint32_t lead_full = mapa_shared(&full[stage], 0);
           if (issued >= pre) {
@@ -804,10 +930,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
-            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * (C::A_BYTES + C::B_TX));
-            tma_load_2d_pair(sB + stage * C::B_BYTES, &tmB, lead_full, kb * BK, b_row, polB);
+            if (leader) mbar_arrive_expect_tx(&full[stage], stage_tx);
+            tma_load_2d_pair(sW + stage * w_stride, &tmB, lead_full, kb * BK, w_row, polB);
           }
-          tma_load_2d_pair(sA + stage * C::A_BYTES, &tmA, lead_full, kb * BK, a_row, polA);
+          tma_load_2d_pair(sX + stage * x_stride, &tmA, lead_full, kb * BK, x_row, polA);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -826,7 +952,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (leader && elect_one()) {
-      constexpr uint32_t idesc = idesc_f8f6f4_f32(2 * BM, BN, kMmaE4M3, wf_mma(WF));  // B = weights
+      // unswapped: A = tokens, B = weights (N = BN); swapped: A = weights, B = tokens (N = nt)
+      uint32_t idesc = idesc_f8f6f4_f32(2 * BM, BN, kMmaE4M3, wf_mma(WF));
+      if constexpr (BN == 256)
+        if (p.swap) idesc = idesc_f8f6f4_f32(2 * BM, p.nt, wf_mma(WF), kMmaE4M3);
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
@@ -878,6 +1007,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     float *scl = sScale + ew * 64;
     int local = 0;
     bool ok = true;
+    bool swap = false;
+    if constexpr (BN == 256) swap = p.swap != 0;
     // a member of the split tail: decided by the schedule alone, so every
     // epilogue warp runs the tail protocol's barriers whatever happens above
     const bool tail_member = p.tail_tiles > 0 && !F32OUT && cid < p.tail_tiles * p.tail_split;
@@ -898,7 +1029,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int row0 = u.m * (2 * BM) + (int)rank * BM + q * 32;
       const int row = row0 + lane;
       float xsr = 0.0f;
-      if (!F32OUT && row < p.T) xsr = __ldg(p.xs + row);
+      if (!F32OUT && !swap && row < p.T) xsr = __ldg(p.xs + row);
       // tcgen05.ld is warp-collective: the whole warp stops or none of it
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[buf], aphase))) {
         ok = false;
@@ -906,7 +1037,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
-      if (u.split < 0) {
+      if (swap) {
+        if constexpr (BN == 256) {
+          // lanes are channels u.n * 256 + rank * 128 + q * 32 + lane, columns tokens
+          const int ch0 = u.n * BN + (int)rank * HALF_N + q * 32;
+          if (u.split < 0) {
+            epilogue_store_swap<F32OUT>(&tmC, tbase, cbuf, p, ch0, u.m * p.nt, lane,
+                                        mapa_shared(&tempty[buf], 0));
+          } else if constexpr (!F32OUT) {
+            tail_j = u.tile - p.full_tiles;
+            tail_m = u.m;
+            tail_n = u.n;
+            tail_r = u.split;
+            float *dst = p.partials + (size_t)(tail_j * p.tail_split + u.split) * p.nt * BN +
+                         (rank * HALF_N + q * 32 + lane);
+            dump_partial_swap(tbase, dst, p.nt, lane, mapa_shared(&tempty[buf], 0));
+            dumped = true;
+          }
+        }
+      } else if (u.split < 0) {
         epilogue_store_tile<BN, F32OUT>(&tmC, tbase, cbuf, scl, p, u.n * BN, row0, xsr, lane,
                                         mapa_shared(&tempty[buf], 0));
       } else if constexpr (!F32OUT) {
@@ -1101,6 +1250,21 @@ bool make_maps(const GemmProblem &pr, uint32_t b_rows, CUtensorMap *tmA, CUtenso
                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// Swapped operands: token tiles of nt / 2 rows a CTA, weight tiles of 128
+// rows a CTA, and an output box of 32 channels x 32 tokens, unswizzled (the
+// epilogue's transposed staging).
+bool make_swap_maps(const GemmProblem &pr, int nt, CUtensorMap *tmA, CUtensorMap *tmB, CUtensorMap *tmC) {
+  if (!make_map_2d(tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, pr.Xq, pr.Ci, pr.T, pr.Ci, BK, (uint32_t)(nt / 2),
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_weight_map(tmB, pr, BM))
+    return false;
+  if (pr.f32_out)
+    return make_map_2d(tmC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, pr.out, pr.Co, pr.T, (uint64_t)pr.Co * 4, 32, 32,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+  return make_map_2d(tmC, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, pr.out, pr.Co, pr.T, (uint64_t)pr.Co * 2, 32, 32,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 // Ring depth of the pair kernel per tile width (the stages fill ~192 KB).
 template <int BN>
 constexpr int pair_stages() {
@@ -1219,6 +1383,8 @@ struct Plan {
   int np, stages, tmem_cols;  // decode kernel only
   bool red_fits;              // decode kernel: the K-split buffer fits in the ring
   int tail_tiles, tail_split; // pair kernel: split tail (0: every tile whole)
+  bool swap;                  // pair kernel: weights as the M operand, nt tokens a tile
+  int nt;
 };
 
 // Time of a 128-wide pair tile relative to half a 256-wide one.  Measured on
@@ -1232,13 +1398,16 @@ constexpr double kPairN128Cost = 1.15;
 // Tuning overrides (not for production use), from the environment:
 // PTPC_FORCE_KERNEL = pair | decode, PTPC_FORCE_PAIR_BN = 128 | 256,
 // PTPC_FORCE_KSPLIT = 1 | 2 | 4 | 8, PTPC_FORCE_SPLIT_TAIL = 0 | 1 (the pair
-// kernel's split tail off, or on wherever it is feasible).  Read once, at the
-// first GEMM call of the process (or again by reload_tuning), not on every call.
+// kernel's split tail off, or on wherever it is feasible), PTPC_FORCE_SWAP =
+// 0 | 1 (the pair kernel's swapped operands off, or on for every pair-kernel
+// shape).  Read once, at the first GEMM call of the process (or again by
+// reload_tuning), not on every call.
 struct Tuning {
   int kernel;   // 0 automatic, 1 pair, 2 decode
   int pair_bn;  // 0 automatic, 128, 256
   int ksplit;   // 0 automatic, 1, 2, 4, 8
   int streamk;  // 0 automatic, 1 off, 2 on wherever feasible
+  int swap;     // 0 automatic, 1 off, 2 on
 };
 
 int env_int(const char *name, int fallback) {
@@ -1250,7 +1419,7 @@ int env_int(const char *name, int fallback) {
 }
 
 Tuning read_tuning() {
-  Tuning t{0, 0, 0};
+  Tuning t{0, 0, 0, 0, 0};
   const char *k = std::getenv("PTPC_FORCE_KERNEL");
   if (k != nullptr && std::strcmp(k, "pair") == 0) t.kernel = 1;
   if (k != nullptr && std::strcmp(k, "decode") == 0) t.kernel = 2;
@@ -1261,16 +1430,19 @@ Tuning read_tuning() {
   const int sk = env_int("PTPC_FORCE_SPLIT_TAIL", -1);
   if (sk == 0) t.streamk = 1;
   if (sk == 1) t.streamk = 2;
+  const int sw = env_int("PTPC_FORCE_SWAP", -1);
+  if (sw == 0) t.swap = 1;
+  if (sw == 1) t.swap = 2;
   return t;
 }
 
-// Packed as kernel | pair_bn / 128 << 2 | ksplit << 4 | streamk << 9, plus
-// bit 8 once read.
+// Packed as kernel | pair_bn / 128 << 2 | ksplit << 4 | streamk << 9 |
+// swap << 11, plus bit 8 once read.
 std::atomic<uint32_t> g_tuning{0};
 
 uint32_t pack_tuning(const Tuning &t) {
   return 0x100u | (uint32_t)t.kernel | (uint32_t)(t.pair_bn / 128) << 2 | (uint32_t)t.ksplit << 4 |
-         (uint32_t)t.streamk << 9;
+         (uint32_t)t.streamk << 9 | (uint32_t)t.swap << 11;
 }
 
 Tuning tuning() {
@@ -1279,7 +1451,8 @@ Tuning tuning() {
     v = pack_tuning(read_tuning());
     g_tuning.store(v, std::memory_order_relaxed);
   }
-  return Tuning{(int)(v & 3u), (int)((v >> 2) & 3u) * 128, (int)((v >> 4) & 15u), (int)((v >> 9) & 3u)};
+  return Tuning{(int)(v & 3u), (int)((v >> 2) & 3u) * 128, (int)((v >> 4) & 15u), (int)((v >> 9) & 3u),
+                (int)((v >> 11) & 3u)};
 }
 
 // Fewest K-blocks a CTA of a K-split cluster streams.
@@ -1343,6 +1516,12 @@ int choose_pair_bn(int T, int Co, const DeviceInfo &d) {
 // time plus the partials' round trip through L2 and the distributed
 // reduction.  Taken only where the caller's workspace holds the partials.
 constexpr int kMinTailKb = 4;
+// Measured on B200 (70B layers, T = 256 ... 3001, split on against off): the
+// split pays only on long K (down-proj, K = 28672: +8% at T = 2048, +13% at
+// T = 3001); at K = 8192 it is within +-2% on gate+up and 1-5% slower on
+// the 10240-wide QKV, since a last wave of few tiles already runs at the
+// higher clock that the idle rest of the GPU leaves it.
+constexpr int kMinTailTotalKb = 128;
 constexpr int kMaxTailPairs = 74;      // bound of the workspace size (a B200's 148 SMs in pairs)
 constexpr size_t kTailCountBytes = 1024;
 
@@ -1355,6 +1534,7 @@ void choose_tail(Plan &pl, size_t ws_bytes) {
   pl.tail_split = 0;
   const int forced = tuning().streamk;          // 0 automatic, 1 off, 2 on
   if (forced == 1 || pl.num_tiles <= pl.ctas) return;
+  if (forced != 2 && pl.num_kb < kMinTailTotalKb) return;
   const int rem = pl.num_tiles % pl.ctas;
   if (rem == 0) return;
   const int pairs = std::min(pl.ctas, kMaxTailPairs);
@@ -1367,11 +1547,40 @@ void choose_tail(Plan &pl, size_t ws_bytes) {
   pl.tail_split = split;
 }
 
-// The prefill kernel's plan: whole tiles on the CTA pairs.
-// Sharing the last partial wave stream-K style (fp32 partial sums through
-// global memory, fixed-order fixup) was measured slower on B200 for these
-// tiles (e.g. 2048 x 4096 -> 6144: 73.8 us shared vs 43.1 us whole;
-// 2048 x 14336 -> 4096: 136.8 vs 109.7).
+// Cost of a swapped pair tile of nt tokens, in unswapped 256 x 256 tile
+// times: F + (1 - F) nt / 256.  The tensor work scales with nt, but every
+// stage still moves the 16 KB-a-CTA weight tile through shared memory
+// (written by TMA, read by the MMA) whatever nt is.  Measured on B200 (70B
+// layers, same tile counts both ways): nt = 160 costs 0.74, 192 0.81, 224
+// 0.87 of an unswapped tile; F = 0.3 fits the small nt, which matter most.
+constexpr double kSwapFixed = 0.3;
+
+double swap_tile_cost(int nt) {
+  const double f = nt / 256.0;
+  return kSwapFixed + (1.0 - kSwapFixed) * f;
+}
+
+// Tile times of `tiles` tiles on `pairs` CTA pairs: whole waves, and a last
+// partial wave that costs a whole tile time, or 1/split of one (plus 0.1 for
+// the partials' round trip) where the split tail takes it (same conditions
+// as choose_tail).
+double est_waves(long long tiles, int pairs, int num_kb, size_t ws_bytes, int bn) {
+  const long long full = tiles / pairs;
+  const long long rem = tiles % pairs;
+  if (rem == 0) return (double)full;
+  const int forced = tuning().streamk;
+  if (full > 0 && forced != 1 && (forced == 2 || num_kb >= kMinTailTotalKb) && (forced == 2 || 2 * rem <= pairs)) {
+    const int split = (int)std::min<long long>(std::min(pairs, kMaxTailPairs) / rem, num_kb / kMinTailKb);
+    if (split >= 2 && kGemmStatusBytes + tail_workspace((int)rem, split, bn) <= ws_bytes)
+      return (double)full + 1.0 / split + 0.1;
+  }
+  return (double)(full + 1);
+}
+
+// The prefill kernel's plan: whole tiles on the CTA pairs, 256 tokens x BN
+// channels a tile, or, with the operands swapped, 256 channels x nt tokens
+// where that finishes the waves sooner (ragged T: the token tiles divide T
+// evenly instead of rounding it up to 256 rows), then the split tail.
 Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d, size_t ws_bytes) {
   Plan pl = {};
   pl.pair = true;
@@ -1383,6 +1592,24 @@ Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d, size_t ws_bytes) {
   pl.num_m = (T + pl.tile_rows - 1) / pl.tile_rows;
   pl.num_n = (Co + pl.bn - 1) / pl.bn;
   pl.num_tiles = pl.num_m * pl.num_n;
+  const int pairs = pl.bn == 128 ? d.pair_clusters128 : d.pair_clusters;
+  // swapped: ceil(T / 256) token tiles of equal size, rounded up to 32
+  const int ntt = (T + 2 * BM - 1) / (2 * BM);
+  const int nt = ((T + ntt - 1) / ntt + 31) / 32 * 32;
+  const long long swap_tiles = (long long)ntt * ((Co + 255) / 256);
+  const double cost_plain = est_waves(pl.num_tiles, pairs, pl.num_kb, ws_bytes, pl.bn) *
+                            (pl.bn == 128 ? 0.5 * kPairN128Cost : 1.0);
+  const double cost_swap = est_waves(swap_tiles, d.pair_clusters, pl.num_kb, ws_bytes, 256) * swap_tile_cost(nt);
+  const int forced = tuning().swap;  // 0 automatic, 1 off, 2 on
+  pl.swap = forced == 2 || (forced == 0 && cost_swap < cost_plain);
+  if (pl.swap) {
+    pl.nt = nt;
+    pl.tile_rows = nt;
+    pl.bn = 256;
+    pl.num_m = ntt;
+    pl.num_n = (Co + 255) / 256;
+    pl.num_tiles = (int)swap_tiles;
+  }
   pl.ctas = std::max(1, std::min(pl.num_tiles, pl.bn == 128 ? d.pair_clusters128 : d.pair_clusters));
   choose_tail(pl, ws_bytes);
   return pl;
@@ -1390,21 +1617,16 @@ Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d, size_t ws_bytes) {
 
 // Which kernel runs a shape.  Measured on B200 with weights streamed from
 // HBM (70B layer shapes): the decode kernel is faster than the pair kernel
-// for every T <= 160; between 192 and 256 only where it splits K (e.g.
-// T = 256, 28672 -> 8192: 63.5 us vs 93.2 us), while with whole tiles it
-// ties at T = 192 and falls behind above (T = 256, 8192 -> 28672: 67.1 us vs
-// 59.0 us).
+// for every T <= 160 and ties at T = 192; above, the pair kernel wins, with a
+// K split in the decode kernel too (T = 256, 28672 -> 8192: 53.8 us against
+// 66.1 us; 8192 -> 8192: 25.3 against 31.4 us).
 // PTPC_FORCE_KERNEL = "pair" or "decode" overrides the choice (tuning only;
 // the decode kernel takes T <= 256 only).
 Plan make_plan(int T, int Ci, int Co, size_t ws_bytes) {
   const DeviceInfo &d = device_info();
   const int force = tuning().kernel;
   if (force == 1) return pair_plan(T, Ci, Co, d, ws_bytes);
-  if (T <= kDecodeMaxT) {
-    const Plan pl = decode_plan(T, Ci, Co, d);
-    if (force == 2) return pl;
-    if (T <= kDecodeWholeMaxT || pl.ksplit > 1) return pl;
-  }
+  if (T <= kDecodeMaxT && (force == 2 || T <= kDecodeWholeMaxT)) return decode_plan(T, Ci, Co, d);
   return pair_plan(T, Ci, Co, d, ws_bytes);
 }
 
@@ -1502,6 +1724,11 @@ int gemm_ksplit(int T, int Ci, int Co) { return make_plan(T, Ci, Co, gemm_worksp
 
 int gemm_tail_split(int T, int Ci, int Co, size_t ws_bytes) { return make_plan(T, Ci, Co, ws_bytes).tail_split; }
 
+int gemm_swap_tokens(int T, int Ci, int Co, size_t ws_bytes) {
+  const Plan pl = make_plan(T, Ci, Co, ws_bytes);
+  return pl.pair && pl.swap ? pl.nt : 0;
+}
+
 size_t gemm_workspace_bytes(int T, int Ci, int Co) {
   // the status word, plus the split tail's counters and partials where the
   // pair kernel could split one (more than one wave, K long enough), sized
@@ -1528,6 +1755,8 @@ cudaError_t launch_scaled_gemm(const GemmProblem &pr, cudaStream_t st) {
   gp.tail_tiles = pl.tail_tiles;
   gp.tail_split = pl.tail_split;
   gp.full_tiles = pl.num_tiles - pl.tail_tiles;
+  gp.swap = pl.swap ? 1 : 0;
+  gp.nt = pl.nt;
   if (pl.tail_tiles > 0) {
     uint8_t *w = reinterpret_cast<uint8_t *>(pr.status);
     gp.tail_count = reinterpret_cast<uint32_t *>(w + kGemmStatusBytes);
@@ -1554,7 +1783,11 @@ cudaError_t launch_scaled_gemm(const GemmProblem &pr, cudaStream_t st) {
     }
   }
   CUtensorMap tmA, tmB, tmC;
-  if (!make_maps(pr, pl.bn / 2, &tmA, &tmB, &tmC)) return cudaErrorInvalidValue;
+  if (pl.swap) {
+    if (!make_swap_maps(pr, pl.nt, &tmA, &tmB, &tmC)) return cudaErrorInvalidValue;
+  } else if (!make_maps(pr, pl.bn / 2, &tmA, &tmB, &tmC)) {
+    return cudaErrorInvalidValue;
+  }
   const int grid = 2 * pl.ctas;
   if (pr.f32_out)
     return pl.bn == 128 ? launch_pair<true, 128>(grid, tmA, tmB, tmC, gp, pr.pdl, st)

@@ -66,6 +66,10 @@ int gemm_ksplit(int T, int Ci, int Co);
 // workspace (0: every tile whole).  For tests and reports.
 int gemm_tail_split(int T, int Ci, int Co, size_t ws_bytes);
 
+// Tokens a tile of the pair kernel's swapped-operand plan holds for a shape
+// (0: the plan is not swapped).  For tests and reports.
+int gemm_swap_tokens(int T, int Ci, int Co, size_t ws_bytes);
+
 // Workspace bytes of a GEMM call (a multiple of 256).
 size_t gemm_workspace_bytes(int T, int Ci, int Co);
 

@@ -250,7 +250,11 @@ PTPC_API int ptpc_linear_fmt(const void *X_dev, int64_t ldx, const uint8_t *Wq_d
  *   PTPC_FORCE_PAIR_BN = 128 | 256       tile width of the prefill kernel,
  *   PTPC_FORCE_KSPLIT  = 1 | 2 | 4 | 8   CTAs per tile of the decode kernel,
  *   PTPC_FORCE_SPLIT_TAIL = 0 | 1        the prefill kernel's split tail off,
- *                                        or on wherever the workspace allows.
+ *                                        or on wherever the workspace allows,
+ *   PTPC_FORCE_SWAP    = 0 | 1           the prefill kernel's swapped operands
+ *                                        (weights as the 256-row operand,
+ *                                        tokens as the tile's columns) off, or
+ *                                        on for every prefill-kernel shape.
  * Each is honoured only where the forced choice is feasible for the shape;
  * results stay within the GEMM's tolerance under every choice.  For tuning
  * and tests, not for production.  Not thread-safe with concurrent GEMM calls
@@ -262,6 +266,15 @@ PTPC_API int ptpc_reload_tuning_overrides(void);
  * computed whole, else the number of CTA pairs that share each tile of the
  * last wave (split along K).  Launches nothing.  No counterpart on the page. */
 PTPC_API int ptpc_gemm_tail_split(int64_t T, int64_t Ci, int64_t Co, size_t ws_bytes);
+
+/* The operand order of the prefill GEMM's plan for a shape on the current
+ * device with ws_bytes of GEMM workspace: 0 if its tiles are 256 tokens x
+ * 128 or 256 channels (or the decode kernel runs the shape), else the number
+ * of tokens a tile holds when the operands are swapped (256 channels x that
+ * many tokens; a multiple of 32, at most 256, chosen so that the token tiles
+ * divide T evenly, e.g. 160 for T = 300).  Launches nothing.  No counterpart
+ * on the page. */
+PTPC_API int ptpc_gemm_swap_tokens(int64_t T, int64_t Ci, int64_t Co, size_t ws_bytes);
 
 /* ptpc_scaled_mm without a caller-provided workspace.  The page has no
  * counterpart: this exists for callers that cannot allocate device memory

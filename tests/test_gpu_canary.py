@@ -103,3 +103,38 @@ def test_naive_path_stays_in_bounds(ptpc, T, Ci, Co):
     ptpc.apply_scales(y.view(torch.float32, (T, Co)), xs, ws, out=out.view(torch.bfloat16, (T, Co)))
     out.check(f"naive step 2 {T}x{Ci}x{Co}")
     assert np.isfinite(out.view(torch.bfloat16, (T, Co)).float().cpu().numpy()).all()
+
+
+@pytest.mark.parametrize("T,Ci,Co,env", [
+    (33, 256, 1040, {"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_SWAP": "1"}),   # swapped, one ragged token tile
+    (300, 2048, 28672, {"PTPC_FORCE_SPLIT_TAIL": "1"}),                        # swapped with a split tail
+    (600, 512, 2064, {"PTPC_FORCE_SWAP": "1"}),
+])
+def test_swapped_gemm_stays_in_bounds(ptpc, monkeypatch, T, Ci, Co, env):
+    for k in ("PTPC_FORCE_SWAP", "PTPC_FORCE_KERNEL", "PTPC_FORCE_SPLIT_TAIL"):
+        monkeypatch.delenv(k, raising=False)
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    ptpc.reload_tuning_overrides()
+    try:
+        assert ptpc.gemm_swap_tokens(T, Ci, Co) > 0
+        X = to_dev_bf16(synthetic.make_x(synthetic.DECODE_70B, 0, T, Ci))
+        Wq_t, ws = ptpc.quantize_weights(to_dev_bf16(synthetic.random_bf16((Ci, Co), seed=T + Co, scale=0.02)))
+        Xq, xs = ptpc.quantize_activations(X)
+        need = ptpc.workspace_size(ptpc.OP_LINEAR, T, Ci, Co)
+        wsg = Guarded(need)
+        wsg.view(torch.uint8, (need,)).zero_()
+        ws_obj = ptpc.Workspace(0, "cuda")
+        ws_obj.buf = wsg.view(torch.uint8, (need,))
+        out = Guarded(T * Co * 2)
+        ptpc.scaled_mm(Xq, xs, Wq_t, ws, out=out.view(torch.bfloat16, (T, Co)), ws=ws_obj)
+        out.check(f"swapped scaled_mm out {T}x{Ci}x{Co}")
+        wsg.check(f"swapped scaled_mm workspace {T}x{Ci}x{Co}")
+        y = Guarded(T * Co * 4)
+        ptpc.unscaled_mm_f32(Xq, Wq_t, out=y.view(torch.float32, (T, Co)))
+        y.check(f"swapped fp32 GEMM out {T}x{Ci}x{Co}")
+        assert ptpc.device_status(ws_obj) == ptpc.OK
+    finally:
+        for k in env:
+            monkeypatch.delenv(k, raising=False)
+        ptpc.reload_tuning_overrides()

@@ -69,7 +69,7 @@ def test_llama8b_prefill_full(ptpc, layer):
     assert_gemm_close(g, r, L.name)
 
 
-@pytest.mark.parametrize("T", [1, 8, 32, 128, 200])
+@pytest.mark.parametrize("T", [1, 8, 32, 128, 192])
 @pytest.mark.parametrize("layer", [0, 1])
 def test_decode_full(ptpc, T, layer):
     w = synthetic.DECODE_70B
@@ -87,14 +87,23 @@ def test_decode_full(ptpc, T, layer):
     (4096, 1024, (8,)), (4096, 2048, (4, 8)), (4112, 2064, (4, 8)), (2048, 4096, (4,)), (1024, 8192, (2,)),
     (4112, 8192, (2,)), (1024, 10240, (1,)),
 ])
-@pytest.mark.parametrize("T", [1, 13, 77, 128, 160, 256])
-def test_decode_cluster_split(ptpc, T, Ci, Co, splits):
-    got_split = ptpc.gemm_ksplit(T, Ci, Co)
-    assert got_split in splits, f"{T}x{Ci}x{Co}: K split {got_split}, expected one of {splits}"
-    X = synthetic.with_edge_rows(synthetic.make_x(synthetic.DECODE_70B, 0, T, Ci), huge_bits=BIG_BF16)
-    W = synthetic.random_bf16((Ci, Co), seed=T * 7 + Ci + Co, scale=0.02)
-    g, r = run_pair(ptpc, X, W)
-    assert_gemm_close(g, r, f"decode {T}x{Ci}x{Co} split {got_split}")
+@pytest.mark.parametrize("T", [1, 13, 77, 128, 160, 192, 256])
+def test_decode_cluster_split(ptpc, monkeypatch, T, Ci, Co, splits):
+    # above T = 192 the plan takes the pair kernel: the decode kernel's largest
+    # token count (256) is reached through the override
+    if T > 192:
+        monkeypatch.setenv("PTPC_FORCE_KERNEL", "decode")
+    ptpc.reload_tuning_overrides()
+    try:
+        got_split = ptpc.gemm_ksplit(T, Ci, Co)
+        assert got_split in splits, f"{T}x{Ci}x{Co}: K split {got_split}, expected one of {splits}"
+        X = synthetic.with_edge_rows(synthetic.make_x(synthetic.DECODE_70B, 0, T, Ci), huge_bits=BIG_BF16)
+        W = synthetic.random_bf16((Ci, Co), seed=T * 7 + Ci + Co, scale=0.02)
+        g, r = run_pair(ptpc, X, W)
+        assert_gemm_close(g, r, f"decode {T}x{Ci}x{Co} split {got_split}")
+    finally:
+        monkeypatch.delenv("PTPC_FORCE_KERNEL", raising=False)
+        ptpc.reload_tuning_overrides()
 
 
 def test_decode_split_matches_naive_step1(ptpc):
@@ -166,7 +175,7 @@ def test_tuning_overrides(ptpc, monkeypatch):
     """PTPC_FORCE_KSPLIT / PTPC_FORCE_PAIR_BN / PTPC_FORCE_KERNEL change the
     plan (where feasible) and every forced plan still matches the oracle.  The
     library reads them once, so every change is followed by a reload."""
-    names = ("PTPC_FORCE_KSPLIT", "PTPC_FORCE_PAIR_BN", "PTPC_FORCE_KERNEL")
+    names = ("PTPC_FORCE_KSPLIT", "PTPC_FORCE_PAIR_BN", "PTPC_FORCE_KERNEL", "PTPC_FORCE_SWAP")
 
     def setenv(env):
         for k in names:
@@ -189,8 +198,10 @@ def test_tuning_overrides(ptpc, monkeypatch):
         assert ptpc.gemm_ksplit(T, Ci, Co) == 1
         X = synthetic.with_edge_rows(synthetic.make_x(synthetic.DECODE_70B, 0, 256, 1024), huge_bits=BIG_BF16)
         W = synthetic.random_bf16((1024, 2064), seed=17, scale=0.02)
-        cases = [({"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_PAIR_BN": "128"}, 100),
-                 ({"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_PAIR_BN": "256"}, 7),
+        cases = [({"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_PAIR_BN": "128", "PTPC_FORCE_SWAP": "0"}, 100),
+                 ({"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_PAIR_BN": "256", "PTPC_FORCE_SWAP": "0"}, 7),
+                 ({"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_SWAP": "1"}, 7),
+                 ({"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_SWAP": "1"}, 256),
                  ({"PTPC_FORCE_KERNEL": "decode"}, 256),
                  ({"PTPC_FORCE_KERNEL": "decode", "PTPC_FORCE_KSPLIT": "1"}, 64),
                  ({"PTPC_FORCE_KSPLIT": "2"}, 13)]
@@ -332,15 +343,29 @@ def test_linear_on_column_slice(ptpc):
     assert torch.equal(dense.view(torch.int16), out.view(torch.int16))
 
 
-@pytest.mark.parametrize("T,Ci,Co,fmt", [(256, 8192, 57344, "e4m3"), (300, 2048, 28672, "e4m3"),
-                                         (512, 4096, 10240, "e4m3"), (1000, 1024, 5120, "e4m3"),
-                                         (300, 2048, 28672, "e2m1"), (512, 4096, 10240, "e3m2")])
-def test_split_tail(ptpc, monkeypatch, T, Ci, Co, fmt):
+@pytest.mark.parametrize("T,Ci,Co,fmt,forced", [
+    (2048, 16384, 8192, "e4m3", False),                   # long K: split by the automatic plan
+    (256, 8192, 57344, "e4m3", True), (300, 2048, 28672, "e4m3", True),
+    (512, 4096, 10240, "e4m3", True), (1000, 1024, 5120, "e4m3", True),
+    (300, 2048, 28672, "e2m1", True), (512, 4096, 10240, "e3m2", True)])
+def test_split_tail(ptpc, monkeypatch, T, Ci, Co, fmt, forced):
     """Prefill shapes whose last wave of tiles is split along K over the GPU
     (partials through the workspace, distributed fixed-order reduction):
     parity with the oracle, agreement with the whole-tile plan, repeated
     calls on one workspace (its counters back at zero after each), no
-    timeout in the status word."""
+    timeout in the status word.  Short-K shapes take the split only when
+    PTPC_FORCE_SPLIT_TAIL=1 asks for it."""
+    if forced:
+        monkeypatch.setenv("PTPC_FORCE_SPLIT_TAIL", "1")
+    ptpc.reload_tuning_overrides()
+    try:
+        _split_tail_case(ptpc, monkeypatch, T, Ci, Co, fmt)
+    finally:
+        monkeypatch.delenv("PTPC_FORCE_SPLIT_TAIL", raising=False)
+        ptpc.reload_tuning_overrides()
+
+
+def _split_tail_case(ptpc, monkeypatch, T, Ci, Co, fmt):
     assert ptpc.gemm_tail_split(T, Ci, Co) >= 2, "shape does not exercise the split tail"
     X = synthetic.with_edge_rows(synthetic.make_x(synthetic.CHAIN_70B, 2, T, Ci), huge_bits=BIG_BF16)
     W = synthetic.make_w(synthetic.CHAIN_70B, 2, Ci, Co)
@@ -376,7 +401,103 @@ def test_split_tail(ptpc, monkeypatch, T, Ci, Co, fmt):
 
 
 def test_split_tail_needs_the_workspace(ptpc):
-    """With only the status word of workspace the same shape runs whole tiles."""
-    assert ptpc.gemm_tail_split(256, 8192, 57344) >= 2
-    assert ptpc.gemm_tail_split(256, 8192, 57344, ws_bytes=256) == 0
+    """With only the status word of workspace the same shape runs whole
+    tiles; short K and a mostly full last wave are not split."""
+    assert ptpc.gemm_tail_split(2048, 16384, 8192) >= 2
+    assert ptpc.gemm_tail_split(2048, 16384, 8192, ws_bytes=256) == 0
+    assert ptpc.gemm_tail_split(256, 8192, 57344) == 0        # K = 8192: not worth it
     assert ptpc.gemm_tail_split(8192, 8192, 57344) == 0       # last wave mostly full: no split
+
+
+def _set_tuning(ptpc, monkeypatch, env):
+    for k in ("PTPC_FORCE_SWAP", "PTPC_FORCE_SPLIT_TAIL", "PTPC_FORCE_KERNEL"):
+        monkeypatch.delenv(k, raising=False)
+    for k, v in env.items():
+        monkeypatch.setenv(k, v)
+    ptpc.reload_tuning_overrides()
+
+
+@pytest.mark.parametrize("T,Ci,Co,fmt,env,nt", [
+    (300, 8192, 10240, "e4m3", {}, 160),                          # 70B QKV at T = 300: chosen by the plan
+    (300, 1024, 1040, "e4m3", {"PTPC_FORCE_SWAP": "1"}, 160),     # channels end inside a 32-wide store box
+    (200, 512, 2064, "e4m3", {"PTPC_FORCE_SWAP": "1"}, 224),      # one token tile, 24 padded tokens
+    (33, 256, 1040, "e4m3", {"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_SWAP": "1"}, 64),
+    (600, 2048, 4096, "e4m3", {"PTPC_FORCE_SWAP": "1"}, 224),     # three token tiles
+    (400, 1024, 2064, "e2m3", {"PTPC_FORCE_SWAP": "1"}, 224),     # FP6 weights as the M operand
+    (300, 2048, 4096, "e2m1", {"PTPC_FORCE_SWAP": "1"}, 160),     # FP4 weights as the M operand
+])
+def test_swapped_operand_tiles(ptpc, monkeypatch, T, Ci, Co, fmt, env, nt):
+    """The prefill kernel with the weights as the 256-row MMA operand and the
+    tokens as the tile's columns (transposed epilogue): parity with the
+    oracle on every row, the same output from linear, agreement with the
+    unswapped plan, deterministic, no timeout."""
+    try:
+        _set_tuning(ptpc, monkeypatch, env)
+        assert ptpc.gemm_swap_tokens(T, Ci, Co) == nt
+        X = synthetic.with_edge_rows(synthetic.make_x(synthetic.CHAIN_70B, 0, T, Ci), huge_bits=BIG_BF16)
+        W = synthetic.make_w(synthetic.CHAIN_70B, 0, Ci, Co)
+        Xd = to_dev_bf16(X)
+        Wq, ws_ = ptpc.quantize_weights_fmt(to_dev_bf16(W), fmt)
+        Xq, xs = ptpc.quantize_activations(Xd)
+        wsp = ptpc.Workspace(ptpc.workspace_size(ptpc.OP_LINEAR, T, Ci, Co), "cuda")
+        a = ptpc.scaled_mm_fmt(Xq, xs, Wq, ws_, fmt, ws=wsp)
+        b = ptpc.scaled_mm_fmt(Xq, xs, Wq, ws_, fmt, ws=wsp)
+        lin = ptpc.linear_fmt(Xd, Wq, ws_, fmt, ws=wsp)
+        assert ptpc.device_status(wsp) == ptpc.OK
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+        assert torch.equal(a.view(torch.int16), lin.view(torch.int16))
+        rXq, rxs = oracle.quant_act(X)
+        assert np.array_equal(Xq.cpu().numpy(), rXq)
+        if fmt == "e4m3":
+            rWq, rws = oracle.quant_weight(W)
+            ref = oracle.scaled_mm_reference(rXq, rxs, rWq, rws)
+        else:
+            codes, rws = oracle.quant_weight_fmt(W, fmt)
+            ref = oracle.scaled_mm_reference_fmt(rXq, rxs, codes, rws, fmt)
+        assert_gemm_close(from_dev_bf16(a), ref, f"swapped {fmt} T={T} {Ci}->{Co}")
+        _set_tuning(ptpc, monkeypatch, {"PTPC_FORCE_SWAP": "0"})
+        assert ptpc.gemm_swap_tokens(T, Ci, Co) == 0
+        plain = ptpc.scaled_mm_fmt(Xq, xs, Wq, ws_, fmt, ws=wsp)
+        assert_gemm_close(from_dev_bf16(a), from_dev_bf16(plain), "swapped vs unswapped")
+    finally:
+        _set_tuning(ptpc, monkeypatch, {})
+
+
+@pytest.mark.parametrize("T,Ci,Co", [(300, 1024, 768), (77, 512, 1040)])
+def test_swapped_naive_path(ptpc, monkeypatch, T, Ci, Co):
+    """The fp32-output GEMM (the naive path's first step) with swapped
+    operands: its accumulator is the oracle's dot product up to fp32
+    accumulation, and scaling it afterwards gives the fused bits."""
+    try:
+        _set_tuning(ptpc, monkeypatch, {"PTPC_FORCE_KERNEL": "pair", "PTPC_FORCE_SWAP": "1"})
+        X = synthetic.make_x(synthetic.LLAMA8B_PREFILL, 0, T, Ci)
+        W = synthetic.make_w(synthetic.LLAMA8B_PREFILL, 0, Ci, Co)
+        Wq_t, ws = ptpc.quantize_weights(to_dev_bf16(W))
+        Xq, xs = ptpc.quantize_activations(to_dev_bf16(X))
+        fused = ptpc.scaled_mm(Xq, xs, Wq_t, ws)
+        y = ptpc.unscaled_mm_f32(Xq, Wq_t)
+        naive = ptpc.apply_scales(y, xs, ws)
+        assert torch.equal(fused.view(torch.int16), naive.view(torch.int16))
+        acc = oracle.gemm_acc64(Xq.cpu().numpy(), Wq_t.cpu().numpy())
+        yy = y.cpu().numpy().astype(np.float64)
+        rms = np.sqrt(np.mean(acc * acc))
+        assert (np.abs(yy - acc) <= 1e-2 * np.abs(acc) + 1e-3 * rms).all()
+    finally:
+        _set_tuning(ptpc, monkeypatch, {})
+
+
+@pytest.mark.parametrize("split", ["0", "1"])
+def test_swapped_70b_gate_up(ptpc, monkeypatch, split):
+    """The 70B gate+up layer at T = 300 takes swapped tiles (with and
+    without a split last wave); sampled rows against the oracle."""
+    T, Ci, Co = 300, 8192, 57344
+    try:
+        _set_tuning(ptpc, monkeypatch, {"PTPC_FORCE_SPLIT_TAIL": split})
+        assert ptpc.gemm_swap_tokens(T, Ci, Co) == 160
+        assert (ptpc.gemm_tail_split(T, Ci, Co) >= 2) == (split == "1")
+        rows = np.unique(np.concatenate([np.arange(0, T, 5), [T - 1]]))
+        w = synthetic.CHAIN_70B
+        g, r = run_pair(ptpc, synthetic.make_x(w, 2, T, Ci), synthetic.make_w(w, 2, Ci, Co), rows=rows)
+        assert_gemm_close(g, r, f"70B gate_up T=300 swapped, split tail {split}")
+    finally:
+        _set_tuning(ptpc, monkeypatch, {})
