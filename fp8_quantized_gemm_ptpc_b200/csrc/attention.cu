@@ -19,20 +19,22 @@
 // with asynchronous copies (cp.async, 16 bytes per copy, zero-filled for
 // positions that are not read) into a ring of three shared-memory stages, so
 // two tiles' bytes are in flight while it computes on a third.  The codes go
-// from shared memory straight into the registers of FlashAttention-style
-// tensor-core MMAs (mma.sync m16n8k16, f16 inputs, fp32 accumulation; the
-// GQA group's query heads are the 16 rows), converted exactly to f16 on the
-// way (cvt e4m3x2 -> f16x2: every E4M3 value is an f16 value).  To make that
-// possible the contraction over d in S = Q K^T runs in a permuted order (the
-// same for Q and K) in which each lane's codes of a position are contiguous,
-// and O's columns are ordered so that each lane's V codes of a position are
-// contiguous too; the two positions a V register pairs are joined by one byte
-// permute.  Online softmax in base 2; the key scales multiply the scores; the
-// value scales enter P relative to the largest value scale seen so far (so P
-// stays in [0, 1] in f16), and the accumulator is kept in units of it.  The
-// warps' states are combined in shared memory and every CTA writes (max, sum,
+// from shared memory straight into the registers of tensor-core MMAs
+// (mma.sync m16n8k16, f16 inputs, fp32 accumulation), converted exactly to
+// f16 on the way (cvt e4m3x2 -> f16x2: every E4M3 value is an f16 value).
+// Both products are taken transposed, S^T = K Q^T and O^T += V^T P^T, so the
+// GQA group's 8 query heads are the MMAs' N = 8 operand and no tensor work is
+// spent on padding rows; P moves between them by a register transpose.  The
+// contraction over d runs in a permuted order (the same for Q and K) in
+// which each lane's K codes of a position are contiguous, and the rows of O^T
+// are ordered so that each lane's V codes of a position are contiguous too.
+// Online softmax in base 2; the key scales multiply the scores; the value
+// scales enter P relative to the largest value scale seen so far (so P stays
+// in [0, 1] in f16), and the accumulator is kept in units of it.  The warps'
+// states are combined in shared memory and every CTA writes (max, sum,
 // accumulator) for its chunk; a second kernel combines the chunks and rounds
 // to bf16.
+#include <atomic>
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -128,19 +130,45 @@ __device__ __forceinline__ int code_off(int pos, int i) {
 __device__ __forceinline__ uint32_t lo16(uint32_t w) { return w & 0xFFFFu; }
 __device__ __forceinline__ uint32_t hi16(uint32_t w) { return w >> 16; }
 
-template <int D, int CHUNK>
-__global__ void __launch_bounds__(kAttnThreads, 3) decode_attn_kernel(const AttnParams p) {
+// Transpose of an 8x8 b16 matrix held as the warp's m8n8 fragment (lane i:
+// row i/4, columns 2(i%4), 2(i%4)+1).
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// The warp computes, per 16-position tile, S^T = K Q^T (M = 16 positions, N =
+// 8 query heads a head tile, K = d) and O^T += V^T P^T (M = 16 values of d,
+// N = 8 heads, K = 16 positions): with the GQA group's 8 heads as the N = 8
+// operand neither product carries padding rows.  Lane (g, c) = (lane / 4,
+// lane % 4).  In S^T it holds positions g and g + 8 for heads 2c, 2c+1, the
+// same heads whose columns it holds in O^T, so the softmax state and the
+// accumulator rescale stay in the lane; P goes from the S^T layout to the B
+// operand of O^T by one register transpose (movmatrix) per 8 x 8 block.
+// Orders that make every lane's code loads contiguous:
+//  * contraction over d in S^T: K step s, lane column c holds d = c*KB + 4s +
+//    {0, 1} (k = 2c, 2c+1) and c*KB + 4s + {2, 3} (k = 2c+8, 2c+9): a lane's
+//    K codes of a position are the KB bytes [c*KB, (c+1)*KB);
+//  * rows of O^T: row tile t, row g holds d = VB*g + 2t, row g + 8 holds
+//    d = VB*g + 2t + 1: a lane's V codes of a position are the VB bytes
+//    [VB*g, VB*(g+1)), and the two positions a register pairs are joined by
+//    one byte permute.
+// NH: head tiles of 8 (2 for groups of 9 to 16 heads).
+template <int D, int CHUNK, int NH>
+__global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 3) decode_attn_kernel(const AttnParams p) {
   using SM = AttnSmem<D, CHUNK>;
-  constexpr int KS = D / 16;        // 16-deep K steps of S = Q K^T
-  constexpr int NT = D / 8;         // 8-wide column tiles of O
-  constexpr int KB = D / 4;         // K code bytes a lane holds per position (its share of D)
+  constexpr int KS = D / 16;        // 16-deep K steps of S^T
+  constexpr int MT = D / 16;        // 16-row tiles of O^T
+  constexpr int KB = D / 4;         // K code bytes a lane holds per position
   constexpr int VB = D / 8;         // V code bytes a lane holds per position
   extern __shared__ __align__(16) uint8_t dsmem[];
   int *s_blk = reinterpret_cast<int *>(dsmem + SM::CODES);
   __shared__ float s_ml[kAttnWarps][16][2];
 
-  const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
   const int L = __ldg(p.context_lens + b);
   const int c0 = split * CHUNK;
   const int c1 = min(c0 + CHUNK, L);
@@ -171,7 +199,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) decode_attn_kernel(const Attn
       if (blk < 0 || slot >= p.num_slots) slot = -1;
     }
     const bool valid = slot >= 0;
-    const int64_t row = valid ? slot * p.Hkv + g : 0;
+    const int64_t row = valid ? slot * p.Hkv + kvh : 0;
     uint8_t *sk = ring + st * SM::STAGE;
     uint8_t *sv = sk + 16 * D;
     const uint8_t *gk = p.kc + row * D;
@@ -191,36 +219,37 @@ __global__ void __launch_bounds__(kAttnThreads, 3) decode_attn_kernel(const Attn
     if (lane == 0) *reinterpret_cast<uint32_t *>(sc + 32) = m;
   };
 
-  // Query fragments (A operand of S = Q K^T; rows = the group's heads, padded
-  // to 16).  The contraction over d is taken in a permuted order: in K step
-  // s, lane column c (lane & 3) holds d = c*KB + 4s + {0, 1} (logical k =
-  // 2c, 2c+1) and c*KB + 4s + {2, 3} (logical 2c+8, 2c+9), so that a lane's K
-  // codes for a position are the KB contiguous bytes [c*KB, (c+1)*KB).
-  const int r0 = lane >> 2, cq = lane & 3;
-  uint32_t qa[KS][4];
+  // Q^T fragments (B operand of S^T): head tile j, head 8j + g, K step s.
+  uint32_t qb[NH][KS][2];
   {
     const uint32_t *q32 = reinterpret_cast<const uint32_t *>(p.q);
-    const int64_t hrow0 = (int64_t)b * p.Hq + (int64_t)g * p.G;
+    const int64_t hrow0 = (int64_t)b * p.Hq + (int64_t)kvh * p.G;
     #pragma unroll
-    for (int kk = 0; kk < KS; ++kk) {
+    for (int j = 0; j < NH; ++j) {
+      const int h = 8 * j + g;
       #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int row = r0 + ((i & 1) ? 8 : 0);
-        const int col = cq * KB + 4 * kk + ((i & 2) ? 2 : 0);
-        qa[kk][i] = row < p.G ? bf16x2_to_f16x2(__ldg(q32 + ((hrow0 + row) * D + col) / 2)) : 0u;
+      for (int s = 0; s < KS; ++s) {
+        #pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int col = c * KB + 4 * s + 2 * i;
+          qb[j][s][i] = h < p.G ? bf16x2_to_f16x2(__ldg(q32 + ((hrow0 + h) * D + col) / 2)) : 0u;
+        }
       }
     }
   }
 
-  // The accumulator is kept in units of `unit`, the largest value scale seen
-  // so far (O = acc * unit); column tile n, columns 2cq, 2cq+1 hold
-  // d = VB*(2cq) + n and VB*(2cq+1) + n (the V operand's d order: lane row r0
-  // holds d = VB*r0 + n, so its V codes for a position are the VB contiguous
-  // bytes [VB*r0, VB*(r0+1))).
-  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.0f, 0.0f}, unit = 0.0f;
-  float acc[NT][4];
+  // Softmax state of heads 8j + 2c + e (e = 0, 1), and the accumulator, kept
+  // in units of `unit`, the largest value scale seen so far (O = acc * unit).
+  float m_h[NH][2], l_h[NH][2];
+  float acc[NH][MT][4];
   #pragma unroll
-  for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.0f;
+  for (int j = 0; j < NH; ++j) {
+    m_h[j][0] = m_h[j][1] = -INFINITY;
+    l_h[j][0] = l_h[j][1] = 0.0f;
+    #pragma unroll
+    for (int t = 0; t < MT; ++t) acc[j][t][0] = acc[j][t][1] = acc[j][t][2] = acc[j][t][3] = 0.0f;
+  }
+  float unit = 0.0f;
 
   constexpr int STEP = kAttnWarps * 16;
   const int first = c0 + warp * 16;
@@ -246,139 +275,127 @@ __global__ void __launch_bounds__(kAttnThreads, 3) decode_attn_kernel(const Attn
     const float *vsc = ksc + 16;
     const uint32_t vmask = *reinterpret_cast<const uint32_t *>(ksc + 32);
 
-    // S = Q K^T: column tile j holds positions 8j .. 8j+7 (B operand: lane
-    // row r0 = position 8j + r0, its KB code bytes)
-    float s[2][4];
-    #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int pos = 8 * j + r0;
-      uint32_t kw[KB / 4];
-      #pragma unroll
-      for (int i = 0; i < KB / 16; ++i) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(sk + code_off<D>(pos, cq * (KB / 16) + i));
-        kw[4 * i] = v.x;
-        kw[4 * i + 1] = v.y;
-        kw[4 * i + 2] = v.z;
-        kw[4 * i + 3] = v.w;
-      }
-      s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
-      #pragma unroll
-      for (int kk = 0; kk < KS; ++kk)
-        mma_f16(s[j], qa[kk], e4m3x2_to_f16x2(lo16(kw[kk])), e4m3x2_to_f16x2(hi16(kw[kk])));
-    }
-
-    // this lane's positions: 2cq, 2cq+1 (column tile 0) and 2cq+8, 2cq+9 (tile 1)
-    const float2 ks01 = *reinterpret_cast<const float2 *>(ksc + 2 * cq);
-    const float2 ks89 = *reinterpret_cast<const float2 *>(ksc + 2 * cq + 8);
-    const float2 vs01 = *reinterpret_cast<const float2 *>(vsc + 2 * cq);
-    const float2 vs89 = *reinterpret_cast<const float2 *>(vsc + 2 * cq + 8);
-    const float kscl[2][2] = {{ks01.x, ks01.y}, {ks89.x, ks89.y}};
-    const float vscl[2][2] = {{vs01.x, vs01.y}, {vs89.x, vs89.y}};
-    bool ok[2][2];
-    float vmax = 0.0f;
-    #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        ok[j][e] = (vmask >> (2 * (8 * j + 2 * cq + e))) & 1u;
-        if (ok[j][e]) vmax = fmaxf(vmax, vscl[j][e]);
-      }
-    }
-    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 1));
-    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 2));
-
-    // key scales, masking, online softmax (rows r0 and r0 + 8)
-    float mx[2] = {-INFINITY, -INFINITY};
-    #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float k2 = kscl[j][e] * p.scale_log2;
-        s[j][e] = ok[j][e] ? s[j][e] * k2 : -INFINITY;
-        s[j][2 + e] = ok[j][e] ? s[j][2 + e] * k2 : -INFINITY;
-        mx[0] = fmaxf(mx[0], s[j][e]);
-        mx[1] = fmaxf(mx[1], s[j][2 + e]);
-      }
-    }
-    float alpha[2], psum[2] = {0.0f, 0.0f};
+    // S^T = K Q^T (A = K: rows g, g + 8 = positions)
+    uint32_t kw[2][KB / 4];
     #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
-      mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
-      const float m_new = fmaxf(m_r[r], mx[r]);
-      // a tile with no readable position leaves the state as it is
-      alpha[r] = m_new == -INFINITY ? 1.0f : exp2f(m_r[r] - m_new);
-      m_r[r] = m_new;
+      const int pos = g + 8 * r;
+      #pragma unroll
+      for (int i = 0; i < KB / 16; ++i) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(sk + code_off<D>(pos, c * (KB / 16) + i));
+        kw[r][4 * i] = v.x;
+        kw[r][4 * i + 1] = v.y;
+        kw[r][4 * i + 2] = v.z;
+        kw[r][4 * i + 3] = v.w;
+      }
     }
+    float s[NH][4];
+    #pragma unroll
+    for (int j = 0; j < NH; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
+    #pragma unroll
+    for (int k = 0; k < KS; ++k) {
+      const uint32_t a[4] = {e4m3x2_to_f16x2(lo16(kw[0][k])), e4m3x2_to_f16x2(lo16(kw[1][k])),
+                             e4m3x2_to_f16x2(hi16(kw[0][k])), e4m3x2_to_f16x2(hi16(kw[1][k]))};
+      #pragma unroll
+      for (int j = 0; j < NH; ++j) mma_f16(s[j], a, qb[j][k][0], qb[j][k][1]);
+    }
+
+    // this lane's positions g (s[.][0..1]) and g + 8 (s[.][2..3])
+    const bool ok0 = (vmask >> (2 * g)) & 1u, ok8 = (vmask >> (2 * (g + 8))) & 1u;
+    const float k0 = ksc[g] * p.scale_log2, k8 = ksc[g + 8] * p.scale_log2;
+    const float v0 = ok0 ? vsc[g] : 0.0f, v8 = ok8 ? vsc[g + 8] : 0.0f;
+    float vmax = fmaxf(v0, v8);
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 4));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 8));
+    vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, 16));
     // the unit grows to this tile's largest value scale where that is larger
     const float new_unit = fmaxf(unit, vmax);
     const float to_unit = new_unit > unit && unit > 0.0f ? __fdividef(unit, new_unit) : 1.0f;
     unit = new_unit;
     const float inv_unit = unit > 0.0f ? __fdividef(1.0f, unit) : 0.0f;
-    uint32_t pa[4];
+    const float vr0 = v0 * inv_unit, vr8 = v8 * inv_unit;
+
+    uint32_t pb[NH][2];
+    bool rescale = false;
+    float alpha[NH][2];
     #pragma unroll
-    for (int j = 0; j < 2; ++j) {
+    for (int j = 0; j < NH; ++j) {
+      // key scales and masking
+      s[j][0] = ok0 ? s[j][0] * k0 : -INFINITY;
+      s[j][1] = ok0 ? s[j][1] * k0 : -INFINITY;
+      s[j][2] = ok8 ? s[j][2] * k8 : -INFINITY;
+      s[j][3] = ok8 ? s[j][3] * k8 : -INFINITY;
       float pv[4];
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const float vr = vscl[j][e] * inv_unit;   // this position's value scale / the unit
-        const float p0 = m_r[0] == -INFINITY ? 0.0f : exp2f(s[j][e] - m_r[0]);
-        const float p1 = m_r[1] == -INFINITY ? 0.0f : exp2f(s[j][2 + e] - m_r[1]);
-        psum[0] += p0;
-        psum[1] += p1;
-        pv[e] = p0 * vr;
-        pv[2 + e] = p1 * vr;
+        // head 8j + 2c + e: its largest score of the tile over the 16 positions
+        float mx = fmaxf(s[j][e], s[j][2 + e]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float m_new = fmaxf(m_h[j][e], mx);
+        // a tile with no readable position leaves the state as it is
+        alpha[j][e] = m_new == -INFINITY ? 1.0f : exp2f(m_h[j][e] - m_new);
+        m_h[j][e] = m_new;
+        const float p0 = m_new == -INFINITY ? 0.0f : exp2f(s[j][e] - m_new);
+        const float p8 = m_new == -INFINITY ? 0.0f : exp2f(s[j][2 + e] - m_new);
+        float ps = p0 + p8;
+        ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+        l_h[j][e] = l_h[j][e] * alpha[j][e] + ps;
+        alpha[j][e] *= to_unit;
+        rescale |= alpha[j][e] != 1.0f;
+        pv[e] = p0 * vr0;
+        pv[2 + e] = p8 * vr8;
       }
-      pa[2 * j] = h2_bits(__floats2half2_rn(pv[0], pv[1]));       // row r0, positions 8j + 2cq, +1
-      pa[2 * j + 1] = h2_bits(__floats2half2_rn(pv[2], pv[3]));   // row r0 + 8
-    }
-    #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      psum[r] += __shfl_xor_sync(0xffffffffu, psum[r], 1);
-      psum[r] += __shfl_xor_sync(0xffffffffu, psum[r], 2);
-      l_r[r] = l_r[r] * alpha[r] + psum[r];
-      alpha[r] *= to_unit;
+      // P' of positions 0..7 and 8..15 as 8 x 8 blocks (row = position,
+      // columns = heads 2c, 2c+1), transposed into the B operand of O^T
+      // (k = positions 2c, 2c+1 and 2c+8, 2c+9, n = head g)
+      pb[j][0] = movmatrix_trans(h2_bits(__floats2half2_rn(pv[0], pv[1])));
+      pb[j][1] = movmatrix_trans(h2_bits(__floats2half2_rn(pv[2], pv[3])));
     }
     // rescale the accumulator only where a factor differs from one
-    if (__any_sync(0xffffffffu, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
+    if (__any_sync(0xffffffffu, rescale)) {
       #pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        acc[n][0] *= alpha[0];
-        acc[n][1] *= alpha[0];
-        acc[n][2] *= alpha[1];
-        acc[n][3] *= alpha[1];
+      for (int j = 0; j < NH; ++j) {
+        #pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          acc[j][t][0] *= alpha[j][0];
+          acc[j][t][1] *= alpha[j][1];
+          acc[j][t][2] *= alpha[j][0];
+          acc[j][t][3] *= alpha[j][1];
+        }
       }
     }
 
-    // O += P V.  A = P (rows r0 / r0 + 8; k = positions 2cq, 2cq+1 and
-    // 2cq+8, 2cq+9); B = V (k = those positions, n = d of column tile n):
-    // lane row r0 holds d = VB*r0 + n, so the two codes of a B register (two
-    // positions, one d) are byte n of two positions' VB-byte runs, paired
-    // with a byte permute before the conversion.
-    const uint32_t a[4] = {pa[0], pa[1], pa[2], pa[3]};
+    // O^T += V^T P'^T (A = V^T: rows = d, k = positions 2c, 2c+1, 2c+8, 2c+9)
     uint32_t vw[4][VB / 4];
     #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const int pos = 2 * cq + (q & 1) + ((q & 2) ? 8 : 0);
+      const int pos = 2 * c + (q & 1) + ((q & 2) ? 8 : 0);
       if constexpr (VB == 16) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(sv + code_off<D>(pos, r0));
+        const uint4 v = *reinterpret_cast<const uint4 *>(sv + code_off<D>(pos, g));
         vw[q][0] = v.x;
         vw[q][1] = v.y;
         vw[q][2] = v.z;
         vw[q][3] = v.w;
       } else {
-        const uint2 v = *reinterpret_cast<const uint2 *>(sv + code_off<D>(pos, r0 >> 1) + 8 * (r0 & 1));
+        const uint2 v = *reinterpret_cast<const uint2 *>(sv + code_off<D>(pos, g >> 1) + 8 * (g & 1));
         vw[q][0] = v.x;
         vw[q][1] = v.y;
       }
     }
     #pragma unroll
-    for (int n = 0; n < NT; n += 2) {
-      const uint32_t sel = (n & 2) ? 0x7362u : 0x5140u;
-      const uint32_t x01 = __byte_perm(vw[0][n >> 2], vw[1][n >> 2], sel);   // positions 2cq, 2cq+1
-      const uint32_t x89 = __byte_perm(vw[2][n >> 2], vw[3][n >> 2], sel);   // positions 2cq+8, 2cq+9
-      mma_f16(acc[n], a, e4m3x2_to_f16x2(lo16(x01)), e4m3x2_to_f16x2(lo16(x89)));
-      mma_f16(acc[n + 1], a, e4m3x2_to_f16x2(hi16(x01)), e4m3x2_to_f16x2(hi16(x89)));
+    for (int t = 0; t < MT; ++t) {
+      // bytes 2t (row g) and 2t + 1 (row g + 8) of the lane's run
+      const uint32_t sel = (t & 1) ? 0x7362u : 0x5140u;
+      const uint32_t x01 = __byte_perm(vw[0][t >> 1], vw[1][t >> 1], sel);   // positions 2c, 2c+1
+      const uint32_t x89 = __byte_perm(vw[2][t >> 1], vw[3][t >> 1], sel);   // positions 2c+8, 2c+9
+      const uint32_t a[4] = {e4m3x2_to_f16x2(lo16(x01)), e4m3x2_to_f16x2(hi16(x01)),
+                             e4m3x2_to_f16x2(lo16(x89)), e4m3x2_to_f16x2(hi16(x89))};
+      #pragma unroll
+      for (int j = 0; j < NH; ++j) mma_f16(acc[j][t], a, pb[j][0], pb[j][1]);
     }
     __syncwarp();  // this stage is refilled two tiles later
     if (++st == kAttnStages) st = 0;
@@ -386,23 +403,30 @@ __global__ void __launch_bounds__(kAttnThreads, 3) decode_attn_kernel(const Attn
   cp_async_wait<0>();
 
   // combine the four warps' states (each accumulator times its unit)
-  if (cq == 0) {
-    s_ml[warp][r0][0] = m_r[0];
-    s_ml[warp][r0][1] = l_r[0];
-    s_ml[warp][r0 + 8][0] = m_r[1];
-    s_ml[warp][r0 + 8][1] = l_r[1];
+  if (g == 0) {
+    #pragma unroll
+    for (int j = 0; j < NH; ++j) {
+      #pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        s_ml[warp][8 * j + 2 * c + e][0] = m_h[j][e];
+        s_ml[warp][8 * j + 2 * c + e][1] = l_h[j][e];
+      }
+    }
   }
   __syncthreads();  // every warp has finished with its ring: the buffer is free
-  float *s_acc = reinterpret_cast<float *>(dsmem);   // [warp][16][D]
+  float *s_acc = reinterpret_cast<float *>(dsmem);   // [warp][16 heads][D]
   #pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    const int d0 = VB * (2 * cq) + n, d1 = VB * (2 * cq + 1) + n;
-    float *row0 = s_acc + ((size_t)warp * 16 + r0) * D;
-    float *row1 = s_acc + ((size_t)warp * 16 + r0 + 8) * D;
-    row0[d0] = acc[n][0] * unit;
-    row0[d1] = acc[n][1] * unit;
-    row1[d0] = acc[n][2] * unit;
-    row1[d1] = acc[n][3] * unit;
+  for (int j = 0; j < NH; ++j) {
+    #pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      const int d0 = VB * g + 2 * t, d8 = d0 + 1;
+      float *h0 = s_acc + ((size_t)warp * 16 + 8 * j + 2 * c) * D;
+      float *h1 = h0 + D;
+      h0[d0] = acc[j][t][0] * unit;
+      h1[d0] = acc[j][t][1] * unit;
+      h0[d8] = acc[j][t][2] * unit;
+      h1[d8] = acc[j][t][3] * unit;
+    }
   }
   __syncthreads();
   for (int i = threadIdx.x; i < p.G * D; i += kAttnThreads) {
@@ -419,7 +443,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) decode_attn_kernel(const Attn
         o += s_acc[((size_t)w * 16 + h) * D + d] * f;
       }
     }
-    const int64_t idx = (((int64_t)b * p.Hq + (int64_t)g * p.G + h) * p.splits + split);
+    const int64_t idx = (((int64_t)b * p.Hq + (int64_t)kvh * p.G + h) * p.splits + split);
     p.part_acc[idx * D + d] = o;
     if (d == 0) {
       p.part_ml[idx * 2] = m;
@@ -451,19 +475,19 @@ __global__ void __launch_bounds__(D) decode_attn_combine_kernel(const float *__r
 
 constexpr int kAttnChunk = 512;
 
-template <int D>
+template <int D, int NH>
 cudaError_t launch_attn(const AttnParams &p, int B, __nv_bfloat16 *out, cudaStream_t st) {
   const size_t smem = AttnSmem<D, kAttnChunk>::BYTES;
-  static bool attr_set[64] = {};
+  static std::atomic<bool> attr_set[64];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t a = cudaFuncSetAttribute(decode_attn_kernel<D, kAttnChunk>,
+  if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
+    cudaError_t a = cudaFuncSetAttribute(decode_attn_kernel<D, kAttnChunk, NH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (a != cudaSuccess) return a;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
-  decode_attn_kernel<D, kAttnChunk><<<dim3(p.splits, p.Hkv, B), kAttnThreads, smem, st>>>(p);
+  decode_attn_kernel<D, kAttnChunk, NH><<<dim3(p.splits, p.Hkv, B), kAttnThreads, smem, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -513,8 +537,8 @@ cudaError_t launch_decode_attention(const void *q, const uint8_t *kc, const uint
   p.part_ml = static_cast<float *>(ws);
   p.part_acc = static_cast<float *>(ws) + n * 2;
   __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
-  if (D == 64) return launch_attn<64>(p, B, o, st);
-  if (D == 128) return launch_attn<128>(p, B, o, st);
+  if (D == 64) return p.G > 8 ? launch_attn<64, 2>(p, B, o, st) : launch_attn<64, 1>(p, B, o, st);
+  if (D == 128) return p.G > 8 ? launch_attn<128, 2>(p, B, o, st) : launch_attn<128, 1>(p, B, o, st);
   return cudaErrorInvalidValue;
 }
 

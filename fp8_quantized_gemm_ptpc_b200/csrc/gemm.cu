@@ -266,7 +266,6 @@ constexpr int kDecMaxStages = 16;
 constexpr int kDecWBytes = BM * BK;   // weight tile of one stage
 constexpr size_t kDecBarBytes = 512;  // barriers and flags after the ring
 constexpr size_t kDecSmemMax = 232448;
-constexpr int kDecPrefetchBytes = 192 * 1024;  // weight bytes an SM prefetches into L2 ahead of its loads
 
 __host__ __device__ constexpr size_t dec_smem_bytes(int np, int stages) {
   return 1024 + (size_t)stages * (kDecWBytes + (size_t)np * BK) + kDecBarBytes;
@@ -441,28 +440,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       Sched sc;
       Unit u;
-      // L2 prefetch of the weight tiles kDecPrefetchBytes ahead of the loads
-      // (a second walk of the same schedule): the ring holds the weights
-      // unpacked, so a sub-byte format keeps only half (FP4) or 3/4 (FP6) of
-      // the ring's bytes in flight from HBM; with the tiles already in L2 the
-      // ring's loads return sooner and the SM's stream keeps up.
-      Sched sa;
-      Unit ua;
-      sa.init(p, blockIdx.x, gridDim.x);
-      bool more_a = sa.next(p, ua);
-      int kba = ua.kb0;
-      auto advance_a = [&]() {
-        if (more_a && ++kba >= ua.kb1) {
-          more_a = sa.next(p, ua);
-          kba = ua.kb0;
-        }
-      };
-      const int pf_ahead = kDecPrefetchBytes / (kDecWBytes * wf_bits(WF) / 8);
-      for (int i = 0; i < pf_ahead; ++i) advance_a();
-      auto prefetch_next = [&]() {
-        if (more_a) tma_prefetch_2d(&tmW, kba * BK, ua.n * BM);
-        advance_a();
-      };
       // The weights never depend on the kernel launched just before this one:
       // the first stages' weight tiles are requested before waiting for it.
       int pre = 0;
@@ -471,7 +448,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (; pre < STAGES && u.kb0 + pre < u.kb1; ++pre) {
           mbar_arrive_expect_tx(&full[pre], stage_tx);
           tma_load_2d(sW + pre * kDecWBytes, &tmW, &full[pre], (u.kb0 + pre) * BK, u.n * BM, polW);
-          prefetch_next();
         }
       }
       griddep_wait();  // Xq may come from the kernel launched just before
@@ -486,7 +462,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             mbar_arrive_expect_tx(&full[stage], stage_tx);
             tma_load_2d(sW + stage * kDecWBytes, &tmW, &full[stage], kb * BK, u.n * BM, polW);
-            prefetch_next();
           }
           tma_load_2d(sX + stage * X_BYTES, &tmX, &full[stage], kb * BK, 0, polX);
           if (++stage == STAGES) {

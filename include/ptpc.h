@@ -155,14 +155,17 @@ PTPC_API int ptpc_quantize_weights(const void *W_dev, int64_t Ci, int64_t Co,
  *               device status word and, for prefill-sized T, room for the
  *               split tail (below), about 19 MB.
  * The sum over k is an fp32 tensor-core accumulation; its order is not
- * specified.  For T <= 256 and few output tiles, K is split over a cluster of
+ * specified.  For T <= 192 and few output tiles, K is split over a cluster of
  * 2, 4 or 8 CTAs (see ptpc_gemm_ksplit) whose fp32 partial sums are added in
- * a fixed order.  For prefill-sized T whose last wave of output tiles would
- * keep at most half the SMs busy, those tiles are split along K over the
- * whole GPU (see ptpc_gemm_tail_split): their fp32 partial sums go through
- * the workspace and are added in a fixed order.  Results are deterministic
- * for a given shape and workspace size.  With a smaller workspace (at least
- * the status word) every tile is computed whole. */
+ * a fixed order.  For prefill-sized T with a long K (at least 16384) whose
+ * last wave of output tiles would keep at most half the SMs busy, those
+ * tiles are split along K over the whole GPU (see ptpc_gemm_tail_split):
+ * their fp32 partial sums go through the workspace and are added in a fixed
+ * order.  Ragged prefill T may run with the operands swapped (see
+ * ptpc_gemm_swap_tokens); the products and their accumulation are the same
+ * kind, only the tiling differs.  Results are deterministic for a given
+ * shape and workspace size.  With a smaller workspace (at least the status
+ * word) every tile is computed whole. */
 PTPC_API int ptpc_scaled_mm(const uint8_t *Xq_dev, const float *x_scale_dev,
                    const uint8_t *Wq_t_dev, const float *w_scale_dev,
                    int64_t T, int64_t Ci, int64_t Co, void *out_dev,
