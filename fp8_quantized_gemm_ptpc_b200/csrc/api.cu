@@ -348,7 +348,7 @@ int ptpc_decode_attention(const void *q, const uint8_t *k_cache, const uint8_t *
   if (s != PTPC_OK) return s;
   if (B < 0 || Hq <= 0 || max_blocks <= 0 || max_context < 0) return PTPC_ERR_INVALID_ARG;
   if (Hq % Hkv != 0 || Hq / Hkv > 16 || B > 65535 || Hkv > 65535 || max_context > kMaxDim ||
-      max_blocks > kMaxDim / block_size)
+      max_blocks > kMaxDim / block_size || num_blocks > kMaxDim / block_size)
     return PTPC_ERR_UNSUPPORTED_SHAPE;
   if (B == 0) return PTPC_OK;
   if (!q || !k_cache || !v_cache || !k_scale || !v_scale || !block_tables || !context_lens || !out || !ws)

@@ -65,12 +65,6 @@ struct AttnParams {
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 v) { return *reinterpret_cast<uint32_t *>(&v); }
 
-// Two bf16 (low half first) -> two f16: exact for magnitudes in f16's range.
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
-  const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w));
-  return h2_bits(__floats2half2_rn(f.x, f.y));
-}
-
 // Two E4M3 codes (low byte first) -> two f16 (exact).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
   const __half2_raw r = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)two_codes, __NV_E4M3);
@@ -84,6 +78,25 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// D (16x8 fp32) += A (16x32 e4m3, row) * B (32x8 e4m3, col); four codes a register.
+__device__ __forceinline__ void mma_e4m3(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two floats -> two E4M3 codes (low byte first), round to nearest even, saturating.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
+}
+
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t two_codes) {
+  const uint32_t h = e4m3x2_to_f16x2(two_codes);
+  return __half22float2(*reinterpret_cast<const __half2 *>(&h));
 }
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
@@ -100,12 +113,12 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-constexpr int kMinBlockSize = 8;   // the chunk's block-table entries fit in shared memory
 constexpr int kAttnStages = 3;     // code stages a warp keeps in flight (two tiles ahead)
 
 // Shared memory of one CTA: every warp's ring of code stages (K and V codes of
 // 16 positions, their scales and the tile's validity mask), which at the end
-// doubles as the warps' accumulators, and the chunk's block-table entries.
+// doubles as the warps' accumulators, and the cache slot of every position of
+// the chunk.
 // A position's D code bytes are stored as D/16 16-byte chunks, chunk i at
 // chunk index i ^ (position mod D/16), so that the fragment loads below hit
 // distinct shared-memory banks.
@@ -115,8 +128,8 @@ struct AttnSmem {
   static constexpr int STAGE = CODES_TILE + 2 * 16 * 4 + 16;          // + k, v scales + validity mask
   static constexpr int RING = kAttnStages * STAGE;
   static constexpr int CODES = kAttnWarps * RING;
-  static constexpr int BLOCKS = (CHUNK / kMinBlockSize + 2) * 4;
-  static constexpr size_t BYTES = (size_t)CODES + BLOCKS;
+  static constexpr int SLOTS = CHUNK * 4;
+  static constexpr size_t BYTES = (size_t)CODES + SLOTS;
   static_assert(kAttnWarps * 16 * D * 4 <= CODES, "combine buffer");
   static_assert(STAGE % 16 == 0, "stage alignment");
 };
@@ -141,29 +154,37 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 // The warp computes, per 16-position tile, S^T = K Q^T (M = 16 positions, N =
 // 8 query heads a head tile, K = d) and O^T += V^T P^T (M = 16 values of d,
 // N = 8 heads, K = 16 positions): with the GQA group's 8 heads as the N = 8
-// operand neither product carries padding rows.  Lane (g, c) = (lane / 4,
+// operand neither product carries padding rows.  S^T is an E4M3 x E4M3 MMA
+// (m16n8k32) that takes the K codes as they are, with no conversion: each
+// head's q is scaled by a power of two sigma (the largest with max |q| sigma
+// <= 448) and written as two E4M3 terms, q sigma = hi + lo / 16 (hi rounded
+// to nearest, lo the rounded remainder times 16); a bf16 q has 8 significant
+// bits and each term 4, so the pair holds it exactly wherever hi is a normal
+// number, and S^T = (K hi + (K lo) / 16) / sigma with each product exact and
+// fp32 accumulation.  O^T stays an f16 MMA (P needs more than 4 bits).  Lane (g, c) = (lane / 4,
 // lane % 4).  In S^T it holds positions g and g + 8 for heads 2c, 2c+1, the
 // same heads whose columns it holds in O^T, so the softmax state and the
 // accumulator rescale stay in the lane; P goes from the S^T layout to the B
 // operand of O^T by one register transpose (movmatrix) per 8 x 8 block.
 // Orders that make every lane's code loads contiguous:
-//  * contraction over d in S^T: K step s, lane column c holds d = c*KB + 4s +
-//    {0, 1} (k = 2c, 2c+1) and c*KB + 4s + {2, 3} (k = 2c+8, 2c+9): a lane's
-//    K codes of a position are the KB bytes [c*KB, (c+1)*KB);
+//  * contraction over d in S^T: 32-deep K step s, lane column c holds d =
+//    c*KB + 8s + {0..3} (k = 4c .. 4c+3) and c*KB + 8s + {4..7} (k = 16+4c ..
+//    16+4c+3): a lane's K codes of a position are the KB bytes [c*KB,
+//    (c+1)*KB), four codes a register;
 //  * rows of O^T: row tile t, row g holds d = VB*g + 2t, row g + 8 holds
 //    d = VB*g + 2t + 1: a lane's V codes of a position are the VB bytes
 //    [VB*g, VB*(g+1)), and the two positions a register pairs are joined by
 //    one byte permute.
 // NH: head tiles of 8 (2 for groups of 9 to 16 heads).
 template <int D, int CHUNK, int NH>
-__global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 3) decode_attn_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 2) decode_attn_kernel(const AttnParams p) {
   using SM = AttnSmem<D, CHUNK>;
-  constexpr int KS = D / 16;        // 16-deep K steps of S^T
+  constexpr int KS = D / 32;        // 32-deep K steps of S^T
   constexpr int MT = D / 16;        // 16-row tiles of O^T
   constexpr int KB = D / 4;         // K code bytes a lane holds per position
   constexpr int VB = D / 8;         // V code bytes a lane holds per position
   extern __shared__ __align__(16) uint8_t dsmem[];
-  int *s_blk = reinterpret_cast<int *>(dsmem + SM::CODES);
+  int *s_slot = reinterpret_cast<int *>(dsmem + SM::CODES);
   __shared__ float s_ml[kAttnWarps][16][2];
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -173,12 +194,19 @@ __global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 3) decode_attn_ker
   const int c0 = split * CHUNK;
   const int c1 = min(c0 + CHUNK, L);
 
-  // the chunk's block-table entries (-1 where there is none)
-  const int bi0 = c0 / p.block_size;
-  const int nbi = c1 > c0 ? (c1 - 1) / p.block_size - bi0 + 1 : 0;
-  for (int i = threadIdx.x; i < nbi; i += kAttnThreads) {
-    const int bi = bi0 + i;
-    s_blk[i] = bi < p.max_blocks ? __ldg(p.block_tables + (int64_t)b * p.max_blocks + bi) : -1;
+  // the cache slot of every position of the chunk, -1 where it is not read
+  // (past the context, no block-table entry, block outside the cache; the
+  // cache has fewer than 2^31 slots)
+  for (int i = threadIdx.x; i < CHUNK; i += kAttnThreads) {
+    const int pos = c0 + i;
+    int slot = -1;
+    if (pos < c1) {
+      const int bi = pos / p.block_size;
+      const int blk = bi < p.max_blocks ? __ldg(p.block_tables + (int64_t)b * p.max_blocks + bi) : -1;
+      const int64_t sl = (int64_t)blk * p.block_size + pos % p.block_size;
+      if (blk >= 0 && sl < p.num_slots) slot = (int)sl;
+    }
+    s_slot[i] = slot;
   }
   __syncthreads();
 
@@ -191,15 +219,9 @@ __global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 3) decode_attn_ker
   // zero-filled and masked.
   auto prefetch = [&](int base, int st) {
     const int kk = lane >> 1, half = lane & 1;
-    const int pos = base + kk;
-    int64_t slot = -1;
-    if (pos < c1) {
-      const int blk = s_blk[pos / p.block_size - bi0];
-      slot = (int64_t)blk * p.block_size + pos % p.block_size;
-      if (blk < 0 || slot >= p.num_slots) slot = -1;
-    }
+    const int slot = s_slot[base - c0 + kk];
     const bool valid = slot >= 0;
-    const int64_t row = valid ? slot * p.Hkv + kvh : 0;
+    const int64_t row = valid ? (int64_t)slot * p.Hkv + kvh : 0;
     uint8_t *sk = ring + st * SM::STAGE;
     uint8_t *sv = sk + 16 * D;
     const uint8_t *gk = p.kc + row * D;
@@ -219,22 +241,61 @@ __global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 3) decode_attn_ker
     if (lane == 0) *reinterpret_cast<uint32_t *>(sc + 32) = m;
   };
 
-  // Q^T fragments (B operand of S^T): head tile j, head 8j + g, K step s.
-  uint32_t qb[NH][KS][2];
+  // Q^T fragments (B operand of S^T) as two E4M3 terms: head tile j, head
+  // 8j + g, K step s, registers b0 (d = c*KB + 8s + 0..3) and b1 (+ 4..7).
+  // inv_sig[j][e]: 1 / sigma of head 8j + 2c + e (the heads of this lane's
+  // S^T columns).
+  uint32_t qh[NH][KS][2], ql[NH][KS][2];
+  float inv_sig[NH][2];
   {
-    const uint32_t *q32 = reinterpret_cast<const uint32_t *>(p.q);
+    const uint2 *q64 = reinterpret_cast<const uint2 *>(p.q);   // 4 bf16 a load
     const int64_t hrow0 = (int64_t)b * p.Hq + (int64_t)kvh * p.G;
     #pragma unroll
     for (int j = 0; j < NH; ++j) {
       const int h = 8 * j + g;
+      float qv[KS][8];
+      float amax = 0.0f;
       #pragma unroll
-      for (int s = 0; s < KS; ++s) {
+      for (int ks = 0; ks < KS; ++ks) {
         #pragma unroll
         for (int i = 0; i < 2; ++i) {
-          const int col = c * KB + 4 * s + 2 * i;
-          qb[j][s][i] = h < p.G ? bf16x2_to_f16x2(__ldg(q32 + ((hrow0 + h) * D + col) / 2)) : 0u;
+          uint2 w = make_uint2(0u, 0u);
+          if (h < p.G) w = __ldg(q64 + ((hrow0 + h) * D + c * KB + 8 * ks + 4 * i) / 4);
+          const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w.x));
+          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w.y));
+          qv[ks][4 * i] = f0.x;
+          qv[ks][4 * i + 1] = f0.y;
+          qv[ks][4 * i + 2] = f1.x;
+          qv[ks][4 * i + 3] = f1.y;
+          amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y))));
         }
       }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      // sigma: 448 / amax with the mantissa cleared (a power of two, so that
+      // amax * sigma <= 448); 1 for an all-zero head
+      const float sig = amax > 0.0f ? __uint_as_float(__float_as_uint(448.0f / amax) & 0x7F800000u) : 1.0f;
+      const float isig = 1.0f / sig;
+      #pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        #pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          uint32_t hi = 0, lo = 0;
+          #pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float x0 = qv[ks][4 * i + 2 * e] * sig, x1 = qv[ks][4 * i + 2 * e + 1] * sig;
+            const uint32_t h2 = f32x2_to_e4m3x2(x0, x1);
+            const float2 d = e4m3x2_to_f32x2(h2);
+            const uint32_t l2 = f32x2_to_e4m3x2((x0 - d.x) * 16.0f, (x1 - d.y) * 16.0f);
+            hi |= h2 << (16 * e);
+            lo |= l2 << (16 * e);
+          }
+          qh[j][ks][i] = hi;
+          ql[j][ks][i] = lo;
+        }
+      }
+      inv_sig[j][0] = __shfl_sync(0xffffffffu, isig, 4 * (2 * c));
+      inv_sig[j][1] = __shfl_sync(0xffffffffu, isig, 4 * (2 * c + 1));
     }
   }
 
@@ -289,15 +350,22 @@ __global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 3) decode_attn_ker
         kw[r][4 * i + 3] = v.w;
       }
     }
-    float s[NH][4];
+    float s[NH][4], sl[NH][4];
     #pragma unroll
-    for (int j = 0; j < NH; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.0f;
+    for (int j = 0; j < NH; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = sl[j][0] = sl[j][1] = sl[j][2] = sl[j][3] = 0.0f;
     #pragma unroll
     for (int k = 0; k < KS; ++k) {
-      const uint32_t a[4] = {e4m3x2_to_f16x2(lo16(kw[0][k])), e4m3x2_to_f16x2(lo16(kw[1][k])),
-                             e4m3x2_to_f16x2(hi16(kw[0][k])), e4m3x2_to_f16x2(hi16(kw[1][k]))};
+      const uint32_t a[4] = {kw[0][2 * k], kw[1][2 * k], kw[0][2 * k + 1], kw[1][2 * k + 1]};
       #pragma unroll
-      for (int j = 0; j < NH; ++j) mma_f16(s[j], a, qb[j][k][0], qb[j][k][1]);
+      for (int j = 0; j < NH; ++j) {
+        mma_e4m3(s[j], a, qh[j][k][0], qh[j][k][1]);
+        mma_e4m3(sl[j], a, ql[j][k][0], ql[j][k][1]);
+      }
+    }
+    #pragma unroll
+    for (int j = 0; j < NH; ++j) {
+      #pragma unroll
+      for (int e = 0; e < 4; ++e) s[j][e] = fmaf(sl[j][e], 0.0625f, s[j][e]) * inv_sig[j][e & 1];
     }
 
     // this lane's positions g (s[.][0..1]) and g + 8 (s[.][2..3])

@@ -336,16 +336,20 @@ PTPC_API int ptpc_kv_cache_append(const void *K_dev, const void *V_dev, const in
 PTPC_API size_t ptpc_decode_attention_workspace_size(int64_t B, int64_t Hq, int64_t D, int64_t max_context);
 
 /* Decode attention (one query per sequence) over the FP8 cache:
- *   q_dev bf16 [B, Hq, D] (|q| < 65504), query head h reads KV head
- *   h / (Hq / Hkv) (Hq / Hkv <= 16);
+ *   q_dev bf16 [B, Hq, D], query head h reads KV head h / (Hq / Hkv)
+ *   (Hq / Hkv <= 16); the cache holds fewer than 2^31 slots
+ *   (num_blocks * block_size; PTPC_ERR_UNSUPPORTED_SHAPE otherwise);
  *   block_tables_dev int32 [B, max_blocks]: the cache blocks of each
  *   sequence in order; context_lens_dev int32 [B]: positions to attend to
  *   (<= max_context; positions whose block-table entry is missing, negative
  *   or past the cache are left out);
  *   out[b][h][d] = bf16_RNE(sum_l p_l * v_scale_l * dec(V_l[d])),
  *   p = softmax_l(softmax_scale * k_scale_l * sum_d q[d] * dec(K_l[d]))
- *   (0 for a sequence with no position), computed in fp32 with f16 tensor-
- *   core products of the exactly decoded codes.  out_dev bf16 [B, Hq, D].
+ *   (0 for a sequence with no position), computed in fp32: q K^T from
+ *   E4M3 tensor-core products of the K codes with q written as two E4M3
+ *   terms (exact for every bf16 q whose first term is a normal number, see
+ *   the kernel), P V from f16 products of the exactly decoded V codes.
+ *   out_dev bf16 [B, Hq, D].
  *   ws_dev: ptpc_decode_attention_workspace_size(B, Hq, D, max_context)
  *   bytes (the context is split into chunks of 512 positions whose partial
  *   results are combined by a second kernel). */

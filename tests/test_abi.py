@@ -183,6 +183,8 @@ def test_kv_cache_argument_checks(ptpc):
     assert at(*bad) == ptpc.ERR_UNSUPPORTED_SHAPE           # Hq not a multiple of Hkv
     bad = list(base); bad[8] = 256; bad[9] = 8
     assert at(*bad) == ptpc.ERR_UNSUPPORTED_SHAPE           # group of 32 query heads
+    bad = list(base); bad[12] = 2 ** 27
+    assert at(*bad) == ptpc.ERR_UNSUPPORTED_SHAPE           # 2^31 cache slots
     bad = list(base); bad[-2] = need - 1
     assert at(*bad) == ptpc.ERR_WORKSPACE_TOO_SMALL
     bad = list(base); bad[7] = 0
