@@ -373,6 +373,7 @@ int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co) {
 
 int ptpc_reload_tuning_overrides(void) {
   ptpc::reload_tuning();
+  ptpc::attn_reload_tuning();
   return PTPC_OK;
 }
 

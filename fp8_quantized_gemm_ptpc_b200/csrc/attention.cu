@@ -34,8 +34,10 @@
 // states are combined in shared memory and every CTA writes (max, sum,
 // accumulator) for its chunk; a second kernel combines the chunks and rounds
 // to bf16.
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -57,6 +59,7 @@ struct AttnParams {
   const int32_t *block_tables; // [B, max_blocks]
   const int32_t *context_lens; // [B]
   int Hq, Hkv, G, block_size, max_blocks, splits;
+  uint64_t bs_magic;           // floor(2^64 / block_size) + 1: pos / block_size = umul64hi(pos, bs_magic)
   int64_t num_slots;           // cache slots (num_blocks * block_size): larger slots are skipped
   float scale_log2;            // softmax_scale * log2(e)
   float *part_ml;              // [B, Hq, splits, 2]: running max (base-2 units), sum
@@ -117,8 +120,8 @@ constexpr int kAttnStages = 3;     // code stages a warp keeps in flight (two ti
 
 // Shared memory of one CTA: every warp's ring of code stages (K and V codes of
 // 16 positions, their scales and the tile's validity mask), which at the end
-// doubles as the warps' accumulators, and the cache slot of every position of
-// the chunk.
+// doubles as the warps' accumulators, and the chunk's block-table entries
+// (blocks hold at least 8 positions).
 // A position's D code bytes are stored as D/16 16-byte chunks, chunk i at
 // chunk index i ^ (position mod D/16), so that the fragment loads below hit
 // distinct shared-memory banks.
@@ -128,8 +131,8 @@ struct AttnSmem {
   static constexpr int STAGE = CODES_TILE + 2 * 16 * 4 + 16;          // + k, v scales + validity mask
   static constexpr int RING = kAttnStages * STAGE;
   static constexpr int CODES = kAttnWarps * RING;
-  static constexpr int SLOTS = CHUNK * 4;
-  static constexpr size_t BYTES = (size_t)CODES + SLOTS;
+  static constexpr int BLOCKS = (CHUNK / 8 + 2) * 4;
+  static constexpr size_t BYTES = (size_t)CODES + BLOCKS;
   static_assert(kAttnWarps * 16 * D * 4 <= CODES, "combine buffer");
   static_assert(STAGE % 16 == 0, "stage alignment");
 };
@@ -184,7 +187,7 @@ __global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 2) decode_attn_ker
   constexpr int KB = D / 4;         // K code bytes a lane holds per position
   constexpr int VB = D / 8;         // V code bytes a lane holds per position
   extern __shared__ __align__(16) uint8_t dsmem[];
-  int *s_slot = reinterpret_cast<int *>(dsmem + SM::CODES);
+  int *s_blk = reinterpret_cast<int *>(dsmem + SM::CODES);
   __shared__ float s_ml[kAttnWarps][16][2];
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -194,19 +197,12 @@ __global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 2) decode_attn_ker
   const int c0 = split * CHUNK;
   const int c1 = min(c0 + CHUNK, L);
 
-  // the cache slot of every position of the chunk, -1 where it is not read
-  // (past the context, no block-table entry, block outside the cache; the
-  // cache has fewer than 2^31 slots)
-  for (int i = threadIdx.x; i < CHUNK; i += kAttnThreads) {
-    const int pos = c0 + i;
-    int slot = -1;
-    if (pos < c1) {
-      const int bi = pos / p.block_size;
-      const int blk = bi < p.max_blocks ? __ldg(p.block_tables + (int64_t)b * p.max_blocks + bi) : -1;
-      const int64_t sl = (int64_t)blk * p.block_size + pos % p.block_size;
-      if (blk >= 0 && sl < p.num_slots) slot = (int)sl;
-    }
-    s_slot[i] = slot;
+  // the chunk's block-table entries (-1 where there is none)
+  const int bi0 = (int)__umul64hi((uint64_t)c0, p.bs_magic);
+  const int nbi = c1 > c0 ? (int)__umul64hi((uint64_t)(c1 - 1), p.bs_magic) - bi0 + 1 : 0;
+  for (int i = threadIdx.x; i < nbi; i += kAttnThreads) {
+    const int bi = bi0 + i;
+    s_blk[i] = bi < p.max_blocks ? __ldg(p.block_tables + (int64_t)b * p.max_blocks + bi) : -1;
   }
   __syncthreads();
 
@@ -219,9 +215,16 @@ __global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 2) decode_attn_ker
   // zero-filled and masked.
   auto prefetch = [&](int base, int st) {
     const int kk = lane >> 1, half = lane & 1;
-    const int slot = s_slot[base - c0 + kk];
+    const int pos = base + kk;
+    int64_t slot = -1;
+    if (pos < c1) {
+      const int bi = (int)__umul64hi((uint64_t)pos, p.bs_magic);   // pos / block_size, exactly
+      const int blk = s_blk[bi - bi0];
+      slot = (int64_t)blk * p.block_size + (pos - bi * p.block_size);
+      if (blk < 0 || slot >= p.num_slots) slot = -1;
+    }
     const bool valid = slot >= 0;
-    const int64_t row = valid ? (int64_t)slot * p.Hkv + kvh : 0;
+    const int64_t row = valid ? slot * p.Hkv + kvh : 0;
     uint8_t *sk = ring + st * SM::STAGE;
     uint8_t *sv = sk + 16 * D;
     const uint8_t *gk = p.kc + row * D;
@@ -541,22 +544,90 @@ __global__ void __launch_bounds__(D) decode_attn_combine_kernel(const float *__r
   out[bh * D + d] = __float2bfloat16_rn(l > 0.0f ? o / l : 0.0f);
 }
 
-constexpr int kAttnChunk = 512;
+// Context chunk of a CTA: 512, 1024 or 2048 positions.  Larger chunks pay the
+// CTA's start (block table, query terms) and end (the warps' combine) over
+// more tiles but leave fewer CTAs to fill the GPU; the launch takes the chunk
+// with the fewest rounds of resident CTAs times positions a CTA (ties: the
+// larger chunk).
+constexpr int kAttnChunkMin = 512;
 
-template <int D, int NH>
-cudaError_t launch_attn(const AttnParams &p, int B, __nv_bfloat16 *out, cudaStream_t st) {
-  const size_t smem = AttnSmem<D, kAttnChunk>::BYTES;
+template <int D, int CHUNK, int NH>
+cudaError_t launch_attn_chunk(const AttnParams &p, int B, cudaStream_t st) {
+  const size_t smem = AttnSmem<D, CHUNK>::BYTES;
   static std::atomic<bool> attr_set[64];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
-    cudaError_t a = cudaFuncSetAttribute(decode_attn_kernel<D, kAttnChunk, NH>,
+    cudaError_t a = cudaFuncSetAttribute(decode_attn_kernel<D, CHUNK, NH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (a != cudaSuccess) return a;
     attr_set[dev].store(true, std::memory_order_release);
   }
-  decode_attn_kernel<D, kAttnChunk, NH><<<dim3(p.splits, p.Hkv, B), kAttnThreads, smem, st>>>(p);
-  cudaError_t e = cudaGetLastError();
+  decode_attn_kernel<D, CHUNK, NH><<<dim3(p.splits, p.Hkv, B), kAttnThreads, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+// CTAs of the attention kernel that can be resident at once on this device.
+template <int D, int NH>
+int attn_resident() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int sms = 148, per_sm = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaFuncSetAttribute(decode_attn_kernel<D, 2048, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)AttnSmem<D, 2048>::BYTES);
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_attn_kernel<D, 2048, NH>, kAttnThreads,
+                                                    AttnSmem<D, 2048>::BYTES) != cudaSuccess || per_sm <= 0)
+    per_sm = 1;
+  cudaGetLastError();
+  const int n = std::max(1, sms * per_sm);
+  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// PTPC_FORCE_ATTN_CHUNK = 512 | 1024 | 2048 (tuning and tests only): read at
+// the first launch, or again by attn_reload_tuning.
+std::atomic<int> g_attn_chunk{-1};
+
+int read_attn_chunk() {
+  const char *v = std::getenv("PTPC_FORCE_ATTN_CHUNK");
+  if (v == nullptr) return 0;
+  const int c = std::atoi(v);
+  return c == 512 || c == 1024 || c == 2048 ? c : 0;
+}
+
+int attn_chunk(int pairs, int max_context, int resident) {
+  int forced = g_attn_chunk.load(std::memory_order_relaxed);
+  if (forced < 0) {
+    forced = read_attn_chunk();
+    g_attn_chunk.store(forced, std::memory_order_relaxed);
+  }
+  if (forced > 0) return forced;
+  int best = kAttnChunkMin;
+  long long best_cost = -1;
+  for (int chunk = kAttnChunkMin; chunk <= 2048; chunk *= 2) {
+    const long long ctas = (long long)pairs * ((std::max(max_context, 1) + chunk - 1) / chunk);
+    const long long cost = (ctas + resident - 1) / resident * chunk;
+    if (best_cost < 0 || cost <= best_cost) {
+      best = chunk;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
+template <int D, int NH>
+cudaError_t launch_attn(AttnParams p, int B, int max_context, __nv_bfloat16 *out, cudaStream_t st) {
+  const int chunk = attn_chunk(B * p.Hkv, max_context, attn_resident<D, NH>());
+  p.splits = (std::max(max_context, 1) + chunk - 1) / chunk;
+  cudaError_t e = chunk == 2048   ? launch_attn_chunk<D, 2048, NH>(p, B, st)
+                  : chunk == 1024 ? launch_attn_chunk<D, 1024, NH>(p, B, st)
+                                  : launch_attn_chunk<D, 512, NH>(p, B, st);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(B * p.Hq);
@@ -573,7 +644,10 @@ cudaError_t launch_attn(const AttnParams &p, int B, __nv_bfloat16 *out, cudaStre
 
 }  // namespace
 
-int attn_splits(int max_context) { return max_context <= 0 ? 1 : (max_context + kAttnChunk - 1) / kAttnChunk; }
+void attn_reload_tuning() { g_attn_chunk.store(read_attn_chunk(), std::memory_order_relaxed); }
+
+// The most chunks a launch can split a context into (the workspace bound).
+int attn_splits(int max_context) { return max_context <= 0 ? 1 : (max_context + kAttnChunkMin - 1) / kAttnChunkMin; }
 
 size_t attn_workspace_bytes(int B, int Hq, int D, int max_context) {
   const size_t n = (size_t)B * Hq * attn_splits(max_context);
@@ -598,15 +672,19 @@ cudaError_t launch_decode_attention(const void *q, const uint8_t *kc, const uint
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
   p.block_size = block_size;
+  // ceil(2^64 / block_size): pos * bs_magic / 2^64 is pos / block_size plus less than 2^-32 for
+  // pos < 2^32, and the fractional part of pos / block_size is at most 1 - 1 / block_size,
+  // so the high word is the exact quotient
+  p.bs_magic = ~0ull / (uint64_t)block_size + 1;
   p.max_blocks = max_blocks;
-  p.splits = attn_splits(max_context);
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
-  const size_t n = (size_t)B * Hq * p.splits;
+  // partial results of up to attn_splits(max_context) chunks a head
+  const size_t n = (size_t)B * Hq * attn_splits(max_context);
   p.part_ml = static_cast<float *>(ws);
   p.part_acc = static_cast<float *>(ws) + n * 2;
   __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
-  if (D == 64) return p.G > 8 ? launch_attn<64, 2>(p, B, o, st) : launch_attn<64, 1>(p, B, o, st);
-  if (D == 128) return p.G > 8 ? launch_attn<128, 2>(p, B, o, st) : launch_attn<128, 1>(p, B, o, st);
+  if (D == 64) return p.G > 8 ? launch_attn<64, 2>(p, B, max_context, o, st) : launch_attn<64, 1>(p, B, max_context, o, st);
+  if (D == 128) return p.G > 8 ? launch_attn<128, 2>(p, B, max_context, o, st) : launch_attn<128, 1>(p, B, max_context, o, st);
   return cudaErrorInvalidValue;
 }
 

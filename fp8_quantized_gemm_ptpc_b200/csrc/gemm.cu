@@ -166,9 +166,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 }
 
 // Stages one warp's 32 rows x 128 bytes in 128-byte-swizzled shared memory and
-// stores them with TMA at (col, row).  `packed` holds this lane's row.
+// stores them with TMA at (col, row).  `packed` holds this lane's row.  The
+// stored lines are marked evict-first in L2: the kernel never reads them, and
+// they must not push out the operand tiles that other CTAs still read.
 __device__ __forceinline__ void stage_and_store(const CUtensorMap *tmC, uint8_t *cbuf, const uint32_t (&packed)[32],
-                                                int col, int row, int lane) {
+                                                int col, int row, int lane, uint64_t pol) {
   // the previous TMA store from this buffer must have finished reading it
   if (lane == 0) bulk_wait_read<0>();
   __syncwarp();
@@ -181,7 +183,7 @@ __device__ __forceinline__ void stage_and_store(const CUtensorMap *tmC, uint8_t 
   fence_async_shared();
   __syncwarp();
   if (lane == 0) {
-    tma_store_2d(tmC, cbuf, col, row);
+    tma_store_2d_hint(tmC, cbuf, col, row, pol);
     bulk_commit();
   }
 }
@@ -218,7 +220,8 @@ __device__ __forceinline__ void scale_pack32(const uint32_t (&r)[32], float xsr,
 template <int BN_T, bool F32OUT>
 __device__ __forceinline__ void epilogue_store_tile(const CUtensorMap *tmC, uint32_t tbase, uint8_t *cbuf,
                                                     float *sc, const GemmParams &p, int col_base,
-                                                    int store_row0, float xsr, int lane, uint32_t release_bar) {
+                                                    int store_row0, float xsr, int lane, uint32_t release_bar,
+                                                    uint64_t pol) {
   constexpr int EPI_COLS = F32OUT ? 32 : 64;
   #pragma unroll 1
   for (int c0 = 0; c0 < BN_T; c0 += EPI_COLS) {
@@ -242,7 +245,7 @@ __device__ __forceinline__ void epilogue_store_tile(const CUtensorMap *tmC, uint
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(release_bar);
     }
-    stage_and_store(tmC, cbuf, packed, col_base + c0, store_row0, lane);
+    stage_and_store(tmC, cbuf, packed, col_base + c0, store_row0, lane, pol);
   }
 }
 
@@ -625,7 +628,7 @@ __device__ __forceinline__ void dump_partial(uint32_t tbase, float *row_dst, int
 template <bool F32OUT>
 __device__ __forceinline__ void epilogue_store_swap(const CUtensorMap *tmC, uint32_t tbase, uint8_t *cbuf,
                                                     const GemmParams &p, int ch0, int t0, int lane,
-                                                    uint32_t release_bar) {
+                                                    uint32_t release_bar, uint64_t pol) {
   const int ch = ch0 + lane;
   float wsr = 0.0f;
   if constexpr (!F32OUT) wsr = ch < p.Co ? __ldg(p.ws + ch) : 0.0f;
@@ -662,7 +665,7 @@ __device__ __forceinline__ void epilogue_store_swap(const CUtensorMap *tmC, uint
     fence_async_shared();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(tmC, cbuf, ch0, t0 + c0);
+      tma_store_2d_hint(tmC, cbuf, ch0, t0 + c0, pol);
       bulk_commit();
     }
   }
@@ -862,8 +865,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
     if (elect_one()) {
+      // Activation tiles are read by every column tile of their group of tile
+      // rows: kept (evict-last).  Weight tiles are read by the group's tile
+      // rows at about the same time: normal priority.  Marked evict-first
+      // (as in the decode kernel, where each weight byte is read once) they
+      // were pushed out of L2 by the output stream before the other rows
+      // read them: 10.8 GB of DRAM reads for the 0.54 GB of operands of the
+      // 70B gate+up layer at T = 8192.
       const uint64_t polA = policy_evict_last();
-      const uint64_t polB = policy_evict_first();
+      const uint64_t polB = policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -987,6 +997,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // a member of the split tail: decided by the schedule alone, so every
     // epilogue warp runs the tail protocol's barriers whatever happens above
     const bool tail_member = p.tail_tiles > 0 && !F32OUT && cid < p.tail_tiles * p.tail_split;
+    const uint64_t polC = policy_evict_first();  // output lines: never read here
     int tail_j = 0, tail_m = 0, tail_n = 0, tail_r = 0;
     bool dumped = false;
     if (tail_member) {
@@ -1018,7 +1029,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int ch0 = u.n * BN + (int)rank * HALF_N + q * 32;
           if (u.split < 0) {
             epilogue_store_swap<F32OUT>(&tmC, tbase, cbuf, p, ch0, u.m * p.nt, lane,
-                                        mapa_shared(&tempty[buf], 0));
+                                        mapa_shared(&tempty[buf], 0), polC);
           } else if constexpr (!F32OUT) {
             tail_j = u.tile - p.full_tiles;
             tail_m = u.m;
@@ -1032,7 +1043,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
       } else if (u.split < 0) {
         epilogue_store_tile<BN, F32OUT>(&tmC, tbase, cbuf, scl, p, u.n * BN, row0, xsr, lane,
-                                        mapa_shared(&tempty[buf], 0));
+                                        mapa_shared(&tempty[buf], 0), polC);
       } else if constexpr (!F32OUT) {
         tail_j = u.tile - p.full_tiles;
         tail_m = u.m;
@@ -1375,7 +1386,8 @@ constexpr double kPairN128Cost = 1.15;
 // PTPC_FORCE_KSPLIT = 1 | 2 | 4 | 8, PTPC_FORCE_SPLIT_TAIL = 0 | 1 (the pair
 // kernel's split tail off, or on wherever it is feasible), PTPC_FORCE_SWAP =
 // 0 | 1 (the pair kernel's swapped operands off, or on for every pair-kernel
-// shape).  Read once, at the first GEMM call of the process (or again by
+// shape), PTPC_FORCE_GROUP_M = 1 .. 63 (tile rows visited together by the pair
+// kernel).  Read once, at the first GEMM call of the process (or again by
 // reload_tuning), not on every call.
 struct Tuning {
   int kernel;   // 0 automatic, 1 pair, 2 decode
@@ -1383,6 +1395,7 @@ struct Tuning {
   int ksplit;   // 0 automatic, 1, 2, 4, 8
   int streamk;  // 0 automatic, 1 off, 2 on wherever feasible
   int swap;     // 0 automatic, 1 off, 2 on
+  int group_m;  // 0 automatic, else tile rows a group (1 .. 63)
 };
 
 int env_int(const char *name, int fallback) {
@@ -1394,7 +1407,7 @@ int env_int(const char *name, int fallback) {
 }
 
 Tuning read_tuning() {
-  Tuning t{0, 0, 0, 0, 0};
+  Tuning t{0, 0, 0, 0, 0, 0};
   const char *k = std::getenv("PTPC_FORCE_KERNEL");
   if (k != nullptr && std::strcmp(k, "pair") == 0) t.kernel = 1;
   if (k != nullptr && std::strcmp(k, "decode") == 0) t.kernel = 2;
@@ -1408,16 +1421,18 @@ Tuning read_tuning() {
   const int sw = env_int("PTPC_FORCE_SWAP", -1);
   if (sw == 0) t.swap = 1;
   if (sw == 1) t.swap = 2;
+  const int gm = env_int("PTPC_FORCE_GROUP_M", 0);
+  if (gm >= 1 && gm <= 63) t.group_m = gm;
   return t;
 }
 
 // Packed as kernel | pair_bn / 128 << 2 | ksplit << 4 | streamk << 9 |
-// swap << 11, plus bit 8 once read.
+// swap << 11 | group_m << 13, plus bit 8 once read.
 std::atomic<uint32_t> g_tuning{0};
 
 uint32_t pack_tuning(const Tuning &t) {
   return 0x100u | (uint32_t)t.kernel | (uint32_t)(t.pair_bn / 128) << 2 | (uint32_t)t.ksplit << 4 |
-         (uint32_t)t.streamk << 9 | (uint32_t)t.swap << 11;
+         (uint32_t)t.streamk << 9 | (uint32_t)t.swap << 11 | (uint32_t)t.group_m << 13;
 }
 
 Tuning tuning() {
@@ -1427,7 +1442,7 @@ Tuning tuning() {
     g_tuning.store(v, std::memory_order_relaxed);
   }
   return Tuning{(int)(v & 3u), (int)((v >> 2) & 3u) * 128, (int)((v >> 4) & 15u), (int)((v >> 9) & 3u),
-                (int)((v >> 11) & 3u)};
+                (int)((v >> 11) & 3u), (int)((v >> 13) & 63u)};
 }
 
 // Fewest K-blocks a CTA of a K-split cluster streams.
@@ -1556,6 +1571,12 @@ double est_waves(long long tiles, int pairs, int num_kb, size_t ws_bytes, int bn
 // channels a tile, or, with the operands swapped, 256 channels x nt tokens
 // where that finishes the waves sooner (ragged T: the token tiles divide T
 // evenly instead of rounding it up to 256 rows), then the split tail.
+// Activation bytes a group of tile rows may keep in L2 (126 MB on B200).
+// Measured on the 70B layers at T = 8192 (32 tile rows): with groups of 8
+// rows the gate+up GEMM read 3.0 GB from DRAM for 0.54 GB of operands (the
+// weights once per group) and down-proj 2.2 GB for 0.47 GB.
+constexpr long long kGroupL2Bytes = 64ll << 20;
+
 Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d, size_t ws_bytes) {
   Plan pl = {};
   pl.pair = true;
@@ -1563,7 +1584,6 @@ Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d, size_t ws_bytes) {
   pl.num_kb = (Ci + BK - 1) / BK;
   pl.tile_rows = 2 * BM;
   pl.bn = choose_pair_bn(T, Co, d);
-  pl.group_m = 8;
   pl.num_m = (T + pl.tile_rows - 1) / pl.tile_rows;
   pl.num_n = (Co + pl.bn - 1) / pl.bn;
   pl.num_tiles = pl.num_m * pl.num_n;
@@ -1585,6 +1605,12 @@ Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d, size_t ws_bytes) {
     pl.num_n = (Co + 255) / 256;
     pl.num_tiles = (int)swap_tiles;
   }
+  // Tile rows visited together: their activation tiles stay in L2 (loaded
+  // evict-last) while the column tiles sweep past, so every weight tile is
+  // read from DRAM once per group.  As many rows as fit in half the L2.
+  const long long row_bytes = (long long)pl.tile_rows * Ci;
+  pl.group_m = (int)std::max(1LL, std::min<long long>(pl.num_m, kGroupL2Bytes / row_bytes));
+  if (tuning().group_m > 0) pl.group_m = std::min(pl.num_m, tuning().group_m);
   pl.ctas = std::max(1, std::min(pl.num_tiles, pl.bn == 128 ? d.pair_clusters128 : d.pair_clusters));
   choose_tail(pl, ws_bytes);
   return pl;

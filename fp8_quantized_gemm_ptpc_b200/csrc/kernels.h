@@ -78,6 +78,7 @@ int num_sms();
 // Re-reads the PTPC_FORCE_* tuning overrides from the environment (they are
 // otherwise read once, at the first GEMM call).
 void reload_tuning();
+void attn_reload_tuning();
 
 // Tensor-map cache counters since the library was loaded.
 void map_cache_stats(uint64_t *hits, uint64_t *misses);

@@ -102,6 +102,14 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *m, const void *s
                : "memory");
 }
 
+// The same with an L2 cache policy for the stored lines.
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap *m, const void *src, int32_t x, int32_t y,
+                                                  uint64_t policy) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;"
+               ::"l"(m), "r"(smem_u32(src)), "r"(x), "r"(y), "l"(policy)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 template <int N>
@@ -124,6 +132,11 @@ __device__ __forceinline__ void fence_async_shared() {
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 __device__ __forceinline__ uint64_t policy_evict_first() {

@@ -257,7 +257,12 @@ PTPC_API int ptpc_linear_fmt(const void *X_dev, int64_t ldx, const uint8_t *Wq_d
  *   PTPC_FORCE_SWAP    = 0 | 1           the prefill kernel's swapped operands
  *                                        (weights as the 256-row operand,
  *                                        tokens as the tile's columns) off, or
- *                                        on for every prefill-kernel shape.
+ *                                        on for every prefill-kernel shape,
+ *   PTPC_FORCE_GROUP_M = 1 .. 63         tile rows the prefill kernel visits
+ *                                        together (their activation tiles
+ *                                        kept in L2 while the columns sweep),
+ *   PTPC_FORCE_ATTN_CHUNK = 512 | 1024 | 2048  context positions a CTA of
+ *                                        ptpc_decode_attention takes.
  * Each is honoured only where the forced choice is feasible for the shape;
  * results stay within the GEMM's tolerance under every choice.  For tuning
  * and tests, not for production.  Not thread-safe with concurrent GEMM calls
@@ -351,8 +356,9 @@ PTPC_API size_t ptpc_decode_attention_workspace_size(int64_t B, int64_t Hq, int6
  *   the kernel), P V from f16 products of the exactly decoded V codes.
  *   out_dev bf16 [B, Hq, D].
  *   ws_dev: ptpc_decode_attention_workspace_size(B, Hq, D, max_context)
- *   bytes (the context is split into chunks of 512 positions whose partial
- *   results are combined by a second kernel). */
+ *   bytes (the context is split into chunks of 512, 1024 or 2048 positions,
+ *   chosen per launch to fill the GPU, whose partial results are combined by
+ *   a second kernel). */
 PTPC_API int ptpc_decode_attention(const void *q_dev, const uint8_t *k_cache_dev, const uint8_t *v_cache_dev,
                                    const float *k_scale_dev, const float *v_scale_dev,
                                    const int32_t *block_tables_dev, const int32_t *context_lens_dev, int64_t B,

@@ -106,6 +106,29 @@ def test_append_bit_exact(ptpc):
     ([0, 5, 2049], 28, 4, 128, 16),
 ])
 def test_decode_attention(ptpc, lens, Hq, Hkv, D, bs):
+    _attention_case(ptpc, lens, Hq, Hkv, D, bs)
+
+
+@pytest.mark.parametrize("chunk", ["1024", "2048"])
+@pytest.mark.parametrize("lens,Hq,Hkv,D,bs", [
+    ([511, 512, 513, 1030, 2047, 2048, 2049, 4100], 64, 8, 128, 16),
+    ([257, 1500, 3000], 32, 2, 64, 24),
+    ([0, 5, 2049], 28, 4, 128, 16),
+])
+def test_decode_attention_chunk_sizes(ptpc, monkeypatch, chunk, lens, Hq, Hkv, D, bs):
+    """The larger context chunks a CTA can take (chosen by the launch for
+    long contexts on many sequences), forced on small cases; a block size
+    that is not a power of two exercises the exact quotient."""
+    monkeypatch.setenv("PTPC_FORCE_ATTN_CHUNK", chunk)
+    ptpc.reload_tuning_overrides()
+    try:
+        _attention_case(ptpc, lens, Hq, Hkv, D, bs)
+    finally:
+        monkeypatch.delenv("PTPC_FORCE_ATTN_CHUNK")
+        ptpc.reload_tuning_overrides()
+
+
+def _attention_case(ptpc, lens, Hq, Hkv, D, bs):
     dev, ref = build_cache(ptpc, lens, Hkv, D, bs, seed=sum(lens) + Hq, holes=True)
     kc, vc, ksc, vsc, tables = dev
     rk, rv, rks, rvs = ref
