@@ -1571,11 +1571,14 @@ double est_waves(long long tiles, int pairs, int num_kb, size_t ws_bytes, int bn
 // channels a tile, or, with the operands swapped, 256 channels x nt tokens
 // where that finishes the waves sooner (ragged T: the token tiles divide T
 // evenly instead of rounding it up to 256 rows), then the split tail.
-// Activation bytes a group of tile rows may keep in L2 (126 MB on B200).
-// Measured on the 70B layers at T = 8192 (32 tile rows): with groups of 8
-// rows the gate+up GEMM read 3.0 GB from DRAM for 0.54 GB of operands (the
-// weights once per group) and down-proj 2.2 GB for 0.47 GB.
+// Tile rows visited together: at most kGroupMaxRows, and no more than keep
+// kGroupL2Bytes of activation tiles (half the 126 MB L2).  Measured on the
+// 70B layers at T = 8192 (32 tile rows; ncu DRAM reads of one launch without
+// a cache flush): gate+up (2 MB of activations a row) 2.53 GB with groups of
+// 8, 1.41 GB with 16, 3.50 GB with 32; down-proj (7.3 MB a row) 2.07 GB with
+// 8, 2.33 GB with 16.
 constexpr long long kGroupL2Bytes = 64ll << 20;
+constexpr int kGroupMaxRows = 16;
 
 Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d, size_t ws_bytes) {
   Plan pl = {};
@@ -1607,9 +1610,9 @@ Plan pair_plan(int T, int Ci, int Co, const DeviceInfo &d, size_t ws_bytes) {
   }
   // Tile rows visited together: their activation tiles stay in L2 (loaded
   // evict-last) while the column tiles sweep past, so every weight tile is
-  // read from DRAM once per group.  As many rows as fit in half the L2.
+  // read from DRAM once per group.
   const long long row_bytes = (long long)pl.tile_rows * Ci;
-  pl.group_m = (int)std::max(1LL, std::min<long long>(pl.num_m, kGroupL2Bytes / row_bytes));
+  pl.group_m = (int)std::max(1LL, std::min<long long>(std::min(pl.num_m, kGroupMaxRows), kGroupL2Bytes / row_bytes));
   if (tuning().group_m > 0) pl.group_m = std::min(pl.num_m, tuning().group_m);
   pl.ctas = std::max(1, std::min(pl.num_tiles, pl.bn == 128 ? d.pair_clusters128 : d.pair_clusters));
   choose_tail(pl, ws_bytes);
