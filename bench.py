@@ -77,7 +77,7 @@ def parse():
                     help="T values of the decode record inside the default line ('' to skip)")
     ap.add_argument("--weight-formats", default="e3m2,e2m1",
                     help="sub-byte weight formats of the decode_subbyte record")
-    ap.add_argument("--record", default=None, choices=["decode", "decode_subbyte", "kv_decode"],
+    ap.add_argument("--record", default=None, choices=["decode", "decode_subbyte", "kv_decode", "prefill_subbyte"],
                     help="print only this sub-record of the default line (a short run for profiling)")
     return ap.parse_args()
 
@@ -479,6 +479,55 @@ def decode_subbyte_record(ptpc, dev, peaks, tokens, steps, fmts=("e3m2", "e2m1")
         del Ls
         torch.cuda.empty_cache()
     return {"workload": wl.name + ", sub-byte per-channel weights, FP8 per-token activations", "steps": steps,
+            "per_format": res}
+
+
+def prefill_subbyte_record(ptpc, dev, peaks, steps, fmts=("e3m2", "e2m1"), T=8192):
+    """The 70B prefill layers (gate+up 8192 -> 57344, down 28672 -> 8192) at
+    T = 8192 with FP6 (E3M2) and FP4 (E2M1) per-channel weights: the same
+    step as the default line (per-token FP8 activations quantised per call)
+    through ptpc_linear_fmt.  The mixed-format MMA runs at the FP8 rate, so
+    the roofline is the same burst FP8 figure."""
+    import torch
+    wl = synthetic.LLAMA70B_PREFILL
+    stream = torch.cuda.current_stream(dev)
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    flops = sum(2.0 * T * L.Ci * L.Co for L in wl.layers)
+    Xs = [torch.from_numpy(synthetic.make_x(wl, i, T, L.Ci).view(np.int16)).to(dev).view(torch.bfloat16)
+          for i, L in enumerate(wl.layers)]
+    outs = [torch.empty((T, L.Co), dtype=torch.bfloat16, device=dev) for L in wl.layers]
+    wsps = [ptpc.Workspace(ptpc.workspace_size(ptpc.OP_LINEAR, T, L.Ci, L.Co), dev) for L in wl.layers]
+    res = {}
+    for fmt in fmts:
+        Ws = []
+        for i, L in enumerate(wl.layers):
+            Wb = torch.from_numpy(synthetic.make_w(wl, i, L.Ci, L.Co).view(np.int16)).to(dev).view(torch.bfloat16)
+            Ws.append(ptpc.quantize_weights_fmt(Wb, fmt))
+            del Wb
+
+        def step():
+            for j, (Wq, ws) in enumerate(Ws):
+                ptpc.linear_fmt(Xs[j], Wq, ws, fmt, out=outs[j], ws=wsps[j])
+
+        for _ in range(3):
+            step()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / steps
+        tf = flops / (ms / 1e3) / 1e12
+        res[fmt] = {"ms_per_step": ms, "tflops": tf, "frac_of_fp8_peak": tf / fp8_peak,
+                    "weight_bytes_vs_fp8": ptpc.WEIGHT_BITS[fmt] / 8}
+        del Ws
+        torch.cuda.empty_cache()
+    del Xs, outs, wsps
+    torch.cuda.empty_cache()
+    return {"workload": f"Llama-3.1-70B prefill T={T} (gate+up, down), sub-byte per-channel weights", "steps": steps,
+            "peak": fp8_peak, "unit": "TFLOP/s", "note": "step TFLOP/s (quantiser + GEMM launches)",
             "per_format": res}
 
 
@@ -893,6 +942,7 @@ def run_gpu(args):
                                                            or dec_tokens[:1], steps=max(20, min(K * 2, 100)))
         if not args.no_kv:
             line["kv_decode"] = kv_decode_record(ptpc, dev, peaks)
+        line["prefill_subbyte"] = prefill_subbyte_record(ptpc, dev, peaks, steps=max(5, min(K, 20)))
         chain_tokens = [int(t) for t in args.chain_tokens.split(",") if t.strip()]
         if chain_tokens:
             Ws = chain_weights(ptpc, dev)
@@ -1169,6 +1219,9 @@ def run_record(args):
     elif args.record == "decode_subbyte":
         rec = decode_subbyte_record(ptpc, dev, peaks, tokens, steps=steps,
                                     fmts=tuple(f for f in args.weight_formats.split(",") if f))
+    elif args.record == "prefill_subbyte":
+        rec = prefill_subbyte_record(ptpc, dev, peaks, steps=steps,
+                                     fmts=tuple(f for f in args.weight_formats.split(",") if f))
     else:
         rec = kv_decode_record(ptpc, dev, peaks, steps=steps)
     print(json.dumps({"record": args.record} | rec), flush=True)
