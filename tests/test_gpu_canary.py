@@ -72,6 +72,7 @@ def test_weight_quantiser_stays_in_bounds(ptpc, Ci, Co):
 @pytest.mark.parametrize("T,Ci,Co", [
     (1, 4096, 2048), (13, 2048, 4096), (128, 1024, 8192), (200, 4112, 8192), (77, 384, 528),
     (300, 640, 1040), (512, 8192, 10240), (2048, 4096, 6144), (1000, 1024, 2064),
+    (1, 1024, 28672), (64, 512, 20512),      # decode, a second partial round of tiles
 ])
 def test_gemm_and_linear_stay_in_bounds(ptpc, T, Ci, Co):
     X = to_dev_bf16(synthetic.make_x(synthetic.DECODE_70B, 0, T, Ci))

@@ -106,6 +106,26 @@ def test_decode_cluster_split(ptpc, monkeypatch, T, Ci, Co, splits):
         ptpc.reload_tuning_overrides()
 
 
+@pytest.mark.parametrize("T,Ci,Co,fmt", [(1, 1024, 28672, "e4m3"), (77, 512, 20512, "e4m3"),
+                                         (1, 1024, 28672, "e2m1"), (32, 1024, 20480, "e3m2")])
+def test_decode_two_rounds_of_tiles(ptpc, T, Ci, Co, fmt):
+    """Decode shapes with more 128-channel tiles than SMs (a second, partial
+    round of tiles): parity on every channel, including the last, partial
+    tile, for FP8 and sub-byte weights."""
+    X = synthetic.with_edge_rows(synthetic.make_x(synthetic.DECODE_70B, 0, T, Ci), huge_bits=BIG_BF16)
+    W = synthetic.random_bf16((Ci, Co), seed=T + Co, scale=0.02)
+    Wq, ws = ptpc.quantize_weights_fmt(to_dev_bf16(W), fmt)
+    Xq, xs = ptpc.quantize_activations(to_dev_bf16(X))
+    out = from_dev_bf16(ptpc.scaled_mm_fmt(Xq, xs, Wq, ws, fmt))
+    rXq, rxs = oracle.quant_act(X)
+    if fmt == "e4m3":
+        ref = oracle.scaled_mm_reference(rXq, rxs, *oracle.quant_weight(W))
+    else:
+        codes, rws = oracle.quant_weight_fmt(W, fmt)
+        ref = oracle.scaled_mm_reference_fmt(rXq, rxs, codes, rws, fmt)
+    assert_gemm_close(out, ref, f"decode, two rounds of tiles {fmt} {T}x{Ci}x{Co}")
+
+
 def test_decode_split_matches_naive_step1(ptpc):
     """The K-split path's fp32 output (naive step 1) is what the fused path
     scales: applying the scales to it gives the fused output bit for bit."""
