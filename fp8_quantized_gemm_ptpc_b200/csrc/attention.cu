@@ -276,8 +276,11 @@ __global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 2) decode_attn_ker
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
       // sigma: 448 / amax with the mantissa cleared (a power of two, so that
-      // amax * sigma <= 448); 1 for an all-zero head
-      const float sig = amax > 0.0f ? __uint_as_float(__float_as_uint(448.0f / amax) & 0x7F800000u) : 1.0f;
+      // amax * sigma <= 448), at most 2^126 (a head of subnormal values); 1
+      // for an all-zero head
+      const float sig = amax > 0.0f ? fminf(__uint_as_float(__float_as_uint(448.0f / amax) & 0x7F800000u),
+                                            __uint_as_float(253u << 23))
+                                    : 1.0f;
       const float isig = 1.0f / sig;
       #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
@@ -368,7 +371,7 @@ __global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 2) decode_attn_ker
     #pragma unroll
     for (int j = 0; j < NH; ++j) {
       #pragma unroll
-      for (int e = 0; e < 4; ++e) s[j][e] = fmaf(sl[j][e], 0.0625f, s[j][e]) * inv_sig[j][e & 1];
+      for (int e = 0; e < 4; ++e) s[j][e] = fmaf(sl[j][e], 0.0625f, s[j][e]);
     }
 
     // this lane's positions g (s[.][0..1]) and g + 8 (s[.][2..3])
@@ -392,10 +395,14 @@ __global__ void __launch_bounds__(kAttnThreads, NH == 1 ? 4 : 2) decode_attn_ker
     #pragma unroll
     for (int j = 0; j < NH; ++j) {
       // key scales and masking
-      s[j][0] = ok0 ? s[j][0] * k0 : -INFINITY;
-      s[j][1] = ok0 ? s[j][1] * k0 : -INFINITY;
-      s[j][2] = ok8 ? s[j][2] * k8 : -INFINITY;
-      s[j][3] = ok8 ? s[j][3] * k8 : -INFINITY;
+      // the key scale and the query's 1 / sigma multiplied first: each may be
+      // far from 1 (a huge query has a tiny 1 / sigma), their product is not
+      const float k0h0 = k0 * inv_sig[j][0], k0h1 = k0 * inv_sig[j][1];
+      const float k8h0 = k8 * inv_sig[j][0], k8h1 = k8 * inv_sig[j][1];
+      s[j][0] = ok0 ? s[j][0] * k0h0 : -INFINITY;
+      s[j][1] = ok0 ? s[j][1] * k0h1 : -INFINITY;
+      s[j][2] = ok8 ? s[j][2] * k8h0 : -INFINITY;
+      s[j][3] = ok8 ? s[j][3] * k8h1 : -INFINITY;
       float pv[4];
       #pragma unroll
       for (int e = 0; e < 2; ++e) {

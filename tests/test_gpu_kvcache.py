@@ -173,3 +173,22 @@ def test_decode_attention_70b_shape(ptpc):
                                 torch.tensor(lens, dtype=torch.int32, device="cuda"), 4096, 1 / math.sqrt(128))
     r = oracle.decode_attention_reference(q, rk, rks, rv, rvs, tables, lens, 16, 1 / math.sqrt(128))
     assert_gemm_close(from_dev_bf16(out), r, "70B decode attention")
+
+
+@pytest.mark.parametrize("q_scale", [1e-39, 1e-20, 1e20, 3e37])
+def test_decode_attention_query_range(ptpc, q_scale):
+    """Query vectors far from unit size (bf16 subnormals up to near the bf16
+    maximum, times a softmax scale that keeps the scores finite): the
+    power-of-two scale of the query's two E4M3 terms keeps them in range."""
+    lens, Hq, Hkv, D, bs = [37, 130], 16, 2, 128, 16
+    dev, ref = build_cache(ptpc, lens, Hkv, D, bs, seed=5)
+    kc, vc, ksc, vsc, tables = dev
+    rk, rv, rks, rvs = ref
+    rng = np.random.Generator(np.random.PCG64(21))
+    qf = rng.standard_normal((len(lens), Hq, D)).astype(np.float32) * np.float32(q_scale)
+    q = synthetic.to_bf16_bits(qf)
+    scale = float(min(1.0, 1.0 / (q_scale * math.sqrt(D))))
+    out = ptpc.decode_attention(to_dev_bf16(q), kc, vc, ksc, vsc, torch.from_numpy(tables).cuda(),
+                                torch.tensor(lens, dtype=torch.int32, device="cuda"), max(lens), scale)
+    r = oracle.decode_attention_reference(q, rk, rks, rv, rvs, tables, lens, bs, scale)
+    assert_gemm_close(from_dev_bf16(out), r, f"attention, |q| ~ {q_scale}")
