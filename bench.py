@@ -591,6 +591,7 @@ def kv_decode_record(ptpc, dev, peaks, B=32, ctx=4096, Hq=64, Hkv=8, D=128, bs=1
     rec = {
         "workload": f"Llama-3.1-70B decode attention: {B} sequences x {ctx} cached positions, {Hq} query / "
                     f"{Hkv} KV heads, D = {D}, {bs}-position blocks (shuffled), E4M3 codes + per-(token, head) scales",
+        "kernel": ptpc.decode_attention_kernel(Hq, Hkv, D, bs),
         "ms_per_step": ms, "algorithmic_bytes": nbytes,
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": gbs / peaks["hbm_gbs"], "peak_src": f"{peaks['src']} HBM copy"},

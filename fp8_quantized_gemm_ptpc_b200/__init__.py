@@ -65,6 +65,7 @@ SIGNATURES = {
     "ptpc_weight_bytes": (ctypes.c_size_t, [ctypes.c_int, _I64, _I64]),
     "ptpc_kv_cache_append": (ctypes.c_int, [_P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P]),
     "ptpc_decode_attention_workspace_size": (ctypes.c_size_t, [_I64, _I64, _I64, _I64]),
+    "ptpc_decode_attention_kernel": (ctypes.c_int, [_I64, _I64, _I64, _I64]),
     "ptpc_decode_attention": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I64,
                                              _I64, _I64, ctypes.c_float, _P, _P, _SZ, _P]),
     "ptpc_act_row_amax": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P]),
@@ -550,6 +551,15 @@ def kv_cache_append(K, V, slots, k_cache, v_cache, k_scale, v_scale):
     _check("ptpc_kv_cache_append",
            lib.ptpc_kv_cache_append(_ptr(K), _ptr(V), _ptr(slots), T, H, D, bs, nb, _ptr(k_cache), _ptr(v_cache),
                                     _ptr(k_scale), _ptr(v_scale), _stream(K.device)))
+
+
+def decode_attention_kernel(Hq: int, Hkv: int, D: int, block_size: int) -> str:
+    """The decode-attention kernel the library runs for this shape: "mma"
+    (warp-level tensor-core tiles) or "tc" (tensor-memory MMAs)."""
+    k = int(lib.ptpc_decode_attention_kernel(Hq, Hkv, D, block_size))
+    if k == 0:
+        raise ValueError("unsupported attention shape")
+    return "tc" if k == 2 else "mma"
 
 
 def decode_attention(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, max_context: int,

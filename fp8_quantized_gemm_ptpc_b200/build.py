@@ -22,8 +22,8 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIB_DIR, "libptpc.so")
-SOURCES = ["api.cu", "gemm.cu", "quant.cu", "attention.cu", "bench_probe.cu"]
-HEADERS = ["sm100.cuh", "kernels.h", "bench_probe.h"]
+SOURCES = ["api.cu", "gemm.cu", "quant.cu", "attention.cu", "attention_tc.cu", "bench_probe.cu"]
+HEADERS = ["sm100.cuh", "kernels.h", "attention_tc.h", "bench_probe.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",

@@ -8,6 +8,7 @@
 
 #include "../../include/ptpc.h"
 #include "bench_probe.h"
+#include "attention_tc.h"
 #include "kernels.h"
 
 namespace {
@@ -363,6 +364,13 @@ int ptpc_decode_attention(const void *q, const uint8_t *k_cache, const uint8_t *
                                                    (int)B, (int)Hq, (int)Hkv, (int)D, (int)block_size,
                                                    (int)max_blocks, num_blocks * block_size, (int)max_context,
                                                    softmax_scale, out, ws, (cudaStream_t)stream));
+}
+
+int ptpc_decode_attention_kernel(int64_t Hq, int64_t Hkv, int64_t D, int64_t block_size) {
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || Hq / Hkv > 16 || (D != 64 && D != 128) || block_size <= 0 ||
+      block_size > kMaxDim)
+    return 0;
+  return ptpc::attn_kernel_choice((int)D, (int)(Hq / Hkv), (int)block_size);
 }
 
 int ptpc_gemm_ksplit(int64_t T, int64_t Ci, int64_t Co) {

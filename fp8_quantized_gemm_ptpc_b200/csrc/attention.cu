@@ -38,11 +38,13 @@
 #include <atomic>
 #include <cstdint>
 #include <cstdlib>
+#include <string>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
+#include "attention_tc.h"
 #include "kernels.h"
 
 namespace ptpc {
@@ -628,14 +630,31 @@ int attn_chunk(int pairs, int max_context, int resident) {
   return best;
 }
 
-template <int D, int NH>
-cudaError_t launch_attn(AttnParams p, int B, int max_context, __nv_bfloat16 *out, cudaStream_t st) {
-  const int chunk = attn_chunk(B * p.Hkv, max_context, attn_resident<D, NH>());
-  p.splits = (std::max(max_context, 1) + chunk - 1) / chunk;
-  cudaError_t e = chunk == 2048   ? launch_attn_chunk<D, 2048, NH>(p, B, st)
-                  : chunk == 1024 ? launch_attn_chunk<D, 1024, NH>(p, B, st)
-                                  : launch_attn_chunk<D, 512, NH>(p, B, st);
-  if (e != cudaSuccess) return e;
+// PTPC_FORCE_ATTN_KERNEL = mma | tc (tuning and tests only): the warp-level
+// kernel above or the tensor-memory kernel of attention_tc.cu where it
+// applies.  Read at the first launch, or again by attn_reload_tuning.
+constexpr int kAttnKernelAuto = 0, kAttnKernelMma = 1, kAttnKernelTc = 2;
+std::atomic<int> g_attn_kernel{-1};
+
+int read_attn_kernel() {
+  const char *v = std::getenv("PTPC_FORCE_ATTN_KERNEL");
+  if (v == nullptr) return kAttnKernelAuto;
+  const std::string s(v);
+  return s == "mma" ? kAttnKernelMma : s == "tc" ? kAttnKernelTc : kAttnKernelAuto;
+}
+
+bool attn_use_tc(int D, int G, int block_size) {
+  int k = g_attn_kernel.load(std::memory_order_relaxed);
+  if (k < 0) {
+    k = read_attn_kernel();
+    g_attn_kernel.store(k, std::memory_order_relaxed);
+  }
+  if (!attn_tc_supported(D, G, block_size)) return false;
+  return k == kAttnKernelTc;
+}
+
+template <int D>
+cudaError_t launch_attn_combine(const AttnParams &p, int B, __nv_bfloat16 *out, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(B * p.Hq);
   cfg.blockDim = dim3(D);
@@ -649,16 +668,46 @@ cudaError_t launch_attn(AttnParams p, int B, int max_context, __nv_bfloat16 *out
                             (const float *)p.part_acc, p.splits, out);
 }
 
+template <int D, int NH>
+cudaError_t launch_attn(AttnParams p, int B, int max_context, __nv_bfloat16 *out, cudaStream_t st) {
+  const int chunk = attn_chunk(B * p.Hkv, max_context, attn_resident<D, NH>());
+  p.splits = (std::max(max_context, 1) + chunk - 1) / chunk;
+  cudaError_t e = chunk == 2048   ? launch_attn_chunk<D, 2048, NH>(p, B, st)
+                  : chunk == 1024 ? launch_attn_chunk<D, 1024, NH>(p, B, st)
+                                  : launch_attn_chunk<D, 512, NH>(p, B, st);
+  if (e != cudaSuccess) return e;
+  return launch_attn_combine<D>(p, B, out, st);
+}
+
+cudaError_t launch_attn_tc_and_combine(AttnParams p, int B, int max_context, uint32_t *status, __nv_bfloat16 *out,
+                                       cudaStream_t st) {
+  const int chunk = attn_chunk(B * p.Hkv, max_context, attn_tc_resident());
+  p.splits = (std::max(max_context, 1) + chunk - 1) / chunk;
+  cudaError_t e = launch_attn_tc(p.q, p.kc, p.vc, p.ks, p.vs, p.block_tables, p.context_lens, B, p.Hq, p.Hkv,
+                                 p.block_size, p.max_blocks, p.num_slots, p.bs_magic, chunk, p.splits, p.scale_log2,
+                                 p.part_ml, p.part_acc, status, st);
+  if (e != cudaSuccess) return e;
+  return launch_attn_combine<128>(p, B, out, st);
+}
+
 }  // namespace
 
-void attn_reload_tuning() { g_attn_chunk.store(read_attn_chunk(), std::memory_order_relaxed); }
+int attn_kernel_choice(int D, int G, int block_size) { return attn_use_tc(D, G, block_size) ? 2 : 1; }
+
+void attn_reload_tuning() {
+  g_attn_chunk.store(read_attn_chunk(), std::memory_order_relaxed);
+  g_attn_kernel.store(read_attn_kernel(), std::memory_order_relaxed);
+}
 
 // The most chunks a launch can split a context into (the workspace bound).
 int attn_splits(int max_context) { return max_context <= 0 ? 1 : (max_context + kAttnChunkMin - 1) / kAttnChunkMin; }
 
+// The device status word (256 bytes reserved), then the partial results.
+constexpr size_t kAttnStatusBytes = 256;
+
 size_t attn_workspace_bytes(int B, int Hq, int D, int max_context) {
   const size_t n = (size_t)B * Hq * attn_splits(max_context);
-  return n * 2 * sizeof(float) + n * D * sizeof(float);
+  return kAttnStatusBytes + n * 2 * sizeof(float) + n * D * sizeof(float);
 }
 
 cudaError_t launch_decode_attention(const void *q, const uint8_t *kc, const uint8_t *vc, const float *ks,
@@ -687,9 +736,11 @@ cudaError_t launch_decode_attention(const void *q, const uint8_t *kc, const uint
   p.scale_log2 = softmax_scale * 1.4426950408889634f;
   // partial results of up to attn_splits(max_context) chunks a head
   const size_t n = (size_t)B * Hq * attn_splits(max_context);
-  p.part_ml = static_cast<float *>(ws);
-  p.part_acc = static_cast<float *>(ws) + n * 2;
+  uint32_t *status = static_cast<uint32_t *>(ws);
+  p.part_ml = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kAttnStatusBytes);
+  p.part_acc = p.part_ml + n * 2;
   __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(out);
+  if (attn_use_tc(D, p.G, block_size)) return launch_attn_tc_and_combine(p, B, max_context, status, o, st);
   if (D == 64) return p.G > 8 ? launch_attn<64, 2>(p, B, max_context, o, st) : launch_attn<64, 1>(p, B, max_context, o, st);
   if (D == 128) return p.G > 8 ? launch_attn<128, 2>(p, B, max_context, o, st) : launch_attn<128, 1>(p, B, max_context, o, st);
   return cudaErrorInvalidValue;

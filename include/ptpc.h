@@ -337,7 +337,8 @@ PTPC_API int ptpc_kv_cache_append(const void *K_dev, const void *V_dev, const in
                                   uint8_t *k_cache_dev, uint8_t *v_cache_dev, float *k_scale_dev,
                                   float *v_scale_dev, void *stream);
 
-/* Workspace bytes of ptpc_decode_attention (0 on invalid arguments). */
+/* Workspace bytes of ptpc_decode_attention (0 on invalid arguments): the
+ * device status word (first 256 bytes) and the chunks' partial results. */
 PTPC_API size_t ptpc_decode_attention_workspace_size(int64_t B, int64_t Hq, int64_t D, int64_t max_context);
 
 /* Decode attention (one query per sequence) over the FP8 cache:
@@ -358,13 +359,30 @@ PTPC_API size_t ptpc_decode_attention_workspace_size(int64_t B, int64_t Hq, int6
  *   ws_dev: ptpc_decode_attention_workspace_size(B, Hq, D, max_context)
  *   bytes (the context is split into chunks of 512, 1024 or 2048 positions,
  *   chosen per launch to fill the GPU, whose partial results are combined by
- *   a second kernel). */
+ *   a second kernel).  It starts with the device status word: the
+ *   tensor-memory kernel (see ptpc_decode_attention_kernel) sets a bit there
+ *   when one of its bounded waits runs out, which ptpc_get_device_status
+ *   reports; the word must be zero before the first call (a zeroed
+ *   workspace). */
 PTPC_API int ptpc_decode_attention(const void *q_dev, const uint8_t *k_cache_dev, const uint8_t *v_cache_dev,
                                    const float *k_scale_dev, const float *v_scale_dev,
                                    const int32_t *block_tables_dev, const int32_t *context_lens_dev, int64_t B,
                                    int64_t Hq, int64_t Hkv, int64_t D, int64_t block_size, int64_t num_blocks,
                                    int64_t max_blocks, int64_t max_context, float softmax_scale, void *out_dev,
                                    void *ws_dev, size_t ws_bytes, void *stream);
+
+/* Which decode-attention kernel ptpc_decode_attention runs for a shape on
+ * this library: 1 the warp-level kernel (mma.sync tensor-core tiles, every
+ * supported shape), 2 the kernel on the fifth-generation tensor cores
+ * (tcgen05 MMAs into tensor memory, TMA loads), which takes D = 128, groups
+ * of at most 8 query heads a KV head and block sizes that are multiples of 8
+ * when selected with PTPC_FORCE_ATTN_KERNEL=tc (PTPC_FORCE_ATTN_KERNEL=mma
+ * forces kernel 1; read at the first launch or by
+ * ptpc_reload_tuning_overrides).  Both compute the same function; the
+ * tensor-memory kernel multiplies P, written as two E4M3 terms (8
+ * significant bits), by the E4M3 V codes, where the warp-level kernel uses
+ * f16 P.  0 on invalid arguments. */
+PTPC_API int ptpc_decode_attention_kernel(int64_t Hq, int64_t Hkv, int64_t D, int64_t block_size);
 
 /* ------------------------------------------------------------------------- */
 /* Measurement-only entry points: the comparison paths the page describes.  */

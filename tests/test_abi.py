@@ -174,7 +174,7 @@ def test_kv_cache_argument_checks(ptpc):
     bad = list(args); bad[3] = 0
     assert ap(*bad) == ptpc.OK
     wsz = lambda *a: call(ptpc, "ptpc_decode_attention_workspace_size", *a)
-    assert wsz(32, 64, 128, 4096) == 32 * 64 * 8 * (2 + 128) * 4
+    assert wsz(32, 64, 128, 4096) == 256 + 32 * 64 * 8 * (2 + 128) * 4   # status word, then the chunks
     assert wsz(32, 64, 96, 4096) == 0
     at = lambda *a: call(ptpc, "ptpc_decode_attention", *a)
     need = wsz(2, 16, 128, 100)
@@ -196,3 +196,29 @@ def test_tensor_map_cache_logic(ptpc):
     shape, emptying at capacity, failed encodes) on a private instance with a
     stand-in encoder: no GPU needed."""
     assert call(ptpc, "ptpc_bench_map_cache_selftest") == ptpc.OK
+
+
+def test_decode_attention_kernel_choice(ptpc, monkeypatch):
+    """Which decode-attention kernel a shape runs: the warp-level kernel by
+    default, the tensor-memory kernel under the override for the shapes it
+    takes (D = 128, groups of at most 8, blocks of a multiple of 8), 0 for
+    invalid arguments.  Host logic only."""
+    k = lambda *a: call(ptpc, "ptpc_decode_attention_kernel", *a)
+    try:
+        monkeypatch.delenv("PTPC_FORCE_ATTN_KERNEL", raising=False)
+        ptpc.reload_tuning_overrides()
+        assert k(64, 8, 128, 16) == 1
+        monkeypatch.setenv("PTPC_FORCE_ATTN_KERNEL", "tc")
+        ptpc.reload_tuning_overrides()
+        assert k(64, 8, 128, 16) == 2 and k(8, 8, 128, 8) == 2 and k(24, 3, 128, 48) == 2
+        assert k(64, 8, 64, 16) == 1                # D = 64
+        assert k(128, 8, 128, 16) == 1              # group of 16
+        assert k(64, 8, 128, 12) == 1               # block of 12 positions
+        assert k(12, 8, 128, 16) == 0 and k(64, 0, 128, 16) == 0 and k(64, 8, 96, 16) == 0
+        assert k(64, 8, 128, 0) == 0
+        monkeypatch.setenv("PTPC_FORCE_ATTN_KERNEL", "mma")
+        ptpc.reload_tuning_overrides()
+        assert k(64, 8, 128, 16) == 1
+    finally:
+        monkeypatch.delenv("PTPC_FORCE_ATTN_KERNEL", raising=False)
+        ptpc.reload_tuning_overrides()

@@ -2,9 +2,12 @@
 kernel's codes and scales bit for bit (the per-token rule on every
 (token, KV head) vector), and decode attention over the paged cache within
 |gpu - ref| <= 1e-2 |ref| + 1e-3 rms(ref) of the oracle's fp64 attention,
-over context lengths around the 16-position tiles and 512-position chunks,
-GQA groups of 1 to 16 query heads, head sizes 64 and 128, and block tables
-with missing entries."""
+over context lengths around the 16- and 128-position tiles and the
+512-position chunks, GQA groups of 1 to 16 query heads, head sizes 64 and
+128, and block tables with missing entries.  Every attention case runs on
+both kernels: the warp-level one ("mma") and the tensor-memory one ("tc",
+for the shapes it takes; the others fall back to "mma", which the test
+checks)."""
 import math
 
 import numpy as np
@@ -24,15 +27,42 @@ def ptpc():
     return p
 
 
-def make_kv(T, H, D, seed):
+@pytest.fixture(params=["mma", "tc"])
+def kernel(request, ptpc, monkeypatch):
+    monkeypatch.setenv("PTPC_FORCE_ATTN_KERNEL", request.param)
+    ptpc.reload_tuning_overrides()
+    yield request.param
+    monkeypatch.delenv("PTPC_FORCE_ATTN_KERNEL")
+    ptpc.reload_tuning_overrides()
+
+
+def expect_kernel(ptpc, kernel, Hq, Hkv, D, bs):
+    tc_shape = D == 128 and Hq // Hkv <= 8 and bs % 8 == 0
+    assert ptpc.decode_attention_kernel(Hq, Hkv, D, bs) == ("tc" if kernel == "tc" and tc_shape else "mma")
+
+
+def run_attention(ptpc, q, kc, vc, ksc, vsc, tables, lens, max_ctx, scale):
+    """decode_attention through an explicit zeroed workspace whose device
+    status word must still be clear afterwards."""
+    B, Hq, D = q.shape
+    ws = ptpc.Workspace(ptpc.lib.ptpc_decode_attention_workspace_size(B, Hq, D, max_ctx), "cuda")
+    out = ptpc.decode_attention(to_dev_bf16(q), kc, vc, ksc, vsc, torch.from_numpy(tables).cuda(),
+                                torch.tensor(lens, dtype=torch.int32, device="cuda"), max_ctx, scale, ws=ws)
+    assert ptpc.device_status(ws) == 0
+    return from_dev_bf16(out)
+
+
+def make_kv(T, H, D, seed, ramp=0.0):
     rng = np.random.Generator(np.random.PCG64(seed))
     x = rng.standard_normal((T, H, D)).astype(np.float32)
     x *= rng.lognormal(0.0, 1.0, size=(T, H, 1)).astype(np.float32)
     x[:, :, rng.choice(D, 2, replace=False)] *= 20.0          # a few outlier channels per head
+    if ramp:
+        x *= (1.0 + ramp * np.arange(T, dtype=np.float32))[:, None, None]
     return synthetic.to_bf16_bits(x)
 
 
-def build_cache(ptpc, lens, Hkv, D, bs, seed, holes=False):
+def build_cache(ptpc, lens, Hkv, D, bs, seed, holes=False, ramp=0.0):
     """Random block tables, K/V appended through the library; returns device
     caches and the oracle's copies."""
     rng = np.random.Generator(np.random.PCG64(seed))
@@ -51,8 +81,8 @@ def build_cache(ptpc, lens, Hkv, D, bs, seed, holes=False):
         for pos in range(l):
             slots.append(tables[b, pos // bs] * bs + pos % bs)
     T = len(slots)
-    K = make_kv(max(T, 1), Hkv, D, seed + 1)[:T]
-    V = make_kv(max(T, 1), Hkv, D, seed + 2)[:T]
+    K = make_kv(max(T, 1), Hkv, D, seed + 1, ramp)[:T]
+    V = make_kv(max(T, 1), Hkv, D, seed + 2, ramp)[:T]
     kc = torch.zeros((nb, bs, Hkv, D), dtype=torch.uint8, device="cuda")
     vc = torch.zeros_like(kc)
     ksc = torch.zeros((nb, bs, Hkv), dtype=torch.float32, device="cuda")
@@ -104,9 +134,11 @@ def test_append_bit_exact(ptpc):
     ([33, 700], 16, 16, 128, 32),
     ([257, 1500], 32, 2, 64, 16),
     ([0, 5, 2049], 28, 4, 128, 16),
+    ([1, 127, 128, 129, 255, 256, 1000, 2047], 24, 3, 128, 8),
+    ([130, 641], 12, 12, 128, 48),
 ])
-def test_decode_attention(ptpc, lens, Hq, Hkv, D, bs):
-    _attention_case(ptpc, lens, Hq, Hkv, D, bs)
+def test_decode_attention(ptpc, kernel, lens, Hq, Hkv, D, bs):
+    _attention_case(ptpc, kernel, lens, Hq, Hkv, D, bs)
 
 
 @pytest.mark.parametrize("chunk", ["1024", "2048"])
@@ -115,21 +147,22 @@ def test_decode_attention(ptpc, lens, Hq, Hkv, D, bs):
     ([257, 1500, 3000], 32, 2, 64, 24),
     ([0, 5, 2049], 28, 4, 128, 16),
 ])
-def test_decode_attention_chunk_sizes(ptpc, monkeypatch, chunk, lens, Hq, Hkv, D, bs):
+def test_decode_attention_chunk_sizes(ptpc, monkeypatch, kernel, chunk, lens, Hq, Hkv, D, bs):
     """The larger context chunks a CTA can take (chosen by the launch for
     long contexts on many sequences), forced on small cases; a block size
     that is not a power of two exercises the exact quotient."""
     monkeypatch.setenv("PTPC_FORCE_ATTN_CHUNK", chunk)
     ptpc.reload_tuning_overrides()
     try:
-        _attention_case(ptpc, lens, Hq, Hkv, D, bs)
+        _attention_case(ptpc, kernel, lens, Hq, Hkv, D, bs)
     finally:
         monkeypatch.delenv("PTPC_FORCE_ATTN_CHUNK")
         ptpc.reload_tuning_overrides()
 
 
-def _attention_case(ptpc, lens, Hq, Hkv, D, bs):
-    dev, ref = build_cache(ptpc, lens, Hkv, D, bs, seed=sum(lens) + Hq, holes=True)
+def _attention_case(ptpc, kernel, lens, Hq, Hkv, D, bs, ramp=0.0):
+    expect_kernel(ptpc, kernel, Hq, Hkv, D, bs)
+    dev, ref = build_cache(ptpc, lens, Hkv, D, bs, seed=sum(lens) + Hq, holes=True, ramp=ramp)
     kc, vc, ksc, vsc, tables = dev
     rk, rv, rks, rvs = ref
     assert np.array_equal(kc.cpu().numpy(), rk) and np.array_equal(vsc.cpu().numpy(), rvs)
@@ -138,10 +171,8 @@ def _attention_case(ptpc, lens, Hq, Hkv, D, bs):
     q = synthetic.to_bf16_bits(rng.standard_normal((B, Hq, D)).astype(np.float32) * 2.0)
     scale = 1.0 / math.sqrt(D)
     max_ctx = max(lens)
-    out = ptpc.decode_attention(to_dev_bf16(q), kc, vc, ksc, vsc, torch.from_numpy(tables).cuda(),
-                                torch.tensor(lens, dtype=torch.int32, device="cuda"), max_ctx, scale)
     # the oracle over the same table (missing entries: positions left out)
-    got = from_dev_bf16(out)
+    got = run_attention(ptpc, q, kc, vc, ksc, vsc, tables, lens, max_ctx, scale)
     for b in range(B):
         L = lens[b]
         pos = [p for p in range(L) if tables[b, p // bs] >= 0]
@@ -160,23 +191,30 @@ def _attention_case(ptpc, lens, Hq, Hkv, D, bs):
         assert_gemm_close(got[b:b + 1], r, f"attention b={b} L={L} Hq={Hq} Hkv={Hkv} D={D}")
 
 
-def test_decode_attention_70b_shape(ptpc):
+def test_decode_attention_growing_scores(ptpc, kernel):
+    """Keys and values whose size grows along the context (x 1 + t / 40):
+    the running maximum of every head and the largest value scale move many
+    times within a chunk, so the kernels rescale their accumulators often."""
+    _attention_case(ptpc, kernel, [300, 1000, 2100], 16, 2, 128, 16, ramp=1.0 / 40)
+
+
+def test_decode_attention_70b_shape(ptpc, kernel):
     """Llama-3.1-70B attention at decode: 64 query heads on 8 KV heads, D =
     128, 16-position blocks; a batch of mixed context lengths."""
+    expect_kernel(ptpc, kernel, 64, 8, 128, 16)
     lens = [4096, 1, 3000, 2048, 777, 4095]
     dev, ref = build_cache(ptpc, lens, 8, 128, 16, seed=70)
     kc, vc, ksc, vsc, tables = dev
     rk, rv, rks, rvs = ref
     rng = np.random.Generator(np.random.PCG64(12))
     q = synthetic.to_bf16_bits(rng.standard_normal((len(lens), 64, 128)).astype(np.float32))
-    out = ptpc.decode_attention(to_dev_bf16(q), kc, vc, ksc, vsc, torch.from_numpy(tables).cuda(),
-                                torch.tensor(lens, dtype=torch.int32, device="cuda"), 4096, 1 / math.sqrt(128))
+    got = run_attention(ptpc, q, kc, vc, ksc, vsc, tables, lens, 4096, 1 / math.sqrt(128))
     r = oracle.decode_attention_reference(q, rk, rks, rv, rvs, tables, lens, 16, 1 / math.sqrt(128))
-    assert_gemm_close(from_dev_bf16(out), r, "70B decode attention")
+    assert_gemm_close(got, r, "70B decode attention")
 
 
 @pytest.mark.parametrize("q_scale", [1e-39, 1e-20, 1e20, 3e37])
-def test_decode_attention_query_range(ptpc, q_scale):
+def test_decode_attention_query_range(ptpc, kernel, q_scale):
     """Query vectors far from unit size (bf16 subnormals up to near the bf16
     maximum, times a softmax scale that keeps the scores finite): the
     power-of-two scale of the query's two E4M3 terms keeps them in range."""
@@ -188,7 +226,6 @@ def test_decode_attention_query_range(ptpc, q_scale):
     qf = rng.standard_normal((len(lens), Hq, D)).astype(np.float32) * np.float32(q_scale)
     q = synthetic.to_bf16_bits(qf)
     scale = float(min(1.0, 1.0 / (q_scale * math.sqrt(D))))
-    out = ptpc.decode_attention(to_dev_bf16(q), kc, vc, ksc, vsc, torch.from_numpy(tables).cuda(),
-                                torch.tensor(lens, dtype=torch.int32, device="cuda"), max(lens), scale)
+    got = run_attention(ptpc, q, kc, vc, ksc, vsc, tables, lens, max(lens), scale)
     r = oracle.decode_attention_reference(q, rk, rks, rv, rvs, tables, lens, bs, scale)
-    assert_gemm_close(from_dev_bf16(out), r, f"attention, |q| ~ {q_scale}")
+    assert_gemm_close(got, r, f"attention, |q| ~ {q_scale}")
