@@ -556,8 +556,8 @@ __global__ void __launch_bounds__(D) decode_attn_combine_kernel(const float *__r
 // Context chunk of a CTA: 512, 1024 or 2048 positions.  Larger chunks pay the
 // CTA's start (block table, query terms) and end (the warps' combine) over
 // more tiles but leave fewer CTAs to fill the GPU; the launch takes the chunk
-// with the fewest rounds of resident CTAs times positions a CTA (ties: the
-// larger chunk).
+// with the fewest rounds of resident CTAs times (positions a CTA + `fixed`,
+// the CTA's start and end counted in positions) (ties: the larger chunk).
 constexpr int kAttnChunkMin = 512;
 
 template <int D, int CHUNK, int NH>
@@ -610,7 +610,7 @@ int read_attn_chunk() {
   return c == 512 || c == 1024 || c == 2048 ? c : 0;
 }
 
-int attn_chunk(int pairs, int max_context, int resident) {
+int attn_chunk(int pairs, int max_context, int resident, int fixed = 0) {
   int forced = g_attn_chunk.load(std::memory_order_relaxed);
   if (forced < 0) {
     forced = read_attn_chunk();
@@ -621,7 +621,7 @@ int attn_chunk(int pairs, int max_context, int resident) {
   long long best_cost = -1;
   for (int chunk = kAttnChunkMin; chunk <= 2048; chunk *= 2) {
     const long long ctas = (long long)pairs * ((std::max(max_context, 1) + chunk - 1) / chunk);
-    const long long cost = (ctas + resident - 1) / resident * chunk;
+    const long long cost = (ctas + resident - 1) / resident * (chunk + fixed);
     if (best_cost < 0 || cost <= best_cost) {
       best = chunk;
       best_cost = cost;
@@ -630,9 +630,12 @@ int attn_chunk(int pairs, int max_context, int resident) {
   return best;
 }
 
-// PTPC_FORCE_ATTN_KERNEL = mma | tc (tuning and tests only): the warp-level
-// kernel above or the tensor-memory kernel of attention_tc.cu where it
-// applies.  Read at the first launch, or again by attn_reload_tuning.
+// Decode attention runs the tensor-memory kernel of attention_tc.cu where it
+// applies (D = 128, groups of at most 8 query heads, blocks of a multiple of
+// 8 positions) and the warp-level kernel above otherwise.
+// PTPC_FORCE_ATTN_KERNEL = mma | tc (tuning and tests only) forces one (tc
+// only where it applies).  Read at the first launch, or again by
+// attn_reload_tuning.
 constexpr int kAttnKernelAuto = 0, kAttnKernelMma = 1, kAttnKernelTc = 2;
 std::atomic<int> g_attn_kernel{-1};
 
@@ -650,7 +653,7 @@ bool attn_use_tc(int D, int G, int block_size) {
     g_attn_kernel.store(k, std::memory_order_relaxed);
   }
   if (!attn_tc_supported(D, G, block_size)) return false;
-  return k == kAttnKernelTc;
+  return k != kAttnKernelMma;
 }
 
 template <int D>
@@ -681,7 +684,9 @@ cudaError_t launch_attn(AttnParams p, int B, int max_context, __nv_bfloat16 *out
 
 cudaError_t launch_attn_tc_and_combine(AttnParams p, int B, int max_context, uint32_t *status, __nv_bfloat16 *out,
                                        cudaStream_t st) {
-  const int chunk = attn_chunk(B * p.Hkv, max_context, attn_tc_resident());
+  // the tensor-memory kernel's start (barriers, tensor memory, the first
+  // tiles' load latency) costs about three 128-position tiles
+  const int chunk = attn_chunk(B * p.Hkv, max_context, attn_tc_resident(), 384);
   p.splits = (std::max(max_context, 1) + chunk - 1) / chunk;
   cudaError_t e = launch_attn_tc(p.q, p.kc, p.vc, p.ks, p.vs, p.block_tables, p.context_lens, B, p.Hq, p.Hkv,
                                  p.block_size, p.max_blocks, p.num_slots, p.bs_magic, chunk, p.splits, p.scale_log2,

@@ -7,8 +7,14 @@
 //
 // A CTA takes one (sequence, KV head) and a chunk of context positions, in
 // tiles of 128 positions.  Warp 0 loads a tile's K and V codes with TMA (a
-// 3-D tensor map over [slot][head][d], boxes of 8 positions into 128-byte
-// swizzled tiles) and its scales with cp.async, into a ring of stages.  Warp 1
+// 3-D tensor map over [slot][head][d], boxes of 16 positions, or 8 where the
+// cache blocks hold an odd multiple of 8, into 128-byte swizzled tiles, one
+// box a lane) into two rings of stages, one for K (a stage is free again once
+// the tile's QK MMAs are done) and one for V (free once its PV MMAs are
+// done), so neither ring waits for the other half's work.  It issues nothing
+// else and runs as far ahead as the rings allow (a TMA instruction takes
+// tens of cycles to issue whatever its box, hence the largest box a block
+// allows).  Warp 1
 // issues the MMAs from one thread:
 //   S^T = K Q^T    (M = 128 positions, N = 16, K = d; A = the K tile, B = q)
 //   O^T += V^T P^T (M = 128 values of d, N = 2 x 16, K = positions; A = the
@@ -21,7 +27,8 @@
 // for P, term 3 in a second MMA), so the terms share the MMAs.  The cache
 // codes go in as they are, with no conversion.
 // Warps 2-5 (thread i = tensor-memory lane i = position i of the tile, and
-// value d = i of O) run the online softmax in base 2: key scales, masking,
+// value d = i of O; each loads its position's two scales two tiles ahead)
+// run the online softmax in base 2: key scales, masking,
 // exponentials, P written to shared memory.  The running maximum and the
 // value-scale unit are lazy: a reference maximum per head moves (and O, in
 // tensor memory, is rescaled) only when a score exceeds it by more than 8
@@ -53,7 +60,7 @@ namespace ptpc {
 namespace {
 
 constexpr int kTcThreads = 192;  // warp 0 producer, warp 1 MMA issuer, warps 2-5 softmax
-constexpr int kTcStages = 3;
+constexpr int kTcStages = 3;   // of each ring
 constexpr int kTcTile = 128;     // positions a tile
 constexpr int kTcD = 128;
 constexpr int kTcKV = kTcTile * kTcD;  // bytes of one K or V tile
@@ -69,6 +76,7 @@ struct TcParams {
   const int32_t *block_tables;  // [B, max_blocks]
   const int32_t *context_lens;  // [B]
   int Hq, Hkv, G, block_size, max_blocks, splits, chunk;
+  int box_rows;                 // positions a TMA box: 16, or 8 (a divisor of block_size)
   uint64_t bs_magic;            // ceil(2^64 / block_size)
   int64_t num_slots;
   float scale_log2;
@@ -81,15 +89,14 @@ struct TcSmem {
   static constexpr int K = 0;                                    // [stage] 16 KB
   static constexpr int V = K + kTcStages * kTcKV;                // [stage] 16 KB
   static constexpr int Q = V + kTcStages * kTcKV;                // 16 rows x 128 B: hi terms, then lo terms
-  static constexpr int P = Q + 16 * 128;                         // [buffer][plane] 128 positions x 16 B
+  static constexpr int P = Q + 16 * 128;                         // [plane] 128 positions x 16 B
   static constexpr int P_PLANE = kTcTile * 16;                   // plane 0: terms 1, 2; plane 1: term 3, zeros
-  static constexpr int SCL = P + 2 * 2 * P_PLANE;                // [stage] k scales, v scales
-  static constexpr int RED = SCL + kTcStages * 2 * kTcTile * 4;  // [warp][16]: per-warp maxima, sums
+  static constexpr int RED = P + 2 * P_PLANE;                    // [warp][16]: per-warp maxima, sums
   static constexpr int SIG = RED + 4 * 16 * 4;                   // [head]: 1 / sigma of q
   static constexpr int BLK = SIG + 16 * 4;
   // then the chunk's block-table entries (size depends on the chunk), then
   // the barriers and the tensor-memory address
-  static constexpr int kBarriers = 2 * kTcStages + 3 * 2 + 2;
+  static constexpr int kBarriers = 4 * kTcStages + 3 * 2 + 2;
 };
 
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uint64_t *bar, int32_t x, int32_t y,
@@ -101,17 +108,17 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *m, uin
       : "memory");
 }
 
-__device__ __forceinline__ void cp_async4_zfill(void *dst, const void *src, bool valid) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 4 : 0)
-               : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-// The barrier tracks this thread's earlier cp.async copies (no extra arrival
-// counted: the barrier's count includes it).
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+// Non-blocking test of a phase (no suspension, unlike try_wait).
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
@@ -207,11 +214,13 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   const int nblk_max = p.chunk / 8 + 2;
   int *s_blk = reinterpret_cast<int *>(sm + TcSmem::BLK);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ((TcSmem::BLK + nblk_max * 4 + 7) & ~7));
-  uint64_t *kv_full = bars;                   // [stage]: TMA bytes + 32 cp.async arrivals + 1
-  uint64_t *kv_empty = kv_full + kTcStages;   // [stage]: the PV MMAs of the tile are done
-  uint64_t *s_full = kv_empty + kTcStages;    // [buffer]: S of a tile is in tensor memory
+  uint64_t *k_full = bars;                    // [stage]: the tile's K bytes have landed
+  uint64_t *k_empty = k_full + kTcStages;     // [stage]: the tile's QK MMAs are done
+  uint64_t *v_full = k_empty + kTcStages;     // [stage]: the tile's V bytes have landed
+  uint64_t *v_empty = v_full + kTcStages;     // [stage]: the tile's PV MMAs are done
+  uint64_t *s_full = v_empty + kTcStages;     // [buffer]: S of a tile is in tensor memory
   uint64_t *s_empty = s_full + 2;             // [buffer]: the softmax has read it (128)
-  uint64_t *p_full = s_empty + 2;             // [buffer]: P written, O corrected (128)
+  uint64_t *p_full = s_empty + 2;             // [tile parity]: P written, O corrected (128)
   uint64_t *o_done = p_full + 2;              // one phase per PV
   uint64_t *drain = o_done + 1;               // the MMA issuer's last commit
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
@@ -234,8 +243,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&kv_full[s], 1 + 32);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -250,9 +261,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     tmem_alloc(tmem_holder, kTcTmemCols);
     tmem_relinquish();
   }
-  // slot of position pos (-1: not read).  A block holds a multiple of 8
-  // positions and tiles start at multiples of 8, so the 8 positions of a TMA
-  // box share one block: the box is read whole or not at all.
+  // slot of position pos (-1: not read).  A block holds a multiple of
+  // box_rows positions and tiles start at multiples of 128, so the positions
+  // of a TMA box share one block: the box is read whole or not at all.
   auto slot_of = [&](int pos) -> int64_t {
     if (pos >= c1) return -1;
     const int bi = (int)__umul64hi((uint64_t)pos, p.bs_magic);
@@ -303,6 +314,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       qs[sw128_off(h + 8, col)] = (uint8_t)(lo & 0xFF);
       qs[sw128_off(h + 8, col + 1)] = (uint8_t)(lo >> 8);
     }
+    // the V ring starts zeroed: rows of boxes that are never loaded then hold
+    // zeros or an earlier tile's codes (finite), which P = 0 cancels
+    uint4 *vz = reinterpret_cast<uint4 *>(sm + TcSmem::V);
+    for (int j = t; j < kTcStages * kTcKV / 16; j += 128) vz[j] = make_uint4(0, 0, 0, 0);
     fence_async_shared();
   }
   tc_fence_before();
@@ -313,53 +328,53 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // Decisions are warp-uniform: a stage is refilled by all 32 lanes or none.
+    // Order: K of tile j + 1, then V of tile j, the order in which the MMAs
+    // free their stages (QK(j - 2) before PV(j - 3)).
+    const int nbox = kTcTile / p.box_rows;
+    const uint32_t box_bytes = (uint32_t)(p.box_rows * kTcD);
     bool ok = true;
-    int issued = 0;
-    for (int i = 0; i < ntiles; ++i) {
+    int k_issued = 0, v_issued = 0;
+    // issue one half (K or V) of tile i into its ring
+    auto issue = [&](int i, bool is_k) -> bool {
       const int s = i % kTcStages;
+      uint64_t *full = is_k ? &k_full[s] : &v_full[s];
       if (i >= kTcStages) {
-        const bool w = mbar_wait(&kv_empty[s], (uint32_t)((i / kTcStages) - 1) & 1u);
-        if (!__all_sync(0xffffffffu, w)) {
-          ok = false;
-          break;
-        }
+        uint64_t *empty = is_k ? &k_empty[s] : &v_empty[s];
+        const bool w = mbar_wait(empty, (uint32_t)((i / kTcStages) - 1) & 1u);
+        if (!__all_sync(0xffffffffu, w)) return false;
       }
-      const int base = c0 + i * kTcTile;
-      // scales: lane l takes positions 4l .. 4l+3 of the tile
-      float *sk = reinterpret_cast<float *>(sm + TcSmem::SCL + s * 2 * kTcTile * 4);
-      #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int pidx = 4 * lane + j;
-        const int64_t sl = slot_of(base + pidx);
-        const int64_t row = sl >= 0 ? sl * p.Hkv + kvh : 0;
-        cp_async4_zfill(sk + pidx, p.ks + row, sl >= 0);
-        cp_async4_zfill(sk + kTcTile + pidx, p.vs + row, sl >= 0);
+      // box j loaded by lane j; a box that is not read leaves its rows as they
+      // were.  The barrier's byte count is set before any copy is issued.
+      const int64_t s0 = lane < nbox ? slot_of(c0 + i * kTcTile + p.box_rows * lane) : -1;
+      const uint32_t boxes = __ballot_sync(0xffffffffu, s0 >= 0);
+      if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)__popc(boxes) * box_bytes);
+      __syncwarp();
+      if (s0 >= 0)
+        tma_load_3d(sm + (is_k ? TcSmem::K : TcSmem::V) + s * kTcKV + lane * (int)box_bytes, is_k ? &tmK : &tmV, full,
+                    0, kvh, (int)s0);
+      return true;
+    };
+    if (ntiles > 0) {
+      ok = issue(0, true);
+      k_issued = ok ? 1 : 0;
+    }
+    for (int j = 0; j < ntiles && ok; ++j) {
+      if (j + 1 < ntiles) {
+        ok = issue(j + 1, true);
+        if (!ok) break;
+        k_issued = j + 2;
       }
-      // codes: 16 boxes of 8 positions; a box that is not read leaves its
-      // rows as they were (the softmax masks them)
-      if (lane == 0) {
-        uint32_t bytes = 0;
-        #pragma unroll 1
-        for (int j = 0; j < 16; ++j)
-          if (slot_of(base + 8 * j) >= 0) bytes += 2 * 8 * kTcD;
-        mbar_arrive_expect_tx(&kv_full[s], bytes);
-        #pragma unroll 1
-        for (int j = 0; j < 16; ++j) {
-          const int64_t s0 = slot_of(base + 8 * j);
-          if (s0 < 0) continue;
-          tma_load_3d(sm + TcSmem::K + s * kTcKV + j * 1024, &tmK, &kv_full[s], 0, kvh, (int)s0);
-          tma_load_3d(sm + TcSmem::V + s * kTcKV + j * 1024, &tmV, &kv_full[s], 0, kvh, (int)s0);
-        }
-      }
-      cp_async_arrive_noinc(&kv_full[s]);
-      issued = i + 1;
+      ok = issue(j, false);
+      if (ok) v_issued = j + 1;
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeoutAttn);
     // every copy this warp issued completes before the CTA ends (bounded)
-    cp_async_wait_all();
-    if (lane == 0)
-      for (int i = std::max(0, issued - kTcStages); i < issued; ++i)
-        mbar_wait(&kv_full[i % kTcStages], (uint32_t)(i / kTcStages) & 1u);
+    if (lane == 0) {
+      for (int i = std::max(0, k_issued - kTcStages); i < k_issued; ++i)
+        mbar_wait(&k_full[i % kTcStages], (uint32_t)(i / kTcStages) & 1u);
+      for (int i = std::max(0, v_issued - kTcStages); i < v_issued; ++i)
+        mbar_wait(&v_full[i % kTcStages], (uint32_t)(i / kTcStages) & 1u);
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
@@ -369,7 +384,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       bool ok = true;
       auto qk = [&](int i) {
         const int s = i % kTcStages, bufi = i & 1;
-        if (!mbar_wait(&kv_full[s], (uint32_t)(i / kTcStages) & 1u)) return false;
+        if (!mbar_wait(&k_full[s], (uint32_t)(i / kTcStages) & 1u)) return false;
         if (i >= 2 && !mbar_wait(&s_empty[bufi], (uint32_t)((i >> 1) - 1) & 1u)) return false;
         tc_fence_after();
         const uint64_t ad = sw128_kmajor_desc(smem_u32(sm + TcSmem::K + s * kTcKV));
@@ -377,13 +392,15 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         #pragma unroll
         for (int kk = 0; kk < kTcD / 32; ++kk) mma_f8f6f4(d, ad + 2 * kk, qd + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
         mma_commit(&s_full[bufi]);
+        mma_commit(&k_empty[s]);
         return true;
       };
       auto pv = [&](int i) {
         const int s = i % kTcStages, bufi = i & 1;
+        if (!mbar_wait(&v_full[s], (uint32_t)(i / kTcStages) & 1u)) return false;
         if (!mbar_wait(&p_full[bufi], (uint32_t)(i >> 1) & 1u)) return false;
         tc_fence_after();
-        const uint32_t pb = smem_u32(sm + TcSmem::P + bufi * 2 * TcSmem::P_PLANE);
+        const uint32_t pb = smem_u32(sm + TcSmem::P);
         const uint32_t vb = smem_u32(sm + TcSmem::V + s * kTcKV);
         #pragma unroll
         for (int kk = 0; kk < kTcTile / 32; ++kk) {
@@ -393,14 +410,22 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           mma_f8f6f4(tmem_base + kTcColO + 16, ad, plain_mnmajor16_desc(pb + TcSmem::P_PLANE + kk * 32 * 16), idesc_pv,
                      acc);
         }
-        mma_commit(&kv_empty[s]);
+        mma_commit(&v_empty[s]);
         mma_commit(o_done);
         return true;
       };
+      // S of tile i + 1 is computed while the softmax works on tile i, but
+      // PV of tile i does not wait for tile i + 1's K codes: QK(i + 1) goes
+      // first only if they have landed.
       if (ntiles > 0) ok = qk(0);
       for (int i = 0; i < ntiles && ok; ++i) {
-        if (i + 1 < ntiles) ok = qk(i + 1);
-        if (ok) ok = pv(i);
+        const bool next = i + 1 < ntiles;
+        if (next && mbar_test(&k_full[(i + 1) % kTcStages], (uint32_t)((i + 1) / kTcStages) & 1u)) {
+          ok = qk(i + 1) && pv(i);
+        } else {
+          ok = pv(i);
+          if (ok && next) ok = qk(i + 1);
+        }
       }
       if (!ok) atomicOr(p.status, kStatusTimeoutAttn);
       // every MMA issued has completed before the CTA ends
@@ -425,7 +450,18 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
     float unit = 0.0f;  // power of two >= every value scale seen (0: none yet)
     bool ok = true;     // this thread's waits; the loop leaves only on a decision all 128 take
-    for (int i = 0; i < ntiles; ++i) {
+    // this position's key and value scales, loaded two tiles ahead (0 where
+    // the position is not read)
+    auto load_scales = [&](int i, float &k, float &v) {
+      const int64_t sl = i < ntiles ? slot_of(c0 + i * kTcTile + pidx) : -1;
+      k = sl >= 0 ? __ldg(p.ks + sl * p.Hkv + kvh) : 0.0f;
+      v = sl >= 0 ? __ldg(p.vs + sl * p.Hkv + kvh) : 0.0f;
+    };
+    // one tile; false when the 128 threads stop together.  The tile's scales
+    // kr, vr were loaded two tiles earlier: two tiles a loop turn, each with
+    // its own registers, reloaded only after use, so no register copy waits
+    // for a load in flight.
+    auto tile_step = [&](int i, const float kr, const float vr) __attribute__((always_inline)) -> bool {
       const int s = i % kTcStages, bufi = i & 1;
       const int pos = c0 + i * kTcTile + pidx;
       bool w = mbar_wait(&s_full[bufi], (uint32_t)(i >> 1) & 1u);
@@ -435,13 +471,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&s_empty[bufi]);
-      // the tile's codes and scales have landed (the MMA waited for them too)
-      w = w && mbar_wait(&kv_full[s], (uint32_t)(i / kTcStages) & 1u);
       ok = ok && w;
-      const float *sk = reinterpret_cast<const float *>(sm + TcSmem::SCL + s * 2 * kTcTile * 4);
       const bool valid = slot_of(pos) >= 0;
-      const float ksc = sk[pidx] * p.scale_log2;
-      const float vsc = valid ? sk[kTcTile + pidx] : 0.0f;
+      const float ksc = kr * p.scale_log2;
+      const float vsc = valid ? vr : 0.0f;
       float sv[8];
       bool need = vsc > unit;
       #pragma unroll
@@ -455,7 +488,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       float fac_o[8];
       bool corr = false;
       if (softmax_bar_count(need || !ok) != 0) {
-        if (!softmax_bar_all(ok)) break;
+        if (!softmax_bar_all(ok)) return false;
         // the tile's maximum per head and its largest value scale
         float tm[9];
         #pragma unroll
@@ -513,9 +546,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         w3[h / 2] = f32x2_e4m3x2((r0 - d2.x) * 16.0f, (r1 - d2.y) * 16.0f);
       }
       // PV of tile i - 1 has completed: O holds tiles 0 .. i-1 (it may be
-      // corrected) and the P buffer of tile i - 2 is free.  (PV of tile i
-      // cannot start before this tile's P, so o_done is never two phases
-      // ahead of this wait.)
+      // corrected) and the P buffer (one, in shared memory) is free again.
+      // (PV of tile i cannot start before this tile's P, so o_done is never
+      // two phases ahead of this wait.)
       if (i >= 1) {
         ok = ok && mbar_wait(o_done, (uint32_t)(i - 1) & 1u);
         tc_fence_after();
@@ -534,19 +567,38 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         tmem_wait_st();
       }
       tc_fence_before();
-      uint8_t *prow = sm + TcSmem::P + bufi * 2 * TcSmem::P_PLANE + pidx * 16;
+      uint8_t *prow = sm + TcSmem::P + pidx * 16;
       *reinterpret_cast<uint4 *>(prow) =
           make_uint4(w1[0] | (w1[1] << 16), w1[2] | (w1[3] << 16), w2[0] | (w2[1] << 16), w2[2] | (w2[3] << 16));
       *reinterpret_cast<uint4 *>(prow + TcSmem::P_PLANE) = make_uint4(w3[0] | (w3[1] << 16), w3[2] | (w3[3] << 16), 0u, 0u);
-      // a position that is not read may hold any bytes in the V tile: zero its
-      // row so that P = 0 times it is 0
-      if (!valid) {
-        uint4 *vrow = reinterpret_cast<uint4 *>(sm + TcSmem::V + s * kTcKV + pidx * 128);
-        #pragma unroll
-        for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0, 0, 0, 0);
+      // the last box of a context that ends inside it is loaded whole: its
+      // rows past the context hold whatever the cache holds there (maybe
+      // NaN codes), so they are zeroed once the box has landed (P = 0 times
+      // them must be 0).  Every other row that is not read holds zeros or an
+      // earlier tile's codes.
+      if (i == ntiles - 1 && c1 % p.box_rows != 0) {
+        ok = ok && mbar_wait(&v_full[s], (uint32_t)(i / kTcStages) & 1u);
+        if (pos >= c1 && pos < (c1 / p.box_rows + 1) * p.box_rows) {
+          uint4 *vrow = reinterpret_cast<uint4 *>(sm + TcSmem::V + s * kTcKV + pidx * 128);
+          #pragma unroll
+          for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0, 0, 0, 0);
+        }
       }
       fence_async_shared();
       mbar_arrive(&p_full[bufi]);
+      return true;
+    };
+    float k0, v0, k1, v1;
+    load_scales(0, k0, v0);
+    load_scales(1, k1, v1);
+    #pragma unroll 1
+    for (int i = 0; i < ntiles; i += 2) {
+      const float ka = k0, va = v0;
+      load_scales(i + 2, k0, v0);
+      if (!tile_step(i, ka, va)) break;
+      const float kb = k1, vb = v1;
+      load_scales(i + 3, k1, v1);
+      if (i + 1 < ntiles && !tile_step(i + 1, kb, vb)) break;
     }
     if (!ok && lane == 0) atomicOr(p.status, kStatusTimeoutAttn);
     // the last PV, then O, the sums and the maxima of the chunk
@@ -623,11 +675,12 @@ TcEncodeFn tc_encode_fn() {
 // 3-D map of a cache [slots][Hkv][128] of bytes: boxes of 128 bytes x 1 head x
 // 8 slots, 128-byte swizzle.  Cached for the last few caches (a decode step
 // calls the kernel once a layer on the same caches).
-bool tc_cache_map(CUtensorMap *m, const void *base, int Hkv, int64_t slots) {
+bool tc_cache_map(CUtensorMap *m, const void *base, int Hkv, int64_t slots, int box_rows) {
   struct Entry {
     const void *base;
     int Hkv;
     int64_t slots;
+    int box_rows;
     CUtensorMap map;
   };
   static std::mutex mu;
@@ -635,7 +688,7 @@ bool tc_cache_map(CUtensorMap *m, const void *base, int Hkv, int64_t slots) {
   static int next = 0;
   std::lock_guard<std::mutex> lock(mu);
   for (const Entry &e : cache)
-    if (e.base == base && e.Hkv == Hkv && e.slots == slots) {
+    if (e.base == base && e.Hkv == Hkv && e.slots == slots && e.box_rows == box_rows) {
       *m = e.map;
       return true;
     }
@@ -643,13 +696,13 @@ bool tc_cache_map(CUtensorMap *m, const void *base, int Hkv, int64_t slots) {
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)kTcD, (cuuint64_t)Hkv, (cuuint64_t)slots};
   cuuint64_t strides[2] = {(cuuint64_t)kTcD, (cuuint64_t)kTcD * (cuuint64_t)Hkv};
-  cuuint32_t box[3] = {(cuuint32_t)kTcD, 1, 8};
+  cuuint32_t box[3] = {(cuuint32_t)kTcD, 1, (cuuint32_t)box_rows};
   cuuint32_t es[3] = {1, 1, 1};
   if (fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, es,
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
-  cache[next] = Entry{base, Hkv, slots, *m};
+  cache[next] = Entry{base, Hkv, slots, box_rows, *m};
   next = (next + 1) % 16;
   return true;
 }
@@ -688,8 +741,10 @@ cudaError_t launch_attn_tc(const void *q, const uint8_t *kc, const uint8_t *vc, 
                            cudaStream_t st) {
   if (chunk % kTcTile != 0 || chunk > 2048 || Hq % Hkv != 0 || !attn_tc_supported(kTcD, Hq / Hkv, block_size))
     return cudaErrorInvalidValue;
+  const int box_rows = block_size % 16 == 0 ? 16 : 8;
   CUtensorMap tmK, tmV;
-  if (!tc_cache_map(&tmK, kc, Hkv, num_slots) || !tc_cache_map(&tmV, vc, Hkv, num_slots)) return cudaErrorInvalidValue;
+  if (!tc_cache_map(&tmK, kc, Hkv, num_slots, box_rows) || !tc_cache_map(&tmV, vc, Hkv, num_slots, box_rows))
+    return cudaErrorInvalidValue;
   TcParams p = {};
   p.q = static_cast<const __nv_bfloat16 *>(q);
   p.ks = ks;
@@ -700,6 +755,7 @@ cudaError_t launch_attn_tc(const void *q, const uint8_t *kc, const uint8_t *vc, 
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
   p.block_size = block_size;
+  p.box_rows = box_rows;
   p.max_blocks = max_blocks;
   p.splits = splits;
   p.chunk = chunk;

@@ -354,7 +354,9 @@ PTPC_API size_t ptpc_decode_attention_workspace_size(int64_t B, int64_t Hq, int6
  *   (0 for a sequence with no position), computed in fp32: q K^T from
  *   E4M3 tensor-core products of the K codes with q written as two E4M3
  *   terms (exact for every bf16 q whose first term is a normal number, see
- *   the kernel), P V from f16 products of the exactly decoded V codes.
+ *   the kernel), P V from tensor-core products of the V codes with P written
+ *   as three E4M3 terms (or, in the warp-level kernel, f16 P times the
+ *   exactly decoded V codes; see ptpc_decode_attention_kernel).
  *   out_dev bf16 [B, Hq, D].
  *   ws_dev: ptpc_decode_attention_workspace_size(B, Hq, D, max_context)
  *   bytes (the context is split into chunks of 512, 1024 or 2048 positions,
@@ -372,16 +374,16 @@ PTPC_API int ptpc_decode_attention(const void *q_dev, const uint8_t *k_cache_dev
                                    void *ws_dev, size_t ws_bytes, void *stream);
 
 /* Which decode-attention kernel ptpc_decode_attention runs for a shape on
- * this library: 1 the warp-level kernel (mma.sync tensor-core tiles, every
- * supported shape), 2 the kernel on the fifth-generation tensor cores
- * (tcgen05 MMAs into tensor memory, TMA loads), which takes D = 128, groups
- * of at most 8 query heads a KV head and block sizes that are multiples of 8
- * when selected with PTPC_FORCE_ATTN_KERNEL=tc (PTPC_FORCE_ATTN_KERNEL=mma
- * forces kernel 1; read at the first launch or by
- * ptpc_reload_tuning_overrides).  Both compute the same function; the
- * tensor-memory kernel multiplies P, written as two E4M3 terms (8
- * significant bits), by the E4M3 V codes, where the warp-level kernel uses
- * f16 P.  0 on invalid arguments. */
+ * this library: 2 the kernel on the fifth-generation tensor cores (tcgen05
+ * MMAs into tensor memory, TMA loads), for D = 128, groups of at most 8
+ * query heads a KV head and block sizes that are multiples of 8; 1 the
+ * warp-level kernel (mma.sync tensor-core tiles) for every other supported
+ * shape.  PTPC_FORCE_ATTN_KERNEL=mma forces kernel 1 and =tc asks for
+ * kernel 2 where it applies (read at the first launch or by
+ * ptpc_reload_tuning_overrides; tuning and tests only).  Both compute the
+ * same function; the tensor-memory kernel multiplies P, written as three
+ * E4M3 terms (about 12 significant bits), by the E4M3 V codes, where the
+ * warp-level kernel uses f16 P (11).  0 on invalid arguments. */
 PTPC_API int ptpc_decode_attention_kernel(int64_t Hq, int64_t Hkv, int64_t D, int64_t block_size);
 
 /* ------------------------------------------------------------------------- */
