@@ -553,11 +553,13 @@ __global__ void __launch_bounds__(D) decode_attn_combine_kernel(const float *__r
   out[bh * D + d] = __float2bfloat16_rn(l > 0.0f ? o / l : 0.0f);
 }
 
-// Context chunk of a CTA: 512, 1024 or 2048 positions.  Larger chunks pay the
+// Context chunk of a CTA: 512, 1024 or 2048 positions (up to 4096 for the
+// tensor-memory kernel).  Larger chunks pay the
 // CTA's start (block table, query terms) and end (the warps' combine) over
 // more tiles but leave fewer CTAs to fill the GPU; the launch takes the chunk
-// with the fewest rounds of resident CTAs times (positions a CTA + `fixed`,
-// the CTA's start and end counted in positions) (ties: the larger chunk).
+// with the fewest rounds of resident CTAs times (positions a CTA — at most the
+// longest context — + `fixed`, the CTA's start and end counted in positions)
+// (ties: the larger chunk).
 constexpr int kAttnChunkMin = 512;
 
 template <int D, int CHUNK, int NH>
@@ -599,7 +601,8 @@ int attn_resident() {
   return n;
 }
 
-// PTPC_FORCE_ATTN_CHUNK = 512 | 1024 | 2048 (tuning and tests only): read at
+// PTPC_FORCE_ATTN_CHUNK = 512 | 1024 | 2048 | 4096 (tuning and tests only;
+// 4096 only for the tensor-memory kernel, the other takes 2048): read at
 // the first launch, or again by attn_reload_tuning.
 std::atomic<int> g_attn_chunk{-1};
 
@@ -607,21 +610,21 @@ int read_attn_chunk() {
   const char *v = std::getenv("PTPC_FORCE_ATTN_CHUNK");
   if (v == nullptr) return 0;
   const int c = std::atoi(v);
-  return c == 512 || c == 1024 || c == 2048 ? c : 0;
+  return c == 512 || c == 1024 || c == 2048 || c == 4096 ? c : 0;
 }
 
-int attn_chunk(int pairs, int max_context, int resident, int fixed = 0) {
+int attn_chunk(int pairs, int max_context, int resident, int fixed = 0, int max_chunk = 2048) {
   int forced = g_attn_chunk.load(std::memory_order_relaxed);
   if (forced < 0) {
     forced = read_attn_chunk();
     g_attn_chunk.store(forced, std::memory_order_relaxed);
   }
-  if (forced > 0) return forced;
+  if (forced > 0) return std::min(forced, max_chunk);
   int best = kAttnChunkMin;
   long long best_cost = -1;
-  for (int chunk = kAttnChunkMin; chunk <= 2048; chunk *= 2) {
+  for (int chunk = kAttnChunkMin; chunk <= max_chunk; chunk *= 2) {
     const long long ctas = (long long)pairs * ((std::max(max_context, 1) + chunk - 1) / chunk);
-    const long long cost = (ctas + resident - 1) / resident * (chunk + fixed);
+    const long long cost = (ctas + resident - 1) / resident * (std::min(chunk, std::max(max_context, 1)) + fixed);
     if (best_cost < 0 || cost <= best_cost) {
       best = chunk;
       best_cost = cost;
@@ -686,12 +689,14 @@ cudaError_t launch_attn_tc_and_combine(AttnParams p, int B, int max_context, uin
                                        cudaStream_t st) {
   // the tensor-memory kernel's start (barriers, tensor memory, the first
   // tiles' load latency) costs about three 128-position tiles
-  const int chunk = attn_chunk(B * p.Hkv, max_context, attn_tc_resident(), 384);
+  const int chunk = attn_chunk(B * p.Hkv, max_context, attn_tc_resident(), 384, 4096);
   p.splits = (std::max(max_context, 1) + chunk - 1) / chunk;
+  // one chunk covers every context: the kernel writes the output itself
+  const bool single = p.splits == 1;
   cudaError_t e = launch_attn_tc(p.q, p.kc, p.vc, p.ks, p.vs, p.block_tables, p.context_lens, B, p.Hq, p.Hkv,
                                  p.block_size, p.max_blocks, p.num_slots, p.bs_magic, chunk, p.splits, p.scale_log2,
-                                 p.part_ml, p.part_acc, status, st);
-  if (e != cudaSuccess) return e;
+                                 p.part_ml, p.part_acc, single ? out : nullptr, status, st);
+  if (e != cudaSuccess || single) return e;
   return launch_attn_combine<128>(p, B, out, st);
 }
 

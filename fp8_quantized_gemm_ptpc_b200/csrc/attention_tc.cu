@@ -39,7 +39,8 @@
 // widely; and the common tile needs one barrier and no reduction.  S
 // has two tensor-memory buffers, so the MMAs of tile i+1 run while the
 // softmax works on tile i.  At the end the CTA writes (max, sum, accumulator)
-// of its chunk for the combine kernel of attention.cu.  Every wait is
+// of its chunk for the combine kernel of attention.cu, or, when one chunk
+// covers every context, the output itself.  Every wait is
 // bounded; a timeout sets a bit in the status word at the front of the
 // workspace and the CTA stops (after letting its copies and MMAs finish).
 #include <algorithm>
@@ -69,6 +70,7 @@ constexpr uint32_t kTcColO = 32;
 constexpr uint32_t kStatusTimeoutAttn = 1u << 3;
 constexpr float kRefLazy = 8.0f;    // a head's reference maximum moves when a score exceeds it by this
 constexpr float kRefBelow = 4.0f;   // ... and then to this below the tile's maximum
+constexpr int kTcMaxChunk = 4096;   // positions a CTA at most
 
 struct TcParams {
   const __nv_bfloat16 *q;       // [B, Hq, D]
@@ -81,6 +83,7 @@ struct TcParams {
   int64_t num_slots;
   float scale_log2;
   float *part_ml, *part_acc;
+  __nv_bfloat16 *out;           // [B, Hq, D] when splits == 1 (no combine), else null
   uint32_t *status;
 };
 
@@ -635,10 +638,18 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     for (int h = 0; h < 8; ++h) {
       if (h >= p.G) break;
       const int64_t idx = (((int64_t)b * p.Hq + (int64_t)kvh * p.G + h) * p.splits + split);
+      const float lsum = red[h] + red[16 + h] + red[32 + h] + red[48 + h];
+      if (p.out != nullptr) {
+        // one chunk covers the context: the combine kernel's arithmetic for
+        // a single chunk (o / l, rounded once), written here
+        const int64_t oh = (int64_t)b * p.Hq + (int64_t)kvh * p.G + h;
+        p.out[oh * kTcD + pidx] = __float2bfloat16_rn(lsum > 0.0f ? o_out[h] / lsum : 0.0f);
+        continue;
+      }
       p.part_acc[idx * kTcD + pidx] = o_out[h];
       if (pidx == 0) {
         p.part_ml[idx * 2] = ntiles > 0 ? m[h] : -INFINITY;
-        p.part_ml[idx * 2 + 1] = red[h] + red[16 + h] + red[32 + h] + red[48 + h];
+        p.part_ml[idx * 2 + 1] = lsum;
       }
     }
   }
@@ -723,8 +734,8 @@ int attn_tc_resident() {
   }
   int sms = 148, per_sm = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaFuncSetAttribute(decode_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem_bytes(2048));
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_attn_tc_kernel, kTcThreads, tc_smem_bytes(2048)) !=
+  cudaFuncSetAttribute(decode_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc_smem_bytes(kTcMaxChunk));
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_attn_tc_kernel, kTcThreads, tc_smem_bytes(kTcMaxChunk)) !=
           cudaSuccess ||
       per_sm <= 0)
     per_sm = 1;
@@ -737,9 +748,9 @@ int attn_tc_resident() {
 cudaError_t launch_attn_tc(const void *q, const uint8_t *kc, const uint8_t *vc, const float *ks, const float *vs,
                            const int32_t *block_tables, const int32_t *context_lens, int B, int Hq, int Hkv,
                            int block_size, int max_blocks, int64_t num_slots, uint64_t bs_magic, int chunk,
-                           int splits, float scale_log2, float *part_ml, float *part_acc, uint32_t *status,
-                           cudaStream_t st) {
-  if (chunk % kTcTile != 0 || chunk > 2048 || Hq % Hkv != 0 || !attn_tc_supported(kTcD, Hq / Hkv, block_size))
+                           int splits, float scale_log2, float *part_ml, float *part_acc, void *out,
+                           uint32_t *status, cudaStream_t st) {
+  if ((out != nullptr && splits != 1) || chunk % kTcTile != 0 || chunk > kTcMaxChunk || Hq % Hkv != 0 || !attn_tc_supported(kTcD, Hq / Hkv, block_size))
     return cudaErrorInvalidValue;
   const int box_rows = block_size % 16 == 0 ? 16 : 8;
   CUtensorMap tmK, tmV;
@@ -764,13 +775,14 @@ cudaError_t launch_attn_tc(const void *q, const uint8_t *kc, const uint8_t *vc, 
   p.scale_log2 = scale_log2;
   p.part_ml = part_ml;
   p.part_acc = part_acc;
+  p.out = static_cast<__nv_bfloat16 *>(out);
   p.status = status;
   static std::atomic<bool> attr_set[64];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
     cudaError_t a = cudaFuncSetAttribute(decode_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)tc_smem_bytes(2048));
+                                         (int)tc_smem_bytes(kTcMaxChunk));
     if (a != cudaSuccess) return a;
     attr_set[dev].store(true, std::memory_order_release);
   }

@@ -18,13 +18,15 @@ int attn_kernel_choice(int D, int G, int block_size);
 int attn_tc_resident();
 size_t attn_tc_smem_bytes(int chunk);
 // One CTA per (chunk of `chunk` positions, KV head, sequence): partial
-// results into part_ml [B, Hq, splits, 2] and part_acc [B, Hq, splits, 128];
-// a bounded wait that runs out sets a bit in *status.  chunk: a multiple of
-// 128, at most 2048.
+// results into part_ml [B, Hq, splits, 2] and part_acc [B, Hq, splits, 128],
+// or, with splits == 1 and out non-null, the bf16 output [B, Hq, 128]
+// directly (the combine kernel's arithmetic for one chunk); a bounded wait
+// that runs out sets a bit in *status.  chunk: a multiple of 128, at most
+// 4096.
 cudaError_t launch_attn_tc(const void *q, const uint8_t *kc, const uint8_t *vc, const float *ks, const float *vs,
                            const int32_t *block_tables, const int32_t *context_lens, int B, int Hq, int Hkv,
                            int block_size, int max_blocks, int64_t num_slots, uint64_t bs_magic, int chunk,
-                           int splits, float scale_log2, float *part_ml, float *part_acc, uint32_t *status,
-                           cudaStream_t st);
+                           int splits, float scale_log2, float *part_ml, float *part_acc, void *out,
+                           uint32_t *status, cudaStream_t st);
 
 }  // namespace ptpc

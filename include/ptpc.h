@@ -359,9 +359,10 @@ PTPC_API size_t ptpc_decode_attention_workspace_size(int64_t B, int64_t Hq, int6
  *   exactly decoded V codes; see ptpc_decode_attention_kernel).
  *   out_dev bf16 [B, Hq, D].
  *   ws_dev: ptpc_decode_attention_workspace_size(B, Hq, D, max_context)
- *   bytes (the context is split into chunks of 512, 1024 or 2048 positions,
- *   chosen per launch to fill the GPU, whose partial results are combined by
- *   a second kernel).  It starts with the device status word: the
+ *   bytes (the context is split into chunks of 512 to 2048 positions, 4096
+ *   with the tensor-memory kernel, chosen per launch to fill the GPU, whose
+ *   partial results are combined by a second kernel; when one chunk covers
+ *   every context the attention kernel writes the output itself).  It starts with the device status word: the
  *   tensor-memory kernel (see ptpc_decode_attention_kernel) sets a bit there
  *   when one of its bounded waits runs out, which ptpc_get_device_status
  *   reports; the word must be zero before the first call (a zeroed

@@ -2,7 +2,8 @@
 inside a larger allocation whose guard bytes before and after must come back
 unchanged, over shapes that exercise every tail path (ragged rows and
 columns, both prefill tile widths, the decode kernel with and without a K
-split, the long-row quantiser, the naive path)."""
+split, the long-row quantiser, the naive path, decode attention on both of
+its kernels)."""
 import ctypes
 
 import numpy as np
@@ -138,4 +139,51 @@ def test_swapped_gemm_stays_in_bounds(ptpc, monkeypatch, T, Ci, Co, env):
     finally:
         for k in env:
             monkeypatch.delenv(k, raising=False)
+        ptpc.reload_tuning_overrides()
+
+
+@pytest.mark.parametrize("kernel,chunk", [("tc", "auto"), ("tc", "1024"), ("mma", "auto")])
+@pytest.mark.parametrize("lens,Hq,Hkv,D,bs", [
+    ([1, 300, 4096, 0, 77], 64, 8, 128, 16),     # one chunk a context: the kernel writes the output itself
+    ([5000, 130], 24, 3, 128, 8),                # several chunks: partial results and the combine kernel
+    ([40, 600], 32, 2, 64, 16),                  # the warp-level kernel's shape
+])
+def test_decode_attention_stays_in_bounds(ptpc, monkeypatch, kernel, chunk, lens, Hq, Hkv, D, bs):
+    """Decode attention's output and workspace (status word, partial results)
+    stay inside their buffers on both kernels, with the output written by the
+    attention kernel itself (one chunk a context) and by the combine kernel."""
+    monkeypatch.setenv("PTPC_FORCE_ATTN_KERNEL", kernel)
+    if chunk != "auto":
+        monkeypatch.setenv("PTPC_FORCE_ATTN_CHUNK", chunk)
+    ptpc.reload_tuning_overrides()
+    try:
+        B = len(lens)
+        max_blocks = max(1, max((l + bs - 1) // bs for l in lens))
+        nb = B * max_blocks + 1
+        rng = np.random.Generator(np.random.PCG64(sum(lens) + Hq))
+        tables = torch.from_numpy(rng.permutation(nb)[:B * max_blocks].astype(np.int32).reshape(B, max_blocks)).cuda()
+        kc = torch.randint(0, 0x7E, (nb, bs, Hkv, D), dtype=torch.uint8, device="cuda")
+        vc = torch.randint(0, 0x7E, (nb, bs, Hkv, D), dtype=torch.uint8, device="cuda")
+        ksc = torch.rand((nb, bs, Hkv), device="cuda") * 0.01
+        vsc = torch.rand((nb, bs, Hkv), device="cuda") * 0.01
+        q = torch.randn((B, Hq, D), device="cuda").to(torch.bfloat16)
+        max_ctx = max(lens)
+        out = Guarded(B * Hq * D * 2)
+        need = int(ptpc.lib.ptpc_decode_attention_workspace_size(B, Hq, D, max_ctx))
+        ws = Guarded(need)
+        ws.view(torch.uint8, (need,)).zero_()
+        lens_d = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        P = ctypes.c_void_p
+        st = P(torch.cuda.current_stream().cuda_stream)
+        r = ptpc.lib.ptpc_decode_attention(P(q.data_ptr()), P(kc.data_ptr()), P(vc.data_ptr()), P(ksc.data_ptr()),
+                                           P(vsc.data_ptr()), P(tables.data_ptr()), P(lens_d.data_ptr()), B, Hq, Hkv,
+                                           D, bs, nb, max_blocks, max_ctx, ctypes.c_float(D ** -0.5), out.ptr(),
+                                           ws.ptr(), need, st)
+        assert r == ptpc.OK
+        out.check(f"attention out {kernel} {lens}")
+        ws.check(f"attention workspace {kernel} {lens}")
+        assert ptpc.lib.ptpc_get_device_status(ws.ptr(), st) == ptpc.OK
+    finally:
+        monkeypatch.delenv("PTPC_FORCE_ATTN_KERNEL", raising=False)
+        monkeypatch.delenv("PTPC_FORCE_ATTN_CHUNK", raising=False)
         ptpc.reload_tuning_overrides()

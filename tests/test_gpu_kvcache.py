@@ -141,16 +141,17 @@ def test_decode_attention(ptpc, kernel, lens, Hq, Hkv, D, bs):
     _attention_case(ptpc, kernel, lens, Hq, Hkv, D, bs)
 
 
-@pytest.mark.parametrize("chunk", ["1024", "2048"])
+@pytest.mark.parametrize("chunk", ["1024", "2048", "4096"])
 @pytest.mark.parametrize("lens,Hq,Hkv,D,bs", [
-    ([511, 512, 513, 1030, 2047, 2048, 2049, 4100], 64, 8, 128, 16),
+    ([511, 512, 513, 1030, 2047, 2048, 2049, 4100, 8200], 64, 8, 128, 16),
     ([257, 1500, 3000], 32, 2, 64, 24),
     ([0, 5, 2049], 28, 4, 128, 16),
 ])
 def test_decode_attention_chunk_sizes(ptpc, monkeypatch, kernel, chunk, lens, Hq, Hkv, D, bs):
     """The larger context chunks a CTA can take (chosen by the launch for
-    long contexts on many sequences), forced on small cases; a block size
-    that is not a power of two exercises the exact quotient."""
+    long contexts on many sequences; 4096 only on the tensor-memory kernel,
+    the warp-level one takes 2048), forced on small cases; a block size that
+    is not a power of two exercises the exact quotient."""
     monkeypatch.setenv("PTPC_FORCE_ATTN_CHUNK", chunk)
     ptpc.reload_tuning_overrides()
     try:
