@@ -12,10 +12,9 @@
 // box a lane) into two rings of stages, one for K (a stage is free again once
 // the tile's QK MMAs are done) and one for V (free once its PV MMAs are
 // done), so neither ring waits for the other half's work.  It issues nothing
-// else and runs as far ahead as the rings allow (a TMA instruction takes
-// tens of cycles to issue whatever its box, hence the largest box a block
-// allows).  Warp 1
-// issues the MMAs from one thread:
+// else and runs as far ahead as the rings allow (a TMA instruction takes tens
+// of cycles to issue whatever its box, hence the largest box a block allows).
+// Warp 1 issues the MMAs from one thread:
 //   S^T = K Q^T    (M = 128 positions, N = 16, K = d; A = the K tile, B = q)
 //   O^T += V^T P^T (M = 128 values of d, N = 2 x 16, K = positions; A = the
 //                   V tile read as an MN-major operand, B = P, MN-major)
@@ -28,21 +27,21 @@
 // codes go in as they are, with no conversion.
 // Warps 2-5 (thread i = tensor-memory lane i = position i of the tile, and
 // value d = i of O; each loads its position's two scales two tiles ahead)
-// run the online softmax in base 2: key scales, masking,
-// exponentials, P written to shared memory.  The running maximum and the
-// value-scale unit are lazy: a reference maximum per head moves (and O, in
-// tensor memory, is rescaled) only when a score exceeds it by more than 8
-// (base-2 units), and then to 4 below the tile's maximum; the unit (a power
-// of two) moves only when a value scale exceeds it.  So P stays below 2^8
-// (E4M3 holds 448) and its largest terms sit well above E4M3's absolute
-// resolution (2^-13 for the two terms), even when the value scales spread
-// widely; and the common tile needs one barrier and no reduction.  S
-// has two tensor-memory buffers, so the MMAs of tile i+1 run while the
-// softmax works on tile i.  At the end the CTA writes (max, sum, accumulator)
-// of its chunk for the combine kernel of attention.cu, or, when one chunk
-// covers every context, the output itself.  Every wait is
-// bounded; a timeout sets a bit in the status word at the front of the
-// workspace and the CTA stops (after letting its copies and MMAs finish).
+// run the online softmax in base 2: key scales, masking, exponentials, P
+// written to shared memory.  The running maximum and the value-scale unit are
+// lazy: a reference maximum per head moves (and O, in tensor memory, is
+// rescaled) only when a score exceeds it by more than 8 (base-2 units), and
+// then to 4 below the tile's maximum; the unit (a power of two) moves only
+// when a value scale exceeds it.  So P stays below 2^8 (E4M3 holds 448), its
+// largest values sit far above the smallest step its three E4M3 terms can
+// express even when the value scales spread widely, and the common tile needs
+// one barrier and no reduction.  S has two tensor-memory buffers, so the MMAs
+// of tile i+1 run while the softmax works on tile i.  At the end the CTA
+// writes (max, sum, accumulator) of its chunk for the combine kernel of
+// attention.cu, or, when one chunk covers every context, the output itself.
+// Every wait is bounded; a timeout sets a bit in the status word at the front
+// of the workspace and the CTA stops (after letting its copies and MMAs
+// finish).
 #include <algorithm>
 #include <atomic>
 #include <cstdint>
@@ -61,7 +60,7 @@ namespace ptpc {
 namespace {
 
 constexpr int kTcThreads = 192;  // warp 0 producer, warp 1 MMA issuer, warps 2-5 softmax
-constexpr int kTcStages = 3;   // of each ring
+constexpr int kTcStages = 3;     // stages of each ring
 constexpr int kTcTile = 128;     // positions a tile
 constexpr int kTcD = 128;
 constexpr int kTcKV = kTcTile * kTcD;  // bytes of one K or V tile
@@ -230,18 +229,25 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Independent loads, issued together: this thread's part of its head's
+  // query (softmax warps), the context length and the block-table entries a
+  // whole chunk spans (-1 past the table; entries past the context are never
+  // read, positions there being rejected first).
+  const int tq = threadIdx.x - 64;  // softmax thread 0..127: head tq / 16, values 8 (tq % 16) ..
+  uint4 qw = make_uint4(0u, 0u, 0u, 0u);
+  if (warp >= 2 && (tq >> 4) < p.G)
+    qw = *reinterpret_cast<const uint4 *>(p.q + ((int64_t)b * p.Hq + (int64_t)kvh * p.G + (tq >> 4)) * kTcD +
+                                          (tq & 15) * 8);
   const int L = __ldg(p.context_lens + b);
   const int c0 = split * p.chunk;
-  const int c1 = min(c0 + p.chunk, L);
-  const int ntiles = c1 > c0 ? (c1 - c0 + kTcTile - 1) / kTcTile : 0;
-
-  // the chunk's block-table entries (-1 where there is none)
   const int bi0 = (int)__umul64hi((uint64_t)c0, p.bs_magic);
-  const int nbi = c1 > c0 ? (int)__umul64hi((uint64_t)(c1 - 1), p.bs_magic) - bi0 + 1 : 0;
+  const int nbi = (int)__umul64hi((uint64_t)(c0 + p.chunk - 1), p.bs_magic) - bi0 + 1;  // <= chunk / 8 + 2
   for (int i = threadIdx.x; i < nbi; i += kTcThreads) {
     const int bi = bi0 + i;
     s_blk[i] = bi < p.max_blocks ? __ldg(p.block_tables + (int64_t)b * p.max_blocks + bi) : -1;
   }
+  const int c1 = min(c0 + p.chunk, L);
+  const int ntiles = c1 > c0 ? (c1 - c0 + kTcTile - 1) / kTcTile : 0;
   if (threadIdx.x == 0) {
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
@@ -278,13 +284,12 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   // softmax warps: q as two E4M3 terms (rows 0..7 = first terms of the heads,
   // rows 8..15 = second terms), 1 / sigma of each head into shared memory
   if (warp >= 2) {
-    const int t = threadIdx.x - 64;  // 0..127
+    const int t = tq;  // 0..127
     const int h = t >> 4, d0 = (t & 15) * 8;
     float x[8];
     float amax = 0.0f;
     if (h < p.G) {
-      const uint4 w = *reinterpret_cast<const uint4 *>(p.q + ((int64_t)b * p.Hq + (int64_t)kvh * p.G + h) * kTcD + d0);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      const uint32_t ww[4] = {qw.x, qw.y, qw.z, qw.w};
       #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ww[i]));
