@@ -77,7 +77,7 @@ def parse():
                     help="T values of the decode record inside the default line ('' to skip)")
     ap.add_argument("--weight-formats", default="e3m2,e2m1",
                     help="sub-byte weight formats of the decode_subbyte record")
-    ap.add_argument("--record", default=None, choices=["decode", "decode_subbyte", "kv_decode", "prefill_subbyte"],
+    ap.add_argument("--record", default=None, choices=["decode", "decode_subbyte", "kv_decode", "kv_decode_405b", "prefill_subbyte"],
                     help="print only this sub-record of the default line (a short run for profiling)")
     return ap.parse_args()
 
@@ -531,9 +531,9 @@ def prefill_subbyte_record(ptpc, dev, peaks, steps, fmts=("e3m2", "e2m1"), T=819
             "per_format": res}
 
 
-def kv_decode_record(ptpc, dev, peaks, B=32, ctx=4096, Hq=64, Hkv=8, D=128, bs=16, steps=50):
+def kv_decode_record(ptpc, dev, peaks, B=32, ctx=4096, Hq=64, Hkv=8, D=128, bs=16, steps=50, model="Llama-3.1-70B"):
     """Decode attention of a Llama-3.1-70B-shaped layer (64 query heads on 8
-    KV heads, D = 128) over the FP8 paged cache: B sequences of ctx cached
+    KV heads, D = 128; Llama-3.1-405B: 128 query heads) over the FP8 paged cache: B sequences of ctx cached
     positions, blocks of bs positions in a shuffled order.  Algorithmic bytes
     per step: the codes of K and V, their scales, q and the output.  Also
     times appending one new token per sequence (the decode step's write)."""
@@ -589,7 +589,7 @@ def kv_decode_record(ptpc, dev, peaks, B=32, ctx=4096, Hq=64, Hkv=8, D=128, bs=1
     ms_app = e0.elapsed_time(e1) / steps
     gbs = nbytes / (ms / 1e3) / 1e9
     rec = {
-        "workload": f"Llama-3.1-70B decode attention: {B} sequences x {ctx} cached positions, {Hq} query / "
+        "workload": f"{model} decode attention: {B} sequences x {ctx} cached positions, {Hq} query / "
                     f"{Hkv} KV heads, D = {D}, {bs}-position blocks (shuffled), E4M3 codes + per-(token, head) scales",
         "kernel": ptpc.decode_attention_kernel(Hq, Hkv, D, bs),
         "ms_per_step": ms, "algorithmic_bytes": nbytes,
@@ -1223,6 +1223,8 @@ def run_record(args):
     elif args.record == "prefill_subbyte":
         rec = prefill_subbyte_record(ptpc, dev, peaks, steps=steps,
                                      fmts=tuple(f for f in args.weight_formats.split(",") if f))
+    elif args.record == "kv_decode_405b":
+        rec = kv_decode_record(ptpc, dev, peaks, Hq=128, steps=steps, model="Llama-3.1-405B")
     else:
         rec = kv_decode_record(ptpc, dev, peaks, steps=steps)
     print(json.dumps({"record": args.record} | rec), flush=True)

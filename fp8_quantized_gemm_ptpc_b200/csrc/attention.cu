@@ -634,8 +634,8 @@ int attn_chunk(int pairs, int max_context, int resident, int fixed = 0, int max_
 }
 
 // Decode attention runs the tensor-memory kernel of attention_tc.cu where it
-// applies (D = 128, groups of at most 8 query heads, blocks of a multiple of
-// 8 positions) and the warp-level kernel above otherwise.
+// applies (D = 128, blocks of a multiple of 8 positions) and the warp-level
+// kernel above otherwise.
 // PTPC_FORCE_ATTN_KERNEL = mma | tc (tuning and tests only) forces one (tc
 // only where it applies).  Read at the first launch, or again by
 // attn_reload_tuning.
@@ -689,7 +689,7 @@ cudaError_t launch_attn_tc_and_combine(AttnParams p, int B, int max_context, uin
                                        cudaStream_t st) {
   // the tensor-memory kernel's start (barriers, tensor memory, the first
   // tiles' load latency) costs about three 128-position tiles
-  const int chunk = attn_chunk(B * p.Hkv, max_context, attn_tc_resident(), 384, 4096);
+  const int chunk = attn_chunk(B * p.Hkv * ((p.G + 7) / 8), max_context, attn_tc_resident(), 384, 4096);
   p.splits = (std::max(max_context, 1) + chunk - 1) / chunk;
   // one chunk covers every context: the kernel writes the output itself
   const bool single = p.splits == 1;

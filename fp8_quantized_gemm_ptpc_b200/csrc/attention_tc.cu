@@ -1,11 +1,13 @@
 // Decode attention over the FP8 (E4M3) paged KV cache on the fifth-generation
-// tensor cores (tcgen05), for head size 128, GQA groups of up to 8 query
+// tensor cores (tcgen05), for head size 128, GQA groups of up to 16 query
 // heads and cache blocks of a multiple of 8 positions.  Same arguments and
 // results as the warp-level kernel in attention.cu (which takes every other
 // shape); same cache layout:
 //   codes  cache[(slot * Hkv + g) * D + d],  scale  scales[slot * Hkv + g].
 //
-// A CTA takes one (sequence, KV head) and a chunk of context positions, in
+// A CTA takes one (sequence, KV head, group of at most 8 of the KV head's
+// query heads — a group of 9 to 16 takes two CTAs, which read the same
+// tiles, the second mostly from L2) and a chunk of context positions, in
 // tiles of 128 positions.  Warp 0 loads a tile's K and V codes with TMA (a
 // 3-D tensor map over [slot][head][d], boxes of 16 positions, or 8 where the
 // cache blocks hold an odd multiple of 8, into 128-byte swizzled tiles, one
@@ -77,6 +79,7 @@ struct TcParams {
   const int32_t *block_tables;  // [B, max_blocks]
   const int32_t *context_lens;  // [B]
   int Hq, Hkv, G, block_size, max_blocks, splits, chunk;
+  int hgroups;                  // CTAs a KV head (query heads 8 a CTA)
   int box_rows;                 // positions a TMA box: 16, or 8 (a divisor of block_size)
   uint64_t bs_magic;            // ceil(2^64 / block_size)
   int64_t num_slots;
@@ -227,7 +230,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   uint64_t *drain = o_done + 1;               // the MMA issuer's last commit
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain + 1);
 
-  const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int split = blockIdx.x, kvh = blockIdx.y / p.hgroups, b = blockIdx.z;
+  // this CTA's query heads: kvh * G + h0 + h, h < GC
+  const int h0 = (blockIdx.y - kvh * p.hgroups) * 8;
+  const int GC = min(8, p.G - h0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Independent loads, issued together: this thread's part of its head's
   // query (softmax warps), the context length and the block-table entries a
@@ -235,8 +241,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   // read, positions there being rejected first).
   const int tq = threadIdx.x - 64;  // softmax thread 0..127: head tq / 16, values 8 (tq % 16) ..
   uint4 qw = make_uint4(0u, 0u, 0u, 0u);
-  if (warp >= 2 && (tq >> 4) < p.G)
-    qw = *reinterpret_cast<const uint4 *>(p.q + ((int64_t)b * p.Hq + (int64_t)kvh * p.G + (tq >> 4)) * kTcD +
+  if (warp >= 2 && (tq >> 4) < GC)
+    qw = *reinterpret_cast<const uint4 *>(p.q + ((int64_t)b * p.Hq + (int64_t)kvh * p.G + h0 + (tq >> 4)) * kTcD +
                                           (tq & 15) * 8);
   const int L = __ldg(p.context_lens + b);
   const int c0 = split * p.chunk;
@@ -288,7 +294,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int h = t >> 4, d0 = (t & 15) * 8;
     float x[8];
     float amax = 0.0f;
-    if (h < p.G) {
+    if (h < GC) {
       const uint32_t ww[4] = {qw.x, qw.y, qw.z, qw.w};
       #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -488,7 +494,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       #pragma unroll
       for (int h = 0; h < 8; ++h) {
         const float sc = fmaf(__uint_as_float(r[8 + h]), 0.0625f, __uint_as_float(r[h]));
-        sv[h] = (valid && h < p.G) ? sc * (ksc * inv_sig[h]) : -INFINITY;
+        sv[h] = (valid && h < GC) ? sc * (ksc * inv_sig[h]) : -INFINITY;
         need = need || sv[h] > m[h] + kRefLazy;
       }
       // one barrier a tile: does any thread need the maxima, or has any wait
@@ -641,13 +647,13 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     softmax_bar();
     #pragma unroll
     for (int h = 0; h < 8; ++h) {
-      if (h >= p.G) break;
-      const int64_t idx = (((int64_t)b * p.Hq + (int64_t)kvh * p.G + h) * p.splits + split);
+      if (h >= GC) break;
+      const int64_t idx = (((int64_t)b * p.Hq + (int64_t)kvh * p.G + h0 + h) * p.splits + split);
       const float lsum = red[h] + red[16 + h] + red[32 + h] + red[48 + h];
       if (p.out != nullptr) {
         // one chunk covers the context: the combine kernel's arithmetic for
         // a single chunk (o / l, rounded once), written here
-        const int64_t oh = (int64_t)b * p.Hq + (int64_t)kvh * p.G + h;
+        const int64_t oh = (int64_t)b * p.Hq + (int64_t)kvh * p.G + h0 + h;
         p.out[oh * kTcD + pidx] = __float2bfloat16_rn(lsum > 0.0f ? o_out[h] / lsum : 0.0f);
         continue;
       }
@@ -725,7 +731,7 @@ bool tc_cache_map(CUtensorMap *m, const void *base, int Hkv, int64_t slots, int 
 
 }  // namespace
 
-bool attn_tc_supported(int D, int G, int block_size) { return D == kTcD && G <= 8 && block_size % 8 == 0; }
+bool attn_tc_supported(int D, int G, int block_size) { return D == kTcD && G >= 1 && G <= 16 && block_size % 8 == 0; }
 
 size_t attn_tc_smem_bytes(int chunk) { return tc_smem_bytes(chunk); }
 
@@ -770,6 +776,7 @@ cudaError_t launch_attn_tc(const void *q, const uint8_t *kc, const uint8_t *vc, 
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
+  p.hgroups = (p.G + 7) / 8;
   p.block_size = block_size;
   p.box_rows = box_rows;
   p.max_blocks = max_blocks;
@@ -791,7 +798,8 @@ cudaError_t launch_attn_tc(const void *q, const uint8_t *kc, const uint8_t *vc, 
     if (a != cudaSuccess) return a;
     attr_set[dev].store(true, std::memory_order_release);
   }
-  decode_attn_tc_kernel<<<dim3(splits, Hkv, B), kTcThreads, tc_smem_bytes(chunk), st>>>(p, tmK, tmV);
+  if ((int64_t)Hkv * p.hgroups > 65535) return cudaErrorInvalidValue;
+  decode_attn_tc_kernel<<<dim3(splits, Hkv * p.hgroups, B), kTcThreads, tc_smem_bytes(chunk), st>>>(p, tmK, tmV);
   return cudaGetLastError();
 }
 

@@ -1,6 +1,6 @@
 // Decode attention on the fifth-generation tensor cores (attention_tc.cu):
-// head size 128, GQA groups of up to 8 heads, cache blocks of a multiple of 8
-// positions.  attention.cu chooses between it and the warp-level kernel and
+// head size 128, GQA groups of up to 16 heads, cache blocks of a multiple of
+// 8 positions.  attention.cu chooses between it and the warp-level kernel and
 // runs the combine kernel after either.
 #pragma once
 
@@ -17,7 +17,8 @@ int attn_kernel_choice(int D, int G, int block_size);
 // CTAs of the kernel that can be resident at once on this device.
 int attn_tc_resident();
 size_t attn_tc_smem_bytes(int chunk);
-// One CTA per (chunk of `chunk` positions, KV head, sequence): partial
+// One CTA per (chunk of `chunk` positions, KV head and group of up to 8 of
+// its query heads, sequence): partial
 // results into part_ml [B, Hq, splits, 2] and part_acc [B, Hq, splits, 128],
 // or, with splits == 1 and out non-null, the bf16 output [B, Hq, 128]
 // directly (the combine kernel's arithmetic for one chunk); a bounded wait

@@ -376,10 +376,10 @@ PTPC_API int ptpc_decode_attention(const void *q_dev, const uint8_t *k_cache_dev
 
 /* Which decode-attention kernel ptpc_decode_attention runs for a shape on
  * this library: 2 the kernel on the fifth-generation tensor cores (tcgen05
- * MMAs into tensor memory, TMA loads), for D = 128, groups of at most 8
- * query heads a KV head and block sizes that are multiples of 8; 1 the
- * warp-level kernel (mma.sync tensor-core tiles) for every other supported
- * shape.  PTPC_FORCE_ATTN_KERNEL=mma forces kernel 1 and =tc asks for
+ * MMAs into tensor memory, TMA loads), for D = 128 and block sizes that are
+ * multiples of 8 (groups of 9 to 16 query heads take two CTAs a KV head);
+ * 1 the warp-level kernel (mma.sync tensor-core tiles) for every other
+ * supported shape.  PTPC_FORCE_ATTN_KERNEL=mma forces kernel 1 and =tc asks for
  * kernel 2 where it applies (read at the first launch or by
  * ptpc_reload_tuning_overrides; tuning and tests only).  Both compute the
  * same function; the tensor-memory kernel multiplies P, written as three

@@ -200,19 +200,19 @@ def test_tensor_map_cache_logic(ptpc):
 
 def test_decode_attention_kernel_choice(ptpc, monkeypatch):
     """Which decode-attention kernel a shape runs: the tensor-memory kernel
-    for the shapes it takes (D = 128, groups of at most 8, blocks of a
-    multiple of 8), the warp-level kernel otherwise or when forced, 0 for
-    invalid arguments.  Host logic only."""
+    for the shapes it takes (D = 128, blocks of a multiple of 8; groups up to
+    16), the warp-level kernel otherwise or when forced, 0 for invalid
+    arguments.  Host logic only."""
     k = lambda *a: call(ptpc, "ptpc_decode_attention_kernel", *a)
     try:
         monkeypatch.delenv("PTPC_FORCE_ATTN_KERNEL", raising=False)
         ptpc.reload_tuning_overrides()
-        assert k(64, 8, 128, 16) == 2 and k(64, 8, 64, 16) == 1 and k(128, 8, 128, 16) == 1
+        assert k(64, 8, 128, 16) == 2 and k(64, 8, 64, 16) == 1 and k(128, 8, 128, 16) == 2
         monkeypatch.setenv("PTPC_FORCE_ATTN_KERNEL", "tc")
         ptpc.reload_tuning_overrides()
         assert k(64, 8, 128, 16) == 2 and k(8, 8, 128, 8) == 2 and k(24, 3, 128, 48) == 2
         assert k(64, 8, 64, 16) == 1                # D = 64
-        assert k(128, 8, 128, 16) == 1              # group of 16
+        assert k(128, 8, 128, 16) == 2 and k(96, 8, 128, 16) == 2   # groups of 16 and 12
         assert k(64, 8, 128, 12) == 1               # block of 12 positions
         assert k(12, 8, 128, 16) == 0 and k(64, 0, 128, 16) == 0 and k(64, 8, 96, 16) == 0
         assert k(64, 8, 128, 0) == 0

@@ -37,7 +37,7 @@ def kernel(request, ptpc, monkeypatch):
 
 
 def expect_kernel(ptpc, kernel, Hq, Hkv, D, bs):
-    tc_shape = D == 128 and Hq // Hkv <= 8 and bs % 8 == 0
+    tc_shape = D == 128 and Hq // Hkv <= 16 and bs % 8 == 0
     assert ptpc.decode_attention_kernel(Hq, Hkv, D, bs) == ("tc" if kernel == "tc" and tc_shape else "mma")
 
 
@@ -136,6 +136,8 @@ def test_append_bit_exact(ptpc):
     ([0, 5, 2049], 28, 4, 128, 16),
     ([1, 127, 128, 129, 255, 256, 1000, 2047], 24, 3, 128, 8),
     ([130, 641], 12, 12, 128, 48),
+    ([1, 300, 1000, 4097], 32, 2, 128, 16),      # groups of 16: two CTAs a KV head
+    ([77, 2100], 24, 2, 128, 8),                 # groups of 12: 8 + 4 heads
 ])
 def test_decode_attention(ptpc, kernel, lens, Hq, Hkv, D, bs):
     _attention_case(ptpc, kernel, lens, Hq, Hkv, D, bs)
