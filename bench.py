@@ -77,7 +77,7 @@ def parse():
                     help="T values of the decode record inside the default line ('' to skip)")
     ap.add_argument("--weight-formats", default="e3m2,e2m1",
                     help="sub-byte weight formats of the decode_subbyte record")
-    ap.add_argument("--record", default=None, choices=["decode", "decode_subbyte", "kv_decode", "kv_decode_405b", "prefill_subbyte"],
+    ap.add_argument("--record", default=None, choices=["decode", "decode_subbyte", "kv_decode", "kv_decode_405b", "kv_decode_long", "prefill_subbyte"],
                     help="print only this sub-record of the default line (a short run for profiling)")
     return ap.parse_args()
 
@@ -1243,6 +1243,8 @@ def run_record(args):
                                      fmts=tuple(f for f in args.weight_formats.split(",") if f))
     elif args.record == "kv_decode_405b":
         rec = kv_decode_record(ptpc, dev, peaks, Hq=128, steps=steps, model="Llama-3.1-405B")
+    elif args.record == "kv_decode_long":
+        rec = kv_decode_record(ptpc, dev, peaks, ctx=32768, steps=steps)
     else:
         rec = kv_decode_record(ptpc, dev, peaks, steps=steps)
     print(json.dumps({"record": args.record} | rec), flush=True)
