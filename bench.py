@@ -961,6 +961,7 @@ def run_gpu(args):
                                                            or dec_tokens[:1], steps=max(20, min(K * 2, 100)))
         if not args.no_kv:
             line["kv_decode"] = kv_decode_record(ptpc, dev, peaks)
+            line["kv_decode_long"] = kv_decode_record(ptpc, dev, peaks, ctx=32768, steps=10)
         line["prefill_subbyte"] = prefill_subbyte_record(ptpc, dev, peaks, steps=max(5, min(K, 20)))
         chain_tokens = [int(t) for t in args.chain_tokens.split(",") if t.strip()]
         if chain_tokens:
