@@ -113,6 +113,19 @@ def status_string(status: int) -> str:
     return lib.ptpc_status_string(int(status)).decode()
 
 
+_size_cache: dict = {}
+
+
+def _ws_need(op: int, T: int, Ci: int, Co: int, device: torch.device) -> int:
+    """workspace_size for a call on `device`, remembered per shape (the size
+    depends on the shape, the device and the tuning overrides only)."""
+    key = (op, T, Ci, Co, device.index)
+    n = _size_cache.get(key)
+    if n is None:
+        n = _size_cache[key] = workspace_size(op, T, Ci, Co)
+    return n
+
+
 def workspace_size(op: int, T: int, Ci: int, Co: int) -> int:
     return int(lib.ptpc_workspace_size(op, T, Ci, Co))
 
@@ -222,13 +235,12 @@ def default_workspace(nbytes: int, device) -> Workspace:
     workspaces and never share the quantised activations or the status word
     a ``linear`` call keeps there, while calls on one stream are ordered by
     that stream, which is what makes sharing one buffer between them safe."""
-    dev = torch.device(device)
-    stream = torch.cuda.current_stream(dev)
-    key = (dev, stream.cuda_stream)
+    dev = device if isinstance(device, torch.device) else torch.device(device)
+    key = (dev, _stream(dev))
     with _ws_lock:
         ws = _ws_cache.get(key)
         if ws is None:
-            with torch.cuda.stream(stream):
+            with torch.cuda.stream(torch.cuda.current_stream(dev)):
                 ws = _ws_cache[key] = Workspace(nbytes, dev)
         return ws.ensure(nbytes)
 
@@ -327,7 +339,7 @@ def scaled_mm_fmt(Xq, x_scale, Wq, w_scale, fmt: str, out: torch.Tensor | None =
     if _packed_ci(Wq, fmt) != Ci or x_scale.shape[0] != T or w_scale.shape[0] != Co:
         raise ValueError("shape mismatch")
     out = torch.empty((T, Co), dtype=torch.bfloat16, device=Xq.device) if out is None else out
-    need = workspace_size(OP_SCALED_MM, T, Ci, Co)
+    need = _ws_need(OP_SCALED_MM, T, Ci, Co, Xq.device)
     ws = default_workspace(need, Xq.device) if ws is None else ws.ensure(need)
     _check("ptpc_scaled_mm_fmt",
            lib.ptpc_scaled_mm_fmt(_ptr(Xq), _ptr(x_scale), _ptr(Wq), _ptr(w_scale), _fmt(fmt), T, Ci, Co,
@@ -345,7 +357,7 @@ def linear_fmt(X, Wq, w_scale, fmt: str, out: torch.Tensor | None = None, ws: Wo
     if _packed_ci(Wq, fmt) != Ci or w_scale.shape[0] != Co:
         raise ValueError("shape mismatch")
     out = torch.empty((T, Co), dtype=torch.bfloat16, device=X.device) if out is None else out
-    need = workspace_size(OP_LINEAR, T, Ci, Co)
+    need = _ws_need(OP_LINEAR, T, Ci, Co, X.device)
     ws = default_workspace(need, X.device) if ws is None else ws.ensure(need)
     _check("ptpc_linear_fmt",
            lib.ptpc_linear_fmt(_ptr(X), ldx, _ptr(Wq), _ptr(w_scale), _fmt(fmt), T, Ci, Co, _ptr(out), ws.ptr(),
@@ -364,7 +376,7 @@ def scaled_mm(Xq, x_scale, Wq_t, w_scale, out: torch.Tensor | None = None, ws: W
     if Wq_t.shape[1] != Ci or x_scale.shape[0] != T or w_scale.shape[0] != Co:
         raise ValueError("shape mismatch")
     out = torch.empty((T, Co), dtype=torch.bfloat16, device=Xq.device) if out is None else out
-    need = workspace_size(OP_SCALED_MM, T, Ci, Co)
+    need = _ws_need(OP_SCALED_MM, T, Ci, Co, Xq.device)
     ws = default_workspace(need, Xq.device) if ws is None else ws.ensure(need)
     _check("ptpc_scaled_mm",
            lib.ptpc_scaled_mm(_ptr(Xq), _ptr(x_scale), _ptr(Wq_t), _ptr(w_scale), T, Ci, Co, _ptr(out),
@@ -383,7 +395,7 @@ def linear(X, Wq_t, w_scale, out: torch.Tensor | None = None, ws: Workspace | No
     if Wq_t.shape[1] != Ci or w_scale.shape[0] != Co:
         raise ValueError("shape mismatch")
     out = torch.empty((T, Co), dtype=torch.bfloat16, device=X.device) if out is None else out
-    need = workspace_size(OP_LINEAR, T, Ci, Co)
+    need = _ws_need(OP_LINEAR, T, Ci, Co, X.device)
     ws = default_workspace(need, X.device) if ws is None else ws.ensure(need)
     _check("ptpc_linear",
            lib.ptpc_linear(_ptr(X), ldx, _ptr(Wq_t), _ptr(w_scale), T, Ci, Co, _ptr(out), ws.ptr(), ws.nbytes,
@@ -420,9 +432,11 @@ def static_scratch_status() -> int:
 
 
 def reload_tuning_overrides():
-    """Re-read PTPC_FORCE_KERNEL / PTPC_FORCE_PAIR_BN / PTPC_FORCE_KSPLIT from
-    the environment (the library reads them once otherwise; tuning only)."""
+    """Re-read the PTPC_FORCE_* overrides from the environment (the library
+    reads them once otherwise; tuning only).  Workspace sizes remembered by
+    the binding are forgotten (a forced plan may need another size)."""
     _check("ptpc_reload_tuning_overrides", lib.ptpc_reload_tuning_overrides())
+    _size_cache.clear()
 
 
 def map_cache_stats():
