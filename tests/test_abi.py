@@ -222,3 +222,17 @@ def test_decode_attention_kernel_choice(ptpc, monkeypatch):
     finally:
         monkeypatch.delenv("PTPC_FORCE_ATTN_KERNEL", raising=False)
         ptpc.reload_tuning_overrides()
+
+
+def test_binding_remembers_workspace_sizes_until_overrides_reload(ptpc):
+    """The binding remembers ptpc_workspace_size per (op, shape, device) and
+    forgets it when the tuning overrides are re-read (a forced plan may need
+    another size).  Host logic only."""
+    import torch
+    dev = torch.device("cuda", 0)
+    for op, T, Ci, Co in ((ptpc.OP_LINEAR, 1, 8192, 8192), (ptpc.OP_LINEAR, 8192, 8192, 57344),
+                          (ptpc.OP_SCALED_MM, 300, 8192, 10240)):
+        assert ptpc._ws_need(op, T, Ci, Co, dev) == ptpc.workspace_size(op, T, Ci, Co)
+    assert len(ptpc._size_cache) >= 3
+    ptpc.reload_tuning_overrides()
+    assert len(ptpc._size_cache) == 0
