@@ -196,3 +196,60 @@ def test_kv_cache_oracle():
     out = oracle.decode_attention_reference(qb[:, :1], cc2, cs2, vc, cs2, np.array([[0, 1]]), [8], bs, 0.5)
     mean = dec[codes[:8, 0]].mean(axis=0)
     assert np.allclose(oracle.bf16_to_float(out[0, 0]), mean, rtol=2 ** -8, atol=1e-12)
+    # a dominant score: q along one key's direction, scaled so its score
+    # exceeds the others by far more than fp64's range of exp; p is then
+    # (1, 0, ...) to the last bit and the output is that token's value
+    kc = np.zeros((2, bs, 1, D), np.uint8); ks = np.ones((2, bs, 1), np.float32)
+    kc[1, 2, 0, 0] = 0x7E                              # key at position 6: e_0 * 448
+    vc3 = np.zeros_like(kc); vc3[:, :, 0, :] = codes[:8, 1].reshape(2, bs, D)
+    q3 = np.zeros((1, 1, D), np.float32); q3[0, 0, 0] = 1.0
+    out = oracle.decode_attention_reference(synthetic.to_bf16_bits(q3), kc, ks, vc3, cs2,
+                                            np.array([[0, 1]]), [8], bs, 64.0)
+    assert np.array_equal(out[0, 0], oracle.bf16_from_double(dec[codes[6, 1]]))
+
+
+def test_decode_attention_oracle_matches_library_attention():
+    """Decode attention against PyTorch's scaled_dot_product_attention in
+    fp64 on the same dequantised keys and values, taken in token order (not
+    through the block table) and with the query-head groups expanded by
+    repeat_interleave.  Pins the paged gather, the query-head to KV-head map,
+    the softmax scale and the reduction over ragged contexts: the oracle's
+    bf16 output is the library's fp64 result rounded to nearest (within one
+    bf16 unit where the two fp64 sums round to opposite sides of a tie)."""
+    rng = np.random.Generator(np.random.PCG64(11))
+    B, Hq, Hkv, D, bs = 3, 8, 2, 32, 4
+    lens = [1, 9, 23]
+    nblk = 24
+    scale = 1.0 / np.sqrt(D)
+    cc = {n: np.zeros((nblk, bs, Hkv, D), np.uint8) for n in "kv"}
+    cs = {n: np.zeros((nblk, bs, Hkv), np.float32) for n in "kv"}
+    perm = rng.permutation(nblk)
+    tables = np.zeros((B, 8), np.int64)
+    tokens = {}
+    used = 0
+    for b, L in enumerate(lens):
+        nb = -(-L // bs)
+        tables[b, :nb] = perm[used:used + nb]
+        used += nb
+        slots = tables[b, np.arange(L) // bs] * bs + np.arange(L) % bs
+        for n in "kv":
+            x = synthetic.to_bf16_bits((rng.standard_normal((L, Hkv, D)) * 2.0).astype(np.float32))
+            c, s = oracle.kv_quantize(x)
+            oracle.kv_cache_write(cc[n], cs[n], c, s, slots, bs)
+            tokens[b, n] = (c, s)
+    qb = synthetic.to_bf16_bits(rng.standard_normal((B, Hq, D)).astype(np.float32))
+    out = oracle.decode_attention_reference(qb, cc["k"], cs["k"], cc["v"], cs["v"], tables, lens, bs, scale)
+    dec = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double()
+    q = torch.from_numpy(qb.astype(np.int32) << 16).view(torch.float32).double()
+    for b, L in enumerate(lens):
+        kv = []
+        for n in "kv":
+            c, s = tokens[b, n]
+            x = dec[torch.from_numpy(c).long()] * torch.from_numpy(s).double()[:, :, None]   # [L, Hkv, D]
+            kv.append(x.permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0))               # [Hq, L, D]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q[b][:, None, :], kv[0], kv[1], scale=scale)[:, 0, :].numpy()
+        got = oracle.bf16_to_float(out[b]).astype(np.float64)
+        ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
+        assert np.all(np.abs(got - ref) <= 0.5 * ulp + 1e-12 * np.abs(ref) + 1e-300), b
+        assert np.mean(oracle.bf16_from_double(ref) == out[b]) > 0.99
