@@ -149,6 +149,9 @@ def test_bf16_rounding_fp64_cases():
     assert f(255.5 * 2.0 ** 120 - 2.0 ** 100) == 0x7F7F
     assert f(2.0 ** 129) == 0x7F80
     assert f(-(2.0 ** 129)) == 0xFF80
+    assert f(float("inf")) == 0x7F80 and f(float("-inf")) == 0xFF80
+    nan = f(float("nan"))
+    assert nan & 0x7F80 == 0x7F80 and nan & 0x007F != 0                # a NaN pattern
 
 
 def test_bf16_to_float_is_exact_widening():

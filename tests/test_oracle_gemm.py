@@ -253,3 +253,101 @@ def test_decode_attention_oracle_matches_library_attention():
         ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
         assert np.all(np.abs(got - ref) <= 0.5 * ulp + 1e-12 * np.abs(ref) + 1e-300), b
         assert np.mean(oracle.bf16_from_double(ref) == out[b]) > 0.99
+
+
+def brute_f32(fr: Fraction):
+    """fp32 round-half-to-even of a non-negative exact rational, by bracketing
+    the monotone positive fp32 bit patterns; None where it rounds to inf
+    (at or above the midpoint between the largest finite value, whose
+    mantissa is odd, and 2^128)."""
+    assert fr >= 0
+    if fr >= Fraction(2 ** 128) - Fraction(2 ** 103):
+        return None
+    val = lambda b: Fraction(float(np.array([b], np.uint32).view(np.float32)[0]))
+    lo, hi = 0, 0x7F7FFFFF
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        if val(mid) <= fr:
+            lo = mid
+        else:
+            hi = mid
+    dl, dh = fr - val(lo), val(hi) - fr
+    return val(lo) if dl < dh or (dl == dh and lo % 2 == 0) else val(hi)
+
+
+def page_order_f32_bits(y, xs, ws) -> int:
+    """bf16 bits of (y * xs) * ws, each product one fp32 rounding, in exact
+    arithmetic with brute-force rounding (positive operands)."""
+    p = brute_f32(Fraction(float(y)) * Fraction(float(xs)))
+    if p is None:
+        return 0x7F80
+    v = brute_f32(p * Fraction(float(ws)))
+    return 0x7F80 if v is None else brute_bf16(v)
+
+
+def near_tie_triples(rng, n, acc=None):
+    """Operands whose final product lies within an fp32 rounding of a bf16
+    midpoint, so that the order and the precision of the two products decide
+    the bf16 bits: y (or the given exact accumulators) and xs random, ws the
+    fp32 quotient of a bf16 midpoint by fp32(y * xs)."""
+    y = (rng.random(n) + 1.0).astype(np.float32) if acc is None else np.asarray(acc, np.float32)
+    xs = (rng.random(n) * 0.01 + 1e-3).astype(np.float32)
+    mid = (1.0 + (rng.integers(0, 128, n) + 0.5) / 128.0) * np.exp2(rng.integers(-4, 5, n))
+    ws = (mid / (y.astype(np.float64) * xs)).astype(np.float32)
+    return y, xs, ws
+
+
+def test_fp32_epilogue_rounds_each_product_left_to_right():
+    """The fp32 epilogues (naive step 2 and the fused one) take the page's
+    order, (acc * token scale) * channel scale, each product one fp32
+    round-to-nearest-even and the result rounded to bf16: checked against
+    exact rational arithmetic with brute-force rounding, on operands where
+    another order or fp64 products give other bits."""
+    rng = np.random.default_rng(21)
+    y, xs, ws = near_tie_triples(rng, 400)
+    expect = np.array([page_order_f32_bits(*t) for t in zip(y, xs, ws)], np.uint16)
+    # the cases discriminate: other orders and fp64 products differ on many
+    other = np.array([brute_bf16(Fraction(float(a)) * Fraction(float(b)) * Fraction(float(c)))
+                      for a, b, c in zip(y, xs, ws)], np.uint16)
+    assert (other != expect).sum() >= 40
+    got = oracle.naive_step2_apply_scales(np.diag(y), xs, ws)
+    assert np.array_equal(np.diag(got), expect)
+    # the fused epilogue: accumulators that are exact dot products of codes
+    codes = rng.integers(0x38, 0x50, (400, 2)).astype(np.uint8)      # 1 .. 7.5, positive
+    dec = oracle.e4m3_decode_table()
+    acc = dec[codes[:, 0]] * dec[codes[:, 1]]
+    a, xs, ws = near_tie_triples(rng, 400, acc)
+    expect = np.array([page_order_f32_bits(*t) for t in zip(a, xs, ws)], np.uint16)
+    for i in range(400):
+        got = oracle.fused_f32(codes[i:i + 1, :1], xs[i:i + 1], codes[i:i + 1, 1:], ws[i:i + 1])
+        assert got[0, 0] == expect[i], i
+
+
+def test_fp32_epilogue_overflows_only_in_the_page_order():
+    """A token scale near the top of the range: acc * token scale overflows
+    fp32 (2^23.6 * 2^110) and stays inf after the channel scale (2^-100),
+    while the exact product (about 2^33.6) is finite, and so is the fp64
+    tolerance reference.  The token scale is reachable: amax = 448 * 2^110 is
+    a finite bf16 value."""
+    Ci = 64
+    Xq = np.full((1, Ci), 0x7E, np.uint8)
+    Wq_t = np.full((1, Ci), 0x7E, np.uint8)
+    xs = np.array([2.0 ** 110], np.float32)
+    ws = np.array([2.0 ** -100], np.float32)
+    assert oracle.fused_f32(Xq, xs, Wq_t, ws)[0, 0] == 0x7F80
+    y = oracle.naive_step1_f32(Xq, Wq_t)
+    assert y[0, 0] == Ci * 448.0 * 448.0
+    assert oracle.naive_step2_apply_scales(y, xs, ws)[0, 0] == 0x7F80
+    exact = Fraction(Ci * 448 * 448) * 2 ** 10
+    assert oracle.scaled_mm_reference(Xq, xs, Wq_t, ws)[0, 0] == brute_bf16(exact) != 0x7F80
+
+
+def test_reference_epilogue_rounds_once():
+    """The tolerance reference rounds the fp64 product straight to bf16: a
+    value above a bf16 midpoint by less than half an fp32 unit rounds up
+    (through fp32 first it would land on the midpoint and round to even)."""
+    acc = np.array([[2.0 ** 12 + 2.0 ** 4 + 2.0 ** -18]])            # a multiple of 2^-18
+    out = oracle.reference_epilogue(acc, np.array([2.0 ** -12], np.float32), np.array([1.0], np.float32))
+    assert out[0, 0] == 0x3F81                                          # 1 + 2^-7
+    assert brute_bf16(Fraction(1) + Fraction(1, 2 ** 8) + Fraction(1, 2 ** 30)) == 0x3F81
+    assert brute_bf16(brute_f32(Fraction(1) + Fraction(1, 2 ** 8) + Fraction(1, 2 ** 30))) == 0x3F80

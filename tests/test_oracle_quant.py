@@ -125,6 +125,25 @@ def test_per_tensor_is_equal_scale_special_case():
     assert np.array_equal(Xq, Pq)
 
 
+def test_per_tensor_is_the_one_token_case():
+    """Per-tensor quantisation is per-token quantisation of the whole tensor
+    read as one token: same codes, and the scale is the tensor's largest
+    magnitude / 448.  The largest magnitude is planted in the last element,
+    then in the first, so a maximum over part of the tensor fails."""
+    X = synthetic.make_x(synthetic.LLAMA8B_PREFILL, 3, 24, 256)
+    for where in (-1, 0):
+        Xp = X.copy().ravel()
+        big = np.abs(oracle.bf16_to_float(X)).max() * 4
+        Xp[where] = (np.float32(-big).view(np.uint32) >> 16).astype(np.uint16)
+        Xp = Xp.reshape(X.shape)
+        q, s = oracle.quant_per_tensor(Xp)
+        q1, s1 = oracle.quant_act(Xp.reshape(1, -1))
+        assert s == s1[0] == np.float32(np.abs(oracle.bf16_to_float(Xp)).max()) / np.float32(448.0)
+        assert np.array_equal(q.ravel(), q1[0])
+        Wq_t, sw = oracle.quant_weight_per_tensor(Xp)
+        assert sw == s and np.array_equal(Wq_t, q.T)
+
+
 def test_weight_quant_is_activation_quant_of_transpose():
     W = synthetic.make_w(synthetic.LLAMA8B_PREFILL, 0, 384, 96)
     Wq_t, ws = oracle.quant_weight(W)

@@ -105,7 +105,7 @@ def _worker(rank, world, port, out):
 @pytest.mark.parametrize("world", [2, 4])
 def test_tensor_parallel_layers_equal_the_unsplit_oracle(world):
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     spans = []
