@@ -155,6 +155,8 @@ def test_row_subset_equals_full_rows():
     rows = [0, 3, 19, 7]
     full = oracle.scaled_mm_reference(Xq, xs, Wq_t, ws)
     assert np.array_equal(oracle.scaled_mm_reference(Xq, xs, Wq_t, ws, rows), full[rows])
+    full = oracle.fused_f32(Xq, xs, Wq_t, ws)
+    assert np.array_equal(oracle.fused_f32(Xq, xs, Wq_t, ws, rows), full[rows])
 
 
 def test_kv_cache_oracle():

@@ -3,8 +3,10 @@ oracle (a dropped term, a wrong sign, index, bias, rounding rule or order of
 operations) each make the pin that covers that function fail.
 
 Each mutant of ptpc_oracle.c is compiled by gcc into a temporary library that
-the oracle module is pointed at for the duration of one pin; the attention
-oracle (numpy) is mutated by re-executing its source with one line changed.
+the oracle module is pointed at for the duration of one pin; the functions
+written in numpy (the attention oracle, the fp64 dot products, the row
+selection of the references) are mutated by re-executing their source with
+one line changed.
 Nothing here touches the CUDA path.  CPU only.
 """
 import inspect
@@ -144,23 +146,51 @@ def test_planted_c_mistake_fails_its_pin(name, orig, planted, pin, c_source, tmp
         monkeypatch.setattr(oracle, "_lib", None)
 
 
-ATTN_MUTANTS = [
-    ("query head mapped modulo", "g = h // group", "g = h % Hkv"),
-    ("softmax scale dropped", "s = softmax_scale * (K[:, g, :] @ q[b, h])", "s = (K[:, g, :] @ q[b, h])"),
-    ("block offset shifted", "offs = pos % block_size", "offs = (pos + 1) % block_size"),
-    ("last context position dropped", "pos = np.arange(L)", "pos = np.arange(max(L - 1, 1))"),
-    ("values scaled by the key scales", "V = dec[v_codes[blocks, offs]] * v_scales", "V = dec[v_codes[blocks, offs]] * k_scales"),
+PY_MUTANTS = [
+    ("decode_attention_reference", "query head mapped modulo", "g = h // group", "g = h % Hkv"),
+    ("decode_attention_reference", "softmax scale dropped",
+     "s = softmax_scale * (K[:, g, :] @ q[b, h])", "s = (K[:, g, :] @ q[b, h])"),
+    ("decode_attention_reference", "block offset shifted", "offs = pos % block_size", "offs = (pos + 1) % block_size"),
+    ("decode_attention_reference", "last context position dropped",
+     "pos = np.arange(L)", "pos = np.arange(max(L - 1, 1))"),
+    ("decode_attention_reference", "values scaled by the key scales",
+     "V = dec[v_codes[blocks, offs]] * v_scales", "V = dec[v_codes[blocks, offs]] * k_scales"),
+    ("kv_quantize", "heads and tokens swapped",
+     "q, s = quant_act(np.ascontiguousarray(KV_bits).reshape(T * H, D))",
+     "q, s = quant_act(np.ascontiguousarray(KV_bits.transpose(1, 0, 2)).reshape(T * H, D))"),
+    ("gemm_acc64", "weight codes reversed along K",
+     "acc[:, o0:o0 + col_chunk] = A @ B.T", "acc[:, o0:o0 + col_chunk] = A @ B[:, ::-1].T"),
+    ("gemm_acc64_fmt", "sub-byte codes decoded as E4M3",
+     "acc[:, o0:o0 + col_chunk] = A @ dec[codes_t[o0:o0 + col_chunk]].T",
+     "acc[:, o0:o0 + col_chunk] = A @ e4m3_decode_table()[codes_t[o0:o0 + col_chunk]].T"),
+    ("scaled_mm_reference_fmt", "token scales not following the chosen rows",
+     "slice(None) if rows is None else np.asarray(rows)])", "slice(None) if rows is None else np.asarray(rows)[::-1]])"),
+    ("fused_f32", "token scales not following the chosen rows",
+     "slice(None) if rows is None else np.asarray(rows)])", "slice(None) if rows is None else np.asarray(rows)[::-1]])"),
+    ("linear_reference_fmt", "one token scale for all tokens",
+     "return scaled_mm_reference_fmt(Xq, xs, codes_t, w_scale, fmt, rows), Xq, xs",
+     "return scaled_mm_reference_fmt(Xq, np.full_like(xs, xs.max()), codes_t, w_scale, fmt, rows), Xq, xs"),
 ]
 
+PY_PINS = {
+    "decode_attention_reference": lambda: gemm.test_decode_attention_oracle_matches_library_attention(),
+    "kv_quantize": lambda: gemm.test_kv_cache_oracle(),
+    "gemm_acc64": lambda: gemm.test_hand_example_gemm(),
+    "gemm_acc64_fmt": lambda: subbyte.test_gemm_exact_against_integer_dot_products("e2m1"),
+    "scaled_mm_reference_fmt": lambda: subbyte.test_reference_row_subset_equals_full_rows("e3m2"),
+    "fused_f32": lambda: gemm.test_row_subset_equals_full_rows(),
+    "linear_reference_fmt": lambda: subbyte.test_generic_reference_with_e4m3_equals_the_ptpc_reference(),
+}
 
-@pytest.mark.parametrize("name,orig,planted", ATTN_MUTANTS, ids=[m[0] for m in ATTN_MUTANTS])
-def test_planted_attention_mistake_fails_its_pin(name, orig, planted, monkeypatch):
-    pin = gemm.test_decode_attention_oracle_matches_library_attention
-    src = inspect.getsource(oracle.decode_attention_reference)
+
+@pytest.mark.parametrize("fn,name,orig,planted", PY_MUTANTS, ids=[f"{m[0]}: {m[1]}" for m in PY_MUTANTS])
+def test_planted_python_mistake_fails_its_pin(fn, name, orig, planted, monkeypatch):
+    pin = PY_PINS[fn]
+    src = inspect.getsource(getattr(oracle, fn))
     assert src.count(orig) == 1, name
     ns = dict(vars(oracle))
     exec(src.replace(orig, planted), ns)
-    pin()
-    monkeypatch.setattr(oracle, "decode_attention_reference", ns["decode_attention_reference"])
+    pin()                                       # the pin holds on the oracle itself
+    monkeypatch.setattr(oracle, fn, ns[fn])
     with pytest.raises(AssertionError):
         pin()

@@ -179,3 +179,31 @@ def test_gemm_exact_against_integer_dot_products(fmt):
     # the E4M3 special case of the generic GEMM is the pinned PTPC GEMM
     rq, _ = oracle.quant_weight(W)
     assert np.array_equal(oracle.gemm_acc64_fmt(Xq, rq, "e4m3"), oracle.gemm_acc64(Xq, rq))
+
+
+def test_generic_reference_with_e4m3_equals_the_ptpc_reference():
+    """The format-generic fused entry with E4M3 weights is the pinned PTPC
+    one: the same bf16 outputs over all tokens and over a subset of rows (the
+    token scales then follow the chosen rows)."""
+    X = synthetic.with_edge_rows(synthetic.make_x(synthetic.TINY, 0, 12, 256))
+    W = synthetic.random_bf16((256, 40), seed=6, scale=0.05)
+    codes, ws = oracle.quant_weight_fmt(W, "e4m3")
+    rows = [11, 0, 5, 7]
+    for r in (None, rows):
+        got, gq, gs = oracle.linear_reference_fmt(X, codes, ws, "e4m3", r)
+        want, wq, wsc = oracle.linear_reference(X, codes, ws, r)
+        assert np.array_equal(got, want) and np.array_equal(gq, wq) and np.array_equal(gs, wsc)
+
+
+@pytest.mark.parametrize("fmt", SUB)
+def test_reference_row_subset_equals_full_rows(fmt):
+    """A subset of token rows of the sub-byte reference equals those rows of
+    the full result (the token scales follow the rows)."""
+    rng = np.random.default_rng(12)
+    X = synthetic.make_x(synthetic.TINY, 0, 16, 256)
+    Xq, xs = oracle.quant_act(X)
+    xs = xs * (rng.random(16) + 0.5).astype(np.float32)         # distinct token scales
+    codes, ws = oracle.quant_weight_fmt(synthetic.random_bf16((256, 24), seed=7, scale=0.05), fmt)
+    rows = [15, 2, 9]
+    full = oracle.scaled_mm_reference_fmt(Xq, xs, codes, ws, fmt)
+    assert np.array_equal(oracle.scaled_mm_reference_fmt(Xq, xs, codes, ws, fmt, rows), full[rows])
