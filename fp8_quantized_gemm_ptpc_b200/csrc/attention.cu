@@ -164,8 +164,8 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 // head's q is scaled by a power of two sigma (the largest with max |q| sigma
 // <= 448) and written as two E4M3 terms, q sigma = hi + lo / 16 (hi rounded
 // to nearest, lo the rounded remainder times 16); a bf16 q has 8 significant
-// bits and each term 4, so the pair holds it exactly wherever hi is a normal
-// number, and S^T = (K hi + (K lo) / 16) / sigma with each product exact and
+// bits and each term 4, so the pair holds it exactly wherever |q sigma| is at
+// least E4M3's smallest normal 2^-6 (below it, within 2^-14), and S^T = (K hi + (K lo) / 16) / sigma with each product exact and
 // fp32 accumulation.  O^T stays an f16 MMA (P needs more than 4 bits).  Lane (g, c) = (lane / 4,
 // lane % 4).  In S^T it holds positions g and g + 8 for heads 2c, 2c+1, the
 // same heads whose columns it holds in O^T, so the softmax state and the

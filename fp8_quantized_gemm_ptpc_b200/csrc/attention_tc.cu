@@ -22,7 +22,8 @@
 //                   V tile read as an MN-major operand, B = P, MN-major)
 // all kind::f8f6f4 E4M3 x E4M3 with fp32 accumulators in tensor memory.  q
 // enters as two E4M3 terms (q = t1 + t2 / 16 after a power-of-two scale: 8
-// significant bits, exact for a bf16 value whose t1 is a normal number) and
+// significant bits, exact for a bf16 value of at least E4M3's smallest normal,
+// 2^-6, after the scale; within 2^-14 below it) and
 // P as three (P = t1 + t2 / 16 + t3 / 256: about 12 significant bits, like
 // f16); the N columns hold term 1 of the group's 8 heads, then term 2 (and,
 // for P, term 3 in a second MMA), so the terms share the MMAs.  The cache

@@ -353,8 +353,8 @@ PTPC_API size_t ptpc_decode_attention_workspace_size(int64_t B, int64_t Hq, int6
  *   p = softmax_l(softmax_scale * k_scale_l * sum_d q[d] * dec(K_l[d]))
  *   (0 for a sequence with no position), computed in fp32: q K^T from
  *   E4M3 tensor-core products of the K codes with q written as two E4M3
- *   terms (exact for every bf16 q whose first term is a normal number, see
- *   the kernel), P V from tensor-core products of the V codes with P written
+ *   terms (exact for every bf16 q whose scaled value is at least E4M3's
+ *   smallest normal 2^-6, see the kernel), P V from tensor-core products of the V codes with P written
  *   as three E4M3 terms (or, in the warp-level kernel, f16 P times the
  *   exactly decoded V codes; see ptpc_decode_attention_kernel).
  *   out_dev bf16 [B, Hq, D].
