@@ -245,6 +245,26 @@ def default_workspace(nbytes: int, device) -> Workspace:
         return ws.ensure(nbytes)
 
 
+def release_default_workspaces(device=None) -> int:
+    """Drop the cached default workspaces of one device (all devices when
+    None) and return how many were dropped; the next call on a stream
+    allocates a fresh one.  A prefill-sized ``linear`` keeps its quantised
+    activations there (hundreds of MB at T = 8192), so a caller that is done
+    with a stream, or with large shapes, can give that memory back.  Safe
+    while work is still queued: each buffer returns to PyTorch's caching
+    allocator, which reuses it only for later work of the stream it was
+    allocated on."""
+    if device is not None:
+        device = torch.device(device)
+        if device.type == "cuda" and device.index is None:
+            device = torch.device("cuda", torch.cuda.current_device())
+    with _ws_lock:
+        keys = [k for k in _ws_cache if device is None or k[0] == device]
+        for k in keys:
+            del _ws_cache[k]
+    return len(keys)
+
+
 # ----------------------------------------------------------------- entry points
 
 def quantize_activations(X: torch.Tensor, Xq: torch.Tensor | None = None, x_scale: torch.Tensor | None = None):

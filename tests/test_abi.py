@@ -236,3 +236,17 @@ def test_binding_remembers_workspace_sizes_until_overrides_reload(ptpc):
     assert len(ptpc._size_cache) >= 3
     ptpc.reload_tuning_overrides()
     assert len(ptpc._size_cache) == 0
+
+
+def test_release_default_workspaces(ptpc, monkeypatch):
+    """The cached default workspaces are dropped per device or all at once
+    (host logic: the cache is filled with placeholders, no device memory)."""
+    import torch
+    cache = {(torch.device("cuda", 0), 11): object(), (torch.device("cuda", 0), 12): object(),
+             (torch.device("cuda", 1), 11): object()}
+    monkeypatch.setattr(ptpc, "_ws_cache", dict(cache))
+    assert ptpc.release_default_workspaces("cuda:1") == 1
+    assert set(ptpc._ws_cache) == {(torch.device("cuda", 0), 11), (torch.device("cuda", 0), 12)}
+    assert ptpc.release_default_workspaces("cuda:3") == 0
+    assert ptpc.release_default_workspaces() == 2
+    assert ptpc._ws_cache == {}
