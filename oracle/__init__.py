@@ -407,7 +407,11 @@ def reference_epilogue(acc64: np.ndarray, x_scale, w_scale) -> np.ndarray:
 # plain definition, in fp64: for query head h (KV head g = h // (Hq / Hkv)),
 #   s_l = softmax_scale * sum_d q[h, d] * dec(K[l, g, d]) * k_scale[l, g],
 #   p = softmax(s),  out[h, d] = sum_l p_l * dec(V[l, g, d]) * v_scale[l, g],
-# rounded to bf16.
+# rounded to bf16, over the positions l < context_len whose block-table entry
+# exists (the table is wide enough), is not negative and lies inside the
+# cache; the others are left out, and a sequence left with no position gets
+# 0 (the softmax of an empty set is undefined: the library's reading, which
+# its header states).
 
 def kv_quantize(KV_bits: np.ndarray):
     """Per-(token, head) E4M3 quantisation of K or V, bf16 [T, H, D]:
@@ -429,17 +433,24 @@ def kv_cache_write(cache_codes, cache_scales, codes, scales, slots, block_size: 
 def decode_attention_reference(q_bits, k_codes, k_scales, v_codes, v_scales, block_tables, context_lens,
                                block_size: int, softmax_scale: float) -> np.ndarray:
     """Decode attention over an E4M3 paged cache, fp64, rounded to bf16.
-    q_bits bf16 [B, Hq, D]; returns bf16 bits [B, Hq, D]."""
+    q_bits bf16 [B, Hq, D]; returns bf16 bits [B, Hq, D].  Positions without
+    a valid block are left out; no position left: the output is 0."""
     B, Hq, D = q_bits.shape
-    Hkv = k_codes.shape[2]
+    num_blocks, Hkv = k_codes.shape[0], k_codes.shape[2]
     group = Hq // Hkv
     dec = e4m3_decode_table()
     q = bf16_to_float(q_bits).astype(np.float64)
-    out = np.empty((B, Hq, D), dtype=np.float64)
+    out = np.zeros((B, Hq, D), dtype=np.float64)
     for b in range(B):
         L = int(context_lens[b])
+        table = np.asarray(block_tables[b])
         pos = np.arange(L)
-        blocks = np.asarray(block_tables[b])[pos // block_size]
+        bi = pos // block_size
+        blocks = np.where(bi < len(table), table[np.minimum(bi, len(table) - 1)], -1) if len(table) else -np.ones(L, int)
+        keep = (blocks >= 0) & (blocks < num_blocks)
+        if not keep.any():
+            continue
+        pos, blocks = pos[keep], blocks[keep]
         offs = pos % block_size
         K = dec[k_codes[blocks, offs]] * k_scales[blocks, offs][:, :, None].astype(np.float64)   # [L, Hkv, D]
         V = dec[v_codes[blocks, offs]] * v_scales[blocks, offs][:, :, None].astype(np.float64)

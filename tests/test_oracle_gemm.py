@@ -353,3 +353,38 @@ def test_reference_epilogue_rounds_once():
     assert out[0, 0] == 0x3F81                                          # 1 + 2^-7
     assert brute_bf16(Fraction(1) + Fraction(1, 2 ** 8) + Fraction(1, 2 ** 30)) == 0x3F81
     assert brute_bf16(brute_f32(Fraction(1) + Fraction(1, 2 ** 8) + Fraction(1, 2 ** 30))) == 0x3F80
+
+
+def test_decode_attention_oracle_edge_cases():
+    """The positions the library leaves out: a context of 0 positions gives 0;
+    positions whose block-table entry is negative, past the cache or past the
+    table's width are left out, and the rest equals PyTorch's fp64 attention
+    over only the positions kept (taken in token order, not through the
+    table)."""
+    rng = np.random.Generator(np.random.PCG64(13))
+    Hq, Hkv, D, bs, nblk = 4, 2, 32, 4, 6
+    scale = 0.25
+    codes = {n: rng.integers(0, 0x7E, (nblk, bs, Hkv, D)).astype(np.uint8) for n in "kv"}
+    scales = {n: (rng.random((nblk, bs, Hkv)) + 0.5).astype(np.float32) for n in "kv"}
+    qb = synthetic.to_bf16_bits(rng.standard_normal((3, Hq, D)).astype(np.float32))
+    # seq 0: no position; seq 1: blocks 2, -1 (hole), 9 (past the cache), 4; seq 2: blocks 5,
+    # 1, -1, 3 and a context of 19, three positions past the table's 16 (left out)
+    tables = np.array([[0, 0, 0, 0], [2, -1, 9, 4], [5, 1, -1, 3]])
+    lens = [0, 15, 19]                              # seq 2: positions 16-18 lie past the table
+    out = oracle.decode_attention_reference(qb, codes["k"], scales["k"], codes["v"], scales["v"],
+                                            tables, lens, bs, scale)
+    assert not out[0].any()
+    dec = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double()
+    q = torch.from_numpy(qb.astype(np.int32) << 16).view(torch.float32).double()
+    kept = {1: [(2, o) for o in range(4)] + [(4, o) for o in range(3)],      # positions 0-3 and 12-14
+            2: [(5, o) for o in range(4)] + [(1, o) for o in range(4)] + [(3, o) for o in range(4)]}
+    for b, slots in kept.items():
+        kv = []
+        for n in "kv":
+            x = torch.stack([dec[torch.from_numpy(codes[n][blk, o]).long()] *
+                             torch.from_numpy(scales[n][blk, o]).double()[:, None] for blk, o in slots])
+            kv.append(x.permute(1, 0, 2).repeat_interleave(Hq // Hkv, dim=0))
+        ref = torch.nn.functional.scaled_dot_product_attention(q[b][:, None, :], kv[0], kv[1], scale=scale)[:, 0, :]
+        got = oracle.bf16_to_float(out[b]).astype(np.float64)
+        ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref.numpy()), 1e-30))) - 7)
+        assert np.all(np.abs(got - ref.numpy()) <= 0.5 * ulp + 1e-12 * np.abs(ref.numpy())), b

@@ -155,6 +155,11 @@ PY_MUTANTS = [
      "pos = np.arange(L)", "pos = np.arange(max(L - 1, 1))"),
     ("decode_attention_reference", "values scaled by the key scales",
      "V = dec[v_codes[blocks, offs]] * v_scales", "V = dec[v_codes[blocks, offs]] * k_scales"),
+    ("decode_attention_reference", "negative block entries read (from the end of the cache)",
+     "keep = (blocks >= 0) & (blocks < num_blocks)", "keep = blocks < num_blocks"),
+    ("decode_attention_reference", "positions past the table read from its last entry",
+     "blocks = np.where(bi < len(table), table[np.minimum(bi, len(table) - 1)], -1)",
+     "blocks = np.where(True, table[np.minimum(bi, len(table) - 1)], -1)"),
     ("kv_quantize", "heads and tokens swapped",
      "q, s = quant_act(np.ascontiguousarray(KV_bits).reshape(T * H, D))",
      "q, s = quant_act(np.ascontiguousarray(KV_bits.transpose(1, 0, 2)).reshape(T * H, D))"),
@@ -173,7 +178,8 @@ PY_MUTANTS = [
 ]
 
 PY_PINS = {
-    "decode_attention_reference": lambda: gemm.test_decode_attention_oracle_matches_library_attention(),
+    "decode_attention_reference": lambda: (gemm.test_decode_attention_oracle_matches_library_attention(),
+                                           gemm.test_decode_attention_oracle_edge_cases()),
     "kv_quantize": lambda: gemm.test_kv_cache_oracle(),
     "gemm_acc64": lambda: gemm.test_hand_example_gemm(),
     "gemm_acc64_fmt": lambda: subbyte.test_gemm_exact_against_integer_dot_products("e2m1"),
