@@ -73,7 +73,7 @@ typedef enum {
     PTPC_ERR_UNSUPPORTED_DEVICE = 5,   /* current device is not compute capability 10.0 */
     PTPC_ERR_CUDA = 6,                 /* a CUDA runtime/driver call failed */
     PTPC_ERR_DEVICE_TIMEOUT = 7,       /* a kernel's bounded wait ran out (device status word) */
-    PTPC_ERR_NOT_IMPLEMENTED = 8
+    PTPC_ERR_NOT_IMPLEMENTED = 8       /* reserved: no entry point returns it at present */
 } ptpc_status;
 
 /* Weight formats.  E4M3 is the PTPC-FP8 format of the entry points above;
