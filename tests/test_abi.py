@@ -250,3 +250,19 @@ def test_release_default_workspaces(ptpc, monkeypatch):
     assert ptpc.release_default_workspaces("cuda:3") == 0
     assert ptpc.release_default_workspaces() == 2
     assert ptpc._ws_cache == {}
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """The package refuses to import when libptpc.so has not been built: no
+    fallback path exists.  (A copy of the binding in a folder with no _lib.)"""
+    import shutil
+    import subprocess
+    import sys
+    src = os.path.join(ROOT, "fp8_quantized_gemm_ptpc_b200", "__init__.py")
+    pkg = tmp_path / "fp8_quantized_gemm_ptpc_b200"
+    pkg.mkdir()
+    shutil.copy(src, pkg / "__init__.py")
+    r = subprocess.run([sys.executable, "-c", "import fp8_quantized_gemm_ptpc_b200"], cwd=tmp_path,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "is missing" in r.stderr
