@@ -261,8 +261,12 @@ PTPC_API int ptpc_linear_fmt(const void *X_dev, int64_t ldx, const uint8_t *Wq_d
  *   PTPC_FORCE_GROUP_M = 1 .. 63         tile rows the prefill kernel visits
  *                                        together (their activation tiles
  *                                        kept in L2 while the columns sweep),
- *   PTPC_FORCE_ATTN_CHUNK = 512 | 1024 | 2048  context positions a CTA of
- *                                        ptpc_decode_attention takes.
+ *   PTPC_FORCE_ATTN_CHUNK = 512 | 1024 | 2048 | 4096  context positions a
+ *                                        CTA of ptpc_decode_attention takes
+ *                                        (4096 only on the tensor-memory
+ *                                        kernel; the other takes at most 2048),
+ *   PTPC_FORCE_ATTN_KERNEL = mma | tc    which decode-attention kernel runs
+ *                                        (tc only where it applies).
  * Each is honoured only where the forced choice is feasible for the shape;
  * results stay within the GEMM's tolerance under every choice.  For tuning
  * and tests, not for production.  Not thread-safe with concurrent GEMM calls
