@@ -45,8 +45,10 @@
  *   - Inputs are assumed finite.  Non-finite inputs do not fault but give
  *     unspecified codes.  The GEMM epilogue multiplies in the order
  *     (acc * x_scale) * w_scale in fp32; outputs are specified where that
- *     intermediate product is finite (|acc * x_scale| < 2^128), which holds
- *     unless a token's amax is within ~2^30 of the bf16 maximum.
+ *     intermediate product is finite (|acc * x_scale| < 2^128).  Since
+ *     |acc| <= Ci * 448^2 and x_scale = amax / 448, that holds whenever a
+ *     token's amax is below 2^128 / (448 * Ci): within 2^24 of the bf16
+ *     maximum at Ci = 28672, 2^26 at Ci = 2^17.
  */
 #ifndef PTPC_H_
 #define PTPC_H_
